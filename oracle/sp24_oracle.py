@@ -1,0 +1,423 @@
+"""CPU oracle for the 2:4 structured-sparse FP8 GEMM path (test infrastructure).
+
+THIS MODULE IS TEST INFRASTRUCTURE.  Only the tests, the package's ``smoke()``
+check and the benchmark's CPU-baseline leg may import it.  The product path
+(the CUDA library behind ``include/sp24.h``) never calls it, shares no code,
+table or constant generator with it, and must fail loudly when its extension
+is missing instead of falling back to anything here.
+
+Every function below is the plain definition of one step of the method,
+written with numpy in float64 (FP8 codes, bf16 bit patterns and metadata are
+integers).  Where the pages leave a step open the reading taken is stated in
+the function's docstring.  Pages cited:
+
+* "Deploying 2:4 Sparsity with FP8 on Hopper: A Production Cookbook"
+  (the cookbook) -- pipeline steps 2-4 and 6, Practical Example 1
+  ("2:4 mask application").
+* "SlideSparse: Fast and Flexible (2N-2):2N Structured Sparsity" (the
+  SlideSparse summary) -- Resumen tecnico §2 Metodologia: "Descomposicion de
+  Ventana Deslizante", "Levantamiento de Activacion", "Pipeline de
+  Implementacion"; the lay "Analogia de la Ventana Deslizante".
+* "La Densite Dynamique et les Noyaux Non Structures ..." (the roadmap) --
+  §Lacunes des noyaux (compressed metadata), §Interaction avec la
+  quantification (per-tensor FP8 scaling).
+
+Conventions shared with the CUDA path (fixed here, from the readings):
+
+* bf16 tensors are passed around as ``uint16`` bit patterns.
+* E4M3 means the OCP FP8 "E4M3FN" format: bias 7, 3 mantissa bits, no
+  infinities, NaN = S.1111.111, largest finite 448.
+* 2:4 groups are 4 contiguous values along K (the last axis).
+* Compressed layout: ``values[n, 2g + t]`` is the t-th kept element of group
+  g in ascending index order; ``meta[n, b]`` holds group 2b in bits 0-3 and
+  group 2b+1 in bits 4-7, each nibble ``i0 | i1 << 2`` with ``i0 < i1``.
+
+All functions are parity-pinned by ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+E4M3_MAX = 448.0
+
+# ---------------------------------------------------------------------------
+# bf16 helpers (definition of the bf16 format: the top 16 bits of a float32)
+# ---------------------------------------------------------------------------
+
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns (uint16) to float32 exactly."""
+    bits = np.asarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def f32_to_bf16_rne(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bf16 bit patterns, round-to-nearest-even.
+
+    Used only to express the bf16 rounding of an output; NaN is not expected.
+    """
+    u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (u >> np.uint64(16)) & np.uint64(1)
+    u = u + np.uint64(0x7FFF) + lsb
+    return (u >> np.uint64(16)).astype(np.uint16)
+
+
+def _require_finite(x: np.ndarray, what: str) -> None:
+    if not np.all(np.isfinite(x)):
+        raise ValueError(f"{what}: the method is defined for finite inputs only")
+
+
+# ---------------------------------------------------------------------------
+# FP8 E4M3 (per-tensor dynamic scaling: the cookbook, pipeline steps 3 and 6;
+# the roadmap, §Interaction avec la quantification)
+# ---------------------------------------------------------------------------
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """Encode float32 values as E4M3 codes: round to nearest even, saturating.
+
+    Written from the format's definition: a value with |v| >= 2**-6 has
+    quantum 2**(e-3) where e = floor(log2 |v|); below that the grid is the
+    subnormal one with quantum 2**-9.  Rounding is to nearest, ties to even
+    (numpy's ``rint``), done in float64 where dividing by a power of two is
+    exact.  Magnitudes that round above 448 saturate to 448 (the
+    "satfinite" reading).  The sign of v is kept, so a negative value that
+    rounds to zero gives the code 0x80.  NaN gives 0x7F.
+    """
+    v = np.asarray(v, dtype=np.float32)
+    a = np.abs(v.astype(np.float64))
+    neg = np.signbit(v)
+    nan = np.isnan(a)
+    a = np.where(nan, 0.0, a)
+    _require_finite(a, "e4m3_encode")
+    _, ex = np.frexp(a)                      # a = m * 2**ex, m in [0.5, 1)
+    e = np.maximum(ex.astype(np.int64) - 1, -6)
+    quantum = np.ldexp(1.0, (e - 3).astype(np.int32))
+    q = np.rint(a / quantum) * quantum       # nearest grid point, ties to even
+    q = np.minimum(q, E4M3_MAX)              # saturate
+    # q is now exactly representable; split it into exponent and mantissa.
+    code = np.zeros(a.shape, dtype=np.int64)
+    sub = q < 2.0 ** -6
+    code = np.where(sub, np.rint(q / 2.0 ** -9).astype(np.int64), code)
+    _, qex = np.frexp(np.where(sub, 1.0, q))
+    qe = qex.astype(np.int64) - 1            # floor(log2 q) for normal q
+    mant = np.rint(np.ldexp(np.where(sub, 1.0, q), (3 - qe).astype(np.int32))).astype(np.int64) - 8
+    normal_code = ((qe + 7) << 3) | mant
+    code = np.where(sub, code, normal_code)
+    code = code | np.where(neg, 0x80, 0)
+    code = np.where(nan, 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """Value of each E4M3 code as float64 (NaN for S.1111.111)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    s = np.where(c & 0x80, -1.0, 1.0)
+    ef = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(ef == 0, m * 2.0 ** -9,
+                   (1.0 + m / 8.0) * np.ldexp(1.0, (ef - 7).astype(np.int32)))
+    val = np.where((ef == 15) & (m == 7), np.nan, val)
+    return s * val
+
+
+def amax(bits: np.ndarray) -> np.float32:
+    """Largest |x| of a bf16 tensor, as float32 (exact: a max of bf16 values)."""
+    x = bf16_to_f32(bits)
+    _require_finite(x, "amax")
+    if x.size == 0:
+        return np.float32(0.0)
+    return np.float32(np.max(np.abs(x)))
+
+
+def scale_from_amax(a: np.float32) -> np.float32:
+    """Per-tensor dequantisation scale s = amax / 448, one fp32 division.
+
+    Reading: when amax is 0 the scale is taken as 1.0 (every code is then 0).
+    """
+    a = np.float32(a)
+    if a == 0:
+        return np.float32(1.0)
+    return np.float32(a / np.float32(E4M3_MAX))
+
+
+def quantize_with_scale(bits: np.ndarray, s: np.float32) -> np.ndarray:
+    """E4M3 codes of x / s, the quotient taken as one correctly rounded fp32
+    division (reading: divide by the dequantisation scale, not multiply by
+    its reciprocal)."""
+    x = bf16_to_f32(bits)
+    v = (x / np.float32(s)).astype(np.float32)
+    return e4m3_encode(v)
+
+
+def quantize_pertensor(bits: np.ndarray):
+    """Per-tensor dynamic E4M3 quantisation: returns (codes, scale)."""
+    s = scale_from_amax(amax(bits))
+    return quantize_with_scale(bits, s), s
+
+
+# ---------------------------------------------------------------------------
+# N:M magnitude pruning along K (the cookbook, pipeline step 4 and Practical
+# Example 1; the SlideSparse summary, §1 for 6:8)
+# ---------------------------------------------------------------------------
+
+
+def keep_mask(bits: np.ndarray, group: int, keep: int) -> np.ndarray:
+    """Magnitude N:M mask along the last axis.
+
+    In every group of ``group`` contiguous values, element i beats element j
+    when |w_i| > |w_j|, or |w_i| == |w_j| and i < j (ties go to the lower
+    index; -0 and +0 are equal).  An element is kept when fewer than ``keep``
+    elements of its group beat it, which keeps exactly ``keep`` per group.
+    """
+    w = bf16_to_f32(bits)
+    _require_finite(w, "keep_mask")
+    if w.shape[-1] % group:
+        raise ValueError(f"K={w.shape[-1]} is not a multiple of {group}")
+    a = np.abs(w).reshape(*w.shape[:-1], w.shape[-1] // group, group).astype(np.float64)
+    idx = np.arange(group)
+    ai = a[..., :, None]
+    aj = a[..., None, :]
+    beats = (aj > ai) | ((aj == ai) & (idx[None, :] < idx[:, None]))
+    rank = beats.sum(axis=-1)
+    return (rank < keep).reshape(w.shape)
+
+
+def prune24_mask(bits: np.ndarray) -> np.ndarray:
+    """2:4 magnitude mask: the two largest |w| of each 4 along K survive."""
+    return keep_mask(bits, 4, 2)
+
+
+def compress24(mask: np.ndarray, payload: np.ndarray):
+    """Compress a 2:4-masked [N, K] array into (values [N, K/2], meta [N, K/8]).
+
+    ``payload`` is whatever is stored per kept element (E4M3 codes or bf16
+    bit patterns).  Requires exactly two kept elements per group of 4.
+    """
+    mask = np.asarray(mask, dtype=bool)
+    n, k = mask.shape
+    if k % 8:
+        raise ValueError("compressed metadata needs K to be a multiple of 8")
+    g = mask.reshape(n, k // 4, 4)
+    if not np.all(g.sum(axis=-1) == 2):
+        raise ValueError("every group of 4 must keep exactly 2 elements")
+    pos = np.nonzero(g)[-1].reshape(n, k // 4, 2)          # ascending per group
+    i0, i1 = pos[..., 0], pos[..., 1]
+    p = np.asarray(payload).reshape(n, k // 4, 4)
+    vals = np.take_along_axis(p, pos, axis=-1).reshape(n, k // 2)
+    nib = (i0 | (i1 << 2)).astype(np.uint8)                # [n, k/4]
+    meta = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    return vals, meta
+
+
+def decompress24(values: np.ndarray, meta: np.ndarray, k: int, fill=0):
+    """Scatter compressed values back to a dense [N, K] array (``fill`` elsewhere)."""
+    values = np.asarray(values)
+    meta = np.asarray(meta, dtype=np.uint8)
+    n = values.shape[0]
+    nib = np.empty((n, k // 4), dtype=np.int64)
+    nib[:, 0::2] = meta & 0xF
+    nib[:, 1::2] = meta >> 4
+    i0 = nib & 3
+    i1 = nib >> 2
+    out = np.full((n, k // 4, 4), fill, dtype=values.dtype)
+    v = values.reshape(n, k // 4, 2)
+    np.put_along_axis(out, i0[..., None], v[..., 0:1], axis=-1)
+    np.put_along_axis(out, i1[..., None], v[..., 1:2], axis=-1)
+    return out.reshape(n, k)
+
+
+def sp24_prune_compress(w_bits: np.ndarray, out_dtype: str = "e4m3"):
+    """The weight path for 2:4: prune, then quantise (E4M3) or keep (bf16), then compress.
+
+    Returns a dict with ``values``, ``meta``, ``mask``, ``scale`` (None for
+    bf16) and ``pruned_dense`` (E4M3 codes with 0x00 at pruned positions, or
+    the pruned bf16 bit patterns with 0x0000 there).
+
+    Reading: pruning ranks the original bf16 magnitudes, before quantisation
+    (pruning is the first step of the pipeline, quantisation the third).  The
+    weight scale is taken from the whole tensor's amax, which equals the
+    pruned tensor's amax because each group's largest element is kept.
+    """
+    w_bits = np.asarray(w_bits, dtype=np.uint16)
+    mask = prune24_mask(w_bits)
+    if out_dtype == "e4m3":
+        s = scale_from_amax(amax(w_bits))
+        codes = quantize_with_scale(w_bits, s)
+        dense = np.where(mask, codes, np.uint8(0)).astype(np.uint8)
+        vals, meta = compress24(mask, codes)
+        return dict(values=vals.astype(np.uint8), meta=meta, mask=mask, scale=s,
+                    pruned_dense=dense)
+    if out_dtype == "bf16":
+        dense = np.where(mask, w_bits, np.uint16(0)).astype(np.uint16)
+        vals, meta = compress24(mask, w_bits)
+        return dict(values=vals.astype(np.uint16), meta=meta, mask=mask, scale=None,
+                    pruned_dense=dense)
+    raise ValueError(out_dtype)
+
+
+# ---------------------------------------------------------------------------
+# The GEMM Y = X W^T (reference) and its error bound
+# ---------------------------------------------------------------------------
+
+
+def gemm_ref(x_vals: np.ndarray, w_vals: np.ndarray, sx=1.0, sw=1.0):
+    """Y[m, n] = sx * sw * sum_k x[m, k] * w[n, k] in float64, and the bound
+    B[m, n] = |sx * sw| * sum_k |x[m, k] * w[n, k]|.
+
+    ``x_vals``/``w_vals`` are the decoded operand values (float64).  Every
+    product of two E4M3 (or bf16) values is exact in float64 and the float64
+    sums carry far less error than any tolerance used against it.
+    """
+    x = np.asarray(x_vals, dtype=np.float64)
+    w = np.asarray(w_vals, dtype=np.float64)
+    s = float(np.float64(sx) * np.float64(sw))
+    y = s * (x @ w.T)
+    b = abs(s) * (np.abs(x) @ np.abs(w).T)
+    return y, b
+
+
+def sparse_gemm_walk(x_vals: np.ndarray, values: np.ndarray, meta: np.ndarray,
+                     sx=1.0, sw=1.0) -> np.ndarray:
+    """Y from the compressed operand directly, in plain loops (tiny shapes only).
+
+    For each output (m, n) and each group g, the two stored values multiply
+    x[m, 4g + i0] and x[m, 4g + i1].  Used to pin the compressed format
+    against the dense reference.
+    """
+    x = np.asarray(x_vals, dtype=np.float64)
+    v = np.asarray(values, dtype=np.float64)
+    m_, k = x.shape
+    n_ = v.shape[0]
+    y = np.zeros((m_, n_))
+    for m in range(m_):
+        for n in range(n_):
+            acc = 0.0
+            for g in range(k // 4):
+                byte = int(meta[n, g // 2])
+                nib = (byte >> (4 * (g % 2))) & 0xF
+                i0, i1 = nib & 3, nib >> 2
+                acc += v[n, 2 * g] * x[m, 4 * g + i0]
+                acc += v[n, 2 * g + 1] * x[m, 4 * g + i1]
+            y[m, n] = acc
+    return float(np.float64(sx) * np.float64(sw)) * y
+
+
+def within_tolerance(y_gpu: np.ndarray, y_ref: np.ndarray, bound: np.ndarray,
+                     rel_bound: float = 1e-3, rel_val: float = 1e-2) -> np.ndarray:
+    """Elementwise pass mask of |y - y_ref| <= 1e-3 * B + 1e-2 * |y_ref|."""
+    y = np.asarray(y_gpu, dtype=np.float64)
+    return np.abs(y - y_ref) <= rel_bound * bound + rel_val * np.abs(y_ref)
+
+
+# ---------------------------------------------------------------------------
+# 6:8 sliding-window decomposition and activation lifting (the SlideSparse
+# summary, §2 Metodologia)
+# ---------------------------------------------------------------------------
+
+
+def prune68_mask(bits: np.ndarray) -> np.ndarray:
+    """6:8 magnitude mask: the six largest |w| of each 8 along K survive
+    (ties to the lower index, as for 2:4)."""
+    return keep_mask(bits, 8, 6)
+
+
+def window_assignment(kept: np.ndarray):
+    """Assign the 6 kept positions of one 8-group to the 3 stride-2 windows.
+
+    Window j covers positions 2j .. 2j+3.  Reading of "the extras spill into
+    the next overlapping window": for j = 0, 1, 2 in turn, window j takes the
+    two lowest-index kept positions in its range that no earlier window took.
+    Returns a list of three (p0, p1) pairs, p0 < p1.
+    """
+    kept = [int(p) for p in np.nonzero(np.asarray(kept, dtype=bool))[0]]
+    if len(kept) != 6:
+        raise ValueError("a 6:8 group must keep exactly 6 positions")
+    taken = set()
+    out = []
+    for j in range(3):
+        cand = [p for p in kept if 2 * j <= p <= 2 * j + 3 and p not in taken]
+        if len(cand) < 2:
+            raise AssertionError("window assignment failed")  # impossible, see tests
+        pick = cand[:2]
+        taken.update(pick)
+        out.append((pick[0], pick[1]))
+    if taken != set(kept):
+        raise AssertionError("window assignment lost a kept position")
+    return out
+
+
+def slide68_expand_mask_and_map(mask68: np.ndarray):
+    """For a 6:8 mask [N, K], build the expanded 2:4 mask [N, 1.5K] and the
+    source column of every kept expanded slot (-1 where the slot is empty).
+
+    Expanded column of window j, slot r of group g is 12g + 4j + r; the
+    element placed there is W[n, 8g + 2j + r].
+    """
+    n, k = mask68.shape
+    kp = k * 3 // 2
+    emask = np.zeros((n, kp), dtype=bool)
+    src = np.full((n, kp), -1, dtype=np.int64)
+    for row in range(n):
+        for g in range(k // 8):
+            pairs = window_assignment(mask68[row, 8 * g:8 * g + 8])
+            for j, (p0, p1) in enumerate(pairs):
+                for p in (p0, p1):
+                    col = 12 * g + 4 * j + (p - 2 * j)
+                    emask[row, col] = True
+                    src[row, col] = 8 * g + p
+    return emask, src
+
+
+def slide68_decompose(w_bits: np.ndarray, out_dtype: str = "e4m3"):
+    """6:8 prune, window decomposition and 2:4 compression over K' = 1.5K.
+
+    Returns values [N, 3K/4], meta [N, 3K/16], the 6:8 mask, the expanded
+    mask [N, 1.5K], the scale (E4M3; None for bf16) and the expanded dense
+    operand W' [N, 1.5K] (codes or bf16 bits, zero in empty slots).
+    """
+    w_bits = np.asarray(w_bits, dtype=np.uint16)
+    n, k = w_bits.shape
+    if k % 8:
+        raise ValueError("6:8 needs K to be a multiple of 8")
+    m68 = prune68_mask(w_bits)
+    emask, src = slide68_expand_mask_and_map(m68)
+    if out_dtype == "e4m3":
+        s = scale_from_amax(amax(w_bits))
+        payload = quantize_with_scale(w_bits, s)
+        zero = np.uint8(0)
+    elif out_dtype == "bf16":
+        s = None
+        payload = w_bits
+        zero = np.uint16(0)
+    else:
+        raise ValueError(out_dtype)
+    rows = np.arange(n)[:, None]
+    wexp = np.where(emask, payload[rows, np.maximum(src, 0)], zero).astype(payload.dtype)
+    vals, meta = compress24(emask, wexp)
+    return dict(values=vals, meta=meta, mask68=m68, emask=emask, scale=s,
+                expanded=wexp, src=src)
+
+
+def lift_columns(k: int) -> np.ndarray:
+    """Source column of X for every lifted column: X'[:, 12g+4j+r] = X[:, 8g+2j+r]."""
+    cols = np.empty(k * 3 // 2, dtype=np.int64)
+    for g in range(k // 8):
+        for j in range(3):
+            for r in range(4):
+                cols[12 * g + 4 * j + r] = 8 * g + 2 * j + r
+    return cols
+
+
+def slide68_lift(x_bits: np.ndarray):
+    """Per-tensor E4M3 quantisation of X fused with the lift to K' = 1.5K.
+
+    The scale is that of X itself (X' holds the same values, so the same
+    amax).  Returns (lifted codes [M, 1.5K], scale).
+    """
+    x_bits = np.asarray(x_bits, dtype=np.uint16)
+    k = x_bits.shape[1]
+    if k % 8:
+        raise ValueError("6:8 lifting needs K to be a multiple of 8")
+    codes, s = quantize_pertensor(x_bits)
+    return codes[:, lift_columns(k)], s

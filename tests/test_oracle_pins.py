@@ -1,0 +1,302 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test ties one oracle function to an independent source: a library
+routine (ml_dtypes / torch FP8 casts), brute force over every small case,
+closed forms, invariants the pages state, or the hand-worked fixtures under
+``tests/golden/``.  No test here needs a GPU.
+"""
+import itertools
+import os
+
+import ml_dtypes
+import numpy as np
+import pytest
+import torch
+
+from oracle import sp24_oracle as O
+from structured_sparse_fp8_b200 import workloads as WL
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# --------------------------------------------------------------------------
+# E4M3 encode / decode
+# --------------------------------------------------------------------------
+
+def _lib_e4m3(v32):
+    return np.asarray(v32, dtype=np.float32).astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+
+
+def test_e4m3_decode_all_codes_match_ml_dtypes():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = O.e4m3_decode(codes)
+    lib = codes.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    same = (ours == lib) | (np.isnan(ours) & np.isnan(lib))
+    assert same.all()
+
+
+def test_e4m3_encode_every_bf16_value_in_range():
+    bits = np.arange(65536, dtype=np.uint16)
+    v = O.bf16_to_f32(bits)
+    ok = np.isfinite(v) & (np.abs(v) <= 448.0)
+    v = v[ok]
+    assert (O.e4m3_encode(v) == _lib_e4m3(v)).all()
+    t = torch.from_numpy(v.copy()).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert (O.e4m3_encode(v) == t).all()
+
+
+def test_e4m3_encode_strided_fp32_sweep_and_ties():
+    # every 97th fp32 bit pattern from +0 up to 464 (beyond the last tie), both signs
+    top = np.float32(464.0).view(np.uint32)
+    pos = np.arange(0, int(top) + 1, 97, dtype=np.uint32).view(np.float32)
+    v = np.concatenate([pos, -pos])
+    assert (O.e4m3_encode(v) == _lib_e4m3(v)).all()
+    # every midpoint between neighbouring E4M3 values, and one fp32 ulp either side
+    grid = np.unique(np.abs(O.e4m3_decode(np.arange(0x7F, dtype=np.uint8))))
+    mids = ((grid[:-1] + grid[1:]) / 2).astype(np.float32)
+    probe = np.concatenate([mids, np.nextafter(mids, np.float32(0)),
+                            np.nextafter(mids, np.float32(1e9))])
+    probe = np.concatenate([probe, -probe])
+    assert (O.e4m3_encode(probe) == _lib_e4m3(probe)).all()
+
+
+def test_e4m3_saturates_above_448_and_keeps_sign_of_zero():
+    big = np.array([448.0, 460.0, 464.0, 465.0, 1000.0, 3.0e38], dtype=np.float32)
+    assert (O.e4m3_encode(big) == 0x7E).all()
+    assert (O.e4m3_encode(-big) == 0xFE).all()
+    tiny = np.array([0.0, 1e-30, 2.0 ** -10], dtype=np.float32)
+    assert (O.e4m3_encode(tiny) == 0x00).all()
+    assert (O.e4m3_encode(-tiny) == 0x80).all()
+
+
+def test_e4m3_golden_landmarks():
+    path = os.path.join(GOLDEN, "e4m3_landmarks.txt")
+    rows = [ln.split("#")[0].split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    vals = np.array([float.fromhex(r[0]) for r in rows], dtype=np.float32)
+    codes = np.array([int(r[1], 16) for r in rows], dtype=np.uint8)
+    assert (O.e4m3_encode(vals) == codes).all()
+
+
+# --------------------------------------------------------------------------
+# Scale and quantisation
+# --------------------------------------------------------------------------
+
+def test_scale_closed_form_and_zero_tensor():
+    x = WL.random_bits((64, 256), 1, scale=3.0)
+    a = O.amax(x)
+    assert a == np.max(np.abs(x.view(ml_dtypes.bfloat16).astype(np.float64)))
+    s = O.scale_from_amax(a)
+    assert s == np.float32(np.float32(a) / np.float32(448.0))
+    codes, s2 = O.quantize_pertensor(x)
+    assert s2 == s
+    # the largest magnitude maps onto the top code 0x7E (= 448) exactly
+    assert (codes & 0x7F).max() == 0x7E
+    z = np.zeros((4, 16), dtype=np.uint16)
+    cz, sz = O.quantize_pertensor(z)
+    assert sz == np.float32(1.0) and (cz == 0).all()
+
+
+def test_quantised_dequantised_error_within_e4m3_half_ulp():
+    x = WL.random_bits((32, 512), 2)
+    codes, s = O.quantize_pertensor(x)
+    xv = O.bf16_to_f32(x).astype(np.float64)
+    back = O.e4m3_decode(codes) * float(s)
+    # relative half-ulp of a 3-bit mantissa, plus the subnormal quantum
+    err = np.abs(back - xv)
+    assert (err <= np.abs(xv) * 2.0 ** -4 + float(s) * 2.0 ** -10 * 1.0001).all()
+
+
+# --------------------------------------------------------------------------
+# 2:4 and 6:8 pruning against brute force
+# --------------------------------------------------------------------------
+
+ALPHABET = [0.0, -0.0, 1.0, -1.0, 2.0]
+
+
+def _brute_keep(group_vals, keep):
+    a = np.abs(np.asarray(group_vals, dtype=np.float64))
+    best = None
+    for subset in itertools.combinations(range(len(a)), keep):
+        key = (-a[list(subset)].sum(), subset)     # max sum, then lexicographically lowest
+        if best is None or key < best:
+            best = key
+    return set(best[1])
+
+
+def test_prune24_exhaustive_over_tie_alphabet():
+    groups = np.array(list(itertools.product(ALPHABET, repeat=4)))
+    bits = WL.to_bf16_bits(groups)
+    mask = O.prune24_mask(bits)
+    for g, m in zip(groups, mask):
+        assert set(np.nonzero(m)[0]) == _brute_keep(g, 2), g
+
+
+def test_prune68_against_brute_force():
+    rng = np.random.default_rng(5)
+    groups = np.array(list(itertools.product([0.0, 1.0, 2.0], repeat=8)))   # 6561 tie-heavy groups
+    groups = np.concatenate([groups * rng.choice([-1, 1], size=groups.shape),
+                             rng.normal(size=(2000, 8))])
+    bits = WL.to_bf16_bits(groups)
+    mask = O.prune68_mask(bits)
+    for g, m in zip(bits, mask):
+        assert set(np.nonzero(m)[0]) == _brute_keep(O.bf16_to_f32(g), 6)
+
+
+def test_prune24_matches_the_cookbook_topk_mask_when_no_ties():
+    # Practical Example 1 of the cookbook keeps topk(2) of |w| per group of 4 along K.
+    w = WL.random_bits((64, 256), 3, scale=0.02)
+    wt = torch.from_numpy(O.bf16_to_f32(w).copy())
+    g = wt.reshape(64, 64, 4).abs()
+    top2 = g.topk(2, dim=-1).indices
+    ref = torch.zeros_like(g, dtype=torch.bool).scatter_(-1, top2, True).reshape(64, 64, 4)
+    # topk leaves the order of equal magnitudes open: compare the tie-free groups only
+    gs = np.sort(g.numpy(), axis=-1)
+    tie_free = (np.diff(gs, axis=-1) != 0).all(-1)
+    assert tie_free.mean() > 0.9
+    ours = O.prune24_mask(w).reshape(64, 64, 4)
+    assert (ours[tie_free] == ref.numpy()[tie_free]).all()
+
+
+def test_prune24_golden_hand_example():
+    path = os.path.join(GOLDEN, "prune24_hand_example.txt")
+    lines = [ln for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    w = np.array([[float(t) for t in ln.split()] for ln in lines[:2]])
+    want_mask = np.array([[int(t) for t in ln.split()] for ln in lines[2:4]], dtype=bool)
+    want_meta = np.array([[int(t, 16) for t in ln.split()] for ln in lines[4:6]], dtype=np.uint8)
+    bits = WL.to_bf16_bits(w)
+    mask = O.prune24_mask(bits)
+    assert (mask == want_mask).all()
+    _, meta = O.compress24(mask, bits)
+    assert (meta == want_meta).all()
+
+
+def test_exactly_two_nonzeros_per_group_on_workload_weights():
+    w = WL.weight_bits(1)                    # 256 x 256, N(0, 0.02)
+    assert (O.bf16_to_f32(w) != 0).all()     # no exact zeros in practice
+    out = O.sp24_prune_compress(w, "bf16")
+    nz = (O.bf16_to_f32(out["pruned_dense"]) != 0).reshape(256, 64, 4).sum(-1)
+    assert (nz == 2).all()
+
+
+# --------------------------------------------------------------------------
+# Compression round trip and metadata validity
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["e4m3", "bf16"])
+def test_compress_roundtrip_bit_exact(dtype):
+    w = WL.random_bits((48, 320), 4, scale=0.02, dist="ties" if dtype == "bf16" else "normal")
+    out = O.sp24_prune_compress(w, dtype)
+    back = O.decompress24(out["values"], out["meta"], 320)
+    assert (back == out["pruned_dense"]).all()
+    nib = np.stack([out["meta"] & 0xF, out["meta"] >> 4], -1).reshape(48, 80)
+    i0, i1 = nib & 3, nib >> 2
+    assert (i0 < i1).all() and (i1 <= 3).all()
+
+
+def test_amax_of_pruned_equals_amax_of_original():
+    for seed in range(4):
+        w = WL.random_bits((32, 256), 10 + seed, dist="student_t3")
+        out = O.sp24_prune_compress(w, "bf16")
+        assert O.amax(out["pruned_dense"]) == O.amax(w)
+
+
+# --------------------------------------------------------------------------
+# GEMM: compressed walk vs dense reference, closed-form special cases
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dist", ["normal", "ties"])
+def test_sparse_walk_equals_dense_reference(dist):
+    x = WL.random_bits((5, 64), 20, dist=dist)
+    w = WL.random_bits((7, 64), 21, scale=0.02, dist=dist)
+    xq, sx = O.quantize_pertensor(x)
+    out = O.sp24_prune_compress(w, "e4m3")
+    walk = O.sparse_gemm_walk(O.e4m3_decode(xq), O.e4m3_decode(out["values"]), out["meta"], sx, out["scale"])
+    dense, _ = O.gemm_ref(O.e4m3_decode(xq), O.e4m3_decode(out["pruned_dense"]), sx, out["scale"])
+    assert np.array_equal(walk, dense)
+
+
+def test_selection_pattern_reduces_gemm_to_column_picks():
+    # Row n of W keeps column c_n with value 1 and a second column with value 0,
+    # so Y[:, n] must be exactly X[:, c_n] (a closed form independent of the GEMM).
+    k, n = 64, 16
+    rng = np.random.default_rng(7)
+    cols = rng.integers(0, k, size=n)
+    w = np.zeros((n, k))
+    w[np.arange(n), cols] = 1.0
+    bits = WL.to_bf16_bits(w)
+    mask = O.prune24_mask(bits)
+    vals, meta = O.compress24(mask, bits)
+    x = O.bf16_to_f32(WL.random_bits((3, k), 8)).astype(np.float64)
+    y = O.sparse_gemm_walk(x, O.bf16_to_f32(vals), meta)
+    assert np.array_equal(y, x[:, cols])
+
+
+def test_tolerance_rule_is_tight_enough_to_catch_a_dropped_group():
+    x = WL.random_bits((4, 256), 30)
+    w = WL.random_bits((8, 256), 31, scale=0.02)
+    xq, sx = O.quantize_pertensor(x)
+    out = O.sp24_prune_compress(w, "e4m3")
+    xv, wv = O.e4m3_decode(xq), O.e4m3_decode(out["pruned_dense"])
+    y, b = O.gemm_ref(xv, wv, sx, out["scale"])
+    wv_bad = wv.copy()
+    wv_bad[:, 0:4] = 0.0                   # drop one group of K
+    y_bad, _ = O.gemm_ref(xv, wv_bad, sx, out["scale"])
+    assert O.within_tolerance(O.bf16_to_f32(O.f32_to_bf16_rne(y.astype(np.float32))), y, b).all()
+    assert not O.within_tolerance(y_bad, y, b).all()
+
+
+# --------------------------------------------------------------------------
+# 6:8 sliding windows and lifting
+# --------------------------------------------------------------------------
+
+def test_every_68_mask_decomposes_into_three_24_windows():
+    for kept in itertools.combinations(range(8), 6):
+        m = np.zeros(8, dtype=bool)
+        m[list(kept)] = True
+        pairs = O.window_assignment(m)
+        assert len(pairs) == 3
+        used = []
+        for j, (p0, p1) in enumerate(pairs):
+            assert 2 * j <= p0 < p1 <= 2 * j + 3
+            used += [p0, p1]
+        assert sorted(used) == sorted(kept)
+
+
+def test_slide68_reconstructs_pruned_groups_and_gemm_exactly():
+    w = WL.random_bits((12, 64), 40, scale=0.02)
+    d = O.slide68_decompose(w, "bf16")
+    assert d["values"].shape == (12, 48) and d["meta"].shape == (12, 12)   # K' = 1.5 K
+    # scatter the expanded operand back onto K: it must equal the 6:8-pruned W
+    recon = np.zeros((12, 64), dtype=np.uint16)
+    rows, cols = np.nonzero(d["emask"])
+    recon[rows, d["src"][rows, cols]] = d["expanded"][rows, cols]
+    assert (recon == np.where(d["mask68"], w, 0)).all()
+    assert (O.decompress24(d["values"], d["meta"], 96) == d["expanded"]).all()
+    x = WL.random_bits((5, 64), 41)
+    xv = O.bf16_to_f32(x).astype(np.float64)
+    xl = xv[:, O.lift_columns(64)]
+    y_lift, _ = O.gemm_ref(xl, O.bf16_to_f32(d["expanded"]))
+    y_68, _ = O.gemm_ref(xv, O.bf16_to_f32(np.where(d["mask68"], w, 0)))
+    assert np.array_equal(y_lift, y_68)
+
+
+def test_slide68_golden_hand_example():
+    path = os.path.join(GOLDEN, "slide68_hand_example.txt")
+    lines = [ln for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    kept = [int(t) for t in lines[0].split()]
+    want = [tuple(int(t) for t in ln.split()) for ln in lines[1:4]]
+    m = np.zeros(8, dtype=bool)
+    m[kept] = True
+    assert O.window_assignment(m) == want
+    want_cols = [int(t) for t in lines[4].split()]
+    assert O.lift_columns(8).tolist() == want_cols
+
+
+def test_lift_codes_are_gathered_codes_and_ratios():
+    x = WL.random_bits((6, 64), 50)
+    lifted, s = O.slide68_lift(x)
+    codes, s2 = O.quantize_pertensor(x)
+    assert s == s2 and (lifted == codes[:, O.lift_columns(64)]).all()
+    assert lifted.shape[1] / x.shape[1] == 1.5           # gamma = (2N-2)/N for N = 4
+    # dense-equivalent work ratio of 6:8-through-2:4 vs dense: 1.5 / 2 = 0.75 -> S_max 4/3
+    assert (1.5 * 0.5) == 0.75 and abs(1 / 0.75 - 4 / 3) < 1e-12

@@ -1,0 +1,195 @@
+/*
+ * sp24.h -- C ABI of the B200 (sm_100a) 2:4 structured-sparse FP8 GEMM library.
+ *
+ * The library implements the hot path of 2:4 structured sparsity with FP8
+ * for the linear and FFN layers of an LLM:
+ *   1. magnitude 2:4 pruning along K, ties to the lower index
+ *      ("Deploying 2:4 Sparsity with FP8 on Hopper: A Production Cookbook",
+ *       pipeline step 4 and Practical Example 1);
+ *   2. compression into an [N, K/2] values array plus 2-bit index metadata
+ *      (the cookbook, pipeline step 2; "La Densite Dynamique et les Noyaux
+ *       Non Structures", §Lacunes des noyaux);
+ *   3. per-tensor dynamic E4M3 quantisation with scale = amax / 448
+ *      (the cookbook, pipeline steps 3 and 6);
+ *   4. the sparse GEMM Y[M,N] = X[M,K] . W^T with fp32 accumulation, both
+ *      scales applied and bf16 output;
+ * and the (2N-2):2N extension for 6:8 ("SlideSparse: Fast and Flexible
+ * (2N-2):2N Structured Sparsity", Resumen tecnico §2 Metodologia): each
+ * 8-group is split into three overlapping stride-2 windows that are each
+ * 2:4 over a lifted K' = 1.5 K, and the activation lift is fused into the
+ * FP8 quantisation pass.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *   never allocates.  Matrices are row-major with K contiguous.  Every
+ *   tensor pointer must be 16-byte aligned (SP24_ERR_ALIGN otherwise).
+ * - bf16 tensors are IEEE bfloat16 bit patterns (uint16); E4M3 tensors are
+ *   OCP FP8 E4M3 ("FN": no infinities, 0x7F/0xFF = NaN, max 448) bytes.
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL means the
+ *   legacy default stream) and returns an int status (SP24_OK or a negative
+ *   SP24_ERR_*).  Arguments are validated on the host before any launch;
+ *   there is no silent dense or CPU fallback.
+ * - Scales are device floats (dequantisation scales: real = code * scale), so
+ *   dynamic scaling never forces a host synchronisation.
+ * - `workspace` is device scratch of at least sp24_workspace_size(...)
+ *   bytes (never less than 256).  It must be zero-filled before its FIRST
+ *   use.  Its first 256 bytes (and, for a split-K GEMM, its tile counters)
+ *   hold counters that every call returns to zero; the rest is scratch that
+ *   a call rewrites before reading.  So one buffer can serve any sequence of
+ *   calls, as long as calls sharing it never run concurrently.
+ * - `status` (nullable) is a device int32 that kernels OR error bits into:
+ *   SP24_STATUS_NONFINITE when an input holds NaN/Inf (the method is defined
+ *   for finite inputs only).  Read it after synchronising the stream.
+ * - The library is for sm_100a (B200).  On any other device the entry
+ *   points return SP24_ERR_ARCH.
+ *
+ * Compressed weight layout (shared by every GEMM entry point)
+ * ------------------------------------------------------------
+ *   values[n, 2g + t] = t-th kept element (ascending index) of group g of row n
+ *   meta[n, b]        = nibble(2b) | nibble(2b + 1) << 4
+ *   nibble(g)         = i0 | i1 << 2, 0 <= i0 < i1 <= 3, the in-group indices
+ *                       of the two kept elements of group g.
+ */
+#ifndef SP24_H
+#define SP24_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *sp24_stream_t; /* identical to cudaStream_t */
+
+/* Return codes */
+#define SP24_OK 0
+#define SP24_ERR_NULL (-1)      /* a required pointer is NULL */
+#define SP24_ERR_SHAPE (-2)     /* a dimension breaks the shape rules of the call */
+#define SP24_ERR_ALIGN (-3)     /* a pointer is not 16-byte aligned */
+#define SP24_ERR_DTYPE (-4)     /* unknown dtype code */
+#define SP24_ERR_CUDA (-5)      /* CUDA launch/runtime error, see sp24_last_cuda_error() */
+#define SP24_ERR_WORKSPACE (-6) /* workspace missing or smaller than required */
+#define SP24_ERR_ARCH (-7)      /* current device is not sm_100 */
+
+/* Device status bits (OR-ed into *status by the kernels) */
+#define SP24_STATUS_NONFINITE 1 /* an input element was NaN or Inf */
+#define SP24_STATUS_TIMEOUT 2   /* a pipeline wait hit its iteration limit */
+
+/* dtype codes */
+#define SP24_DTYPE_E4M3 0
+#define SP24_DTYPE_BF16 1
+
+/* op codes for sp24_workspace_size */
+#define SP24_OP_QUANTIZE 0
+#define SP24_OP_PRUNE_COMPRESS 1
+#define SP24_OP_SLIDE68_DECOMPOSE 2
+#define SP24_OP_SLIDE68_LIFT 3
+#define SP24_OP_GEMM 4
+#define SP24_OP_GEMM_DENSE 5
+
+/*
+ * Weight path, 2:4.  W: bf16 [N, K].  For every row and every group of 4
+ * contiguous K-values the two largest |w| are kept (equal magnitudes go to the
+ * lower index; -0 equals +0).  Pruning ranks the bf16 magnitudes before any
+ * quantisation.
+ *   out_dtype = SP24_DTYPE_E4M3: w_scale <- amax|W| / 448 (1.0 when amax = 0),
+ *     values <- E4M3(w / w_scale) of the kept elements (u8 [N, K/2]; the
+ *     quotient is one correctly rounded fp32 division, then round to nearest
+ *     even with saturation to +-448), pruned_dense (nullable) <- u8 [N, K]
+ *     with the same codes at kept positions and 0x00 elsewhere.
+ *   out_dtype = SP24_DTYPE_BF16: values <- the kept bf16 values (u16 [N, K/2]),
+ *     w_scale is ignored (may be NULL), pruned_dense (nullable) <- bf16 [N, K].
+ * meta <- u8 [N, K/8] in the layout above.
+ * Shape rules: N >= 1, K >= 8, K % 8 == 0.
+ */
+int sp24_prune_compress(const void *W, int N, int K, int out_dtype, void *values,
+                        uint8_t *meta, float *w_scale, void *pruned_dense, void *workspace,
+                        size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+
+/*
+ * Per-tensor dynamic E4M3 quantisation (the cookbook, pipeline step 3).
+ * X: bf16 [rows, cols] -> q: u8 [rows, cols], scale <- amax|X| / 448 (1.0 when
+ * amax = 0), q = E4M3(x / scale) as above.  Also used for the weights of the
+ * dense FP8 comparison GEMM.  Shape rules: rows >= 1, cols >= 1, cols % 16 == 0.
+ */
+int fp8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, uint8_t *q, float *scale,
+                           void *workspace, size_t ws_bytes, int32_t *status,
+                           sp24_stream_t stream);
+
+/*
+ * Weight path, 6:8 through 2:4 windows (SlideSparse, §2 "Descomposicion de
+ * Ventana Deslizante").  W: bf16 [N, K].  Each group of 8 contiguous K-values
+ * keeps its six largest |w| (ties to the lower index).  Window j = 0, 1, 2 of
+ * group g covers positions 2j .. 2j+3; in that order each window takes the two
+ * lowest-index kept positions in its range not taken by an earlier window.  A
+ * position p taken by window j goes to expanded column 12g + 4j + (p - 2j) of
+ * W' [N, K' = 3K/2], which is then 2:4 and stored compressed:
+ * values [N, 3K/4] (E4M3 codes with w_scale as for 2:4, or bf16) and
+ * meta [N, 3K/16].  Shape rules: N >= 1, K % 16 == 0.
+ */
+int slide68_decompose(const void *W, int N, int K, int out_dtype, void *values, uint8_t *meta,
+                      float *w_scale, void *workspace, size_t ws_bytes, int32_t *status,
+                      sp24_stream_t stream);
+
+/*
+ * Activation lift fused with per-tensor E4M3 quantisation (SlideSparse, §2
+ * "Levantamiento de Activacion").  X: bf16 [M, K] -> q_lifted: u8 [M, 3K/2]
+ * with q_lifted[m, 12g + 4j + r] = E4M3(X[m, 8g + 2j + r] / scale), scale <-
+ * amax|X| / 448.  Shape rules: M >= 1, K % 16 == 0.
+ */
+int slide68_lift(const void *X, int M, int K, uint8_t *q_lifted, float *scale, void *workspace,
+                 size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+
+/*
+ * Sparse GEMM Y[M, N] = bf16( x_scale * w_scale * sum_k X[m, k] * W[n, k] ),
+ * accumulated in fp32 over the kept K positions only, on the 5th-generation
+ * tensor cores (sparse tcgen05 MMA, accumulators in tensor memory).
+ *   dtype = SP24_DTYPE_E4M3: Xq u8 [M, K], w_values u8 [N, K/2] (E4M3), scales
+ *     are device floats (NULL means 1.0).
+ *   dtype = SP24_DTYPE_BF16: Xq bf16 [M, K], w_values bf16 [N, K/2], scales
+ *     ignored (may be NULL).
+ * w_meta u8 [N, K/8]; Y bf16 [M, N].  K is the K of the compressed operand
+ * (for 6:8 weights pass K' = 3K/2 and the lifted activations).
+ * Shape rules: M >= 1, N % 128 == 0, K % 128 == 0 (E4M3) or K % 64 == 0 (BF16).
+ * Y must not alias any input.
+ */
+int sp24_gemm(const void *Xq, const float *x_scale, const void *w_values, const uint8_t *w_meta,
+              const float *w_scale, void *Y, int M, int N, int K, int dtype, void *workspace,
+              size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+
+/*
+ * Dense FP8 GEMM of the same kernel family (comparison baseline for the
+ * sparse speedup): Y[M, N] = bf16( x_scale * w_scale * sum_k Xq[m,k] Wq[n,k] )
+ * with Xq u8 [M, K], Wq u8 [N, K] (E4M3, e.g. the pruned_dense output of
+ * sp24_prune_compress).  Shape rules: M >= 1, N % 128 == 0, K % 128 == 0.
+ */
+int fp8_gemm_dense(const uint8_t *Xq, const float *x_scale, const uint8_t *Wq,
+                   const float *w_scale, void *Y, int M, int N, int K, void *workspace,
+                   size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+
+/* Bytes of workspace the op needs for these sizes (0 is a valid answer). */
+size_t sp24_workspace_size(int op, int64_t M, int64_t N, int64_t K, int dtype);
+
+/* Human-readable text for a return code. */
+const char *sp24_status_str(int code);
+
+/* The last cudaError_t seen by a call that returned SP24_ERR_CUDA (per thread). */
+int sp24_last_cuda_error(void);
+
+/*
+ * Test hook: E4M3 encoding of fp32 values with the same device routine the
+ * quantisation kernels use (round to nearest even, saturate to +-448, sign of
+ * zero kept).  v: f32 [n] -> out: u8 [n].  n >= 0.
+ */
+int sp24_debug_e4m3_encode(const float *v, uint8_t *out, int64_t n, sp24_stream_t stream);
+
+/* Library version string. */
+const char *sp24_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SP24_H */

@@ -1,0 +1,200 @@
+"""B200-native 2:4 structured-sparse FP8 GEMM.
+
+Thin Python binding over the C ABI in ``include/sp24.h``: every function
+below only allocates output tensors with torch (device memory plumbing),
+marshals pointers and the current CUDA stream, and calls into
+``libsp24.so``.  All arithmetic runs in the library's sm_100a kernels.
+
+Entry points (same names as the C ABI):
+    sp24_prune_compress, fp8_quantize_pertensor, slide68_decompose,
+    slide68_lift, sp24_gemm, fp8_gemm_dense
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+from ._lib import DTYPE_BF16, DTYPE_E4M3, Sp24Error  # noqa: F401
+
+__all__ = [
+    "sp24_prune_compress", "fp8_quantize_pertensor", "slide68_decompose", "slide68_lift",
+    "sp24_gemm", "fp8_gemm_dense", "Workspace", "Sp24Error", "DTYPE_E4M3", "DTYPE_BF16",
+]
+
+_DT = {"e4m3": DTYPE_E4M3, "bf16": DTYPE_BF16, DTYPE_E4M3: DTYPE_E4M3, DTYPE_BF16: DTYPE_BF16}
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise Sp24Error("tensors must be contiguous CUDA tensors")
+
+
+class Workspace:
+    """Zero-filled device scratch shared by calls on one stream.
+
+    Every library call leaves its workspace zero-filled, so a buffer can be
+    reused by calls that do not run concurrently (one Workspace per stream).
+    """
+
+    _by_key: dict = {}
+
+    def __init__(self, device):
+        self.device = torch.device(device)
+        self.buf = torch.zeros(4096, dtype=torch.uint8, device=self.device)
+
+    def get(self, nbytes: int):
+        if nbytes > self.buf.numel():
+            self.buf = torch.zeros(max(nbytes, 2 * self.buf.numel()), dtype=torch.uint8,
+                                   device=self.device)
+        return self.buf
+
+    @classmethod
+    def for_current_stream(cls, device) -> "Workspace":
+        device = torch.device(device)
+        key = (device.index, _stream(device))
+        ws = cls._by_key.get(key)
+        if ws is None:
+            ws = cls._by_key[key] = cls(device)
+        return ws
+
+
+def _ws(device, op, m, n, k, dtype=DTYPE_E4M3, workspace=None):
+    lib = _lib.load()
+    need = lib.sp24_workspace_size(op, m, n, k, dtype)
+    ws = workspace or Workspace.for_current_stream(device)
+    buf = ws.get(max(need, 256))
+    return buf, buf.numel()
+
+
+def sp24_prune_compress(W: torch.Tensor, out_dtype="e4m3", pruned_dense: bool = False,
+                        status: torch.Tensor | None = None, workspace: Workspace | None = None):
+    """2:4 magnitude prune + (E4M3 quantise) + compress of W bf16 [N, K].
+
+    Returns dict(values, meta, scale, pruned_dense).
+    """
+    lib = _lib.load()
+    _require_cuda(W, status)
+    if W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise Sp24Error("W must be a 2-D bf16 tensor")
+    dt = _DT[out_dtype]
+    N, K = W.shape
+    vdt = torch.uint8 if dt == DTYPE_E4M3 else torch.bfloat16
+    values = torch.empty((N, K // 2), dtype=vdt, device=W.device)
+    meta = torch.empty((N, K // 8), dtype=torch.uint8, device=W.device)
+    scale = torch.empty((1,), dtype=torch.float32, device=W.device) if dt == DTYPE_E4M3 else None
+    dense = torch.empty((N, K), dtype=vdt, device=W.device) if pruned_dense else None
+    ws, wsn = _ws(W.device, _lib.OP_PRUNE_COMPRESS, 0, N, K, dt, workspace)
+    rc = lib.sp24_prune_compress(_ptr(W), N, K, dt, _ptr(values), _ptr(meta), _ptr(scale),
+                                 _ptr(dense), _ptr(ws), wsn, _ptr(status), _stream(W.device))
+    _lib.check(rc, "sp24_prune_compress")
+    return dict(values=values, meta=meta, scale=scale, pruned_dense=dense)
+
+
+def fp8_quantize_pertensor(X: torch.Tensor, status: torch.Tensor | None = None,
+                           out: torch.Tensor | None = None, scale: torch.Tensor | None = None,
+                           workspace: Workspace | None = None):
+    """Per-tensor E4M3 quantisation of X bf16 [rows, cols] -> (codes u8, scale f32[1])."""
+    lib = _lib.load()
+    _require_cuda(X, status, out, scale)
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise Sp24Error("X must be a 2-D bf16 tensor")
+    rows, cols = X.shape
+    q = out if out is not None else torch.empty((rows, cols), dtype=torch.uint8, device=X.device)
+    s = scale if scale is not None else torch.empty((1,), dtype=torch.float32, device=X.device)
+    ws, wsn = _ws(X.device, _lib.OP_QUANTIZE, rows, 0, cols, DTYPE_E4M3, workspace)
+    rc = lib.fp8_quantize_pertensor(_ptr(X), rows, cols, _ptr(q), _ptr(s), _ptr(ws), wsn,
+                                    _ptr(status), _stream(X.device))
+    _lib.check(rc, "fp8_quantize_pertensor")
+    return q, s
+
+
+def slide68_decompose(W: torch.Tensor, out_dtype="e4m3", status: torch.Tensor | None = None,
+                      workspace: Workspace | None = None):
+    """6:8 prune + sliding-window decomposition of W bf16 [N, K] into 2:4 over K' = 1.5 K."""
+    lib = _lib.load()
+    _require_cuda(W, status)
+    if W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise Sp24Error("W must be a 2-D bf16 tensor")
+    dt = _DT[out_dtype]
+    N, K = W.shape
+    vdt = torch.uint8 if dt == DTYPE_E4M3 else torch.bfloat16
+    values = torch.empty((N, 3 * K // 4), dtype=vdt, device=W.device)
+    meta = torch.empty((N, 3 * K // 16), dtype=torch.uint8, device=W.device)
+    scale = torch.empty((1,), dtype=torch.float32, device=W.device) if dt == DTYPE_E4M3 else None
+    ws, wsn = _ws(W.device, _lib.OP_SLIDE68_DECOMPOSE, 0, N, K, dt, workspace)
+    rc = lib.slide68_decompose(_ptr(W), N, K, dt, _ptr(values), _ptr(meta), _ptr(scale), _ptr(ws),
+                               wsn, _ptr(status), _stream(W.device))
+    _lib.check(rc, "slide68_decompose")
+    return dict(values=values, meta=meta, scale=scale)
+
+
+def slide68_lift(X: torch.Tensor, status: torch.Tensor | None = None,
+                 out: torch.Tensor | None = None, scale: torch.Tensor | None = None,
+                 workspace: Workspace | None = None):
+    """Quantise X bf16 [M, K] to E4M3 and lift it to [M, 1.5 K] -> (codes, scale)."""
+    lib = _lib.load()
+    _require_cuda(X, status, out, scale)
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise Sp24Error("X must be a 2-D bf16 tensor")
+    M, K = X.shape
+    q = out if out is not None else torch.empty((M, 3 * K // 2), dtype=torch.uint8, device=X.device)
+    s = scale if scale is not None else torch.empty((1,), dtype=torch.float32, device=X.device)
+    ws, wsn = _ws(X.device, _lib.OP_SLIDE68_LIFT, M, 0, K, DTYPE_E4M3, workspace)
+    rc = lib.slide68_lift(_ptr(X), M, K, _ptr(q), _ptr(s), _ptr(ws), wsn, _ptr(status),
+                          _stream(X.device))
+    _lib.check(rc, "slide68_lift")
+    return q, s
+
+
+def sp24_gemm(xq: torch.Tensor, x_scale, values: torch.Tensor, meta: torch.Tensor, w_scale,
+              dtype="e4m3", out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+              workspace: Workspace | None = None):
+    """Sparse GEMM Y[M, N] = bf16(sx * sw * Xq . W^T) with W 2:4-compressed."""
+    lib = _lib.load()
+    _require_cuda(xq, x_scale, values, meta, w_scale, out, status)
+    dt = _DT[dtype]
+    M, K = xq.shape
+    N = values.shape[0]
+    if values.shape[1] * 2 != K or meta.shape != (N, K // 8):
+        raise Sp24Error("operand shapes disagree")
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    ws, wsn = _ws(xq.device, _lib.OP_GEMM, M, N, K, dt, workspace)
+    rc = lib.sp24_gemm(_ptr(xq), _ptr(x_scale), _ptr(values), _ptr(meta), _ptr(w_scale), _ptr(y),
+                       M, N, K, dt, _ptr(ws), wsn, _ptr(status), _stream(xq.device))
+    _lib.check(rc, "sp24_gemm")
+    return y
+
+
+def fp8_gemm_dense(xq: torch.Tensor, x_scale, wq: torch.Tensor, w_scale,
+                   out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                   workspace: Workspace | None = None):
+    """Dense FP8 GEMM of the same kernel family (sparse-speedup baseline)."""
+    lib = _lib.load()
+    _require_cuda(xq, x_scale, wq, w_scale, out, status)
+    M, K = xq.shape
+    N = wq.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    ws, wsn = _ws(xq.device, _lib.OP_GEMM_DENSE, M, N, K, DTYPE_E4M3, workspace)
+    rc = lib.fp8_gemm_dense(_ptr(xq), _ptr(x_scale), _ptr(wq), _ptr(w_scale), _ptr(y), M, N, K,
+                            _ptr(ws), wsn, _ptr(status), _stream(xq.device))
+    _lib.check(rc, "fp8_gemm_dense")
+    return y
+
+
+def debug_e4m3_encode(v: torch.Tensor) -> torch.Tensor:
+    """E4M3 codes of fp32 values via the kernels' own device routine (test hook)."""
+    lib = _lib.load()
+    _require_cuda(v)
+    out = torch.empty(v.shape, dtype=torch.uint8, device=v.device)
+    _lib.check(lib.sp24_debug_e4m3_encode(_ptr(v), _ptr(out), v.numel(), _stream(v.device)),
+               "sp24_debug_e4m3_encode")
+    return out

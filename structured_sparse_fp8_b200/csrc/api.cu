@@ -1,0 +1,209 @@
+// api.cu -- the extern "C" entry points declared in include/sp24.h: argument
+// validation on the host, workspace bookkeeping and kernel launches.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kernels.h"
+#include "sp24.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices];
+int g_arch_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 not sm_100
+
+// SM count of the current device, or -1 when the device is not sm_100.
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  if (g_arch_ok[dev] == 0) {
+    int major = 0, minor = 0, sms = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    g_sm_count[dev] = sms;
+    g_arch_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  return g_arch_ok[dev] == 1 ? g_sm_count[dev] : -1;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SP24_OK;
+  g_last_cuda_error = static_cast<int>(e);
+  return SP24_ERR_CUDA;
+}
+
+// Runs the amax reduction, which also writes the per-tensor scale.
+int amax_then(const void *x, int64_t nelem, void *workspace, size_t ws_bytes, float *scale,
+              int32_t *status, int sms, cudaStream_t st) {
+  if (!workspace) return SP24_ERR_WORKSPACE;
+  if (ws_bytes < sp24::kAmaxWorkspaceBytes) return SP24_ERR_WORKSPACE;
+  return cuda_status(sp24::launch_amax_scale(x, nelem, static_cast<uint32_t *>(workspace), scale,
+                                             status, sms, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sp24_version(void) { return "sp24 0.1 (sm_100a)"; }
+
+int sp24_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char *sp24_status_str(int code) {
+  switch (code) {
+    case SP24_OK: return "ok";
+    case SP24_ERR_NULL: return "a required pointer is NULL";
+    case SP24_ERR_SHAPE: return "a dimension breaks the shape rules of the call";
+    case SP24_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case SP24_ERR_DTYPE: return "unknown dtype";
+    case SP24_ERR_CUDA: return "CUDA error (see sp24_last_cuda_error)";
+    case SP24_ERR_WORKSPACE: return "workspace missing or too small";
+    case SP24_ERR_ARCH: return "the current device is not sm_100 (B200)";
+    default: return "unknown status";
+  }
+}
+
+size_t sp24_workspace_size(int op, int64_t M, int64_t N, int64_t K, int dtype) {
+  switch (op) {
+    case SP24_OP_QUANTIZE:
+    case SP24_OP_PRUNE_COMPRESS:
+    case SP24_OP_SLIDE68_DECOMPOSE:
+    case SP24_OP_SLIDE68_LIFT:
+      return sp24::kAmaxWorkspaceBytes;
+    case SP24_OP_GEMM:
+    case SP24_OP_GEMM_DENSE: {
+      if (M < 1 || N < 128 || K < 128 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return 0;
+      int sms = device_sm_count();
+      if (sms <= 0) sms = 148;
+      const sp24::GemmKind kind =
+          op == SP24_OP_GEMM_DENSE ? sp24::kDenseE4M3
+                                   : (dtype == SP24_DTYPE_BF16 ? sp24::kSparseBF16 : sp24::kSparseE4M3);
+      return sp24::plan_gemm(kind, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sms)
+          .workspace_bytes();
+    }
+    default:
+      return 0;
+  }
+}
+
+int sp24_prune_compress(const void *W, int N, int K, int out_dtype, void *values, uint8_t *meta,
+                        float *w_scale, void *pruned_dense, void *workspace, size_t ws_bytes,
+                        int32_t *status, sp24_stream_t stream) {
+  if (out_dtype != SP24_DTYPE_E4M3 && out_dtype != SP24_DTYPE_BF16) return SP24_ERR_DTYPE;
+  if (!W || !values || !meta) return SP24_ERR_NULL;
+  if (out_dtype == SP24_DTYPE_E4M3 && !w_scale) return SP24_ERR_NULL;
+  if (N < 1 || K < 8 || K % 8 != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(values) || !aligned16(meta) ||
+      (pruned_dense && !aligned16(pruned_dense)))
+    return SP24_ERR_ALIGN;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t nelem = static_cast<int64_t>(N) * K;
+  const bool fp8 = out_dtype == SP24_DTYPE_E4M3;
+  int rc = amax_then(W, nelem, workspace, ws_bytes, fp8 ? w_scale : nullptr, status, sms, st);
+  if (rc != SP24_OK) return rc;
+  return cuda_status(sp24::launch_prune24(W, nelem, fp8, w_scale, values, meta, pruned_dense, sms, st));
+}
+
+int fp8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, uint8_t *q, float *scale,
+                           void *workspace, size_t ws_bytes, int32_t *status,
+                           sp24_stream_t stream) {
+  if (!X || !q || !scale) return SP24_ERR_NULL;
+  if (rows < 1 || cols < 1 || cols % 16 != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(q)) return SP24_ERR_ALIGN;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t nelem = rows * cols;
+  int rc = amax_then(X, nelem, workspace, ws_bytes, scale, status, sms, st);
+  if (rc != SP24_OK) return rc;
+  return cuda_status(sp24::launch_quantize(X, nelem, scale, q, sms, st));
+}
+
+int slide68_decompose(const void *W, int N, int K, int out_dtype, void *values, uint8_t *meta,
+                      float *w_scale, void *workspace, size_t ws_bytes, int32_t *status,
+                      sp24_stream_t stream) {
+  if (out_dtype != SP24_DTYPE_E4M3 && out_dtype != SP24_DTYPE_BF16) return SP24_ERR_DTYPE;
+  if (!W || !values || !meta) return SP24_ERR_NULL;
+  if (out_dtype == SP24_DTYPE_E4M3 && !w_scale) return SP24_ERR_NULL;
+  if (N < 1 || K < 16 || K % 16 != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(values) || !aligned16(meta)) return SP24_ERR_ALIGN;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t nelem = static_cast<int64_t>(N) * K;
+  const bool fp8 = out_dtype == SP24_DTYPE_E4M3;
+  int rc = amax_then(W, nelem, workspace, ws_bytes, fp8 ? w_scale : nullptr, status, sms, st);
+  if (rc != SP24_OK) return rc;
+  return cuda_status(sp24::launch_slide68(W, nelem, fp8, w_scale, values, meta, sms, st));
+}
+
+int slide68_lift(const void *X, int M, int K, uint8_t *q_lifted, float *scale, void *workspace,
+                 size_t ws_bytes, int32_t *status, sp24_stream_t stream) {
+  if (!X || !q_lifted || !scale) return SP24_ERR_NULL;
+  if (M < 1 || K < 16 || K % 16 != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(q_lifted)) return SP24_ERR_ALIGN;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t nelem = static_cast<int64_t>(M) * K;
+  int rc = amax_then(X, nelem, workspace, ws_bytes, scale, status, sms, st);
+  if (rc != SP24_OK) return rc;
+  return cuda_status(sp24::launch_lift_quantize(X, nelem, scale, q_lifted, sms, st));
+}
+
+static int gemm_common(sp24::GemmKind kind, const void *Xq, const float *x_scale,
+                       const void *w_values, const uint8_t *w_meta, const float *w_scale, void *Y,
+                       int M, int N, int K, void *workspace, size_t ws_bytes, int32_t *status,
+                       sp24_stream_t stream) {
+  const bool sparse = kind != sp24::kDenseE4M3;
+  if (!Xq || !w_values || !Y || (sparse && !w_meta)) return SP24_ERR_NULL;
+  const int kmod = kind == sp24::kSparseBF16 ? 64 : 128;
+  if (M < 1 || N < 128 || N % 128 != 0 || K < kmod || K % kmod != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(Xq) || !aligned16(w_values) || !aligned16(Y) || (sparse && !aligned16(w_meta)))
+    return SP24_ERR_ALIGN;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  const sp24::GemmPlan pl = sp24::plan_gemm(kind, M, N, K, sms);
+  if (pl.workspace_bytes() > 0) {
+    if (!workspace || ws_bytes < pl.workspace_bytes()) return SP24_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SP24_ERR_ALIGN;
+  }
+  return cuda_status(sp24::launch_gemm(kind, pl, Xq, x_scale, w_values, w_meta, w_scale, Y, M, N, K,
+                                       workspace, status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sp24_gemm(const void *Xq, const float *x_scale, const void *w_values, const uint8_t *w_meta,
+              const float *w_scale, void *Y, int M, int N, int K, int dtype, void *workspace,
+              size_t ws_bytes, int32_t *status, sp24_stream_t stream) {
+  if (dtype == SP24_DTYPE_E4M3)
+    return gemm_common(sp24::kSparseE4M3, Xq, x_scale, w_values, w_meta, w_scale, Y, M, N, K,
+                       workspace, ws_bytes, status, stream);
+  if (dtype == SP24_DTYPE_BF16)
+    return gemm_common(sp24::kSparseBF16, Xq, nullptr, w_values, w_meta, nullptr, Y, M, N, K,
+                       workspace, ws_bytes, status, stream);
+  return SP24_ERR_DTYPE;
+}
+
+int fp8_gemm_dense(const uint8_t *Xq, const float *x_scale, const uint8_t *Wq,
+                   const float *w_scale, void *Y, int M, int N, int K, void *workspace,
+                   size_t ws_bytes, int32_t *status, sp24_stream_t stream) {
+  return gemm_common(sp24::kDenseE4M3, Xq, x_scale, Wq, nullptr, w_scale, Y, M, N, K, workspace,
+                     ws_bytes, status, stream);
+}
+
+int sp24_debug_e4m3_encode(const float *v, uint8_t *out, int64_t n, sp24_stream_t stream) {
+  if (n < 0) return SP24_ERR_SHAPE;
+  if (n > 0 && (!v || !out)) return SP24_ERR_NULL;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  return cuda_status(sp24::launch_e4m3_encode(v, out, n, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

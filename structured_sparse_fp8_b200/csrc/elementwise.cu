@@ -1,0 +1,398 @@
+// elementwise.cu -- the bandwidth-bound kernels of the path:
+//   * amax + per-tensor scale (one pass, last-block finalisation),
+//   * E4M3 quantisation of activations (and the fused 6:8 lift),
+//   * 2:4 magnitude prune + quantise + compress of weights,
+//   * 6:8 prune + sliding-window decomposition of weights.
+// All of them read 16-byte vectors with streaming loads and use grid-stride
+// loops over a grid sized to the SM count.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kernels.h"
+#include "sp24.h"
+
+namespace sp24 {
+
+// ----------------------------------------------------------------- helpers
+
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t h) { return __uint_as_float(h << 16); }
+
+// E4M3 code of one fp32 value: round to nearest even, saturate to +-448, and
+// keep the sign of a value that rounds to zero (code 0x80 for negatives).
+__device__ __forceinline__ uint32_t e4m3_code(float v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+  uint32_t c = r & 0xFFu;
+  return c | ((__float_as_uint(v) >> 24) & 0x80u);
+}
+
+// Code of the bf16 value h divided by the dequantisation scale s (one
+// correctly rounded fp32 division, as in the definition).
+__device__ __forceinline__ uint32_t quant_bf16(uint32_t h, float s) {
+  return e4m3_code(__fdiv_rn(bf16_bits_to_float(h), s));
+}
+
+// Largest magnitude bit pattern among the 8 bf16 values of a 16-byte vector.
+// For finite bf16 the unsigned order of (bits & 0x7FFF) is the order of |x|;
+// NaN/Inf patterns (>= 0x7F80) sort above every finite value.
+__device__ __forceinline__ uint32_t absmax8(uint4 v) {
+  const uint32_t m = 0x7FFF7FFFu;
+  uint32_t a = __vmaxu2(__vmaxu2(v.x & m, v.y & m), __vmaxu2(v.z & m, v.w & m));
+  return max(a & 0xFFFFu, a >> 16);
+}
+
+// ----------------------------------------------------------------- amax
+
+// ws[0]: running max of |x| bits, ws[1]: finished-block ticket.  The last
+// block to finish turns the max into the scale amax/448 (1.0 for amax == 0),
+// flags non-finite input and re-zeroes ws.
+__global__ void __launch_bounds__(256) amax_scale_kernel(const uint4 *__restrict__ x, int64_t nvec,
+                                                         uint32_t *ws, float *scale_out,
+                                                         int32_t *status) {
+  uint32_t m = 0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec;
+       i += stride)
+    m = max(m, absmax8(ld_stream(x + i)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ uint32_t part[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) part[warp] = m;
+  __syncthreads();
+  if (warp == 0) {
+    m = lane < (blockDim.x >> 5) ? part[lane] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) {
+      atomicMax(&ws[0], m);
+      __threadfence();
+      const uint32_t ticket = atomicAdd(&ws[1], 1u);
+      if (ticket == gridDim.x - 1) {
+        __threadfence();
+        const uint32_t a = atomicOr(&ws[0], 0u);
+        if (a >= 0x7F80u && status) atomicOr(status, SP24_STATUS_NONFINITE);
+        const float amax = bf16_bits_to_float(a);
+        if (scale_out) *scale_out = (a == 0u) ? 1.0f : __fdiv_rn(amax, 448.0f);
+        ws[0] = 0u;
+        ws[1] = 0u;
+        __threadfence();
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------------------- quantise
+
+// 16 bf16 -> 16 E4M3 codes per iteration (two 16-byte loads, one store).
+__global__ void __launch_bounds__(256) quantize_kernel(const uint4 *__restrict__ x, int64_t n16,
+                                                       const float *__restrict__ scale,
+                                                       uint4 *__restrict__ q) {
+  const float s = *scale;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += stride) {
+    const uint4 a = ld_stream(x + 2 * i), b = ld_stream(x + 2 * i + 1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t lo = w[2 * j], hi = w[2 * j + 1];
+      o[j] = quant_bf16(lo & 0xFFFFu, s) | (quant_bf16(lo >> 16, s) << 8) |
+             (quant_bf16(hi & 0xFFFFu, s) << 16) | (quant_bf16(hi >> 16, s) << 24);
+    }
+    q[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// Fused quantise + 6:8 lift.  Each thread takes 16 consecutive values of a
+// row (two 8-groups) and writes the 24 lifted codes
+//   out[12*gl + 4*j + r] = E4M3(x[8*gl + 2*j + r] / s),  gl in {0,1}.
+__global__ void __launch_bounds__(256) lift_quantize_kernel(const uint4 *__restrict__ x,
+                                                            int64_t n16,
+                                                            const float *__restrict__ scale,
+                                                            uint2 *__restrict__ q) {
+  const float s = *scale;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += stride) {
+    const uint4 a = ld_stream(x + 2 * i), b = ld_stream(x + 2 * i + 1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t c[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      c[2 * j] = quant_bf16(w[j] & 0xFFFFu, s);
+      c[2 * j + 1] = quant_bf16(w[j] >> 16, s);
+    }
+    uint32_t out[6];
+#pragma unroll
+    for (int o = 0; o < 6; ++o) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int b8 = 0; b8 < 4; ++b8) {
+        const int t = 4 * o + b8;  // lifted index within the 24
+        const int gl = t / 12, j = (t % 12) / 4, r = t % 4;
+        word |= c[8 * gl + 2 * j + r] << (8 * b8);
+      }
+      out[o] = word;
+    }
+    uint2 *dst = q + 3 * i;
+    dst[0] = make_uint2(out[0], out[1]);
+    dst[1] = make_uint2(out[2], out[3]);
+    dst[2] = make_uint2(out[4], out[5]);
+  }
+}
+
+// ----------------------------------------------------------------- 2:4 prune
+
+// Kept-position mask (4 bits) of one group: element i is kept when fewer than
+// two elements beat it (larger |w|, or equal |w| at a lower index).
+__device__ __forceinline__ uint32_t keep2of4(const uint32_t a[4]) {
+  uint32_t mask = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int beaten = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (j != i) beaten += (a[j] > a[i]) || (a[j] == a[i] && j < i);
+    mask |= (beaten < 2 ? 1u : 0u) << i;
+  }
+  return mask;
+}
+
+// One thread per 8 K-values (two groups, one metadata byte).
+template <bool FP8>
+__global__ void __launch_bounds__(256) prune24_kernel(const uint4 *__restrict__ w, int64_t n8,
+                                                      const float *__restrict__ scale,
+                                                      void *__restrict__ values,
+                                                      uint8_t *__restrict__ meta,
+                                                      void *__restrict__ dense) {
+  const float s = FP8 ? *scale : 1.0f;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += stride) {
+    const uint4 v = ld_stream(w + i);
+    const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+    uint32_t h[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      h[2 * j] = words[j] & 0xFFFFu;
+      h[2 * j + 1] = words[j] >> 16;
+    }
+    uint32_t kept_vals[4];  // bf16 bits or codes of the 4 kept elements
+    uint32_t meta_byte = 0;
+    uint32_t dense_out[8];
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      uint32_t a[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) a[t] = h[4 * g + t] & 0x7FFFu;
+      const uint32_t mk = keep2of4(a);
+      const int i0 = __ffs(mk) - 1;
+      const int i1 = __ffs(mk & (mk - 1)) - 1;
+      meta_byte |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * g);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const uint32_t val = FP8 ? quant_bf16(h[4 * g + t], s) : h[4 * g + t];
+        dense_out[4 * g + t] = ((mk >> t) & 1u) ? val : 0u;
+        if (t == i0) kept_vals[2 * g] = val;
+        if (t == i1) kept_vals[2 * g + 1] = val;
+      }
+    }
+    meta[i] = static_cast<uint8_t>(meta_byte);
+    if (FP8) {
+      reinterpret_cast<uint32_t *>(values)[i] =
+          kept_vals[0] | (kept_vals[1] << 8) | (kept_vals[2] << 16) | (kept_vals[3] << 24);
+      if (dense) {
+        uint2 d;
+        d.x = dense_out[0] | (dense_out[1] << 8) | (dense_out[2] << 16) | (dense_out[3] << 24);
+        d.y = dense_out[4] | (dense_out[5] << 8) | (dense_out[6] << 16) | (dense_out[7] << 24);
+        reinterpret_cast<uint2 *>(dense)[i] = d;
+      }
+    } else {
+      reinterpret_cast<uint2 *>(values)[i] =
+          make_uint2(kept_vals[0] | (kept_vals[1] << 16), kept_vals[2] | (kept_vals[3] << 16));
+      if (dense)
+        reinterpret_cast<uint4 *>(dense)[i] =
+            make_uint4(dense_out[0] | (dense_out[1] << 16), dense_out[2] | (dense_out[3] << 16),
+                       dense_out[4] | (dense_out[5] << 16), dense_out[6] | (dense_out[7] << 16));
+    }
+  }
+}
+
+// ----------------------------------------------------------------- 6:8 decompose
+
+// 6:8 keep mask (8 bits): element i is kept when fewer than six elements beat it.
+__device__ __forceinline__ uint32_t keep6of8(const uint32_t a[8]) {
+  uint32_t mask = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int beaten = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j != i) beaten += (a[j] > a[i]) || (a[j] == a[i] && j < i);
+    mask |= (beaten < 6 ? 1u : 0u) << i;
+  }
+  return mask;
+}
+
+// Greedy window assignment: window j (positions 2j..2j+3) takes the two
+// lowest kept positions in its range that no earlier window took.
+// pos[2j], pos[2j+1] receive the positions, ascending.
+__device__ __forceinline__ void assign_windows(uint32_t kept, int pos[6]) {
+  uint32_t left = kept;
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    uint32_t cand = left & (0xFu << (2 * j));
+    const int p0 = __ffs(cand) - 1;
+    cand &= cand - 1;
+    const int p1 = __ffs(cand) - 1;
+    pos[2 * j] = p0;
+    pos[2 * j + 1] = p1;
+    left &= ~((1u << p0) | (1u << p1));
+  }
+}
+
+// One thread per 16 K-values (two 8-groups -> 12 values, 6 nibbles = 3 bytes).
+template <bool FP8>
+__global__ void __launch_bounds__(256) slide68_kernel(const uint4 *__restrict__ w, int64_t n16,
+                                                      const float *__restrict__ scale,
+                                                      void *__restrict__ values,
+                                                      uint8_t *__restrict__ meta) {
+  const float s = FP8 ? *scale : 1.0f;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += stride) {
+    uint32_t vals[12];
+    uint32_t nib[6];
+#pragma unroll
+    for (int gl = 0; gl < 2; ++gl) {
+      const uint4 v = ld_stream(w + 2 * i + gl);
+      const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+      uint32_t h[8], a[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        h[2 * j] = words[j] & 0xFFFFu;
+        h[2 * j + 1] = words[j] >> 16;
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) a[t] = h[t] & 0x7FFFu;
+      int pos[6];
+      assign_windows(keep6of8(a), pos);
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        const int p0 = pos[2 * j], p1 = pos[2 * j + 1];
+        nib[3 * gl + j] = static_cast<uint32_t>((p0 - 2 * j) | ((p1 - 2 * j) << 2));
+        uint32_t h0 = 0, h1 = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (t == p0) h0 = h[t];
+          if (t == p1) h1 = h[t];
+        }
+        vals[6 * gl + 2 * j] = FP8 ? quant_bf16(h0, s) : h0;
+        vals[6 * gl + 2 * j + 1] = FP8 ? quant_bf16(h1, s) : h1;
+      }
+    }
+    uint8_t *mrow = meta + 3 * i;
+    mrow[0] = static_cast<uint8_t>(nib[0] | (nib[1] << 4));
+    mrow[1] = static_cast<uint8_t>(nib[2] | (nib[3] << 4));
+    mrow[2] = static_cast<uint8_t>(nib[4] | (nib[5] << 4));
+    if (FP8) {
+      uint32_t *dst = reinterpret_cast<uint32_t *>(values) + 3 * i;
+#pragma unroll
+      for (int o = 0; o < 3; ++o)
+        dst[o] = vals[4 * o] | (vals[4 * o + 1] << 8) | (vals[4 * o + 2] << 16) |
+                 (vals[4 * o + 3] << 24);
+    } else {
+      uint2 *dst = reinterpret_cast<uint2 *>(values) + 3 * i;
+#pragma unroll
+      for (int o = 0; o < 3; ++o)
+        dst[o] = make_uint2(vals[4 * o] | (vals[4 * o + 1] << 16),
+                            vals[4 * o + 2] | (vals[4 * o + 3] << 16));
+    }
+  }
+}
+
+// ----------------------------------------------------------------- test hook
+__global__ void e4m3_encode_kernel(const float *__restrict__ v, uint8_t *__restrict__ out,
+                                   int64_t n) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += stride)
+    out[i] = static_cast<uint8_t>(e4m3_code(v[i]));
+}
+
+// ----------------------------------------------------------------- launchers
+
+static int grid_for(int64_t work, int sm_count) {
+  const int64_t want = (work + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+  return static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
+}
+
+cudaError_t launch_amax_scale(const void *x, int64_t nelem, uint32_t *ws, float *scale,
+                              int32_t *status, int sm_count, cudaStream_t st) {
+  const int64_t nvec = nelem / 8;
+  amax_scale_kernel<<<grid_for(nvec, sm_count), 256, 0, st>>>(
+      static_cast<const uint4 *>(x), nvec, ws, scale, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const void *x, int64_t nelem, const float *scale, uint8_t *q,
+                            int sm_count, cudaStream_t st) {
+  const int64_t n16 = nelem / 16;
+  quantize_kernel<<<grid_for(n16, sm_count), 256, 0, st>>>(static_cast<const uint4 *>(x), n16,
+                                                           scale, reinterpret_cast<uint4 *>(q));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lift_quantize(const void *x, int64_t nelem, const float *scale, uint8_t *q,
+                                 int sm_count, cudaStream_t st) {
+  const int64_t n16 = nelem / 16;
+  lift_quantize_kernel<<<grid_for(n16, sm_count), 256, 0, st>>>(
+      static_cast<const uint4 *>(x), n16, scale, reinterpret_cast<uint2 *>(q));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prune24(const void *w, int64_t nelem, bool fp8, const float *scale,
+                           void *values, uint8_t *meta, void *dense, int sm_count,
+                           cudaStream_t st) {
+  const int64_t n8 = nelem / 8;
+  if (fp8)
+    prune24_kernel<true><<<grid_for(n8, sm_count), 256, 0, st>>>(
+        static_cast<const uint4 *>(w), n8, scale, values, meta, dense);
+  else
+    prune24_kernel<false><<<grid_for(n8, sm_count), 256, 0, st>>>(
+        static_cast<const uint4 *>(w), n8, scale, values, meta, dense);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_slide68(const void *w, int64_t nelem, bool fp8, const float *scale,
+                           void *values, uint8_t *meta, int sm_count, cudaStream_t st) {
+  const int64_t n16 = nelem / 16;
+  if (fp8)
+    slide68_kernel<true><<<grid_for(n16, sm_count), 256, 0, st>>>(
+        static_cast<const uint4 *>(w), n16, scale, values, meta);
+  else
+    slide68_kernel<false><<<grid_for(n16, sm_count), 256, 0, st>>>(
+        static_cast<const uint4 *>(w), n16, scale, values, meta);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_e4m3_encode(const float *v, uint8_t *out, int64_t n, int sm_count,
+                               cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  e4m3_encode_kernel<<<grid_for(n, sm_count), 256, 0, st>>>(v, out, n);
+  return cudaGetLastError();
+}
+
+}  // namespace sp24

@@ -1,0 +1,56 @@
+// kernels.h -- internal launch interface between the C ABI (api.cu) and the
+// kernels (elementwise.cu, gemm.cu).  Not installed; not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sp24 {
+
+// ---- elementwise.cu
+cudaError_t launch_amax_scale(const void *x, int64_t nelem, uint32_t *ws, float *scale,
+                              int32_t *status, int sm_count, cudaStream_t st);
+cudaError_t launch_quantize(const void *x, int64_t nelem, const float *scale, uint8_t *q,
+                            int sm_count, cudaStream_t st);
+cudaError_t launch_lift_quantize(const void *x, int64_t nelem, const float *scale, uint8_t *q,
+                                 int sm_count, cudaStream_t st);
+cudaError_t launch_prune24(const void *w, int64_t nelem, bool fp8, const float *scale,
+                           void *values, uint8_t *meta, void *dense, int sm_count,
+                           cudaStream_t st);
+cudaError_t launch_slide68(const void *w, int64_t nelem, bool fp8, const float *scale,
+                           void *values, uint8_t *meta, int sm_count, cudaStream_t st);
+cudaError_t launch_e4m3_encode(const float *v, uint8_t *out, int64_t n, int sm_count,
+                               cudaStream_t st);
+
+// Bytes of scratch the amax/scale reduction uses (two counters, padded).
+constexpr size_t kAmaxWorkspaceBytes = 256;
+
+// ---- gemm.cu
+enum GemmKind : int { kSparseE4M3 = 0, kDenseE4M3 = 1, kSparseBF16 = 2 };
+
+// How a GEMM call is cut into CTAs: tile shape, split-K factor and the
+// scratch the split-K reduction needs.
+struct GemmPlan {
+  int bn;            // tokens per tile (MMA N)
+  int bk;            // logical K per pipeline stage
+  int tiles_n;       // N / 128
+  int tiles_m;       // ceil(M / bn)
+  int num_kb;        // K / bk
+  int kb_per_split;  // k-blocks per split
+  int splits;        // number of non-empty splits
+  size_t partial_bytes;
+  size_t counter_bytes;
+  size_t workspace_bytes() const { return splits > 1 ? partial_bytes + counter_bytes : 0; }
+};
+
+GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count);
+
+// Launch the tcgen05 GEMM.  `workspace` must hold plan.workspace_bytes()
+// zero-initialised bytes when plan.splits > 1.
+cudaError_t launch_gemm(GemmKind kind, const GemmPlan &plan, const void *xq, const float *x_scale,
+                        const void *w_values, const uint8_t *w_meta, const float *w_scale,
+                        void *y, int M, int N, int K, void *workspace, int32_t *status,
+                        cudaStream_t st);
+
+}  // namespace sp24

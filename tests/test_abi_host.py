@@ -1,0 +1,77 @@
+"""Host-side checks of the C ABI: the library builds, loads and exports every
+function the header declares, and argument validation rejects bad calls
+before anything touches a GPU.  No test here needs a GPU."""
+import ctypes
+
+import pytest
+
+from structured_sparse_fp8_b200 import _lib
+from structured_sparse_fp8_b200 import build as B
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return _lib.load()
+
+
+def test_every_declared_function_is_exported(lib):
+    names = _lib.header_functions()
+    assert len(names) >= 10
+    for name in names:
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks a signature for {name}"
+
+
+def test_status_strings_and_version(lib):
+    assert lib.sp24_status_str(0) == b"ok"
+    for code in range(-7, 0):
+        assert lib.sp24_status_str(code) not in (b"ok", b"unknown status")
+    assert b"sm_100a" in lib.sp24_version()
+
+
+def test_workspace_sizes(lib):
+    for op in range(4):
+        assert lib.sp24_workspace_size(op, 16, 256, 256, 0) == 256
+    # a prefill-sized GEMM fills the machine without split-K: no scratch
+    assert lib.sp24_workspace_size(_lib.OP_GEMM, 4096, 12288, 4096, 0) == 0
+    # a decode-sized GEMM splits K and needs counters + fp32 partial tiles
+    ws = lib.sp24_workspace_size(_lib.OP_GEMM, 1, 11008, 4096, 0)
+    assert ws > 0 and ws % 256 == 0
+    assert lib.sp24_workspace_size(_lib.OP_GEMM, 0, 11008, 4096, 0) == 0
+
+
+FAKE = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: calls fail validation first
+
+
+def test_validation_rejects_bad_arguments_without_a_gpu(lib):
+    ws = 256
+    # null pointers
+    assert lib.sp24_prune_compress(None, 128, 128, 0, FAKE, FAKE, FAKE, None, FAKE, ws, None, None) == _lib.SP24_ERR_NULL
+    assert lib.fp8_quantize_pertensor(FAKE, 4, 32, None, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_NULL
+    assert lib.sp24_gemm(FAKE, None, FAKE, None, None, FAKE, 4, 128, 128, 0, FAKE, ws, None, None) == _lib.SP24_ERR_NULL
+    # dtype
+    assert lib.sp24_prune_compress(FAKE, 128, 128, 7, FAKE, FAKE, FAKE, None, FAKE, ws, None, None) == _lib.SP24_ERR_DTYPE
+    assert lib.sp24_gemm(FAKE, None, FAKE, FAKE, None, FAKE, 4, 128, 128, 9, FAKE, ws, None, None) == _lib.SP24_ERR_DTYPE
+    # shapes: K not a multiple of the group/tile sizes, N not a multiple of 128, empty M
+    assert lib.sp24_prune_compress(FAKE, 128, 12, 0, FAKE, FAKE, FAKE, None, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.slide68_decompose(FAKE, 128, 24, 0, FAKE, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.slide68_lift(FAKE, 0, 64, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.fp8_quantize_pertensor(FAKE, 4, 24, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.sp24_gemm(FAKE, None, FAKE, FAKE, None, FAKE, 4, 128, 192, 0, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.sp24_gemm(FAKE, None, FAKE, FAKE, None, FAKE, 4, 200, 256, 0, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.sp24_gemm(FAKE, None, FAKE, FAKE, None, FAKE, 0, 128, 256, 0, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.fp8_gemm_dense(FAKE, None, FAKE, None, FAKE, 4, 128, 64, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    # alignment
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.fp8_quantize_pertensor(odd, 4, 32, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
+    assert lib.sp24_gemm(FAKE, None, odd, FAKE, None, FAKE, 4, 128, 128, 0, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
+
+
+def test_no_silent_fallback_without_a_sm100_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; the GPU suite covers real calls")
+    # valid arguments on a machine without an sm_100 device: the call must refuse
+    rc = lib.fp8_quantize_pertensor(FAKE, 4, 32, FAKE, FAKE, FAKE, 256, None, None)
+    assert rc == _lib.SP24_ERR_ARCH

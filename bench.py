@@ -1,0 +1,623 @@
+#!/usr/bin/env python
+"""Benchmark of the 2:4 structured-sparse FP8 hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input.
+Default workload (``--workload decode``): the decode-shaped MLP up-projection
+W[11008, 4096] (bf16, N(0, 0.02)) with X[M, 4096] (N(0, 1)) for M in
+{1, 8, 32, 64}.  Each step
+
+  * prunes, quantises and compresses one layer's weights (weight amax +
+    2:4 prune/quantise/compress: ``sp24_prune_compress``), and
+  * for each M: quantises X (``fp8_quantize_pertensor``) and runs the sparse
+    GEMM (``sp24_gemm``) against another layer's compressed weights.
+
+Layers rotate over pools larger than the 126 MB L2 (4 bf16 weight copies,
+8 compressed layers), so every kernel reads weights that were last touched a
+full step earlier: inputs larger than L2, no flush needed.
+
+Timing: W warm-up steps, then exactly K steps captured in one CUDA graph and
+timed with CUDA events on the launching stream, bracketed by a barrier and
+``torch.cuda.synchronize()``; max over ranks.  A second replay of the same K
+steps with an event between every call gives the per-kernel durations used
+for the roofline.  ``e2e`` repeats the K steps eagerly through the public
+API with the step's inputs copied from pinned host memory and the outputs
+read back every step.
+
+``--impl reference`` times the CPU oracle instead (a bounded sample per
+step), on the same metric.  Multi-GPU (torchrun): every rank runs its own
+independent replica of the workload (weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse FP8 GEMM TFLOPS & HBM GB/s vs roofline; speedup over dense FP8"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------- workloads
+# Algorithmic bytes / flops per call (the minimum traffic each op must move).
+
+def bytes_prune24(n, k):
+    return 2 * n * k + n * k // 2 + n * k // 8 + 4
+
+
+def bytes_quant(m, k):
+    return 3 * m * k + 4
+
+
+def bytes_sparse_gemm(m, n, k):
+    return n * k // 2 + n * k // 8 + m * k + 2 * m * n + 8
+
+
+def bytes_dense_gemm(m, n, k):
+    return n * k + m * k + 2 * m * n + 8
+
+
+def bytes_slide68(n, k):
+    return 2 * n * k + 3 * n * k // 4 + 3 * n * k // 16 + 4
+
+
+def bytes_lift(m, k):
+    return 2 * m * k + 3 * m * k // 2 + 4
+
+
+WORKLOADS = {
+    "decode": dict(cfg=2, n=11008, k=4096, ms=(1, 8, 32, 64), pattern="2:4",
+                   name="decode MLP up-proj W[11008,4096], M in {1,8,32,64}, 2:4 FP8 E4M3"),
+    "prefill": dict(cfg=3, n=12288, k=4096, ms=(4096,), pattern="2:4",
+                    name="prefill fused QKV M4096 N12288 K4096, 2:4 FP8 E4M3"),
+    "downproj": dict(cfg=4, n=4096, k=14336, ms=(256,), pattern="2:4",
+                     name="MLP down-proj M256 N4096 K14336, 2:4 FP8 E4M3"),
+    "slide68": dict(cfg=5, n=4096, k=4096, ms=(64, 2048), pattern="6:8",
+                    name="6:8 sliding-window W[4096,4096] K'=6144, M in {64,2048}"),
+}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "structured_sparse_fp8_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return {}
+    d = json.load(open(path))
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return {}
+    return d.get("per_launch_bytes", {})
+
+
+# ---------------------------------------------------------------- ranks
+
+def max_over_ranks(seconds: float, device=None) -> float:
+    """Largest of every rank's measured time (identity on one process)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return seconds
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_gbs(step_bytes: int, steps: int, world: int, seconds: float) -> float:
+    """Whole-job throughput: the bytes every rank processed over the slowest rank's time."""
+    return step_bytes * steps * world / seconds / 1e9
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index, period=0.002):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self.period = period
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - NVML unavailable: report no clocks
+            self.nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        for bit, name in self.REASONS.items():
+            if r & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:  # noqa: BLE001
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self._stop.set()
+            self._t.join()
+            try:
+                self._sample()
+            except Exception:  # noqa: BLE001
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return None
+        busy = [s for s in self.samples]
+        return {"sm_mhz": float(statistics.median(busy)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(busy)}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+class GpuWorkload:
+    """Device buffers, rotating pools and the step for one workload."""
+
+    def __init__(self, wl, device):
+        import torch
+
+        import structured_sparse_fp8_b200 as sp
+        from structured_sparse_fp8_b200 import workloads as WL
+        self.torch, self.sp, self.wl, self.dev = torch, sp, wl, device
+        n, k, ms = wl["n"], wl["k"], wl["ms"]
+        self.n, self.k, self.ms = n, k, ms
+        self.is68 = wl["pattern"] == "6:8"
+        self.kc = k * 3 // 2 if self.is68 else k   # K of the compressed operand
+        w_host = WL.weight_bits(wl["cfg"])
+        self.w_host_pinned = torch.from_numpy(w_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+        w_dev = self.w_host_pinned.to(device)
+        wbytes = n * k * 2
+        self.R_w = max(2, -(-3 * L2_BYTES // wbytes))
+        self.w_pool = [w_dev.clone() for _ in range(self.R_w)]
+        comp_bytes = n * self.kc // 2 + n * self.kc // 8
+        self.R_g = max(2 * len(ms), -(-3 * L2_BYTES // comp_bytes))
+        self.R_g = -(-self.R_g // len(ms)) * len(ms)
+        self.ws = sp.Workspace(device)
+        self.ws.get(max(sp._lib.load().sp24_workspace_size(sp._lib.OP_GEMM, m, n, self.kc, 0) for m in ms) + 4096)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+        def new_comp():
+            return dict(values=torch.empty((n, self.kc // 2), dtype=torch.uint8, device=device),
+                        meta=torch.empty((n, self.kc // 8), dtype=torch.uint8, device=device),
+                        scale=torch.empty((1,), dtype=torch.float32, device=device))
+        self.prune_out = [new_comp() for _ in range(2)]
+        self.weight_op(w_dev, self.prune_out[0])
+        self.g_pool = []
+        for _ in range(self.R_g):
+            c = new_comp()
+            for key in c:
+                c[key].copy_(self.prune_out[0][key])
+            self.g_pool.append(c)
+        self.x_host = {}
+        self.x_dev, self.xq, self.sx, self.y = {}, {}, {}, {}
+        for m in ms:
+            xb = WL.activation_bits(wl["cfg"], m)
+            self.x_host[m] = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+            self.x_dev[m] = self.x_host[m].to(device)
+            self.xq[m] = torch.empty((m, self.kc), dtype=torch.uint8, device=device)
+            self.sx[m] = torch.empty((1,), dtype=torch.float32, device=device)
+            self.y[m] = torch.empty((m, n), dtype=torch.bfloat16, device=device)
+        self.y_host = {m: torch.empty((m, n), dtype=torch.bfloat16).pin_memory() for m in ms}
+        del w_dev
+        torch.cuda.synchronize()
+
+    # one call of each kind -------------------------------------------------
+    def weight_op(self, w, out):
+        if self.is68:
+            return self.sp.slide68_decompose(w, "e4m3", status=self.status, workspace=self.ws, out=out)
+        return self.sp.sp24_prune_compress(w, "e4m3", status=self.status, workspace=self.ws, out=out)
+
+    def act_op(self, m):
+        if self.is68:
+            return self.sp.slide68_lift(self.x_dev[m], status=self.status, out=self.xq[m],
+                                        scale=self.sx[m], workspace=self.ws)
+        return self.sp.fp8_quantize_pertensor(self.x_dev[m], status=self.status, out=self.xq[m],
+                                              scale=self.sx[m], workspace=self.ws)
+
+    def gemm_op(self, m, layer):
+        c = self.g_pool[layer]
+        return self.sp.sp24_gemm(self.xq[m], self.sx[m], c["values"], c["meta"], c["scale"],
+                                 out=self.y[m], status=self.status, workspace=self.ws)
+
+    def ops_of_step(self, s):
+        """(name, callable, algorithmic bytes, flops, kernel launches) of step s."""
+        n, k, kc = self.n, self.k, self.kc
+        ops = []
+        wi = s % self.R_w
+        wname = "slide68_decompose" if self.is68 else "sp24_prune_compress"
+        wbytes = bytes_slide68(n, k) if self.is68 else bytes_prune24(n, k)
+        ops.append((wname, lambda: self.weight_op(self.w_pool[wi], self.prune_out[s % 2]), wbytes, 0, 2))
+        for j, m in enumerate(self.ms):
+            layer = (s * len(self.ms) + j) % self.R_g
+            aname = "slide68_lift" if self.is68 else "fp8_quantize_pertensor"
+            abytes = bytes_lift(m, k) if self.is68 else bytes_quant(m, k)
+            ops.append((aname, (lambda m=m: self.act_op(m)), abytes, 0, 2))
+            ops.append(("sp24_gemm", (lambda m=m, layer=layer: self.gemm_op(m, layer)),
+                        bytes_sparse_gemm(m, n, kc), 2 * m * n * kc, 1))
+        return ops
+
+    def step_bytes(self):
+        return sum(o[2] for o in self.ops_of_step(0))
+
+    def step_launches(self):
+        return sum(o[4] for o in self.ops_of_step(0))
+
+    def capture(self, steps, first, events):
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        evs = []
+        with torch.cuda.graph(g):
+            for s in range(first, first + steps):
+                for (name, fn, nb, fl, nl) in self.ops_of_step(s):
+                    if events:
+                        e0 = torch.cuda.Event(enable_timing=True, external=True)
+                        e1 = torch.cuda.Event(enable_timing=True, external=True)
+                        e0.record()
+                        fn()
+                        e1.record()
+                        evs.append((name, nb, fl, e0, e1))
+                    else:
+                        fn()
+        return g, evs
+
+    # dense FP8 comparison for the GEMM shapes of this workload ------------
+    def dense_compare(self, reps=50):
+        """Sparse GEMM of this workload vs the dense FP8 GEMM of the same
+        layer (dense W[N, K] with X quantised at K), each timed as a CUDA
+        graph of `reps` launches over rotating weight copies."""
+        torch, sp = self.torch, self.sp
+        n, k, kc = self.n, self.k, self.kc
+        out = {}
+        wq, sw = sp.fp8_quantize_pertensor(self.w_pool[0], workspace=self.ws)
+        ndense = max(2, -(-3 * L2_BYTES // (n * k)))
+        dpool = [wq.clone() for _ in range(ndense)]
+        for m in self.ms:
+            xqd, sxd = sp.fp8_quantize_pertensor(self.x_dev[m], workspace=self.ws)
+            res = {}
+            for kind in ("sparse", "dense"):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    for r in range(reps):
+                        if kind == "dense":
+                            sp.fp8_gemm_dense(xqd, sxd, dpool[r % ndense], sw,
+                                              out=self.y[m], workspace=self.ws)
+                        else:
+                            c = self.g_pool[r % self.R_g]
+                            sp.sp24_gemm(self.xq[m], self.sx[m], c["values"], c["meta"], c["scale"],
+                                         out=self.y[m], workspace=self.ws)
+                g.replay()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                g.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                res[kind] = e0.elapsed_time(e1) * 1000.0 / reps
+                del g
+            out[str(m)] = {"sparse_us": round(res["sparse"], 3), "dense_us": round(res["dense"], 3),
+                           "speedup": round(res["dense"] / res["sparse"], 3),
+                           "sparse_gbs": round(bytes_sparse_gemm(m, n, kc) / res["sparse"] / 1e3, 1),
+                           "dense_gbs": round(bytes_dense_gemm(m, n, k) / res["dense"] / 1e3, 1),
+                           "sparse_tflops_dense_equiv": round(2 * m * n * kc / res["sparse"] / 1e6, 2),
+                           "dense_tflops": round(2 * m * n * k / res["dense"] / 1e6, 2)}
+        del dpool
+        return out
+
+    # e2e through the public API with host buffers ---------------------------
+    def e2e(self, steps):
+        torch = self.torch
+        h2d = self.n * self.k * 2 + sum(m * self.k * 2 for m in self.ms)
+        d2h = sum(m * self.n * 2 for m in self.ms)
+        for s in range(2):
+            self._e2e_step(s)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for s in range(steps):
+            self._e2e_step(s)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3, h2d, d2h
+
+    def _e2e_step(self, s):
+        w = self.w_pool[s % self.R_w]
+        w.copy_(self.w_host_pinned, non_blocking=True)
+        for m in self.ms:
+            self.x_dev[m].copy_(self.x_host[m], non_blocking=True)
+        for (name, fn, nb, fl, nl) in self.ops_of_step(s):
+            fn()
+        for m in self.ms:
+            self.y_host[m].copy_(self.y[m], non_blocking=True)
+
+
+def run_gpu(args, wl, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    import __graft_entry__
+    __graft_entry__.build()
+    gw = GpuWorkload(wl, device)
+    peaks = load_peaks()
+
+    # warm-up: W eager steps (first calls set kernel attributes), then graphs
+    for s in range(args.warmup):
+        for op in gw.ops_of_step(s):
+            op[1]()
+    torch.cuda.synchronize()
+    g_warm, _ = gw.capture(args.warmup, 0, events=False)
+    g_timed, _ = gw.capture(args.steps, args.warmup, events=False)
+    g_detail, evs = gw.capture(args.steps, args.warmup, events=True)
+    g_warm.replay()
+    torch.cuda.synchronize()
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        start.record()
+        g_timed.replay()
+        end.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    elapsed = max_over_ranks(start.elapsed_time(end) / 1e3, device)
+
+    # per-call durations (second replay of the same K steps, events between calls)
+    g_detail.replay()
+    torch.cuda.synchronize()
+    per = {}
+    for name, nb, fl, e0, e1 in evs:
+        d = per.setdefault(name, dict(t=0.0, bytes=0, flops=0, n=0))
+        d["t"] += e0.elapsed_time(e1) / 1e3
+        d["bytes"] += nb
+        d["flops"] += fl
+        d["n"] += 1
+    assert int(gw.status.item()) == 0, "device status word set during the benchmark"
+
+    step_bytes = gw.step_bytes()
+    value = aggregate_gbs(step_bytes, args.steps, world, elapsed)
+    detail_total = sum(d["t"] for d in per.values())
+    dominant = max(per, key=lambda k: per[k]["t"])
+    dom = per[dominant]
+    traffic = load_traffic()
+    gemm_flops = per.get("sp24_gemm", {}).get("flops", 0)
+    gemm_t = per.get("sp24_gemm", {}).get("t", 1.0)
+    tensor_bound = wl["ms"][-1] >= 1024 and dominant == "sp24_gemm"
+    if tensor_bound:
+        achieved = dom["flops"] / dom["t"] / 1e12
+        peak = peaks["bf16_tflops"] * 4.0   # 2:4 sparse FP8 = 2 x FP8 = 4 x bf16 (nominal ratio)
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "kernel": dominant, "peak_source": f"{peaks['source']} bf16 burst x4 (2:4 sparse FP8 dense-equivalent)"}
+    else:
+        achieved = dom["bytes"] / dom["t"] / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": round(peak, 1),
+                "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "kernel": dominant, "peak_source": f"{peaks['source']} hbm_gbs"}
+    tr = traffic.get(f"{args.workload}:{dominant}")
+    roof["traffic"] = tr
+    kernels = {k: {"calls": v["n"] // args.steps, "us_per_call": round(v["t"] / v["n"] * 1e6, 3),
+                   "share": round(v["t"] / detail_total, 4),
+                   "gbs": round(v["bytes"] / v["t"] / 1e9, 1),
+                   "frac_hbm": round(v["bytes"] / v["t"] / 1e9 / peaks["hbm_gbs"], 4)}
+               for k, v in per.items()}
+    if gemm_flops:
+        kernels["sp24_gemm"]["tflops"] = round(gemm_flops / gemm_t / 1e12, 2)
+
+    compare = gw.dense_compare() if rank == 0 and not args.no_compare else None
+    e2e_t, h2d, d2h = gw.e2e(args.steps)
+    e2e_t = max_over_ranks(e2e_t, device)
+    del g_timed, g_detail, g_warm
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(elapsed / args.steps * 1e3, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3",
+        "data": "synthetic (seeded, bf16 N(0,0.02) weights / N(0,1) activations; see workloads.py)",
+        "config": {"workload": wl["name"], "n": wl["n"], "k": wl["k"], "m": list(wl["ms"]),
+                   "step": "weight prune/quantise/compress + per-M activation quantise + sparse GEMM",
+                   "algorithmic_bytes_per_step": step_bytes,
+                   "l2": f"inputs larger than L2: rotating pools of {gw.R_w} bf16 weight copies and "
+                         f"{gw.R_g} compressed layers",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof,
+        "kernels": kernels,
+        "sparse_vs_dense": compare,
+        "e2e": {"value": round(aggregate_gbs(step_bytes, args.steps, world, e2e_t), 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": gw.step_launches() * args.steps,
+        "clocks": clocks.summary(),
+        "peaks": peaks,
+    }
+    return line, gw
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample_step(wl, rows, rng_seed, m_cap=64):
+    """One bounded oracle step: the workload's weight op on `rows` rows of W,
+    then for every M (capped at `m_cap` token rows): activation quantisation
+    and the float64 GEMM against those weight rows.  Returns (algorithmic
+    bytes of the sample, seconds)."""
+    from oracle import sp24_oracle as O
+    from structured_sparse_fp8_b200 import workloads as WL
+    k = wl["k"]
+    w = WL.weight_bits(wl["cfg"], n=rows, k=k, layer=rng_seed + 1)
+    xs = {min(m, m_cap): WL.activation_bits(wl["cfg"], m)[:min(m, m_cap)] for m in wl["ms"]}
+    t0 = time.perf_counter()
+    nbytes = 0
+    if wl["pattern"] == "6:8":
+        d = O.slide68_decompose(w, "e4m3")
+        wv = O.e4m3_decode(d["expanded"])
+        sw = d["scale"]
+        nbytes += bytes_slide68(rows, k)
+        kc = 3 * k // 2
+    else:
+        c = O.sp24_prune_compress(w, "e4m3")
+        wv = O.e4m3_decode(O.decompress24(c["values"], c["meta"], k))
+        sw = c["scale"]
+        nbytes += bytes_prune24(rows, k)
+        kc = k
+    for m, x in xs.items():
+        if wl["pattern"] == "6:8":
+            xq, sx = O.slide68_lift(x)
+            nbytes += bytes_lift(m, k)
+        else:
+            xq, sx = O.quantize_pertensor(x)
+            nbytes += bytes_quant(m, k)
+        O.gemm_ref(O.e4m3_decode(xq), wv, sx, sw)
+        nbytes += bytes_sparse_gemm(m, rows, kc)
+    return nbytes, time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, budget_s=10.0, rows=128):
+    total_b, total_t, n = 0, 0.0, 0
+    while total_t < budget_s and n < 200:
+        b, t = oracle_sample_step(wl, rows, n)
+        total_b += b
+        total_t += t
+        n += 1
+    return {"value": round(total_b / total_t / 1e9, 4), "unit": "GB/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{n} oracle steps, each on {rows} of {wl['n']} weight rows and up to 64 "
+                      f"token rows per M, {total_t:.1f} s of CPU work"}
+
+
+def run_reference(args, wl):
+    rows = 64 if wl["ms"][-1] >= 1024 else 128
+    for s in range(args.warmup):
+        oracle_sample_step(wl, rows, s)
+    total_b, total_t = 0, 0.0
+    for s in range(args.steps):
+        b, t = oracle_sample_step(wl, rows, s)
+        total_b += b
+        total_t += t
+    value = total_b / total_t / 1e9
+    cb = {"value": round(value, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+          "sample": f"each step: the oracle on {rows} of {wl['n']} weight rows and up to 64 "
+                    "token rows per M of the workload"}
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_t / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded; see workloads.py)",
+            "config": {"workload": wl["name"], "n": wl["n"], "k": wl["k"], "m": list(wl["ms"]),
+                       "parallelism": "cpu oracle"},
+            "cpu_baseline": cb,
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["sp24", "reference"], default="sp24")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--no-compare", action="store_true", help="skip the dense-FP8 comparison")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, wl)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=__import__("torch").device("cuda", local_rank))
+    line, gw = run_gpu(args, wl, rank, world, local_rank)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

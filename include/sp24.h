@@ -152,7 +152,12 @@ int slide68_lift(const void *X, int M, int K, uint8_t *q_lifted, float *scale, v
  *     ignored (may be NULL).
  * w_meta u8 [N, K/8]; Y bf16 [M, N].  K is the K of the compressed operand
  * (for 6:8 weights pass K' = 3K/2 and the lifted activations).
- * Shape rules: M >= 1, N % 128 == 0, K % 128 == 0 (E4M3) or K % 64 == 0 (BF16).
+ * When there are too few output tiles to fill the GPU, K is split over a
+ * thread-block cluster of up to 8 CTAs whose partial tiles are reduced
+ * through distributed shared memory in a fixed order (deterministic output).
+ * The GEMMs use no workspace: sp24_workspace_size() returns 0 and
+ * `workspace` may be NULL.
+ * Shape rules: M >= 1, N % 128 == 0, K % 128 == 0 (both dtypes).
  * Y must not alias any input.
  */
 int sp24_gemm(const void *Xq, const float *x_scale, const void *w_values, const uint8_t *w_meta,

@@ -76,10 +76,12 @@ def _ws(device, op, m, n, k, dtype=DTYPE_E4M3, workspace=None):
 
 
 def sp24_prune_compress(W: torch.Tensor, out_dtype="e4m3", pruned_dense: bool = False,
-                        status: torch.Tensor | None = None, workspace: Workspace | None = None):
+                        status: torch.Tensor | None = None, workspace: Workspace | None = None,
+                        out: dict | None = None):
     """2:4 magnitude prune + (E4M3 quantise) + compress of W bf16 [N, K].
 
-    Returns dict(values, meta, scale, pruned_dense).
+    Returns dict(values, meta, scale, pruned_dense); ``out`` may supply any
+    of these tensors preallocated.
     """
     lib = _lib.load()
     _require_cuda(W, status)
@@ -87,11 +89,23 @@ def sp24_prune_compress(W: torch.Tensor, out_dtype="e4m3", pruned_dense: bool = 
         raise Sp24Error("W must be a 2-D bf16 tensor")
     dt = _DT[out_dtype]
     N, K = W.shape
+    out = out or {}
     vdt = torch.uint8 if dt == DTYPE_E4M3 else torch.bfloat16
-    values = torch.empty((N, K // 2), dtype=vdt, device=W.device)
-    meta = torch.empty((N, K // 8), dtype=torch.uint8, device=W.device)
-    scale = torch.empty((1,), dtype=torch.float32, device=W.device) if dt == DTYPE_E4M3 else None
-    dense = torch.empty((N, K), dtype=vdt, device=W.device) if pruned_dense else None
+    values = out.get("values")
+    if values is None:
+        values = torch.empty((N, K // 2), dtype=vdt, device=W.device)
+    meta = out.get("meta")
+    if meta is None:
+        meta = torch.empty((N, K // 8), dtype=torch.uint8, device=W.device)
+    scale = out.get("scale")
+    if scale is None and dt == DTYPE_E4M3:
+        scale = torch.empty((1,), dtype=torch.float32, device=W.device)
+    dense = out.get("pruned_dense")
+    if dense is None and pruned_dense:
+        dense = torch.empty((N, K), dtype=vdt, device=W.device)
+    _require_cuda(values, meta, scale, dense)
+    if values.shape != (N, K // 2) or values.dtype != vdt or meta.shape != (N, K // 8):
+        raise Sp24Error("output tensors have the wrong shape or dtype")
     ws, wsn = _ws(W.device, _lib.OP_PRUNE_COMPRESS, 0, N, K, dt, workspace)
     rc = lib.sp24_prune_compress(_ptr(W), N, K, dt, _ptr(values), _ptr(meta), _ptr(scale),
                                  _ptr(dense), _ptr(ws), wsn, _ptr(status), _stream(W.device))
@@ -118,7 +132,7 @@ def fp8_quantize_pertensor(X: torch.Tensor, status: torch.Tensor | None = None,
 
 
 def slide68_decompose(W: torch.Tensor, out_dtype="e4m3", status: torch.Tensor | None = None,
-                      workspace: Workspace | None = None):
+                      workspace: Workspace | None = None, out: dict | None = None):
     """6:8 prune + sliding-window decomposition of W bf16 [N, K] into 2:4 over K' = 1.5 K."""
     lib = _lib.load()
     _require_cuda(W, status)
@@ -126,10 +140,20 @@ def slide68_decompose(W: torch.Tensor, out_dtype="e4m3", status: torch.Tensor | 
         raise Sp24Error("W must be a 2-D bf16 tensor")
     dt = _DT[out_dtype]
     N, K = W.shape
+    out = out or {}
     vdt = torch.uint8 if dt == DTYPE_E4M3 else torch.bfloat16
-    values = torch.empty((N, 3 * K // 4), dtype=vdt, device=W.device)
-    meta = torch.empty((N, 3 * K // 16), dtype=torch.uint8, device=W.device)
-    scale = torch.empty((1,), dtype=torch.float32, device=W.device) if dt == DTYPE_E4M3 else None
+    values = out.get("values")
+    if values is None:
+        values = torch.empty((N, 3 * K // 4), dtype=vdt, device=W.device)
+    meta = out.get("meta")
+    if meta is None:
+        meta = torch.empty((N, 3 * K // 16), dtype=torch.uint8, device=W.device)
+    scale = out.get("scale")
+    if scale is None and dt == DTYPE_E4M3:
+        scale = torch.empty((1,), dtype=torch.float32, device=W.device)
+    _require_cuda(values, meta, scale)
+    if values.shape != (N, 3 * K // 4) or values.dtype != vdt or meta.shape != (N, 3 * K // 16):
+        raise Sp24Error("output tensors have the wrong shape or dtype")
     ws, wsn = _ws(W.device, _lib.OP_SLIDE68_DECOMPOSE, 0, N, K, dt, workspace)
     rc = lib.slide68_decompose(_ptr(W), N, K, dt, _ptr(values), _ptr(meta), _ptr(scale), _ptr(ws),
                                wsn, _ptr(status), _stream(W.device))

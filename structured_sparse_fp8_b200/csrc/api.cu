@@ -108,7 +108,7 @@ int sp24_prune_compress(const void *W, int N, int K, int out_dtype, void *values
   const bool fp8 = out_dtype == SP24_DTYPE_E4M3;
   int rc = amax_then(W, nelem, workspace, ws_bytes, fp8 ? w_scale : nullptr, status, sms, st);
   if (rc != SP24_OK) return rc;
-  return cuda_status(sp24::launch_prune24(W, nelem, fp8, w_scale, values, meta, pruned_dense, sms, st));
+  return cuda_status(sp24::launch_prune24(W, nelem, K, fp8, w_scale, values, meta, pruned_dense, sms, st));
 }
 
 int fp8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, uint8_t *q, float *scale,
@@ -164,7 +164,7 @@ static int gemm_common(sp24::GemmKind kind, const void *Xq, const float *x_scale
                        sp24_stream_t stream) {
   const bool sparse = kind != sp24::kDenseE4M3;
   if (!Xq || !w_values || !Y || (sparse && !w_meta)) return SP24_ERR_NULL;
-  const int kmod = kind == sp24::kSparseBF16 ? 64 : 128;
+  const int kmod = 128;
   if (M < 1 || N < 128 || N % 128 != 0 || K < kmod || K % kmod != 0) return SP24_ERR_SHAPE;
   if (!aligned16(Xq) || !aligned16(w_values) || !aligned16(Y) || (sparse && !aligned16(w_meta)))
     return SP24_ERR_ALIGN;

@@ -60,9 +60,13 @@ __global__ void __launch_bounds__(256) amax_scale_kernel(const uint4 *__restrict
                                                          int32_t *status) {
   uint32_t m = 0;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec;
-       i += stride)
-    m = max(m, absmax8(ld_stream(x + i)));
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < nvec; i += 4 * stride) {  // four 16-byte loads in flight
+    const uint4 a = ld_stream(x + i), b = ld_stream(x + i + stride);
+    const uint4 c = ld_stream(x + i + 2 * stride), d = ld_stream(x + i + 3 * stride);
+    m = max(m, max(max(absmax8(a), absmax8(b)), max(absmax8(c), absmax8(d))));
+  }
+  for (; i < nvec; i += stride) m = max(m, absmax8(ld_stream(x + i)));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   __shared__ uint32_t part[32];
@@ -169,37 +173,30 @@ __device__ __forceinline__ uint32_t keep2of4(const uint32_t a[4]) {
   return mask;
 }
 
-// One thread per 8 K-values (two groups, one metadata byte).
-template <bool FP8>
-__global__ void __launch_bounds__(256) prune24_kernel(const uint4 *__restrict__ w, int64_t n8,
-                                                      const float *__restrict__ scale,
-                                                      void *__restrict__ values,
-                                                      uint8_t *__restrict__ meta,
-                                                      void *__restrict__ dense) {
-  const float s = FP8 ? *scale : 1.0f;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-       i += stride) {
-    const uint4 v = ld_stream(w + i);
-    const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-    uint32_t h[8];
+// Prune/quantise/compress 8 K-values (two groups, one metadata byte).
+// Codes are computed for the kept elements only, unless the pruned-dense copy
+// is wanted as well.
+template <bool FP8, bool DENSE>
+__device__ __forceinline__ void prune8(const uint4 v, float s, uint32_t kept_vals[4],
+                                       uint32_t &meta_byte, uint32_t dense_out[8]) {
+  const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+  uint32_t h[8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      h[2 * j] = words[j] & 0xFFFFu;
-      h[2 * j + 1] = words[j] >> 16;
-    }
-    uint32_t kept_vals[4];  // bf16 bits or codes of the 4 kept elements
-    uint32_t meta_byte = 0;
-    uint32_t dense_out[8];
+  for (int j = 0; j < 4; ++j) {
+    h[2 * j] = words[j] & 0xFFFFu;
+    h[2 * j + 1] = words[j] >> 16;
+  }
+  meta_byte = 0;
 #pragma unroll
-    for (int g = 0; g < 2; ++g) {
-      uint32_t a[4];
+  for (int g = 0; g < 2; ++g) {
+    uint32_t a[4];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) a[t] = h[4 * g + t] & 0x7FFFu;
-      const uint32_t mk = keep2of4(a);
-      const int i0 = __ffs(mk) - 1;
-      const int i1 = __ffs(mk & (mk - 1)) - 1;
-      meta_byte |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * g);
+    for (int t = 0; t < 4; ++t) a[t] = h[4 * g + t] & 0x7FFFu;
+    const uint32_t mk = keep2of4(a);
+    const int i0 = __ffs(mk) - 1;
+    const int i1 = __ffs(mk & (mk - 1)) - 1;
+    meta_byte |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * g);
+    if (DENSE) {
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const uint32_t val = FP8 ? quant_bf16(h[4 * g + t], s) : h[4 * g + t];
@@ -207,24 +204,71 @@ __global__ void __launch_bounds__(256) prune24_kernel(const uint4 *__restrict__ 
         if (t == i0) kept_vals[2 * g] = val;
         if (t == i1) kept_vals[2 * g + 1] = val;
       }
+    } else {
+      uint32_t h0 = 0, h1 = 0;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        if (t == i0) h0 = h[4 * g + t];
+        if (t == i1) h1 = h[4 * g + t];
+      }
+      kept_vals[2 * g] = FP8 ? quant_bf16(h0, s) : h0;
+      kept_vals[2 * g + 1] = FP8 ? quant_bf16(h1, s) : h1;
     }
-    meta[i] = static_cast<uint8_t>(meta_byte);
+  }
+}
+
+// One thread per CHUNKS x 8 consecutive K-values (CHUNKS = 4 when K % 32 == 0:
+// 64-byte loads, 16-byte value stores and one 4-byte metadata store).
+template <bool FP8, bool DENSE, int CHUNKS>
+__global__ void __launch_bounds__(256) prune24_kernel(const uint4 *__restrict__ w, int64_t nwork,
+                                                      const float *__restrict__ scale,
+                                                      void *__restrict__ values,
+                                                      uint8_t *__restrict__ meta,
+                                                      void *__restrict__ dense) {
+  const float s = FP8 ? *scale : 1.0f;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nwork;
+       i += stride) {
+    uint4 v[CHUNKS];
+#pragma unroll
+    for (int c = 0; c < CHUNKS; ++c) v[c] = ld_stream(w + i * CHUNKS + c);
+    uint32_t kv[CHUNKS][4], mb[CHUNKS], dn[CHUNKS][8];
+#pragma unroll
+    for (int c = 0; c < CHUNKS; ++c) prune8<FP8, DENSE>(v[c], s, kv[c], mb[c], dn[c]);
+    if (CHUNKS == 4) {
+      reinterpret_cast<uint32_t *>(meta)[i] = mb[0] | (mb[1] << 8) | (mb[2] << 16) | (mb[3] << 24);
+    } else {
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) meta[i * CHUNKS + c] = static_cast<uint8_t>(mb[c]);
+    }
     if (FP8) {
-      reinterpret_cast<uint32_t *>(values)[i] =
-          kept_vals[0] | (kept_vals[1] << 8) | (kept_vals[2] << 16) | (kept_vals[3] << 24);
-      if (dense) {
-        uint2 d;
-        d.x = dense_out[0] | (dense_out[1] << 8) | (dense_out[2] << 16) | (dense_out[3] << 24);
-        d.y = dense_out[4] | (dense_out[5] << 8) | (dense_out[6] << 16) | (dense_out[7] << 24);
-        reinterpret_cast<uint2 *>(dense)[i] = d;
+      uint32_t word[CHUNKS];
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c)
+        word[c] = kv[c][0] | (kv[c][1] << 8) | (kv[c][2] << 16) | (kv[c][3] << 24);
+      if (CHUNKS == 4)
+        reinterpret_cast<uint4 *>(values)[i] = make_uint4(word[0], word[1], word[2], word[3]);
+      else
+        for (int c = 0; c < CHUNKS; ++c) reinterpret_cast<uint32_t *>(values)[i * CHUNKS + c] = word[c];
+      if (DENSE) {
+#pragma unroll
+        for (int c = 0; c < CHUNKS; ++c) {
+          uint2 d;
+          d.x = dn[c][0] | (dn[c][1] << 8) | (dn[c][2] << 16) | (dn[c][3] << 24);
+          d.y = dn[c][4] | (dn[c][5] << 8) | (dn[c][6] << 16) | (dn[c][7] << 24);
+          reinterpret_cast<uint2 *>(dense)[i * CHUNKS + c] = d;
+        }
       }
     } else {
-      reinterpret_cast<uint2 *>(values)[i] =
-          make_uint2(kept_vals[0] | (kept_vals[1] << 16), kept_vals[2] | (kept_vals[3] << 16));
-      if (dense)
-        reinterpret_cast<uint4 *>(dense)[i] =
-            make_uint4(dense_out[0] | (dense_out[1] << 16), dense_out[2] | (dense_out[3] << 16),
-                       dense_out[4] | (dense_out[5] << 16), dense_out[6] | (dense_out[7] << 16));
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) {
+        reinterpret_cast<uint2 *>(values)[i * CHUNKS + c] =
+            make_uint2(kv[c][0] | (kv[c][1] << 16), kv[c][2] | (kv[c][3] << 16));
+        if (DENSE)
+          reinterpret_cast<uint4 *>(dense)[i * CHUNKS + c] =
+              make_uint4(dn[c][0] | (dn[c][1] << 16), dn[c][2] | (dn[c][3] << 16),
+                         dn[c][4] | (dn[c][5] << 16), dn[c][6] | (dn[c][7] << 16));
+      }
     }
   }
 }
@@ -363,16 +407,32 @@ cudaError_t launch_lift_quantize(const void *x, int64_t nelem, const float *scal
   return cudaGetLastError();
 }
 
-cudaError_t launch_prune24(const void *w, int64_t nelem, bool fp8, const float *scale,
+template <bool FP8, bool DENSE>
+static void prune24_dispatch(const void *w, int64_t nelem, bool wide, const float *scale,
+                             void *values, uint8_t *meta, void *dense, int sm_count,
+                             cudaStream_t st) {
+  if (wide) {
+    const int64_t n32 = nelem / 32;
+    prune24_kernel<FP8, DENSE, 4><<<grid_for(n32, sm_count), 256, 0, st>>>(
+        static_cast<const uint4 *>(w), n32, scale, values, meta, dense);
+  } else {
+    const int64_t n8 = nelem / 8;
+    prune24_kernel<FP8, DENSE, 1><<<grid_for(n8, sm_count), 256, 0, st>>>(
+        static_cast<const uint4 *>(w), n8, scale, values, meta, dense);
+  }
+}
+
+cudaError_t launch_prune24(const void *w, int64_t nelem, int64_t k, bool fp8, const float *scale,
                            void *values, uint8_t *meta, void *dense, int sm_count,
                            cudaStream_t st) {
-  const int64_t n8 = nelem / 8;
-  if (fp8)
-    prune24_kernel<true><<<grid_for(n8, sm_count), 256, 0, st>>>(
-        static_cast<const uint4 *>(w), n8, scale, values, meta, dense);
-  else
-    prune24_kernel<false><<<grid_for(n8, sm_count), 256, 0, st>>>(
-        static_cast<const uint4 *>(w), n8, scale, values, meta, dense);
+  const bool wide = k % 32 == 0;
+  if (fp8) {
+    if (dense) prune24_dispatch<true, true>(w, nelem, wide, scale, values, meta, dense, sm_count, st);
+    else prune24_dispatch<true, false>(w, nelem, wide, scale, values, meta, dense, sm_count, st);
+  } else {
+    if (dense) prune24_dispatch<false, true>(w, nelem, wide, scale, values, meta, dense, sm_count, st);
+    else prune24_dispatch<false, false>(w, nelem, wide, scale, values, meta, dense, sm_count, st);
+  }
   return cudaGetLastError();
 }
 

@@ -53,6 +53,9 @@ struct KindTraits<kSparseE4M3> {
   static constexpr uint32_t kFmt = 0;
   static constexpr int kAElemBytes = 1;
   static constexpr int kBElemBytes = 1;
+  static constexpr int kBBoxElems = 128;     // one 128-byte swizzle row of X per box
+  static constexpr bool kMetaTransform = false;
+  static constexpr int kMetaColsPerMma = 2;  // 64 metadata bits per row per MMA
 };
 
 // Dense E4M3 (comparison kernel): 128 logical K per stage, 4 MMAs of K = 32.
@@ -71,6 +74,34 @@ struct KindTraits<kDenseE4M3> {
   static constexpr uint32_t kFmt = 0;
   static constexpr int kAElemBytes = 1;
   static constexpr int kBElemBytes = 1;
+  static constexpr int kBBoxElems = 128;
+  static constexpr bool kMetaTransform = false;
+  static constexpr int kMetaColsPerMma = 0;
+};
+
+// 2:4 sparse BF16 (kind::f16): per stage 128 logical K = 64 bf16 values (128 B)
+// + 16 metadata bytes per W row, 256 bytes (two 128-byte boxes) per token;
+// 4 MMAs of K = 32.  For 16-bit operands the MMA reads the metadata of rows
+// m and m + 8 from one TMEM lane (16 bits each), so the epilogue warps
+// re-arrange each stage's metadata in shared memory before it is copied.
+template <>
+struct KindTraits<kSparseBF16> {
+  static constexpr bool kSparse = true;
+  static constexpr int kBK = 128;
+  static constexpr int kARowBytes = 128;
+  static constexpr uint32_t kASwizzle = kSwizzle128B;
+  static constexpr int kASbo = 8 * 128;
+  static constexpr int kBRowBytes = 256;
+  static constexpr int kERowBytes = 16;
+  static constexpr int kMmas = 4;
+  static constexpr int kAStep = 32;  // 16 compressed bf16 per MMA
+  static constexpr int kBStep = 64;  // 32 bf16 per MMA
+  static constexpr uint32_t kFmt = 1;
+  static constexpr int kAElemBytes = 2;
+  static constexpr int kBElemBytes = 2;
+  static constexpr int kBBoxElems = 64;
+  static constexpr bool kMetaTransform = true;
+  static constexpr int kMetaColsPerMma = 1;
 };
 
 template <int KIND, int BN>
@@ -79,20 +110,26 @@ struct Config {
   static constexpr uint32_t kABytes = 128 * T::kARowBytes;
   static constexpr uint32_t kBBytes = BN * T::kBRowBytes;
   static constexpr uint32_t kEBytes = 128 * T::kERowBytes;
-  static constexpr uint32_t kStageBytes = kABytes + kBBytes + kEBytes;
+  static constexpr uint32_t kTBytes = T::kMetaTransform ? 128 * 16 : 0;  // TMEM-ready metadata
+  static constexpr uint32_t kTmaBytes = kABytes + kBBytes + kEBytes;
+  static constexpr uint32_t kStageBytes = kTmaBytes + kTBytes;
+  static constexpr int kBSub = T::kBRowBytes / 128;   // 128-byte X boxes per stage
   // Small token tiles run two CTAs per SM (more loads in flight for the
   // bandwidth-bound decode shapes); large ones one CTA with a deep ring.
   static constexpr int kCtasPerSm = BN <= 64 ? 2 : 1;
   static constexpr uint32_t kSmemBudget = kCtasPerSm == 2 ? 110 * 1024 : 220 * 1024;
   static constexpr int kStagesRaw = static_cast<int>(kSmemBudget / kStageBytes);
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*bars*/;
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 512 /*bars*/;
   static constexpr uint32_t kTmemNeed = BN + (T::kSparse ? 4 : 0);
   static constexpr uint32_t kTmemCols =
       kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
   static_assert(kStages >= 2, "shared-memory ring too shallow");
+  static_assert(kStages * kStageBytes >= BN * 128 * 4, "split-K tile must fit in the idle ring");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be a multiple of 16 in [16,256]");
 };
+
+constexpr int kMaxSplits = 8;  // portable thread-block cluster size
 
 struct GemmArgs {
   int M, N, K;
@@ -102,8 +139,6 @@ struct GemmArgs {
   uint16_t *y;
   const float *x_scale;
   const float *w_scale;
-  float *partials;     // [tiles][splits][BN][128]
-  uint32_t *counters;  // [tiles]
   int32_t *status;
 };
 
@@ -126,9 +161,9 @@ __global__ void __launch_bounds__(192, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * C::kStageBytes);
   uint64_t *empty = full + S;
-  uint64_t *accum_bar = empty + S;
+  uint64_t *meta_ready = empty + S;
+  uint64_t *accum_bar = meta_ready + S;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum_bar + 1);
-  uint32_t *last_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -146,6 +181,7 @@ __global__ void __launch_bounds__(192, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&meta_ready[s], 128);
     }
     mbar_init(accum_bar, 1);
     fence_mbar_init();
@@ -170,10 +206,12 @@ __global__ void __launch_bounds__(192, 1)
         if (i >= S && !mbar_wait(&empty[s], ph ^ 1u, p.status)) break;
         uint8_t *st = smem + s * C::kStageBytes;
         const int kb = kb_begin + i;
-        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+        mbar_arrive_expect_tx(&full[s], C::kTmaBytes);
         tma_load_2d(st, &tmA, &full[s], kb * (T::kARowBytes / T::kAElemBytes), n0, stream_w);
-        tma_load_2d(st + C::kABytes, &tmB, &full[s], kb * (T::kBRowBytes / T::kBElemBytes), m0,
-                    keep_x);
+#pragma unroll
+        for (int sub = 0; sub < C::kBSub; ++sub)
+          tma_load_2d(st + C::kABytes + sub * BN * 128, &tmB, &full[s],
+                      kb * (T::kBRowBytes / T::kBElemBytes) + sub * T::kBBoxElems, m0, keep_x);
         if (T::kSparse)
           tma_load_2d(st + C::kABytes + C::kBBytes, &tmE, &full[s], kb * T::kERowBytes, n0,
                       stream_w);
@@ -190,23 +228,31 @@ __global__ void __launch_bounds__(192, 1)
         const int s = i % S;
         const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
         if (!mbar_wait(&full[s], ph, p.status)) break;
+        if (T::kMetaTransform && !mbar_wait(&meta_ready[s], ph, p.status)) break;
         tc_fence_after();
         const uint32_t a_addr = smem_addr(smem + s * C::kStageBytes);
         const uint32_t b_addr = a_addr + C::kABytes;
         if (T::kSparse) {
-          const uint32_t e_addr = b_addr + C::kBBytes;
           // 128 rows x 16 B, rows contiguous: core matrices of 8 rows are 128 B apart.
+          const uint32_t e_addr = b_addr + C::kBBytes + (T::kMetaTransform ? C::kEBytes : 0);
           tmem_copy_128x128b(e_tmem, smem_desc(e_addr, 2048, 128, kSwizzleNone));
         }
 #pragma unroll
         for (int kk = 0; kk < T::kMmas; ++kk) {
           const uint64_t ad = smem_desc(a_addr + kk * T::kAStep, 16, T::kASbo, T::kASwizzle);
-          const uint64_t bd = smem_desc(b_addr + kk * T::kBStep, 16, 8 * 128, kSwizzle128B);
+          const uint32_t boff = (kk * T::kBStep / 128) * (BN * 128) + (kk * T::kBStep) % 128;
+          const uint64_t bd = smem_desc(b_addr + boff, 16, 8 * 128, kSwizzle128B);
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          if constexpr (T::kSparse)
+          if constexpr (KIND == kSparseE4M3) {
             mma_f8_sparse(d_tmem, ad, bd, idesc, e_tmem + 2 * kk, acc);
-          else
+          } else if constexpr (KIND == kSparseBF16) {
+            // one metadata column per MMA; columns are addressed in pairs and
+            // the instruction descriptor's selector picks the column of the pair
+            mma_bf16_sparse(d_tmem, ad, bd, idesc | static_cast<uint32_t>(kk & 1),
+                            e_tmem + (kk & ~1), acc);
+          } else {
             mma_f8_dense(d_tmem, ad, bd, idesc, acc);
+          }
         }
         mma_commit(&empty[s]);
       }
@@ -218,6 +264,30 @@ __global__ void __launch_bounds__(192, 1)
     const int q = warp & 3;            // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;     // W row within the tile == accumulator lane
     const int n = n0 + row;
+    if constexpr (T::kMetaTransform) {
+      // Lane L = r0 + 8h + 16g of the TMEM metadata holds, for each of the
+      // stage's 4 MMAs j, the 16 bits of K-half h of row 16g + r0 (low half)
+      // and of row 16g + 8 + r0 (high half).
+      const int t = threadIdx.x - 64;
+      const int r0 = t & 7, h = (t >> 3) & 1, g = t >> 4;
+      const int ra = 16 * g + r0, rb = ra + 8;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % S;
+        const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
+        if (!mbar_wait(&full[s], ph, p.status)) break;
+        const uint8_t *e = smem + s * C::kStageBytes + C::kABytes + C::kBBytes;
+        const uint16_t *ea = reinterpret_cast<const uint16_t *>(e + ra * 16);
+        const uint16_t *eb = reinterpret_cast<const uint16_t *>(e + rb * 16);
+        uint4 w;
+        w.x = ea[0 + h] | (static_cast<uint32_t>(eb[0 + h]) << 16);
+        w.y = ea[2 + h] | (static_cast<uint32_t>(eb[2 + h]) << 16);
+        w.z = ea[4 + h] | (static_cast<uint32_t>(eb[4 + h]) << 16);
+        w.w = ea[6 + h] | (static_cast<uint32_t>(eb[6 + h]) << 16);
+        *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(e) + C::kEBytes + t * 16) = w;
+        fence_proxy_async_smem();
+        mbar_arrive(&meta_ready[s]);
+      }
+    }
     mbar_wait(accum_bar, 0, p.status);
     tc_fence_after();
     const float sx = p.x_scale ? __ldg(p.x_scale) : 1.0f;
@@ -237,37 +307,54 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
     } else {
-      const int tile = m_tile * gridDim.x + n_tile;
-      float *mine = p.partials + (static_cast<size_t>(tile) * p.splits + split) * BN * 128;
+      // Split-K: park this split's fp32 tile (valid token columns only) in
+      // this CTA's shared memory, red[c * 128 + row]; the ring is idle now.
+      float *red = reinterpret_cast<float *>(smem);
+      const int mvalid = min(BN, p.M - m0);
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 16) {
+      for (int c = 0; c < mvalid; c += 16) {
         uint32_t r[16];
         tmem_ld_32x32b_x16(t_row + c, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) __stcg(mine + (c + j) * 128 + row, __uint_as_float(r[j]));
-      }
-      __threadfence();
-      named_bar_sync(1, 128);
-      if (threadIdx.x == 64) {
-        const uint32_t done = atomicAdd(&p.counters[tile], 1u);
-        *last_flag = (done == static_cast<uint32_t>(p.splits - 1)) ? 1u : 0u;
-      }
-      named_bar_sync(1, 128);
-      if (*last_flag) {
-        __threadfence();
-        const float *base = p.partials + static_cast<size_t>(tile) * p.splits * BN * 128;
-#pragma unroll 1
-        for (int c = 0; c < BN; ++c) {
-          const int m = m0 + c;
-          if (m >= p.M) break;
-          float acc = 0.0f;
-          for (int s2 = 0; s2 < p.splits; ++s2) acc += __ldcg(base + (static_cast<size_t>(s2) * BN + c) * 128 + row);
-          p.y[static_cast<size_t>(m) * p.N + n] = f32_to_bf16_bits(acc * sc);
-        }
-        if (threadIdx.x == 64) p.counters[tile] = 0u;  // leave the workspace zeroed
+        for (int j = 0; j < 16; ++j) red[(c + j) * 128 + row] = __uint_as_float(r[j]);
       }
     }
+  }
+
+  if (p.splits > 1) {
+    // The K-splits of one output tile form a thread-block cluster.  After the
+    // first cluster barrier every split's partial tile is in its CTA's shared
+    // memory; CTA `rank` then reduces the token columns c = rank (mod splits),
+    // reading all partials through distributed shared memory in split order
+    // (deterministic), and the second barrier keeps every CTA's shared memory
+    // alive until its peers have finished reading it.
+    cluster_sync_all();
+    if (warp >= 2) {
+      const int q = warp & 3;
+      const int row = q * 32 + lane;
+      const int n = n0 + row;
+      const int S2 = p.splits;
+      const uint32_t rank = cluster_ctarank();
+      const int mvalid = min(BN, p.M - m0);
+      const float sx = p.x_scale ? __ldg(p.x_scale) : 1.0f;
+      const float sw = p.w_scale ? __ldg(p.w_scale) : 1.0f;
+      const float sc = sx * sw;
+      const uint32_t red_base = smem_addr(smem) + static_cast<uint32_t>(row) * 4u;
+#pragma unroll 1
+      for (int c = static_cast<int>(rank); c < mvalid; c += S2) {
+        const uint32_t local = red_base + static_cast<uint32_t>(c) * 128u * 4u;
+        float v[kMaxSplits];
+#pragma unroll
+        for (int s2 = 0; s2 < kMaxSplits; ++s2)
+          v[s2] = s2 < S2 ? ld_dsmem_f32(dsmem_map(local, static_cast<uint32_t>(s2))) : 0.0f;
+        float acc = 0.0f;
+#pragma unroll
+        for (int s2 = 0; s2 < kMaxSplits; ++s2) acc += v[s2];
+        p.y[static_cast<size_t>(m0 + c) * p.N + n] = f32_to_bf16_bits(acc * sc);
+      }
+    }
+    cluster_sync_all();
   }
 
   tc_fence_before();
@@ -313,11 +400,11 @@ static bool make_map(CUtensorMap *map, const void *ptr, CUtensorMapDataType dt, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static int choose_bn(int M) {
+static int choose_bn(GemmKind kind, int M) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
   if (M <= 64) return 64;
-  if (M <= 128) return 128;
+  if (M <= 128 || kind == kSparseBF16) return 128;  // bf16 X stages are twice as large
   return 256;
 }
 
@@ -325,9 +412,8 @@ static int ctas_per_sm(int bn) { return bn <= 64 ? 2 : 1; }
 
 GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   GemmPlan pl{};
-  pl.bn = choose_bn(M);
+  pl.bn = choose_bn(kind, M);
   pl.bk = 128;
-  (void)kind;
   pl.tiles_n = N / 128;
   pl.tiles_m = (M + pl.bn - 1) / pl.bn;
   pl.num_kb = K / pl.bk;
@@ -336,10 +422,12 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   pl.kb_per_split = pl.num_kb;
   pl.splits = 1;
   if (tiles * 2 <= slots) {
-    // Split K so that the CTAs fill the machine; each split keeps >= 4 stages.
+    // Split K over a cluster of up to 8 CTAs so that the CTAs fill the
+    // machine; each split keeps >= 4 pipeline stages of work.
     double best = -1.0;
     for (int kps = pl.num_kb; kps >= 4; --kps) {
       const int s = (pl.num_kb + kps - 1) / kps;
+      if (s > kMaxSplits) break;
       const long units = static_cast<long>(tiles) * s;
       const long waves = (units + slots - 1) / slots;
       const double eff = static_cast<double>(units) / static_cast<double>(waves * slots);
@@ -350,8 +438,8 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
       }
     }
   }
-  pl.partial_bytes = static_cast<size_t>(tiles) * pl.splits * pl.bn * 128 * sizeof(float);
-  pl.counter_bytes = (static_cast<size_t>(tiles) * sizeof(uint32_t) + 255) & ~static_cast<size_t>(255);
+  pl.partial_bytes = 0;
+  pl.counter_bytes = 0;
   return pl;
 }
 
@@ -371,16 +459,21 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   if (attr_err != cudaSuccess) return attr_err;
 
   CUtensorMap tmA, tmB, tmE;
-  const CUtensorMapDataType dt8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const CUtensorMapDataType dtA =
+      T::kAElemBytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const CUtensorMapDataType dtB =
+      T::kBElemBytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const uint64_t a_row = T::kSparse ? static_cast<uint64_t>(K) / 2 : static_cast<uint64_t>(K);
   const CUtensorMapSwizzle a_sw =
       T::kASwizzle == kSwizzle64B ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-  if (!make_map(&tmA, w_values, dt8, 1, a_row, N, T::kARowBytes, 128, a_sw)) return cudaErrorInvalidValue;
-  if (!make_map(&tmB, xq, dt8, 1, K, M, T::kBRowBytes, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_map(&tmA, w_values, dtA, T::kAElemBytes, a_row, N, T::kARowBytes / T::kAElemBytes,
+                128, a_sw))
+    return cudaErrorInvalidValue;
+  if (!make_map(&tmB, xq, dtB, T::kBElemBytes, K, M, T::kBBoxElems, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (T::kSparse) {
-    if (!make_map(&tmE, w_meta, dt8, 1, static_cast<uint64_t>(K) / 8, N, 16, 128,
-                  CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!make_map(&tmE, w_meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(K) / 8, N,
+                  16, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   } else {
     tmE = tmA;  // unused
@@ -395,16 +488,21 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   a.y = static_cast<uint16_t *>(y);
   a.x_scale = x_scale;
   a.w_scale = w_scale;
-  // Workspace layout: tile counters first (kept at zero between calls), then
-  // the fp32 partial tiles (scratch, fully rewritten before being read).
-  a.counters = pl.splits > 1 ? static_cast<uint32_t *>(workspace) : nullptr;
-  a.partials = pl.splits > 1
-                   ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + pl.counter_bytes)
-                   : nullptr;
   a.status = status;
-  dim3 grid(pl.tiles_n, pl.tiles_m, pl.splits);
-  gemm_kernel<KIND, BN><<<grid, 192, C::kSmemBytes, st>>>(tmA, tmB, tmE, a);
-  return cudaGetLastError();
+  (void)workspace;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.tiles_n, pl.tiles_m, pl.splits);
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = static_cast<unsigned>(pl.splits);
+  cfg.attrs = attr;
+  cfg.numAttrs = pl.splits > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN>, tmA, tmB, tmE, a);
 }
 
 template <int KIND>
@@ -431,6 +529,8 @@ cudaError_t launch_gemm(GemmKind kind, const GemmPlan &pl, const void *xq, const
       return launch_kind<kSparseE4M3>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
     case kDenseE4M3:
       return launch_kind<kDenseE4M3>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
+    case kSparseBF16:
+      return launch_kind<kSparseBF16>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
     default:
       return cudaErrorInvalidValue;
   }

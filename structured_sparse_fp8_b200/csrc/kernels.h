@@ -15,7 +15,7 @@ cudaError_t launch_quantize(const void *x, int64_t nelem, const float *scale, ui
                             int sm_count, cudaStream_t st);
 cudaError_t launch_lift_quantize(const void *x, int64_t nelem, const float *scale, uint8_t *q,
                                  int sm_count, cudaStream_t st);
-cudaError_t launch_prune24(const void *w, int64_t nelem, bool fp8, const float *scale,
+cudaError_t launch_prune24(const void *w, int64_t nelem, int64_t k, bool fp8, const float *scale,
                            void *values, uint8_t *meta, void *dense, int sm_count,
                            cudaStream_t st);
 cudaError_t launch_slide68(const void *w, int64_t nelem, bool fp8, const float *scale,

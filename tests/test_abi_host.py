@@ -33,12 +33,10 @@ def test_status_strings_and_version(lib):
 def test_workspace_sizes(lib):
     for op in range(4):
         assert lib.sp24_workspace_size(op, 16, 256, 256, 0) == 256
-    # a prefill-sized GEMM fills the machine without split-K: no scratch
-    assert lib.sp24_workspace_size(_lib.OP_GEMM, 4096, 12288, 4096, 0) == 0
-    # a decode-sized GEMM splits K and needs counters + fp32 partial tiles
-    ws = lib.sp24_workspace_size(_lib.OP_GEMM, 1, 11008, 4096, 0)
-    assert ws > 0 and ws % 256 == 0
-    assert lib.sp24_workspace_size(_lib.OP_GEMM, 0, 11008, 4096, 0) == 0
+    # the GEMMs reduce split-K partials in distributed shared memory: no scratch
+    for m in (1, 64, 256, 4096):
+        assert lib.sp24_workspace_size(_lib.OP_GEMM, m, 11008, 4096, 0) == 0
+        assert lib.sp24_workspace_size(_lib.OP_GEMM_DENSE, m, 11008, 4096, 0) == 0
 
 
 FAKE = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: calls fail validation first

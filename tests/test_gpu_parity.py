@@ -274,7 +274,7 @@ def test_slide68_workload_gemm(m):
     assert_gemm_close(torch.from_numpy(yh.view(np.int16)).view(torch.bfloat16), y_ref, b, f"6:8 M={m}")
 
 
-def test_gemm_rejects_bad_workspace_and_shapes():
+def test_gemm_needs_no_workspace_and_rejects_bad_shapes():
     m = sp()
     xq = torch.zeros((1, 4096), dtype=torch.uint8, device=DEV)
     vals = torch.zeros((11008, 2048), dtype=torch.uint8, device=DEV)
@@ -282,11 +282,52 @@ def test_gemm_rejects_bad_workspace_and_shapes():
     s = torch.ones(1, dtype=torch.float32, device=DEV)
     y = torch.empty((1, 11008), dtype=torch.bfloat16, device=DEV)
     lib = m._lib.load()
+    stream = torch.cuda.current_stream().cuda_stream
     rc = lib.sp24_gemm(xq.data_ptr(), s.data_ptr(), vals.data_ptr(), meta.data_ptr(), s.data_ptr(),
-                       y.data_ptr(), 1, 11008, 4096, 0, None, 0, None,
-                       torch.cuda.current_stream().cuda_stream)
-    assert rc == m._lib.SP24_ERR_WORKSPACE
+                       y.data_ptr(), 1, 11008, 4096, 0, None, 0, None, stream)
+    assert rc == m._lib.SP24_OK
+    torch.cuda.synchronize()
+    assert (host(y) == 0).all()
     rc = lib.sp24_gemm(xq.data_ptr(), s.data_ptr(), vals.data_ptr(), meta.data_ptr(), s.data_ptr(),
-                       y.data_ptr(), 1, 11008, 4000, 0, None, 0, None,
-                       torch.cuda.current_stream().cuda_stream)
+                       y.data_ptr(), 1, 11008, 4000, 0, None, 0, None, stream)
     assert rc == m._lib.SP24_ERR_SHAPE
+
+
+def test_back_to_back_gemm_shapes_share_one_workspace():
+    """Regression: GEMMs of different shapes on one stream, one after another."""
+    for (mm, n, k) in [(300, 384, 1152), (1, 11008, 4096), (17, 384, 640), (64, 11008, 4096)]:
+        x = WL.random_bits((mm, k), 500 + mm)
+        w = WL.random_bits((n, k), 600 + n, scale=0.02)
+        y, _, xq, sx, vals, meta, sw = _run_sparse(x, w)
+        y_ref, b = _ref(xq, sx, vals, meta, sw, k)
+        assert_gemm_close(y, y_ref, b, f"sequence {mm}x{n}x{k}")
+
+
+# ------------------------------------------------------------ BF16-operand sparse GEMM
+
+def _run_sparse_bf16(x_bits, w_bits):
+    st = new_status()
+    c = sp().sp24_prune_compress(dev_bf16(w_bits), "bf16", status=st)
+    y = sp().sp24_gemm(dev_bf16(x_bits), None, c["values"], c["meta"], None, dtype="bf16", status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = O.sp24_prune_compress(w_bits, "bf16")
+    assert np.array_equal(host(c["values"]), ref["values"])
+    assert np.array_equal(host(c["meta"]), ref["meta"])
+    y_ref, b = O.gemm_ref(O.bf16_to_f32(x_bits), O.bf16_to_f32(ref["pruned_dense"]))
+    return y, y_ref, b
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 128, 128), (16, 256, 256), (33, 128, 640), (130, 384, 512),
+                                   (257, 256, 384), (64, 1024, 2048)])
+def test_sparse_gemm_bf16_small_shapes(m, n, k):
+    x = WL.random_bits((m, k), 300 + m)
+    w = WL.random_bits((n, k), 400 + n, scale=0.02)
+    y, y_ref, b = _run_sparse_bf16(x, w)
+    assert_gemm_close(y, y_ref, b, f"bf16 sparse {m}x{n}x{k}")
+
+
+def test_down_proj_workload_gemm_bf16():
+    w, x = WL.weight_bits(4), WL.activation_bits(4, 256)
+    y, y_ref, b = _run_sparse_bf16(x, w)
+    assert_gemm_close(y, y_ref, b, "down-proj bf16")

@@ -35,11 +35,44 @@ __device__ __forceinline__ uint32_t e4m3_code(float v) {
   return c | ((__float_as_uint(v) >> 24) & 0x80u);
 }
 
-// Code of the bf16 value h divided by the dequantisation scale s (one
-// correctly rounded fp32 division, as in the definition).
-__device__ __forceinline__ uint32_t quant_bf16(uint32_t h, float s) {
-  return e4m3_code(__fdiv_rn(bf16_bits_to_float(h), s));
-}
+// E4M3 code of the bf16 value h divided by the dequantisation scale s, where
+// the definition takes the quotient as one correctly rounded fp32 division;
+// computed without a full division in almost every case.
+//
+// With rs = RN(1/s), q0 = RN(x * rs) is within 1.5 ulp of x/s, and one
+// residual step q1 = RN(q0 + RN(x - q0*s) * rs) (Markstein's correction,
+// P. Markstein, IBM J. Res. Dev. 34(1), 1990) is within 0.5 ulp + a tiny
+// fraction of an ulp of x/s, hence within 1 ulp of the correctly rounded
+// quotient q* = RN(x/s).  The E4M3 code of an fp32 value in the E4M3 normal
+// range depends only on which side of the grid midpoints (fp32 values whose
+// low 20 mantissa bits are 0x80000) it lies, so cvt(q1) == cvt(q*) whenever
+// q1 is more than 2 ulps away from every midpoint.  The remaining cases --
+// within 2 ulps of a midpoint, or in the E4M3 subnormal range -- take the
+// correctly rounded division.  Quotients below 2^-12 are code +-0 for any
+// value within 1 ulp, so they need no division at all.
+struct FastQuant {
+  float s, rs;
+  bool fast;  // scale and reciprocal are normal, so the residual step is valid
+  __device__ __forceinline__ explicit FastQuant(float scale) : s(scale) {
+    rs = __frcp_rn(scale);
+    const uint32_t es = (__float_as_uint(scale) >> 23) & 0xFFu;
+    const uint32_t er = (__float_as_uint(rs) >> 23) & 0xFFu;
+    fast = es > 8u && es < 247u && er > 8u && er < 247u;
+  }
+  __device__ __forceinline__ uint32_t operator()(uint32_t h) const {
+    const float x = bf16_bits_to_float(h);
+    if (!fast) return e4m3_code(__fdiv_rn(x, s));
+    const float q0 = x * rs;
+    const float r = fmaf(-q0, s, x);
+    const float q1 = fmaf(r, rs, q0);
+    const uint32_t u = __float_as_uint(q1);
+    const uint32_t mag = u & 0x7FFFFFFFu;
+    if (mag < 0x39800000u) return (h >> 8) & 0x80u;  // |q| < 2^-12: +-0 with the sign of x
+    const bool near_mid = ((u - 0x7FFFEu) & 0xFFFFFu) <= 4u;
+    if (mag < 0x3C800000u || near_mid) return e4m3_code(__fdiv_rn(x, s));  // < 2^-6 or tie zone
+    return e4m3_code(q1);
+  }
+};
 
 // Largest magnitude bit pattern among the 8 bf16 values of a 16-byte vector.
 // For finite bf16 the unsigned order of (bits & 0x7FFF) is the order of |x|;
@@ -101,7 +134,7 @@ __global__ void __launch_bounds__(256) amax_scale_kernel(const uint4 *__restrict
 __global__ void __launch_bounds__(256) quantize_kernel(const uint4 *__restrict__ x, int64_t n16,
                                                        const float *__restrict__ scale,
                                                        uint4 *__restrict__ q) {
-  const float s = *scale;
+  const FastQuant qz(*scale);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
        i += stride) {
@@ -111,8 +144,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint4 *__restrict__
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint32_t lo = w[2 * j], hi = w[2 * j + 1];
-      o[j] = quant_bf16(lo & 0xFFFFu, s) | (quant_bf16(lo >> 16, s) << 8) |
-             (quant_bf16(hi & 0xFFFFu, s) << 16) | (quant_bf16(hi >> 16, s) << 24);
+      o[j] = qz(lo & 0xFFFFu) | (qz(lo >> 16) << 8) | (qz(hi & 0xFFFFu) << 16) | (qz(hi >> 16) << 24);
     }
     q[i] = make_uint4(o[0], o[1], o[2], o[3]);
   }
@@ -125,7 +157,7 @@ __global__ void __launch_bounds__(256) lift_quantize_kernel(const uint4 *__restr
                                                             int64_t n16,
                                                             const float *__restrict__ scale,
                                                             uint2 *__restrict__ q) {
-  const float s = *scale;
+  const FastQuant qz(*scale);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
        i += stride) {
@@ -134,8 +166,8 @@ __global__ void __launch_bounds__(256) lift_quantize_kernel(const uint4 *__restr
     uint32_t c[16];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      c[2 * j] = quant_bf16(w[j] & 0xFFFFu, s);
-      c[2 * j + 1] = quant_bf16(w[j] >> 16, s);
+      c[2 * j] = qz(w[j] & 0xFFFFu);
+      c[2 * j + 1] = qz(w[j] >> 16);
     }
     uint32_t out[6];
 #pragma unroll
@@ -159,25 +191,24 @@ __global__ void __launch_bounds__(256) lift_quantize_kernel(const uint4 *__restr
 // ----------------------------------------------------------------- 2:4 prune
 
 // Kept-position mask (4 bits) of one group: element i is kept when fewer than
-// two elements beat it (larger |w|, or equal |w| at a lower index).
+// two elements beat it (larger |w|, or equal |w| at a lower index).  With the
+// unique keys k_i = |w_i| << 2 | (3 - i) "beats" is plain ">", so the kept pair
+// is the two largest keys, found with a min/max network.
 __device__ __forceinline__ uint32_t keep2of4(const uint32_t a[4]) {
-  uint32_t mask = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    int beaten = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (j != i) beaten += (a[j] > a[i]) || (a[j] == a[i] && j < i);
-    mask |= (beaten < 2 ? 1u : 0u) << i;
-  }
-  return mask;
+  const uint32_t k0 = (a[0] << 2) | 3u, k1 = (a[1] << 2) | 2u;
+  const uint32_t k2 = (a[2] << 2) | 1u, k3 = a[3] << 2;
+  const uint32_t hi01 = max(k0, k1), lo01 = min(k0, k1);
+  const uint32_t hi23 = max(k2, k3), lo23 = min(k2, k3);
+  const uint32_t first = max(hi01, hi23);
+  const uint32_t second = max(min(hi01, hi23), max(lo01, lo23));
+  return (1u << (3u - (first & 3u))) | (1u << (3u - (second & 3u)));
 }
 
 // Prune/quantise/compress 8 K-values (two groups, one metadata byte).
 // Codes are computed for the kept elements only, unless the pruned-dense copy
 // is wanted as well.
 template <bool FP8, bool DENSE>
-__device__ __forceinline__ void prune8(const uint4 v, float s, uint32_t kept_vals[4],
+__device__ __forceinline__ void prune8(const uint4 v, const FastQuant &qz, uint32_t kept_vals[4],
                                        uint32_t &meta_byte, uint32_t dense_out[8]) {
   const uint32_t words[4] = {v.x, v.y, v.z, v.w};
   uint32_t h[8];
@@ -199,7 +230,7 @@ __device__ __forceinline__ void prune8(const uint4 v, float s, uint32_t kept_val
     if (DENSE) {
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const uint32_t val = FP8 ? quant_bf16(h[4 * g + t], s) : h[4 * g + t];
+        const uint32_t val = FP8 ? qz(h[4 * g + t]) : h[4 * g + t];
         dense_out[4 * g + t] = ((mk >> t) & 1u) ? val : 0u;
         if (t == i0) kept_vals[2 * g] = val;
         if (t == i1) kept_vals[2 * g + 1] = val;
@@ -211,8 +242,8 @@ __device__ __forceinline__ void prune8(const uint4 v, float s, uint32_t kept_val
         if (t == i0) h0 = h[4 * g + t];
         if (t == i1) h1 = h[4 * g + t];
       }
-      kept_vals[2 * g] = FP8 ? quant_bf16(h0, s) : h0;
-      kept_vals[2 * g + 1] = FP8 ? quant_bf16(h1, s) : h1;
+      kept_vals[2 * g] = FP8 ? qz(h0) : h0;
+      kept_vals[2 * g + 1] = FP8 ? qz(h1) : h1;
     }
   }
 }
@@ -225,7 +256,7 @@ __global__ void __launch_bounds__(256) prune24_kernel(const uint4 *__restrict__ 
                                                       void *__restrict__ values,
                                                       uint8_t *__restrict__ meta,
                                                       void *__restrict__ dense) {
-  const float s = FP8 ? *scale : 1.0f;
+  const FastQuant qz(FP8 ? *scale : 1.0f);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nwork;
        i += stride) {
@@ -234,7 +265,7 @@ __global__ void __launch_bounds__(256) prune24_kernel(const uint4 *__restrict__ 
     for (int c = 0; c < CHUNKS; ++c) v[c] = ld_stream(w + i * CHUNKS + c);
     uint32_t kv[CHUNKS][4], mb[CHUNKS], dn[CHUNKS][8];
 #pragma unroll
-    for (int c = 0; c < CHUNKS; ++c) prune8<FP8, DENSE>(v[c], s, kv[c], mb[c], dn[c]);
+    for (int c = 0; c < CHUNKS; ++c) prune8<FP8, DENSE>(v[c], qz, kv[c], mb[c], dn[c]);
     if (CHUNKS == 4) {
       reinterpret_cast<uint32_t *>(meta)[i] = mb[0] | (mb[1] << 8) | (mb[2] << 16) | (mb[3] << 24);
     } else {
@@ -275,18 +306,17 @@ __global__ void __launch_bounds__(256) prune24_kernel(const uint4 *__restrict__ 
 
 // ----------------------------------------------------------------- 6:8 decompose
 
-// 6:8 keep mask (8 bits): element i is kept when fewer than six elements beat it.
+// 6:8 keep mask (8 bits): element i is kept when fewer than six elements beat
+// it, i.e. everything but the two smallest unique keys k_i = |w_i| << 3 | (7 - i).
 __device__ __forceinline__ uint32_t keep6of8(const uint32_t a[8]) {
-  uint32_t mask = 0;
+  uint32_t k[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int beaten = 0;
+  for (int i = 0; i < 8; ++i) k[i] = (a[i] << 3) | static_cast<uint32_t>(7 - i);
+  uint32_t lo1 = min(min(min(k[0], k[1]), min(k[2], k[3])), min(min(k[4], k[5]), min(k[6], k[7])));
+  uint32_t lo2 = 0xFFFFFFFFu;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (j != i) beaten += (a[j] > a[i]) || (a[j] == a[i] && j < i);
-    mask |= (beaten < 6 ? 1u : 0u) << i;
-  }
-  return mask;
+  for (int i = 0; i < 8; ++i) lo2 = min(lo2, k[i] == lo1 ? 0xFFFFFFFFu : k[i]);
+  return 0xFFu & ~((1u << (7u - (lo1 & 7u))) | (1u << (7u - (lo2 & 7u))));
 }
 
 // Greedy window assignment: window j (positions 2j..2j+3) takes the two
@@ -312,7 +342,7 @@ __global__ void __launch_bounds__(256) slide68_kernel(const uint4 *__restrict__ 
                                                       const float *__restrict__ scale,
                                                       void *__restrict__ values,
                                                       uint8_t *__restrict__ meta) {
-  const float s = FP8 ? *scale : 1.0f;
+  const FastQuant qz(FP8 ? *scale : 1.0f);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
        i += stride) {
@@ -342,8 +372,8 @@ __global__ void __launch_bounds__(256) slide68_kernel(const uint4 *__restrict__ 
           if (t == p0) h0 = h[t];
           if (t == p1) h1 = h[t];
         }
-        vals[6 * gl + 2 * j] = FP8 ? quant_bf16(h0, s) : h0;
-        vals[6 * gl + 2 * j + 1] = FP8 ? quant_bf16(h1, s) : h1;
+        vals[6 * gl + 2 * j] = FP8 ? qz(h0) : h0;
+        vals[6 * gl + 2 * j + 1] = FP8 ? qz(h1) : h1;
       }
     }
     uint8_t *mrow = meta + 3 * i;

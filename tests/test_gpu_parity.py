@@ -331,3 +331,28 @@ def test_down_proj_workload_gemm_bf16():
     w, x = WL.weight_bits(4), WL.activation_bits(4, 256)
     y, y_ref, b = _run_sparse_bf16(x, w)
     assert_gemm_close(y, y_ref, b, "down-proj bf16")
+
+
+# ------------------------------------------------------------ quotient rounding corner cases
+
+@pytest.mark.parametrize("amax_bits", [0x3F80, 0x3FE0, 0x4049, 0x3C23, 0x43E0, 0x0080, 0x1234, 0x7F7F])
+def test_quantize_every_bf16_magnitude_against_oracle(amax_bits):
+    """Every finite bf16 value up to a chosen amax (both signs), so that the
+    kernels' quotient x / s meets every E4M3 rounding midpoint the scale
+    produces; amax from 1.0 up to the largest finite bf16 and down to the
+    smallest normal."""
+    mags = np.arange(0, amax_bits + 1, dtype=np.uint16)
+    x = np.concatenate([mags, mags | 0x8000]).astype(np.uint16)
+    pad = (-x.size) % 256
+    x = np.concatenate([x, np.zeros(pad, np.uint16)]).reshape(-1, 256)
+    q, s = sp().fp8_quantize_pertensor(dev_bf16(x))
+    ref_q, ref_s = O.quantize_pertensor(x)
+    assert host(s)[0] == ref_s
+    got = host(q)
+    assert np.array_equal(got, ref_q), np.argwhere(got != ref_q)[:5]
+    # the same values through the prune kernel (codes of kept elements)
+    w = x[:, :256]
+    c = sp().sp24_prune_compress(dev_bf16(w), "e4m3", pruned_dense=True)
+    ref = O.sp24_prune_compress(w, "e4m3")
+    assert np.array_equal(host(c["pruned_dense"]), ref["pruned_dense"])
+    assert np.array_equal(host(c["values"]), ref["values"])

@@ -174,6 +174,29 @@ int fp8_gemm_dense(const uint8_t *Xq, const float *x_scale, const uint8_t *Wq,
                    const float *w_scale, void *Y, int M, int N, int K, void *workspace,
                    size_t ws_bytes, int32_t *status, sp24_stream_t stream);
 
+/*
+ * fp8_quantize_pertensor for callers that cannot allocate device memory (the
+ * pages have no counterpart: this is a deployment convenience).  Engines and
+ * plugin hosts that own every device allocation, or hot loops that cannot
+ * afford the implicit synchronisation of cudaMalloc/cudaFree, may have no
+ * workspace to pass.  This entry point computes exactly what
+ * fp8_quantize_pertensor computes (same arguments except the workspace) and
+ * keeps the scratch of its amax reduction in a 256-byte static device array
+ * inside the library instead; every GPU that loads the library holds those
+ * bytes until the process exits.  It calls no allocating routine.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call clears the array's counters on `stream` before using them.
+ *     All calls share the one array, so calls that overlap on the GPU (other
+ *     streams, other threads) race: serialise them.
+ *   - The scratch needed does not grow with the tensor; a configuration whose
+ *     need exceeded the array would be rejected with SP24_ERR_WORKSPACE.
+ * Shape rules and errors as fp8_quantize_pertensor.
+ */
+int fp8_quantize_pertensor_static(const void *X, int64_t rows, int64_t cols, uint8_t *q,
+                                  float *scale, int32_t *status, sp24_stream_t stream);
+
 /* Bytes of workspace the op needs for these sizes (0 is a valid answer). */
 size_t sp24_workspace_size(int op, int64_t M, int64_t N, int64_t K, int dtype);
 

@@ -34,6 +34,7 @@ _sz = ctypes.c_size_t
 SIGNATURES = {
     "sp24_prune_compress": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _sz, _p, _p]),
     "fp8_quantize_pertensor": (_i, [_p, _i64, _i64, _p, _p, _p, _sz, _p, _p]),
+    "fp8_quantize_pertensor_static": (_i, [_p, _i64, _i64, _p, _p, _p, _p]),
     "slide68_decompose": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _sz, _p, _p]),
     "slide68_lift": (_i, [_p, _i, _i, _p, _p, _p, _sz, _p, _p]),
     "sp24_gemm": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _sz, _p, _p]),

@@ -48,6 +48,8 @@ int amax_then(const void *x, int64_t nelem, void *workspace, size_t ws_bytes, fl
 
 }  // namespace
 
+void sp24::set_last_cuda_error(int e) { g_last_cuda_error = e; }
+
 extern "C" {
 
 const char *sp24_version(void) { return "sp24 0.1 (sm_100a)"; }

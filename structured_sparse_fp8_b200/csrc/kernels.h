@@ -23,6 +23,9 @@ cudaError_t launch_slide68(const void *w, int64_t nelem, bool fp8, const float *
 cudaError_t launch_e4m3_encode(const float *v, uint8_t *out, int64_t n, int sm_count,
                                cudaStream_t st);
 
+// Records the CUDA error reported by sp24_last_cuda_error() (api.cu).
+void set_last_cuda_error(int e);
+
 // Bytes of scratch the amax/scale reduction uses (two counters, padded).
 constexpr size_t kAmaxWorkspaceBytes = 256;
 

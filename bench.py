@@ -221,6 +221,7 @@ class GpuWorkload:
         self.w_pool = [w_dev.clone() for _ in range(self.R_w)]
         comp_bytes = n * self.kc // 2 + n * self.kc // 8
         self.R_g = max(2 * len(ms), -(-3 * L2_BYTES // comp_bytes))
+        self.comp_bytes = comp_bytes
         self.R_g = -(-self.R_g // len(ms)) * len(ms)
         self.ws = sp.Workspace(device)
         self.ws.get(max(sp._lib.load().sp24_workspace_size(sp._lib.OP_GEMM, m, n, self.kc, 0) for m in ms) + 4096)
@@ -229,7 +230,9 @@ class GpuWorkload:
         def new_comp():
             return dict(values=torch.empty((n, self.kc // 2), dtype=torch.uint8, device=device),
                         meta=torch.empty((n, self.kc // 8), dtype=torch.uint8, device=device),
-                        scale=torch.empty((1,), dtype=torch.float32, device=device))
+                        scale=torch.empty((1,), dtype=torch.float32, device=device),
+                        packed=torch.empty(n * self.kc // 2 + n * self.kc // 8, dtype=torch.uint8,
+                                           device=device))
         self.prune_out = [new_comp() for _ in range(2)]
         self.weight_op(w_dev, self.prune_out[0])
         self.g_pool = []
@@ -238,6 +241,9 @@ class GpuWorkload:
             for key in c:
                 c[key].copy_(self.prune_out[0][key])
             self.g_pool.append(c)
+        # the GEMM streams the packed copy only: drop the canonical arrays of the pool
+        for c in self.g_pool:
+            del c["values"], c["meta"]
         self.x_host = {}
         self.x_dev, self.xq, self.sx, self.y = {}, {}, {}, {}
         for m in ms:
@@ -253,9 +259,13 @@ class GpuWorkload:
 
     # one call of each kind -------------------------------------------------
     def weight_op(self, w, out):
+        """Weight path: prune/quantise/compress (2:4) or decompose (6:8), then
+        the tile-packed copy the GEMM streams."""
         if self.is68:
-            return self.sp.slide68_decompose(w, "e4m3", status=self.status, workspace=self.ws, out=out)
-        return self.sp.sp24_prune_compress(w, "e4m3", status=self.status, workspace=self.ws, out=out)
+            self.sp.slide68_decompose(w, "e4m3", status=self.status, workspace=self.ws, out=out)
+        else:
+            self.sp.sp24_prune_compress(w, "e4m3", status=self.status, workspace=self.ws, out=out)
+        return self.sp.sp24_pack_weights(out["values"], out["meta"], out=out["packed"])
 
     def act_op(self, m):
         if self.is68:
@@ -266,23 +276,23 @@ class GpuWorkload:
 
     def gemm_op(self, m, layer):
         c = self.g_pool[layer]
-        return self.sp.sp24_gemm(self.xq[m], self.sx[m], c["values"], c["meta"], c["scale"],
-                                 out=self.y[m], status=self.status, workspace=self.ws)
+        return self.sp.sp24_gemm_packed(self.xq[m], self.sx[m], c["packed"], c["scale"], self.n,
+                                        out=self.y[m], status=self.status, workspace=self.ws)
 
     def ops_of_step(self, s):
         """(name, callable, algorithmic bytes, flops, kernel launches) of step s."""
         n, k, kc = self.n, self.k, self.kc
         ops = []
         wi = s % self.R_w
-        wname = "slide68_decompose" if self.is68 else "sp24_prune_compress"
-        wbytes = bytes_slide68(n, k) if self.is68 else bytes_prune24(n, k)
+        wname = "slide68_decompose+pack" if self.is68 else "sp24_prune_compress+pack"
+        wbytes = (bytes_slide68(n, k) if self.is68 else bytes_prune24(n, k)) + 2 * self.comp_bytes
         ops.append((wname, lambda: self.weight_op(self.w_pool[wi], self.prune_out[s % 2]), wbytes, 0, 2))
         for j, m in enumerate(self.ms):
             layer = (s * len(self.ms) + j) % self.R_g
             aname = "slide68_lift" if self.is68 else "fp8_quantize_pertensor"
             abytes = bytes_lift(m, k) if self.is68 else bytes_quant(m, k)
-            ops.append((aname, (lambda m=m: self.act_op(m)), abytes, 0, 2))
-            ops.append(("sp24_gemm", (lambda m=m, layer=layer: self.gemm_op(m, layer)),
+            ops.append((aname, (lambda m=m: self.act_op(m)), abytes, 0, 1))
+            ops.append(("sp24_gemm_packed", (lambda m=m, layer=layer: self.gemm_op(m, layer)),
                         bytes_sparse_gemm(m, n, kc), 2 * m * n * kc, 1))
         return ops
 
@@ -290,7 +300,7 @@ class GpuWorkload:
         return sum(o[2] for o in self.ops_of_step(0))
 
     def step_launches(self):
-        return sum(o[4] for o in self.ops_of_step(0))
+        return sum(o[4] for o in self.ops_of_step(0))  # one kernel per op, two for the weight path
 
     def capture(self, steps, first, events):
         torch = self.torch
@@ -333,8 +343,8 @@ class GpuWorkload:
                                               out=self.y[m], workspace=self.ws)
                         else:
                             c = self.g_pool[r % self.R_g]
-                            sp.sp24_gemm(self.xq[m], self.sx[m], c["values"], c["meta"], c["scale"],
-                                         out=self.y[m], workspace=self.ws)
+                            sp.sp24_gemm_packed(self.xq[m], self.sx[m], c["packed"], c["scale"], n,
+                                                out=self.y[m], workspace=self.ws)
                 g.replay()
                 torch.cuda.synchronize()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -432,9 +442,9 @@ def run_gpu(args, wl, rank, world, local_rank):
     dominant = max(per, key=lambda k: per[k]["t"])
     dom = per[dominant]
     traffic = load_traffic()
-    gemm_flops = per.get("sp24_gemm", {}).get("flops", 0)
-    gemm_t = per.get("sp24_gemm", {}).get("t", 1.0)
-    tensor_bound = wl["ms"][-1] >= 1024 and dominant == "sp24_gemm"
+    gemm_flops = per.get("sp24_gemm_packed", {}).get("flops", 0)
+    gemm_t = per.get("sp24_gemm_packed", {}).get("t", 1.0)
+    tensor_bound = wl["ms"][-1] >= 1024 and dominant == "sp24_gemm_packed"
     if tensor_bound:
         achieved = dom["flops"] / dom["t"] / 1e12
         peak = peaks["bf16_tflops"] * 4.0   # 2:4 sparse FP8 = 2 x FP8 = 4 x bf16 (nominal ratio)
@@ -455,7 +465,7 @@ def run_gpu(args, wl, rank, world, local_rank):
                    "frac_hbm": round(v["bytes"] / v["t"] / 1e9 / peaks["hbm_gbs"], 4)}
                for k, v in per.items()}
     if gemm_flops:
-        kernels["sp24_gemm"]["tflops"] = round(gemm_flops / gemm_t / 1e12, 2)
+        kernels["sp24_gemm_packed"]["tflops"] = round(gemm_flops / gemm_t / 1e12, 2)
 
     compare = gw.dense_compare() if rank == 0 and not args.no_compare else None
     e2e_t, h2d, d2h = gw.e2e(args.steps)
@@ -476,7 +486,7 @@ def run_gpu(args, wl, rank, world, local_rank):
         "dtype": "e4m3",
         "data": "synthetic (seeded, bf16 N(0,0.02) weights / N(0,1) activations; see workloads.py)",
         "config": {"workload": wl["name"], "n": wl["n"], "k": wl["k"], "m": list(wl["ms"]),
-                   "step": "weight prune/quantise/compress + per-M activation quantise + sparse GEMM",
+                   "step": "weight prune/quantise/compress + tile-pack, then per M: activation quantise + sparse GEMM",
                    "algorithmic_bytes_per_step": step_bytes,
                    "l2": f"inputs larger than L2: rotating pools of {gw.R_w} bf16 weight copies and "
                          f"{gw.R_g} compressed layers",

@@ -88,6 +88,7 @@ typedef struct CUstream_st *sp24_stream_t; /* identical to cudaStream_t */
 #define SP24_OP_SLIDE68_LIFT 3
 #define SP24_OP_GEMM 4
 #define SP24_OP_GEMM_DENSE 5
+#define SP24_OP_GEMM_PACKED 6
 
 /*
  * Weight path, 2:4.  W: bf16 [N, K].  For every row and every group of 4
@@ -152,17 +153,44 @@ int slide68_lift(const void *X, int M, int K, uint8_t *q_lifted, float *scale, v
  *     ignored (may be NULL).
  * w_meta u8 [N, K/8]; Y bf16 [M, N].  K is the K of the compressed operand
  * (for 6:8 weights pass K' = 3K/2 and the lifted activations).
- * When there are too few output tiles to fill the GPU, K is split over a
- * thread-block cluster of up to 8 CTAs whose partial tiles are reduced
- * through distributed shared memory in a fixed order (deterministic output).
- * The GEMMs use no workspace: sp24_workspace_size() returns 0 and
- * `workspace` may be NULL.
+ * The kernel is persistent (at most one CTA per SM).  With many output tiles
+ * each CTA takes whole tiles and needs no workspace.  With few tiles (decode
+ * shapes) the (tile, K-block) work is split evenly over the CTAs (stream-K):
+ * tiles shared by several CTAs are finished by the CTA holding their first
+ * K-block, which adds the others' fp32 partials in a fixed order, so the
+ * output is deterministic.  That needs sp24_workspace_size(SP24_OP_GEMM, ...)
+ * bytes of workspace: a 16 KB prefix of counters (zero before the first
+ * use, zero again after every call) followed by the partial tiles.
  * Shape rules: M >= 1, N % 128 == 0, K % 128 == 0 (both dtypes).
  * Y must not alias any input.
  */
 int sp24_gemm(const void *Xq, const float *x_scale, const void *w_values, const uint8_t *w_meta,
               const float *w_scale, void *Y, int M, int N, int K, int dtype, void *workspace,
               size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+
+/*
+ * Tile-packed 2:4 E4M3 weights ("tile-aligned packing" of the compressed
+ * values and metadata, as the roadmap page's §Lacunes des noyaux advises).
+ * The canonical layout stores every row's values and metadata contiguously,
+ * so one 128-row x 128-K GEMM stage touches 128 separate 64-byte and 16-byte
+ * pieces; the packed layout makes each such stage one contiguous 10240-byte
+ * block, read with a single bulk copy.  packed (u8, N*K/2 + N*K/8 bytes):
+ * block (t, kb) at byte ((t * K/128) + kb) * 10240 holds, for rows
+ * r = 0..127 of tile t, the 64 value bytes of K-block kb with 16-byte chunk c
+ * stored at chunk position c ^ ((r >> 1) & 3), followed by the 128 rows x 16
+ * metadata bytes of K-block kb.  It is a pure permutation of the canonical
+ * bytes.  Shape rules: N % 128 == 0, K % 128 == 0.
+ */
+int sp24_pack_weights(const uint8_t *values, const uint8_t *meta, int N, int K, void *packed,
+                      sp24_stream_t stream);
+
+/*
+ * sp24_gemm (E4M3) with tile-packed weights (sp24_pack_weights); same result.
+ * Workspace from sp24_workspace_size(SP24_OP_GEMM_PACKED, M, N, K, 0).
+ */
+int sp24_gemm_packed(const void *Xq, const float *x_scale, const void *packed,
+                     const float *w_scale, void *Y, int M, int N, int K, void *workspace,
+                     size_t ws_bytes, int32_t *status, sp24_stream_t stream);
 
 /*
  * Dense FP8 GEMM of the same kernel family (comparison baseline for the

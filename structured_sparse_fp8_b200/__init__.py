@@ -18,7 +18,8 @@ from ._lib import DTYPE_BF16, DTYPE_E4M3, Sp24Error  # noqa: F401
 
 __all__ = [
     "sp24_prune_compress", "fp8_quantize_pertensor", "slide68_decompose", "slide68_lift",
-    "sp24_gemm", "fp8_gemm_dense", "Workspace", "Sp24Error", "DTYPE_E4M3", "DTYPE_BF16",
+    "sp24_gemm", "fp8_gemm_dense", "sp24_pack_weights", "sp24_gemm_packed", "Workspace",
+    "Sp24Error", "DTYPE_E4M3", "DTYPE_BF16",
 ]
 
 _DT = {"e4m3": DTYPE_E4M3, "bf16": DTYPE_BF16, DTYPE_E4M3: DTYPE_E4M3, DTYPE_BF16: DTYPE_BF16}
@@ -195,6 +196,37 @@ def sp24_gemm(xq: torch.Tensor, x_scale, values: torch.Tensor, meta: torch.Tenso
     rc = lib.sp24_gemm(_ptr(xq), _ptr(x_scale), _ptr(values), _ptr(meta), _ptr(w_scale), _ptr(y),
                        M, N, K, dt, _ptr(ws), wsn, _ptr(status), _stream(xq.device))
     _lib.check(rc, "sp24_gemm")
+    return y
+
+
+def sp24_pack_weights(values: torch.Tensor, meta: torch.Tensor, out: torch.Tensor | None = None):
+    """Tile-packed copy of 2:4 E4M3 weights (values u8 [N, K/2], meta u8 [N, K/8])."""
+    lib = _lib.load()
+    _require_cuda(values, meta, out)
+    N, K = values.shape[0], values.shape[1] * 2
+    if meta.shape != (N, K // 8) or values.dtype != torch.uint8:
+        raise Sp24Error("values/meta shapes disagree")
+    packed = out if out is not None else torch.empty(N * K // 2 + N * K // 8, dtype=torch.uint8,
+                                                     device=values.device)
+    rc = lib.sp24_pack_weights(_ptr(values), _ptr(meta), N, K, _ptr(packed), _stream(values.device))
+    _lib.check(rc, "sp24_pack_weights")
+    return packed
+
+
+def sp24_gemm_packed(xq: torch.Tensor, x_scale, packed: torch.Tensor, w_scale, n: int,
+                     out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                     workspace: Workspace | None = None):
+    """Sparse E4M3 GEMM with tile-packed weights (see sp24_pack_weights)."""
+    lib = _lib.load()
+    _require_cuda(xq, x_scale, packed, w_scale, out, status)
+    M, K = xq.shape
+    if packed.numel() != n * K // 2 + n * K // 8:
+        raise Sp24Error("packed weights do not match N x K")
+    y = out if out is not None else torch.empty((M, n), dtype=torch.bfloat16, device=xq.device)
+    ws, wsn = _ws(xq.device, _lib.OP_GEMM_PACKED, M, n, K, DTYPE_E4M3, workspace)
+    rc = lib.sp24_gemm_packed(_ptr(xq), _ptr(x_scale), _ptr(packed), _ptr(w_scale), _ptr(y), M, n, K,
+                              _ptr(ws), wsn, _ptr(status), _stream(xq.device))
+    _lib.check(rc, "sp24_gemm_packed")
     return y
 
 

@@ -37,13 +37,11 @@ int cuda_status(cudaError_t e) {
   return SP24_ERR_CUDA;
 }
 
-// Runs the amax reduction, which also writes the per-tensor scale.
-int amax_then(const void *x, int64_t nelem, void *workspace, size_t ws_bytes, float *scale,
-              int32_t *status, int sms, cudaStream_t st) {
-  if (!workspace) return SP24_ERR_WORKSPACE;
-  if (ws_bytes < sp24::kAmaxWorkspaceBytes) return SP24_ERR_WORKSPACE;
-  return cuda_status(sp24::launch_amax_scale(x, nelem, static_cast<uint32_t *>(workspace), scale,
-                                             status, sms, st));
+// The single-launch kernels keep their amax counters in the workspace.
+int check_workspace(const void *workspace, size_t ws_bytes) {
+  if (!workspace || ws_bytes < sp24::kAmaxWorkspaceBytes) return SP24_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 15u) return SP24_ERR_ALIGN;
+  return SP24_OK;
 }
 
 }  // namespace
@@ -78,13 +76,15 @@ size_t sp24_workspace_size(int op, int64_t M, int64_t N, int64_t K, int dtype) {
     case SP24_OP_SLIDE68_LIFT:
       return sp24::kAmaxWorkspaceBytes;
     case SP24_OP_GEMM:
+    case SP24_OP_GEMM_PACKED:
     case SP24_OP_GEMM_DENSE: {
       if (M < 1 || N < 128 || K < 128 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return 0;
       int sms = device_sm_count();
       if (sms <= 0) sms = 148;
       const sp24::GemmKind kind =
-          op == SP24_OP_GEMM_DENSE ? sp24::kDenseE4M3
-                                   : (dtype == SP24_DTYPE_BF16 ? sp24::kSparseBF16 : sp24::kSparseE4M3);
+          op == SP24_OP_GEMM_DENSE    ? sp24::kDenseE4M3
+          : op == SP24_OP_GEMM_PACKED ? sp24::kSparseE4M3Packed
+                                      : (dtype == SP24_DTYPE_BF16 ? sp24::kSparseBF16 : sp24::kSparseE4M3);
       return sp24::plan_gemm(kind, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sms)
           .workspace_bytes();
     }
@@ -108,9 +108,11 @@ int sp24_prune_compress(const void *W, int N, int K, int out_dtype, void *values
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t nelem = static_cast<int64_t>(N) * K;
   const bool fp8 = out_dtype == SP24_DTYPE_E4M3;
-  int rc = amax_then(W, nelem, workspace, ws_bytes, fp8 ? w_scale : nullptr, status, sms, st);
+  const int rc = check_workspace(workspace, ws_bytes);
   if (rc != SP24_OK) return rc;
-  return cuda_status(sp24::launch_prune24(W, nelem, K, fp8, w_scale, values, meta, pruned_dense, sms, st));
+  return cuda_status(sp24::launch_prune24_fused(W, nelem, fp8, static_cast<uint32_t *>(workspace),
+                                                fp8 ? w_scale : nullptr, values, meta, pruned_dense,
+                                                status, sms, st));
 }
 
 int fp8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, uint8_t *q, float *scale,
@@ -123,9 +125,10 @@ int fp8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, uint8_t *q
   if (sms < 0) return SP24_ERR_ARCH;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t nelem = rows * cols;
-  int rc = amax_then(X, nelem, workspace, ws_bytes, scale, status, sms, st);
+  const int rc = check_workspace(workspace, ws_bytes);
   if (rc != SP24_OK) return rc;
-  return cuda_status(sp24::launch_quantize(X, nelem, scale, q, sms, st));
+  return cuda_status(sp24::launch_quantize_fused(X, nelem, static_cast<uint32_t *>(workspace), scale,
+                                                 q, status, sms, st));
 }
 
 int slide68_decompose(const void *W, int N, int K, int out_dtype, void *values, uint8_t *meta,
@@ -141,9 +144,11 @@ int slide68_decompose(const void *W, int N, int K, int out_dtype, void *values, 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t nelem = static_cast<int64_t>(N) * K;
   const bool fp8 = out_dtype == SP24_DTYPE_E4M3;
-  int rc = amax_then(W, nelem, workspace, ws_bytes, fp8 ? w_scale : nullptr, status, sms, st);
+  const int rc = check_workspace(workspace, ws_bytes);
   if (rc != SP24_OK) return rc;
-  return cuda_status(sp24::launch_slide68(W, nelem, fp8, w_scale, values, meta, sms, st));
+  return cuda_status(sp24::launch_slide68_fused(W, nelem, fp8, static_cast<uint32_t *>(workspace),
+                                                fp8 ? w_scale : nullptr, values, meta, status, sms,
+                                                st));
 }
 
 int slide68_lift(const void *X, int M, int K, uint8_t *q_lifted, float *scale, void *workspace,
@@ -155,16 +160,17 @@ int slide68_lift(const void *X, int M, int K, uint8_t *q_lifted, float *scale, v
   if (sms < 0) return SP24_ERR_ARCH;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t nelem = static_cast<int64_t>(M) * K;
-  int rc = amax_then(X, nelem, workspace, ws_bytes, scale, status, sms, st);
+  const int rc = check_workspace(workspace, ws_bytes);
   if (rc != SP24_OK) return rc;
-  return cuda_status(sp24::launch_lift_quantize(X, nelem, scale, q_lifted, sms, st));
+  return cuda_status(sp24::launch_lift_fused(X, nelem, static_cast<uint32_t *>(workspace), scale,
+                                             q_lifted, status, sms, st));
 }
 
 static int gemm_common(sp24::GemmKind kind, const void *Xq, const float *x_scale,
                        const void *w_values, const uint8_t *w_meta, const float *w_scale, void *Y,
                        int M, int N, int K, void *workspace, size_t ws_bytes, int32_t *status,
                        sp24_stream_t stream) {
-  const bool sparse = kind != sp24::kDenseE4M3;
+  const bool sparse = kind != sp24::kDenseE4M3 && kind != sp24::kSparseE4M3Packed;
   if (!Xq || !w_values || !Y || (sparse && !w_meta)) return SP24_ERR_NULL;
   const int kmod = 128;
   if (M < 1 || N < 128 || N % 128 != 0 || K < kmod || K % kmod != 0) return SP24_ERR_SHAPE;
@@ -191,6 +197,24 @@ int sp24_gemm(const void *Xq, const float *x_scale, const void *w_values, const 
     return gemm_common(sp24::kSparseBF16, Xq, nullptr, w_values, w_meta, nullptr, Y, M, N, K,
                        workspace, ws_bytes, status, stream);
   return SP24_ERR_DTYPE;
+}
+
+int sp24_pack_weights(const uint8_t *values, const uint8_t *meta, int N, int K, void *packed,
+                      sp24_stream_t stream) {
+  if (!values || !meta || !packed) return SP24_ERR_NULL;
+  if (N < 128 || N % 128 != 0 || K < 128 || K % 128 != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(values) || !aligned16(meta) || !aligned16(packed)) return SP24_ERR_ALIGN;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  return cuda_status(sp24::launch_pack_weights(values, meta, N, K, static_cast<uint8_t *>(packed), sms,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sp24_gemm_packed(const void *Xq, const float *x_scale, const void *packed, const float *w_scale,
+                     void *Y, int M, int N, int K, void *workspace, size_t ws_bytes, int32_t *status,
+                     sp24_stream_t stream) {
+  return gemm_common(sp24::kSparseE4M3Packed, Xq, x_scale, packed, nullptr, w_scale, Y, M, N, K,
+                     workspace, ws_bytes, status, stream);
 }
 
 int fp8_gemm_dense(const uint8_t *Xq, const float *x_scale, const uint8_t *Wq,

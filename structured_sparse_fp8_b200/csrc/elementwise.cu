@@ -10,78 +10,10 @@
 #include <stdint.h>
 
 #include "kernels.h"
+#include "quant_common.cuh"
 #include "sp24.h"
 
 namespace sp24 {
-
-// ----------------------------------------------------------------- helpers
-
-__device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-__device__ __forceinline__ float bf16_bits_to_float(uint32_t h) { return __uint_as_float(h << 16); }
-
-// E4M3 code of one fp32 value: round to nearest even, saturate to +-448, and
-// keep the sign of a value that rounds to zero (code 0x80 for negatives).
-__device__ __forceinline__ uint32_t e4m3_code(float v) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
-  uint32_t c = r & 0xFFu;
-  return c | ((__float_as_uint(v) >> 24) & 0x80u);
-}
-
-// E4M3 code of the bf16 value h divided by the dequantisation scale s, where
-// the definition takes the quotient as one correctly rounded fp32 division;
-// computed without a full division in almost every case.
-//
-// With rs = RN(1/s), q0 = RN(x * rs) is within 1.5 ulp of x/s, and one
-// residual step q1 = RN(q0 + RN(x - q0*s) * rs) (Markstein's correction,
-// P. Markstein, IBM J. Res. Dev. 34(1), 1990) is within 0.5 ulp + a tiny
-// fraction of an ulp of x/s, hence within 1 ulp of the correctly rounded
-// quotient q* = RN(x/s).  The E4M3 code of an fp32 value in the E4M3 normal
-// range depends only on which side of the grid midpoints (fp32 values whose
-// low 20 mantissa bits are 0x80000) it lies, so cvt(q1) == cvt(q*) whenever
-// q1 is more than 2 ulps away from every midpoint.  The remaining cases --
-// within 2 ulps of a midpoint, or in the E4M3 subnormal range -- take the
-// correctly rounded division.  Quotients below 2^-12 are code +-0 for any
-// value within 1 ulp, so they need no division at all.
-struct FastQuant {
-  float s, rs;
-  bool fast;  // scale and reciprocal are normal, so the residual step is valid
-  __device__ __forceinline__ explicit FastQuant(float scale) : s(scale) {
-    rs = __frcp_rn(scale);
-    const uint32_t es = (__float_as_uint(scale) >> 23) & 0xFFu;
-    const uint32_t er = (__float_as_uint(rs) >> 23) & 0xFFu;
-    fast = es > 8u && es < 247u && er > 8u && er < 247u;
-  }
-  __device__ __forceinline__ uint32_t operator()(uint32_t h) const {
-    const float x = bf16_bits_to_float(h);
-    if (!fast) return e4m3_code(__fdiv_rn(x, s));
-    const float q0 = x * rs;
-    const float r = fmaf(-q0, s, x);
-    const float q1 = fmaf(r, rs, q0);
-    const uint32_t u = __float_as_uint(q1);
-    const uint32_t mag = u & 0x7FFFFFFFu;
-    if (mag < 0x39800000u) return (h >> 8) & 0x80u;  // |q| < 2^-12: +-0 with the sign of x
-    const bool near_mid = ((u - 0x7FFFEu) & 0xFFFFFu) <= 4u;
-    if (mag < 0x3C800000u || near_mid) return e4m3_code(__fdiv_rn(x, s));  // < 2^-6 or tie zone
-    return e4m3_code(q1);
-  }
-};
-
-// Largest magnitude bit pattern among the 8 bf16 values of a 16-byte vector.
-// For finite bf16 the unsigned order of (bits & 0x7FFF) is the order of |x|;
-// NaN/Inf patterns (>= 0x7F80) sort above every finite value.
-__device__ __forceinline__ uint32_t absmax8(uint4 v) {
-  const uint32_t m = 0x7FFF7FFFu;
-  uint32_t a = __vmaxu2(__vmaxu2(v.x & m, v.y & m), __vmaxu2(v.z & m, v.w & m));
-  return max(a & 0xFFFFu, a >> 16);
-}
 
 // ----------------------------------------------------------------- amax
 
@@ -190,20 +122,6 @@ __global__ void __launch_bounds__(256) lift_quantize_kernel(const uint4 *__restr
 
 // ----------------------------------------------------------------- 2:4 prune
 
-// Kept-position mask (4 bits) of one group: element i is kept when fewer than
-// two elements beat it (larger |w|, or equal |w| at a lower index).  With the
-// unique keys k_i = |w_i| << 2 | (3 - i) "beats" is plain ">", so the kept pair
-// is the two largest keys, found with a min/max network.
-__device__ __forceinline__ uint32_t keep2of4(const uint32_t a[4]) {
-  const uint32_t k0 = (a[0] << 2) | 3u, k1 = (a[1] << 2) | 2u;
-  const uint32_t k2 = (a[2] << 2) | 1u, k3 = a[3] << 2;
-  const uint32_t hi01 = max(k0, k1), lo01 = min(k0, k1);
-  const uint32_t hi23 = max(k2, k3), lo23 = min(k2, k3);
-  const uint32_t first = max(hi01, hi23);
-  const uint32_t second = max(min(hi01, hi23), max(lo01, lo23));
-  return (1u << (3u - (first & 3u))) | (1u << (3u - (second & 3u)));
-}
-
 // Prune/quantise/compress 8 K-values (two groups, one metadata byte).
 // Codes are computed for the kept elements only, unless the pruned-dense copy
 // is wanted as well.
@@ -306,36 +224,6 @@ __global__ void __launch_bounds__(256) prune24_kernel(const uint4 *__restrict__ 
 
 // ----------------------------------------------------------------- 6:8 decompose
 
-// 6:8 keep mask (8 bits): element i is kept when fewer than six elements beat
-// it, i.e. everything but the two smallest unique keys k_i = |w_i| << 3 | (7 - i).
-__device__ __forceinline__ uint32_t keep6of8(const uint32_t a[8]) {
-  uint32_t k[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) k[i] = (a[i] << 3) | static_cast<uint32_t>(7 - i);
-  uint32_t lo1 = min(min(min(k[0], k[1]), min(k[2], k[3])), min(min(k[4], k[5]), min(k[6], k[7])));
-  uint32_t lo2 = 0xFFFFFFFFu;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) lo2 = min(lo2, k[i] == lo1 ? 0xFFFFFFFFu : k[i]);
-  return 0xFFu & ~((1u << (7u - (lo1 & 7u))) | (1u << (7u - (lo2 & 7u))));
-}
-
-// Greedy window assignment: window j (positions 2j..2j+3) takes the two
-// lowest kept positions in its range that no earlier window took.
-// pos[2j], pos[2j+1] receive the positions, ascending.
-__device__ __forceinline__ void assign_windows(uint32_t kept, int pos[6]) {
-  uint32_t left = kept;
-#pragma unroll
-  for (int j = 0; j < 3; ++j) {
-    uint32_t cand = left & (0xFu << (2 * j));
-    const int p0 = __ffs(cand) - 1;
-    cand &= cand - 1;
-    const int p1 = __ffs(cand) - 1;
-    pos[2 * j] = p0;
-    pos[2 * j + 1] = p1;
-    left &= ~((1u << p0) | (1u << p1));
-  }
-}
-
 // One thread per 16 K-values (two 8-groups -> 12 values, 6 nibbles = 3 bytes).
 template <bool FP8>
 __global__ void __launch_bounds__(256) slide68_kernel(const uint4 *__restrict__ w, int64_t n16,
@@ -403,6 +291,35 @@ __global__ void e4m3_encode_kernel(const float *__restrict__ v, uint8_t *__restr
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += stride)
     out[i] = static_cast<uint8_t>(e4m3_code(v[i]));
+}
+
+// ----------------------------------------------------------------- weight packing
+// Block (t, kb) of the packed layout = 128 rows x 64 bytes of values, each
+// row's 16-byte chunk c stored at position c ^ ((r >> 1) & 3) (the placement
+// of the 64-byte shared-memory swizzle), then 128 rows x 16 bytes of
+// metadata.  One thread per 16-byte output chunk.
+__global__ void __launch_bounds__(256) pack_kernel(const uint8_t *__restrict__ values,
+                                                   const uint8_t *__restrict__ meta, int K,
+                                                   int64_t nblocks, uint8_t *__restrict__ packed) {
+  const int KB = K / 128;
+  const int64_t nchunks = nblocks * (kPackedBlockBytes / 16);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < nchunks;
+       q += stride) {
+    const int64_t blk = q / (kPackedBlockBytes / 16);
+    const int w = static_cast<int>(q % (kPackedBlockBytes / 16));
+    const int64_t t = blk / KB;
+    const int kb = static_cast<int>(blk % KB);
+    const uint8_t *src;
+    if (w < 512) {
+      const int r = w >> 2, c = (w & 3) ^ ((r >> 1) & 3);
+      src = values + (t * 128 + r) * static_cast<int64_t>(K / 2) + kb * 64 + c * 16;
+    } else {
+      const int r = w - 512;
+      src = meta + (t * 128 + r) * static_cast<int64_t>(K / 8) + kb * 16;
+    }
+    reinterpret_cast<uint4 *>(packed + blk * kPackedBlockBytes)[w] = ld_stream(reinterpret_cast<const uint4 *>(src));
+  }
 }
 
 // ----------------------------------------------------------------- launchers
@@ -475,6 +392,14 @@ cudaError_t launch_slide68(const void *w, int64_t nelem, bool fp8, const float *
   else
     slide68_kernel<false><<<grid_for(n16, sm_count), 256, 0, st>>>(
         static_cast<const uint4 *>(w), n16, scale, values, meta);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_weights(const uint8_t *values, const uint8_t *meta, int N, int K,
+                                uint8_t *packed, int sm_count, cudaStream_t st) {
+  const int64_t nblocks = static_cast<int64_t>(N / 128) * (K / 128);
+  pack_kernel<<<grid_for(nblocks * (kPackedBlockBytes / 16), sm_count), 256, 0, st>>>(values, meta, K,
+                                                                                    nblocks, packed);
   return cudaGetLastError();
 }
 

@@ -11,8 +11,10 @@
 //               into TMEM (tcgen05.cp) and issues the tcgen05.mma(.sp)
 //               instructions, releasing each stage with tcgen05.commit;
 //   warps 2-5   epilogue: tcgen05.ld the accumulator, apply x_scale * w_scale,
-//               round to bf16 and store Y (or, under split-K, store an fp32
-//               partial and let the last CTA of the tile reduce in split order).
+//               round to bf16 and store Y (stream-K: see GemmArgs).
+// The kernel is persistent: one CTA per SM walks a list of (tile, k-range)
+// segments; two TMEM accumulators (when they fit) let the epilogue of one
+// segment overlap the main loop of the next.
 //
 // 2:4 metadata in TMEM: for kind::f8f6f4 with M = 128 every accumulator lane
 // (one W row) holds the 4-bit group descriptors of that row in K order, 64
@@ -56,6 +58,15 @@ struct KindTraits<kSparseE4M3> {
   static constexpr int kBBoxElems = 128;     // one 128-byte swizzle row of X per box
   static constexpr bool kMetaTransform = false;
   static constexpr int kMetaColsPerMma = 2;  // 64 metadata bits per row per MMA
+  static constexpr bool kPacked = false;
+};
+
+// The same MMA with the weights in the tile-packed layout: each stage's
+// values (already in the 64-byte-swizzled shared-memory order) and metadata
+// are one contiguous 10240-byte block, fetched with a single bulk copy.
+template <>
+struct KindTraits<kSparseE4M3Packed> : KindTraits<kSparseE4M3> {
+  static constexpr bool kPacked = true;
 };
 
 // Dense E4M3 (comparison kernel): 128 logical K per stage, 4 MMAs of K = 32.
@@ -77,6 +88,7 @@ struct KindTraits<kDenseE4M3> {
   static constexpr int kBBoxElems = 128;
   static constexpr bool kMetaTransform = false;
   static constexpr int kMetaColsPerMma = 0;
+  static constexpr bool kPacked = false;
 };
 
 // 2:4 sparse BF16 (kind::f16): per stage 128 logical K = 64 bf16 values (128 B)
@@ -102,6 +114,7 @@ struct KindTraits<kSparseBF16> {
   static constexpr int kBBoxElems = 64;
   static constexpr bool kMetaTransform = true;
   static constexpr int kMetaColsPerMma = 1;
+  static constexpr bool kPacked = false;
 };
 
 template <int KIND, int BN>
@@ -113,37 +126,111 @@ struct Config {
   static constexpr uint32_t kTBytes = T::kMetaTransform ? 128 * 16 : 0;  // TMEM-ready metadata
   static constexpr uint32_t kTmaBytes = kABytes + kBBytes + kEBytes;
   static constexpr uint32_t kStageBytes = kTmaBytes + kTBytes;
-  static constexpr int kBSub = T::kBRowBytes / 128;   // 128-byte X boxes per stage
-  // Small token tiles run two CTAs per SM (more loads in flight for the
-  // bandwidth-bound decode shapes); large ones one CTA with a deep ring.
-  static constexpr int kCtasPerSm = BN <= 64 ? 2 : 1;
-  static constexpr uint32_t kSmemBudget = kCtasPerSm == 2 ? 110 * 1024 : 220 * 1024;
+  static constexpr int kBSub = T::kBRowBytes / 128;  // 128-byte X boxes per stage
+  // Stage layout: [A][B][E][T] (tensor-mapped weights) or [A][E][B] (packed:
+  // A and E arrive together in one bulk copy).
+  static constexpr uint32_t kBOff = T::kPacked ? kABytes + kEBytes : kABytes;
+  static constexpr uint32_t kEOff = T::kPacked ? kABytes : kABytes + kBBytes;
+  // Persistent CTAs.  Small token tiles (decode shapes, stream-K) keep the
+  // footprint to half an SM, so that the next kernel's CTAs can already be
+  // resident, and streaming weights, while this kernel drains; large tiles
+  // take the whole SM for a deep ring.
+  static constexpr uint32_t kSmemBudget = BN <= 64 ? 108 * 1024 : 214 * 1024;
   static constexpr int kStagesRaw = static_cast<int>(kSmemBudget / kStageBytes);
-  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 512 /*bars*/;
-  static constexpr uint32_t kTmemNeed = BN + (T::kSparse ? 4 : 0);
+  static constexpr int kStages = kStagesRaw > 16 ? 16 : kStagesRaw;
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*bars*/;
+  // Two accumulators (the epilogue of one output tile overlaps the main loop
+  // of the next) whenever they fit in the 512 TMEM columns next to the 4
+  // metadata columns.
+  static constexpr uint32_t kMetaCols = T::kSparse ? 4 : 0;
+  static constexpr int kAccBufs = (2 * BN + kMetaCols <= 512) ? 2 : 1;
+  static constexpr uint32_t kTmemNeed = kAccBufs * BN + kMetaCols;
   static constexpr uint32_t kTmemCols =
       kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
   static_assert(kStages >= 2, "shared-memory ring too shallow");
-  static_assert(kStages * kStageBytes >= BN * 128 * 4, "split-K tile must fit in the idle ring");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be a multiple of 16 in [16,256]");
 };
 
-constexpr int kMaxSplits = 8;  // portable thread-block cluster size
-
+// Work decomposition.  With stream_k == 0 every CTA takes whole output tiles
+// blockIdx.x, blockIdx.x + gridDim.x, ...  With stream_k == 1 the
+// (tile, k-block) pairs are numbered u = tile * num_kb + kb and CTA g takes
+// the contiguous range [g U / G, (g + 1) U / G), so every CTA streams the same
+// number of weight bytes.  A tile split between CTAs is finished by the CTA
+// that computed its k-block 0 (the owner): the others (contributors) leave
+// fp32 partial tiles in the workspace and count themselves in the tile's
+// counter; the owner waits for them, adds the partials in CTA order
+// (deterministic) and writes Y.  A CTA's only contributor segment is its
+// first, so it never waits for anybody and owners always make progress.
 struct GemmArgs {
   int M, N, K;
   int num_kb;
-  int kb_per_split;
-  int splits;
+  int tiles_n;
+  int num_tiles;
+  int stream_k;
+  int64_t units;
   uint16_t *y;
   const float *x_scale;
   const float *w_scale;
+  float *partials;     // stream-K: [gridDim.x][128][BN] fp32
+  uint32_t *counters;  // stream-K: [num_tiles], zero between calls
   int32_t *status;
+  const uint8_t *packed;  // tile-packed weights (packed kind only)
 };
+
+enum SegRole : int { kWhole = 0, kOwner = 1, kContrib = 2 };
+
+struct Segment {
+  int tile, kb0, kb1, role;
+};
+
+struct SegIter {
+  int64_t u, u_end;
+  int tile;
+  __device__ __forceinline__ void init(const GemmArgs &p) {
+    if (p.stream_k) {
+      u = static_cast<int64_t>(blockIdx.x) * p.units / gridDim.x;
+      u_end = static_cast<int64_t>(blockIdx.x + 1) * p.units / gridDim.x;
+    } else {
+      tile = blockIdx.x;
+    }
+  }
+  __device__ __forceinline__ bool next(const GemmArgs &p, Segment &s) {
+    if (p.stream_k) {
+      if (u >= u_end) return false;
+      s.tile = static_cast<int>(u / p.num_kb);
+      s.kb0 = static_cast<int>(u % p.num_kb);
+      s.kb1 = static_cast<int>(min(static_cast<int64_t>(p.num_kb), s.kb0 + (u_end - u)));
+      s.role = s.kb0 != 0 ? kContrib : (s.kb1 == p.num_kb ? kWhole : kOwner);
+      u += s.kb1 - s.kb0;
+      return true;
+    }
+    if (tile >= p.num_tiles) return false;
+    s.tile = tile;
+    s.kb0 = 0;
+    s.kb1 = p.num_kb;
+    s.role = kWhole;
+    tile += gridDim.x;
+    return true;
+  }
+};
+
+// CTA whose stream-K range holds unit u.
+__device__ __forceinline__ int cta_of_unit(int64_t u, int64_t units, int grid) {
+  return static_cast<int>(((u + 1) * grid + units - 1) / units) - 1;
+}
 
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+__device__ __forceinline__ void red_release_add_gpu(uint32_t *p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
 // ------------------------------------------------------------------ kernel
@@ -155,6 +242,7 @@ __global__ void __launch_bounds__(192, 1)
   using T = KindTraits<KIND>;
   using C = Config<KIND, BN>;
   constexpr int S = C::kStages;
+  constexpr int NB = C::kAccBufs;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -162,28 +250,27 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * C::kStageBytes);
   uint64_t *empty = full + S;
   uint64_t *meta_ready = empty + S;
-  uint64_t *accum_bar = meta_ready + S;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum_bar + 1);
+  uint64_t *tmem_full = meta_ready + S;
+  uint64_t *tmem_empty = tmem_full + NB;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tmem_empty + NB);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_tile = blockIdx.x, m_tile = blockIdx.y, split = blockIdx.z;
-  const int n0 = n_tile * 128;
-  const int m0 = m_tile * BN;
-  const int kb_begin = split * p.kb_per_split;
-  const int kb_end = min(p.num_kb, kb_begin + p.kb_per_split);
-  const int nkb = kb_end - kb_begin;
+  const int tiles_m = (p.num_tiles + p.tiles_n - 1) / p.tiles_n;
 
   if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&tmA);
+    if (!T::kPacked) prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
-    if (T::kSparse) prefetch_tensormap(&tmE);
+    if (T::kSparse && !T::kPacked) prefetch_tensormap(&tmE);
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&meta_ready[s], 128);
     }
-    mbar_init(accum_bar, 1);
+    for (int b = 0; b < NB; ++b) {
+      mbar_init(&tmem_full[b], 1);
+      mbar_init(&tmem_empty[b], 128);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -194,27 +281,75 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Programmatic dependent launch.  This grid may start while the previous
+  // kernel in the stream is still running.  Compressed weights are only ever
+  // written by the weight-path kernels (prune/compress, decompose), which do
+  // not release their dependents early, so the producer may stream weight
+  // tiles right away; activations, scales and Y are touched only after
+  // griddepcontrol.wait, i.e. after the previous kernel has completed.
+  if (threadIdx.x != 0) grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const uint64_t keep_x = l2_policy_evict_last();    // X tiles are re-read by many CTAs
-      const uint64_t stream_w = l2_policy_evict_first();  // weights are read once
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % S;
-        const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
-        if (i >= S && !mbar_wait(&empty[s], ph ^ 1u, p.status)) break;
-        uint8_t *st = smem + s * C::kStageBytes;
-        const int kb = kb_begin + i;
-        mbar_arrive_expect_tx(&full[s], C::kTmaBytes);
-        tma_load_2d(st, &tmA, &full[s], kb * (T::kARowBytes / T::kAElemBytes), n0, stream_w);
+      const uint64_t keep_x = l2_policy_evict_last();  // X tiles are re-read by many CTAs
+      // Weights are read once when there is a single token tile; otherwise
+      // every token tile re-reads them and they should stay in L2.
+      const uint64_t stream_w = tiles_m == 1 ? l2_policy_evict_first() : l2_policy_evict_normal();
+      // weight half of a stage: values + metadata of rows n0.., k-block kb
+      auto load_weights = [&](uint8_t *st, uint64_t *bar, int n0, int kb) {
+        if constexpr (T::kPacked) {
+          const uint8_t *blk = p.packed +
+                               (static_cast<int64_t>(n0 / 128) * p.num_kb + kb) * kPackedBlockBytes;
+          bulk_load_g2s(st, blk, kPackedBlockBytes, bar, stream_w);
+        } else {
+          tma_load_2d(st, &tmA, bar, kb * (T::kARowBytes / T::kAElemBytes), n0, stream_w);
+          if (T::kSparse) tma_load_2d(st + C::kEOff, &tmE, bar, kb * T::kERowBytes, n0, stream_w);
+        }
+      };
+      // Pass 1 (before the grid dependency resolves): the weight half of the
+      // first S stages.  Pass 2: everything else, in the same stage order.
+      SegIter it;
+      it.init(p);
+      Segment sg;
+      int i = 0;
+      bool ok = true;
+      int pre = 0;  // stages whose weight tiles were issued ahead
+      {
+        SegIter it0;
+        it0.init(p);
+        Segment s0;
+        while (pre < S && it0.next(p, s0)) {
+          const int n0 = (s0.tile % p.tiles_n) * 128;
+          for (int kb = s0.kb0; kb < s0.kb1 && pre < S; ++kb, ++pre) {
+            uint8_t *st = smem + pre * C::kStageBytes;
+            mbar_arrive_expect_tx(&full[pre], C::kTmaBytes);
+            load_weights(st, &full[pre], n0, kb);
+          }
+        }
+      }
+      grid_dependency_wait();
+      while (ok && it.next(p, sg)) {
+        const int n0 = (sg.tile % p.tiles_n) * 128;
+        const int m0 = (sg.tile / p.tiles_n) * BN;
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++i) {
+          const int s = i % S;
+          const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
+          uint8_t *st = smem + s * C::kStageBytes;
+          if (i >= pre) {
+            if (i >= S && !mbar_wait(&empty[s], ph ^ 1u, p.status)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[s], C::kTmaBytes);
+            load_weights(st, &full[s], n0, kb);
+          }
 #pragma unroll
-        for (int sub = 0; sub < C::kBSub; ++sub)
-          tma_load_2d(st + C::kABytes + sub * BN * 128, &tmB, &full[s],
-                      kb * (T::kBRowBytes / T::kBElemBytes) + sub * T::kBBoxElems, m0, keep_x);
-        if (T::kSparse)
-          tma_load_2d(st + C::kABytes + C::kBBytes, &tmE, &full[s], kb * T::kERowBytes, n0,
-                      stream_w);
+          for (int sub = 0; sub < C::kBSub; ++sub)
+            tma_load_2d(st + C::kBOff + sub * BN * 128, &tmB, &full[s],
+                        kb * (T::kBRowBytes / T::kBElemBytes) + sub * T::kBBoxElems, m0, keep_x);
+        }
       }
     }
     __syncwarp();
@@ -222,139 +357,179 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = mma_idesc(128, BN, T::kFmt, T::kSparse);
-      const uint32_t d_tmem = tmem_base;
-      const uint32_t e_tmem = tmem_base + BN;
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % S;
-        const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
-        if (!mbar_wait(&full[s], ph, p.status)) break;
-        if (T::kMetaTransform && !mbar_wait(&meta_ready[s], ph, p.status)) break;
+      const uint32_t e_tmem = tmem_base + NB * BN;
+      SegIter it;
+      it.init(p);
+      Segment sg;
+      int i = 0, j = 0;
+      bool ok = true;
+      while (ok && it.next(p, sg)) {
+        const int b = j % NB;
+        const int r = j / NB;
+        if (r >= 1 && !mbar_wait(&tmem_empty[b], static_cast<uint32_t>(r - 1) & 1u, p.status)) break;
         tc_fence_after();
-        const uint32_t a_addr = smem_addr(smem + s * C::kStageBytes);
-        const uint32_t b_addr = a_addr + C::kABytes;
-        if (T::kSparse) {
-          // 128 rows x 16 B, rows contiguous: core matrices of 8 rows are 128 B apart.
-          const uint32_t e_addr = b_addr + C::kBBytes + (T::kMetaTransform ? C::kEBytes : 0);
-          tmem_copy_128x128b(e_tmem, smem_desc(e_addr, 2048, 128, kSwizzleNone));
-        }
-#pragma unroll
-        for (int kk = 0; kk < T::kMmas; ++kk) {
-          const uint64_t ad = smem_desc(a_addr + kk * T::kAStep, 16, T::kASbo, T::kASwizzle);
-          const uint32_t boff = (kk * T::kBStep / 128) * (BN * 128) + (kk * T::kBStep) % 128;
-          const uint64_t bd = smem_desc(b_addr + boff, 16, 8 * 128, kSwizzle128B);
-          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          if constexpr (KIND == kSparseE4M3) {
-            mma_f8_sparse(d_tmem, ad, bd, idesc, e_tmem + 2 * kk, acc);
-          } else if constexpr (KIND == kSparseBF16) {
-            // one metadata column per MMA; columns are addressed in pairs and
-            // the instruction descriptor's selector picks the column of the pair
-            mma_bf16_sparse(d_tmem, ad, bd, idesc | static_cast<uint32_t>(kk & 1),
-                            e_tmem + (kk & ~1), acc);
-          } else {
-            mma_f8_dense(d_tmem, ad, bd, idesc, acc);
+        const uint32_t d_tmem = tmem_base + b * BN;
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++i) {
+          const int s = i % S;
+          const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
+          if (!mbar_wait(&full[s], ph, p.status) ||
+              (T::kMetaTransform && !mbar_wait(&meta_ready[s], ph, p.status))) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          const uint32_t a_addr = smem_addr(smem + s * C::kStageBytes);
+          const uint32_t b_addr = a_addr + C::kBOff;
+          if (T::kSparse) {
+            // 128 rows x 16 B, rows contiguous: core matrices of 8 rows are 128 B apart.
+            const uint32_t e_addr = a_addr + C::kEOff + (T::kMetaTransform ? C::kEBytes : 0);
+            tmem_copy_128x128b(e_tmem, smem_desc(e_addr, 2048, 128, kSwizzleNone));
+          }
+#pragma unroll
+          for (int kk = 0; kk < T::kMmas; ++kk) {
+            const uint64_t ad = smem_desc(a_addr + kk * T::kAStep, 16, T::kASbo, T::kASwizzle);
+            const uint32_t boff = (kk * T::kBStep / 128) * (BN * 128) + (kk * T::kBStep) % 128;
+            const uint64_t bd = smem_desc(b_addr + boff, 16, 8 * 128, kSwizzle128B);
+            const uint32_t acc = (kb > sg.kb0 || kk > 0) ? 1u : 0u;
+            if constexpr (KIND == kSparseE4M3 || KIND == kSparseE4M3Packed) {
+              mma_f8_sparse(d_tmem, ad, bd, idesc, e_tmem + 2 * kk, acc);
+            } else if constexpr (KIND == kSparseBF16) {
+              // one metadata column per MMA; columns are addressed in pairs and
+              // the instruction descriptor's selector picks the column of the pair
+              mma_bf16_sparse(d_tmem, ad, bd, idesc | static_cast<uint32_t>(kk & 1),
+                              e_tmem + (kk & ~1), acc);
+            } else {
+              mma_f8_dense(d_tmem, ad, bd, idesc, acc);
+            }
+          }
+          mma_commit(&empty[s]);
         }
-        mma_commit(&empty[s]);
+        mma_commit(&tmem_full[b]);
+        ++j;
       }
-      mma_commit(accum_bar);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------ epilogue
-    const int q = warp & 3;            // TMEM lane quarter this warp may access
-    const int row = q * 32 + lane;     // W row within the tile == accumulator lane
-    const int n = n0 + row;
-    if constexpr (T::kMetaTransform) {
-      // Lane L = r0 + 8h + 16g of the TMEM metadata holds, for each of the
-      // stage's 4 MMAs j, the 16 bits of K-half h of row 16g + r0 (low half)
-      // and of row 16g + 8 + r0 (high half).
-      const int t = threadIdx.x - 64;
-      const int r0 = t & 7, h = (t >> 3) & 1, g = t >> 4;
-      const int ra = 16 * g + r0, rb = ra + 8;
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % S;
-        const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
-        if (!mbar_wait(&full[s], ph, p.status)) break;
-        const uint8_t *e = smem + s * C::kStageBytes + C::kABytes + C::kBBytes;
-        const uint16_t *ea = reinterpret_cast<const uint16_t *>(e + ra * 16);
-        const uint16_t *eb = reinterpret_cast<const uint16_t *>(e + rb * 16);
-        uint4 w;
-        w.x = ea[0 + h] | (static_cast<uint32_t>(eb[0 + h]) << 16);
-        w.y = ea[2 + h] | (static_cast<uint32_t>(eb[2 + h]) << 16);
-        w.z = ea[4 + h] | (static_cast<uint32_t>(eb[4 + h]) << 16);
-        w.w = ea[6 + h] | (static_cast<uint32_t>(eb[6 + h]) << 16);
-        *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(e) + C::kEBytes + t * 16) = w;
-        fence_proxy_async_smem();
-        mbar_arrive(&meta_ready[s]);
-      }
-    }
-    mbar_wait(accum_bar, 0, p.status);
-    tc_fence_after();
+    // ------------------------------------------------------ epilogue warps
+    const int q = warp & 3;          // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;   // W row within the tile == accumulator lane
+    const int t = threadIdx.x - 64;  // 0..127
     const float sx = p.x_scale ? __ldg(p.x_scale) : 1.0f;
     const float sw = p.w_scale ? __ldg(p.w_scale) : 1.0f;
     const float sc = sx * sw;
-    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    if (p.splits == 1) {
-#pragma unroll 1
-      for (int c = 0; c < BN; c += 16) {
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(t_row + c, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int m = m0 + c + j;
-          if (m < p.M) p.y[static_cast<size_t>(m) * p.N + n] = f32_to_bf16_bits(__uint_as_float(r[j]) * sc);
+    SegIter it;
+    it.init(p);
+    Segment sg;
+    int i = 0, j = 0;
+    while (it.next(p, sg)) {
+      if constexpr (T::kMetaTransform) {
+        // Lane L = r0 + 8h + 16g of the TMEM metadata holds, for each of the
+        // stage's 4 MMAs, the 16 bits of K-half h of row 16g + r0 (low half)
+        // and of row 16g + 8 + r0 (high half).
+        const int r0 = t & 7, h = (t >> 3) & 1, g = t >> 4;
+        const int ra = 16 * g + r0, rb = ra + 8;
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++i) {
+          const int s = i % S;
+          const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
+          if (!mbar_wait(&full[s], ph, p.status)) break;
+          const uint8_t *e = smem + s * C::kStageBytes + C::kEOff;
+          const uint16_t *ea = reinterpret_cast<const uint16_t *>(e + ra * 16);
+          const uint16_t *eb = reinterpret_cast<const uint16_t *>(e + rb * 16);
+          uint4 w;
+          w.x = ea[0 + h] | (static_cast<uint32_t>(eb[0 + h]) << 16);
+          w.y = ea[2 + h] | (static_cast<uint32_t>(eb[2 + h]) << 16);
+          w.z = ea[4 + h] | (static_cast<uint32_t>(eb[4 + h]) << 16);
+          w.w = ea[6 + h] | (static_cast<uint32_t>(eb[6 + h]) << 16);
+          *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(e) + C::kEBytes + t * 16) = w;
+          fence_proxy_async_smem();
+          mbar_arrive(&meta_ready[s]);
         }
       }
-    } else {
-      // Split-K: park this split's fp32 tile (valid token columns only) in
-      // this CTA's shared memory, red[c * 128 + row]; the ring is idle now.
-      float *red = reinterpret_cast<float *>(smem);
-      const int mvalid = min(BN, p.M - m0);
-#pragma unroll 1
-      for (int c = 0; c < mvalid; c += 16) {
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(t_row + c, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) red[(c + j) * 128 + row] = __uint_as_float(r[j]);
-      }
-    }
-  }
-
-  if (p.splits > 1) {
-    // The K-splits of one output tile form a thread-block cluster.  After the
-    // first cluster barrier every split's partial tile is in its CTA's shared
-    // memory; CTA `rank` then reduces the token columns c = rank (mod splits),
-    // reading all partials through distributed shared memory in split order
-    // (deterministic), and the second barrier keeps every CTA's shared memory
-    // alive until its peers have finished reading it.
-    cluster_sync_all();
-    if (warp >= 2) {
-      const int q = warp & 3;
-      const int row = q * 32 + lane;
+      const int b = j % NB;
+      const int r = j / NB;
+      mbar_wait(&tmem_full[b], static_cast<uint32_t>(r) & 1u, p.status);
+      tc_fence_after();
+      const int n0 = (sg.tile % p.tiles_n) * 128;
+      const int m0 = (sg.tile / p.tiles_n) * BN;
       const int n = n0 + row;
-      const int S2 = p.splits;
-      const uint32_t rank = cluster_ctarank();
       const int mvalid = min(BN, p.M - m0);
-      const float sx = p.x_scale ? __ldg(p.x_scale) : 1.0f;
-      const float sw = p.w_scale ? __ldg(p.w_scale) : 1.0f;
-      const float sc = sx * sw;
-      const uint32_t red_base = smem_addr(smem) + static_cast<uint32_t>(row) * 4u;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
+
+      if (sg.role == kContrib) {
+        // leave the fp32 partial tile (valid token columns) for the owner
+        float *mine = p.partials + (static_cast<size_t>(blockIdx.x) * 128 + row) * BN;
 #pragma unroll 1
-      for (int c = static_cast<int>(rank); c < mvalid; c += S2) {
-        const uint32_t local = red_base + static_cast<uint32_t>(c) * 128u * 4u;
-        float v[kMaxSplits];
+        for (int c = 0; c < mvalid; c += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_row + c, v);
+          tmem_ld_wait();
 #pragma unroll
-        for (int s2 = 0; s2 < kMaxSplits; ++s2)
-          v[s2] = s2 < S2 ? ld_dsmem_f32(dsmem_map(local, static_cast<uint32_t>(s2))) : 0.0f;
-        float acc = 0.0f;
+          for (int k4 = 0; k4 < 4; ++k4)
+            __stcg(reinterpret_cast<float4 *>(mine + c) + k4,
+                   make_float4(__uint_as_float(v[4 * k4]), __uint_as_float(v[4 * k4 + 1]),
+                               __uint_as_float(v[4 * k4 + 2]), __uint_as_float(v[4 * k4 + 3])));
+        }
+        tc_fence_before();
+        mbar_arrive(&tmem_empty[b]);
+        // The barrier orders every thread's partial stores before thread 0's
+        // release increment (release is cumulative), which the owner acquires.
+        named_bar_sync(1, 128);
+        if (t == 0) red_release_add_gpu(&p.counters[sg.tile], 1u);
+      } else {
+        int first = 0, last = -1;  // contributor CTAs of an owned tile
+        if (sg.role == kOwner) {
+          const int64_t u_first = static_cast<int64_t>(sg.tile) * p.num_kb;
+          first = static_cast<int>(blockIdx.x) + 1;
+          last = cta_of_unit(u_first + p.num_kb - 1, p.units, gridDim.x);
+          if (t == 0) {
+            const uint32_t expect = static_cast<uint32_t>(last - first + 1);
+            const uint64_t t0 = global_timer_ns();
+            uint32_t polls = 0;
+            while (ld_acquire_gpu(&p.counters[sg.tile]) < expect) {
+              __nanosleep(20);
+              if ((++polls & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+                if (p.status) atomicOr(p.status, SP24_STATUS_TIMEOUT);
+                break;
+              }
+            }
+            p.counters[sg.tile] = 0u;  // leave the workspace counters at zero
+          }
+          named_bar_sync(1, 128);  // the acquire by thread 0 covers the whole CTA's reads
+        }
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          if (c >= mvalid) break;
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_row + c, v);
+          tmem_ld_wait();
+          float acc[16];
 #pragma unroll
-        for (int s2 = 0; s2 < kMaxSplits; ++s2) acc += v[s2];
-        p.y[static_cast<size_t>(m0 + c) * p.N + n] = f32_to_bf16_bits(acc * sc);
+          for (int k = 0; k < 16; ++k) acc[k] = __uint_as_float(v[k]);
+          for (int g2 = first; g2 <= last; ++g2) {
+            const float4 *src =
+                reinterpret_cast<const float4 *>(p.partials + (static_cast<size_t>(g2) * 128 + row) * BN + c);
+            float4 pv[4];
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) pv[k4] = __ldcg(src + k4);
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              acc[4 * k4] += pv[k4].x;
+              acc[4 * k4 + 1] += pv[k4].y;
+              acc[4 * k4 + 2] += pv[k4].z;
+              acc[4 * k4 + 3] += pv[k4].w;
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int m = m0 + c + k;
+            if (m < p.M) p.y[static_cast<size_t>(m) * p.N + n] = f32_to_bf16_bits(acc[k] * sc);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&tmem_empty[b]);
       }
+      ++j;
     }
-    cluster_sync_all();
   }
 
   tc_fence_before();
@@ -400,15 +575,17 @@ static bool make_map(CUtensorMap *map, const void *ptr, CUtensorMapDataType dt, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Token-tile width: the MMA N.  Small token counts use the smallest tile
+// that holds them; large ones prefer 224 (two accumulators fit in tensor
+// memory, so epilogues overlap main loops) unless it pads more than 10%.
 static int choose_bn(GemmKind kind, int M) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
   if (M <= 64) return 64;
   if (M <= 128 || kind == kSparseBF16) return 128;  // bf16 X stages are twice as large
-  return 256;
+  const long pad224 = static_cast<long>((M + 223) / 224) * 224;
+  return (M >= 1024 && pad224 * 10 <= static_cast<long>(M) * 11) ? 224 : 256;
 }
-
-static int ctas_per_sm(int bn) { return bn <= 64 ? 2 : 1; }
 
 GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   GemmPlan pl{};
@@ -417,29 +594,21 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   pl.tiles_n = N / 128;
   pl.tiles_m = (M + pl.bn - 1) / pl.bn;
   pl.num_kb = K / pl.bk;
-  const int tiles = pl.tiles_n * pl.tiles_m;
-  const int slots = sm_count * ctas_per_sm(pl.bn);
-  pl.kb_per_split = pl.num_kb;
-  pl.splits = 1;
-  if (tiles * 2 <= slots) {
-    // Split K over a cluster of up to 8 CTAs so that the CTAs fill the
-    // machine; each split keeps >= 4 pipeline stages of work.
-    double best = -1.0;
-    for (int kps = pl.num_kb; kps >= 4; --kps) {
-      const int s = (pl.num_kb + kps - 1) / kps;
-      if (s > kMaxSplits) break;
-      const long units = static_cast<long>(tiles) * s;
-      const long waves = (units + slots - 1) / slots;
-      const double eff = static_cast<double>(units) / static_cast<double>(waves * slots);
-      if (eff > best + 1e-9) {
-        best = eff;
-        pl.kb_per_split = kps;
-        pl.splits = s;
-      }
-    }
+  pl.num_tiles = pl.tiles_n * pl.tiles_m;
+  pl.units = static_cast<int64_t>(pl.num_tiles) * pl.num_kb;
+  // Few tiles: stream-K over (tile, k-block) units so that every SM streams
+  // the same number of weight bytes.  Many tiles: persistent whole tiles.
+  pl.stream_k = pl.num_tiles < 2 * sm_count;
+  if (pl.stream_k) {
+    const int64_t by_work = pl.units / 4;  // at least ~4 k-blocks per CTA
+    pl.grid = static_cast<int>(by_work < 1 ? 1 : (by_work < sm_count ? by_work : sm_count));
+    if (pl.grid <= pl.num_tiles && pl.grid >= 1 && pl.units / pl.grid >= pl.num_kb)
+      ;  // whole tiles per CTA still possible; stream-K handles it uniformly
+  } else {
+    pl.grid = pl.num_tiles < sm_count ? pl.num_tiles : sm_count;
   }
-  pl.partial_bytes = 0;
-  pl.counter_bytes = 0;
+  pl.counter_bytes = pl.stream_k ? kGemmCounterBytes : 0;
+  pl.partial_bytes = pl.stream_k ? static_cast<size_t>(pl.grid) * 128 * pl.bn * sizeof(float) : 0;
   return pl;
 }
 
@@ -466,42 +635,56 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   const uint64_t a_row = T::kSparse ? static_cast<uint64_t>(K) / 2 : static_cast<uint64_t>(K);
   const CUtensorMapSwizzle a_sw =
       T::kASwizzle == kSwizzle64B ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-  if (!make_map(&tmA, w_values, dtA, T::kAElemBytes, a_row, N, T::kARowBytes / T::kAElemBytes,
-                128, a_sw))
+  if (T::kPacked) {
+    tmA = {};
+  } else if (!make_map(&tmA, w_values, dtA, T::kAElemBytes, a_row, N, T::kARowBytes / T::kAElemBytes,
+                       128, a_sw)) {
     return cudaErrorInvalidValue;
+  }
   if (!make_map(&tmB, xq, dtB, T::kBElemBytes, K, M, T::kBBoxElems, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  if (T::kSparse) {
+  if (T::kSparse && !T::kPacked) {
     if (!make_map(&tmE, w_meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(K) / 8, N,
                   16, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   } else {
-    tmE = tmA;  // unused
+    tmE = tmB;  // unused
   }
+  if (T::kPacked) tmA = tmB;  // unused
   GemmArgs a;
   a.M = M;
   a.N = N;
   a.K = K;
   a.num_kb = pl.num_kb;
-  a.kb_per_split = pl.kb_per_split;
-  a.splits = pl.splits;
+  a.tiles_n = pl.tiles_n;
+  a.num_tiles = pl.num_tiles;
+  a.stream_k = pl.stream_k ? 1 : 0;
+  a.units = pl.units;
   a.y = static_cast<uint16_t *>(y);
   a.x_scale = x_scale;
   a.w_scale = w_scale;
+  // Workspace layout: tile counters in a fixed-size prefix (zero between
+  // calls, whatever the shape), then the fp32 partial tiles (scratch).
+  a.counters = pl.stream_k ? static_cast<uint32_t *>(workspace) : nullptr;
+  a.partials = pl.stream_k
+                   ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kGemmCounterBytes)
+                   : nullptr;
   a.status = status;
-  (void)workspace;
+  a.packed = T::kPacked ? static_cast<const uint8_t *>(w_values) : nullptr;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pl.tiles_n, pl.tiles_m, pl.splits);
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.grid), 1, 1);
   cfg.blockDim = dim3(192, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = static_cast<unsigned>(pl.splits);
-  cfg.attrs = attr;
-  cfg.numAttrs = pl.splits > 1 ? 1 : 0;
+  // Programmatic dependent launch (see the kernel).  Stream-K owners wait
+  // for contributor CTAs; with at most one CTA per SM every CTA becomes
+  // resident once the SMs still held by the previous kernel drain, and each
+  // wait is bounded anyway.
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN>, tmA, tmB, tmE, a);
 }
 
@@ -515,6 +698,7 @@ static cudaError_t launch_kind(const GemmPlan &pl, const void *xq, const float *
     case 32: return launch_typed<KIND, 32>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
     case 64: return launch_typed<KIND, 64>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
     case 128: return launch_typed<KIND, 128>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+    case 224: return launch_typed<KIND, 224>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
     case 256: return launch_typed<KIND, 256>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
     default: return cudaErrorInvalidValue;
   }
@@ -531,6 +715,8 @@ cudaError_t launch_gemm(GemmKind kind, const GemmPlan &pl, const void *xq, const
       return launch_kind<kDenseE4M3>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
     case kSparseBF16:
       return launch_kind<kSparseBF16>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
+    case kSparseE4M3Packed:
+      return launch_kind<kSparseE4M3Packed>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
     default:
       return cudaErrorInvalidValue;
   }

@@ -22,6 +22,25 @@ cudaError_t launch_slide68(const void *w, int64_t nelem, bool fp8, const float *
                            void *values, uint8_t *meta, int sm_count, cudaStream_t st);
 cudaError_t launch_e4m3_encode(const float *v, uint8_t *out, int64_t n, int sm_count,
                                cudaStream_t st);
+// Re-lay 2:4 E4M3 weights (canonical values + metadata) into the GEMM's
+// tile-packed layout: one 10240-byte block per (128-row tile, 128-K block).
+cudaError_t launch_pack_weights(const uint8_t *values, const uint8_t *meta, int N, int K,
+                                uint8_t *packed, int sm_count, cudaStream_t st);
+constexpr int kPackedBlockBytes = 128 * 64 + 128 * 16;
+
+// ---- stream.cu: single-launch TMA-streamed kernels (cooperative grid).
+// `ws` must hold kAmaxWorkspaceBytes of zeroed counters; they are zero again
+// when the kernel ends.
+cudaError_t launch_quantize_fused(const void *x, int64_t nelem, uint32_t *ws, float *scale,
+                                  uint8_t *q, int32_t *status, int sm_count, cudaStream_t st);
+cudaError_t launch_lift_fused(const void *x, int64_t nelem, uint32_t *ws, float *scale,
+                              uint8_t *q, int32_t *status, int sm_count, cudaStream_t st);
+cudaError_t launch_prune24_fused(const void *w, int64_t nelem, bool fp8, uint32_t *ws,
+                                 float *scale, void *values, uint8_t *meta, void *dense,
+                                 int32_t *status, int sm_count, cudaStream_t st);
+cudaError_t launch_slide68_fused(const void *w, int64_t nelem, bool fp8, uint32_t *ws,
+                                 float *scale, void *values, uint8_t *meta, int32_t *status,
+                                 int sm_count, cudaStream_t st);
 
 // Records the CUDA error reported by sp24_last_cuda_error() (api.cu).
 void set_last_cuda_error(int e);
@@ -30,27 +49,31 @@ void set_last_cuda_error(int e);
 constexpr size_t kAmaxWorkspaceBytes = 256;
 
 // ---- gemm.cu
-enum GemmKind : int { kSparseE4M3 = 0, kDenseE4M3 = 1, kSparseBF16 = 2 };
+enum GemmKind : int { kSparseE4M3 = 0, kDenseE4M3 = 1, kSparseBF16 = 2, kSparseE4M3Packed = 3 };
 
-// How a GEMM call is cut into CTAs: tile shape, split-K factor and the
-// scratch the split-K reduction needs.
+// How a GEMM call is cut into CTAs: tile shape, work decomposition and the
+// scratch a stream-K reduction needs.
+constexpr size_t kGemmCounterBytes = 16384;  // tile counters: a fixed workspace prefix
+
 struct GemmPlan {
   int bn;            // tokens per tile (MMA N)
   int bk;            // logical K per pipeline stage
   int tiles_n;       // N / 128
   int tiles_m;       // ceil(M / bn)
   int num_kb;        // K / bk
-  int kb_per_split;  // k-blocks per split
-  int splits;        // number of non-empty splits
+  int num_tiles;
+  int64_t units;     // num_tiles * num_kb
+  bool stream_k;     // stream-K over (tile, k-block) units, else whole tiles
+  int grid;          // persistent CTAs (one per SM at most)
   size_t partial_bytes;
   size_t counter_bytes;
-  size_t workspace_bytes() const { return splits > 1 ? partial_bytes + counter_bytes : 0; }
+  size_t workspace_bytes() const { return stream_k ? counter_bytes + partial_bytes : 0; }
 };
 
 GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count);
 
 // Launch the tcgen05 GEMM.  `workspace` must hold plan.workspace_bytes()
-// zero-initialised bytes when plan.splits > 1.
+// bytes whose counter prefix is zero (it is zero again afterwards).
 cudaError_t launch_gemm(GemmKind kind, const GemmPlan &plan, const void *xq, const float *x_scale,
                         const void *w_values, const uint8_t *w_meta, const float *w_scale,
                         void *y, int M, int N, int K, void *workspace, int32_t *status,

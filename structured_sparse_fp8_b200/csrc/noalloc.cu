@@ -74,8 +74,8 @@ extern "C" int fp8_quantize_pertensor_static(const void *X, int64_t rows, int64_
   e = cudaMemsetAsync(scratch, 0, sp24::kAmaxWorkspaceBytes, st);
   const int64_t nelem = rows * cols;
   if (e == cudaSuccess)
-    e = sp24::launch_amax_scale(X, nelem, static_cast<uint32_t *>(scratch), scale, status, sms, st);
-  if (e == cudaSuccess) e = sp24::launch_quantize(X, nelem, scale, q, sms, st);
+    e = sp24::launch_quantize_fused(X, nelem, static_cast<uint32_t *>(scratch), scale, q, status,
+                                    sms, st);
   if (e != cudaSuccess) {
     sp24::set_last_cuda_error(static_cast<int>(e));
     return SP24_ERR_CUDA;

@@ -33,10 +33,14 @@ def test_status_strings_and_version(lib):
 def test_workspace_sizes(lib):
     for op in range(4):
         assert lib.sp24_workspace_size(op, 16, 256, 256, 0) == 256
-    # the GEMMs reduce split-K partials in distributed shared memory: no scratch
-    for m in (1, 64, 256, 4096):
-        assert lib.sp24_workspace_size(_lib.OP_GEMM, m, 11008, 4096, 0) == 0
-        assert lib.sp24_workspace_size(_lib.OP_GEMM_DENSE, m, 11008, 4096, 0) == 0
+    # prefill-sized GEMMs run whole tiles on persistent CTAs: no scratch
+    assert lib.sp24_workspace_size(_lib.OP_GEMM, 4096, 12288, 4096, 0) == 0
+    assert lib.sp24_workspace_size(_lib.OP_GEMM_DENSE, 4096, 12288, 4096, 0) == 0
+    # decode-sized GEMMs use stream-K: a 16 KB counter prefix + fp32 partial tiles
+    for m in (1, 64):
+        ws = lib.sp24_workspace_size(_lib.OP_GEMM, m, 11008, 4096, 0)
+        assert ws > 16384 and ws % 16 == 0
+    assert lib.sp24_workspace_size(_lib.OP_GEMM, 0, 11008, 4096, 0) == 0
 
 
 FAKE = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: calls fail validation first

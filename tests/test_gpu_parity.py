@@ -274,7 +274,7 @@ def test_slide68_workload_gemm(m):
     assert_gemm_close(torch.from_numpy(yh.view(np.int16)).view(torch.bfloat16), y_ref, b, f"6:8 M={m}")
 
 
-def test_gemm_needs_no_workspace_and_rejects_bad_shapes():
+def test_gemm_workspace_and_shape_errors():
     m = sp()
     xq = torch.zeros((1, 4096), dtype=torch.uint8, device=DEV)
     vals = torch.zeros((11008, 2048), dtype=torch.uint8, device=DEV)
@@ -283,13 +283,22 @@ def test_gemm_needs_no_workspace_and_rejects_bad_shapes():
     y = torch.empty((1, 11008), dtype=torch.bfloat16, device=DEV)
     lib = m._lib.load()
     stream = torch.cuda.current_stream().cuda_stream
+    need = lib.sp24_workspace_size(m._lib.OP_GEMM, 1, 11008, 4096, 0)
     rc = lib.sp24_gemm(xq.data_ptr(), s.data_ptr(), vals.data_ptr(), meta.data_ptr(), s.data_ptr(),
                        y.data_ptr(), 1, 11008, 4096, 0, None, 0, None, stream)
+    assert rc == m._lib.SP24_ERR_WORKSPACE
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    rc = lib.sp24_gemm(xq.data_ptr(), s.data_ptr(), vals.data_ptr(), meta.data_ptr(), s.data_ptr(),
+                       y.data_ptr(), 1, 11008, 4096, 0, ws.data_ptr(), need - 16, None, stream)
+    assert rc == m._lib.SP24_ERR_WORKSPACE
+    rc = lib.sp24_gemm(xq.data_ptr(), s.data_ptr(), vals.data_ptr(), meta.data_ptr(), s.data_ptr(),
+                       y.data_ptr(), 1, 11008, 4096, 0, ws.data_ptr(), need, None, stream)
     assert rc == m._lib.SP24_OK
     torch.cuda.synchronize()
     assert (host(y) == 0).all()
+    assert (host(ws[:16384]) == 0).all()        # the counter prefix is zero again
     rc = lib.sp24_gemm(xq.data_ptr(), s.data_ptr(), vals.data_ptr(), meta.data_ptr(), s.data_ptr(),
-                       y.data_ptr(), 1, 11008, 4000, 0, None, 0, None, stream)
+                       y.data_ptr(), 1, 11008, 4000, 0, ws.data_ptr(), need, None, stream)
     assert rc == m._lib.SP24_ERR_SHAPE
 
 
@@ -356,3 +365,57 @@ def test_quantize_every_bf16_magnitude_against_oracle(amax_bits):
     ref = O.sp24_prune_compress(w, "e4m3")
     assert np.array_equal(host(c["pruned_dense"]), ref["pruned_dense"])
     assert np.array_equal(host(c["values"]), ref["values"])
+
+
+# ------------------------------------------------------------ tile-packed weights
+
+def _pack_reference(values, meta, n, k):
+    """The documented packed layout, as a pure byte permutation (numpy)."""
+    kb_n = k // 128
+    out = np.empty(n * k // 2 + n * k // 8, dtype=np.uint8)
+    blocks = out.reshape(n // 128, kb_n, 10240)
+    v = values.reshape(n // 128, 128, kb_n, 4, 16)          # tile, row, kb, chunk, byte
+    r = np.arange(128)
+    for c in range(4):
+        pos = c ^ ((r >> 1) & 3)                             # stored chunk position per row
+        for rr in range(128):
+            blocks[:, :, rr * 64 + pos[rr] * 16: rr * 64 + pos[rr] * 16 + 16] = v[:, rr, :, c, :]
+    blocks[:, :, 8192:] = meta.reshape(n // 128, 128, kb_n, 16).transpose(0, 2, 1, 3).reshape(n // 128, kb_n, 2048)
+    return out
+
+
+@pytest.mark.parametrize("n,k", [(128, 128), (256, 512), (11008, 4096)])
+def test_pack_weights_is_the_documented_permutation(n, k):
+    w = WL.random_bits((n, k), 700 + n, scale=0.02) if n < 1024 else WL.weight_bits(2)
+    c = sp().sp24_prune_compress(dev_bf16(w), "e4m3")
+    packed = sp().sp24_pack_weights(c["values"], c["meta"])
+    want = _pack_reference(host(c["values"]), host(c["meta"]), n, k)
+    assert np.array_equal(host(packed), want)
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 128, 128), (5, 256, 512), (64, 384, 1024), (300, 256, 1152)])
+def test_packed_gemm_small(m, n, k):
+    x = WL.random_bits((m, k), 800 + m)
+    w = WL.random_bits((n, k), 900 + n, scale=0.02)
+    st = new_status()
+    c = sp().sp24_prune_compress(dev_bf16(w), "e4m3", status=st)
+    xq, sx = sp().fp8_quantize_pertensor(dev_bf16(x), status=st)
+    packed = sp().sp24_pack_weights(c["values"], c["meta"])
+    y = sp().sp24_gemm_packed(xq, sx, packed, c["scale"], n, status=st)
+    y2 = sp().sp24_gemm(xq, sx, c["values"], c["meta"], c["scale"], status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    y_ref, b = _ref(host(xq), host(sx)[0], host(c["values"]), host(c["meta"]), host(c["scale"])[0], k)
+    assert_gemm_close(y, y_ref, b, f"packed {m}x{n}x{k}")
+    assert torch.equal(y, y2)
+
+
+@pytest.mark.parametrize("m", [1, 8, 32, 64])
+def test_packed_gemm_decode_workload(m):
+    w, x = WL.weight_bits(2), WL.activation_bits(2, m)
+    c = sp().sp24_prune_compress(dev_bf16(w), "e4m3")
+    xq, sx = sp().fp8_quantize_pertensor(dev_bf16(x))
+    packed = sp().sp24_pack_weights(c["values"], c["meta"])
+    y = sp().sp24_gemm_packed(xq, sx, packed, c["scale"], 11008)
+    y_ref, b = _ref(host(xq), host(sx)[0], host(c["values"]), host(c["meta"]), host(c["scale"])[0], 4096)
+    assert_gemm_close(y, y_ref, b, f"packed decode M={m}")

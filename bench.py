@@ -7,13 +7,16 @@ W[11008, 4096] (bf16, N(0, 0.02)) with X[M, 4096] (N(0, 1)) for M in
 {1, 8, 32, 64}.  Each step
 
   * prunes, quantises and compresses one layer's weights (weight amax +
-    2:4 prune/quantise/compress: ``sp24_prune_compress``), and
+    2:4 prune/quantise/compress, written in the GEMM's tile-packed layout:
+    ``sp24_prune_compress_packed``), and
   * for each M: quantises X (``fp8_quantize_pertensor``) and runs the sparse
-    GEMM (``sp24_gemm``) against another layer's compressed weights.
+    GEMM (``sp24_gemm_packed``) against another layer's compressed weights.
+The 6:8 workload decomposes (``slide68_decompose``), tile-packs
+(``sp24_pack_weights``), lifts and quantises X (``slide68_lift``) instead.
 
-Layers rotate over pools larger than the 126 MB L2 (4 bf16 weight copies,
-8 compressed layers), so every kernel reads weights that were last touched a
-full step earlier: inputs larger than L2, no flush needed.
+Layers rotate over pools of at least three times the 126 MB L2 (bf16 weight
+copies and compressed layers), so every kernel reads weights that were last
+touched more than a full L2 ago: inputs larger than L2, no flush needed.
 
 Timing: W warm-up steps, then exactly K steps captured in one CUDA graph and
 timed with CUDA events on the launching stream, bracketed by a barrier and
@@ -227,23 +230,22 @@ class GpuWorkload:
         self.ws.get(max(sp._lib.load().sp24_workspace_size(sp._lib.OP_GEMM, m, n, self.kc, 0) for m in ms) + 4096)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
-        def new_comp():
-            return dict(values=torch.empty((n, self.kc // 2), dtype=torch.uint8, device=device),
-                        meta=torch.empty((n, self.kc // 8), dtype=torch.uint8, device=device),
-                        scale=torch.empty((1,), dtype=torch.float32, device=device),
-                        packed=torch.empty(n * self.kc // 2 + n * self.kc // 8, dtype=torch.uint8,
-                                           device=device))
-        self.prune_out = [new_comp() for _ in range(2)]
+        def new_comp(canonical):
+            c = dict(scale=torch.empty((1,), dtype=torch.float32, device=device),
+                     packed=torch.empty(n * self.kc // 2 + n * self.kc // 8, dtype=torch.uint8,
+                                        device=device))
+            if canonical:   # 6:8 decomposes into the canonical arrays, then packs
+                c["values"] = torch.empty((n, self.kc // 2), dtype=torch.uint8, device=device)
+                c["meta"] = torch.empty((n, self.kc // 8), dtype=torch.uint8, device=device)
+            return c
+        self.prune_out = [new_comp(self.is68) for _ in range(2)]
         self.weight_op(w_dev, self.prune_out[0])
-        self.g_pool = []
+        self.g_pool = []   # the GEMM streams the packed copy only
         for _ in range(self.R_g):
-            c = new_comp()
+            c = new_comp(False)
             for key in c:
                 c[key].copy_(self.prune_out[0][key])
             self.g_pool.append(c)
-        # the GEMM streams the packed copy only: drop the canonical arrays of the pool
-        for c in self.g_pool:
-            del c["values"], c["meta"]
         self.x_host = {}
         self.x_dev, self.xq, self.sx, self.y = {}, {}, {}, {}
         for m in ms:
@@ -259,13 +261,14 @@ class GpuWorkload:
 
     # one call of each kind -------------------------------------------------
     def weight_op(self, w, out):
-        """Weight path: prune/quantise/compress (2:4) or decompose (6:8), then
-        the tile-packed copy the GEMM streams."""
+        """Weight path into the tile-packed layout the GEMM streams: 2:4
+        prune/quantise/compress in one kernel; 6:8 decomposition, then the
+        tile-packed copy."""
         if self.is68:
             self.sp.slide68_decompose(w, "e4m3", status=self.status, workspace=self.ws, out=out)
-        else:
-            self.sp.sp24_prune_compress(w, "e4m3", status=self.status, workspace=self.ws, out=out)
-        return self.sp.sp24_pack_weights(out["values"], out["meta"], out=out["packed"])
+            return self.sp.sp24_pack_weights(out["values"], out["meta"], out=out["packed"])
+        return self.sp.sp24_prune_compress_packed(w, status=self.status, workspace=self.ws,
+                                                  out=out["packed"], scale=out["scale"])
 
     def act_op(self, m):
         if self.is68:
@@ -284,9 +287,11 @@ class GpuWorkload:
         n, k, kc = self.n, self.k, self.kc
         ops = []
         wi = s % self.R_w
-        wname = "slide68_decompose+pack" if self.is68 else "sp24_prune_compress+pack"
-        wbytes = (bytes_slide68(n, k) if self.is68 else bytes_prune24(n, k)) + 2 * self.comp_bytes
-        ops.append((wname, lambda: self.weight_op(self.w_pool[wi], self.prune_out[s % 2]), wbytes, 0, 2))
+        if self.is68:
+            wname, wbytes, wl = "slide68_decompose+pack", bytes_slide68(n, k) + 2 * self.comp_bytes, 2
+        else:
+            wname, wbytes, wl = "sp24_prune_compress_packed", bytes_prune24(n, k), 1
+        ops.append((wname, lambda: self.weight_op(self.w_pool[wi], self.prune_out[s % 2]), wbytes, 0, wl))
         for j, m in enumerate(self.ms):
             layer = (s * len(self.ms) + j) % self.R_g
             aname = "slide68_lift" if self.is68 else "fp8_quantize_pertensor"
@@ -300,7 +305,7 @@ class GpuWorkload:
         return sum(o[2] for o in self.ops_of_step(0))
 
     def step_launches(self):
-        return sum(o[4] for o in self.ops_of_step(0))  # one kernel per op, two for the weight path
+        return sum(o[4] for o in self.ops_of_step(0))
 
     def capture(self, steps, first, events):
         torch = self.torch
@@ -486,7 +491,9 @@ def run_gpu(args, wl, rank, world, local_rank):
         "dtype": "e4m3",
         "data": "synthetic (seeded, bf16 N(0,0.02) weights / N(0,1) activations; see workloads.py)",
         "config": {"workload": wl["name"], "n": wl["n"], "k": wl["k"], "m": list(wl["ms"]),
-                   "step": "weight prune/quantise/compress + tile-pack, then per M: activation quantise + sparse GEMM",
+                   "step": ("weight 6:8 decompose + tile-pack" if gw.is68 else
+                            "weight 2:4 prune/quantise/compress into the tile-packed layout")
+                           + ", then per M: activation quantise + sparse GEMM",
                    "algorithmic_bytes_per_step": step_bytes,
                    "l2": f"inputs larger than L2: rotating pools of {gw.R_w} bf16 weight copies and "
                          f"{gw.R_g} compressed layers",

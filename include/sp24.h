@@ -185,6 +185,20 @@ int sp24_pack_weights(const uint8_t *values, const uint8_t *meta, int N, int K, 
                       sp24_stream_t stream);
 
 /*
+ * The E4M3 2:4 weight path of sp24_prune_compress written straight into the
+ * tile-packed layout: packed receives, byte for byte, what
+ * sp24_pack_weights would make of the values and metadata that
+ * sp24_prune_compress(W, N, K, SP24_DTYPE_E4M3, ...) computes, without the
+ * canonical arrays ever being stored; w_scale <- amax|W| / 448 as there.
+ * packed: u8, N*K/2 + N*K/8 bytes.  Workspace: sp24_workspace_size(
+ * SP24_OP_PRUNE_COMPRESS, ...).  Shape rules: N % 128 == 0, K % 128 == 0,
+ * N * K <= 2^38.
+ */
+int sp24_prune_compress_packed(const void *W, int N, int K, void *packed, float *w_scale,
+                               void *workspace, size_t ws_bytes, int32_t *status,
+                               sp24_stream_t stream);
+
+/*
  * sp24_gemm (E4M3) with tile-packed weights (sp24_pack_weights); same result.
  * Workspace from sp24_workspace_size(SP24_OP_GEMM_PACKED, M, N, K, 0).
  */

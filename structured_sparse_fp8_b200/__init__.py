@@ -18,7 +18,8 @@ from ._lib import DTYPE_BF16, DTYPE_E4M3, Sp24Error  # noqa: F401
 
 __all__ = [
     "sp24_prune_compress", "fp8_quantize_pertensor", "slide68_decompose", "slide68_lift",
-    "sp24_gemm", "fp8_gemm_dense", "sp24_pack_weights", "sp24_gemm_packed", "Workspace",
+    "sp24_gemm", "fp8_gemm_dense", "sp24_pack_weights", "sp24_prune_compress_packed", "sp24_gemm_packed",
+    "Workspace",
     "Sp24Error", "DTYPE_E4M3", "DTYPE_BF16",
 ]
 
@@ -211,6 +212,31 @@ def sp24_pack_weights(values: torch.Tensor, meta: torch.Tensor, out: torch.Tenso
     rc = lib.sp24_pack_weights(_ptr(values), _ptr(meta), N, K, _ptr(packed), _stream(values.device))
     _lib.check(rc, "sp24_pack_weights")
     return packed
+
+
+def sp24_prune_compress_packed(W: torch.Tensor, status: torch.Tensor | None = None,
+                               workspace: Workspace | None = None, out: torch.Tensor | None = None,
+                               scale: torch.Tensor | None = None):
+    """E4M3 2:4 prune + quantise of W bf16 [N, K] straight into the tile-packed
+    layout (what sp24_pack_weights makes of sp24_prune_compress's output).
+
+    Returns (packed u8 [N*K/2 + N*K/8], scale f32 [1]).
+    """
+    lib = _lib.load()
+    _require_cuda(W, status, out, scale)
+    if W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise Sp24Error("W must be a 2-D bf16 tensor")
+    N, K = W.shape
+    packed = out if out is not None else torch.empty(N * K // 2 + N * K // 8, dtype=torch.uint8,
+                                                     device=W.device)
+    if packed.numel() != N * K // 2 + N * K // 8 or packed.dtype != torch.uint8:
+        raise Sp24Error("packed output has the wrong size or dtype")
+    sc = scale if scale is not None else torch.empty((1,), dtype=torch.float32, device=W.device)
+    ws, wsn = _ws(W.device, _lib.OP_PRUNE_COMPRESS, 0, N, K, DTYPE_E4M3, workspace)
+    rc = lib.sp24_prune_compress_packed(_ptr(W), N, K, _ptr(packed), _ptr(sc), _ptr(ws), wsn,
+                                        _ptr(status), _stream(W.device))
+    _lib.check(rc, "sp24_prune_compress_packed")
+    return packed, sc
 
 
 def sp24_gemm_packed(xq: torch.Tensor, x_scale, packed: torch.Tensor, w_scale, n: int,

@@ -149,30 +149,33 @@ struct Config {
       kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
   static_assert(kStages >= 2, "shared-memory ring too shallow");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be a multiple of 16 in [16,256]");
+  static constexpr int kEpiCols = BN % 32 == 0 ? 32 : 16;  // token columns per epilogue pass
 };
 
-// Work decomposition.  With stream_k == 0 every CTA takes whole output tiles
-// blockIdx.x, blockIdx.x + gridDim.x, ...  With stream_k == 1 the
-// (tile, k-block) pairs are numbered u = tile * num_kb + kb and CTA g takes
-// the contiguous range [g U / G, (g + 1) U / G), so every CTA streams the same
-// number of weight bytes.  A tile split between CTAs is finished by the CTA
-// that computed its k-block 0 (the owner): the others (contributors) leave
-// fp32 partial tiles in the workspace and count themselves in the tile's
-// counter; the owner waits for them, adds the partials in CTA order
-// (deterministic) and writes Y.  A CTA's only contributor segment is its
-// first, so it never waits for anybody and owners always make progress.
+// Work decomposition ("data-parallel + stream-K").  The first dp_tiles tiles
+// are taken whole: CTA g gets tiles g, g + G, ...  The remaining sk_tiles
+// tiles are cut into (tile, k-block) units u = t * num_kb + kb, and CTA
+// g < sk_grid takes the contiguous range [g U / sk_grid, (g + 1) U / sk_grid),
+// so the leftover work is spread evenly instead of forming a partial wave.
+// A tile split between CTAs is finished by the CTA that computed its k-block
+// 0 (the owner): the others (contributors) leave fp32 partial tiles in the
+// workspace and count themselves in the tile's counter; the owner waits for
+// them, adds the partials in CTA order (deterministic) and writes Y.  A CTA's
+// only contributor segment is the first of its range, so it never waits for
+// anybody and owners always make progress.
 struct GemmArgs {
   int M, N, K;
   int num_kb;
   int tiles_n;
   int num_tiles;
-  int stream_k;
-  int64_t units;
+  int dp_tiles;        // tiles taken whole
+  int sk_grid;         // CTAs sharing the stream-K units
+  int64_t sk_units;    // (num_tiles - dp_tiles) * num_kb
   uint16_t *y;
   const float *x_scale;
   const float *w_scale;
-  float *partials;     // stream-K: [gridDim.x][128][BN] fp32
-  uint32_t *counters;  // stream-K: [num_tiles], zero between calls
+  float *partials;     // stream-K: [sk_grid][128][BN] fp32
+  uint32_t *counters;  // stream-K: [num_tiles - dp_tiles], zero between calls
   int32_t *status;
   const uint8_t *packed;  // tile-packed weights (packed kind only)
 };
@@ -187,29 +190,28 @@ struct SegIter {
   int64_t u, u_end;
   int tile;
   __device__ __forceinline__ void init(const GemmArgs &p) {
-    if (p.stream_k) {
-      u = static_cast<int64_t>(blockIdx.x) * p.units / gridDim.x;
-      u_end = static_cast<int64_t>(blockIdx.x + 1) * p.units / gridDim.x;
-    } else {
-      tile = blockIdx.x;
+    tile = blockIdx.x;
+    u = u_end = 0;
+    if (static_cast<int>(blockIdx.x) < p.sk_grid) {
+      u = static_cast<int64_t>(blockIdx.x) * p.sk_units / p.sk_grid;
+      u_end = static_cast<int64_t>(blockIdx.x + 1) * p.sk_units / p.sk_grid;
     }
   }
   __device__ __forceinline__ bool next(const GemmArgs &p, Segment &s) {
-    if (p.stream_k) {
-      if (u >= u_end) return false;
-      s.tile = static_cast<int>(u / p.num_kb);
-      s.kb0 = static_cast<int>(u % p.num_kb);
-      s.kb1 = static_cast<int>(min(static_cast<int64_t>(p.num_kb), s.kb0 + (u_end - u)));
-      s.role = s.kb0 != 0 ? kContrib : (s.kb1 == p.num_kb ? kWhole : kOwner);
-      u += s.kb1 - s.kb0;
+    if (tile < p.dp_tiles) {
+      s.tile = tile;
+      s.kb0 = 0;
+      s.kb1 = p.num_kb;
+      s.role = kWhole;
+      tile += gridDim.x;
       return true;
     }
-    if (tile >= p.num_tiles) return false;
-    s.tile = tile;
-    s.kb0 = 0;
-    s.kb1 = p.num_kb;
-    s.role = kWhole;
-    tile += gridDim.x;
+    if (u >= u_end) return false;
+    s.tile = p.dp_tiles + static_cast<int>(u / p.num_kb);
+    s.kb0 = static_cast<int>(u % p.num_kb);
+    s.kb1 = static_cast<int>(min(static_cast<int64_t>(p.num_kb), s.kb0 + (u_end - u)));
+    s.role = s.kb0 != 0 ? kContrib : (s.kb1 == p.num_kb ? kWhole : kOwner);
+    u += s.kb1 - s.kb0;
     return true;
   }
 };
@@ -417,6 +419,7 @@ __global__ void __launch_bounds__(192, 1)
     const float sx = p.x_scale ? __ldg(p.x_scale) : 1.0f;
     const float sw = p.w_scale ? __ldg(p.w_scale) : 1.0f;
     const float sc = sx * sw;
+    constexpr int kW = C::kEpiCols;
     SegIter it;
     it.init(p);
     Segment sg;
@@ -474,53 +477,80 @@ __global__ void __launch_bounds__(192, 1)
         // The barrier orders every thread's partial stores before thread 0's
         // release increment (release is cumulative), which the owner acquires.
         named_bar_sync(1, 128);
-        if (t == 0) red_release_add_gpu(&p.counters[sg.tile], 1u);
+        if (t == 0) red_release_add_gpu(&p.counters[sg.tile - p.dp_tiles], 1u);
       } else {
         int first = 0, last = -1;  // contributor CTAs of an owned tile
         if (sg.role == kOwner) {
-          const int64_t u_first = static_cast<int64_t>(sg.tile) * p.num_kb;
+          const int64_t u_first = static_cast<int64_t>(sg.tile - p.dp_tiles) * p.num_kb;
           first = static_cast<int>(blockIdx.x) + 1;
-          last = cta_of_unit(u_first + p.num_kb - 1, p.units, gridDim.x);
+          last = cta_of_unit(u_first + p.num_kb - 1, p.sk_units, p.sk_grid);
           if (t == 0) {
             const uint32_t expect = static_cast<uint32_t>(last - first + 1);
             const uint64_t t0 = global_timer_ns();
             uint32_t polls = 0;
-            while (ld_acquire_gpu(&p.counters[sg.tile]) < expect) {
+            while (ld_acquire_gpu(&p.counters[sg.tile - p.dp_tiles]) < expect) {
               __nanosleep(20);
               if ((++polls & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
                 if (p.status) atomicOr(p.status, SP24_STATUS_TIMEOUT);
                 break;
               }
             }
-            p.counters[sg.tile] = 0u;  // leave the workspace counters at zero
+            p.counters[sg.tile - p.dp_tiles] = 0u;  // leave the workspace counters at zero
           }
           named_bar_sync(1, 128);  // the acquire by thread 0 covers the whole CTA's reads
         }
+        // kW token columns per pass.  The first contributor's partial for the
+        // next pass is loaded while this pass is summed and stored, so an
+        // owned tile costs about one L2 round trip, not one per pass.
+        const float *part0 =
+            p.partials + (static_cast<size_t>(first) * 128 + row) * BN;
+        float4 nxt[8];
+        if (first <= last) {
+#pragma unroll
+          for (int k4 = 0; k4 < kW / 4; ++k4) nxt[k4] = __ldcg(reinterpret_cast<const float4 *>(part0) + k4);
+        }
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-          if (c >= mvalid) break;
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(t_row + c, v);
+        for (int c = 0; c < mvalid; c += kW) {
+          uint32_t v[2][16];
+          tmem_ld_32x32b_x16(t_row + c, v[0]);
+          if constexpr (kW == 32) tmem_ld_32x32b_x16(t_row + c + 16, v[1]);
           tmem_ld_wait();
-          float acc[16];
+          float acc[32];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) acc[k] = __uint_as_float(v[k]);
-          for (int g2 = first; g2 <= last; ++g2) {
-            const float4 *src =
-                reinterpret_cast<const float4 *>(p.partials + (static_cast<size_t>(g2) * 128 + row) * BN + c);
-            float4 pv[4];
+          for (int k = 0; k < kW; ++k) acc[k] = __uint_as_float(v[k >> 4][k & 15]);
+          if (first <= last) {
+            float4 cur[8];
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) pv[k4] = __ldcg(src + k4);
+            for (int k4 = 0; k4 < kW / 4; ++k4) cur[k4] = nxt[k4];
+            if (c + kW < mvalid) {
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-              acc[4 * k4] += pv[k4].x;
-              acc[4 * k4 + 1] += pv[k4].y;
-              acc[4 * k4 + 2] += pv[k4].z;
-              acc[4 * k4 + 3] += pv[k4].w;
+              for (int k4 = 0; k4 < kW / 4; ++k4)
+                nxt[k4] = __ldcg(reinterpret_cast<const float4 *>(part0 + c + kW) + k4);
+            }
+#pragma unroll
+            for (int k4 = 0; k4 < kW / 4; ++k4) {
+              acc[4 * k4] += cur[k4].x;
+              acc[4 * k4 + 1] += cur[k4].y;
+              acc[4 * k4 + 2] += cur[k4].z;
+              acc[4 * k4 + 3] += cur[k4].w;
+            }
+            for (int g2 = first + 1; g2 <= last; ++g2) {  // further contributors, in CTA order
+              const float4 *src = reinterpret_cast<const float4 *>(
+                  p.partials + (static_cast<size_t>(g2) * 128 + row) * BN + c);
+              float4 pv[8];
+#pragma unroll
+              for (int k4 = 0; k4 < kW / 4; ++k4) pv[k4] = __ldcg(src + k4);
+#pragma unroll
+              for (int k4 = 0; k4 < kW / 4; ++k4) {
+                acc[4 * k4] += pv[k4].x;
+                acc[4 * k4 + 1] += pv[k4].y;
+                acc[4 * k4 + 2] += pv[k4].z;
+                acc[4 * k4 + 3] += pv[k4].w;
+              }
             }
           }
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
+          for (int k = 0; k < kW; ++k) {
             const int m = m0 + c + k;
             if (m < p.M) p.y[static_cast<size_t>(m) * p.N + n] = f32_to_bf16_bits(acc[k] * sc);
           }
@@ -561,9 +591,9 @@ static EncodeTiledFn encode_fn() {
 }
 
 // Row-major 2-D map: `inner` elements per row (contiguous), `outer` rows.
-static bool make_map(CUtensorMap *map, const void *ptr, CUtensorMapDataType dt, int elem_bytes,
-                     uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
-                     CUtensorMapSwizzle sw) {
+bool make_tensor_map_2d(CUtensorMap *map, const void *ptr, CUtensorMapDataType dt, int elem_bytes,
+                        uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+                        CUtensorMapSwizzle sw) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -578,13 +608,17 @@ static bool make_map(CUtensorMap *map, const void *ptr, CUtensorMapDataType dt, 
 // Token-tile width: the MMA N.  Small token counts use the smallest tile
 // that holds them; large ones prefer 224 (two accumulators fit in tensor
 // memory, so epilogues overlap main loops) unless it pads more than 10%.
+// Token-tile width: the MMA N.  Small token counts use the smallest tile
+// that holds them; medium ones 128 (two accumulators); large ones prefer 224
+// (still two accumulators, so epilogues overlap main loops) unless it pads
+// more than 10% over 256.
 static int choose_bn(GemmKind kind, int M) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
   if (M <= 64) return 64;
-  if (M <= 128 || kind == kSparseBF16) return 128;  // bf16 X stages are twice as large
+  if (M < 1024 || kind == kSparseBF16) return 128;
   const long pad224 = static_cast<long>((M + 223) / 224) * 224;
-  return (M >= 1024 && pad224 * 10 <= static_cast<long>(M) * 11) ? 224 : 256;
+  return pad224 * 10 <= static_cast<long>(M) * 11 ? 224 : 256;
 }
 
 GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
@@ -596,19 +630,29 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   pl.num_kb = K / pl.bk;
   pl.num_tiles = pl.tiles_n * pl.tiles_m;
   pl.units = static_cast<int64_t>(pl.num_tiles) * pl.num_kb;
-  // Few tiles: stream-K over (tile, k-block) units so that every SM streams
-  // the same number of weight bytes.  Many tiles: persistent whole tiles.
-  pl.stream_k = pl.num_tiles < 2 * sm_count;
-  if (pl.stream_k) {
-    const int64_t by_work = pl.units / 4;  // at least ~4 k-blocks per CTA
-    pl.grid = static_cast<int>(by_work < 1 ? 1 : (by_work < sm_count ? by_work : sm_count));
-    if (pl.grid <= pl.num_tiles && pl.grid >= 1 && pl.units / pl.grid >= pl.num_kb)
-      ;  // whole tiles per CTA still possible; stream-K handles it uniformly
-  } else {
-    pl.grid = pl.num_tiles < sm_count ? pl.num_tiles : sm_count;
-  }
+  // Persistent grid: one CTA per SM, fewer only when there are fewer than
+  // two k-blocks per CTA.
+  int64_t G = pl.units / 2;
+  if (G > sm_count) G = sm_count;
+  if (G < 1) G = 1;
+  pl.grid = static_cast<int>(G);
+  // Whole tiles for the full waves, stream-K over the leftover tiles so that
+  // the last partial wave is spread over every CTA.
+  pl.dp_tiles = (pl.num_tiles / pl.grid) * pl.grid;
+  const int rem = pl.num_tiles - pl.dp_tiles;
+  pl.sk_units = static_cast<int64_t>(rem) * pl.num_kb;
+  // Tiles wider than 64 tokens are split at most two ways: their owners then
+  // read a single, prefetched partial.  Narrower (decode) tiles have at most
+  // two epilogue passes, so they split as finely as the grid allows.
+  int64_t skg = pl.sk_units / 2;  // at least two k-blocks per CTA
+  if (skg > pl.grid) skg = pl.grid;
+  if (pl.bn > 64 && skg > 2 * static_cast<int64_t>(rem)) skg = 2 * static_cast<int64_t>(rem);
+  if (skg < rem) skg = rem;
+  pl.sk_grid = rem > 0 ? static_cast<int>(skg) : 0;
+  if (pl.dp_tiles == 0) pl.grid = pl.sk_grid;  // no idle CTAs when every tile is split
+  pl.stream_k = rem > 0;
   pl.counter_bytes = pl.stream_k ? kGemmCounterBytes : 0;
-  pl.partial_bytes = pl.stream_k ? static_cast<size_t>(pl.grid) * 128 * pl.bn * sizeof(float) : 0;
+  pl.partial_bytes = pl.stream_k ? static_cast<size_t>(pl.sk_grid) * 128 * pl.bn * sizeof(float) : 0;
   return pl;
 }
 
@@ -637,14 +681,14 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
       T::kASwizzle == kSwizzle64B ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   if (T::kPacked) {
     tmA = {};
-  } else if (!make_map(&tmA, w_values, dtA, T::kAElemBytes, a_row, N, T::kARowBytes / T::kAElemBytes,
+  } else if (!make_tensor_map_2d(&tmA, w_values, dtA, T::kAElemBytes, a_row, N, T::kARowBytes / T::kAElemBytes,
                        128, a_sw)) {
     return cudaErrorInvalidValue;
   }
-  if (!make_map(&tmB, xq, dtB, T::kBElemBytes, K, M, T::kBBoxElems, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_tensor_map_2d(&tmB, xq, dtB, T::kBElemBytes, K, M, T::kBBoxElems, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (T::kSparse && !T::kPacked) {
-    if (!make_map(&tmE, w_meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(K) / 8, N,
+    if (!make_tensor_map_2d(&tmE, w_meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(K) / 8, N,
                   16, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   } else {
@@ -658,8 +702,9 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   a.num_kb = pl.num_kb;
   a.tiles_n = pl.tiles_n;
   a.num_tiles = pl.num_tiles;
-  a.stream_k = pl.stream_k ? 1 : 0;
-  a.units = pl.units;
+  a.dp_tiles = pl.dp_tiles;
+  a.sk_grid = pl.sk_grid;
+  a.sk_units = pl.sk_units;
   a.y = static_cast<uint16_t *>(y);
   a.x_scale = x_scale;
   a.w_scale = w_scale;

@@ -1,25 +1,24 @@
 // kernels.h -- internal launch interface between the C ABI (api.cu) and the
-// kernels (elementwise.cu, gemm.cu).  Not installed; not part of the ABI.
+// kernels (elementwise.cu, gemm.cu, stream.cu).  Not installed; not part of
+// the ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
 
 namespace sp24 {
 
+// 2-D tiled TMA descriptor of a row-major [outer, inner] tensor of
+// elem_bytes-sized elements (row pitch inner * elem_bytes), box
+// [box_outer, box_inner].  False when the driver entry point is missing or
+// the encoder rejects the arguments.
+bool make_tensor_map_2d(CUtensorMap *map, const void *ptr, CUtensorMapDataType dt, int elem_bytes,
+                        uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+                        CUtensorMapSwizzle sw);
+
 // ---- elementwise.cu
-cudaError_t launch_amax_scale(const void *x, int64_t nelem, uint32_t *ws, float *scale,
-                              int32_t *status, int sm_count, cudaStream_t st);
-cudaError_t launch_quantize(const void *x, int64_t nelem, const float *scale, uint8_t *q,
-                            int sm_count, cudaStream_t st);
-cudaError_t launch_lift_quantize(const void *x, int64_t nelem, const float *scale, uint8_t *q,
-                                 int sm_count, cudaStream_t st);
-cudaError_t launch_prune24(const void *w, int64_t nelem, int64_t k, bool fp8, const float *scale,
-                           void *values, uint8_t *meta, void *dense, int sm_count,
-                           cudaStream_t st);
-cudaError_t launch_slide68(const void *w, int64_t nelem, bool fp8, const float *scale,
-                           void *values, uint8_t *meta, int sm_count, cudaStream_t st);
 cudaError_t launch_e4m3_encode(const float *v, uint8_t *out, int64_t n, int sm_count,
                                cudaStream_t st);
 // Re-lay 2:4 E4M3 weights (canonical values + metadata) into the GEMM's
@@ -38,6 +37,11 @@ cudaError_t launch_lift_fused(const void *x, int64_t nelem, uint32_t *ws, float 
 cudaError_t launch_prune24_fused(const void *w, int64_t nelem, bool fp8, uint32_t *ws,
                                  float *scale, void *values, uint8_t *meta, void *dense,
                                  int32_t *status, int sm_count, cudaStream_t st);
+// 2:4 prune + E4M3 quantise written straight into the tile-packed layout
+// (N % 128 == 0, K % 128 == 0).
+cudaError_t launch_prune24_packed_fused(const void *w, int N, int K, uint32_t *ws, float *scale,
+                                        uint8_t *packed, int32_t *status, int sm_count,
+                                        cudaStream_t st);
 cudaError_t launch_slide68_fused(const void *w, int64_t nelem, bool fp8, uint32_t *ws,
                                  float *scale, void *values, uint8_t *meta, int32_t *status,
                                  int sm_count, cudaStream_t st);
@@ -63,8 +67,11 @@ struct GemmPlan {
   int num_kb;        // K / bk
   int num_tiles;
   int64_t units;     // num_tiles * num_kb
-  bool stream_k;     // stream-K over (tile, k-block) units, else whole tiles
+  bool stream_k;     // some tiles are split over CTAs (needs the workspace)
   int grid;          // persistent CTAs (one per SM at most)
+  int dp_tiles;      // tiles taken whole
+  int sk_grid;       // CTAs sharing the leftover tiles' (tile, k-block) units
+  int64_t sk_units;
   size_t partial_bytes;
   size_t counter_bytes;
   size_t workspace_bytes() const { return stream_k ? counter_bytes + partial_bytes : 0; }

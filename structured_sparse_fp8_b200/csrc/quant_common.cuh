@@ -29,52 +29,13 @@ __device__ __forceinline__ uint32_t e4m3_code(float v) {
   return c | ((__float_as_uint(v) >> 24) & 0x80u);
 }
 
-// E4M3 code of the bf16 value h divided by the dequantisation scale s, where
-// the definition takes the quotient as one correctly rounded fp32 division;
-// computed without a full division in almost every case.
-//
-// With rs = RN(1/s), q0 = RN(x * rs) is within 1.5 ulp of x/s, and one
-// residual step q1 = RN(q0 + RN(x - q0*s) * rs) (Markstein's correction,
-// P. Markstein, IBM J. Res. Dev. 34(1), 1990) is within 0.5 ulp + a tiny
-// fraction of an ulp of x/s, hence within 1 ulp of the correctly rounded
-// quotient q* = RN(x/s).  The E4M3 code of an fp32 value in the E4M3 normal
-// range depends only on which side of the grid midpoints (fp32 values whose
-// low 20 mantissa bits are 0x80000) it lies, so cvt(q1) == cvt(q*) whenever
-// q1 is more than 2 ulps away from every midpoint.  The remaining cases --
-// within 2 ulps of a midpoint, or in the E4M3 subnormal range -- take the
-// correctly rounded division.  Quotients below 2^-12 are code +-0 for any
-// value within 1 ulp, so they need no division at all.
-struct FastQuant {
-  float s, rs;
-  bool fast;  // scale and reciprocal are normal, so the residual step is valid
-  __device__ __forceinline__ explicit FastQuant(float scale) : s(scale) {
-    rs = __frcp_rn(scale);
-    const uint32_t es = (__float_as_uint(scale) >> 23) & 0xFFu;
-    const uint32_t er = (__float_as_uint(rs) >> 23) & 0xFFu;
-    fast = es > 8u && es < 247u && er > 8u && er < 247u;
-  }
-  __device__ __forceinline__ uint32_t operator()(uint32_t h) const {
-    const float x = bf16_bits_to_float(h);
-    if (!fast) return e4m3_code(__fdiv_rn(x, s));
-    const float q0 = x * rs;
-    const float r = fmaf(-q0, s, x);
-    const float q1 = fmaf(r, rs, q0);
-    const uint32_t u = __float_as_uint(q1);
-    const uint32_t mag = u & 0x7FFFFFFFu;
-    if (mag < 0x39800000u) return (h >> 8) & 0x80u;  // |q| < 2^-12: +-0 with the sign of x
-    const bool near_mid = ((u - 0x7FFFEu) & 0xFFFFFu) <= 4u;
-    if (mag < 0x3C800000u || near_mid) return e4m3_code(__fdiv_rn(x, s));  // < 2^-6 or tie zone
-    return e4m3_code(q1);
-  }
-};
-
-// Largest magnitude bit pattern among the 8 bf16 values of a 16-byte vector.
-// For finite bf16 the unsigned order of (bits & 0x7FFF) is the order of |x|;
-// NaN/Inf patterns (>= 0x7F80) sort above every finite value.
-__device__ __forceinline__ uint32_t absmax8(uint4 v) {
+// Largest magnitude bit patterns of the 8 bf16 values of a 16-byte vector,
+// per 16-bit lane (the larger lane is the vector's).  For finite bf16 the
+// unsigned order of (bits & 0x7FFF) is the order of |x|; NaN/Inf patterns
+// (>= 0x7F80) sort above every finite value.
+__device__ __forceinline__ uint32_t absmax8x2(uint4 v) {
   const uint32_t m = 0x7FFF7FFFu;
-  uint32_t a = __vmaxu2(__vmaxu2(v.x & m, v.y & m), __vmaxu2(v.z & m, v.w & m));
-  return max(a & 0xFFFFu, a >> 16);
+  return __vmaxu2(__vmaxu2(v.x & m, v.y & m), __vmaxu2(v.z & m, v.w & m));
 }
 
 // Kept-position mask (4 bits) of one group: element i is kept when fewer than

@@ -3,27 +3,33 @@
 //   kOpQuantize  per-tensor E4M3 quantisation of activations,
 //   kOpLift      the same fused with the 6:8 activation lift,
 //   kOpPrune24   2:4 magnitude prune + quantise + compress of weights,
+//   kOpPrune24Packed  the same, written in the GEMM's tile-packed layout,
 //   kOpSlide68   6:8 prune + sliding-window decomposition of weights.
 //
 // One CTA per SM (cooperative launch: all CTAs resident), each owning a
-// contiguous range of 32 KB chunks of the bf16 input.  A producer warp
-// streams the chunks into a 6-stage shared-memory ring with bulk TMA copies
-// (full/empty mbarriers per slot), 16 consumer warps work on interleaved
-// 16-byte units of each chunk.
-//   Phase 1: amax of the slice (and, for the prune ops, the group selection,
-//            whose metadata is written straight to global memory).
+// contiguous range of 32 KB chunks of the bf16 input (for the packed 2:4 op a
+// chunk is the 128 x 128 box of W behind one packed block, read with a 2-D
+// tensor copy).  A producer warp streams the chunks into a 5-stage
+// shared-memory ring (full/empty mbarriers per slot), 16 consumer warps work
+// on interleaved 16-byte units of each chunk.
+//   Phase 1: amax of the slice, and for the prune ops the group selection,
+//            whose metadata goes straight to global memory (this phase is
+//            bound by HBM, so the selection's arithmetic hides under it).
 //   Grid barrier: the CTAs combine their amax through device counters that
 //            the last CTA to leave resets; every CTA derives s = amax / 448
-//            and fills a 3 KB code table in shared memory with the E4M3 code
-//            of every bf16 magnitude that can produce a nonzero code (the 24
-//            binades below amax), each entry computed as the definition
-//            states: E4M3(RN_fp32(x / s)).
-//   Phase 2: codes by table lookup; the slice comes from the ring again when
-//            the CTA's whole range fitted in it, else it is re-streamed
-//            (normally from L2).
+//            and fills a 64 KB table in shared memory with the E4M3 code of
+//            every bf16 bit pattern: the 24 binades below amax computed as
+//            the definition states, E4M3(RN_fp32(x / s)), signed zeros for
+//            everything smaller.
+//   Phase 2: codes by table lookup (2:4: of the kept pair named by the
+//            metadata, read back one chunk ahead); the slice comes from the
+//            ring again when the CTA's whole range fitted in it, else it is
+//            re-streamed in reverse chunk order, so the chunks phase 1 read
+//            last, the likeliest to still be in L2, are read first.
 // The bf16-output prune ops need no scale and finish after phase 1.
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #include <mutex>
 
@@ -39,11 +45,13 @@ namespace {
 constexpr int kConsumers = 512;              // 16 consumer warps
 constexpr int kThreads = kConsumers + 32;    // + one producer warp
 constexpr int kChunkBytes = 32768;
-constexpr int kStages = 6;
-constexpr int kTab = 24 * 128;               // 24 binades x 128 mantissas
-constexpr uint32_t kSmemBytes = kStages * kChunkBytes + kTab + 2 * kStages * 8 + 128;
+constexpr int kStages = 5;
+constexpr int kTab = 24 * 128;               // binades x mantissas that can give a nonzero code
+constexpr int kTabBytes = 65536;             // code of every bf16 bit pattern
+constexpr uint32_t kSmemBytes = kStages * kChunkBytes + kTabBytes + 2 * kStages * 8 + 128;
+static_assert(kSmemBytes + 2048 <= 227 * 1024, "ring + table exceed the shared memory of a CTA");
 
-enum StreamOp : int { kOpQuantize = 0, kOpLift = 1, kOpPrune24 = 2, kOpSlide68 = 3 };
+enum StreamOp : int { kOpQuantize = 0, kOpLift = 1, kOpPrune24 = 2, kOpSlide68 = 3, kOpPrune24Packed = 4 };
 
 // Bytes of input one consumer thread handles as one unit: 8 bf16 (one
 // metadata byte of 2:4, one 8-group of the lift) or 16 bf16 for 6:8 (two
@@ -55,15 +63,20 @@ template <int OP>
 __host__ __device__ constexpr int unit_bytes() { return OP == kOpSlide68 ? 32 : 16; }
 
 struct StreamArgs {
+  // kOpPrune24Packed reads W through this 2-D map (box 128 rows x 128 bf16):
+  // chunk c is the input of packed block c, rows 128 (c / kblocks) ..,
+  // columns 128 (c % kblocks) ..
+  CUtensorMap wmap;
   const uint8_t *x;  // bf16 input
   int64_t nbytes;    // input bytes, a multiple of 32
   int64_t nchunks;
   uint32_t *ws;      // [0] amax bits, [1] arrivals, [2] departures
   float *scale_out;
   int32_t *status;
-  uint8_t *out;      // codes / kept values
+  uint8_t *out;      // codes / kept values (the packed blocks for kOpPrune24Packed)
   uint8_t *meta;
   uint8_t *dense;
+  uint32_t kblocks;  // kOpPrune24Packed: K / 128
 };
 
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
@@ -75,40 +88,58 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
       : "memory");
 }
 
+__device__ __forceinline__ void red_max_relaxed_gpu(uint32_t *p, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_add_release_gpu(uint32_t *p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 
-// E4M3 code of a bf16 pattern by lookup: entry i of the table holds the
-// magnitude code of exponent field (base7 >> 7) + i / 128, mantissa i % 128.
-// Smaller magnitudes are below 2^-13 after division and encode to +-0.
-// With `direct` set (tensors too small to amortise the table) the code is
-// computed by the same division directly.
+// E4M3 code of a bf16 pattern by lookup: entry h of the 64 KB table is the
+// code of the bf16 pattern h.  Only the 24 binades at and below amax's can
+// give a nonzero code (smaller magnitudes are below 2^-13 after division);
+// every other pattern holds the zero code of its sign.  DIRECT (tensors too
+// small to amortise the table) computes the code by the same division.
+template <bool DIRECT>
 struct CodeTable {
   const uint8_t *tab;
-  int base7;
   float s;
-  bool direct;
   __device__ __forceinline__ uint32_t operator()(uint32_t h) const {
-    if (direct) return e4m3_code(__fdiv_rn(bf16_bits_to_float(h), s));
-    const int idx = static_cast<int>(h & 0x7FFFu) - base7;
-    const uint32_t c = static_cast<unsigned>(idx) < static_cast<unsigned>(kTab) ? tab[idx] : 0u;
-    return c | ((h >> 8) & 0x80u);
+    if constexpr (DIRECT)
+      return e4m3_code(__fdiv_rn(bf16_bits_to_float(h), s));
+    else
+      return tab[h];
   }
 };
 
-__device__ __forceinline__ void build_table(uint8_t *tab, uint32_t amax_bits, float s, int t) {
+// The table: signed zeros everywhere (zero_table, before phase 1), then the
+// 24 binades below amax (fill_table), each entry as the definition states,
+// E4M3(RN_fp32(x / s)) (the code of -x is the code of x with the sign bit).
+__device__ __forceinline__ void zero_table(uint8_t *tab, int t) {
+  uint4 *t4 = reinterpret_cast<uint4 *>(tab);
+  for (int i = t; i < kTabBytes / 16; i += kConsumers) {
+    const uint32_t z = i < kTabBytes / 32 ? 0u : 0x80808080u;
+    t4[i] = make_uint4(z, z, z, z);
+  }
+}
+
+__device__ __forceinline__ void fill_table(uint8_t *tab, uint32_t amax_bits, float s, int t) {
   const int e_base = static_cast<int>(amax_bits >> 7) - 23;
   for (int i = t; i < kTab; i += kConsumers) {
     const int e = e_base + i / 128;
-    uint32_t c = 0;
     if (e >= 0 && e < 255) {
       const uint32_t h = (static_cast<uint32_t>(e) << 7) | static_cast<uint32_t>(i & 127);
-      c = e4m3_code(__fdiv_rn(bf16_bits_to_float(h), s)) & 0x7Fu;
+      const uint32_t c = e4m3_code(__fdiv_rn(bf16_bits_to_float(h), s)) & 0x7Fu;
+      tab[h] = static_cast<uint8_t>(c);
+      tab[h | 0x8000u] = static_cast<uint8_t>(c | 0x80u);
     }
-    tab[i] = static_cast<uint8_t>(c);
   }
 }
 
@@ -117,10 +148,152 @@ __device__ __forceinline__ void halves(const uint4 v, uint32_t h[8]) {
   h[4] = v.z & 0xFFFFu; h[5] = v.z >> 16; h[6] = v.w & 0xFFFFu; h[7] = v.w >> 16;
 }
 
-// ------------------------------------------------------------------ phase 1
-// One unit: `p` its bytes in shared memory, `e0` the index of its first element.
+// A chunk's first element e (a multiple of kChunkBytes / 2).  Unit u of the
+// chunk starts at element e + u * kUnit / 2; addresses are formed as
+// per-chunk 64-bit bases plus 32-bit offsets of u.
+struct Chunk {
+  uint64_t e;
+  uint64_t idx;  // the chunk's index (= its packed block for kOpPrune24Packed)
+};
+
+// ------------------------------------------------------------------ 2:4 + E4M3
+// The 2:4 selection and E4M3 codes of one 8-element unit (two groups), from
+// its four 32-bit words (two bf16 each, lower index in the low half).
+// Every element gets the key  |w| << 17 | (3 - i) << 1 | sign:  keys are
+// unique, and "larger key" is exactly "beats" of the rule (larger |w|, or
+// equal |w| at the lower index), so the kept pair is the two largest keys,
+// found with a min/max network.  The sign rides along in bit 0, below the
+// index, where it cannot affect the order.  Returns the four codes (kept
+// elements in ascending index order, group 0 first); `mb` receives the
+// metadata byte, `dn` (DENSE) the 8 codes with zeros at pruned positions.
+template <bool DENSE, class Code>
+__device__ __forceinline__ uint32_t prune24_encode(const uint4 v, const Code &code, uint32_t &mb,
+                                                   uint2 &dn) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out = 0;
+  mb = 0;
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const uint32_t lo = w[2 * g], hi = w[2 * g + 1];
+    // rotate the element's magnitude to bits 17..31 and its sign to bit 0
+    const uint32_t k0 = (__funnelshift_l(lo, lo, 17) & 0xFFFE0001u) | (3u << 1);
+    const uint32_t k1 = (__funnelshift_l(lo, lo, 1) & 0xFFFE0001u) | (2u << 1);
+    const uint32_t k2 = (__funnelshift_l(hi, hi, 17) & 0xFFFE0001u) | (1u << 1);
+    const uint32_t k3 = __funnelshift_l(hi, hi, 1) & 0xFFFE0001u;
+    const uint32_t hi01 = max(k0, k1), lo01 = min(k0, k1);
+    const uint32_t hi23 = max(k2, k3), lo23 = min(k2, k3);
+    const uint32_t f = max(hi01, hi23);
+    const uint32_t sc = max(min(hi01, hi23), max(lo01, lo23));
+    // a = the kept element of lower index (larger 3 - i), b = the other one
+    const bool f_lower = (f & 6u) > (sc & 6u);
+    const uint32_t ka = f_lower ? f : sc, kb = f_lower ? sc : f;
+    const uint32_t ia = 3u - ((ka >> 1) & 3u), ib = 3u - ((kb >> 1) & 3u);
+    mb |= (ia | (ib << 2)) << (4 * g);
+    const uint32_t ca = code((ka >> 17) | ((ka & 1u) << 15));
+    const uint32_t cb = code((kb >> 17) | ((kb & 1u) << 15));
+    out |= (ca | (cb << 8)) << (16 * g);
+    if (DENSE) (g ? dn.y : dn.x) = (ca << (8 * ia)) | (cb << (8 * ib));
+  }
+  return out;
+}
+
+// The same selection with both groups in the two 16-bit lanes of a word,
+// split over the two phases: phase 1 (memory-bound) selects and stores the
+// metadata byte, phase 2 reads it back and only encodes the kept pair.
+// A_i = (|w| of element i of group 1) << 16 | (|w| of element i of group 0);
+// for j < i, (A_j | 0x80008000) - A_i has bit 15 (group 0) and bit 31
+// (group 1) set exactly when |w_j| >= |w_i|, i.e. when j beats i (the lower
+// index wins ties); when it is clear, i beats j.  The six such bits of a
+// group decide the kept pair, so a 64-entry table maps them to the pair's
+// metadata nibble.
+__device__ __forceinline__ void build_select_tables(uint32_t *nib64, uint32_t *sel16, int t) {
+  if (t < 64) {
+    // bit order of the index: g01, g02, g03, g12, g13, g23 (g_ji = j beats i);
+    // element i is kept when fewer than two elements beat it
+    const int g01 = t & 1, g02 = (t >> 1) & 1, g03 = (t >> 2) & 1;
+    const int g12 = (t >> 3) & 1, g13 = (t >> 4) & 1, g23 = (t >> 5) & 1;
+    const int beaten0 = 3 - g01 - g02 - g03;
+    const int beaten1 = g01 + 2 - g12 - g13;
+    const int beaten2 = g02 + g12 + 1 - g23;
+    const int beaten3 = g03 + g13 + g23;
+    const uint32_t keep = (beaten0 < 2 ? 1u : 0u) | (beaten1 < 2 ? 2u : 0u) | (beaten2 < 2 ? 4u : 0u) |
+                          (beaten3 < 2 ? 8u : 0u);
+    uint32_t nib = 0;
+    if (__popc(keep) == 2) {  // patterns that no input produces keep nibble 0
+      const uint32_t lo = __ffs(keep) - 1, hi = 31 - __clz(keep);
+      nib = lo | (hi << 2);
+    }
+    nib64[t] = nib * 17u;  // the nibble in both halves of the byte
+  }
+  // metadata nibble -> the byte-permute selector of its kept pair: element i
+  // of a group is bytes 2i and 2i + 1 of the group's two words (16 words, one
+  // per bank, so lookups never conflict)
+  if (t < 16) {
+    const uint32_t lo = t & 3u, hi = (t >> 2) & 3u;
+    sel16[t] = (2 * lo) | ((2 * lo + 1) << 4) | ((2 * hi) << 8) | ((2 * hi + 1) << 12);
+  }
+}
+
+// Phase 1: the metadata byte of a unit; amax2 accumulates the lane-wise
+// largest magnitude bits (both halves of the word).
+__device__ __forceinline__ uint32_t prune24_select(const uint4 v, const uint32_t *nib64, uint32_t &amax2) {
+  const uint32_t a0 = __byte_perm(v.x, v.z, 0x5410), a1 = __byte_perm(v.x, v.z, 0x7632);
+  const uint32_t a2 = __byte_perm(v.y, v.w, 0x5410), a3 = __byte_perm(v.y, v.w, 0x7632);
+  constexpr uint32_t kMag = 0x7FFF7FFFu, kTop = 0x80008000u;
+  const uint32_t m0 = a0 & kMag, m1 = a1 & kMag, m2 = a2 & kMag, m3 = a3 & kMag;
+  amax2 = __vmaxu2(amax2, __vmaxu2(__vmaxu2(m0, m1), __vmaxu2(m2, m3)));
+  const uint32_t h0 = a0 | kTop, h1 = a1 | kTop, h2 = a2 | kTop;
+  uint32_t bits = (h0 - m1) & kTop;                        // g01
+  bits = (bits >> 1) | ((h0 - m2) & kTop);                 // g02
+  bits = (bits >> 1) | ((h0 - m3) & kTop);                 // g03
+  bits = (bits >> 1) | ((h1 - m2) & kTop);                 // g12
+  bits = (bits >> 1) | ((h1 - m3) & kTop);                 // g13
+  bits = (bits >> 1) | ((h2 - m3) & kTop);                 // g23
+  return (nib64[(bits >> 10) & 63u] & 0x0Fu) | (nib64[bits >> 26] & 0xF0u);
+}
+
+// Phase 2: the four E4M3 codes of a unit whose metadata byte is mb (kept
+// elements in ascending index order, group 0 first).
+template <class Code>
+__device__ __forceinline__ uint32_t prune24_codes(const uint4 v, uint32_t mb, const uint32_t *sel16,
+                                                  const Code &code) {
+  const uint32_t p0 = __byte_perm(v.x, v.y, sel16[mb & 15u]);         // kept pair of group 0
+  const uint32_t p1 = __byte_perm(v.z, v.w, sel16[(mb >> 4) & 15u]);  // and of group 1
+  const uint32_t c0 = code(p0 & 0xFFFFu), c1 = code(p0 >> 16);
+  const uint32_t c2 = code(p1 & 0xFFFFu), c3 = code(p1 >> 16);
+  return c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
+}
+
+// Byte offset, in its packed block, of the 4 value bytes of unit u (row
+// u / 16, columns 8 (u % 16) ..): row r's 16-byte chunk c sits at chunk
+// position c ^ ((r >> 1) & 3).
+__device__ __forceinline__ uint32_t packed_value_offset(uint32_t u) {
+  const uint32_t r = u >> 4, cchunk = (u >> 2) & 3u;
+  return r * 64 + (((cchunk ^ (r >> 1)) & 3u) << 4) + (u & 3u) * 4;
+}
+
+// E4M3 2:4 ops whose selection runs in phase 1 (the DENSE variant selects and
+// encodes in phase 2).
 template <int OP, bool FP8, bool DENSE>
-__device__ __forceinline__ uint32_t phase1_unit(const uint8_t *p, int64_t e0, const StreamArgs &a) {
+__host__ __device__ constexpr bool selects_in_phase1() {
+  return OP == kOpPrune24Packed || (OP == kOpPrune24 && FP8 && !DENSE);
+}
+
+// Where phase 1 leaves a unit's 2:4 metadata byte for phase 2.
+template <int OP>
+__device__ __forceinline__ uint8_t *meta_byte(const StreamArgs &a, const Chunk &ch, uint32_t u) {
+  if constexpr (OP == kOpPrune24Packed)
+    return a.out + ch.idx * kPackedBlockBytes + 128 * 64 + u;
+  else
+    return a.meta + (ch.e >> 3) + u;
+}
+
+// ------------------------------------------------------------------ phase 1
+// One unit: `p` its bytes in shared memory, u its index in chunk `ch`; mx2
+// accumulates the per-lane largest magnitude bits.
+template <int OP, bool FP8, bool DENSE>
+__device__ __forceinline__ void phase1_unit(const uint8_t *p, const Chunk &ch, uint32_t u,
+                                            const StreamArgs &a, const uint32_t *nib64, uint32_t &mx2) {
   if constexpr (OP == kOpSlide68) {
     const uint4 v0 = reinterpret_cast<const uint4 *>(p)[0];
     const uint4 v1 = reinterpret_cast<const uint4 *>(p)[1];
@@ -149,21 +322,23 @@ __device__ __forceinline__ uint32_t phase1_unit(const uint8_t *p, int64_t e0, co
         }
       }
     }
-    const int64_t unit = e0 / 16;
-    uint8_t *m = a.meta + 3 * unit;
+    uint8_t *m = a.meta + 3 * (ch.e >> 4) + 3 * u;
     m[0] = static_cast<uint8_t>(nib[0] | (nib[1] << 4));
     m[1] = static_cast<uint8_t>(nib[2] | (nib[3] << 4));
     m[2] = static_cast<uint8_t>(nib[4] | (nib[5] << 4));
     if (!FP8) {
-      uint2 *d = reinterpret_cast<uint2 *>(a.out + 24 * unit);
+      uint2 *d = reinterpret_cast<uint2 *>(a.out + 24 * (ch.e >> 4) + 24 * u);
 #pragma unroll
       for (int o = 0; o < 3; ++o)
         d[o] = make_uint2(vals[4 * o] | (vals[4 * o + 1] << 16), vals[4 * o + 2] | (vals[4 * o + 3] << 16));
     }
-    return max(absmax8(v0), absmax8(v1));
+    mx2 = __vmaxu2(mx2, __vmaxu2(absmax8x2(v0), absmax8x2(v1)));
   } else {
     const uint4 v = *reinterpret_cast<const uint4 *>(p);
-    if constexpr (OP == kOpPrune24) {
+    if constexpr (selects_in_phase1<OP, FP8, DENSE>()) {
+      *meta_byte<OP>(a, ch, u) = static_cast<uint8_t>(prune24_select(v, nib64, mx2));
+      return;
+    } else if constexpr (OP == kOpPrune24 && !FP8) {
       uint32_t h[8];
       halves(v, h);
       uint32_t mb = 0, kept[4], dn[8];
@@ -174,39 +349,34 @@ __device__ __forceinline__ uint32_t phase1_unit(const uint8_t *p, int64_t e0, co
         const uint32_t mk = keep2of4(aa);
         const int i0 = __ffs(mk) - 1, i1 = __ffs(mk & (mk - 1)) - 1;
         mb |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * g);
-        if (!FP8) {
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            if (t == i0) kept[2 * g] = h[4 * g + t];
-            if (t == i1) kept[2 * g + 1] = h[4 * g + t];
-            if (DENSE) dn[4 * g + t] = ((mk >> t) & 1u) ? h[4 * g + t] : 0u;
-          }
+        for (int t = 0; t < 4; ++t) {
+          if (t == i0) kept[2 * g] = h[4 * g + t];
+          if (t == i1) kept[2 * g + 1] = h[4 * g + t];
+          if (DENSE) dn[4 * g + t] = ((mk >> t) & 1u) ? h[4 * g + t] : 0u;
         }
       }
-      a.meta[e0 / 8] = static_cast<uint8_t>(mb);
-      if (!FP8) {
-        *reinterpret_cast<uint2 *>(a.out + e0) =
-            make_uint2(kept[0] | (kept[1] << 16), kept[2] | (kept[3] << 16));
-        if (DENSE)
-          *reinterpret_cast<uint4 *>(a.dense + 2 * e0) =
-              make_uint4(dn[0] | (dn[1] << 16), dn[2] | (dn[3] << 16), dn[4] | (dn[5] << 16),
-                         dn[6] | (dn[7] << 16));
-      }
+      a.meta[(ch.e >> 3) + u] = static_cast<uint8_t>(mb);
+      *reinterpret_cast<uint2 *>(a.out + ch.e + 8 * u) =
+          make_uint2(kept[0] | (kept[1] << 16), kept[2] | (kept[3] << 16));
+      if (DENSE)
+        *reinterpret_cast<uint4 *>(a.dense + 2 * ch.e + 16 * u) =
+            make_uint4(dn[0] | (dn[1] << 16), dn[2] | (dn[3] << 16), dn[4] | (dn[5] << 16),
+                       dn[6] | (dn[7] << 16));
     }
-    return absmax8(v);
+    mx2 = __vmaxu2(mx2, absmax8x2(v));
   }
 }
 
 // ------------------------------------------------------------------ phase 2
 // `meta_in` is the unit's metadata (one byte for 2:4, three for 6:8), loaded
 // before the chunk's stores so that the loads overlap.
-template <int OP, bool DENSE>
-__device__ __forceinline__ void phase2_unit(const uint8_t *p, int64_t e0, uint32_t meta_in,
-                                            const StreamArgs &a, const CodeTable &code) {
+template <int OP, bool DENSE, class Code>
+__device__ __forceinline__ void phase2_unit(const uint8_t *p, const Chunk &ch, uint32_t u, uint32_t meta_in,
+                                            const StreamArgs &a, const Code &code, const uint32_t *sel16) {
   if constexpr (OP == kOpSlide68) {
     const uint4 v0 = reinterpret_cast<const uint4 *>(p)[0];
     const uint4 v1 = reinterpret_cast<const uint4 *>(p)[1];
-    const int64_t unit = e0 / 16;
     const uint32_t m3 = meta_in;
     uint32_t c[12];
 #pragma unroll
@@ -227,62 +397,58 @@ __device__ __forceinline__ void phase2_unit(const uint8_t *p, int64_t e0, uint32
         c[6 * gl + 2 * j + 1] = code(h1);
       }
     }
-    uint32_t *d = reinterpret_cast<uint32_t *>(a.out + 12 * unit);
+    uint32_t *d = reinterpret_cast<uint32_t *>(a.out + 12 * (ch.e >> 4) + 12 * u);
 #pragma unroll
     for (int o = 0; o < 3; ++o)
       d[o] = c[4 * o] | (c[4 * o + 1] << 8) | (c[4 * o + 2] << 16) | (c[4 * o + 3] << 24);
   } else {
     const uint4 v = *reinterpret_cast<const uint4 *>(p);
-    uint32_t h[8];
-    halves(v, h);
-    if constexpr (OP == kOpQuantize) {
-      *reinterpret_cast<uint2 *>(a.out + e0) =
-          make_uint2(code(h[0]) | (code(h[1]) << 8) | (code(h[2]) << 16) | (code(h[3]) << 24),
-                     code(h[4]) | (code(h[5]) << 8) | (code(h[6]) << 16) | (code(h[7]) << 24));
-    } else if constexpr (OP == kOpLift) {
-      // lifted[12 g + 4 j + r] = code(x[8 g + 2 j + r]) for the 8-group g
-      uint32_t c[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) c[t] = code(h[t]);
-      uint32_t *d = reinterpret_cast<uint32_t *>(a.out + 12 * (e0 / 8));
-      d[0] = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-      d[1] = c[2] | (c[3] << 8) | (c[4] << 16) | (c[5] << 24);
-      d[2] = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+    if constexpr (OP == kOpPrune24Packed) {
+      *reinterpret_cast<uint32_t *>(a.out + ch.idx * kPackedBlockBytes + packed_value_offset(u)) =
+          prune24_codes(v, meta_in, sel16, code);
+    } else if constexpr (OP == kOpPrune24 && !DENSE) {
+      *reinterpret_cast<uint32_t *>(a.out + (ch.e >> 1) + 4 * u) = prune24_codes(v, meta_in, sel16, code);
     } else if constexpr (OP == kOpPrune24) {
-      const uint32_t mb = meta_in;
-      uint32_t c[4], dn[2];
+      uint32_t mb;
+      uint2 dn;
+      *reinterpret_cast<uint32_t *>(a.out + (ch.e >> 1) + 4 * u) = prune24_encode<true>(v, code, mb, dn);
+      *reinterpret_cast<uint2 *>(a.dense + ch.e + 8 * u) = dn;
+      a.meta[(ch.e >> 3) + u] = static_cast<uint8_t>(mb);
+    } else {
+      uint32_t h[8];
+      halves(v, h);
+      if constexpr (OP == kOpQuantize) {
+        *reinterpret_cast<uint2 *>(a.out + ch.e + 8 * u) =
+            make_uint2(code(h[0]) | (code(h[1]) << 8) | (code(h[2]) << 16) | (code(h[3]) << 24),
+                       code(h[4]) | (code(h[5]) << 8) | (code(h[6]) << 16) | (code(h[7]) << 24));
+      } else if constexpr (OP == kOpLift) {
+        // lifted[12 g + 4 j + r] = code(x[8 g + 2 j + r]) for the 8-group g
+        uint32_t c[8];
 #pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        const uint32_t nib = (mb >> (4 * g)) & 0xFu;
-        const uint32_t i0 = nib & 3u, i1 = nib >> 2;
-        uint32_t h0 = h[4 * g], h1 = h[4 * g + 1];
-#pragma unroll
-        for (int t = 1; t < 4; ++t) {
-          if (i0 == static_cast<uint32_t>(t)) h0 = h[4 * g + t];
-          if (i1 == static_cast<uint32_t>(t)) h1 = h[4 * g + t];
-        }
-        c[2 * g] = code(h0);
-        c[2 * g + 1] = code(h1);
-        if (DENSE) dn[g] = (c[2 * g] << (8 * i0)) | (c[2 * g + 1] << (8 * i1));
+        for (int t = 0; t < 8; ++t) c[t] = code(h[t]);
+        uint32_t *d = reinterpret_cast<uint32_t *>(a.out + 12 * (ch.e >> 3) + 12 * u);
+        d[0] = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+        d[1] = c[2] | (c[3] << 8) | (c[4] << 16) | (c[5] << 24);
+        d[2] = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
       }
-      *reinterpret_cast<uint32_t *>(a.out + e0 / 2) = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-      if (DENSE) *reinterpret_cast<uint2 *>(a.dense + e0) = make_uint2(dn[0], dn[1]);
     }
   }
 }
 
 // ------------------------------------------------------------------ kernel
 template <int OP, bool FP8, bool DENSE>
-__global__ void __launch_bounds__(kThreads, 1) stream_kernel(const StreamArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_constant__ StreamArgs a) {
   constexpr int kUnit = unit_bytes<OP>();
   constexpr int kRows = kChunkBytes / (kConsumers * kUnit);  // units per thread per chunk
   extern __shared__ uint8_t smem_raw[];
   uint8_t *ring = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
   uint8_t *tab = ring + kStages * kChunkBytes;
-  uint64_t *full = reinterpret_cast<uint64_t *>(tab + kTab);
+  uint64_t *full = reinterpret_cast<uint64_t *>(tab + kTabBytes);
   uint64_t *empty = full + kStages;
   __shared__ uint32_t s_red[kConsumers / 32];
+  __shared__ uint32_t s_nib64[64];    // 2:4: comparison bits -> metadata nibble
+  __shared__ uint32_t s_sel16[16];    // 2:4: metadata nibble -> byte-permute selector
   __shared__ uint32_t s_amax;
 
   const int tid = threadIdx.x;
@@ -300,6 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const StreamArgs a)
     }
     fence_mbar_init();
   }
+  if constexpr (selects_in_phase1<OP, FP8, DENSE>()) build_select_tables(s_nib64, s_sel16, tid);
   __syncthreads();
   grid_dependency_wait();
   // Activation kernels let the next kernel (a GEMM) launch early; the weight
@@ -309,44 +476,72 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const StreamArgs a)
 
   if (warp == kConsumers / 32) {
     // ------------------------------------------------------------ producer
-    // Load L brings chunk c0 + L % n_my into slot L % kStages.  The second
-    // pass over the chunks (phase 2) is prefetched as soon as slots free up.
+    // Load L < n_my brings chunk c0 + L, load n_my + i chunk c0 + n_my - 1 - i
+    // (phase 2 walks the range backwards), into slot L % kStages.  The second
+    // pass is prefetched as soon as slots free up.
     if ((tid & 31) == 0) {
+      if constexpr (OP == kOpPrune24Packed) prefetch_tensormap(&a.wmap);
       for (int L = 0; L < n_loads; ++L) {
         const int slot = L % kStages;
         if (L >= kStages &&
             !mbar_wait(&empty[slot], static_cast<uint32_t>(L / kStages - 1) & 1u, a.status))
           break;
-        const int64_t c = c0 + L % n_my;
+        const int64_t c = L < n_my ? c0 + L : c0 + 2 * n_my - 1 - L;
         const uint32_t nb =
             static_cast<uint32_t>(min(static_cast<int64_t>(kChunkBytes), a.nbytes - c * kChunkBytes));
         mbar_arrive_expect_tx(&full[slot], nb);
-        bulk_load(ring + slot * kChunkBytes, a.x + c * kChunkBytes, nb, &full[slot]);
+        if constexpr (OP == kOpPrune24Packed) {
+          const uint32_t t = static_cast<uint32_t>(c) / a.kblocks;
+          const uint32_t kb = static_cast<uint32_t>(c) - t * a.kblocks;
+          tma_load_2d(ring + slot * kChunkBytes, &a.wmap, &full[slot], static_cast<int32_t>(kb * 128),
+                      static_cast<int32_t>(t * 128), l2_policy_evict_normal());
+        } else {
+          bulk_load(ring + slot * kChunkBytes, a.x + c * kChunkBytes, nb, &full[slot]);
+        }
       }
     }
     return;
   }
 
   // -------------------------------------------------------------- consumers
+  // fn(unit bytes in shared memory, unit index) for this thread's units of
+  // chunk c; full chunks (all but possibly the tensor's last) need no checks.
   auto for_units = [&](const uint8_t *chunk, int64_t c, auto &&fn) {
     const int64_t nb = min(static_cast<int64_t>(kChunkBytes), a.nbytes - c * kChunkBytes);
+    if (nb == kChunkBytes) {
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) {
-      const int off = (r * kConsumers + tid) * kUnit;
-      if (off < nb) fn(chunk + off, (c * kChunkBytes + off) / 2);
+      for (int r = 0; r < kRows; ++r) {
+        const uint32_t u = static_cast<uint32_t>(r * kConsumers + tid);
+        fn(chunk + u * kUnit, u);
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) {
+        const uint32_t u = static_cast<uint32_t>(r * kConsumers + tid);
+        if (static_cast<int64_t>(u) * kUnit < nb) fn(chunk + u * kUnit, u);
+      }
     }
   };
+  auto chunk_of = [](int64_t c) {
+    return Chunk{static_cast<uint64_t>(c) * (kChunkBytes / 2), static_cast<uint64_t>(c)};
+  };
 
-  uint32_t mx = 0;
+  // The table costs about as much as dividing 2 chunks' elements directly.
+  const bool direct = n_my <= 2;
+  if (FP8 && !direct) zero_table(tab, tid);  // ordered before its entries by the barriers below
+
+  uint32_t mx2 = 0;  // per-lane largest magnitude bits
   for (int i = 0; i < n_my; ++i) {
     const int slot = i % kStages;
     mbar_wait(&full[slot], static_cast<uint32_t>(i / kStages) & 1u, a.status);
-    for_units(ring + slot * kChunkBytes, c0 + i, [&](const uint8_t *p, int64_t e0) {
-      mx = max(mx, phase1_unit<OP, FP8, DENSE>(p, e0, a));
+    const Chunk ch = chunk_of(c0 + i);
+    for_units(ring + slot * kChunkBytes, c0 + i, [&](const uint8_t *p, uint32_t u) {
+      phase1_unit<OP, FP8, DENSE>(p, ch, u, a, s_nib64, mx2);
     });
     __syncwarp();
     if (!resident && (tid & 31) == 0) mbar_arrive(&empty[slot]);
   }
+  uint32_t mx = max(mx2 & 0xFFFFu, mx2 >> 16);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
   if ((tid & 31) == 0) s_red[warp] = mx;
@@ -362,14 +557,17 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const StreamArgs a)
     if (tid == 0 && mx >= 0x7F80u && a.status) atomicOr(a.status, SP24_STATUS_NONFINITE);
   } else {
     // ------------------------------------------------ grid barrier on amax
+    // The amax and the arrival are posted without waiting (the release on the
+    // arrival orders the max before it); the departure count that lets the
+    // last CTA re-zero the counters is taken at the end of the kernel, off
+    // the critical path.
     if (tid == 0) {
-      atomicMax(&a.ws[0], mx);
-      __threadfence();
-      atomicAdd(&a.ws[1], 1u);
+      red_max_relaxed_gpu(&a.ws[0], mx);
+      red_add_release_gpu(&a.ws[1], 1u);
       const uint64_t t0 = global_timer_ns();
       uint32_t polls = 0;
       while (ld_acquire_u32(&a.ws[1]) < gridDim.x) {
-        __nanosleep(64);
+        __nanosleep(32);
         if ((++polls & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
           if (a.status) atomicOr(a.status, SP24_STATUS_TIMEOUT);
           break;
@@ -377,13 +575,6 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const StreamArgs a)
       }
       const uint32_t amax = ld_acquire_u32(&a.ws[0]);
       s_amax = amax;
-      __threadfence();
-      if (atomicAdd(&a.ws[2], 1u) == gridDim.x - 1) {  // last to leave: reset the counters
-        a.ws[0] = 0u;
-        a.ws[1] = 0u;
-        a.ws[2] = 0u;
-        __threadfence();
-      }
       if (blockIdx.x == 0) {
         if (amax >= 0x7F80u && a.status) atomicOr(a.status, SP24_STATUS_NONFINITE);
         if (a.scale_out) *a.scale_out = amax == 0u ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax), 448.0f);
@@ -392,46 +583,82 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const StreamArgs a)
     named_bar_sync(1, kConsumers);
     const uint32_t amax = s_amax;
     const float s = amax == 0u ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax), 448.0f);
-    const bool direct = static_cast<int64_t>(n_my) * kChunkBytes < 2 * kTab * 2 * 8;
-    if (!direct) build_table(tab, amax, s, tid);
+    if (!direct) fill_table(tab, amax, s, tid);
     named_bar_sync(1, kConsumers);
-    const CodeTable code{tab, (static_cast<int>(amax >> 7) - 23) * 128, s, direct};
 
     // ---------------------------------------------------------- phase 2
-    for (int i = 0; i < n_my; ++i) {
-      int slot = i;
-      const int L = n_my + i;
-      if (!resident) {
-        slot = L % kStages;
-        mbar_wait(&full[slot], static_cast<uint32_t>(L / kStages) & 1u, a.status);
-      }
-      const int64_t c = c0 + i;
+    // The units' metadata (1 byte for 2:4, 3 for 6:8; this thread wrote it in
+    // phase 1) of chunk c, loaded one chunk ahead so the L2 latency overlaps
+    // the previous chunk's work.
+    constexpr bool kMetaIn = OP == kOpSlide68 || selects_in_phase1<OP, FP8, DENSE>();
+    auto load_meta = [&](int64_t c, uint32_t (&m)[kRows]) {
+      const Chunk ch = chunk_of(c);
       const int64_t nb = min(static_cast<int64_t>(kChunkBytes), a.nbytes - c * kChunkBytes);
-      uint32_t mrow[kRows];
 #pragma unroll
       for (int r = 0; r < kRows; ++r) {
-        const int off = (r * kConsumers + tid) * kUnit;
-        const int64_t e0 = (c * kChunkBytes + off) / 2;
-        mrow[r] = 0;
-        if (off < nb) {
-          if constexpr (OP == kOpPrune24) {
-            mrow[r] = __ldcg(a.meta + e0 / 8);
-          } else if constexpr (OP == kOpSlide68) {
-            const uint8_t *mp = a.meta + 3 * (e0 / 16);
-            mrow[r] = __ldcg(mp) | (static_cast<uint32_t>(__ldcg(mp + 1)) << 8) |
-                      (static_cast<uint32_t>(__ldcg(mp + 2)) << 16);
+        const uint32_t u = static_cast<uint32_t>(r * kConsumers + tid);
+        m[r] = 0;
+        if (static_cast<int64_t>(u) * kUnit < nb) {
+          if constexpr (OP == kOpSlide68) {
+            const uint8_t *mp = a.meta + 3 * (ch.e >> 4) + 3 * u;
+            m[r] = __ldcg(mp) | (static_cast<uint32_t>(__ldcg(mp + 1)) << 8) |
+                   (static_cast<uint32_t>(__ldcg(mp + 2)) << 16);
+          } else {
+            m[r] = __ldcg(meta_byte<OP>(a, ch, u));
           }
         }
       }
+    };
+
+    // ---------------------------------------------------------- phase 2
+    auto phase2 = [&](const auto &code) {
+      [[maybe_unused]] uint32_t mnext[kRows];
+      if constexpr (kMetaIn) load_meta(c0 + n_my - 1, mnext);
+      for (int i = 0; i < n_my; ++i) {
+        const int j = n_my - 1 - i;  // chunk of the range, last first
+        int slot = j;                // resident: where phase 1 left it
+        const int L = n_my + i;
+        [[maybe_unused]] uint32_t mrow[kRows];
+        if constexpr (kMetaIn) {
 #pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        const int off = (r * kConsumers + tid) * kUnit;
-        if (off < nb)
-          phase2_unit<OP, DENSE>(ring + slot * kChunkBytes + off, (c * kChunkBytes + off) / 2, mrow[r], a,
-                                 code);
+          for (int r = 0; r < kRows; ++r) mrow[r] = mnext[r];
+          if (j > 0) load_meta(c0 + j - 1, mnext);
+        }
+        if (!resident) {
+          slot = L % kStages;
+          mbar_wait(&full[slot], static_cast<uint32_t>(L / kStages) & 1u, a.status);
+        }
+        const int64_t c = c0 + j;
+        const Chunk ch = chunk_of(c);
+        const uint8_t *chunk = ring + slot * kChunkBytes;
+        if constexpr (kMetaIn) {
+          const int64_t nb = min(static_cast<int64_t>(kChunkBytes), a.nbytes - c * kChunkBytes);
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            const uint32_t u = static_cast<uint32_t>(r * kConsumers + tid);
+            if (static_cast<int64_t>(u) * kUnit < nb)
+              phase2_unit<OP, DENSE>(chunk + u * kUnit, ch, u, mrow[r], a, code, s_sel16);
+          }
+        } else {
+          for_units(chunk, c, [&](const uint8_t *p, uint32_t u) {
+            phase2_unit<OP, DENSE>(p, ch, u, 0u, a, code, s_sel16);
+          });
+        }
+        __syncwarp();
+        if (!resident && (tid & 31) == 0) mbar_arrive(&empty[slot]);
       }
-      __syncwarp();
-      if (!resident && (tid & 31) == 0) mbar_arrive(&empty[slot]);
+    };
+    if (direct)
+      phase2(CodeTable<true>{tab, s});
+    else
+      phase2(CodeTable<false>{tab, s});
+    if (tid == 0) {
+      __threadfence();
+      if (atomicAdd(&a.ws[2], 1u) == gridDim.x - 1) {  // last to leave: re-zero the counters
+        a.ws[0] = 0u;
+        a.ws[1] = 0u;
+        a.ws[2] = 0u;
+      }
     }
   }
 }
@@ -462,6 +689,7 @@ cudaError_t launch_stream_typed(const StreamArgs &a, int sm_count, cudaStream_t 
 StreamArgs make_args(const void *x, int64_t nelem, uint32_t *ws, float *scale, int32_t *status,
                      void *out, uint8_t *meta, void *dense) {
   StreamArgs a;
+  memset(&a, 0, sizeof(a));
   a.x = static_cast<const uint8_t *>(x);
   a.nbytes = nelem * 2;
   a.nchunks = (a.nbytes + kChunkBytes - 1) / kChunkBytes;
@@ -471,6 +699,7 @@ StreamArgs make_args(const void *x, int64_t nelem, uint32_t *ws, float *scale, i
   a.out = static_cast<uint8_t *>(out);
   a.meta = meta;
   a.dense = static_cast<uint8_t *>(dense);
+  a.kblocks = 0;
   return a;
 }
 
@@ -497,6 +726,19 @@ cudaError_t launch_prune24_fused(const void *w, int64_t nelem, bool fp8, uint32_
                  : launch_stream_typed<kOpPrune24, true, false>(a, sm_count, st);
   return dense ? launch_stream_typed<kOpPrune24, false, true>(a, sm_count, st)
                : launch_stream_typed<kOpPrune24, false, false>(a, sm_count, st);
+}
+
+cudaError_t launch_prune24_packed_fused(const void *w, int N, int K, uint32_t *ws, float *scale,
+                                        uint8_t *packed, int32_t *status, int sm_count,
+                                        cudaStream_t st) {
+  StreamArgs a = make_args(w, static_cast<int64_t>(N) * K, ws, scale, status, packed, nullptr, nullptr);
+  a.kblocks = static_cast<uint32_t>(K / 128);
+  // chunk = one 128-row x 128-column box of W = the input of one packed block
+  static_assert(kChunkBytes == 128 * 128 * 2, "a chunk must be one packed block's input");
+  if (!make_tensor_map_2d(&a.wmap, w, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, static_cast<uint64_t>(K),
+                          static_cast<uint64_t>(N), 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  return launch_stream_typed<kOpPrune24Packed, true, false>(a, sm_count, st);
 }
 
 cudaError_t launch_slide68_fused(const void *w, int64_t nelem, bool fp8, uint32_t *ws,

@@ -33,13 +33,25 @@ def test_status_strings_and_version(lib):
 def test_workspace_sizes(lib):
     for op in range(4):
         assert lib.sp24_workspace_size(op, 16, 256, 256, 0) == 256
-    # prefill-sized GEMMs run whole tiles on persistent CTAs: no scratch
-    assert lib.sp24_workspace_size(_lib.OP_GEMM, 4096, 12288, 4096, 0) == 0
-    assert lib.sp24_workspace_size(_lib.OP_GEMM_DENSE, 4096, 12288, 4096, 0) == 0
-    # decode-sized GEMMs use stream-K: a 16 KB counter prefix + fp32 partial tiles
+    # Shapes whose tiles fill whole waves of the 148 SMs need no scratch:
+    # M=256 -> 128-token tiles, 2 x (18944 / 128) = 296 tiles = 2 waves.
+    assert lib.sp24_workspace_size(_lib.OP_GEMM, 256, 18944, 4096, 0) == 0
+    assert lib.sp24_workspace_size(_lib.OP_GEMM_DENSE, 256, 18944, 4096, 0) == 0
+    # Otherwise the leftover tiles are split by k-blocks over up to every CTA
+    # (at most two ways for tiles wider than 64 tokens): a 16 KB counter
+    # prefix + one fp32 128 x BN partial tile per splitting CTA.  Prefill
+    # M=4096 uses 224-token tiles: 19 x 96 = 1824 tiles = 12 waves + 48
+    # leftover, split over 96 CTAs.
+    assert lib.sp24_workspace_size(_lib.OP_GEMM, 4096, 12288, 4096, 0) == 16384 + 96 * 128 * 224 * 4
+    # down-proj M=256: 64 tiles of 112 k-blocks, each split over 2 CTAs
+    assert lib.sp24_workspace_size(_lib.OP_GEMM, 256, 4096, 14336, 0) == 16384 + 128 * 128 * 128 * 4
+    # decode: 16-token tiles
+    assert lib.sp24_workspace_size(_lib.OP_GEMM, 1, 11008, 4096, 0) == 16384 + 148 * 128 * 16 * 4
     for m in (1, 64):
         ws = lib.sp24_workspace_size(_lib.OP_GEMM, m, 11008, 4096, 0)
         assert ws > 16384 and ws % 16 == 0
+    # tiny: 2 tiles x 2 k-blocks -> 2 CTAs with one whole tile each
+    assert lib.sp24_workspace_size(_lib.OP_GEMM, 16, 256, 256, 0) == 0
     assert lib.sp24_workspace_size(_lib.OP_GEMM, 0, 11008, 4096, 0) == 0
 
 
@@ -64,8 +76,12 @@ def test_validation_rejects_bad_arguments_without_a_gpu(lib):
     assert lib.sp24_gemm(FAKE, None, FAKE, FAKE, None, FAKE, 4, 200, 256, 0, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
     assert lib.sp24_gemm(FAKE, None, FAKE, FAKE, None, FAKE, 0, 128, 256, 0, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
     assert lib.fp8_gemm_dense(FAKE, None, FAKE, None, FAKE, 4, 128, 64, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.sp24_prune_compress_packed(FAKE, 128, 192, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.sp24_prune_compress_packed(FAKE, 64, 128, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.sp24_prune_compress_packed(FAKE, 128, 128, FAKE, None, FAKE, ws, None, None) == _lib.SP24_ERR_NULL
     # alignment
     odd = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.sp24_prune_compress_packed(FAKE, 128, 128, odd, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.fp8_quantize_pertensor(odd, 4, 32, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.sp24_gemm(FAKE, None, odd, FAKE, None, FAKE, 4, 128, 128, 0, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
 

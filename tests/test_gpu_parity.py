@@ -217,6 +217,25 @@ def test_sparse_gemm_small_shapes(m, n, k):
     assert_gemm_close(yd, y_ref, b, f"dense {m}x{n}x{k}")
 
 
+@pytest.mark.parametrize("m,n,k", [(40, 19200, 1024), (200, 19072, 512), (1100, 9600, 640)])
+def test_gemm_whole_waves_plus_stream_k_tail(m, n, k):
+    """More tiles than SMs and not a whole number of waves: the full waves run
+    as whole tiles and the leftover tiles are split over CTAs by k-blocks
+    (4-way, 2-way and 2-3-way splits here; the last shape also has a ragged
+    token tile).  The split result must also be deterministic."""
+    x = WL.random_bits((m, k), 500 + m, scale=1.0)
+    w = WL.random_bits((n, k), 600 + n, scale=0.02)
+    y, yd, xq, sx, vals, meta, sw = _run_sparse(x, w, dense_too=True)
+    y_ref, b = _ref(xq, sx, vals, meta, sw, k)
+    assert_gemm_close(y, y_ref, b, f"hybrid sparse {m}x{n}x{k}")
+    assert_gemm_close(yd, y_ref, b, f"hybrid dense {m}x{n}x{k}")
+    xq_d = torch.from_numpy(xq).to(DEV)
+    sx_d = torch.tensor([sx], dtype=torch.float32, device=DEV)
+    again = sp().sp24_gemm(xq_d, sx_d, torch.from_numpy(vals).to(DEV), torch.from_numpy(meta).to(DEV),
+                           torch.tensor([sw], dtype=torch.float32, device=DEV))
+    assert torch.equal(again, y)
+
+
 def test_sparse_gemm_tie_heavy_and_zero_activation():
     x = WL.random_bits((8, 256), 7, dist="ties")
     w = WL.random_bits((128, 256), 8, scale=0.5, dist="ties")
@@ -336,6 +355,13 @@ def test_sparse_gemm_bf16_small_shapes(m, n, k):
     assert_gemm_close(y, y_ref, b, f"bf16 sparse {m}x{n}x{k}")
 
 
+def test_sparse_gemm_bf16_stream_k_tail():
+    x = WL.random_bits((200, 512), 310)
+    w = WL.random_bits((19072, 512), 410, scale=0.02)
+    y, y_ref, b = _run_sparse_bf16(x, w)
+    assert_gemm_close(y, y_ref, b, "bf16 sparse 200x19072x512")
+
+
 def test_down_proj_workload_gemm_bf16():
     w, x = WL.weight_bits(4), WL.activation_bits(4, 256)
     y, y_ref, b = _run_sparse_bf16(x, w)
@@ -391,6 +417,36 @@ def test_pack_weights_is_the_documented_permutation(n, k):
     packed = sp().sp24_pack_weights(c["values"], c["meta"])
     want = _pack_reference(host(c["values"]), host(c["meta"]), n, k)
     assert np.array_equal(host(packed), want)
+
+
+@pytest.mark.parametrize("n,k,dist", [(128, 128, "normal"), (256, 512, "ties"), (384, 14336, "student_t3"),
+                                      (1024, 1152, "normal"), (2048, 4096, "ties")])
+def test_prune_compress_packed_matches_oracle(n, k, dist):
+    """Direct packed output == the documented packing of the oracle's values
+    and metadata, byte for byte (K/128 = 1, 4, 112, 9, 32 exercise the
+    division by the K-block count; the first case runs the whole tensor in
+    one CTA with direct division instead of the code table)."""
+    w = WL.random_bits((n, k), 1000 + n, scale=0.02, dist=dist)
+    st = new_status()
+    packed, scale = sp().sp24_prune_compress_packed(dev_bf16(w), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = O.sp24_prune_compress(w, "e4m3")
+    assert host(scale)[0] == np.float32(ref["scale"])
+    want = _pack_reference(ref["values"], ref["meta"], n, k)
+    got = host(packed)
+    if not np.array_equal(got, want):
+        bad = np.flatnonzero(got != want)
+        raise AssertionError(f"{bad.size} bytes differ, first at {bad[:8].tolist()}")
+
+
+@pytest.mark.parametrize("cfg", [2, 4, 5])
+def test_prune_compress_packed_workload_equals_pack_of_canonical(cfg):
+    w = dev_bf16(WL.weight_bits(cfg))
+    c = sp().sp24_prune_compress(w, "e4m3")
+    packed, scale = sp().sp24_prune_compress_packed(w)
+    assert torch.equal(packed, sp().sp24_pack_weights(c["values"], c["meta"]))
+    assert torch.equal(scale, c["scale"])
 
 
 @pytest.mark.parametrize("m,n,k", [(1, 128, 128), (5, 256, 512), (64, 384, 1024), (300, 256, 1152)])

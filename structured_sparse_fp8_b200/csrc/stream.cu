@@ -48,8 +48,17 @@ constexpr int kChunkBytes = 32768;
 constexpr int kStages = 5;
 constexpr int kTab = 24 * 128;               // binades x mantissas that can give a nonzero code
 constexpr int kTabBytes = 65536;             // code of every bf16 bit pattern
-constexpr uint32_t kSmemBytes = kStages * kChunkBytes + kTabBytes + 2 * kStages * 8 + 128;
-static_assert(kSmemBytes + 2048 <= 227 * 1024, "ring + table exceed the shared memory of a CTA");
+// SMALL instantiations serve tensors of at most 2 chunks per CTA: they keep
+// the whole slice resident in a 2-slot ring and divide directly, so they need
+// no table and little shared memory (which leaves room on the SM for the
+// next kernel's CTAs to start early).
+template <bool SMALL> __host__ __device__ constexpr int ring_stages() { return SMALL ? 2 : kStages; }
+template <bool SMALL> __host__ __device__ constexpr int table_bytes() { return SMALL ? 0 : kTabBytes; }
+template <bool SMALL>
+constexpr uint32_t smem_bytes() {
+  return ring_stages<SMALL>() * kChunkBytes + table_bytes<SMALL>() + 2 * ring_stages<SMALL>() * 8 + 128;
+}
+static_assert(smem_bytes<false>() + 2048 <= 227 * 1024, "ring + table exceed the shared memory of a CTA");
 
 enum StreamOp : int { kOpQuantize = 0, kOpLift = 1, kOpPrune24 = 2, kOpSlide68 = 3, kOpPrune24Packed = 4 };
 
@@ -436,16 +445,17 @@ __device__ __forceinline__ void phase2_unit(const uint8_t *p, const Chunk &ch, u
 }
 
 // ------------------------------------------------------------------ kernel
-template <int OP, bool FP8, bool DENSE>
+template <int OP, bool FP8, bool DENSE, bool SMALL>
 __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_constant__ StreamArgs a) {
+  constexpr int kS = ring_stages<SMALL>();
   constexpr int kUnit = unit_bytes<OP>();
   constexpr int kRows = kChunkBytes / (kConsumers * kUnit);  // units per thread per chunk
   extern __shared__ uint8_t smem_raw[];
   uint8_t *ring = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
-  uint8_t *tab = ring + kStages * kChunkBytes;
-  uint64_t *full = reinterpret_cast<uint64_t *>(tab + kTabBytes);
-  uint64_t *empty = full + kStages;
+  uint8_t *tab = ring + kS * kChunkBytes;
+  uint64_t *full = reinterpret_cast<uint64_t *>(tab + table_bytes<SMALL>());
+  uint64_t *empty = full + kS;
   __shared__ uint32_t s_red[kConsumers / 32];
   __shared__ uint32_t s_nib64[64];    // 2:4: comparison bits -> metadata nibble
   __shared__ uint32_t s_sel16[16];    // 2:4: metadata nibble -> byte-permute selector
@@ -456,11 +466,11 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * a.nchunks / gridDim.x;
   const int64_t c1 = static_cast<int64_t>(blockIdx.x + 1) * a.nchunks / gridDim.x;
   const int n_my = static_cast<int>(c1 - c0);
-  const bool resident = n_my <= kStages;             // phase 2 reuses the ring contents
+  const bool resident = n_my <= kS;                  // phase 2 reuses the ring contents
   const int n_loads = (FP8 && !resident) ? 2 * n_my : n_my;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumers / 32);
     }
@@ -477,14 +487,13 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
   if (warp == kConsumers / 32) {
     // ------------------------------------------------------------ producer
     // Load L < n_my brings chunk c0 + L, load n_my + i chunk c0 + n_my - 1 - i
-    // (phase 2 walks the range backwards), into slot L % kStages.  The second
+    // (phase 2 walks the range backwards), into slot L % kS.  The second
     // pass is prefetched as soon as slots free up.
     if ((tid & 31) == 0) {
       if constexpr (OP == kOpPrune24Packed) prefetch_tensormap(&a.wmap);
       for (int L = 0; L < n_loads; ++L) {
-        const int slot = L % kStages;
-        if (L >= kStages &&
-            !mbar_wait(&empty[slot], static_cast<uint32_t>(L / kStages - 1) & 1u, a.status))
+        const int slot = L % kS;
+        if (L >= kS && !mbar_wait(&empty[slot], static_cast<uint32_t>(L / kS - 1) & 1u, a.status))
           break;
         const int64_t c = L < n_my ? c0 + L : c0 + 2 * n_my - 1 - L;
         const uint32_t nb =
@@ -527,13 +536,15 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
   };
 
   // The table costs about as much as dividing 2 chunks' elements directly.
-  const bool direct = n_my <= 2;
-  if (FP8 && !direct) zero_table(tab, tid);  // ordered before its entries by the barriers below
+  const bool direct = SMALL || n_my <= 2;
+  if constexpr (FP8 && !SMALL) {
+    if (!direct) zero_table(tab, tid);  // ordered before its entries by the barriers below
+  }
 
   uint32_t mx2 = 0;  // per-lane largest magnitude bits
   for (int i = 0; i < n_my; ++i) {
-    const int slot = i % kStages;
-    mbar_wait(&full[slot], static_cast<uint32_t>(i / kStages) & 1u, a.status);
+    const int slot = i % kS;
+    mbar_wait(&full[slot], static_cast<uint32_t>(i / kS) & 1u, a.status);
     const Chunk ch = chunk_of(c0 + i);
     for_units(ring + slot * kChunkBytes, c0 + i, [&](const uint8_t *p, uint32_t u) {
       phase1_unit<OP, FP8, DENSE>(p, ch, u, a, s_nib64, mx2);
@@ -583,7 +594,9 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     named_bar_sync(1, kConsumers);
     const uint32_t amax = s_amax;
     const float s = amax == 0u ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax), 448.0f);
-    if (!direct) fill_table(tab, amax, s, tid);
+    if constexpr (!SMALL) {
+      if (!direct) fill_table(tab, amax, s, tid);
+    }
     named_bar_sync(1, kConsumers);
 
     // ---------------------------------------------------------- phase 2
@@ -625,8 +638,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
           if (j > 0) load_meta(c0 + j - 1, mnext);
         }
         if (!resident) {
-          slot = L % kStages;
-          mbar_wait(&full[slot], static_cast<uint32_t>(L / kStages) & 1u, a.status);
+          slot = L % kS;
+          mbar_wait(&full[slot], static_cast<uint32_t>(L / kS) & 1u, a.status);
         }
         const int64_t c = c0 + j;
         const Chunk ch = chunk_of(c);
@@ -648,10 +661,14 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
         if (!resident && (tid & 31) == 0) mbar_arrive(&empty[slot]);
       }
     };
-    if (direct)
+    if constexpr (SMALL) {
       phase2(CodeTable<true>{tab, s});
-    else
-      phase2(CodeTable<false>{tab, s});
+    } else {
+      if (direct)
+        phase2(CodeTable<true>{tab, s});
+      else
+        phase2(CodeTable<false>{tab, s});
+    }
     if (tid == 0) {
       __threadfence();
       if (atomicAdd(&a.ws[2], 1u) == gridDim.x - 1) {  // last to leave: re-zero the counters
@@ -663,27 +680,35 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
   }
 }
 
-template <int OP, bool FP8, bool DENSE>
-cudaError_t launch_stream_typed(const StreamArgs &a, int sm_count, cudaStream_t st) {
+template <int OP, bool FP8, bool DENSE, bool SMALL>
+cudaError_t launch_stream_variant(const StreamArgs &a, int64_t grid, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(stream_kernel<OP, FP8, DENSE>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    attr_err = cudaFuncSetAttribute(stream_kernel<OP, FP8, DENSE, SMALL>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<SMALL>());
   });
   if (attr_err != cudaSuccess) return attr_err;
   cudaLaunchConfig_t cfg = {};
-  const int64_t grid = a.nchunks < sm_count ? a.nchunks : sm_count;
-  cfg.gridDim = dim3(static_cast<unsigned>(grid < 1 ? 1 : grid), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = smem_bytes<SMALL>();
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = FP8 ? 1 : 0;  // only the two-phase kernels wait on each other
-  return cudaLaunchKernelEx(&cfg, stream_kernel<OP, FP8, DENSE>, a);
+  return cudaLaunchKernelEx(&cfg, stream_kernel<OP, FP8, DENSE, SMALL>, a);
+}
+
+template <int OP, bool FP8, bool DENSE>
+cudaError_t launch_stream_typed(const StreamArgs &a, int sm_count, cudaStream_t st) {
+  int64_t grid = a.nchunks < sm_count ? a.nchunks : sm_count;
+  if (grid < 1) grid = 1;
+  const int64_t per_cta = (a.nchunks + grid - 1) / grid;
+  return per_cta <= 2 ? launch_stream_variant<OP, FP8, DENSE, true>(a, grid, st)
+                      : launch_stream_variant<OP, FP8, DENSE, false>(a, grid, st);
 }
 
 StreamArgs make_args(const void *x, int64_t nelem, uint32_t *ws, float *scale, int32_t *status,

@@ -99,24 +99,31 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
-def kernel_source_hash():
+def source_hash(files):
+    """Hash of the named kernel sources (under structured_sparse_fp8_b200/csrc)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "structured_sparse_fp8_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in files:
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def load_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources (else None)."""
+    """DRAM bytes per launch ("workload:op" -> bytes) from the committed ncu
+    summaries, for the entries whose kernel sources are unchanged since the
+    capture (an entry whose sources changed is dropped: its traffic is null)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return {}
     d = json.load(open(path))
-    if d.get("kernel_source_hash") != kernel_source_hash():
-        return {}
-    return d.get("per_launch_bytes", {})
+    out = {}
+    for key, e in d.get("entries", {}).items():
+        try:
+            if source_hash(e["sources"]) == e["source_hash"]:
+                out[key] = e["bytes_per_launch"]
+        except (OSError, KeyError):
+            pass
+    return out
 
 
 # ---------------------------------------------------------------- ranks

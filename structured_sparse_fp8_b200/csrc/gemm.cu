@@ -117,39 +117,67 @@ struct KindTraits<kSparseBF16> {
   static constexpr bool kPacked = false;
 };
 
-template <int KIND, int BN>
+// MT = 128-row W tiles per CTA tile (1 or 2).  With MT = 2 each stage
+// carries two weight tiles and one activation tile, and every k-block issues
+// the MMAs of both row tiles against the same activation tile: the same
+// activation bytes feed twice the tensor work, which is what bounds large
+// token tiles (operand ingest into shared memory, not the tensor pipe).
+template <int KIND, int BN, int MT = 1>
 struct Config {
   using T = KindTraits<KIND>;
-  static constexpr uint32_t kABytes = 128 * T::kARowBytes;
+  static constexpr int kRows = 128 * MT;
+  static constexpr uint32_t kWTile = T::kPacked ? kPackedBlockBytes : 0;  // packed: one block per row tile
+  static constexpr uint32_t kABytes = kRows * T::kARowBytes;
   static constexpr uint32_t kBBytes = BN * T::kBRowBytes;
-  static constexpr uint32_t kEBytes = 128 * T::kERowBytes;
+  static constexpr uint32_t kEBytes = kRows * T::kERowBytes;
   static constexpr uint32_t kTBytes = T::kMetaTransform ? 128 * 16 : 0;  // TMEM-ready metadata
   static constexpr uint32_t kTmaBytes = kABytes + kBBytes + kEBytes;
   static constexpr uint32_t kStageBytes = kTmaBytes + kTBytes;
   static constexpr int kBSub = T::kBRowBytes / 128;  // 128-byte X boxes per stage
-  // Stage layout: [A][B][E][T] (tensor-mapped weights) or [A][E][B] (packed:
-  // A and E arrive together in one bulk copy).
-  static constexpr uint32_t kBOff = T::kPacked ? kABytes + kEBytes : kABytes;
-  static constexpr uint32_t kEOff = T::kPacked ? kABytes : kABytes + kBBytes;
+  // Stage layout: [A][B][E][T] (tensor-mapped weights; A and E hold all kRows
+  // rows, row tile i at 128 i rows) or [A0 E0][A1 E1][B] (packed: each row
+  // tile's values and metadata arrive together in one bulk copy).
+  static constexpr uint32_t kBOff = T::kPacked ? MT * kPackedBlockBytes : kABytes;
+  static constexpr uint32_t kEOff = T::kPacked ? 128 * T::kARowBytes : kABytes + kBBytes;
+  __host__ __device__ static constexpr uint32_t a_off(int i) {
+    return T::kPacked ? i * kPackedBlockBytes : i * 128 * T::kARowBytes;
+  }
+  __host__ __device__ static constexpr uint32_t e_off(int i) {
+    return T::kPacked ? i * kPackedBlockBytes + 128 * T::kARowBytes : kEOff + i * 128 * T::kERowBytes;
+  }
   // Persistent CTAs.  Small token tiles (decode shapes, stream-K) keep the
   // footprint to half an SM, so that the next kernel's CTAs can already be
   // resident, and streaming weights, while this kernel drains; large tiles
   // take the whole SM for a deep ring.
   static constexpr uint32_t kSmemBudget = BN <= 64 ? 108 * 1024 : 214 * 1024;
-  static constexpr int kStagesRaw = static_cast<int>(kSmemBudget / kStageBytes);
+  // Wide token tiles write Y through shared memory: each epilogue warp
+  // stages its 32 rows x 32 tokens of a pass (2 KB of bf16) in one of two
+  // buffers of its own and stores them with a 2-D bulk tensor copy, so the
+  // warps never wait for each other (scattered 2-byte stores into Y rows cost
+  // ~10 us per 128 x 224 tile).
+  static constexpr bool kTmaStoreY = BN >= 224;
+  static constexpr uint32_t kStageY = 32 * 32 * 2;          // one warp's pass
+  static constexpr uint32_t kYBytes = kTmaStoreY ? 4 * 2 * kStageY : 0;
+  static constexpr int kStagesRaw = static_cast<int>((kSmemBudget - kYBytes) / kStageBytes);
   static constexpr int kStages = kStagesRaw > 16 ? 16 : kStagesRaw;
-  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*bars*/;
-  // Two accumulators (the epilogue of one output tile overlaps the main loop
-  // of the next) whenever they fit in the 512 TMEM columns next to the 4
-  // metadata columns.
-  static constexpr uint32_t kMetaCols = T::kSparse ? 4 : 0;
-  static constexpr int kAccBufs = (2 * BN + kMetaCols <= 512) ? 2 : 1;
-  static constexpr uint32_t kTmemNeed = kAccBufs * BN + kMetaCols;
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kYBytes + 1024 /*align*/ + 1024 /*bars*/;
+  // Accumulators: MT x BN columns each; two of them (the epilogue of one
+  // output tile overlaps the main loop of the next) whenever they fit in the
+  // 512 TMEM columns next to the 4 metadata columns per row tile.
+  static constexpr uint32_t kMetaCols = T::kSparse ? 4 * MT : 0;
+  static constexpr int kAccBufs = (2 * MT * BN + kMetaCols <= 512) ? 2 : 1;
+  static constexpr uint32_t kAccCols = MT * BN;
+  static constexpr uint32_t kTmemNeed = kAccBufs * kAccCols + kMetaCols;
   static constexpr uint32_t kTmemCols =
       kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
   static_assert(kStages >= 2, "shared-memory ring too shallow");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be a multiple of 16 in [16,256]");
+  static_assert(MT == 1 || MT == 2, "one or two 128-row W tiles per CTA tile");
+  static_assert(MT == 1 || !T::kMetaTransform, "the BF16 metadata re-layout handles one row tile");
+  static_assert(kTmemNeed <= 512, "accumulators and metadata exceed tensor memory");
+  static_assert(kBOff % 1024 == 0 && kStageBytes % 1024 == 0, "128-byte-swizzled tiles need 1 KB alignment");
   static constexpr int kEpiCols = BN % 32 == 0 ? 32 : 16;  // token columns per epilogue pass
+  static_assert(!kTmaStoreY || kEpiCols == 32, "staged Y passes are 32 tokens wide");
 };
 
 // Work decomposition ("data-parallel + stream-K").  The first dp_tiles tiles
@@ -174,7 +202,7 @@ struct GemmArgs {
   uint16_t *y;
   const float *x_scale;
   const float *w_scale;
-  float *partials;     // stream-K: [sk_grid][128][BN] fp32
+  float *partials;     // stream-K: [sk_grid][128 MT][BN] fp32
   uint32_t *counters;  // stream-K: [num_tiles - dp_tiles], zero between calls
   int32_t *status;
   const uint8_t *packed;  // tile-packed weights (packed kind only)
@@ -237,19 +265,21 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
 
 // ------------------------------------------------------------------ kernel
 
-template <int KIND, int BN>
+template <int KIND, int BN, int MT>
 __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmE, const GemmArgs p) {
+                const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
+                const GemmArgs p) {
   using T = KindTraits<KIND>;
-  using C = Config<KIND, BN>;
+  using C = Config<KIND, BN, MT>;
   constexpr int S = C::kStages;
   constexpr int NB = C::kAccBufs;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * C::kStageBytes);
+  uint8_t *ystage = smem + S * C::kStageBytes;  // kYBytes: two staged Y passes
+  uint64_t *full = reinterpret_cast<uint64_t *>(ystage + C::kYBytes);
   uint64_t *empty = full + S;
   uint64_t *meta_ready = empty + S;
   uint64_t *tmem_full = meta_ready + S;
@@ -264,6 +294,7 @@ __global__ void __launch_bounds__(192, 1)
     if (!T::kPacked) prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
     if (T::kSparse && !T::kPacked) prefetch_tensormap(&tmE);
+    if (C::kTmaStoreY) prefetch_tensormap(&tmY);
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -302,9 +333,12 @@ __global__ void __launch_bounds__(192, 1)
       // weight half of a stage: values + metadata of rows n0.., k-block kb
       auto load_weights = [&](uint8_t *st, uint64_t *bar, int n0, int kb) {
         if constexpr (T::kPacked) {
-          const uint8_t *blk = p.packed +
-                               (static_cast<int64_t>(n0 / 128) * p.num_kb + kb) * kPackedBlockBytes;
-          bulk_load_g2s(st, blk, kPackedBlockBytes, bar, stream_w);
+#pragma unroll
+          for (int i = 0; i < MT; ++i) {
+            const uint8_t *blk = p.packed +
+                                 (static_cast<int64_t>(n0 / 128 + i) * p.num_kb + kb) * kPackedBlockBytes;
+            bulk_load_g2s(st + C::a_off(i), blk, kPackedBlockBytes, bar, stream_w);
+          }
         } else {
           tma_load_2d(st, &tmA, bar, kb * (T::kARowBytes / T::kAElemBytes), n0, stream_w);
           if (T::kSparse) tma_load_2d(st + C::kEOff, &tmE, bar, kb * T::kERowBytes, n0, stream_w);
@@ -323,7 +357,7 @@ __global__ void __launch_bounds__(192, 1)
         it0.init(p);
         Segment s0;
         while (pre < S && it0.next(p, s0)) {
-          const int n0 = (s0.tile % p.tiles_n) * 128;
+          const int n0 = (s0.tile % p.tiles_n) * C::kRows;
           for (int kb = s0.kb0; kb < s0.kb1 && pre < S; ++kb, ++pre) {
             uint8_t *st = smem + pre * C::kStageBytes;
             mbar_arrive_expect_tx(&full[pre], C::kTmaBytes);
@@ -333,7 +367,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       grid_dependency_wait();
       while (ok && it.next(p, sg)) {
-        const int n0 = (sg.tile % p.tiles_n) * 128;
+        const int n0 = (sg.tile % p.tiles_n) * C::kRows;
         const int m0 = (sg.tile / p.tiles_n) * BN;
         for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++i) {
           const int s = i % S;
@@ -359,7 +393,8 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = mma_idesc(128, BN, T::kFmt, T::kSparse);
-      const uint32_t e_tmem = tmem_base + NB * BN;
+      // metadata of row tile i: 4 TMEM columns after all accumulators
+      const uint32_t e_tmem = tmem_base + NB * C::kAccCols;
       SegIter it;
       it.init(p);
       Segment sg;
@@ -370,7 +405,7 @@ __global__ void __launch_bounds__(192, 1)
         const int r = j / NB;
         if (r >= 1 && !mbar_wait(&tmem_empty[b], static_cast<uint32_t>(r - 1) & 1u, p.status)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + b * BN;
+        const uint32_t d_tmem = tmem_base + b * C::kAccCols;  // row tile rt at + rt * BN
         for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++i) {
           const int s = i % S;
           const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
@@ -380,28 +415,35 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_addr(smem + s * C::kStageBytes);
-          const uint32_t b_addr = a_addr + C::kBOff;
+          const uint32_t st_addr = smem_addr(smem + s * C::kStageBytes);
+          const uint32_t b_addr = st_addr + C::kBOff;
           if (T::kSparse) {
             // 128 rows x 16 B, rows contiguous: core matrices of 8 rows are 128 B apart.
-            const uint32_t e_addr = a_addr + C::kEOff + (T::kMetaTransform ? C::kEBytes : 0);
-            tmem_copy_128x128b(e_tmem, smem_desc(e_addr, 2048, 128, kSwizzleNone));
+#pragma unroll
+            for (int rt = 0; rt < MT; ++rt) {
+              const uint32_t e_addr = st_addr + C::e_off(rt) + (T::kMetaTransform ? C::kEBytes : 0);
+              tmem_copy_128x128b(e_tmem + 4 * rt, smem_desc(e_addr, 2048, 128, kSwizzleNone));
+            }
           }
 #pragma unroll
-          for (int kk = 0; kk < T::kMmas; ++kk) {
-            const uint64_t ad = smem_desc(a_addr + kk * T::kAStep, 16, T::kASbo, T::kASwizzle);
-            const uint32_t boff = (kk * T::kBStep / 128) * (BN * 128) + (kk * T::kBStep) % 128;
-            const uint64_t bd = smem_desc(b_addr + boff, 16, 8 * 128, kSwizzle128B);
-            const uint32_t acc = (kb > sg.kb0 || kk > 0) ? 1u : 0u;
-            if constexpr (KIND == kSparseE4M3 || KIND == kSparseE4M3Packed) {
-              mma_f8_sparse(d_tmem, ad, bd, idesc, e_tmem + 2 * kk, acc);
-            } else if constexpr (KIND == kSparseBF16) {
-              // one metadata column per MMA; columns are addressed in pairs and
-              // the instruction descriptor's selector picks the column of the pair
-              mma_bf16_sparse(d_tmem, ad, bd, idesc | static_cast<uint32_t>(kk & 1),
-                              e_tmem + (kk & ~1), acc);
-            } else {
-              mma_f8_dense(d_tmem, ad, bd, idesc, acc);
+          for (int rt = 0; rt < MT; ++rt) {
+            const uint32_t a_addr = st_addr + C::a_off(rt);
+#pragma unroll
+            for (int kk = 0; kk < T::kMmas; ++kk) {
+              const uint64_t ad = smem_desc(a_addr + kk * T::kAStep, 16, T::kASbo, T::kASwizzle);
+              const uint32_t boff = (kk * T::kBStep / 128) * (BN * 128) + (kk * T::kBStep) % 128;
+              const uint64_t bd = smem_desc(b_addr + boff, 16, 8 * 128, kSwizzle128B);
+              const uint32_t acc = (kb > sg.kb0 || kk > 0) ? 1u : 0u;
+              const uint32_t d = d_tmem + rt * BN;
+              if constexpr (KIND == kSparseE4M3 || KIND == kSparseE4M3Packed) {
+                mma_f8_sparse(d, ad, bd, idesc, e_tmem + 4 * rt + 2 * kk, acc);
+              } else if constexpr (KIND == kSparseBF16) {
+                // one metadata column per MMA; columns are addressed in pairs and
+                // the instruction descriptor's selector picks the column of the pair
+                mma_bf16_sparse(d, ad, bd, idesc | static_cast<uint32_t>(kk & 1), e_tmem + (kk & ~1), acc);
+              } else {
+                mma_f8_dense(d, ad, bd, idesc, acc);
+              }
             }
           }
           mma_commit(&empty[s]);
@@ -420,6 +462,7 @@ __global__ void __launch_bounds__(192, 1)
     const float sw = p.w_scale ? __ldg(p.w_scale) : 1.0f;
     const float sc = sx * sw;
     constexpr int kW = C::kEpiCols;
+    [[maybe_unused]] uint32_t ypass = 0;  // staged Y passes issued so far
     SegIter it;
     it.init(p);
     Segment sg;
@@ -452,25 +495,32 @@ __global__ void __launch_bounds__(192, 1)
       const int r = j / NB;
       mbar_wait(&tmem_full[b], static_cast<uint32_t>(r) & 1u, p.status);
       tc_fence_after();
-      const int n0 = (sg.tile % p.tiles_n) * 128;
+      const int n0 = (sg.tile % p.tiles_n) * C::kRows;
       const int m0 = (sg.tile / p.tiles_n) * BN;
-      const int n = n0 + row;
       const int mvalid = min(BN, p.M - m0);
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
+      // lane quarter of this warp, accumulator b; row tile rt at + rt * BN
+      const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::kAccCols;
+      // fp32 partial tile of CTA g, row tile rt, for this thread's row
+      auto partial_row = [&](int g, int rt) {
+        return p.partials + ((static_cast<size_t>(g) * MT + rt) * 128 + row) * BN;
+      };
 
       if (sg.role == kContrib) {
         // leave the fp32 partial tile (valid token columns) for the owner
-        float *mine = p.partials + (static_cast<size_t>(blockIdx.x) * 128 + row) * BN;
 #pragma unroll 1
-        for (int c = 0; c < mvalid; c += 16) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(t_row + c, v);
-          tmem_ld_wait();
+        for (int rt = 0; rt < MT; ++rt) {
+          float *mine = partial_row(blockIdx.x, rt);
+#pragma unroll 1
+          for (int c = 0; c < mvalid; c += 16) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(t_acc + rt * BN + c, v);
+            tmem_ld_wait();
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4)
-            __stcg(reinterpret_cast<float4 *>(mine + c) + k4,
-                   make_float4(__uint_as_float(v[4 * k4]), __uint_as_float(v[4 * k4 + 1]),
-                               __uint_as_float(v[4 * k4 + 2]), __uint_as_float(v[4 * k4 + 3])));
+            for (int k4 = 0; k4 < 4; ++k4)
+              __stcg(reinterpret_cast<float4 *>(mine + c) + k4,
+                     make_float4(__uint_as_float(v[4 * k4]), __uint_as_float(v[4 * k4 + 1]),
+                                 __uint_as_float(v[4 * k4 + 2]), __uint_as_float(v[4 * k4 + 3])));
+          }
         }
         tc_fence_before();
         mbar_arrive(&tmem_empty[b]);
@@ -499,66 +549,126 @@ __global__ void __launch_bounds__(192, 1)
           }
           named_bar_sync(1, 128);  // the acquire by thread 0 covers the whole CTA's reads
         }
-        // kW token columns per pass.  The first contributor's partial for the
-        // next pass is loaded while this pass is summed and stored, so an
-        // owned tile costs about one L2 round trip, not one per pass.
-        const float *part0 =
-            p.partials + (static_cast<size_t>(first) * 128 + row) * BN;
-        float4 nxt[8];
-        if (first <= last) {
-#pragma unroll
-          for (int k4 = 0; k4 < kW / 4; ++k4) nxt[k4] = __ldcg(reinterpret_cast<const float4 *>(part0) + k4);
-        }
 #pragma unroll 1
-        for (int c = 0; c < mvalid; c += kW) {
-          uint32_t v[2][16];
-          tmem_ld_32x32b_x16(t_row + c, v[0]);
-          if constexpr (kW == 32) tmem_ld_32x32b_x16(t_row + c + 16, v[1]);
-          tmem_ld_wait();
-          float acc[32];
-#pragma unroll
-          for (int k = 0; k < kW; ++k) acc[k] = __uint_as_float(v[k >> 4][k & 15]);
+        for (int rt = 0; rt < MT; ++rt) {
+          const int n = n0 + rt * 128 + row;
+          const uint32_t t_row = t_acc + rt * BN;
+          // kW token columns per pass.  The first contributor's partial for
+          // the next pass is loaded while this pass is summed and stored, so
+          // an owned tile costs about one L2 round trip, not one per pass.
+          const float *part0 = partial_row(first, rt);
+          float4 nxt[8];
           if (first <= last) {
-            float4 cur[8];
 #pragma unroll
-            for (int k4 = 0; k4 < kW / 4; ++k4) cur[k4] = nxt[k4];
-            if (c + kW < mvalid) {
+            for (int k4 = 0; k4 < kW / 4; ++k4) nxt[k4] = __ldcg(reinterpret_cast<const float4 *>(part0) + k4);
+          }
+          // Y through shared memory: this warp's 32 rows of one 32-token pass
+          // (see Config), staged token-major as rows of Y.  Lane 0 issues the
+          // warp's stores; before a buffer is rewritten it waits until the
+          // store issued from it two passes ago has read it.
+          auto store_pass = [&](int c, auto &&value_of) {
+            uint16_t *buf = reinterpret_cast<uint16_t *>(ystage + (q * 2 + (ypass & 1)) * C::kStageY);
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
 #pragma unroll
-              for (int k4 = 0; k4 < kW / 4; ++k4)
-                nxt[k4] = __ldcg(reinterpret_cast<const float4 *>(part0 + c + kW) + k4);
+            for (int k = 0; k < 32; k += 2) {  // two tokens per conversion
+              const __nv_bfloat162 h2 = __floats2bfloat162_rn(value_of(k) * sc, value_of(k + 1) * sc);
+              buf[k * 32 + lane] = __bfloat16_as_ushort(h2.x);
+              buf[(k + 1) * 32 + lane] = __bfloat16_as_ushort(h2.y);
             }
-#pragma unroll
-            for (int k4 = 0; k4 < kW / 4; ++k4) {
-              acc[4 * k4] += cur[k4].x;
-              acc[4 * k4 + 1] += cur[k4].y;
-              acc[4 * k4 + 2] += cur[k4].z;
-              acc[4 * k4 + 3] += cur[k4].w;
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, buf, n0 + rt * 128 + q * 32, m0 + c);
+              bulk_commit_group();
             }
-            for (int g2 = first + 1; g2 <= last; ++g2) {  // further contributors, in CTA order
-              const float4 *src = reinterpret_cast<const float4 *>(
-                  p.partials + (static_cast<size_t>(g2) * 128 + row) * BN + c);
-              float4 pv[8];
+            ++ypass;
+          };
+          if constexpr (C::kTmaStoreY) {
+            if (first > last) {
+              // Whole tile: up to 128 accumulator columns per TMEM wait (the
+              // wait, not the arithmetic, dominates a pass), stored as 32-token
+              // passes.  Tokens past M fall outside the tensor map.
+#pragma unroll 1
+              for (int c2 = 0; c2 < mvalid; c2 += 128) {
+                uint32_t w0[64], w1[64];
+                tmem_ld_32x32b_x64(t_row + c2, w0);
+                if (c2 + 64 < BN) tmem_ld_32x32b_x64(t_row + c2 + 64, w1);
+                tmem_ld_wait();
+                tmem_regs_ready(w0);
+                tmem_regs_ready(w1);
 #pragma unroll
-              for (int k4 = 0; k4 < kW / 4; ++k4) pv[k4] = __ldcg(src + k4);
-#pragma unroll
-              for (int k4 = 0; k4 < kW / 4; ++k4) {
-                acc[4 * k4] += pv[k4].x;
-                acc[4 * k4 + 1] += pv[k4].y;
-                acc[4 * k4 + 2] += pv[k4].z;
-                acc[4 * k4 + 3] += pv[k4].w;
+                for (int h = 0; h < 4; ++h) {
+                  if (c2 + 32 * h < mvalid)
+                    store_pass(c2 + 32 * h, [&](int k) {
+                      return __uint_as_float(h < 2 ? w0[32 * h + k] : w1[32 * (h - 2) + k]);
+                    });
+                }
               }
+              continue;
             }
           }
+#pragma unroll 1
+          for (int c = 0; c < mvalid; c += kW) {
+            uint32_t v[2][16];
+            tmem_ld_32x32b_x16(t_row + c, v[0]);
+            if constexpr (kW == 32) tmem_ld_32x32b_x16(t_row + c + 16, v[1]);
+            tmem_ld_wait();
+            tmem_regs_ready(v[0]);
+            tmem_regs_ready(v[1]);
+            float acc[32];
 #pragma unroll
-          for (int k = 0; k < kW; ++k) {
-            const int m = m0 + c + k;
-            if (m < p.M) p.y[static_cast<size_t>(m) * p.N + n] = f32_to_bf16_bits(acc[k] * sc);
+            for (int k = 0; k < kW; ++k) acc[k] = __uint_as_float(v[k >> 4][k & 15]);
+            if (first <= last) {
+              float4 cur[8];
+#pragma unroll
+              for (int k4 = 0; k4 < kW / 4; ++k4) cur[k4] = nxt[k4];
+              if (c + kW < mvalid) {
+#pragma unroll
+                for (int k4 = 0; k4 < kW / 4; ++k4)
+                  nxt[k4] = __ldcg(reinterpret_cast<const float4 *>(part0 + c + kW) + k4);
+              }
+#pragma unroll
+              for (int k4 = 0; k4 < kW / 4; ++k4) {
+                acc[4 * k4] += cur[k4].x;
+                acc[4 * k4 + 1] += cur[k4].y;
+                acc[4 * k4 + 2] += cur[k4].z;
+                acc[4 * k4 + 3] += cur[k4].w;
+              }
+              for (int g2 = first + 1; g2 <= last; ++g2) {  // further contributors, in CTA order
+                const float4 *src = reinterpret_cast<const float4 *>(partial_row(g2, rt) + c);
+                float4 pv[8];
+#pragma unroll
+                for (int k4 = 0; k4 < kW / 4; ++k4) pv[k4] = __ldcg(src + k4);
+#pragma unroll
+                for (int k4 = 0; k4 < kW / 4; ++k4) {
+                  acc[4 * k4] += pv[k4].x;
+                  acc[4 * k4 + 1] += pv[k4].y;
+                  acc[4 * k4 + 2] += pv[k4].z;
+                  acc[4 * k4 + 3] += pv[k4].w;
+                }
+              }
+            }
+            if constexpr (C::kTmaStoreY) {
+              // Stage the pass token-major, as rows of Y (32 tokens x 128 W
+              // rows), and store it with one bulk tensor copy.
+              store_pass(c, [&](int k) { return acc[k]; });
+            } else {
+#pragma unroll
+              for (int k = 0; k < kW; ++k) {
+                const int m = m0 + c + k;
+                if (m < p.M) p.y[static_cast<size_t>(m) * p.N + n] = f32_to_bf16_bits(acc[k] * sc);
+              }
+            }
           }
         }
         tc_fence_before();
         mbar_arrive(&tmem_empty[b]);
       }
       ++j;
+    }
+    if constexpr (C::kTmaStoreY) {
+      if (lane == 0) bulk_wait_group_all();  // Y written before the CTA leaves
     }
   }
 
@@ -606,9 +716,6 @@ bool make_tensor_map_2d(CUtensorMap *map, const void *ptr, CUtensorMapDataType d
 }
 
 // Token-tile width: the MMA N.  Small token counts use the smallest tile
-// that holds them; large ones prefer 224 (two accumulators fit in tensor
-// memory, so epilogues overlap main loops) unless it pads more than 10%.
-// Token-tile width: the MMA N.  Small token counts use the smallest tile
 // that holds them; medium ones 128 (two accumulators); large ones prefer 224
 // (still two accumulators, so epilogues overlap main loops) unless it pads
 // more than 10% over 256.
@@ -624,8 +731,11 @@ static int choose_bn(GemmKind kind, int M) {
 GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   GemmPlan pl{};
   pl.bn = choose_bn(kind, M);
+  // Large token tiles (224 tokens: many tiles, bound by operand ingest) pair
+  // two 128-row W tiles on one activation tile when N allows it.
+  pl.mt = (pl.bn == 224 && kind != kSparseBF16 && N % 256 == 0) ? 2 : 1;
   pl.bk = 128;
-  pl.tiles_n = N / 128;
+  pl.tiles_n = N / (128 * pl.mt);
   pl.tiles_m = (M + pl.bn - 1) / pl.bn;
   pl.num_kb = K / pl.bk;
   pl.num_tiles = pl.tiles_n * pl.tiles_m;
@@ -652,21 +762,22 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   if (pl.dp_tiles == 0) pl.grid = pl.sk_grid;  // no idle CTAs when every tile is split
   pl.stream_k = rem > 0;
   pl.counter_bytes = pl.stream_k ? kGemmCounterBytes : 0;
-  pl.partial_bytes = pl.stream_k ? static_cast<size_t>(pl.sk_grid) * 128 * pl.bn * sizeof(float) : 0;
+  pl.partial_bytes =
+      pl.stream_k ? static_cast<size_t>(pl.sk_grid) * 128 * pl.mt * pl.bn * sizeof(float) : 0;
   return pl;
 }
 
-template <int KIND, int BN>
+template <int KIND, int BN, int MT>
 static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float *x_scale,
                                 const void *w_values, const uint8_t *w_meta, const float *w_scale,
                                 void *y, int M, int N, int K, void *workspace, int32_t *status,
                                 cudaStream_t st) {
   using T = KindTraits<KIND>;
-  using C = Config<KIND, BN>;
+  using C = Config<KIND, BN, MT>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN>,
+    attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN, MT>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
@@ -681,20 +792,24 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
       T::kASwizzle == kSwizzle64B ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   if (T::kPacked) {
     tmA = {};
-  } else if (!make_tensor_map_2d(&tmA, w_values, dtA, T::kAElemBytes, a_row, N, T::kARowBytes / T::kAElemBytes,
-                       128, a_sw)) {
+  } else if (!make_tensor_map_2d(&tmA, w_values, dtA, T::kAElemBytes, a_row, N,
+                                 T::kARowBytes / T::kAElemBytes, C::kRows, a_sw)) {
     return cudaErrorInvalidValue;
   }
   if (!make_tensor_map_2d(&tmB, xq, dtB, T::kBElemBytes, K, M, T::kBBoxElems, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (T::kSparse && !T::kPacked) {
     if (!make_tensor_map_2d(&tmE, w_meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(K) / 8, N,
-                  16, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+                            16, C::kRows, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   } else {
     tmE = tmB;  // unused
   }
   if (T::kPacked) tmA = tmB;  // unused
+  CUtensorMap tmY = tmB;       // unused unless Y is stored through shared memory
+  if (C::kTmaStoreY &&
+      !make_tensor_map_2d(&tmY, y, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, N, M, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
   GemmArgs a;
   a.M = M;
   a.N = N;
@@ -730,7 +845,7 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   attrs[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN>, tmA, tmB, tmE, a);
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, MT>, tmA, tmB, tmE, tmY, a);
 }
 
 template <int KIND>
@@ -739,12 +854,17 @@ static cudaError_t launch_kind(const GemmPlan &pl, const void *xq, const float *
                                void *y, int M, int N, int K, void *ws, int32_t *status,
                                cudaStream_t st) {
   switch (pl.bn) {
-    case 16: return launch_typed<KIND, 16>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-    case 32: return launch_typed<KIND, 32>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-    case 64: return launch_typed<KIND, 64>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-    case 128: return launch_typed<KIND, 128>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-    case 224: return launch_typed<KIND, 224>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-    case 256: return launch_typed<KIND, 256>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+    case 16: return launch_typed<KIND, 16, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+    case 32: return launch_typed<KIND, 32, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+    case 64: return launch_typed<KIND, 64, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+    case 128: return launch_typed<KIND, 128, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+    case 224:
+      if constexpr (KIND != kSparseBF16) {
+        if (pl.mt == 2)
+          return launch_typed<KIND, 224, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+      }
+      return launch_typed<KIND, 224, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+    case 256: return launch_typed<KIND, 256, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
     default: return cudaErrorInvalidValue;
   }
 }

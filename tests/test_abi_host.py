@@ -39,10 +39,13 @@ def test_workspace_sizes(lib):
     assert lib.sp24_workspace_size(_lib.OP_GEMM_DENSE, 256, 18944, 4096, 0) == 0
     # Otherwise the leftover tiles are split by k-blocks over up to every CTA
     # (at most two ways for tiles wider than 64 tokens): a 16 KB counter
-    # prefix + one fp32 128 x BN partial tile per splitting CTA.  Prefill
-    # M=4096 uses 224-token tiles: 19 x 96 = 1824 tiles = 12 waves + 48
-    # leftover, split over 96 CTAs.
-    assert lib.sp24_workspace_size(_lib.OP_GEMM, 4096, 12288, 4096, 0) == 16384 + 96 * 128 * 224 * 4
+    # prefix + one fp32 (rows x BN) partial tile per splitting CTA.  Prefill
+    # M=4096 uses 224-token tiles of 256 W rows (N % 256 == 0): 19 x 48 = 912
+    # tiles = 6 waves + 24 leftover, split over 48 CTAs.
+    assert lib.sp24_workspace_size(_lib.OP_GEMM, 4096, 12288, 4096, 0) == 16384 + 48 * 256 * 224 * 4
+    # N not a multiple of 256: 128-row tiles, 19 x 75 = 1425 tiles = 9 waves +
+    # 93 leftover over 148 CTAs
+    assert lib.sp24_workspace_size(_lib.OP_GEMM, 4096, 9600, 4096, 0) == 16384 + 148 * 128 * 224 * 4
     # down-proj M=256: 64 tiles of 112 k-blocks, each split over 2 CTAs
     assert lib.sp24_workspace_size(_lib.OP_GEMM, 256, 4096, 14336, 0) == 16384 + 128 * 128 * 128 * 4
     # decode: 16-token tiles

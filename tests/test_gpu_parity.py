@@ -217,12 +217,15 @@ def test_sparse_gemm_small_shapes(m, n, k):
     assert_gemm_close(yd, y_ref, b, f"dense {m}x{n}x{k}")
 
 
-@pytest.mark.parametrize("m,n,k", [(40, 19200, 1024), (200, 19072, 512), (1100, 9600, 640)])
+@pytest.mark.parametrize("m,n,k", [(40, 19200, 1024), (200, 19072, 512), (1100, 9600, 640),
+                                   (1100, 9728, 640), (1024, 512, 1024)])
 def test_gemm_whole_waves_plus_stream_k_tail(m, n, k):
     """More tiles than SMs and not a whole number of waves: the full waves run
     as whole tiles and the leftover tiles are split over CTAs by k-blocks
-    (4-way, 2-way and 2-3-way splits here; the last shape also has a ragged
-    token tile).  The split result must also be deterministic."""
+    (4-way, 2-way and 2-3-way splits here; M=1100 also has a ragged token
+    tile).  N = 9728 and 512 (multiples of 256) with 224-token tiles pair two
+    128-row weight tiles per CTA tile, sparse and dense.  The split result
+    must also be deterministic."""
     x = WL.random_bits((m, k), 500 + m, scale=1.0)
     w = WL.random_bits((n, k), 600 + n, scale=0.02)
     y, yd, xq, sx, vals, meta, sw = _run_sparse(x, w, dense_too=True)

@@ -154,8 +154,9 @@ struct Config {
   // stages its 32 rows x 32 tokens of a pass (2 KB of bf16) in one of two
   // buffers of its own and stores them with a 2-D bulk tensor copy, so the
   // warps never wait for each other (scattered 2-byte stores into Y rows cost
-  // ~10 us per 128 x 224 tile).
-  static constexpr bool kTmaStoreY = BN >= 224;
+  // ~10 us per 128 x 224 tile).  Decode-sized tiles (BN <= 64) keep direct
+  // stores and the deeper ring.
+  static constexpr bool kTmaStoreY = BN >= 128;
   static constexpr uint32_t kStageY = 32 * 32 * 2;          // one warp's pass
   static constexpr uint32_t kYBytes = kTmaStoreY ? 4 * 2 * kStageY : 0;
   static constexpr int kStagesRaw = static_cast<int>((kSmemBudget - kYBytes) / kStageBytes);
@@ -500,24 +501,27 @@ __global__ void __launch_bounds__(192, 1)
       const int mvalid = min(BN, p.M - m0);
       // lane quarter of this warp, accumulator b; row tile rt at + rt * BN
       const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::kAccCols;
-      // fp32 partial tile of CTA g, row tile rt, for this thread's row
-      auto partial_row = [&](int g, int rt) {
-        return p.partials + ((static_cast<size_t>(g) * MT + rt) * 128 + row) * BN;
+      // fp32 partial tile of CTA g, row tile rt, in quads of 4 token columns
+      // laid out [column quad][row][4], so that a warp's 32 rows of one quad
+      // are 512 contiguous bytes: quad cq of this thread's row.
+      auto part4 = [&](int g, int rt, int cq) {
+        return reinterpret_cast<float4 *>(p.partials) +
+               ((static_cast<size_t>(g) * MT + rt) * (BN / 4) + cq) * 128 + row;
       };
 
       if (sg.role == kContrib) {
         // leave the fp32 partial tile (valid token columns) for the owner
 #pragma unroll 1
         for (int rt = 0; rt < MT; ++rt) {
-          float *mine = partial_row(blockIdx.x, rt);
 #pragma unroll 1
           for (int c = 0; c < mvalid; c += 16) {
             uint32_t v[16];
             tmem_ld_32x32b_x16(t_acc + rt * BN + c, v);
             tmem_ld_wait();
+            tmem_regs_ready(v);
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4)
-              __stcg(reinterpret_cast<float4 *>(mine + c) + k4,
+              __stcg(part4(blockIdx.x, rt, c / 4 + k4),
                      make_float4(__uint_as_float(v[4 * k4]), __uint_as_float(v[4 * k4 + 1]),
                                  __uint_as_float(v[4 * k4 + 2]), __uint_as_float(v[4 * k4 + 3])));
           }
@@ -556,11 +560,10 @@ __global__ void __launch_bounds__(192, 1)
           // kW token columns per pass.  The first contributor's partial for
           // the next pass is loaded while this pass is summed and stored, so
           // an owned tile costs about one L2 round trip, not one per pass.
-          const float *part0 = partial_row(first, rt);
           float4 nxt[8];
           if (first <= last) {
 #pragma unroll
-            for (int k4 = 0; k4 < kW / 4; ++k4) nxt[k4] = __ldcg(reinterpret_cast<const float4 *>(part0) + k4);
+            for (int k4 = 0; k4 < kW / 4; ++k4) nxt[k4] = __ldcg(part4(first, rt, k4));
           }
           // Y through shared memory: this warp's 32 rows of one 32-token pass
           // (see Config), staged token-major as rows of Y.  Lane 0 issues the
@@ -625,8 +628,7 @@ __global__ void __launch_bounds__(192, 1)
               for (int k4 = 0; k4 < kW / 4; ++k4) cur[k4] = nxt[k4];
               if (c + kW < mvalid) {
 #pragma unroll
-                for (int k4 = 0; k4 < kW / 4; ++k4)
-                  nxt[k4] = __ldcg(reinterpret_cast<const float4 *>(part0 + c + kW) + k4);
+                for (int k4 = 0; k4 < kW / 4; ++k4) nxt[k4] = __ldcg(part4(first, rt, (c + kW) / 4 + k4));
               }
 #pragma unroll
               for (int k4 = 0; k4 < kW / 4; ++k4) {
@@ -636,10 +638,9 @@ __global__ void __launch_bounds__(192, 1)
                 acc[4 * k4 + 3] += cur[k4].w;
               }
               for (int g2 = first + 1; g2 <= last; ++g2) {  // further contributors, in CTA order
-                const float4 *src = reinterpret_cast<const float4 *>(partial_row(g2, rt) + c);
                 float4 pv[8];
 #pragma unroll
-                for (int k4 = 0; k4 < kW / 4; ++k4) pv[k4] = __ldcg(src + k4);
+                for (int k4 = 0; k4 < kW / 4; ++k4) pv[k4] = __ldcg(part4(g2, rt, c / 4 + k4));
 #pragma unroll
                 for (int k4 = 0; k4 < kW / 4; ++k4) {
                   acc[4 * k4] += pv[k4].x;

@@ -11,8 +11,9 @@ W[11008, 4096] (bf16, N(0, 0.02)) with X[M, 4096] (N(0, 1)) for M in
     ``sp24_prune_compress_packed``), and
   * for each M: quantises X (``fp8_quantize_pertensor``) and runs the sparse
     GEMM (``sp24_gemm_packed``) against another layer's compressed weights.
-The 6:8 workload decomposes (``slide68_decompose``), tile-packs
-(``sp24_pack_weights``), lifts and quantises X (``slide68_lift``) instead.
+The 6:8 workload decomposes into the packed layout
+(``slide68_decompose_packed``) and lifts and quantises X (``slide68_lift``)
+instead.
 
 Layers rotate over pools of at least three times the 126 MB L2 (bf16 weight
 copies and compressed layers), so every kernel reads weights that were last
@@ -237,19 +238,15 @@ class GpuWorkload:
         self.ws.get(max(sp._lib.load().sp24_workspace_size(sp._lib.OP_GEMM, m, n, self.kc, 0) for m in ms) + 4096)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
-        def new_comp(canonical):
-            c = dict(scale=torch.empty((1,), dtype=torch.float32, device=device),
-                     packed=torch.empty(n * self.kc // 2 + n * self.kc // 8, dtype=torch.uint8,
-                                        device=device))
-            if canonical:   # 6:8 decomposes into the canonical arrays, then packs
-                c["values"] = torch.empty((n, self.kc // 2), dtype=torch.uint8, device=device)
-                c["meta"] = torch.empty((n, self.kc // 8), dtype=torch.uint8, device=device)
-            return c
-        self.prune_out = [new_comp(self.is68) for _ in range(2)]
+        def new_comp():
+            return dict(scale=torch.empty((1,), dtype=torch.float32, device=device),
+                        packed=torch.empty(n * self.kc // 2 + n * self.kc // 8, dtype=torch.uint8,
+                                           device=device))
+        self.prune_out = [new_comp() for _ in range(2)]
         self.weight_op(w_dev, self.prune_out[0])
         self.g_pool = []   # the GEMM streams the packed copy only
         for _ in range(self.R_g):
-            c = new_comp(False)
+            c = new_comp()
             for key in c:
                 c[key].copy_(self.prune_out[0][key])
             self.g_pool.append(c)
@@ -268,14 +265,10 @@ class GpuWorkload:
 
     # one call of each kind -------------------------------------------------
     def weight_op(self, w, out):
-        """Weight path into the tile-packed layout the GEMM streams: 2:4
-        prune/quantise/compress in one kernel; 6:8 decomposition, then the
-        tile-packed copy."""
-        if self.is68:
-            self.sp.slide68_decompose(w, "e4m3", status=self.status, workspace=self.ws, out=out)
-            return self.sp.sp24_pack_weights(out["values"], out["meta"], out=out["packed"])
-        return self.sp.sp24_prune_compress_packed(w, status=self.status, workspace=self.ws,
-                                                  out=out["packed"], scale=out["scale"])
+        """Weight path straight into the tile-packed layout the GEMM streams
+        (one kernel: 2:4 prune/quantise/compress, or 6:8 decomposition)."""
+        fn = self.sp.slide68_decompose_packed if self.is68 else self.sp.sp24_prune_compress_packed
+        return fn(w, status=self.status, workspace=self.ws, out=out["packed"], scale=out["scale"])
 
     def act_op(self, m):
         if self.is68:
@@ -295,7 +288,7 @@ class GpuWorkload:
         ops = []
         wi = s % self.R_w
         if self.is68:
-            wname, wbytes, wl = "slide68_decompose+pack", bytes_slide68(n, k) + 2 * self.comp_bytes, 2
+            wname, wbytes, wl = "slide68_decompose_packed", bytes_slide68(n, k), 1
         else:
             wname, wbytes, wl = "sp24_prune_compress_packed", bytes_prune24(n, k), 1
         ops.append((wname, lambda: self.weight_op(self.w_pool[wi], self.prune_out[s % 2]), wbytes, 0, wl))
@@ -498,9 +491,10 @@ def run_gpu(args, wl, rank, world, local_rank):
         "dtype": "e4m3",
         "data": "synthetic (seeded, bf16 N(0,0.02) weights / N(0,1) activations; see workloads.py)",
         "config": {"workload": wl["name"], "n": wl["n"], "k": wl["k"], "m": list(wl["ms"]),
-                   "step": ("weight 6:8 decompose + tile-pack" if gw.is68 else
-                            "weight 2:4 prune/quantise/compress into the tile-packed layout")
-                           + ", then per M: activation quantise + sparse GEMM",
+                   "step": ("weight 6:8 decomposition" if gw.is68 else
+                            "weight 2:4 prune/quantise/compress")
+                           + " into the tile-packed layout, then per M: activation quantise"
+                           + (" + lift" if gw.is68 else "") + " + sparse GEMM",
                    "algorithmic_bytes_per_step": step_bytes,
                    "l2": f"inputs larger than L2: rotating pools of {gw.R_w} bf16 weight copies and "
                          f"{gw.R_g} compressed layers",

@@ -199,6 +199,19 @@ int sp24_prune_compress_packed(const void *W, int N, int K, void *packed, float 
                                sp24_stream_t stream);
 
 /*
+ * The E4M3 path of slide68_decompose written straight into the tile-packed
+ * layout of the lifted 2:4 operand (K' = 3K/2): packed receives, byte for
+ * byte, what sp24_pack_weights(values, meta, N, K') would make of the values
+ * and metadata that slide68_decompose(W, N, K, SP24_DTYPE_E4M3, ...)
+ * computes; w_scale <- amax|W| / 448.  packed: u8, N*K'/2 + N*K'/8 bytes.
+ * Workspace: sp24_workspace_size(SP24_OP_SLIDE68_DECOMPOSE, ...).
+ * Shape rules: N % 128 == 0, K % 256 == 0, N * K <= 2^38.
+ */
+int slide68_decompose_packed(const void *W, int N, int K, void *packed, float *w_scale,
+                             void *workspace, size_t ws_bytes, int32_t *status,
+                             sp24_stream_t stream);
+
+/*
  * sp24_gemm (E4M3) with tile-packed weights (sp24_pack_weights); same result.
  * Workspace from sp24_workspace_size(SP24_OP_GEMM_PACKED, M, N, K, 0).
  */

@@ -18,7 +18,8 @@ from ._lib import DTYPE_BF16, DTYPE_E4M3, Sp24Error  # noqa: F401
 
 __all__ = [
     "sp24_prune_compress", "fp8_quantize_pertensor", "slide68_decompose", "slide68_lift",
-    "sp24_gemm", "fp8_gemm_dense", "sp24_pack_weights", "sp24_prune_compress_packed", "sp24_gemm_packed",
+    "sp24_gemm", "fp8_gemm_dense", "sp24_pack_weights", "sp24_prune_compress_packed", "slide68_decompose_packed",
+    "sp24_gemm_packed",
     "Workspace",
     "Sp24Error", "DTYPE_E4M3", "DTYPE_BF16",
 ]
@@ -236,6 +237,33 @@ def sp24_prune_compress_packed(W: torch.Tensor, status: torch.Tensor | None = No
     rc = lib.sp24_prune_compress_packed(_ptr(W), N, K, _ptr(packed), _ptr(sc), _ptr(ws), wsn,
                                         _ptr(status), _stream(W.device))
     _lib.check(rc, "sp24_prune_compress_packed")
+    return packed, sc
+
+
+def slide68_decompose_packed(W: torch.Tensor, status: torch.Tensor | None = None,
+                             workspace: Workspace | None = None, out: torch.Tensor | None = None,
+                             scale: torch.Tensor | None = None):
+    """E4M3 6:8 decomposition of W bf16 [N, K] straight into the tile-packed
+    layout of the lifted 2:4 operand (K' = 3K/2): what sp24_pack_weights
+    makes of slide68_decompose's output.
+
+    Returns (packed u8 [N*K'/2 + N*K'/8], scale f32 [1]).
+    """
+    lib = _lib.load()
+    _require_cuda(W, status, out, scale)
+    if W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise Sp24Error("W must be a 2-D bf16 tensor")
+    N, K = W.shape
+    kl = 3 * K // 2
+    packed = out if out is not None else torch.empty(N * kl // 2 + N * kl // 8, dtype=torch.uint8,
+                                                     device=W.device)
+    if packed.numel() != N * kl // 2 + N * kl // 8 or packed.dtype != torch.uint8:
+        raise Sp24Error("packed output has the wrong size or dtype")
+    sc = scale if scale is not None else torch.empty((1,), dtype=torch.float32, device=W.device)
+    ws, wsn = _ws(W.device, _lib.OP_SLIDE68_DECOMPOSE, 0, N, K, DTYPE_E4M3, workspace)
+    rc = lib.slide68_decompose_packed(_ptr(W), N, K, _ptr(packed), _ptr(sc), _ptr(ws), wsn,
+                                      _ptr(status), _stream(W.device))
+    _lib.check(rc, "slide68_decompose_packed")
     return packed, sc
 
 

@@ -41,6 +41,7 @@ SIGNATURES = {
     "fp8_gemm_dense": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _sz, _p, _p]),
     "sp24_pack_weights": (_i, [_p, _p, _i, _i, _p, _p]),
     "sp24_prune_compress_packed": (_i, [_p, _i, _i, _p, _p, _p, _sz, _p, _p]),
+    "slide68_decompose_packed": (_i, [_p, _i, _i, _p, _p, _p, _sz, _p, _p]),
     "sp24_gemm_packed": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _sz, _p, _p]),
     "sp24_workspace_size": (_sz, [_i, _i64, _i64, _i64, _i]),
     "sp24_status_str": (ctypes.c_char_p, [_i]),

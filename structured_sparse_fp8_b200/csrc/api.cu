@@ -132,6 +132,23 @@ int sp24_prune_compress_packed(const void *W, int N, int K, void *packed, float 
                                                        sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int slide68_decompose_packed(const void *W, int N, int K, void *packed, float *w_scale,
+                             void *workspace, size_t ws_bytes, int32_t *status,
+                             sp24_stream_t stream) {
+  if (!W || !packed || !w_scale) return SP24_ERR_NULL;
+  if (N < 128 || K < 256 || N % 128 != 0 || K % 256 != 0 ||
+      static_cast<int64_t>(N) * K > (static_cast<int64_t>(1) << 38))
+    return SP24_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(packed)) return SP24_ERR_ALIGN;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  const int rc = check_workspace(workspace, ws_bytes);
+  if (rc != SP24_OK) return rc;
+  return cuda_status(sp24::launch_slide68_packed_fused(W, N, K, static_cast<uint32_t *>(workspace),
+                                                       w_scale, static_cast<uint8_t *>(packed), status,
+                                                       sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int fp8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, uint8_t *q, float *scale,
                            void *workspace, size_t ws_bytes, int32_t *status,
                            sp24_stream_t stream) {

@@ -42,6 +42,11 @@ cudaError_t launch_prune24_fused(const void *w, int64_t nelem, bool fp8, uint32_
 cudaError_t launch_prune24_packed_fused(const void *w, int N, int K, uint32_t *ws, float *scale,
                                         uint8_t *packed, int32_t *status, int sm_count,
                                         cudaStream_t st);
+// 6:8 decomposition + E4M3 quantise written straight into the tile-packed
+// layout of the lifted 2:4 operand (N % 128 == 0, K % 256 == 0).
+cudaError_t launch_slide68_packed_fused(const void *w, int N, int K, uint32_t *ws, float *scale,
+                                        uint8_t *packed, int32_t *status, int sm_count,
+                                        cudaStream_t st);
 cudaError_t launch_slide68_fused(const void *w, int64_t nelem, bool fp8, uint32_t *ws,
                                  float *scale, void *values, uint8_t *meta, int32_t *status,
                                  int sm_count, cudaStream_t st);

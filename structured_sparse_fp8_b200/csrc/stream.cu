@@ -4,7 +4,8 @@
 //   kOpLift      the same fused with the 6:8 activation lift,
 //   kOpPrune24   2:4 magnitude prune + quantise + compress of weights,
 //   kOpPrune24Packed  the same, written in the GEMM's tile-packed layout,
-//   kOpSlide68   6:8 prune + sliding-window decomposition of weights.
+//   kOpSlide68   6:8 prune + sliding-window decomposition of weights,
+//   kOpSlide68Packed  the same, written in the GEMM's tile-packed layout.
 //
 // One CTA per SM (cooperative launch: all CTAs resident), each owning a
 // contiguous range of 32 KB chunks of the bf16 input (for the packed 2:4 op a
@@ -60,7 +61,14 @@ constexpr uint32_t smem_bytes() {
 }
 static_assert(smem_bytes<false>() + 2048 <= 227 * 1024, "ring + table exceed the shared memory of a CTA");
 
-enum StreamOp : int { kOpQuantize = 0, kOpLift = 1, kOpPrune24 = 2, kOpSlide68 = 3, kOpPrune24Packed = 4 };
+enum StreamOp : int {
+  kOpQuantize = 0,
+  kOpLift = 1,
+  kOpPrune24 = 2,
+  kOpSlide68 = 3,
+  kOpPrune24Packed = 4,
+  kOpSlide68Packed = 5
+};
 
 // Bytes of input one consumer thread handles as one unit: 8 bf16 (one
 // metadata byte of 2:4, one 8-group of the lift) or 16 bf16 for 6:8 (two
@@ -69,12 +77,14 @@ enum StreamOp : int { kOpQuantize = 0, kOpLift = 1, kOpPrune24 = 2, kOpSlide68 =
 // consecutive 16-byte words (no shared-memory bank conflicts) and write
 // consecutive outputs.
 template <int OP>
-__host__ __device__ constexpr int unit_bytes() { return OP == kOpSlide68 ? 32 : 16; }
+__host__ __device__ constexpr int unit_bytes() { return OP == kOpSlide68 || OP == kOpSlide68Packed ? 32 : 16; }
 
 struct StreamArgs {
-  // kOpPrune24Packed reads W through this 2-D map (box 128 rows x 128 bf16):
-  // chunk c is the input of packed block c, rows 128 (c / kblocks) ..,
-  // columns 128 (c % kblocks) ..
+  // The packed ops read W through this 2-D map.  kOpPrune24Packed: box 128
+  // rows x 128 bf16, chunk c is the input of packed block c (rows
+  // 128 (c / kblocks) .., columns 128 (c % kblocks) ..).  kOpSlide68Packed:
+  // box 64 rows x 256 bf16 = the input of rows 64 h .. of packed blocks
+  // 3 kg .. 3 kg + 2 of row tile t, for chunk c = (t K/256 + kg) 2 + h.
   CUtensorMap wmap;
   const uint8_t *x;  // bf16 input
   int64_t nbytes;    // input bytes, a multiple of 32
@@ -85,7 +95,7 @@ struct StreamArgs {
   uint8_t *out;      // codes / kept values (the packed blocks for kOpPrune24Packed)
   uint8_t *meta;
   uint8_t *dense;
-  uint32_t kblocks;  // kOpPrune24Packed: K / 128
+  uint32_t kblocks;  // packed ops: K-blocks of the compressed operand per row (K / 128, 6:8: K' / 128)
 };
 
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
@@ -162,7 +172,9 @@ __device__ __forceinline__ void halves(const uint4 v, uint32_t h[8]) {
 // per-chunk 64-bit bases plus 32-bit offsets of u.
 struct Chunk {
   uint64_t e;
-  uint64_t idx;  // the chunk's index (= its packed block for kOpPrune24Packed)
+  uint64_t idx;     // the chunk's index (= its packed block for kOpPrune24Packed)
+  uint8_t *group;   // kOpSlide68Packed: packed block (t, 3 kg) of the chunk
+  uint32_t row0;    // kOpSlide68Packed: first row in the row tile (0 or 64)
 };
 
 // ------------------------------------------------------------------ 2:4 + E4M3
@@ -297,13 +309,49 @@ __device__ __forceinline__ uint8_t *meta_byte(const StreamArgs &a, const Chunk &
     return a.meta + (ch.e >> 3) + u;
 }
 
+// kOpSlide68Packed: where unit u of chunk `ch` lands.  Row r of row tile t,
+// K'-group kg (three packed blocks); the unit is 16 W columns = 24 K'
+// columns: value bytes 12 j .. 12 j + 11 and metadata bytes 3 j .. 3 j + 2 of
+// the group's 192 / 48 bytes per row (j = unit in the row).
+struct Slide68Place {
+  uint8_t *group;  // packed block (t, 3 kg)
+  uint32_t r, j;
+};
+
+// the chunk's packed block group and first row, once per chunk:
+// chunk c = (t K/256 + kg) 2 + h covers rows 64 h .. of row tile t
+__device__ __forceinline__ void slide68_chunk(const StreamArgs &a, Chunk &ch) {
+  const uint32_t kgroups = a.kblocks / 3;
+  const uint32_t c = static_cast<uint32_t>(ch.idx);
+  const uint32_t t = c / (2 * kgroups), rem = c - t * (2 * kgroups);
+  ch.group = a.out + (static_cast<uint64_t>(t) * a.kblocks + 3 * (rem >> 1)) * kPackedBlockBytes;
+  ch.row0 = 64 * (rem & 1u);
+}
+
+__device__ __forceinline__ Slide68Place slide68_place(const StreamArgs &, const Chunk &ch, uint32_t u) {
+  return Slide68Place{ch.group, ch.row0 + (u >> 4), u & 15u};
+}
+
+// metadata byte b (0..47) of the place's row
+__device__ __forceinline__ uint8_t *slide68_meta_at(const Slide68Place &pl, uint32_t b) {
+  return pl.group + (b >> 4) * kPackedBlockBytes + 128 * 64 + pl.r * 16 + (b & 15u);
+}
+
+// 4-byte value word at row byte o (0..188, a multiple of 4) of the place's row,
+// inside the 64-byte-swizzled chunk placement of its block
+__device__ __forceinline__ uint32_t *slide68_value_at(const Slide68Place &pl, uint32_t o) {
+  const uint32_t ob = o & 63u;
+  return reinterpret_cast<uint32_t *>(pl.group + (o >> 6) * kPackedBlockBytes + pl.r * 64 +
+                                      ((((ob >> 4) ^ (pl.r >> 1)) & 3u) << 4) + (ob & 15u));
+}
+
 // ------------------------------------------------------------------ phase 1
 // One unit: `p` its bytes in shared memory, u its index in chunk `ch`; mx2
 // accumulates the per-lane largest magnitude bits.
 template <int OP, bool FP8, bool DENSE>
 __device__ __forceinline__ void phase1_unit(const uint8_t *p, const Chunk &ch, uint32_t u,
                                             const StreamArgs &a, const uint32_t *nib64, uint32_t &mx2) {
-  if constexpr (OP == kOpSlide68) {
+  if constexpr (OP == kOpSlide68 || OP == kOpSlide68Packed) {
     const uint4 v0 = reinterpret_cast<const uint4 *>(p)[0];
     const uint4 v1 = reinterpret_cast<const uint4 *>(p)[1];
     uint32_t nib[6], vals[12];
@@ -331,10 +379,17 @@ __device__ __forceinline__ void phase1_unit(const uint8_t *p, const Chunk &ch, u
         }
       }
     }
-    uint8_t *m = a.meta + 3 * (ch.e >> 4) + 3 * u;
-    m[0] = static_cast<uint8_t>(nib[0] | (nib[1] << 4));
-    m[1] = static_cast<uint8_t>(nib[2] | (nib[3] << 4));
-    m[2] = static_cast<uint8_t>(nib[4] | (nib[5] << 4));
+    if constexpr (OP == kOpSlide68Packed) {
+      const Slide68Place pl = slide68_place(a, ch, u);
+#pragma unroll
+      for (int b = 0; b < 3; ++b)
+        *slide68_meta_at(pl, 3 * pl.j + b) = static_cast<uint8_t>(nib[2 * b] | (nib[2 * b + 1] << 4));
+    } else {
+      uint8_t *m = a.meta + 3 * (ch.e >> 4) + 3 * u;
+      m[0] = static_cast<uint8_t>(nib[0] | (nib[1] << 4));
+      m[1] = static_cast<uint8_t>(nib[2] | (nib[3] << 4));
+      m[2] = static_cast<uint8_t>(nib[4] | (nib[5] << 4));
+    }
     if (!FP8) {
       uint2 *d = reinterpret_cast<uint2 *>(a.out + 24 * (ch.e >> 4) + 24 * u);
 #pragma unroll
@@ -383,7 +438,7 @@ __device__ __forceinline__ void phase1_unit(const uint8_t *p, const Chunk &ch, u
 template <int OP, bool DENSE, class Code>
 __device__ __forceinline__ void phase2_unit(const uint8_t *p, const Chunk &ch, uint32_t u, uint32_t meta_in,
                                             const StreamArgs &a, const Code &code, const uint32_t *sel16) {
-  if constexpr (OP == kOpSlide68) {
+  if constexpr (OP == kOpSlide68 || OP == kOpSlide68Packed) {
     const uint4 v0 = reinterpret_cast<const uint4 *>(p)[0];
     const uint4 v1 = reinterpret_cast<const uint4 *>(p)[1];
     const uint32_t m3 = meta_in;
@@ -406,10 +461,18 @@ __device__ __forceinline__ void phase2_unit(const uint8_t *p, const Chunk &ch, u
         c[6 * gl + 2 * j + 1] = code(h1);
       }
     }
-    uint32_t *d = reinterpret_cast<uint32_t *>(a.out + 12 * (ch.e >> 4) + 12 * u);
+    if constexpr (OP == kOpSlide68Packed) {
+      const Slide68Place pl = slide68_place(a, ch, u);
 #pragma unroll
-    for (int o = 0; o < 3; ++o)
-      d[o] = c[4 * o] | (c[4 * o + 1] << 8) | (c[4 * o + 2] << 16) | (c[4 * o + 3] << 24);
+      for (int o = 0; o < 3; ++o)
+        *slide68_value_at(pl, 12 * pl.j + 4 * o) =
+            c[4 * o] | (c[4 * o + 1] << 8) | (c[4 * o + 2] << 16) | (c[4 * o + 3] << 24);
+    } else {
+      uint32_t *d = reinterpret_cast<uint32_t *>(a.out + 12 * (ch.e >> 4) + 12 * u);
+#pragma unroll
+      for (int o = 0; o < 3; ++o)
+        d[o] = c[4 * o] | (c[4 * o + 1] << 8) | (c[4 * o + 2] << 16) | (c[4 * o + 3] << 24);
+    }
   } else {
     const uint4 v = *reinterpret_cast<const uint4 *>(p);
     if constexpr (OP == kOpPrune24Packed) {
@@ -490,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     // (phase 2 walks the range backwards), into slot L % kS.  The second
     // pass is prefetched as soon as slots free up.
     if ((tid & 31) == 0) {
-      if constexpr (OP == kOpPrune24Packed) prefetch_tensormap(&a.wmap);
+      if constexpr (OP == kOpPrune24Packed || OP == kOpSlide68Packed) prefetch_tensormap(&a.wmap);
       for (int L = 0; L < n_loads; ++L) {
         const int slot = L % kS;
         if (L >= kS && !mbar_wait(&empty[slot], static_cast<uint32_t>(L / kS - 1) & 1u, a.status))
@@ -504,6 +567,12 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
           const uint32_t kb = static_cast<uint32_t>(c) - t * a.kblocks;
           tma_load_2d(ring + slot * kChunkBytes, &a.wmap, &full[slot], static_cast<int32_t>(kb * 128),
                       static_cast<int32_t>(t * 128), l2_policy_evict_normal());
+        } else if constexpr (OP == kOpSlide68Packed) {
+          const uint32_t kgroups = a.kblocks / 3;
+          const uint32_t t = static_cast<uint32_t>(c) / (2 * kgroups);
+          const uint32_t rem = static_cast<uint32_t>(c) - t * (2 * kgroups);
+          tma_load_2d(ring + slot * kChunkBytes, &a.wmap, &full[slot], static_cast<int32_t>((rem >> 1) * 256),
+                      static_cast<int32_t>(t * 128 + (rem & 1u) * 64), l2_policy_evict_normal());
         } else {
           bulk_load(ring + slot * kChunkBytes, a.x + c * kChunkBytes, nb, &full[slot]);
         }
@@ -531,8 +600,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
       }
     }
   };
-  auto chunk_of = [](int64_t c) {
-    return Chunk{static_cast<uint64_t>(c) * (kChunkBytes / 2), static_cast<uint64_t>(c)};
+  auto chunk_of = [&](int64_t c) {
+    Chunk ch{static_cast<uint64_t>(c) * (kChunkBytes / 2), static_cast<uint64_t>(c), nullptr, 0};
+    if constexpr (OP == kOpSlide68Packed) slide68_chunk(a, ch);
+    return ch;
   };
 
   // The table costs about as much as dividing 2 chunks' elements directly.
@@ -603,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     // The units' metadata (1 byte for 2:4, 3 for 6:8; this thread wrote it in
     // phase 1) of chunk c, loaded one chunk ahead so the L2 latency overlaps
     // the previous chunk's work.
-    constexpr bool kMetaIn = OP == kOpSlide68 || selects_in_phase1<OP, FP8, DENSE>();
+    constexpr bool kMetaIn = OP == kOpSlide68 || OP == kOpSlide68Packed || selects_in_phase1<OP, FP8, DENSE>();
     auto load_meta = [&](int64_t c, uint32_t (&m)[kRows]) {
       const Chunk ch = chunk_of(c);
       const int64_t nb = min(static_cast<int64_t>(kChunkBytes), a.nbytes - c * kChunkBytes);
@@ -616,6 +687,11 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
             const uint8_t *mp = a.meta + 3 * (ch.e >> 4) + 3 * u;
             m[r] = __ldcg(mp) | (static_cast<uint32_t>(__ldcg(mp + 1)) << 8) |
                    (static_cast<uint32_t>(__ldcg(mp + 2)) << 16);
+          } else if constexpr (OP == kOpSlide68Packed) {
+            const Slide68Place pl = slide68_place(a, ch, u);
+            m[r] = __ldcg(slide68_meta_at(pl, 3 * pl.j)) |
+                   (static_cast<uint32_t>(__ldcg(slide68_meta_at(pl, 3 * pl.j + 1))) << 8) |
+                   (static_cast<uint32_t>(__ldcg(slide68_meta_at(pl, 3 * pl.j + 2))) << 16);
           } else {
             m[r] = __ldcg(meta_byte<OP>(a, ch, u));
           }
@@ -764,6 +840,19 @@ cudaError_t launch_prune24_packed_fused(const void *w, int N, int K, uint32_t *w
                           static_cast<uint64_t>(N), 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   return launch_stream_typed<kOpPrune24Packed, true, false>(a, sm_count, st);
+}
+
+cudaError_t launch_slide68_packed_fused(const void *w, int N, int K, uint32_t *ws, float *scale,
+                                        uint8_t *packed, int32_t *status, int sm_count,
+                                        cudaStream_t st) {
+  StreamArgs a = make_args(w, static_cast<int64_t>(N) * K, ws, scale, status, packed, nullptr, nullptr);
+  a.kblocks = static_cast<uint32_t>(3 * K / 256);  // K' / 128
+  // chunk = 64 rows x 256 columns of W = rows 64 h .. of three packed blocks
+  static_assert(kChunkBytes == 64 * 256 * 2, "a chunk must be half the input of three packed blocks");
+  if (!make_tensor_map_2d(&a.wmap, w, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, static_cast<uint64_t>(K),
+                          static_cast<uint64_t>(N), 256, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  return launch_stream_typed<kOpSlide68Packed, true, false>(a, sm_count, st);
 }
 
 cudaError_t launch_slide68_fused(const void *w, int64_t nelem, bool fp8, uint32_t *ws,

@@ -82,6 +82,8 @@ def test_validation_rejects_bad_arguments_without_a_gpu(lib):
     assert lib.sp24_prune_compress_packed(FAKE, 128, 192, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
     assert lib.sp24_prune_compress_packed(FAKE, 64, 128, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
     assert lib.sp24_prune_compress_packed(FAKE, 128, 128, FAKE, None, FAKE, ws, None, None) == _lib.SP24_ERR_NULL
+    assert lib.slide68_decompose_packed(FAKE, 128, 128, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.slide68_decompose_packed(FAKE, 96, 256, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
     # alignment
     odd = ctypes.c_void_p((1 << 20) + 8)
     assert lib.sp24_prune_compress_packed(FAKE, 128, 128, odd, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN

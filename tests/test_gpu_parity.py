@@ -452,6 +452,33 @@ def test_prune_compress_packed_workload_equals_pack_of_canonical(cfg):
     assert torch.equal(scale, c["scale"])
 
 
+@pytest.mark.parametrize("n,k,dist", [(128, 256, "normal"), (256, 512, "ties"), (384, 2304, "student_t3"),
+                                      (1024, 4096, "normal")])
+def test_slide68_decompose_packed_matches_oracle(n, k, dist):
+    """Direct packed 6:8 output == the documented packing of the oracle's
+    lifted 2:4 values and metadata (K' = 1.5 K), byte for byte."""
+    w = WL.random_bits((n, k), 1100 + n, scale=0.02, dist=dist)
+    st = new_status()
+    packed, scale = sp().slide68_decompose_packed(dev_bf16(w), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = O.slide68_decompose(w, "e4m3")
+    assert host(scale)[0] == np.float32(ref["scale"])
+    want = _pack_reference(ref["values"], ref["meta"], n, 3 * k // 2)
+    got = host(packed)
+    if not np.array_equal(got, want):
+        bad = np.flatnonzero(got != want)
+        raise AssertionError(f"{bad.size} bytes differ, first at {bad[:8].tolist()}")
+
+
+def test_slide68_decompose_packed_workload_equals_pack_of_canonical():
+    w = dev_bf16(WL.weight_bits(5))
+    c = sp().slide68_decompose(w, "e4m3")
+    packed, scale = sp().slide68_decompose_packed(w)
+    assert torch.equal(packed, sp().sp24_pack_weights(c["values"], c["meta"]))
+    assert torch.equal(scale, c["scale"])
+
+
 @pytest.mark.parametrize("m,n,k", [(1, 128, 128), (5, 256, 512), (64, 384, 1024), (300, 256, 1152)])
 def test_packed_gemm_small(m, n, k):
     x = WL.random_bits((m, k), 800 + m)

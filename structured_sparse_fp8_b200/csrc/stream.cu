@@ -770,11 +770,22 @@ cudaError_t launch_stream_variant(const StreamArgs &a, int64_t grid, cudaStream_
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem_bytes<SMALL>();
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  // Cooperative: only the two-phase kernels wait on each other.
+  // Programmatic dependent launch: the grid may start while the previous
+  // kernel finishes; every CTA passes griddepcontrol.wait before touching
+  // memory.
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (FP8) {
+    attr[na].id = cudaLaunchAttributeCooperative;
+    attr[na].val.cooperative = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = FP8 ? 1 : 0;  // only the two-phase kernels wait on each other
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, stream_kernel<OP, FP8, DENSE, SMALL>, a);
 }
 

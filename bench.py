@@ -9,11 +9,15 @@ W[11008, 4096] (bf16, N(0, 0.02)) with X[M, 4096] (N(0, 1)) for M in
   * prunes, quantises and compresses one layer's weights (weight amax +
     2:4 prune/quantise/compress, written in the GEMM's tile-packed layout:
     ``sp24_prune_compress_packed``), and
-  * for each M: quantises X (``fp8_quantize_pertensor``) and runs the sparse
-    GEMM (``sp24_gemm_packed``) against another layer's compressed weights.
+  * for each M: quantises X and runs the sparse GEMM against another layer's
+    compressed weights: for M <= 256 in one launch
+    (``sp24_quantize_gemm_packed``), otherwise as ``fp8_quantize_pertensor``
+    followed by ``sp24_gemm_packed``.
 The 6:8 workload decomposes into the packed layout
-(``slide68_decompose_packed``) and lifts and quantises X (``slide68_lift``)
-instead.
+(``slide68_decompose_packed``) and lifts and quantises X instead
+(``slide68_lift_gemm_packed``, or ``slide68_lift`` + ``sp24_gemm_packed``).
+``--unfused`` keeps the two launches at every M; ``fused_vs_unfused`` in the
+output times both forms of each small-M GEMM.
 
 Layers rotate over pools of at least three times the 126 MB L2 (bf16 weight
 copies and compressed layers), so every kernel reads weights that were last
@@ -76,6 +80,15 @@ def bytes_slide68(n, k):
 
 def bytes_lift(m, k):
     return 2 * m * k + 3 * m * k // 2 + 4
+
+
+def bytes_fused_gemm(m, n, k, kc):
+    """Quantise (or lift) + GEMM in one launch: packed weights, X in bf16, the
+    codes written out, Y."""
+    return n * kc // 2 + n * kc // 8 + 2 * m * k + m * kc + 2 * m * n + 8
+
+
+FUSED_MAX_M = 64  # above this the full-grid quantiser launch is faster
 
 
 WORKLOADS = {
@@ -214,7 +227,7 @@ class ClockSampler:
 class GpuWorkload:
     """Device buffers, rotating pools and the step for one workload."""
 
-    def __init__(self, wl, device):
+    def __init__(self, wl, device, unfused=False):
         import torch
 
         import structured_sparse_fp8_b200 as sp
@@ -223,6 +236,7 @@ class GpuWorkload:
         n, k, ms = wl["n"], wl["k"], wl["ms"]
         self.n, self.k, self.ms = n, k, ms
         self.is68 = wl["pattern"] == "6:8"
+        self.fused = {m: (not unfused) and m <= FUSED_MAX_M for m in ms}
         self.kc = k * 3 // 2 if self.is68 else k   # K of the compressed operand
         w_host = WL.weight_bits(wl["cfg"])
         self.w_host_pinned = torch.from_numpy(w_host.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -282,6 +296,15 @@ class GpuWorkload:
         return self.sp.sp24_gemm_packed(self.xq[m], self.sx[m], c["packed"], c["scale"], self.n,
                                         out=self.y[m], status=self.status, workspace=self.ws)
 
+    def fused_name(self):
+        return "slide68_lift_gemm_packed" if self.is68 else "sp24_quantize_gemm_packed"
+
+    def fused_op(self, m, layer):
+        c = self.g_pool[layer]
+        fn = getattr(self.sp, self.fused_name())
+        return fn(self.x_dev[m], c["packed"], c["scale"], self.n, out=self.y[m], xq_out=self.xq[m],
+                  x_scale_out=self.sx[m], status=self.status, workspace=self.ws)
+
     def ops_of_step(self, s):
         """(name, callable, algorithmic bytes, flops, kernel launches) of step s."""
         n, k, kc = self.n, self.k, self.kc
@@ -294,6 +317,10 @@ class GpuWorkload:
         ops.append((wname, lambda: self.weight_op(self.w_pool[wi], self.prune_out[s % 2]), wbytes, 0, wl))
         for j, m in enumerate(self.ms):
             layer = (s * len(self.ms) + j) % self.R_g
+            if self.fused[m]:
+                ops.append((self.fused_name(), (lambda m=m, layer=layer: self.fused_op(m, layer)),
+                            bytes_fused_gemm(m, n, k, kc), 2 * m * n * kc, 1))
+                continue
             aname = "slide68_lift" if self.is68 else "fp8_quantize_pertensor"
             abytes = bytes_lift(m, k) if self.is68 else bytes_quant(m, k)
             ops.append((aname, (lambda m=m: self.act_op(m)), abytes, 0, 1))
@@ -368,6 +395,40 @@ class GpuWorkload:
         del dpool
         return out
 
+    def fusion_compare(self, reps=50):
+        """For every M that the step runs fused: the fused launch against the
+        activation kernel + GEMM pair it replaces, each as a CUDA graph of
+        `reps` back-to-back repetitions over rotating weights."""
+        torch = self.torch
+        out = {}
+        for m in self.ms:
+            if m > FUSED_MAX_M:
+                continue
+            res = {}
+            for kind in ("fused", "unfused"):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    for r in range(reps):
+                        if kind == "fused":
+                            self.fused_op(m, r % self.R_g)
+                        else:
+                            self.act_op(m)
+                            self.gemm_op(m, r % self.R_g)
+                g.replay()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                g.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                res[kind] = e0.elapsed_time(e1) * 1000.0 / reps
+                del g
+            nb = bytes_fused_gemm(m, self.n, self.k, self.kc)
+            out[str(m)] = {"fused_us": round(res["fused"], 3), "unfused_us": round(res["unfused"], 3),
+                           "speedup": round(res["unfused"] / res["fused"], 3),
+                           "fused_gbs": round(nb / res["fused"] / 1e3, 1)}
+        return out
+
     # e2e through the public API with host buffers ---------------------------
     def e2e(self, steps):
         torch = self.torch
@@ -402,7 +463,7 @@ def run_gpu(args, wl, rank, world, local_rank):
     torch.cuda.set_device(device)
     import __graft_entry__
     __graft_entry__.build()
-    gw = GpuWorkload(wl, device)
+    gw = GpuWorkload(wl, device, unfused=args.unfused)
     peaks = load_peaks()
 
     # warm-up: W eager steps (first calls set kernel attributes), then graphs
@@ -447,8 +508,6 @@ def run_gpu(args, wl, rank, world, local_rank):
     dominant = max(per, key=lambda k: per[k]["t"])
     dom = per[dominant]
     traffic = load_traffic()
-    gemm_flops = per.get("sp24_gemm_packed", {}).get("flops", 0)
-    gemm_t = per.get("sp24_gemm_packed", {}).get("t", 1.0)
     tensor_bound = wl["ms"][-1] >= 1024 and dominant == "sp24_gemm_packed"
     if tensor_bound:
         achieved = dom["flops"] / dom["t"] / 1e12
@@ -469,10 +528,12 @@ def run_gpu(args, wl, rank, world, local_rank):
                    "gbs": round(v["bytes"] / v["t"] / 1e9, 1),
                    "frac_hbm": round(v["bytes"] / v["t"] / 1e9 / peaks["hbm_gbs"], 4)}
                for k, v in per.items()}
-    if gemm_flops:
-        kernels["sp24_gemm_packed"]["tflops"] = round(gemm_flops / gemm_t / 1e12, 2)
+    for k, v in per.items():
+        if v["flops"]:
+            kernels[k]["tflops"] = round(v["flops"] / v["t"] / 1e12, 2)
 
     compare = gw.dense_compare() if rank == 0 and not args.no_compare else None
+    fusion = gw.fusion_compare() if rank == 0 and not args.no_compare else None
     e2e_t, h2d, d2h = gw.e2e(args.steps)
     e2e_t = max_over_ranks(e2e_t, device)
     del g_timed, g_detail, g_warm
@@ -494,7 +555,9 @@ def run_gpu(args, wl, rank, world, local_rank):
                    "step": ("weight 6:8 decomposition" if gw.is68 else
                             "weight 2:4 prune/quantise/compress")
                            + " into the tile-packed layout, then per M: activation quantise"
-                           + (" + lift" if gw.is68 else "") + " + sparse GEMM",
+                           + (" + lift" if gw.is68 else "") + " + sparse GEMM"
+                           + ("" if args.unfused else
+                              f" (one fused launch for M <= {FUSED_MAX_M})"),
                    "algorithmic_bytes_per_step": step_bytes,
                    "l2": f"inputs larger than L2: rotating pools of {gw.R_w} bf16 weight copies and "
                          f"{gw.R_g} compressed layers",
@@ -502,6 +565,7 @@ def run_gpu(args, wl, rank, world, local_rank):
         "roofline": roof,
         "kernels": kernels,
         "sparse_vs_dense": compare,
+        "fused_vs_unfused": fusion,
         "e2e": {"value": round(aggregate_gbs(step_bytes, args.steps, world, e2e_t), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": gw.step_launches() * args.steps,
@@ -606,6 +670,8 @@ def main():
     ap.add_argument("--impl", choices=["sp24", "reference"], default="sp24")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     ap.add_argument("--no-compare", action="store_true", help="skip the dense-FP8 comparison")
+    ap.add_argument("--unfused", action="store_true",
+                    help="quantise activations in their own launch at every M (no fused quantise + GEMM)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

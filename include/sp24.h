@@ -89,6 +89,8 @@ typedef struct CUstream_st *sp24_stream_t; /* identical to cudaStream_t */
 #define SP24_OP_GEMM 4
 #define SP24_OP_GEMM_DENSE 5
 #define SP24_OP_GEMM_PACKED 6
+#define SP24_OP_QUANTIZE_GEMM_PACKED 7 /* K = the columns of X */
+#define SP24_OP_LIFT_GEMM_PACKED 8     /* K = the columns of X (the GEMM runs over 3K/2) */
 
 /*
  * Weight path, 2:4.  W: bf16 [N, K].  For every row and every group of 4
@@ -218,6 +220,41 @@ int slide68_decompose_packed(const void *W, int N, int K, void *packed, float *w
 int sp24_gemm_packed(const void *Xq, const float *x_scale, const void *packed,
                      const float *w_scale, void *Y, int M, int N, int K, void *workspace,
                      size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+
+/*
+ * Per-tensor activation quantisation and the packed sparse GEMM in one
+ * launch, for small token counts (decode).  Computes exactly what
+ *   fp8_quantize_pertensor(X, M, K, Xq, x_scale, ...) followed by
+ *   sp24_gemm_packed(Xq, x_scale, packed, w_scale, Y, M, N, K, ...)
+ * computes: Xq u8 [M, K] <- E4M3(x / x_scale), x_scale <- amax|X| / 448
+ * (1.0 when amax = 0), Y bf16 [M, N]; Xq and x_scale are outputs (the codes
+ * can feed further GEMMs of the same X).  X: bf16 [M, K].  The GEMM's CTAs
+ * compute the amax of X between them, encode it, and start their tensor-core
+ * work on the codes, while the packed weights already stream in.  Workspace:
+ * sp24_workspace_size(SP24_OP_QUANTIZE_GEMM_PACKED, M, N, K, 0) (its first
+ * 256 bytes are counters, zero before the first use and after every call).
+ * Shape rules: 1 <= M <= 256, N % 128 == 0, K % 128 == 0.  Xq and Y must not
+ * alias X or each other.  SP24_STATUS_NONFINITE is set as by
+ * fp8_quantize_pertensor.
+ */
+int sp24_quantize_gemm_packed(const void *X, int M, int N, int K, const void *packed,
+                              const float *w_scale, uint8_t *Xq, float *x_scale, void *Y,
+                              void *workspace, size_t ws_bytes, int32_t *status,
+                              sp24_stream_t stream);
+
+/*
+ * The same with the SlideSparse activation lift (SlideSparse, §2
+ * "Levantamiento de Activacion"): what slide68_lift(X, M, K, Xq_lifted,
+ * x_scale, ...) followed by sp24_gemm_packed over K' = 3K/2 against 6:8
+ * weights from slide68_decompose_packed computes.  X: bf16 [M, K];
+ * Xq_lifted u8 [M, 3K/2]; packed over K'.  Workspace:
+ * sp24_workspace_size(SP24_OP_LIFT_GEMM_PACKED, M, N, K, 0).
+ * Shape rules: 1 <= M <= 256, N % 128 == 0, K % 256 == 0.
+ */
+int slide68_lift_gemm_packed(const void *X, int M, int N, int K, const void *packed,
+                             const float *w_scale, uint8_t *Xq_lifted, float *x_scale, void *Y,
+                             void *workspace, size_t ws_bytes, int32_t *status,
+                             sp24_stream_t stream);
 
 /*
  * Dense FP8 GEMM of the same kernel family (comparison baseline for the

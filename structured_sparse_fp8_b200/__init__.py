@@ -7,7 +7,9 @@ marshals pointers and the current CUDA stream, and calls into
 
 Entry points (same names as the C ABI):
     sp24_prune_compress, fp8_quantize_pertensor, slide68_decompose,
-    slide68_lift, sp24_gemm, fp8_gemm_dense
+    slide68_lift, sp24_gemm, fp8_gemm_dense, sp24_pack_weights,
+    sp24_prune_compress_packed, slide68_decompose_packed, sp24_gemm_packed,
+    sp24_quantize_gemm_packed, slide68_lift_gemm_packed
 """
 from __future__ import annotations
 
@@ -19,7 +21,7 @@ from ._lib import DTYPE_BF16, DTYPE_E4M3, Sp24Error  # noqa: F401
 __all__ = [
     "sp24_prune_compress", "fp8_quantize_pertensor", "slide68_decompose", "slide68_lift",
     "sp24_gemm", "fp8_gemm_dense", "sp24_pack_weights", "sp24_prune_compress_packed", "slide68_decompose_packed",
-    "sp24_gemm_packed",
+    "sp24_gemm_packed", "sp24_quantize_gemm_packed", "slide68_lift_gemm_packed",
     "Workspace",
     "Sp24Error", "DTYPE_E4M3", "DTYPE_BF16",
 ]
@@ -282,6 +284,49 @@ def sp24_gemm_packed(xq: torch.Tensor, x_scale, packed: torch.Tensor, w_scale, n
                               _ptr(ws), wsn, _ptr(status), _stream(xq.device))
     _lib.check(rc, "sp24_gemm_packed")
     return y
+
+
+def _quant_gemm(name, op, klift, X, packed, w_scale, n, out, xq_out, x_scale_out, status, workspace):
+    lib = _lib.load()
+    _require_cuda(X, packed, w_scale, out, xq_out, x_scale_out, status)
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise Sp24Error("X must be a 2-D bf16 tensor")
+    M, K = X.shape
+    kg = klift(K)
+    if packed.numel() != n * kg // 2 + n * kg // 8:
+        raise Sp24Error("packed weights do not match N x K")
+    y = out if out is not None else torch.empty((M, n), dtype=torch.bfloat16, device=X.device)
+    xq = xq_out if xq_out is not None else torch.empty((M, kg), dtype=torch.uint8, device=X.device)
+    if xq.numel() != M * kg or xq.dtype != torch.uint8:
+        raise Sp24Error("code output has the wrong size or dtype")
+    sx = x_scale_out if x_scale_out is not None else torch.empty((1,), dtype=torch.float32, device=X.device)
+    ws, wsn = _ws(X.device, op, M, n, K, DTYPE_E4M3, workspace)
+    rc = getattr(lib, name)(_ptr(X), M, n, K, _ptr(packed), _ptr(w_scale), _ptr(xq), _ptr(sx), _ptr(y),
+                            _ptr(ws), wsn, _ptr(status), _stream(X.device))
+    _lib.check(rc, name)
+    return y, xq, sx
+
+
+def sp24_quantize_gemm_packed(X: torch.Tensor, packed: torch.Tensor, w_scale, n: int,
+                              out: torch.Tensor | None = None, xq_out: torch.Tensor | None = None,
+                              x_scale_out: torch.Tensor | None = None,
+                              status: torch.Tensor | None = None, workspace: Workspace | None = None):
+    """Per-tensor E4M3 quantisation of X bf16 [M, K] (M <= 256) fused with the
+    packed sparse GEMM: fp8_quantize_pertensor followed by sp24_gemm_packed
+    in one launch.  Returns (Y bf16 [M, n], Xq u8 [M, K], x_scale f32 [1])."""
+    return _quant_gemm("sp24_quantize_gemm_packed", _lib.OP_QUANTIZE_GEMM_PACKED, lambda k: k, X, packed,
+                       w_scale, n, out, xq_out, x_scale_out, status, workspace)
+
+
+def slide68_lift_gemm_packed(X: torch.Tensor, packed: torch.Tensor, w_scale, n: int,
+                             out: torch.Tensor | None = None, xq_out: torch.Tensor | None = None,
+                             x_scale_out: torch.Tensor | None = None,
+                             status: torch.Tensor | None = None, workspace: Workspace | None = None):
+    """slide68_lift of X bf16 [M, K] (M <= 256) fused with the packed sparse GEMM
+    over K' = 3K/2 (weights from slide68_decompose_packed).  Returns
+    (Y bf16 [M, n], lifted codes u8 [M, K'], x_scale f32 [1])."""
+    return _quant_gemm("slide68_lift_gemm_packed", _lib.OP_LIFT_GEMM_PACKED, lambda k: 3 * k // 2, X, packed,
+                       w_scale, n, out, xq_out, x_scale_out, status, workspace)
 
 
 def fp8_gemm_dense(xq: torch.Tensor, x_scale, wq: torch.Tensor, w_scale,

@@ -24,7 +24,8 @@ SP24_STATUS_NONFINITE = 1
 SP24_STATUS_TIMEOUT = 2
 DTYPE_E4M3 = 0
 DTYPE_BF16 = 1
-OP_QUANTIZE, OP_PRUNE_COMPRESS, OP_SLIDE68_DECOMPOSE, OP_SLIDE68_LIFT, OP_GEMM, OP_GEMM_DENSE, OP_GEMM_PACKED = range(7)
+(OP_QUANTIZE, OP_PRUNE_COMPRESS, OP_SLIDE68_DECOMPOSE, OP_SLIDE68_LIFT, OP_GEMM, OP_GEMM_DENSE,
+ OP_GEMM_PACKED, OP_QUANTIZE_GEMM_PACKED, OP_LIFT_GEMM_PACKED) = range(9)
 
 _p = ctypes.c_void_p
 _i = ctypes.c_int
@@ -43,6 +44,8 @@ SIGNATURES = {
     "sp24_prune_compress_packed": (_i, [_p, _i, _i, _p, _p, _p, _sz, _p, _p]),
     "slide68_decompose_packed": (_i, [_p, _i, _i, _p, _p, _p, _sz, _p, _p]),
     "sp24_gemm_packed": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _sz, _p, _p]),
+    "sp24_quantize_gemm_packed": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _sz, _p, _p]),
+    "slide68_lift_gemm_packed": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _sz, _p, _p]),
     "sp24_workspace_size": (_sz, [_i, _i64, _i64, _i64, _i]),
     "sp24_status_str": (ctypes.c_char_p, [_i]),
     "sp24_last_cuda_error": (_i, []),

@@ -47,7 +47,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
            "-Xcompiler", "-fPIC", "-shared", "-cudart", "static",
            "-I", INCLUDE, "-I", CSRC,
            "-Xptxas", "-v" if verbose else "-O3",
-           *[os.path.join(CSRC, f) for f in SOURCES], "-o", tmp, "-lcuda" if False else "-ldl"]
+           *[os.path.join(CSRC, f) for f in SOURCES], "-o", tmp, "-ldl"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)

@@ -75,6 +75,18 @@ size_t sp24_workspace_size(int op, int64_t M, int64_t N, int64_t K, int dtype) {
     case SP24_OP_SLIDE68_DECOMPOSE:
     case SP24_OP_SLIDE68_LIFT:
       return sp24::kAmaxWorkspaceBytes;
+    case SP24_OP_QUANTIZE_GEMM_PACKED:
+    case SP24_OP_LIFT_GEMM_PACKED: {
+      // counters of the fused quantisation, then the GEMM's own workspace
+      const int64_t Kg = op == SP24_OP_LIFT_GEMM_PACKED ? K / 2 * 3 : K;
+      if (M < 1 || N < 128 || Kg < 128 || M > INT32_MAX || N > INT32_MAX || Kg > INT32_MAX) return 0;
+      int sms = device_sm_count();
+      if (sms <= 0) sms = 148;
+      return sp24::kAmaxWorkspaceBytes +
+             sp24::plan_gemm(sp24::kSparseE4M3Packed, static_cast<int>(M), static_cast<int>(N),
+                             static_cast<int>(Kg), sms)
+                 .workspace_bytes();
+    }
     case SP24_OP_GEMM:
     case SP24_OP_GEMM_PACKED:
     case SP24_OP_GEMM_DENSE: {
@@ -249,6 +261,47 @@ int sp24_gemm_packed(const void *Xq, const float *x_scale, const void *packed, c
                      sp24_stream_t stream) {
   return gemm_common(sp24::kSparseE4M3Packed, Xq, x_scale, packed, nullptr, w_scale, Y, M, N, K,
                      workspace, ws_bytes, status, stream);
+}
+
+static int quant_gemm_common(bool lift, const void *X, int M, int N, int K, const void *packed,
+                             const float *w_scale, uint8_t *Xq, float *x_scale, void *Y,
+                             void *workspace, size_t ws_bytes, int32_t *status,
+                             sp24_stream_t stream) {
+  if (!X || !packed || !Xq || !x_scale || !Y) return SP24_ERR_NULL;
+  if (M < 1 || M > 256 || N < 128 || N % 128 != 0 || K < 128 || K % (lift ? 256 : 128) != 0)
+    return SP24_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(packed) || !aligned16(Xq) || !aligned16(Y)) return SP24_ERR_ALIGN;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  const int Kg = lift ? K / 2 * 3 : K;
+  const sp24::GemmPlan pl = sp24::plan_gemm(sp24::kSparseE4M3Packed, M, N, Kg, sms);
+  if (!workspace || ws_bytes < sp24::kAmaxWorkspaceBytes + pl.workspace_bytes()) return SP24_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SP24_ERR_ALIGN;
+  sp24::GemmFusedX fx;
+  fx.x = X;
+  fx.lift = lift ? 1 : 0;
+  fx.xq = Xq;
+  fx.x_scale = x_scale;
+  fx.counters = static_cast<uint32_t *>(workspace);
+  return cuda_status(sp24::launch_gemm_quant(pl, fx, packed, w_scale, Y, M, N, Kg,
+                                             static_cast<uint8_t *>(workspace) + sp24::kAmaxWorkspaceBytes,
+                                             status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sp24_quantize_gemm_packed(const void *X, int M, int N, int K, const void *packed,
+                              const float *w_scale, uint8_t *Xq, float *x_scale, void *Y,
+                              void *workspace, size_t ws_bytes, int32_t *status,
+                              sp24_stream_t stream) {
+  return quant_gemm_common(false, X, M, N, K, packed, w_scale, Xq, x_scale, Y, workspace, ws_bytes,
+                           status, stream);
+}
+
+int slide68_lift_gemm_packed(const void *X, int M, int N, int K, const void *packed,
+                             const float *w_scale, uint8_t *Xq_lifted, float *x_scale, void *Y,
+                             void *workspace, size_t ws_bytes, int32_t *status,
+                             sp24_stream_t stream) {
+  return quant_gemm_common(true, X, M, N, K, packed, w_scale, Xq_lifted, x_scale, Y, workspace,
+                           ws_bytes, status, stream);
 }
 
 int fp8_gemm_dense(const uint8_t *Xq, const float *x_scale, const uint8_t *Wq,

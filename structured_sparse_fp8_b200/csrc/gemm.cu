@@ -29,6 +29,7 @@
 #include <mutex>
 
 #include "kernels.h"
+#include "quant_common.cuh"
 #include "sm100_ptx.cuh"
 
 namespace sp24 {
@@ -207,6 +208,15 @@ struct GemmArgs {
   uint32_t *counters;  // stream-K: [num_tiles - dp_tiles], zero between calls
   int32_t *status;
   const uint8_t *packed;  // tile-packed weights (packed kind only)
+  // Fused activation quantisation (XQ != 0): bf16 X of xvec 8-element
+  // vectors in, its E4M3 codes (lifted for XQ = 2) out to xq, which is the
+  // B operand the kernel then loads; xbar = [amax bits, arrivals, codes
+  // written, departures], zero between calls.
+  const uint16_t *x;
+  uint8_t *xq;
+  float *x_scale_out;
+  uint32_t *xbar;
+  int64_t xvec;
 };
 
 enum SegRole : int { kWhole = 0, kOwner = 1, kContrib = 2 };
@@ -258,15 +268,92 @@ __device__ __forceinline__ void red_release_add_gpu(uint32_t *p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ void red_max_relaxed_gpu(uint32_t *p, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 
+// Spin (bounded) until *p reaches `expect`; acquire semantics.
+__device__ __forceinline__ void wait_count_gpu(const uint32_t *p, uint32_t expect, int32_t *status) {
+  const uint64_t t0 = global_timer_ns();
+  uint32_t polls = 0;
+  while (ld_acquire_gpu(p) < expect) {
+    __nanosleep(32);
+    if ((++polls & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+      if (status) atomicOr(status, SP24_STATUS_TIMEOUT);
+      break;
+    }
+  }
+}
+
+// Per-tensor E4M3 quantisation of the activations fused in front of the
+// GEMM, run by the 128 epilogue threads (t = 0..127) while the producer
+// already streams weights: (1) amax of this CTA's slice of X (a contiguous
+// range of 8-element vectors), (2) a grid-wide max through xbar[0] and an
+// arrival count, (3) s = amax / 448 (1 when amax = 0) and this slice's codes
+// E4M3(RN_fp32(x / s)) written to xq (XQ = 2: the SlideSparse lift, each
+// 8-group g of a row becoming the 12 codes of windows 2j..2j+3, j = 0..2),
+// (4) a second count that the producer waits for before it loads X codes.
+// Every CTA is resident (at most one per SM, cooperative launch), so both
+// counts complete; each wait is bounded anyway.  Returns s.
+template <int XQ>
+__device__ float fused_quantize(const GemmArgs &p, int t, uint32_t *s_red, float *s_scale) {
+  const int64_t v0 = static_cast<int64_t>(blockIdx.x) * p.xvec / gridDim.x;
+  const int64_t v1 = static_cast<int64_t>(blockIdx.x + 1) * p.xvec / gridDim.x;
+  const uint4 *xv = reinterpret_cast<const uint4 *>(p.x);
+  uint32_t m2 = 0;
+  for (int64_t v = v0 + t; v < v1; v += 128) m2 = __vmaxu2(m2, absmax8x2(__ldg(xv + v)));
+  uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
+  if ((t & 31) == 0) s_red[t >> 5] = mx;
+  named_bar_sync(1, 128);
+  if (t == 0) {
+    mx = max(max(s_red[0], s_red[1]), max(s_red[2], s_red[3]));
+    red_max_relaxed_gpu(&p.xbar[0], mx);
+    red_release_add_gpu(&p.xbar[1], 1u);  // orders the max before the arrival
+    wait_count_gpu(&p.xbar[1], gridDim.x, p.status);
+    const uint32_t amax = ld_acquire_gpu(&p.xbar[0]);
+    const float sx = amax == 0u ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax), 448.0f);
+    if (blockIdx.x == 0) {
+      if (amax >= 0x7F80u && p.status) atomicOr(p.status, SP24_STATUS_NONFINITE);
+      *p.x_scale_out = sx;
+    }
+    *s_scale = sx;
+  }
+  named_bar_sync(1, 128);
+  const float sx = *s_scale;
+  for (int64_t v = v0 + t; v < v1; v += 128) {
+    const uint4 w = __ldg(xv + v);
+    const uint32_t h[4] = {w.x, w.y, w.z, w.w};
+    uint32_t c[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      c[2 * i] = e4m3_code(__fdiv_rn(bf16_bits_to_float(h[i] & 0xFFFFu), sx));
+      c[2 * i + 1] = e4m3_code(__fdiv_rn(bf16_bits_to_float(h[i] >> 16), sx));
+    }
+    if constexpr (XQ == 1) {
+      *reinterpret_cast<uint2 *>(p.xq + 8 * v) =
+          make_uint2(c[0] | c[1] << 8 | c[2] << 16 | c[3] << 24, c[4] | c[5] << 8 | c[6] << 16 | c[7] << 24);
+    } else {
+      uint32_t *o = reinterpret_cast<uint32_t *>(p.xq + 12 * v);
+      o[0] = c[0] | c[1] << 8 | c[2] << 16 | c[3] << 24;
+      o[1] = c[2] | c[3] << 8 | c[4] << 16 | c[5] << 24;
+      o[2] = c[4] | c[5] << 8 | c[6] << 16 | c[7] << 24;
+    }
+  }
+  fence_proxy_async_global();  // the codes are read back by TMA loads
+  named_bar_sync(1, 128);
+  if (t == 0) red_release_add_gpu(&p.xbar[2], 1u);
+  return sx;
+}
+
 // ------------------------------------------------------------------ kernel
 
-template <int KIND, int BN, int MT>
+template <int KIND, int BN, int MT, int XQ>
 __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
@@ -286,6 +373,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t *tmem_full = meta_ready + S;
   uint64_t *tmem_empty = tmem_full + NB;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tmem_empty + NB);
+  [[maybe_unused]] __shared__ uint32_t s_xred[4];
+  [[maybe_unused]] __shared__ float s_xscale;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -367,6 +456,11 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       grid_dependency_wait();
+      if constexpr (XQ != 0) {
+        // the activation codes are written by this grid's epilogue warps
+        wait_count_gpu(&p.xbar[2], gridDim.x, p.status);
+        fence_proxy_async_global();
+      }
       while (ok && it.next(p, sg)) {
         const int n0 = (sg.tile % p.tiles_n) * C::kRows;
         const int m0 = (sg.tile / p.tiles_n) * BN;
@@ -459,7 +553,11 @@ __global__ void __launch_bounds__(192, 1)
     const int q = warp & 3;          // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;   // W row within the tile == accumulator lane
     const int t = threadIdx.x - 64;  // 0..127
-    const float sx = p.x_scale ? __ldg(p.x_scale) : 1.0f;
+    float sx;
+    if constexpr (XQ != 0)
+      sx = fused_quantize<XQ>(p, t, s_xred, &s_xscale);
+    else
+      sx = p.x_scale ? __ldg(p.x_scale) : 1.0f;
     const float sw = p.w_scale ? __ldg(p.w_scale) : 1.0f;
     const float sc = sx * sw;
     constexpr int kW = C::kEpiCols;
@@ -679,6 +777,19 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
+  if constexpr (XQ != 0) {
+    // Every thread of this CTA is past its waits on xbar; the last CTA to
+    // get here returns the counters to zero for the next call.
+    if (threadIdx.x == 64) {
+      __threadfence();
+      if (atomicAdd(&p.xbar[3], 1u) == gridDim.x - 1) {
+        p.xbar[0] = 0u;
+        p.xbar[1] = 0u;
+        p.xbar[2] = 0u;
+        p.xbar[3] = 0u;
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -768,17 +879,18 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   return pl;
 }
 
-template <int KIND, int BN, int MT>
+template <int KIND, int BN, int MT, int XQ = 0>
 static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float *x_scale,
                                 const void *w_values, const uint8_t *w_meta, const float *w_scale,
                                 void *y, int M, int N, int K, void *workspace, int32_t *status,
-                                cudaStream_t st) {
+                                cudaStream_t st, const GemmFusedX *fx = nullptr) {
   using T = KindTraits<KIND>;
   using C = Config<KIND, BN, MT>;
+  static_assert(XQ == 0 || KIND == kSparseE4M3Packed, "fused quantisation feeds the packed E4M3 GEMM");
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN, MT>,
+    attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN, MT, XQ>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
@@ -832,6 +944,18 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
                    : nullptr;
   a.status = status;
   a.packed = T::kPacked ? static_cast<const uint8_t *>(w_values) : nullptr;
+  a.x = nullptr;
+  a.xq = nullptr;
+  a.x_scale_out = nullptr;
+  a.xbar = nullptr;
+  a.xvec = 0;
+  if constexpr (XQ != 0) {
+    a.x = static_cast<const uint16_t *>(fx->x);
+    a.xq = fx->xq;
+    a.x_scale_out = fx->x_scale;
+    a.xbar = fx->counters;
+    a.xvec = static_cast<int64_t>(M) * (XQ == 2 ? K / 3 * 2 : K) / 8;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(pl.grid), 1, 1);
   cfg.blockDim = dim3(192, 1, 1);
@@ -841,12 +965,16 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   // for contributor CTAs; with at most one CTA per SM every CTA becomes
   // resident once the SMs still held by the previous kernel drain, and each
   // wait is bounded anyway.
-  cudaLaunchAttribute attrs[1];
+  // The fused quantisation's grid-wide counts need every CTA resident at
+  // once: a cooperative launch, which the driver refuses otherwise.
+  cudaLaunchAttribute attrs[2];
   attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  attrs[1].id = cudaLaunchAttributeCooperative;
+  attrs[1].val.cooperative = 1;
   cfg.attrs = attrs;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, MT>, tmA, tmB, tmE, tmY, a);
+  cfg.numAttrs = XQ != 0 ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, MT, XQ>, tmA, tmB, tmE, tmY, a);
 }
 
 template <int KIND>
@@ -868,6 +996,28 @@ static cudaError_t launch_kind(const GemmPlan &pl, const void *xq, const float *
     case 256: return launch_typed<KIND, 256, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+template <int XQ>
+static cudaError_t launch_quant_bn(const GemmPlan &pl, const GemmFusedX &fx, const void *packed,
+                                   const float *w_scale, void *y, int M, int N, int K, void *ws,
+                                   int32_t *status, cudaStream_t st) {
+  constexpr int P = kSparseE4M3Packed;
+  switch (pl.bn) {
+    case 16: return launch_typed<P, 16, 1, XQ>(pl, fx.xq, nullptr, packed, nullptr, w_scale, y, M, N, K, ws, status, st, &fx);
+    case 32: return launch_typed<P, 32, 1, XQ>(pl, fx.xq, nullptr, packed, nullptr, w_scale, y, M, N, K, ws, status, st, &fx);
+    case 64: return launch_typed<P, 64, 1, XQ>(pl, fx.xq, nullptr, packed, nullptr, w_scale, y, M, N, K, ws, status, st, &fx);
+    case 128: return launch_typed<P, 128, 1, XQ>(pl, fx.xq, nullptr, packed, nullptr, w_scale, y, M, N, K, ws, status, st, &fx);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_gemm_quant(const GemmPlan &pl, const GemmFusedX &fx, const void *packed,
+                              const float *w_scale, void *y, int M, int N, int K, void *workspace,
+                              int32_t *status, cudaStream_t st) {
+  if (pl.mt != 1) return cudaErrorInvalidValue;
+  return fx.lift ? launch_quant_bn<2>(pl, fx, packed, w_scale, y, M, N, K, workspace, status, st)
+                 : launch_quant_bn<1>(pl, fx, packed, w_scale, y, M, N, K, workspace, status, st);
 }
 
 cudaError_t launch_gemm(GemmKind kind, const GemmPlan &pl, const void *xq, const float *x_scale,

@@ -92,4 +92,18 @@ cudaError_t launch_gemm(GemmKind kind, const GemmPlan &plan, const void *xq, con
                         void *y, int M, int N, int K, void *workspace, int32_t *status,
                         cudaStream_t st);
 
+// The packed E4M3 GEMM with the per-tensor quantisation of its activations
+// fused in front (plan from plan_gemm(kSparseE4M3Packed, M, N, K); bn <= 128,
+// mt == 1).  K is the GEMM's K: the columns of X, or 3/2 of them with lift.
+struct GemmFusedX {
+  const void *x;       // bf16 [M, Kx]
+  int lift;            // 0: codes [M, Kx]; 1: SlideSparse lift, codes [M, 3 Kx / 2]
+  uint8_t *xq;         // out: the E4M3 codes (the GEMM's B operand)
+  float *x_scale;      // out: amax|X| / 448 (1 when amax = 0)
+  uint32_t *counters;  // 4 words, zero before the call and after it
+};
+cudaError_t launch_gemm_quant(const GemmPlan &plan, const GemmFusedX &fx, const void *packed,
+                              const float *w_scale, void *y, int M, int N, int K, void *workspace,
+                              int32_t *status, cudaStream_t st);
+
 }  // namespace sp24

@@ -78,6 +78,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// The same between generic-proxy global-memory accesses and async-proxy ones
+// (a TMA load of data that generic stores wrote, here or in another CTA).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 // 2-D tiled bulk tensor load global -> shared, completion counted on `bar`.
 // x is the innermost coordinate (in elements of the map); callers keep

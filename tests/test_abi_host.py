@@ -56,6 +56,14 @@ def test_workspace_sizes(lib):
     # tiny: 2 tiles x 2 k-blocks -> 2 CTAs with one whole tile each
     assert lib.sp24_workspace_size(_lib.OP_GEMM, 16, 256, 256, 0) == 0
     assert lib.sp24_workspace_size(_lib.OP_GEMM, 0, 11008, 4096, 0) == 0
+    # fused quantise (or lift) + GEMM: 256 bytes of counters, then the GEMM's
+    # workspace at K (or K' = 3K/2)
+    for m in (1, 8, 32, 64, 256):
+        assert (lib.sp24_workspace_size(_lib.OP_QUANTIZE_GEMM_PACKED, m, 11008, 4096, 0)
+                == 256 + lib.sp24_workspace_size(_lib.OP_GEMM_PACKED, m, 11008, 4096, 0))
+        assert (lib.sp24_workspace_size(_lib.OP_LIFT_GEMM_PACKED, m, 4096, 4096, 0)
+                == 256 + lib.sp24_workspace_size(_lib.OP_GEMM_PACKED, m, 4096, 6144, 0))
+    assert lib.sp24_workspace_size(_lib.OP_QUANTIZE_GEMM_PACKED, 16, 256, 256, 0) == 256
 
 
 FAKE = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: calls fail validation first
@@ -84,8 +92,21 @@ def test_validation_rejects_bad_arguments_without_a_gpu(lib):
     assert lib.sp24_prune_compress_packed(FAKE, 128, 128, FAKE, None, FAKE, ws, None, None) == _lib.SP24_ERR_NULL
     assert lib.slide68_decompose_packed(FAKE, 128, 128, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
     assert lib.slide68_decompose_packed(FAKE, 96, 256, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    # fused quantise + GEMM: M in [1, 256], N % 128, K % 128 (K % 256 with the lift)
+    big = 1 << 30
+    qg = lib.sp24_quantize_gemm_packed
+    lg = lib.slide68_lift_gemm_packed
+    assert qg(FAKE, 0, 128, 128, FAKE, None, FAKE, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_SHAPE
+    assert qg(FAKE, 257, 128, 128, FAKE, None, FAKE, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_SHAPE
+    assert qg(FAKE, 4, 192, 128, FAKE, None, FAKE, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_SHAPE
+    assert qg(FAKE, 4, 128, 192, FAKE, None, FAKE, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_SHAPE
+    assert lg(FAKE, 4, 128, 128, FAKE, None, FAKE, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_SHAPE
+    assert qg(FAKE, 4, 128, 128, FAKE, None, None, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_NULL
+    assert qg(FAKE, 4, 128, 128, FAKE, None, FAKE, None, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_NULL
+    assert lg(None, 4, 128, 256, FAKE, None, FAKE, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_NULL
     # alignment
     odd = ctypes.c_void_p((1 << 20) + 8)
+    assert qg(FAKE, 4, 128, 128, FAKE, None, odd, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.sp24_prune_compress_packed(FAKE, 128, 128, odd, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.fp8_quantize_pertensor(odd, 4, 32, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.sp24_gemm(FAKE, None, odd, FAKE, None, FAKE, 4, 128, 128, 0, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN

@@ -505,3 +505,109 @@ def test_packed_gemm_decode_workload(m):
     y = sp().sp24_gemm_packed(xq, sx, packed, c["scale"], 11008)
     y_ref, b = _ref(host(xq), host(sx)[0], host(c["values"]), host(c["meta"]), host(c["scale"])[0], 4096)
     assert_gemm_close(y, y_ref, b, f"packed decode M={m}")
+
+
+# ------------------------------------------------------------ fused quantise + GEMM
+
+def _fused_weights(w, lift):
+    st = new_status()
+    if lift:
+        packed, sw = sp().slide68_decompose_packed(dev_bf16(w), status=st)
+        ref_w = O.slide68_decompose(w, "e4m3")
+        wv = O.e4m3_decode(ref_w["expanded"])
+    else:
+        packed, sw = sp().sp24_prune_compress_packed(dev_bf16(w), status=st)
+        ref_w = O.sp24_prune_compress(w, "e4m3")
+        wv = O.e4m3_decode(ref_w["pruned_dense"])
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0 and host(sw)[0] == ref_w["scale"]
+    return packed, sw, wv, ref_w["scale"]
+
+
+def _fused_check(x, wts, n, what, lift=False):
+    """The fused launch against the oracle: codes and scale bit-exact, Y within
+    tolerance, and Y identical to the two-launch path on the same codes."""
+    packed, sw, wv, ref_sw = wts
+    st = new_status()
+    if lift:
+        y, xq, sx = sp().slide68_lift_gemm_packed(dev_bf16(x), packed, sw, n, status=st)
+        ref_q, ref_s = O.slide68_lift(x)
+    else:
+        y, xq, sx = sp().sp24_quantize_gemm_packed(dev_bf16(x), packed, sw, n, status=st)
+        ref_q, ref_s = O.quantize_pertensor(x)
+    y2 = sp().sp24_gemm_packed(xq, sx, packed, sw, n, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, what
+    assert host(sx)[0] == ref_s, what
+    assert np.array_equal(host(xq), ref_q), what
+    y_ref, b = O.gemm_ref(O.e4m3_decode(ref_q), wv, ref_s, ref_sw)
+    assert_gemm_close(y, y_ref, b, what)
+    assert torch.equal(y, y2), what
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 128, 128), (7, 256, 384), (16, 256, 256), (33, 384, 1024),
+                                   (64, 128, 640), (100, 256, 512), (256, 384, 1152)])
+def test_quantize_gemm_packed_small(m, n, k):
+    x = WL.random_bits((m, k), 1000 + m)
+    w = WL.random_bits((n, k), 1100 + n, scale=0.02)
+    _fused_check(x, _fused_weights(w, False), n, f"fused {m}x{n}x{k}")
+
+
+def test_quantize_gemm_packed_decode_workload():
+    wts = _fused_weights(WL.weight_bits(2), False)
+    for m in (1, 8, 32, 64):
+        _fused_check(WL.activation_bits(2, m), wts, 11008, f"fused decode M={m}")
+
+
+def test_quantize_gemm_packed_down_proj_workload():
+    _fused_check(WL.activation_bits(4, 256), _fused_weights(WL.weight_bits(4), False), 4096,
+                 "fused down-proj M=256")
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 128, 256), (17, 256, 512), (64, 384, 768), (200, 128, 1024)])
+def test_lift_gemm_packed_small(m, n, k):
+    x = WL.random_bits((m, k), 1200 + m)
+    w = WL.random_bits((n, k), 1300 + n, scale=0.02)
+    _fused_check(x, _fused_weights(w, True), n, f"fused lift {m}x{n}x{k}", lift=True)
+
+
+def test_lift_gemm_packed_slide68_workload():
+    wts = _fused_weights(WL.weight_bits(5), True)
+    for m in (1, 64):
+        _fused_check(WL.activation_bits(5, m), wts, 4096, f"fused 6:8 M={m}", lift=True)
+
+
+def test_quantize_gemm_packed_zero_and_nonfinite_inputs():
+    w = WL.random_bits((256, 512), 1400, scale=0.02)
+    packed, sw = sp().sp24_prune_compress_packed(dev_bf16(w))
+    st = new_status()
+    y, xq, sx = sp().sp24_quantize_gemm_packed(dev_bf16(np.zeros((5, 512), np.uint16)), packed, sw, 256,
+                                                status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0 and host(sx)[0] == 1.0
+    assert (host(xq) == 0).all() and (host(y) == 0).all()
+    x = WL.random_bits((5, 512), 1401)
+    x[3, 100] = 0x7F80                       # +Inf
+    st = new_status()
+    sp().sp24_quantize_gemm_packed(dev_bf16(x), packed, sw, 256, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & 1
+
+
+def test_quantize_gemm_packed_reuses_its_workspace():
+    """Back-to-back fused calls of different shapes on one workspace: every
+    call must leave its counters at zero for the next one."""
+    ws = sp().Workspace(DEV)
+    w = WL.random_bits((384, 1024), 1500, scale=0.02)
+    packed, sw = sp().sp24_prune_compress_packed(dev_bf16(w))
+    outs = []
+    for rep in range(2):
+        for m in (1, 40, 256):
+            x = WL.random_bits((m, 1024), 1600 + m)
+            y, xq, sx = sp().sp24_quantize_gemm_packed(dev_bf16(x), packed, sw, 384, workspace=ws)
+            y2 = sp().sp24_gemm_packed(xq, sx, packed, sw, 384, workspace=ws)
+            outs.append((host(y), host(y2)))
+    torch.cuda.synchronize()
+    assert (ws.buf[:256] == 0).all()
+    for (a, b), (c, d) in zip(outs[:3], outs[3:]):
+        assert np.array_equal(a, b) and np.array_equal(a, c) and np.array_equal(c, d)

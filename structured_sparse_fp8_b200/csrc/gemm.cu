@@ -3,7 +3,7 @@
 // W is the A operand of the MMA (128 rows per CTA, 2:4-compressed for the
 // sparse kinds), the activations X are the B operand (BN tokens per CTA), so
 // the fp32 accumulator tile lives in tensor memory as 128 lanes (W rows) x BN
-// columns (tokens).  One CTA = 6 warps:
+// columns (tokens).  One CTA = 6 warps (10 for two-row-tile tiles):
 //   warp 0      TMA producer: W values, X tile and 2:4 metadata for each
 //               K-stage into a ring of shared-memory stages (mbarrier
 //               full/empty pairs);
@@ -11,7 +11,7 @@
 //               into TMEM (tcgen05.cp) and issues the tcgen05.mma(.sp)
 //               instructions, releasing each stage with tcgen05.commit;
 //   warps 2-5   epilogue: tcgen05.ld the accumulator, apply x_scale * w_scale,
-//               round to bf16 and store Y (stream-K: see GemmArgs).
+//   (2-9)       round to bf16 and store Y (stream-K: see GemmArgs).
 // The kernel is persistent: one CTA per SM walks a list of (tile, k-range)
 // segments; two TMEM accumulators (when they fit) let the epilogue of one
 // segment overlap the main loop of the next.
@@ -150,7 +150,14 @@ struct Config {
   // footprint to half an SM, so that the next kernel's CTAs can already be
   // resident, and streaming weights, while this kernel drains; large tiles
   // take the whole SM for a deep ring.
-  static constexpr uint32_t kSmemBudget = BN <= 64 ? 108 * 1024 : 214 * 1024;
+  // Epilogue warps: two per TMEM lane quarter for two-row-tile tiles (one
+  // per row tile), whose single accumulator leaves the epilogue exposed
+  // between main loops; one per quarter otherwise.
+  static constexpr int kEpiWarps = MT == 2 ? 8 : 4;
+  static constexpr int kEpiThreads = 32 * kEpiWarps;
+  static constexpr int kThreads = 64 + kEpiThreads;
+  static constexpr int kRtPerWarp = MT * 4 / kEpiWarps;  // row tiles each epilogue warp drains
+  static constexpr uint32_t kSmemBudget = BN <= 64 ? 108 * 1024 : (kEpiWarps == 8 ? 224 * 1024 : 214 * 1024);
   // Wide token tiles write Y through shared memory: each epilogue warp
   // stages its 32 rows x 32 tokens of a pass (2 KB of bf16) in one of two
   // buffers of its own and stores them with a 2-D bulk tensor copy, so the
@@ -159,7 +166,7 @@ struct Config {
   // stores and the deeper ring.
   static constexpr bool kTmaStoreY = BN >= 128;
   static constexpr uint32_t kStageY = 32 * 32 * 2;          // one warp's pass
-  static constexpr uint32_t kYBytes = kTmaStoreY ? 4 * 2 * kStageY : 0;
+  static constexpr uint32_t kYBytes = kTmaStoreY ? kEpiWarps * 2 * kStageY : 0;
   static constexpr int kStagesRaw = static_cast<int>((kSmemBudget - kYBytes) / kStageBytes);
   static constexpr int kStages = kStagesRaw > 16 ? 16 : kStagesRaw;
   static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kYBytes + 1024 /*align*/ + 1024 /*bars*/;
@@ -354,7 +361,7 @@ __device__ float fused_quantize(const GemmArgs &p, int t, uint32_t *s_red, float
 // ------------------------------------------------------------------ kernel
 
 template <int KIND, int BN, int MT, int XQ>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Config<KIND, BN, MT>::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
                 const GemmArgs p) {
@@ -392,7 +399,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < NB; ++b) {
       mbar_init(&tmem_full[b], 1);
-      mbar_init(&tmem_empty[b], 128);
+      mbar_init(&tmem_empty[b], C::kEpiThreads);
     }
     fence_mbar_init();
   }
@@ -550,9 +557,12 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------ epilogue warps
+    static_assert(XQ == 0 || C::kEpiWarps == 4, "the fused quantisation runs on four epilogue warps");
+    const int e = warp - 2;          // epilogue warp index
     const int q = warp & 3;          // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;   // W row within the tile == accumulator lane
-    const int t = threadIdx.x - 64;  // 0..127
+    const int t = threadIdx.x - 64;  // 0 .. kEpiThreads - 1
+    const int rt0 = (e >> 2) * C::kRtPerWarp;  // first row tile this warp drains
     float sx;
     if constexpr (XQ != 0)
       sx = fused_quantize<XQ>(p, t, s_xred, &s_xscale);
@@ -610,7 +620,7 @@ __global__ void __launch_bounds__(192, 1)
       if (sg.role == kContrib) {
         // leave the fp32 partial tile (valid token columns) for the owner
 #pragma unroll 1
-        for (int rt = 0; rt < MT; ++rt) {
+        for (int rt = rt0; rt < rt0 + C::kRtPerWarp; ++rt) {
 #pragma unroll 1
           for (int c = 0; c < mvalid; c += 16) {
             uint32_t v[16];
@@ -628,7 +638,7 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive(&tmem_empty[b]);
         // The barrier orders every thread's partial stores before thread 0's
         // release increment (release is cumulative), which the owner acquires.
-        named_bar_sync(1, 128);
+        named_bar_sync(1, C::kEpiThreads);
         if (t == 0) red_release_add_gpu(&p.counters[sg.tile - p.dp_tiles], 1u);
       } else {
         int first = 0, last = -1;  // contributor CTAs of an owned tile
@@ -649,10 +659,10 @@ __global__ void __launch_bounds__(192, 1)
             }
             p.counters[sg.tile - p.dp_tiles] = 0u;  // leave the workspace counters at zero
           }
-          named_bar_sync(1, 128);  // the acquire by thread 0 covers the whole CTA's reads
+          named_bar_sync(1, C::kEpiThreads);  // the acquire by thread 0 covers the whole CTA's reads
         }
 #pragma unroll 1
-        for (int rt = 0; rt < MT; ++rt) {
+        for (int rt = rt0; rt < rt0 + C::kRtPerWarp; ++rt) {
           const int n = n0 + rt * 128 + row;
           const uint32_t t_row = t_acc + rt * BN;
           // kW token columns per pass.  The first contributor's partial for
@@ -668,7 +678,7 @@ __global__ void __launch_bounds__(192, 1)
           // warp's stores; before a buffer is rewritten it waits until the
           // store issued from it two passes ago has read it.
           auto store_pass = [&](int c, auto &&value_of) {
-            uint16_t *buf = reinterpret_cast<uint16_t *>(ystage + (q * 2 + (ypass & 1)) * C::kStageY);
+            uint16_t *buf = reinterpret_cast<uint16_t *>(ystage + (e * 2 + (ypass & 1)) * C::kStageY);
             if (lane == 0) bulk_wait_group_read<1>();
             __syncwarp();
 #pragma unroll
@@ -958,7 +968,7 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(pl.grid), 1, 1);
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = st;
   // Programmatic dependent launch (see the kernel).  Stream-K owners wait

@@ -521,10 +521,17 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT>::kThreads, 1)
           const uint32_t b_addr = st_addr + C::kBOff;
           if (T::kSparse) {
             // 128 rows x 16 B, rows contiguous: core matrices of 8 rows are 128 B apart.
+            if constexpr (MT == 2 && T::kPacked) {
+              // both row tiles' metadata in one copy: the second 16-byte
+              // column is the next packed block's metadata
+              tmem_copy_128x256b(e_tmem, smem_desc(st_addr + C::e_off(0), C::e_off(1) - C::e_off(0), 128,
+                                                   kSwizzleNone));
+            } else {
 #pragma unroll
-            for (int rt = 0; rt < MT; ++rt) {
-              const uint32_t e_addr = st_addr + C::e_off(rt) + (T::kMetaTransform ? C::kEBytes : 0);
-              tmem_copy_128x128b(e_tmem + 4 * rt, smem_desc(e_addr, 2048, 128, kSwizzleNone));
+              for (int rt = 0; rt < MT; ++rt) {
+                const uint32_t e_addr = st_addr + C::e_off(rt) + (T::kMetaTransform ? C::kEBytes : 0);
+                tmem_copy_128x128b(e_tmem + 4 * rt, smem_desc(e_addr, 2048, 128, kSwizzleNone));
+              }
             }
           }
 #pragma unroll

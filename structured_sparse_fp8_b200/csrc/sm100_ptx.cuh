@@ -265,6 +265,14 @@ __device__ __forceinline__ void tmem_copy_128x128b(uint32_t taddr, uint64_t sdes
   asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+// Copy 128 rows x 32 bytes (two 16-byte core-matrix columns, the second at
+// the descriptor's leading-dimension byte offset) into TMEM lanes 0..127,
+// 8 columns starting at taddr: the first 16 bytes of each row to columns
+// 0..3, the second to columns 4..7.
+__device__ __forceinline__ void tmem_copy_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // ---------------------------------------------------------------- TMEM -> registers
 // 32 lanes x 32 bit, 16 consecutive columns: thread t of the warp receives
 // lane (warp%4)*32 + t, columns [taddr.col, taddr.col + 16).

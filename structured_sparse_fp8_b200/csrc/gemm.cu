@@ -123,28 +123,37 @@ struct KindTraits<kSparseBF16> {
 // the MMAs of both row tiles against the same activation tile: the same
 // activation bytes feed twice the tensor work, which is what bounds large
 // token tiles (operand ingest into shared memory, not the tensor pipe).
-template <int KIND, int BN, int MT = 1>
+//
+// KB = 128-K blocks per pipeline stage (1 or 2).  Decode-sized tiles do
+// little tensor work per stage, so the fixed cost of a stage (barrier wait,
+// metadata copy, commit, each issued by one thread) bounds their main loop;
+// two blocks per stage halve it.  Packed weights only: the stage's two
+// blocks of a row tile are adjacent in memory (one bulk copy) and their
+// metadata is one 128x256b copy.
+template <int KIND, int BN, int MT = 1, int KB = 1>
 struct Config {
   using T = KindTraits<KIND>;
+  static_assert(KB == 1 || (KB == 2 && T::kPacked && MT == 1), "two-block stages are for packed, one-row-tile tiles");
   static constexpr int kRows = 128 * MT;
-  static constexpr uint32_t kWTile = T::kPacked ? kPackedBlockBytes : 0;  // packed: one block per row tile
-  static constexpr uint32_t kABytes = kRows * T::kARowBytes;
-  static constexpr uint32_t kBBytes = BN * T::kBRowBytes;
-  static constexpr uint32_t kEBytes = kRows * T::kERowBytes;
+  static constexpr uint32_t kABytes = kRows * T::kARowBytes * KB;
+  static constexpr uint32_t kBBytes = BN * T::kBRowBytes * KB;
+  static constexpr uint32_t kEBytes = kRows * T::kERowBytes * KB;
   static constexpr uint32_t kTBytes = T::kMetaTransform ? 128 * 16 : 0;  // TMEM-ready metadata
   static constexpr uint32_t kTmaBytes = kABytes + kBBytes + kEBytes;
   static constexpr uint32_t kStageBytes = kTmaBytes + kTBytes;
-  static constexpr int kBSub = T::kBRowBytes / 128;  // 128-byte X boxes per stage
+  static constexpr int kBSub = T::kBRowBytes * KB / 128;  // 128-byte X boxes per stage
+  static constexpr int kMmas = T::kMmas * KB;             // MMAs per row tile per stage
   // Stage layout: [A][B][E][T] (tensor-mapped weights; A and E hold all kRows
-  // rows, row tile i at 128 i rows) or [A0 E0][A1 E1][B] (packed: each row
-  // tile's values and metadata arrive together in one bulk copy).
-  static constexpr uint32_t kBOff = T::kPacked ? MT * kPackedBlockBytes : kABytes;
+  // rows, row tile i at 128 i rows) or [A0 E0 (A0' E0')][A1 E1][B] (packed:
+  // each row tile's values and metadata arrive together in one bulk copy,
+  // the KB blocks of a row tile back to back).
+  static constexpr uint32_t kBOff = T::kPacked ? MT * KB * kPackedBlockBytes : kABytes;
   static constexpr uint32_t kEOff = T::kPacked ? 128 * T::kARowBytes : kABytes + kBBytes;
   __host__ __device__ static constexpr uint32_t a_off(int i) {
-    return T::kPacked ? i * kPackedBlockBytes : i * 128 * T::kARowBytes;
+    return T::kPacked ? i * KB * kPackedBlockBytes : i * 128 * T::kARowBytes;
   }
   __host__ __device__ static constexpr uint32_t e_off(int i) {
-    return T::kPacked ? i * kPackedBlockBytes + 128 * T::kARowBytes : kEOff + i * 128 * T::kERowBytes;
+    return T::kPacked ? i * KB * kPackedBlockBytes + 128 * T::kARowBytes : kEOff + i * 128 * T::kERowBytes;
   }
   // Persistent CTAs.  Small token tiles (decode shapes, stream-K) keep the
   // footprint to half an SM, so that the next kernel's CTAs can already be
@@ -173,7 +182,7 @@ struct Config {
   // Accumulators: MT x BN columns each; two of them (the epilogue of one
   // output tile overlaps the main loop of the next) whenever they fit in the
   // 512 TMEM columns next to the 4 metadata columns per row tile.
-  static constexpr uint32_t kMetaCols = T::kSparse ? 4 * MT : 0;
+  static constexpr uint32_t kMetaCols = T::kSparse ? 4 * MT * KB : 0;
   static constexpr int kAccBufs = (2 * MT * BN + kMetaCols <= 512) ? 2 : 1;
   static constexpr uint32_t kAccCols = MT * BN;
   static constexpr uint32_t kTmemNeed = kAccBufs * kAccCols + kMetaCols;
@@ -360,13 +369,13 @@ __device__ float fused_quantize(const GemmArgs &p, int t, uint32_t *s_red, float
 
 // ------------------------------------------------------------------ kernel
 
-template <int KIND, int BN, int MT, int XQ>
-__global__ void __launch_bounds__(Config<KIND, BN, MT>::kThreads, 1)
+template <int KIND, int BN, int MT, int XQ, int KB>
+__global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
                 const GemmArgs p) {
   using T = KindTraits<KIND>;
-  using C = Config<KIND, BN, MT>;
+  using C = Config<KIND, BN, MT, KB>;
   constexpr int S = C::kStages;
   constexpr int NB = C::kAccBufs;
 
@@ -433,8 +442,8 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT>::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < MT; ++i) {
             const uint8_t *blk = p.packed +
-                                 (static_cast<int64_t>(n0 / 128 + i) * p.num_kb + kb) * kPackedBlockBytes;
-            bulk_load_g2s(st + C::a_off(i), blk, kPackedBlockBytes, bar, stream_w);
+                                 ((static_cast<int64_t>(n0 / 128 + i) * p.num_kb + kb) * KB) * kPackedBlockBytes;
+            bulk_load_g2s(st + C::a_off(i), blk, KB * kPackedBlockBytes, bar, stream_w);
           }
         } else {
           tma_load_2d(st, &tmA, bar, kb * (T::kARowBytes / T::kAElemBytes), n0, stream_w);
@@ -486,7 +495,7 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT>::kThreads, 1)
 #pragma unroll
           for (int sub = 0; sub < C::kBSub; ++sub)
             tma_load_2d(st + C::kBOff + sub * BN * 128, &tmB, &full[s],
-                        kb * (T::kBRowBytes / T::kBElemBytes) + sub * T::kBBoxElems, m0, keep_x);
+                        kb * (T::kBRowBytes * KB / T::kBElemBytes) + sub * T::kBBoxElems, m0, keep_x);
         }
       }
     }
@@ -521,11 +530,11 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT>::kThreads, 1)
           const uint32_t b_addr = st_addr + C::kBOff;
           if (T::kSparse) {
             // 128 rows x 16 B, rows contiguous: core matrices of 8 rows are 128 B apart.
-            if constexpr (MT == 2 && T::kPacked) {
-              // both row tiles' metadata in one copy: the second 16-byte
-              // column is the next packed block's metadata
-              tmem_copy_128x256b(e_tmem, smem_desc(st_addr + C::e_off(0), C::e_off(1) - C::e_off(0), 128,
-                                                   kSwizzleNone));
+            if constexpr (T::kPacked && MT * KB == 2) {
+              // two packed blocks' metadata in one copy (both row tiles, or
+              // both k-blocks of one row tile): the second 16-byte column is
+              // the next block's metadata, 10240 bytes on
+              tmem_copy_128x256b(e_tmem, smem_desc(st_addr + C::e_off(0), kPackedBlockBytes, 128, kSwizzleNone));
             } else {
 #pragma unroll
               for (int rt = 0; rt < MT; ++rt) {
@@ -538,8 +547,12 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT>::kThreads, 1)
           for (int rt = 0; rt < MT; ++rt) {
             const uint32_t a_addr = st_addr + C::a_off(rt);
 #pragma unroll
-            for (int kk = 0; kk < T::kMmas; ++kk) {
-              const uint64_t ad = smem_desc(a_addr + kk * T::kAStep, 16, T::kASbo, T::kASwizzle);
+            for (int kk = 0; kk < C::kMmas; ++kk) {
+              // MMA kk reads block kk / kMmas of the stage (packed blocks are
+              // 10240 bytes apart), step kk % kMmas within it
+              const uint32_t a_k = KB == 1 ? kk * T::kAStep
+                                           : (kk / T::kMmas) * kPackedBlockBytes + (kk % T::kMmas) * T::kAStep;
+              const uint64_t ad = smem_desc(a_addr + a_k, 16, T::kASbo, T::kASwizzle);
               const uint32_t boff = (kk * T::kBStep / 128) * (BN * 128) + (kk * T::kBStep) % 128;
               const uint64_t bd = smem_desc(b_addr + boff, 16, 8 * 128, kSwizzle128B);
               const uint32_t acc = (kb > sg.kb0 || kk > 0) ? 1u : 0u;
@@ -863,7 +876,9 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   // Large token tiles (224 tokens: many tiles, bound by operand ingest) pair
   // two 128-row W tiles on one activation tile when N allows it.
   pl.mt = (pl.bn == 224 && kind != kSparseBF16 && N % 256 == 0) ? 2 : 1;
-  pl.bk = 128;
+  // Decode-sized tiles over packed weights take two 128-K blocks per stage.
+  pl.kb = (kind == kSparseE4M3Packed && pl.bn <= 64 && pl.mt == 1 && K % 256 == 0) ? 2 : 1;
+  pl.bk = 128 * pl.kb;
   pl.tiles_n = N / (128 * pl.mt);
   pl.tiles_m = (M + pl.bn - 1) / pl.bn;
   pl.num_kb = K / pl.bk;
@@ -896,18 +911,18 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   return pl;
 }
 
-template <int KIND, int BN, int MT, int XQ = 0>
+template <int KIND, int BN, int MT, int XQ = 0, int KB = 1>
 static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float *x_scale,
                                 const void *w_values, const uint8_t *w_meta, const float *w_scale,
                                 void *y, int M, int N, int K, void *workspace, int32_t *status,
                                 cudaStream_t st, const GemmFusedX *fx = nullptr) {
   using T = KindTraits<KIND>;
-  using C = Config<KIND, BN, MT>;
+  using C = Config<KIND, BN, MT, KB>;
   static_assert(XQ == 0 || KIND == kSparseE4M3Packed, "fused quantisation feeds the packed E4M3 GEMM");
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN, MT, XQ>,
+    attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN, MT, XQ, KB>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
@@ -991,7 +1006,7 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   attrs[1].val.cooperative = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = XQ != 0 ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, MT, XQ>, tmA, tmB, tmE, tmY, a);
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, MT, XQ, KB>, tmA, tmB, tmE, tmY, a);
 }
 
 template <int KIND>
@@ -999,6 +1014,16 @@ static cudaError_t launch_kind(const GemmPlan &pl, const void *xq, const float *
                                const void *w_values, const uint8_t *w_meta, const float *w_scale,
                                void *y, int M, int N, int K, void *ws, int32_t *status,
                                cudaStream_t st) {
+  if constexpr (KIND == kSparseE4M3Packed) {
+    if (pl.kb == 2) {
+      switch (pl.bn) {
+        case 16: return launch_typed<KIND, 16, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+        case 32: return launch_typed<KIND, 32, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+        case 64: return launch_typed<KIND, 64, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+        default: return cudaErrorInvalidValue;
+      }
+    }
+  }
   switch (pl.bn) {
     case 16: return launch_typed<KIND, 16, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
     case 32: return launch_typed<KIND, 32, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
@@ -1020,6 +1045,14 @@ static cudaError_t launch_quant_bn(const GemmPlan &pl, const GemmFusedX &fx, con
                                    const float *w_scale, void *y, int M, int N, int K, void *ws,
                                    int32_t *status, cudaStream_t st) {
   constexpr int P = kSparseE4M3Packed;
+  if (pl.kb == 2) {
+    switch (pl.bn) {
+      case 16: return launch_typed<P, 16, 1, XQ, 2>(pl, fx.xq, nullptr, packed, nullptr, w_scale, y, M, N, K, ws, status, st, &fx);
+      case 32: return launch_typed<P, 32, 1, XQ, 2>(pl, fx.xq, nullptr, packed, nullptr, w_scale, y, M, N, K, ws, status, st, &fx);
+      case 64: return launch_typed<P, 64, 1, XQ, 2>(pl, fx.xq, nullptr, packed, nullptr, w_scale, y, M, N, K, ws, status, st, &fx);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (pl.bn) {
     case 16: return launch_typed<P, 16, 1, XQ>(pl, fx.xq, nullptr, packed, nullptr, w_scale, y, M, N, K, ws, status, st, &fx);
     case 32: return launch_typed<P, 32, 1, XQ>(pl, fx.xq, nullptr, packed, nullptr, w_scale, y, M, N, K, ws, status, st, &fx);

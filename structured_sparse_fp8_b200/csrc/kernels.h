@@ -67,7 +67,8 @@ constexpr size_t kGemmCounterBytes = 16384;  // tile counters: a fixed workspace
 struct GemmPlan {
   int bn;            // tokens per tile (MMA N)
   int mt;            // 128-row W tiles per CTA tile (1 or 2)
-  int bk;            // logical K per pipeline stage
+  int kb;            // 128-K blocks per pipeline stage (1 or 2)
+  int bk;            // logical K per pipeline stage (128 kb)
   int tiles_n;       // N / (128 mt)
   int tiles_m;       // ceil(M / bn)
   int num_kb;        // K / bk

@@ -309,30 +309,69 @@ __device__ __forceinline__ void wait_count_gpu(const uint32_t *p, uint32_t expec
 
 // Per-tensor E4M3 quantisation of the activations fused in front of the
 // GEMM, run by the 128 epilogue threads (t = 0..127) while the producer
-// already streams weights: (1) amax of this CTA's slice of X (a contiguous
-// range of 8-element vectors), (2) a grid-wide max through xbar[0] and an
-// arrival count, (3) s = amax / 448 (1 when amax = 0) and this slice's codes
-// E4M3(RN_fp32(x / s)) written to xq (XQ = 2: the SlideSparse lift, each
-// 8-group g of a row becoming the 12 codes of windows 2j..2j+3, j = 0..2),
-// (4) a second count that the producer waits for before it loads X codes.
-// Every CTA is resident (at most one per SM, cooperative launch), so both
-// counts complete; each wait is bounded anyway.  Returns s.
+// already streams weights.  Two forms:
+//  * grid-wide (the usual one): (1) amax of this CTA's slice of X (a
+//    contiguous range of 8-element vectors), (2) a grid-wide max through
+//    xbar[0] and an arrival count, (3) s = amax / 448 (1 when amax = 0) and
+//    this slice's codes E4M3(RN_fp32(x / s)) written to xq, (4) a second
+//    count, xbar[2], that every CTA's producer waits for before it loads X
+//    codes.  Every CTA is resident (at most one per SM, cooperative launch),
+//    so both counts complete; each wait is bounded anyway.
+//  * local (X of at most kLocalXVec vectors): every CTA takes the amax of
+//    all of X and encodes all of it itself, so no CTA waits for another; the
+//    codes every CTA writes are identical, and each CTA's producer waits
+//    only for its own CTA (x_ready).
+//  * between the two (X of at most kLocalAmaxXVec vectors): every CTA takes
+//    the amax of all of X (no first count), then encodes its slice as in
+//    the grid-wide form.
+// XQ = 2 writes the SlideSparse lift: each 8-group g of a row becomes the 12
+// codes of windows 2j..2j+3, j = 0..2.  Returns s.
+constexpr int64_t kLocalXVec = 1024;
+constexpr int64_t kLocalAmaxXVec = 4096;
+
 template <int XQ>
-__device__ float fused_quantize(const GemmArgs &p, int t, uint32_t *s_red, float *s_scale) {
-  const int64_t v0 = static_cast<int64_t>(blockIdx.x) * p.xvec / gridDim.x;
-  const int64_t v1 = static_cast<int64_t>(blockIdx.x + 1) * p.xvec / gridDim.x;
+__device__ __forceinline__ void encode_xvec(const GemmArgs &p, int64_t v, float sx) {
+  const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p.x) + v);
+  const uint32_t h[4] = {w.x, w.y, w.z, w.w};
+  uint32_t c[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    c[2 * i] = e4m3_code(__fdiv_rn(bf16_bits_to_float(h[i] & 0xFFFFu), sx));
+    c[2 * i + 1] = e4m3_code(__fdiv_rn(bf16_bits_to_float(h[i] >> 16), sx));
+  }
+  if constexpr (XQ == 1) {
+    *reinterpret_cast<uint2 *>(p.xq + 8 * v) =
+        make_uint2(c[0] | c[1] << 8 | c[2] << 16 | c[3] << 24, c[4] | c[5] << 8 | c[6] << 16 | c[7] << 24);
+  } else {
+    uint32_t *o = reinterpret_cast<uint32_t *>(p.xq + 12 * v);
+    o[0] = c[0] | c[1] << 8 | c[2] << 16 | c[3] << 24;
+    o[1] = c[2] | c[3] << 8 | c[4] << 16 | c[5] << 24;
+    o[2] = c[4] | c[5] << 8 | c[6] << 16 | c[7] << 24;
+  }
+}
+
+template <int XQ>
+__device__ float fused_quantize(const GemmArgs &p, int t, uint32_t *s_red, float *s_scale, uint64_t *x_ready) {
+  const bool local = p.xvec <= kLocalXVec;
+  const bool local_amax = p.xvec <= kLocalAmaxXVec;
+  const int64_t v0 = local ? 0 : static_cast<int64_t>(blockIdx.x) * p.xvec / gridDim.x;
+  const int64_t v1 = local ? p.xvec : static_cast<int64_t>(blockIdx.x + 1) * p.xvec / gridDim.x;
   const uint4 *xv = reinterpret_cast<const uint4 *>(p.x);
   uint32_t m2 = 0;
-  for (int64_t v = v0 + t; v < v1; v += 128) m2 = __vmaxu2(m2, absmax8x2(__ldg(xv + v)));
+  for (int64_t v = (local_amax ? 0 : v0) + t; v < (local_amax ? p.xvec : v1); v += 128)
+    m2 = __vmaxu2(m2, absmax8x2(__ldg(xv + v)));
   uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
   if ((t & 31) == 0) s_red[t >> 5] = mx;
   named_bar_sync(1, 128);
   if (t == 0) {
     mx = max(max(s_red[0], s_red[1]), max(s_red[2], s_red[3]));
-    red_max_relaxed_gpu(&p.xbar[0], mx);
-    red_release_add_gpu(&p.xbar[1], 1u);  // orders the max before the arrival
-    wait_count_gpu(&p.xbar[1], gridDim.x, p.status);
-    const uint32_t amax = ld_acquire_gpu(&p.xbar[0]);
+    uint32_t amax = mx;
+    if (!local_amax) {
+      red_max_relaxed_gpu(&p.xbar[0], mx);
+      red_release_add_gpu(&p.xbar[1], 1u);  // orders the max before the arrival
+      wait_count_gpu(&p.xbar[1], gridDim.x, p.status);
+      amax = ld_acquire_gpu(&p.xbar[0]);
+    }
     const float sx = amax == 0u ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax), 448.0f);
     if (blockIdx.x == 0) {
       if (amax >= 0x7F80u && p.status) atomicOr(p.status, SP24_STATUS_NONFINITE);
@@ -342,28 +381,15 @@ __device__ float fused_quantize(const GemmArgs &p, int t, uint32_t *s_red, float
   }
   named_bar_sync(1, 128);
   const float sx = *s_scale;
-  for (int64_t v = v0 + t; v < v1; v += 128) {
-    const uint4 w = __ldg(xv + v);
-    const uint32_t h[4] = {w.x, w.y, w.z, w.w};
-    uint32_t c[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      c[2 * i] = e4m3_code(__fdiv_rn(bf16_bits_to_float(h[i] & 0xFFFFu), sx));
-      c[2 * i + 1] = e4m3_code(__fdiv_rn(bf16_bits_to_float(h[i] >> 16), sx));
-    }
-    if constexpr (XQ == 1) {
-      *reinterpret_cast<uint2 *>(p.xq + 8 * v) =
-          make_uint2(c[0] | c[1] << 8 | c[2] << 16 | c[3] << 24, c[4] | c[5] << 8 | c[6] << 16 | c[7] << 24);
-    } else {
-      uint32_t *o = reinterpret_cast<uint32_t *>(p.xq + 12 * v);
-      o[0] = c[0] | c[1] << 8 | c[2] << 16 | c[3] << 24;
-      o[1] = c[2] | c[3] << 8 | c[4] << 16 | c[5] << 24;
-      o[2] = c[4] | c[5] << 8 | c[6] << 16 | c[7] << 24;
-    }
-  }
+  for (int64_t v = v0 + t; v < v1; v += 128) encode_xvec<XQ>(p, v, sx);
   fence_proxy_async_global();  // the codes are read back by TMA loads
   named_bar_sync(1, 128);
-  if (t == 0) red_release_add_gpu(&p.xbar[2], 1u);
+  if (t == 0) {
+    if (local)
+      mbar_arrive(x_ready);
+    else
+      red_release_add_gpu(&p.xbar[2], 1u);
+  }
   return sx;
 }
 
@@ -388,7 +414,8 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
   uint64_t *meta_ready = empty + S;
   uint64_t *tmem_full = meta_ready + S;
   uint64_t *tmem_empty = tmem_full + NB;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tmem_empty + NB);
+  uint64_t *x_ready = tmem_empty + NB;  // fused local quantisation: codes written
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(x_ready + 1);
   [[maybe_unused]] __shared__ uint32_t s_xred[4];
   [[maybe_unused]] __shared__ float s_xscale;
 
@@ -410,6 +437,7 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
       mbar_init(&tmem_full[b], 1);
       mbar_init(&tmem_empty[b], C::kEpiThreads);
     }
+    mbar_init(x_ready, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -473,8 +501,12 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
       }
       grid_dependency_wait();
       if constexpr (XQ != 0) {
-        // the activation codes are written by this grid's epilogue warps
-        wait_count_gpu(&p.xbar[2], gridDim.x, p.status);
+        // the activation codes are written by the epilogue warps: of this
+        // CTA (local form) or of the whole grid
+        if (p.xvec <= kLocalXVec)
+          mbar_wait(x_ready, 0u, p.status);
+        else
+          wait_count_gpu(&p.xbar[2], gridDim.x, p.status);
         fence_proxy_async_global();
       }
       while (ok && it.next(p, sg)) {
@@ -585,7 +617,7 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
     const int rt0 = (e >> 2) * C::kRtPerWarp;  // first row tile this warp drains
     float sx;
     if constexpr (XQ != 0)
-      sx = fused_quantize<XQ>(p, t, s_xred, &s_xscale);
+      sx = fused_quantize<XQ>(p, t, s_xred, &s_xscale, x_ready);
     else
       sx = p.x_scale ? __ldg(p.x_scale) : 1.0f;
     const float sw = p.w_scale ? __ldg(p.w_scale) : 1.0f;

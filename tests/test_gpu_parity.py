@@ -545,8 +545,10 @@ def _fused_check(x, wts, n, what, lift=False):
     assert torch.equal(y, y2), what
 
 
-@pytest.mark.parametrize("m,n,k", [(1, 128, 128), (7, 256, 384), (16, 256, 256), (33, 384, 1024),
-                                   (64, 128, 640), (100, 256, 512), (256, 384, 1152)])
+# M*K/8 at most 1024: every CTA quantises all of X; at most 4096: every CTA
+# takes the whole amax and encodes a slice; above: amax and codes grid-wide
+@pytest.mark.parametrize("m,n,k", [(1, 128, 128), (7, 256, 384), (16, 256, 256), (20, 256, 1024),
+                                   (33, 384, 1024), (64, 128, 640), (100, 256, 512), (256, 384, 1152)])
 def test_quantize_gemm_packed_small(m, n, k):
     x = WL.random_bits((m, k), 1000 + m)
     w = WL.random_bits((n, k), 1100 + n, scale=0.02)

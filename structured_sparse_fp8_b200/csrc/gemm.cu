@@ -330,8 +330,7 @@ constexpr int64_t kLocalXVec = 1024;
 constexpr int64_t kLocalAmaxXVec = 4096;
 
 template <int XQ>
-__device__ __forceinline__ void encode_xvec(const GemmArgs &p, int64_t v, float sx) {
-  const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p.x) + v);
+__device__ __forceinline__ void encode_xvec(const GemmArgs &p, int64_t v, const uint4 w, float sx) {
   const uint32_t h[4] = {w.x, w.y, w.z, w.w};
   uint32_t c[8];
 #pragma unroll
@@ -357,9 +356,20 @@ __device__ float fused_quantize(const GemmArgs &p, int t, uint32_t *s_red, float
   const int64_t v0 = local ? 0 : static_cast<int64_t>(blockIdx.x) * p.xvec / gridDim.x;
   const int64_t v1 = local ? p.xvec : static_cast<int64_t>(blockIdx.x + 1) * p.xvec / gridDim.x;
   const uint4 *xv = reinterpret_cast<const uint4 *>(p.x);
+  // kXBatch independent 16-byte loads per thread in flight at a time
+  constexpr int kXBatch = 8;
   uint32_t m2 = 0;
-  for (int64_t v = (local_amax ? 0 : v0) + t; v < (local_amax ? p.xvec : v1); v += 128)
-    m2 = __vmaxu2(m2, absmax8x2(__ldg(xv + v)));
+  {
+    const int64_t a0 = local_amax ? 0 : v0, a1 = local_amax ? p.xvec : v1;
+    for (int64_t v = a0 + t; v < a1; v += 128 * kXBatch) {
+      uint4 w[kXBatch];
+#pragma unroll
+      for (int u = 0; u < kXBatch; ++u)
+        w[u] = v + 128 * u < a1 ? __ldg(xv + v + 128 * u) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int u = 0; u < kXBatch; ++u) m2 = __vmaxu2(m2, absmax8x2(w[u]));
+    }
+  }
   uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
   if ((t & 31) == 0) s_red[t >> 5] = mx;
   named_bar_sync(1, 128);
@@ -381,7 +391,15 @@ __device__ float fused_quantize(const GemmArgs &p, int t, uint32_t *s_red, float
   }
   named_bar_sync(1, 128);
   const float sx = *s_scale;
-  for (int64_t v = v0 + t; v < v1; v += 128) encode_xvec<XQ>(p, v, sx);
+  for (int64_t v = v0 + t; v < v1; v += 128 * kXBatch) {
+    uint4 w[kXBatch];
+#pragma unroll
+    for (int u = 0; u < kXBatch; ++u)
+      if (v + 128 * u < v1) w[u] = __ldg(xv + v + 128 * u);
+#pragma unroll
+    for (int u = 0; u < kXBatch; ++u)
+      if (v + 128 * u < v1) encode_xvec<XQ>(p, v + 128 * u, w[u], sx);
+  }
   fence_proxy_async_global();  // the codes are read back by TMA loads
   named_bar_sync(1, 128);
   if (t == 0) {

@@ -672,13 +672,6 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
       }
       const int b = j % NB;
       const int r = j / NB;
-      mbar_wait(&tmem_full[b], static_cast<uint32_t>(r) & 1u, p.status);
-      tc_fence_after();
-      const int n0 = (sg.tile % p.tiles_n) * C::kRows;
-      const int m0 = (sg.tile / p.tiles_n) * BN;
-      const int mvalid = min(BN, p.M - m0);
-      // lane quarter of this warp, accumulator b; row tile rt at + rt * BN
-      const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::kAccCols;
       // fp32 partial tile of CTA g, row tile rt, in quads of 4 token columns
       // laid out [column quad][row][4], so that a warp's 32 rows of one quad
       // are 512 contiguous bytes: quad cq of this thread's row.
@@ -686,6 +679,43 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
         return reinterpret_cast<float4 *>(p.partials) +
                ((static_cast<size_t>(g) * MT + rt) * (BN / 4) + cq) * 128 + row;
       };
+      // Owner of a split tile: its contributors (the next CTAs) compute this
+      // tile's later k-blocks as the first segment of their range, so they
+      // are normally done before this CTA's own k-blocks are.  Wait for them
+      // and start loading the first contributor's first pass before the
+      // accumulator is ready, so that the L2 round trip overlaps the last
+      // MMAs instead of following them.
+      static_assert(C::kRtPerWarp == 1, "each epilogue warp drains one row tile");
+      int first = 0, last = -1;  // contributor CTAs of an owned tile
+      float4 nxt[8];             // the next pass's first-contributor partial
+      if (sg.role == kOwner) {
+        const int64_t u_first = static_cast<int64_t>(sg.tile - p.dp_tiles) * p.num_kb;
+        first = static_cast<int>(blockIdx.x) + 1;
+        last = cta_of_unit(u_first + p.num_kb - 1, p.sk_units, p.sk_grid);
+        if (t == 0) {
+          const uint32_t expect = static_cast<uint32_t>(last - first + 1);
+          const uint64_t t0 = global_timer_ns();
+          uint32_t polls = 0;
+          while (ld_acquire_gpu(&p.counters[sg.tile - p.dp_tiles]) < expect) {
+            __nanosleep(20);
+            if ((++polls & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+              if (p.status) atomicOr(p.status, SP24_STATUS_TIMEOUT);
+              break;
+            }
+          }
+          p.counters[sg.tile - p.dp_tiles] = 0u;  // leave the workspace counters at zero
+        }
+        named_bar_sync(1, C::kEpiThreads);  // the acquire by thread 0 covers the whole CTA's reads
+#pragma unroll
+        for (int k4 = 0; k4 < kW / 4; ++k4) nxt[k4] = __ldcg(part4(first, rt0, k4));
+      }
+      mbar_wait(&tmem_full[b], static_cast<uint32_t>(r) & 1u, p.status);
+      tc_fence_after();
+      const int n0 = (sg.tile % p.tiles_n) * C::kRows;
+      const int m0 = (sg.tile / p.tiles_n) * BN;
+      const int mvalid = min(BN, p.M - m0);
+      // lane quarter of this warp, accumulator b; row tile rt at + rt * BN
+      const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::kAccCols;
 
       if (sg.role == kContrib) {
         // leave the fp32 partial tile (valid token columns) for the owner
@@ -711,38 +741,14 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
         named_bar_sync(1, C::kEpiThreads);
         if (t == 0) red_release_add_gpu(&p.counters[sg.tile - p.dp_tiles], 1u);
       } else {
-        int first = 0, last = -1;  // contributor CTAs of an owned tile
-        if (sg.role == kOwner) {
-          const int64_t u_first = static_cast<int64_t>(sg.tile - p.dp_tiles) * p.num_kb;
-          first = static_cast<int>(blockIdx.x) + 1;
-          last = cta_of_unit(u_first + p.num_kb - 1, p.sk_units, p.sk_grid);
-          if (t == 0) {
-            const uint32_t expect = static_cast<uint32_t>(last - first + 1);
-            const uint64_t t0 = global_timer_ns();
-            uint32_t polls = 0;
-            while (ld_acquire_gpu(&p.counters[sg.tile - p.dp_tiles]) < expect) {
-              __nanosleep(20);
-              if ((++polls & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
-                if (p.status) atomicOr(p.status, SP24_STATUS_TIMEOUT);
-                break;
-              }
-            }
-            p.counters[sg.tile - p.dp_tiles] = 0u;  // leave the workspace counters at zero
-          }
-          named_bar_sync(1, C::kEpiThreads);  // the acquire by thread 0 covers the whole CTA's reads
-        }
 #pragma unroll 1
         for (int rt = rt0; rt < rt0 + C::kRtPerWarp; ++rt) {
           const int n = n0 + rt * 128 + row;
           const uint32_t t_row = t_acc + rt * BN;
           // kW token columns per pass.  The first contributor's partial for
-          // the next pass is loaded while this pass is summed and stored, so
-          // an owned tile costs about one L2 round trip, not one per pass.
-          float4 nxt[8];
-          if (first <= last) {
-#pragma unroll
-            for (int k4 = 0; k4 < kW / 4; ++k4) nxt[k4] = __ldcg(part4(first, rt, k4));
-          }
+          // the next pass is loaded while this pass is summed and stored (for
+          // the first pass: before the accumulator was ready, above), so an
+          // owned tile costs about one L2 round trip, not one per pass.
           // Y through shared memory: this warp's 32 rows of one 32-token pass
           // (see Config), staged token-major as rows of Y.  Lane 0 issues the
           // warp's stores; before a buffer is rewritten it waits until the

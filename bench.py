@@ -74,6 +74,10 @@ def bytes_dense_gemm(m, n, k):
     return n * k + m * k + 2 * m * n + 8
 
 
+def bytes_bf16_sparse_gemm(m, n, k):
+    return n * k + n * k // 8 + 2 * m * k + 2 * m * n
+
+
 def bytes_slide68(n, k):
     return 2 * n * k + 3 * n * k // 4 + 3 * n * k // 16 + 4
 
@@ -249,7 +253,14 @@ class GpuWorkload:
         self.comp_bytes = comp_bytes
         self.R_g = -(-self.R_g // len(ms)) * len(ms)
         self.ws = sp.Workspace(device)
-        self.ws.get(max(sp._lib.load().sp24_workspace_size(sp._lib.OP_GEMM, m, n, self.kc, 0) for m in ms) + 4096)
+        lib = sp._lib.load()
+        # every GEMM this workload times (packed, fused, canonical, BF16, dense),
+        # sized once here so that no workspace is allocated inside a graph
+        self.ws.get(max(max(lib.sp24_workspace_size(sp._lib.OP_GEMM, m, n, self.kc, 0),
+                            lib.sp24_workspace_size(sp._lib.OP_LIFT_GEMM_PACKED if self.is68
+                                                    else sp._lib.OP_QUANTIZE_GEMM_PACKED, m, n, k, 0),
+                            lib.sp24_workspace_size(sp._lib.OP_GEMM, m, n, k, 1),
+                            lib.sp24_workspace_size(sp._lib.OP_GEMM_DENSE, m, n, k, 0)) for m in ms) + 4096)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
         def new_comp():
@@ -356,23 +367,45 @@ class GpuWorkload:
     def dense_compare(self, reps=50):
         """Sparse GEMM of this workload vs the dense FP8 GEMM of the same
         layer (dense W[N, K] with X quantised at K), each timed as a CUDA
-        graph of `reps` launches over rotating weight copies."""
+        graph of `reps` launches over rotating weight copies.  The same
+        sparse GEMM on the canonical (unpacked) weight layout and, for 2:4,
+        with BF16 operands (values bf16 [N, K/2], X bf16) is timed alongside."""
         torch, sp = self.torch, self.sp
         n, k, kc = self.n, self.k, self.kc
         out = {}
         wq, sw = sp.fp8_quantize_pertensor(self.w_pool[0], workspace=self.ws)
         ndense = max(2, -(-3 * L2_BYTES // (n * k)))
         dpool = [wq.clone() for _ in range(ndense)]
+        if self.is68:
+            canon = sp.slide68_decompose(self.w_pool[0], "e4m3", workspace=self.ws)
+            bf = None
+        else:
+            canon = sp.sp24_prune_compress(self.w_pool[0], "e4m3", workspace=self.ws)
+            bf = sp.sp24_prune_compress(self.w_pool[0], "bf16", workspace=self.ws)
+        ncanon = max(2, -(-3 * L2_BYTES // self.comp_bytes))
+        cpool = [(canon["values"].clone(), canon["meta"].clone()) for _ in range(ncanon)]
+        if bf is not None:
+            nbf = max(2, -(-3 * L2_BYTES // (n * k + n * k // 8)))
+            bpool = [(bf["values"].clone(), bf["meta"].clone()) for _ in range(nbf)]
+        kinds = ("sparse", "dense", "canonical") + (("bf16",) if bf is not None else ())
         for m in self.ms:
             xqd, sxd = sp.fp8_quantize_pertensor(self.x_dev[m], workspace=self.ws)
             res = {}
-            for kind in ("sparse", "dense"):
+            for kind in kinds:
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g):
                     for r in range(reps):
                         if kind == "dense":
                             sp.fp8_gemm_dense(xqd, sxd, dpool[r % ndense], sw,
                                               out=self.y[m], workspace=self.ws)
+                        elif kind == "canonical":
+                            v, e = cpool[r % ncanon]
+                            sp.sp24_gemm(self.xq[m], self.sx[m], v, e, canon["scale"],
+                                         out=self.y[m], workspace=self.ws)
+                        elif kind == "bf16":
+                            v, e = bpool[r % nbf]
+                            sp.sp24_gemm(self.x_dev[m], None, v, e, None, dtype="bf16",
+                                         out=self.y[m], workspace=self.ws)
                         else:
                             c = self.g_pool[r % self.R_g]
                             sp.sp24_gemm_packed(self.xq[m], self.sx[m], c["packed"], c["scale"], n,
@@ -391,8 +424,14 @@ class GpuWorkload:
                            "sparse_gbs": round(bytes_sparse_gemm(m, n, kc) / res["sparse"] / 1e3, 1),
                            "dense_gbs": round(bytes_dense_gemm(m, n, k) / res["dense"] / 1e3, 1),
                            "sparse_tflops_dense_equiv": round(2 * m * n * kc / res["sparse"] / 1e6, 2),
-                           "dense_tflops": round(2 * m * n * k / res["dense"] / 1e6, 2)}
-        del dpool
+                           "dense_tflops": round(2 * m * n * k / res["dense"] / 1e6, 2),
+                           "canonical_layout_us": round(res["canonical"], 3),
+                           "canonical_layout_gbs": round(bytes_sparse_gemm(m, n, kc) / res["canonical"] / 1e3, 1)}
+            if "bf16" in res:
+                out[str(m)]["bf16_sparse_us"] = round(res["bf16"], 3)
+                out[str(m)]["bf16_sparse_gbs"] = round(bytes_bf16_sparse_gemm(m, n, k) / res["bf16"] / 1e3, 1)
+                out[str(m)]["bf16_sparse_tflops"] = round(2 * m * n * k / res["bf16"] / 1e6, 2)
+        del dpool, cpool
         return out
 
     def fusion_compare(self, reps=50):

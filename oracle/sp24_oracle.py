@@ -311,6 +311,62 @@ def within_tolerance(y_gpu: np.ndarray, y_ref: np.ndarray, bound: np.ndarray,
 
 
 # ---------------------------------------------------------------------------
+# Per-token activation scales and per-channel weight scales (the SlideSparse
+# summary, §2 "Pipeline de Implementacion": its fused quantisation kernel
+# scales each token; the roadmap, §Interaction avec la quantification:
+# finer-grained scales for layers with outliers)
+# ---------------------------------------------------------------------------
+
+
+def quantize_pertoken(bits: np.ndarray):
+    """Per-token dynamic E4M3 quantisation of X [M, K]: row m gets its own
+    scale s_m = amax|X[m, :]| / 448 (1.0 for an all-zero row) and the codes
+    E4M3(x / s_m).  Returns (codes uint8 [M, K], scales float32 [M]).
+
+    Reading: the per-tensor rule (scale_from_amax, quantize_with_scale)
+    applied to each row on its own.
+    """
+    bits = np.asarray(bits, dtype=np.uint16)
+    codes = np.empty(bits.shape, dtype=np.uint8)
+    scales = np.empty(bits.shape[0], dtype=np.float32)
+    for m in range(bits.shape[0]):
+        codes[m], scales[m] = quantize_pertensor(bits[m])
+    return codes, scales
+
+
+def sp24_prune_compress_perchannel(w_bits: np.ndarray):
+    """2:4 prune + per-output-channel E4M3 quantisation + compress: the same
+    selection and layout as sp24_prune_compress, with row n of W quantised by
+    its own scale s_n = amax|W[n, :]| / 448 (the amax of the pruned row too:
+    each group's largest element is kept).  Returns a dict with ``values``,
+    ``meta``, ``mask``, ``scales`` (float32 [N]) and ``pruned_dense``.
+    """
+    w_bits = np.asarray(w_bits, dtype=np.uint16)
+    mask = prune24_mask(w_bits)
+    codes = np.empty(w_bits.shape, dtype=np.uint8)
+    scales = np.empty(w_bits.shape[0], dtype=np.float32)
+    for n in range(w_bits.shape[0]):
+        scales[n] = scale_from_amax(amax(w_bits[n]))
+        codes[n] = quantize_with_scale(w_bits[n], scales[n])
+    dense = np.where(mask, codes, np.uint8(0)).astype(np.uint8)
+    vals, meta = compress24(mask, codes)
+    return dict(values=vals.astype(np.uint8), meta=meta, mask=mask, scales=scales,
+                pruned_dense=dense)
+
+
+def gemm_ref_scaled(x_vals: np.ndarray, w_vals: np.ndarray, sx: np.ndarray, sw: np.ndarray):
+    """Y[m, n] = sx[m] * sw[n] * sum_k x[m, k] * w[n, k] in float64 and the
+    bound B[m, n] = |sx[m] * sw[n]| * sum_k |x[m, k] * w[n, k]|; a scalar
+    sx or sw is the same scale for every row or column."""
+    x = np.asarray(x_vals, dtype=np.float64)
+    w = np.asarray(w_vals, dtype=np.float64)
+    a = np.broadcast_to(np.asarray(sx, dtype=np.float64).reshape(-1), (x.shape[0],))
+    b = np.broadcast_to(np.asarray(sw, dtype=np.float64).reshape(-1), (w.shape[0],))
+    s = a[:, None] * b[None, :]
+    return s * (x @ w.T), np.abs(s) * (np.abs(x) @ np.abs(w).T)
+
+
+# ---------------------------------------------------------------------------
 # 6:8 sliding-window decomposition and activation lifting (the SlideSparse
 # summary, §2 Metodologia)
 # ---------------------------------------------------------------------------

@@ -300,3 +300,68 @@ def test_lift_codes_are_gathered_codes_and_ratios():
     assert lifted.shape[1] / x.shape[1] == 1.5           # gamma = (2N-2)/N for N = 4
     # dense-equivalent work ratio of 6:8-through-2:4 vs dense: 1.5 / 2 = 0.75 -> S_max 4/3
     assert (1.5 * 0.5) == 0.75 and abs(1 / 0.75 - 4 / 3) < 1e-12
+
+
+# --------------------------------------------------------------------------
+# Per-token activation scales, per-channel weight scales
+# --------------------------------------------------------------------------
+
+def _powers_of_two_rows(base_bits, n_rows):
+    """Rows base * 2^j (exact in bf16: the exponent field of every nonzero
+    value moves up by j)."""
+    base = np.asarray(base_bits, dtype=np.uint16)
+    nz = (base & 0x7FFF) != 0
+    rows = [np.where(nz, base + np.uint16(j << 7), base).astype(np.uint16) for j in range(n_rows)]
+    return np.stack(rows)
+
+
+def test_pertoken_scales_follow_row_magnitude_exactly():
+    base = WL.random_bits((1, 256), 71)[0]
+    x = _powers_of_two_rows(base, 6)
+    codes, scales = O.quantize_pertoken(x)
+    assert scales.dtype == np.float32 and codes.dtype == np.uint8
+    for j in range(6):
+        # scaling a row by 2^j scales its amax, hence its scale, by 2^j and
+        # leaves every quotient x / s, hence every code, unchanged
+        assert scales[j] == np.float32(scales[0] * 2.0 ** j)
+        assert np.array_equal(codes[j], codes[0])
+        # the row's largest magnitude maps exactly to 448 (code 0x7E)
+        assert (codes[j] & 0x7F).max() == 0x7E
+    # a single row is quantised exactly as the per-tensor path quantises it
+    c1, s1 = O.quantize_pertensor(x[3])
+    assert np.array_equal(codes[3], c1) and scales[3] == s1
+
+
+def test_pertoken_zero_row_takes_scale_one():
+    x = WL.random_bits((3, 64), 72)
+    x[1] = 0
+    codes, scales = O.quantize_pertoken(x)
+    assert scales[1] == np.float32(1.0) and not codes[1].any()
+
+
+def test_perchannel_prune_selects_like_per_tensor_and_scales_each_row():
+    base = WL.random_bits((1, 512), 73, scale=0.02)[0]
+    w = _powers_of_two_rows(base, 5)
+    r = O.sp24_prune_compress_perchannel(w)
+    assert np.array_equal(r["mask"], O.prune24_mask(w))
+    for j in range(5):
+        assert r["scales"][j] == np.float32(r["scales"][0] * 2.0 ** j)
+        assert np.array_equal(r["values"][j], r["values"][0])
+        assert np.array_equal(r["meta"][j], r["meta"][0])
+        assert (r["values"][j] & 0x7F).max() == 0x7E
+    # one row alone is the per-tensor weight path of that row
+    one = O.sp24_prune_compress(w[2:3], "e4m3")
+    assert np.array_equal(r["values"][2], one["values"][0]) and r["scales"][2] == one["scale"]
+
+
+def test_scaled_gemm_reduces_to_the_pinned_reference():
+    x = O.e4m3_decode(WL.random_bits((4, 64), 74).astype(np.uint8) & 0x7E)
+    w = O.e4m3_decode(WL.random_bits((6, 64), 75).astype(np.uint8) & 0x7E)
+    y0, b0 = O.gemm_ref(x, w)
+    sx = np.array([2.0 ** m for m in range(4)], dtype=np.float32)
+    sw = np.array([2.0 ** -n for n in range(6)], dtype=np.float32)
+    y, b = O.gemm_ref_scaled(x, w, sx, sw)
+    assert np.array_equal(y, y0 * np.outer(sx, sw)) and np.array_equal(b, b0 * np.outer(sx, sw))
+    y1, b1 = O.gemm_ref_scaled(x, w, np.float32(0.5), np.float32(3.0))
+    y2, b2 = O.gemm_ref(x, w, np.float32(0.5), np.float32(3.0))
+    assert np.array_equal(y1, y2) and np.array_equal(b1, b2)

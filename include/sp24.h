@@ -257,6 +257,46 @@ int slide68_lift_gemm_packed(const void *X, int M, int N, int K, const void *pac
                              sp24_stream_t stream);
 
 /*
+ * Finer-grained scales (SlideSparse, §2 "Pipeline de Implementacion": its
+ * fused quantiser scales each token; the roadmap, §Interaction avec la
+ * quantification: finer scales for outlier layers).  The per-tensor rule of
+ * fp8_quantize_pertensor applied to each row on its own.
+ *
+ * Per-token quantisation: X bf16 [rows, cols] -> q u8 [rows, cols] and
+ * scales f32 [rows]: scales[m] = amax|X[m, :]| / 448 (1.0 for an all-zero
+ * row), q[m, k] = E4M3(X[m, k] / scales[m]) (correctly rounded fp32
+ * quotient, then round to nearest even with saturation).  No workspace.
+ * SP24_STATUS_NONFINITE when a row holds NaN/Inf.  Shape rules: rows >= 1,
+ * cols % 8 == 0.
+ */
+int fp8_quantize_pertoken(const void *X, int64_t rows, int64_t cols, uint8_t *q, float *scales,
+                          int32_t *status, sp24_stream_t stream);
+
+/*
+ * Per-channel 2:4 weight path: the selection of sp24_prune_compress (two
+ * largest |w| of each 4, ties to the lower index) with one scale per output
+ * channel: w_scales[n] = amax|W[n, :]| / 448 (1.0 for an all-zero row),
+ * values u8 [N, K/2] = E4M3 codes of the kept elements of row n divided by
+ * w_scales[n], meta u8 [N, K/8] in the canonical layout (sp24_pack_weights
+ * makes the tile-packed form).  No workspace.  Shape rules: N >= 1,
+ * K % 8 == 0.
+ */
+int sp24_prune_compress_perchannel(const void *W, int N, int K, uint8_t *values, uint8_t *meta,
+                                   float *w_scales, int32_t *status, sp24_stream_t stream);
+
+/*
+ * sp24_gemm_packed with scale vectors: Y[m, n] = bf16( x_scale(m) *
+ * w_scale(n) * sum_k Xq[m, k] * W[n, k] ), where x_scale(m) = x_scales[m]
+ * when x_per_token (M floats), else x_scales[0], and w_scale(n) =
+ * w_scales[n] when w_per_channel (N floats), else w_scales[0].  Workspace,
+ * layouts and shape rules as sp24_gemm_packed; both scale pointers are
+ * required.
+ */
+int sp24_gemm_packed_scaled(const void *Xq, const float *x_scales, int x_per_token, const void *packed,
+                            const float *w_scales, int w_per_channel, void *Y, int M, int N, int K,
+                            void *workspace, size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+
+/*
  * Dense FP8 GEMM of the same kernel family (comparison baseline for the
  * sparse speedup): Y[M, N] = bf16( x_scale * w_scale * sum_k Xq[m,k] Wq[n,k] )
  * with Xq u8 [M, K], Wq u8 [N, K] (E4M3, e.g. the pruned_dense output of

@@ -9,7 +9,8 @@ Entry points (same names as the C ABI):
     sp24_prune_compress, fp8_quantize_pertensor, slide68_decompose,
     slide68_lift, sp24_gemm, fp8_gemm_dense, sp24_pack_weights,
     sp24_prune_compress_packed, slide68_decompose_packed, sp24_gemm_packed,
-    sp24_quantize_gemm_packed, slide68_lift_gemm_packed
+    sp24_quantize_gemm_packed, slide68_lift_gemm_packed, fp8_quantize_pertoken,
+    sp24_prune_compress_perchannel, sp24_gemm_packed_scaled
 """
 from __future__ import annotations
 
@@ -22,6 +23,7 @@ __all__ = [
     "sp24_prune_compress", "fp8_quantize_pertensor", "slide68_decompose", "slide68_lift",
     "sp24_gemm", "fp8_gemm_dense", "sp24_pack_weights", "sp24_prune_compress_packed", "slide68_decompose_packed",
     "sp24_gemm_packed", "sp24_quantize_gemm_packed", "slide68_lift_gemm_packed",
+    "fp8_quantize_pertoken", "sp24_prune_compress_perchannel", "sp24_gemm_packed_scaled",
     "Workspace",
     "Sp24Error", "DTYPE_E4M3", "DTYPE_BF16",
 ]
@@ -327,6 +329,70 @@ def slide68_lift_gemm_packed(X: torch.Tensor, packed: torch.Tensor, w_scale, n: 
     (Y bf16 [M, n], lifted codes u8 [M, K'], x_scale f32 [1])."""
     return _quant_gemm("slide68_lift_gemm_packed", _lib.OP_LIFT_GEMM_PACKED, lambda k: 3 * k // 2, X, packed,
                        w_scale, n, out, xq_out, x_scale_out, status, workspace)
+
+
+def fp8_quantize_pertoken(X: torch.Tensor, status: torch.Tensor | None = None,
+                          out: torch.Tensor | None = None, scales: torch.Tensor | None = None):
+    """Per-token E4M3 quantisation of X bf16 [M, K]: returns (codes u8 [M, K],
+    scales f32 [M]) with scales[m] = amax|X[m, :]| / 448."""
+    lib = _lib.load()
+    _require_cuda(X, status, out, scales)
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise Sp24Error("X must be a 2-D bf16 tensor")
+    M, K = X.shape
+    q = out if out is not None else torch.empty((M, K), dtype=torch.uint8, device=X.device)
+    sc = scales if scales is not None else torch.empty((M,), dtype=torch.float32, device=X.device)
+    if q.shape != (M, K) or q.dtype != torch.uint8 or sc.numel() != M or sc.dtype != torch.float32:
+        raise Sp24Error("output tensors have the wrong shape or dtype")
+    rc = lib.fp8_quantize_pertoken(_ptr(X), M, K, _ptr(q), _ptr(sc), _ptr(status), _stream(X.device))
+    _lib.check(rc, "fp8_quantize_pertoken")
+    return q, sc
+
+
+def sp24_prune_compress_perchannel(W: torch.Tensor, status: torch.Tensor | None = None, out: dict | None = None):
+    """2:4 prune + per-output-channel E4M3 quantise + compress of W bf16 [N, K].
+    Returns dict(values u8 [N, K/2], meta u8 [N, K/8], scales f32 [N])."""
+    lib = _lib.load()
+    _require_cuda(W, status)
+    if W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise Sp24Error("W must be a 2-D bf16 tensor")
+    N, K = W.shape
+    out = dict(out or {})
+    values = out.get("values")
+    if values is None:
+        values = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    meta = out.get("meta")
+    if meta is None:
+        meta = torch.empty((N, K // 8), dtype=torch.uint8, device=W.device)
+    scales = out.get("scales")
+    if scales is None:
+        scales = torch.empty((N,), dtype=torch.float32, device=W.device)
+    _require_cuda(values, meta, scales)
+    rc = lib.sp24_prune_compress_perchannel(_ptr(W), N, K, _ptr(values), _ptr(meta), _ptr(scales),
+                                            _ptr(status), _stream(W.device))
+    _lib.check(rc, "sp24_prune_compress_perchannel")
+    return dict(values=values, meta=meta, scales=scales)
+
+
+def sp24_gemm_packed_scaled(xq: torch.Tensor, x_scales: torch.Tensor, packed: torch.Tensor,
+                            w_scales: torch.Tensor, n: int, out: torch.Tensor | None = None,
+                            status: torch.Tensor | None = None, workspace: Workspace | None = None):
+    """sp24_gemm_packed with a per-token scale vector (x_scales of M floats,
+    or one) and a per-channel one (w_scales of n floats, or one)."""
+    lib = _lib.load()
+    _require_cuda(xq, x_scales, packed, w_scales, out, status)
+    M, K = xq.shape
+    if packed.numel() != n * K // 2 + n * K // 8:
+        raise Sp24Error("packed weights do not match N x K")
+    xv, wv = x_scales.numel() != 1, w_scales.numel() != 1
+    if (xv and x_scales.numel() != M) or (wv and w_scales.numel() != n):
+        raise Sp24Error("scale vectors must hold one value or one per token / channel")
+    y = out if out is not None else torch.empty((M, n), dtype=torch.bfloat16, device=xq.device)
+    ws, wsn = _ws(xq.device, _lib.OP_GEMM_PACKED, M, n, K, DTYPE_E4M3, workspace)
+    rc = lib.sp24_gemm_packed_scaled(_ptr(xq), _ptr(x_scales), int(xv), _ptr(packed), _ptr(w_scales), int(wv),
+                                     _ptr(y), M, n, K, _ptr(ws), wsn, _ptr(status), _stream(xq.device))
+    _lib.check(rc, "sp24_gemm_packed_scaled")
+    return y
 
 
 def fp8_gemm_dense(xq: torch.Tensor, x_scale, wq: torch.Tensor, w_scale,

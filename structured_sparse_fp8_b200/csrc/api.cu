@@ -304,6 +304,45 @@ int slide68_lift_gemm_packed(const void *X, int M, int N, int K, const void *pac
                            ws_bytes, status, stream);
 }
 
+int fp8_quantize_pertoken(const void *X, int64_t rows, int64_t cols, uint8_t *q, float *scales,
+                          int32_t *status, sp24_stream_t stream) {
+  if (!X || !q || !scales) return SP24_ERR_NULL;
+  if (rows < 1 || cols < 8 || cols % 8 != 0 || rows > INT32_MAX * 8ll) return SP24_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(q) || !aligned16(scales)) return SP24_ERR_ALIGN;
+  if (device_sm_count() < 0) return SP24_ERR_ARCH;
+  return cuda_status(sp24::launch_quantize_pertoken(X, rows, cols, q, scales, status,
+                                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sp24_prune_compress_perchannel(const void *W, int N, int K, uint8_t *values, uint8_t *meta,
+                                   float *w_scales, int32_t *status, sp24_stream_t stream) {
+  if (!W || !values || !meta || !w_scales) return SP24_ERR_NULL;
+  if (N < 1 || K < 8 || K % 8 != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(values) || !aligned16(meta) || !aligned16(w_scales)) return SP24_ERR_ALIGN;
+  if (device_sm_count() < 0) return SP24_ERR_ARCH;
+  return cuda_status(sp24::launch_prune24_perchannel(W, N, K, values, meta, w_scales, status,
+                                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sp24_gemm_packed_scaled(const void *Xq, const float *x_scales, int x_per_token, const void *packed,
+                            const float *w_scales, int w_per_channel, void *Y, int M, int N, int K,
+                            void *workspace, size_t ws_bytes, int32_t *status, sp24_stream_t stream) {
+  if (!Xq || !x_scales || !packed || !w_scales || !Y) return SP24_ERR_NULL;
+  if (M < 1 || N < 128 || N % 128 != 0 || K < 128 || K % 128 != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(Xq) || !aligned16(packed) || !aligned16(Y) || !aligned16(x_scales) || !aligned16(w_scales))
+    return SP24_ERR_ALIGN;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  const sp24::GemmPlan pl = sp24::plan_gemm(sp24::kSparseE4M3Packed, M, N, K, sms);
+  if (pl.workspace_bytes() > 0) {
+    if (!workspace || ws_bytes < pl.workspace_bytes()) return SP24_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SP24_ERR_ALIGN;
+  }
+  return cuda_status(sp24::launch_gemm_scaled(pl, Xq, x_scales, x_per_token ? 1 : 0, packed, w_scales,
+                                              w_per_channel ? 1 : 0, Y, M, N, K, workspace, status,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int fp8_gemm_dense(const uint8_t *Xq, const float *x_scale, const uint8_t *Wq,
                    const float *w_scale, void *Y, int M, int N, int K, void *workspace,
                    size_t ws_bytes, int32_t *status, sp24_stream_t stream) {

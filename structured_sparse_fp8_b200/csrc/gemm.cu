@@ -233,6 +233,9 @@ struct GemmArgs {
   float *x_scale_out;
   uint32_t *xbar;
   int64_t xvec;
+  // Scale vectors (VS kernels): x_scale holds M per-token scales when x_vec,
+  // w_scale N per-channel scales when w_vec; otherwise one value each.
+  int x_vec, w_vec;
 };
 
 enum SegRole : int { kWhole = 0, kOwner = 1, kContrib = 2 };
@@ -411,9 +414,16 @@ __device__ float fused_quantize(const GemmArgs &p, int t, uint32_t *s_red, float
   return sx;
 }
 
+// Scale of token m for the VS epilogue: the per-token vector, or the single
+// scale (0 for the padding tokens past M, which are never stored).
+__device__ __forceinline__ float token_scale(const GemmArgs &p, int m, float sx) {
+  if (!p.x_vec) return sx;
+  return m < p.M ? __ldg(p.x_scale + m) : 0.0f;
+}
+
 // ------------------------------------------------------------------ kernel
 
-template <int KIND, int BN, int MT, int XQ, int KB>
+template <int KIND, int BN, int MT, int XQ, int KB, bool VS>
 __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
@@ -682,9 +692,11 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
       // Owner of a split tile: its contributors (the next CTAs) compute this
       // tile's later k-blocks as the first segment of their range, so they
       // are normally done before this CTA's own k-blocks are.  Wait for them
-      // and start loading the first contributor's first pass before the
-      // accumulator is ready, so that the L2 round trip overlaps the last
-      // MMAs instead of following them.
+      // and (decode-sized tiles, where the tail matters) start loading the
+      // first contributor's first pass before the accumulator is ready, so
+      // that the L2 round trip overlaps the last MMAs instead of following
+      // them.  Wide tiles load it after the accumulator wait: keeping the
+      // registers live through their epilogue would spill.
       static_assert(C::kRtPerWarp == 1, "each epilogue warp drains one row tile");
       int first = 0, last = -1;  // contributor CTAs of an owned tile
       float4 nxt[8];             // the next pass's first-contributor partial
@@ -706,8 +718,10 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
           p.counters[sg.tile - p.dp_tiles] = 0u;  // leave the workspace counters at zero
         }
         named_bar_sync(1, C::kEpiThreads);  // the acquire by thread 0 covers the whole CTA's reads
+        if constexpr (!C::kTmaStoreY) {
 #pragma unroll
-        for (int k4 = 0; k4 < kW / 4; ++k4) nxt[k4] = __ldcg(part4(first, rt0, k4));
+          for (int k4 = 0; k4 < kW / 4; ++k4) nxt[k4] = __ldcg(part4(first, rt0, k4));
+        }
       }
       mbar_wait(&tmem_full[b], static_cast<uint32_t>(r) & 1u, p.status);
       tc_fence_after();
@@ -744,22 +758,41 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
 #pragma unroll 1
         for (int rt = rt0; rt < rt0 + C::kRtPerWarp; ++rt) {
           const int n = n0 + rt * 128 + row;
+          // VS: y = acc * sx[m] * sw[n]; this thread's W row n has one sw,
+          // and the pass's token scales are held one per lane (token_scale)
+          // and shuffled to every lane.
+          [[maybe_unused]] float swn = 0.0f;
+          if constexpr (VS) swn = p.w_vec ? __ldg(p.w_scale + n) : sw;
           const uint32_t t_row = t_acc + rt * BN;
           // kW token columns per pass.  The first contributor's partial for
           // the next pass is loaded while this pass is summed and stored (for
-          // the first pass: before the accumulator was ready, above), so an
-          // owned tile costs about one L2 round trip, not one per pass.
+          // the first pass of a narrow tile: before the accumulator was
+          // ready, above), so an owned tile costs about one L2 round trip,
+          // not one per pass.
+          if constexpr (C::kTmaStoreY) {
+            if (first <= last) {
+#pragma unroll
+              for (int k4 = 0; k4 < kW / 4; ++k4) nxt[k4] = __ldcg(part4(first, rt, k4));
+            }
+          }
           // Y through shared memory: this warp's 32 rows of one 32-token pass
           // (see Config), staged token-major as rows of Y.  Lane 0 issues the
           // warp's stores; before a buffer is rewritten it waits until the
           // store issued from it two passes ago has read it.
           auto store_pass = [&](int c, auto &&value_of) {
             uint16_t *buf = reinterpret_cast<uint16_t *>(ystage + (e * 2 + (ypass & 1)) * C::kStageY);
+            [[maybe_unused]] float xs = 0.0f;
+            if constexpr (VS) xs = token_scale(p, m0 + c + lane, sx);
             if (lane == 0) bulk_wait_group_read<1>();
             __syncwarp();
 #pragma unroll
             for (int k = 0; k < 32; k += 2) {  // two tokens per conversion
-              const __nv_bfloat162 h2 = __floats2bfloat162_rn(value_of(k) * sc, value_of(k + 1) * sc);
+              float f0 = sc, f1 = sc;
+              if constexpr (VS) {
+                f0 = __shfl_sync(0xFFFFFFFFu, xs, k) * swn;
+                f1 = __shfl_sync(0xFFFFFFFFu, xs, k + 1) * swn;
+              }
+              const __nv_bfloat162 h2 = __floats2bfloat162_rn(value_of(k) * f0, value_of(k + 1) * f1);
               buf[k * 32 + lane] = __bfloat16_as_ushort(h2.x);
               buf[(k + 1) * 32 + lane] = __bfloat16_as_ushort(h2.y);
             }
@@ -776,16 +809,18 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
               // Whole tile: up to 128 accumulator columns per TMEM wait (the
               // wait, not the arithmetic, dominates a pass), stored as 32-token
               // passes.  Tokens past M fall outside the tensor map.
+              // (64 columns per wait with scale vectors, for register room)
+              constexpr int kStep = VS ? 64 : 128;
 #pragma unroll 1
-              for (int c2 = 0; c2 < mvalid; c2 += 128) {
+              for (int c2 = 0; c2 < mvalid; c2 += kStep) {
                 uint32_t w0[64], w1[64];
                 tmem_ld_32x32b_x64(t_row + c2, w0);
-                if (c2 + 64 < BN) tmem_ld_32x32b_x64(t_row + c2 + 64, w1);
+                if (!VS && c2 + 64 < BN) tmem_ld_32x32b_x64(t_row + c2 + 64, w1);
                 tmem_ld_wait();
                 tmem_regs_ready(w0);
-                tmem_regs_ready(w1);
+                if constexpr (!VS) tmem_regs_ready(w1);
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
+                for (int h = 0; h < kStep / 32; ++h) {
                   if (c2 + 32 * h < mvalid)
                     store_pass(c2 + 32 * h, [&](int k) {
                       return __uint_as_float(h < 2 ? w0[32 * h + k] : w1[32 * (h - 2) + k]);
@@ -839,10 +874,14 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
               // rows), and store it with one bulk tensor copy.
               store_pass(c, [&](int k) { return acc[k]; });
             } else {
+              [[maybe_unused]] float xs = 0.0f;
+              if constexpr (VS) xs = token_scale(p, m0 + c + lane, sx);
 #pragma unroll
               for (int k = 0; k < kW; ++k) {
                 const int m = m0 + c + k;
-                if (m < p.M) p.y[static_cast<size_t>(m) * p.N + n] = f32_to_bf16_bits(acc[k] * sc);
+                float f = sc;
+                if constexpr (VS) f = __shfl_sync(0xFFFFFFFFu, xs, k) * swn;
+                if (m < p.M) p.y[static_cast<size_t>(m) * p.N + n] = f32_to_bf16_bits(acc[k] * f);
               }
             }
           }
@@ -967,18 +1006,19 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   return pl;
 }
 
-template <int KIND, int BN, int MT, int XQ = 0, int KB = 1>
+template <int KIND, int BN, int MT, int XQ = 0, int KB = 1, bool VS = false>
 static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float *x_scale,
                                 const void *w_values, const uint8_t *w_meta, const float *w_scale,
                                 void *y, int M, int N, int K, void *workspace, int32_t *status,
-                                cudaStream_t st, const GemmFusedX *fx = nullptr) {
+                                cudaStream_t st, const GemmFusedX *fx = nullptr, int x_vec = 0,
+                                int w_vec = 0) {
   using T = KindTraits<KIND>;
   using C = Config<KIND, BN, MT, KB>;
   static_assert(XQ == 0 || KIND == kSparseE4M3Packed, "fused quantisation feeds the packed E4M3 GEMM");
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN, MT, XQ, KB>,
+    attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN, MT, XQ, KB, VS>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
@@ -1037,6 +1077,8 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   a.x_scale_out = nullptr;
   a.xbar = nullptr;
   a.xvec = 0;
+  a.x_vec = x_vec;
+  a.w_vec = w_vec;
   if constexpr (XQ != 0) {
     a.x = static_cast<const uint16_t *>(fx->x);
     a.xq = fx->xq;
@@ -1062,7 +1104,7 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   attrs[1].val.cooperative = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = XQ != 0 ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, MT, XQ, KB>, tmA, tmB, tmE, tmY, a);
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, MT, XQ, KB, VS>, tmA, tmB, tmE, tmY, a);
 }
 
 template <int KIND>
@@ -1116,6 +1158,35 @@ static cudaError_t launch_quant_bn(const GemmPlan &pl, const GemmFusedX &fx, con
     case 128: return launch_typed<P, 128, 1, XQ>(pl, fx.xq, nullptr, packed, nullptr, w_scale, y, M, N, K, ws, status, st, &fx);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_gemm_scaled(const GemmPlan &pl, const void *xq, const float *x_scales, int x_vec,
+                               const void *packed, const float *w_scales, int w_vec, void *y, int M, int N,
+                               int K, void *ws, int32_t *status, cudaStream_t st) {
+  constexpr int P = kSparseE4M3Packed;
+#define SP24_SCALED(BN_, MT_, KB_)                                                                        \
+  return launch_typed<P, BN_, MT_, 0, KB_, true>(pl, xq, x_scales, packed, nullptr, w_scales, y, M, N, K, ws, \
+                                                 status, st, nullptr, x_vec, w_vec)
+  if (pl.kb == 2) {
+    switch (pl.bn) {
+      case 16: SP24_SCALED(16, 1, 2);
+      case 32: SP24_SCALED(32, 1, 2);
+      case 64: SP24_SCALED(64, 1, 2);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  switch (pl.bn) {
+    case 16: SP24_SCALED(16, 1, 1);
+    case 32: SP24_SCALED(32, 1, 1);
+    case 64: SP24_SCALED(64, 1, 1);
+    case 128: SP24_SCALED(128, 1, 1);
+    case 224:
+      if (pl.mt == 2) SP24_SCALED(224, 2, 1);
+      SP24_SCALED(224, 1, 1);
+    case 256: SP24_SCALED(256, 1, 1);
+    default: return cudaErrorInvalidValue;
+  }
+#undef SP24_SCALED
 }
 
 cudaError_t launch_gemm_quant(const GemmPlan &pl, const GemmFusedX &fx, const void *packed,

@@ -51,6 +51,12 @@ cudaError_t launch_slide68_fused(const void *w, int64_t nelem, bool fp8, uint32_
                                  float *scale, void *values, uint8_t *meta, int32_t *status,
                                  int sm_count, cudaStream_t st);
 
+// ---- rowscale.cu: per-token / per-channel scales (one warp per row).
+cudaError_t launch_quantize_pertoken(const void *x, int64_t rows, int64_t cols, uint8_t *q, float *scales,
+                                     int32_t *status, cudaStream_t st);
+cudaError_t launch_prune24_perchannel(const void *w, int N, int K, uint8_t *values, uint8_t *meta,
+                                      float *scales, int32_t *status, cudaStream_t st);
+
 // Records the CUDA error reported by sp24_last_cuda_error() (api.cu).
 void set_last_cuda_error(int e);
 
@@ -92,6 +98,12 @@ cudaError_t launch_gemm(GemmKind kind, const GemmPlan &plan, const void *xq, con
                         const void *w_values, const uint8_t *w_meta, const float *w_scale,
                         void *y, int M, int N, int K, void *workspace, int32_t *status,
                         cudaStream_t st);
+
+// The packed E4M3 GEMM with scale vectors: x_scales holds M per-token scales
+// when x_vec (else one), w_scales N per-channel scales when w_vec (else one).
+cudaError_t launch_gemm_scaled(const GemmPlan &plan, const void *xq, const float *x_scales, int x_vec,
+                               const void *packed, const float *w_scales, int w_vec, void *y, int M, int N,
+                               int K, void *workspace, int32_t *status, cudaStream_t st);
 
 // The packed E4M3 GEMM with the per-tensor quantisation of its activations
 // fused in front (plan from plan_gemm(kSparseE4M3Packed, M, N, K); bn <= 128,

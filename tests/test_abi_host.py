@@ -104,9 +104,19 @@ def test_validation_rejects_bad_arguments_without_a_gpu(lib):
     assert qg(FAKE, 4, 128, 128, FAKE, None, None, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_NULL
     assert qg(FAKE, 4, 128, 128, FAKE, None, FAKE, None, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_NULL
     assert lg(None, 4, 128, 256, FAKE, None, FAKE, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_NULL
+    # per-token / per-channel scales
+    assert lib.fp8_quantize_pertoken(FAKE, 4, 12, FAKE, FAKE, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.fp8_quantize_pertoken(FAKE, 0, 16, FAKE, FAKE, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.fp8_quantize_pertoken(FAKE, 4, 16, FAKE, None, None, None) == _lib.SP24_ERR_NULL
+    assert lib.sp24_prune_compress_perchannel(FAKE, 4, 12, FAKE, FAKE, FAKE, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.sp24_prune_compress_perchannel(FAKE, 4, 16, FAKE, None, FAKE, None, None) == _lib.SP24_ERR_NULL
+    gs = lib.sp24_gemm_packed_scaled
+    assert gs(FAKE, FAKE, 1, FAKE, FAKE, 1, FAKE, 4, 192, 128, FAKE, big, None, None) == _lib.SP24_ERR_SHAPE
+    assert gs(FAKE, None, 1, FAKE, FAKE, 1, FAKE, 4, 128, 128, FAKE, big, None, None) == _lib.SP24_ERR_NULL
     # alignment
     odd = ctypes.c_void_p((1 << 20) + 8)
     assert qg(FAKE, 4, 128, 128, FAKE, None, odd, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_ALIGN
+    assert lib.fp8_quantize_pertoken(FAKE, 4, 16, odd, FAKE, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.sp24_prune_compress_packed(FAKE, 128, 128, odd, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.fp8_quantize_pertensor(odd, 4, 32, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.sp24_gemm(FAKE, None, odd, FAKE, None, FAKE, 4, 128, 128, 0, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN

@@ -613,3 +613,91 @@ def test_quantize_gemm_packed_reuses_its_workspace():
     assert (ws.buf[:256] == 0).all()
     for (a, b), (c, d) in zip(outs[:3], outs[3:]):
         assert np.array_equal(a, b) and np.array_equal(a, c) and np.array_equal(c, d)
+
+
+# ------------------------------------------------------------ per-token / per-channel scales
+
+@pytest.mark.parametrize("shape,seed", [((1, 8), 1), ((3, 48), 2), ((16, 256), 3), ((37, 1000), 4)])
+def test_quantize_pertoken_bit_exact(shape, seed):
+    x = WL.random_bits(shape, 2100 + seed)
+    q, s = sp().fp8_quantize_pertoken(dev_bf16(x))
+    ref_q, ref_s = O.quantize_pertoken(x)
+    assert np.array_equal(host(s), ref_s) and np.array_equal(host(q), ref_q)
+
+
+def test_quantize_pertoken_workload_activations():
+    for cfg, m in ((2, 64), (3, 4096), (4, 256)):
+        x = WL.activation_bits(cfg, m)          # cfg 3 carries the outlier columns
+        q, s = sp().fp8_quantize_pertoken(dev_bf16(x))
+        ref_q, ref_s = O.quantize_pertoken(x)
+        assert np.array_equal(host(s), ref_s) and np.array_equal(host(q), ref_q), cfg
+
+
+def test_quantize_pertoken_zero_row_and_nonfinite_status():
+    x = WL.random_bits((4, 64), 2200)
+    x[2] = 0
+    st = new_status()
+    q, s = sp().fp8_quantize_pertoken(dev_bf16(x), status=st)
+    torch.cuda.synchronize()
+    assert host(s)[2] == 1.0 and (host(q)[2] == 0).all() and int(st.item()) == 0
+    x[1, 7] = 0x7FC0
+    st = new_status()
+    sp().fp8_quantize_pertoken(dev_bf16(x), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & 1
+
+
+@pytest.mark.parametrize("n,k,dist", [(1, 8, "normal"), (128, 128, "normal"), (256, 512, "ties"),
+                                      (384, 1024, "student_t3")])
+def test_prune_compress_perchannel_bit_exact(n, k, dist):
+    w = WL.random_bits((n, k), 2300 + n, scale=0.02, dist=dist)
+    r = sp().sp24_prune_compress_perchannel(dev_bf16(w))
+    ref = O.sp24_prune_compress_perchannel(w)
+    assert np.array_equal(host(r["scales"]), ref["scales"])
+    assert np.array_equal(host(r["values"]), ref["values"]) and np.array_equal(host(r["meta"]), ref["meta"])
+
+
+def test_prune_compress_perchannel_workload_weights():
+    w = WL.weight_bits(4)                        # Student-t(3), the outlier-heavy weights
+    r = sp().sp24_prune_compress_perchannel(dev_bf16(w))
+    rows = np.sort(np.random.default_rng(81).choice(w.shape[0], 96, replace=False))
+    ref = O.sp24_prune_compress_perchannel(w[rows])
+    assert np.array_equal(host(r["scales"])[rows], ref["scales"])
+    assert np.array_equal(host(r["values"])[rows], ref["values"]) and np.array_equal(host(r["meta"])[rows], ref["meta"])
+
+
+def _scaled_check(m, n, k, x_vec, w_vec, seed):
+    x = WL.random_bits((m, k), 2400 + seed)
+    w = WL.random_bits((n, k), 2500 + seed, scale=0.02)
+    st = new_status()
+    if x_vec:
+        xq, sx = sp().fp8_quantize_pertoken(dev_bf16(x), status=st)
+        ref_q, ref_sx = O.quantize_pertoken(x)
+    else:
+        xq, sx = sp().fp8_quantize_pertensor(dev_bf16(x), status=st)
+        ref_q, ref_sx = O.quantize_pertensor(x)
+    if w_vec:
+        r = sp().sp24_prune_compress_perchannel(dev_bf16(w), status=st)
+        values, meta, sw = r["values"], r["meta"], r["scales"]
+        ref_w = O.sp24_prune_compress_perchannel(w)
+        ref_sw = ref_w["scales"]
+    else:
+        c = sp().sp24_prune_compress(dev_bf16(w), "e4m3", status=st)
+        values, meta, sw = c["values"], c["meta"], c["scale"]
+        ref_w = O.sp24_prune_compress(w, "e4m3")
+        ref_sw = ref_w["scale"]
+    packed = sp().sp24_pack_weights(values, meta)
+    y = sp().sp24_gemm_packed_scaled(xq, sx, packed, sw, n, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(host(xq), ref_q) and np.array_equal(host(values), ref_w["values"])
+    y_ref, b = O.gemm_ref_scaled(O.e4m3_decode(ref_q), O.e4m3_decode(ref_w["pruned_dense"]), ref_sx, ref_sw)
+    assert_gemm_close(y, y_ref, b, f"scaled {m}x{n}x{k} x_vec={x_vec} w_vec={w_vec}")
+
+
+# decode tiles (256-K stages), a ragged M, stream-K splits, and 256-row tiles
+@pytest.mark.parametrize("m,n,k", [(1, 256, 512), (13, 384, 1024), (64, 128, 640), (300, 256, 1152),
+                                   (1100, 9728, 640)])
+@pytest.mark.parametrize("x_vec,w_vec", [(True, True), (True, False), (False, True), (False, False)])
+def test_sparse_gemm_packed_scaled(m, n, k, x_vec, w_vec):
+    _scaled_check(m, n, k, x_vec, w_vec, m + n)

@@ -434,6 +434,53 @@ class GpuWorkload:
         del dpool, cpool
         return out
 
+    def _graph_us(self, fn, reps):
+        """Average µs per call of `fn(r)` over a CUDA graph of `reps` calls."""
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for r in range(reps):
+                fn(r)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) * 1000.0 / reps
+
+    def finer_scales(self, reps=50):
+        """Per-token activation scales and per-channel weight scales on this
+        workload's shapes (2:4 only): the per-token quantiser, the per-channel
+        weight path and the GEMM with both scale vectors, each timed as a
+        CUDA graph over rotating inputs."""
+        if self.is68:
+            return None
+        torch, sp = self.torch, self.sp
+        n, k = self.n, self.k
+        out = {}
+        vals = torch.empty((n, k // 2), dtype=torch.uint8, device=self.dev)
+        meta = torch.empty((n, k // 8), dtype=torch.uint8, device=self.dev)
+        wsc = torch.empty((n,), dtype=torch.float32, device=self.dev)
+        t = self._graph_us(lambda r: sp.sp24_prune_compress_perchannel(
+            self.w_pool[r % self.R_w], out=dict(values=vals, meta=meta, scales=wsc)), max(4, reps // 5))
+        out["perchannel_prune"] = {"us": round(t, 3),
+                                   "gbs": round((bytes_prune24(n, k) + 4 * n) / t / 1e3, 1)}
+        for m in self.ms:
+            q = torch.empty((m, k), dtype=torch.uint8, device=self.dev)
+            xs = torch.empty((m,), dtype=torch.float32, device=self.dev)
+            tq = self._graph_us(lambda r: sp.fp8_quantize_pertoken(self.x_dev[m], out=q, scales=xs), reps)
+            tg = self._graph_us(lambda r: sp.sp24_gemm_packed_scaled(
+                q, xs, self.g_pool[r % self.R_g]["packed"], wsc, n, out=self.y[m], workspace=self.ws), reps)
+            out[str(m)] = {"pertoken_quantize_us": round(tq, 3),
+                           "pertoken_quantize_gbs": round((bytes_quant(m, k) + 4 * m) / tq / 1e3, 1),
+                           "scaled_gemm_us": round(tg, 3),
+                           "scaled_gemm_gbs": round((bytes_sparse_gemm(m, n, k) + 4 * m + 4 * n) / tg / 1e3, 1),
+                           "scaled_gemm_tflops_dense_equiv": round(2 * m * n * k / tg / 1e6, 2)}
+        return out
+
     def fusion_compare(self, reps=50):
         """For every M that the step runs fused: the fused launch against the
         activation kernel + GEMM pair it replaces, each as a CUDA graph of
@@ -573,6 +620,7 @@ def run_gpu(args, wl, rank, world, local_rank):
 
     compare = gw.dense_compare() if rank == 0 and not args.no_compare else None
     fusion = gw.fusion_compare() if rank == 0 and not args.no_compare else None
+    finer = gw.finer_scales() if rank == 0 and not args.no_compare else None
     e2e_t, h2d, d2h = gw.e2e(args.steps)
     e2e_t = max_over_ranks(e2e_t, device)
     del g_timed, g_detail, g_warm
@@ -605,6 +653,7 @@ def run_gpu(args, wl, rank, world, local_rank):
         "kernels": kernels,
         "sparse_vs_dense": compare,
         "fused_vs_unfused": fusion,
+        "finer_scales": finer,
         "e2e": {"value": round(aggregate_gbs(step_bytes, args.steps, world, e2e_t), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": gw.step_launches() * args.steps,

@@ -311,6 +311,91 @@ def within_tolerance(y_gpu: np.ndarray, y_ref: np.ndarray, bound: np.ndarray,
 
 
 # ---------------------------------------------------------------------------
+# General (2N-2):2N through 2:4 windows (the SlideSparse summary, §2
+# Metodologia: N-1 overlapping windows of 4 with stride 2 per 2N-group,
+# expansion (2N-2)/N; 6:8 is N = 4)
+# ---------------------------------------------------------------------------
+
+
+def slide_mask(bits: np.ndarray, n: int) -> np.ndarray:
+    """(2n-2):2n magnitude mask: the 2n-2 largest |w| of each 2n along K survive
+    (ties to the lower index)."""
+    return keep_mask(bits, 2 * n, 2 * n - 2)
+
+
+def slide_windows(kept: np.ndarray, n: int):
+    """Assign the 2n-2 kept positions of one 2n-group to its n-1 windows (window
+    j covers positions 2j .. 2j+3): for j = 0 .. n-2 in turn, window j takes the
+    two lowest-index kept positions in its range that no earlier window took
+    (the reading of the 6:8 case, for any n).  Returns n-1 pairs (p0, p1)."""
+    kept = [int(p) for p in np.nonzero(np.asarray(kept, dtype=bool))[0]]
+    if len(kept) != 2 * n - 2:
+        raise ValueError("a (2n-2):2n group must keep exactly 2n-2 positions")
+    taken, out = set(), []
+    for j in range(n - 1):
+        cand = [p for p in kept if 2 * j <= p <= 2 * j + 3 and p not in taken]
+        if len(cand) < 2:
+            raise AssertionError("window assignment failed")
+        taken.update(cand[:2])
+        out.append((cand[0], cand[1]))
+    if taken != set(kept):
+        raise AssertionError("window assignment lost a kept position")
+    return out
+
+
+def slide_decompose(w_bits: np.ndarray, n: int):
+    """(2n-2):2n prune, window decomposition and 2:4 compression over
+    K' = K (2n-2)/n, E4M3 with the per-tensor weight scale.  Window j of group
+    g owns expanded columns 4((n-1)g + j) .. +3; the element at position p of
+    the group sits at slot p - 2j.  Returns values [N, K'/2], meta [N, K'/8],
+    the mask, the expanded mask and codes [N, K'], the scale and ``src``."""
+    w_bits = np.asarray(w_bits, dtype=np.uint16)
+    rows_, k = w_bits.shape
+    g2 = 2 * n
+    if k % g2:
+        raise ValueError("K must be a multiple of 2n")
+    kp = k // g2 * 4 * (n - 1)
+    mask = slide_mask(w_bits, n)
+    emask = np.zeros((rows_, kp), dtype=bool)
+    src = np.full((rows_, kp), -1, dtype=np.int64)
+    for row in range(rows_):
+        for g in range(k // g2):
+            for j, (p0, p1) in enumerate(slide_windows(mask[row, g2 * g:g2 * g + g2], n)):
+                for p in (p0, p1):
+                    col = 4 * ((n - 1) * g + j) + (p - 2 * j)
+                    emask[row, col] = True
+                    src[row, col] = g2 * g + p
+    s = scale_from_amax(amax(w_bits))
+    codes = quantize_with_scale(w_bits, s)
+    r = np.arange(rows_)[:, None]
+    wexp = np.where(emask, codes[r, np.maximum(src, 0)], np.uint8(0)).astype(np.uint8)
+    vals, meta = compress24(emask, wexp)
+    return dict(values=vals, meta=meta, mask=mask, emask=emask, scale=s, expanded=wexp, src=src)
+
+
+def slide_lift_columns(k: int, n: int) -> np.ndarray:
+    """Source column of X for every lifted column:
+    X'[:, 4((n-1)g + j) + r] = X[:, 2n g + 2j + r]."""
+    g2 = 2 * n
+    cols = np.empty(k // g2 * 4 * (n - 1), dtype=np.int64)
+    for g in range(k // g2):
+        for j in range(n - 1):
+            for r in range(4):
+                cols[4 * ((n - 1) * g + j) + r] = g2 * g + 2 * j + r
+    return cols
+
+
+def slide_lift(x_bits: np.ndarray, n: int):
+    """Per-tensor E4M3 quantisation of X fused with the lift to K' = K (2n-2)/n:
+    returns (lifted codes [M, K'], scale)."""
+    x_bits = np.asarray(x_bits, dtype=np.uint16)
+    if x_bits.shape[1] % (2 * n):
+        raise ValueError("K must be a multiple of 2n")
+    codes, s = quantize_pertensor(x_bits)
+    return codes[:, slide_lift_columns(x_bits.shape[1], n)], s
+
+
+# ---------------------------------------------------------------------------
 # Per-token activation scales and per-channel weight scales (the SlideSparse
 # summary, §2 "Pipeline de Implementacion": its fused quantisation kernel
 # scales each token; the roadmap, §Interaction avec la quantification:

@@ -365,3 +365,55 @@ def test_scaled_gemm_reduces_to_the_pinned_reference():
     y1, b1 = O.gemm_ref_scaled(x, w, np.float32(0.5), np.float32(3.0))
     y2, b2 = O.gemm_ref(x, w, np.float32(0.5), np.float32(3.0))
     assert np.array_equal(y1, y2) and np.array_equal(b1, b2)
+
+
+# --------------------------------------------------------------------------
+# General (2N-2):2N windows
+# --------------------------------------------------------------------------
+
+def test_general_slide_reduces_to_the_pinned_68_functions():
+    w = WL.random_bits((5, 64), 91, scale=0.02, dist="ties")
+    g, r68 = O.slide_decompose(w, 4), O.slide68_decompose(w, "e4m3")
+    for key in ("values", "meta", "emask", "expanded"):
+        assert np.array_equal(g[key], r68[key]), key
+    assert g["scale"] == r68["scale"]
+    assert np.array_equal(O.slide_lift_columns(64, 4), O.lift_columns(64))
+
+
+@pytest.mark.parametrize("n", [3, 4, 5])
+def test_general_slide_every_mask_fills_its_windows(n):
+    g2 = 2 * n
+    for pruned in itertools.combinations(range(g2), 2):
+        kept = np.ones(g2, dtype=bool)
+        kept[list(pruned)] = False
+        pairs = O.slide_windows(kept, n)
+        assert len(pairs) == n - 1
+        for j, (p0, p1) in enumerate(pairs):
+            assert 2 * j <= p0 < p1 <= 2 * j + 3
+        assert sorted(p for pr in pairs for p in pr) == list(np.nonzero(kept)[0])
+
+
+@pytest.mark.parametrize("n", [3, 5])
+def test_general_slide_reconstructs_and_gemm_is_exact(n):
+    k = 4 * n * 2
+    w = WL.random_bits((6, k), 92 + n, scale=0.02)
+    x = WL.random_bits((3, k), 94 + n)
+    d = O.slide_decompose(w, n)
+    kp = k * (2 * n - 2) // n
+    assert d["expanded"].shape == (6, kp) and kp / k == (2 * n - 2) / n
+    # every window is 2:4 and scattering the expanded operand back gives the
+    # pruned, quantised W exactly
+    assert (d["emask"].reshape(6, -1, 4).sum(axis=2) == 2).all()
+    codes = O.quantize_with_scale(w, d["scale"])
+    back = np.zeros_like(codes)
+    for row in range(6):
+        for col in np.nonzero(d["emask"][row])[0]:
+            back[row, d["src"][row, col]] = d["expanded"][row, col]
+    assert np.array_equal(back, np.where(d["mask"], codes, np.uint8(0)))
+    # X' W'^T = X W_pruned^T exactly in float64 (products of E4M3 values)
+    xq, sx = O.quantize_pertensor(x)
+    xl, sxl = O.slide_lift(x, n)
+    assert sxl == sx
+    y1, _ = O.gemm_ref(O.e4m3_decode(xl), O.e4m3_decode(d["expanded"]))
+    y2, _ = O.gemm_ref(O.e4m3_decode(xq), O.e4m3_decode(back))
+    assert np.array_equal(y1, y2)

@@ -481,6 +481,55 @@ class GpuWorkload:
                            "scaled_gemm_tflops_dense_equiv": round(2 * m * n * k / tg / 1e6, 2)}
         return out
 
+    def general_slide(self, reps=50):
+        """The (2N-2):2N decomposition for N = 3 (4:6) and 5 (8:10) on the 6:8
+        layer's shape, with K chosen so that K' = 6144 as for 6:8 (K = 4608,
+        3840): the weight decomposition, the lift of each M and the sparse GEMM
+        over K' from tile-packed weights, each a CUDA graph over rotating
+        inputs larger than L2 (timing pools drawn on the device, N(0, 0.02))."""
+        if not self.is68:
+            return None
+        torch, sp = self.torch, self.sp
+        n, out = self.n, {}
+        gen = torch.Generator(device=self.dev)
+        for nn, k in ((3, 4608), (5, 3840)):
+            gen.manual_seed(600 + nn)
+            kp = k // (2 * nn) * 4 * (nn - 1)
+            r_w = max(2, -(-3 * L2_BYTES // (2 * n * k)))
+            r_g = max(2, -(-3 * L2_BYTES // (n * kp * 5 // 8)))
+            wpool = [(torch.randn((n, k), generator=gen, device=self.dev) * 0.02).to(torch.bfloat16)
+                     for _ in range(max(r_w, r_g))]
+            vals = torch.empty((n, kp // 2), dtype=torch.uint8, device=self.dev)
+            meta = torch.empty((n, kp // 8), dtype=torch.uint8, device=self.dev)
+            sw = torch.empty((1,), dtype=torch.float32, device=self.dev)
+            td = self._graph_us(lambda r: sp.slide_decompose(
+                wpool[r % r_w], nn, workspace=self.ws, out=dict(values=vals, meta=meta, scale=sw)),
+                max(4, reps // 5))
+            wbytes = 2 * n * k + n * kp // 2 + n * kp // 8 + 4
+            res = {"k": k, "k_prime": kp, "decompose_us": round(td, 3),
+                   "decompose_gbs": round(wbytes / td / 1e3, 1)}
+            layers = []
+            for r in range(r_g):
+                d = sp.slide_decompose(wpool[r], nn, workspace=self.ws)
+                layers.append((sp.sp24_pack_weights(d["values"], d["meta"]), d["scale"]))
+            del wpool
+            for m in self.ms:
+                x = (torch.randn((m, k), generator=gen, device=self.dev)).to(torch.bfloat16)
+                xl = torch.empty((m, kp), dtype=torch.uint8, device=self.dev)
+                sx = torch.empty((1,), dtype=torch.float32, device=self.dev)
+                y = torch.empty((m, n), dtype=torch.bfloat16, device=self.dev)
+                tl = self._graph_us(lambda r: sp.slide_lift(x, nn, workspace=self.ws, out=xl, scale=sx), reps)
+                tg = self._graph_us(lambda r: sp.sp24_gemm_packed(
+                    xl, sx, layers[r % r_g][0], layers[r % r_g][1], n, out=y, workspace=self.ws), reps)
+                res[str(m)] = {"lift_us": round(tl, 3),
+                               "lift_gbs": round((2 * m * k + m * kp + 4) / tl / 1e3, 1),
+                               "gemm_us": round(tg, 3),
+                               "gemm_gbs": round(bytes_sparse_gemm(m, n, kp) / tg / 1e3, 1),
+                               "gemm_tflops_dense_equiv": round(2 * m * n * k / tg / 1e6, 2)}
+            del layers
+            out[f"{2 * nn - 2}:{2 * nn}"] = res
+        return out
+
     def fusion_compare(self, reps=50):
         """For every M that the step runs fused: the fused launch against the
         activation kernel + GEMM pair it replaces, each as a CUDA graph of
@@ -621,6 +670,7 @@ def run_gpu(args, wl, rank, world, local_rank):
     compare = gw.dense_compare() if rank == 0 and not args.no_compare else None
     fusion = gw.fusion_compare() if rank == 0 and not args.no_compare else None
     finer = gw.finer_scales() if rank == 0 and not args.no_compare else None
+    general = gw.general_slide() if rank == 0 and not args.no_compare else None
     e2e_t, h2d, d2h = gw.e2e(args.steps)
     e2e_t = max_over_ranks(e2e_t, device)
     del g_timed, g_detail, g_warm
@@ -654,6 +704,7 @@ def run_gpu(args, wl, rank, world, local_rank):
         "sparse_vs_dense": compare,
         "fused_vs_unfused": fusion,
         "finer_scales": finer,
+        "general_slide": general,
         "e2e": {"value": round(aggregate_gbs(step_bytes, args.steps, world, e2e_t), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": gw.step_launches() * args.steps,

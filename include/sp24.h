@@ -257,6 +257,30 @@ int slide68_lift_gemm_packed(const void *X, int M, int N, int K, const void *pac
                              sp24_stream_t stream);
 
 /*
+ * The general (2N-2):2N case through 2:4 windows (SlideSparse, §2
+ * "Descomposicion de Ventana Deslizante": N-1 overlapping windows of 4 with
+ * stride 2 per 2N-group, expansion (2N-2)/N), for n = N = 3 (4:6), 4 (6:8,
+ * the same results as slide68_decompose / slide68_lift) or 5 (8:10).  Each
+ * 2n-group keeps its 2n-2 largest |w| (ties to the lower index); window j
+ * (positions 2j .. 2j+3) takes, for j = 0 .. n-2 in turn, the two
+ * lowest-index kept positions of its range not taken by an earlier window;
+ * position p of group g taken by window j goes to column 4((n-1)g + j) +
+ * (p - 2j) of W' [N, K' = K (2n-2)/n], stored 2:4-compressed with E4M3
+ * codes and the per-tensor w_scale: values [N, K'/2], meta [N, K'/8].
+ * slide_lift: X bf16 [M, K] -> q_lifted u8 [M, K'],
+ * q_lifted[m, 4((n-1)g + j) + r] = E4M3(X[m, 2n g + 2j + r] / scale), scale
+ * <- amax|X| / 448.  Workspace: sp24_workspace_size(SP24_OP_SLIDE68_DECOMPOSE
+ * or SP24_OP_SLIDE68_LIFT, ...) (256 bytes of counters).  Shape rules:
+ * 3 <= n <= 5, K % 2n == 0, K' % 16 == 0, rows * K % 8 == 0; the GEMM over
+ * K' (sp24_gemm, or sp24_gemm_packed after sp24_pack_weights) further needs
+ * K' % 128 == 0.
+ */
+int slide_decompose(const void *W, int N, int K, int n, uint8_t *values, uint8_t *meta, float *w_scale,
+                    void *workspace, size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+int slide_lift(const void *X, int M, int K, int n, uint8_t *q_lifted, float *scale, void *workspace,
+               size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+
+/*
  * Finer-grained scales (SlideSparse, §2 "Pipeline de Implementacion": its
  * fused quantiser scales each token; the roadmap, §Interaction avec la
  * quantification: finer scales for outlier layers).  The per-tensor rule of

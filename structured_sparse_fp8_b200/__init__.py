@@ -10,7 +10,7 @@ Entry points (same names as the C ABI):
     slide68_lift, sp24_gemm, fp8_gemm_dense, sp24_pack_weights,
     sp24_prune_compress_packed, slide68_decompose_packed, sp24_gemm_packed,
     sp24_quantize_gemm_packed, slide68_lift_gemm_packed, fp8_quantize_pertoken,
-    sp24_prune_compress_perchannel, sp24_gemm_packed_scaled
+    sp24_prune_compress_perchannel, sp24_gemm_packed_scaled, slide_decompose, slide_lift
 """
 from __future__ import annotations
 
@@ -24,6 +24,7 @@ __all__ = [
     "sp24_gemm", "fp8_gemm_dense", "sp24_pack_weights", "sp24_prune_compress_packed", "slide68_decompose_packed",
     "sp24_gemm_packed", "sp24_quantize_gemm_packed", "slide68_lift_gemm_packed",
     "fp8_quantize_pertoken", "sp24_prune_compress_perchannel", "sp24_gemm_packed_scaled",
+    "slide_decompose", "slide_lift",
     "Workspace",
     "Sp24Error", "DTYPE_E4M3", "DTYPE_BF16",
 ]
@@ -329,6 +330,56 @@ def slide68_lift_gemm_packed(X: torch.Tensor, packed: torch.Tensor, w_scale, n: 
     (Y bf16 [M, n], lifted codes u8 [M, K'], x_scale f32 [1])."""
     return _quant_gemm("slide68_lift_gemm_packed", _lib.OP_LIFT_GEMM_PACKED, lambda k: 3 * k // 2, X, packed,
                        w_scale, n, out, xq_out, x_scale_out, status, workspace)
+
+
+def _slide_kprime(k: int, n: int) -> int:
+    if k % (2 * n):
+        raise Sp24Error("K must be a multiple of 2n")
+    return k // (2 * n) * 4 * (n - 1)
+
+
+def slide_decompose(W: torch.Tensor, n: int, status: torch.Tensor | None = None,
+                    workspace: Workspace | None = None, out: dict | None = None):
+    """(2n-2):2n decomposition (n = 3, 4, 5) of W bf16 [N, K] into 2:4 E4M3 over
+    K' = K (2n-2)/n: returns dict(values [N, K'/2], meta [N, K'/8], scale);
+    ``out`` may supply any of these preallocated."""
+    lib = _lib.load()
+    out = out or {}
+    _require_cuda(W, status, *out.values())
+    if W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise Sp24Error("W must be a 2-D bf16 tensor")
+    N, K = W.shape
+    kp = _slide_kprime(K, n)
+    values = out.get("values")
+    values = values if values is not None else torch.empty((N, kp // 2), dtype=torch.uint8, device=W.device)
+    meta = out.get("meta")
+    meta = meta if meta is not None else torch.empty((N, kp // 8), dtype=torch.uint8, device=W.device)
+    scale = out.get("scale")
+    scale = scale if scale is not None else torch.empty((1,), dtype=torch.float32, device=W.device)
+    ws, wsn = _ws(W.device, _lib.OP_SLIDE68_DECOMPOSE, 0, N, K, DTYPE_E4M3, workspace)
+    rc = lib.slide_decompose(_ptr(W), N, K, n, _ptr(values), _ptr(meta), _ptr(scale), _ptr(ws), wsn,
+                             _ptr(status), _stream(W.device))
+    _lib.check(rc, "slide_decompose")
+    return dict(values=values, meta=meta, scale=scale)
+
+
+def slide_lift(X: torch.Tensor, n: int, status: torch.Tensor | None = None,
+               workspace: Workspace | None = None, out: torch.Tensor | None = None,
+               scale: torch.Tensor | None = None):
+    """Lift of X bf16 [M, K] to K' = K (2n-2)/n fused with per-tensor E4M3
+    quantisation: returns (codes u8 [M, K'], scale f32 [1])."""
+    lib = _lib.load()
+    _require_cuda(X, status, out, scale)
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise Sp24Error("X must be a 2-D bf16 tensor")
+    M, K = X.shape
+    kp = _slide_kprime(K, n)
+    q = out if out is not None else torch.empty((M, kp), dtype=torch.uint8, device=X.device)
+    sc = scale if scale is not None else torch.empty((1,), dtype=torch.float32, device=X.device)
+    ws, wsn = _ws(X.device, _lib.OP_SLIDE68_LIFT, M, 0, K, DTYPE_E4M3, workspace)
+    rc = lib.slide_lift(_ptr(X), M, K, n, _ptr(q), _ptr(sc), _ptr(ws), wsn, _ptr(status), _stream(X.device))
+    _lib.check(rc, "slide_lift")
+    return q, sc
 
 
 def fp8_quantize_pertoken(X: torch.Tensor, status: torch.Tensor | None = None,

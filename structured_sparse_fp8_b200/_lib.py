@@ -47,6 +47,8 @@ SIGNATURES = {
     "sp24_quantize_gemm_packed": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _sz, _p, _p]),
     "slide68_lift_gemm_packed": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _sz, _p, _p]),
     "fp8_quantize_pertoken": (_i, [_p, _i64, _i64, _p, _p, _p, _p]),
+    "slide_decompose": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _sz, _p, _p]),
+    "slide_lift": (_i, [_p, _i, _i, _i, _p, _p, _p, _sz, _p, _p]),
     "sp24_prune_compress_perchannel": (_i, [_p, _i, _i, _p, _p, _p, _p, _p]),
     "sp24_gemm_packed_scaled": (_i, [_p, _p, _i, _p, _p, _i, _p, _i, _i, _i, _p, _sz, _p, _p]),
     "sp24_workspace_size": (_sz, [_i, _i64, _i64, _i64, _i]),

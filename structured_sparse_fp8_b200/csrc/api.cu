@@ -304,6 +304,42 @@ int slide68_lift_gemm_packed(const void *X, int M, int N, int K, const void *pac
                            ws_bytes, status, stream);
 }
 
+// K' = K (2n - 2) / n for the (2n-2):2n decomposition; 0 when K does not fit.
+static int64_t slide_kprime(int64_t K, int n) {
+  if (n < 3 || n > 5 || K % (2 * n) != 0) return 0;
+  const int64_t kp = K / (2 * n) * 4 * (n - 1);
+  return kp % 16 == 0 ? kp : 0;
+}
+
+int slide_decompose(const void *W, int N, int K, int n, uint8_t *values, uint8_t *meta, float *w_scale,
+                    void *workspace, size_t ws_bytes, int32_t *status, sp24_stream_t stream) {
+  if (n == 4) return slide68_decompose(W, N, K, SP24_DTYPE_E4M3, values, meta, w_scale, workspace, ws_bytes,
+                                       status, stream);
+  if (!W || !values || !meta || !w_scale) return SP24_ERR_NULL;
+  if (N < 1 || slide_kprime(K, n) == 0 || (static_cast<int64_t>(N) * K) % 8 != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(values) || !aligned16(meta) || !aligned16(w_scale)) return SP24_ERR_ALIGN;
+  const int rc = check_workspace(workspace, ws_bytes);
+  if (rc != SP24_OK) return rc;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  return cuda_status(sp24::launch_slide_decompose(W, N, K, n, static_cast<uint32_t *>(workspace), w_scale, values,
+                                                  meta, status, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int slide_lift(const void *X, int M, int K, int n, uint8_t *q_lifted, float *scale, void *workspace,
+               size_t ws_bytes, int32_t *status, sp24_stream_t stream) {
+  if (n == 4) return slide68_lift(X, M, K, q_lifted, scale, workspace, ws_bytes, status, stream);
+  if (!X || !q_lifted || !scale) return SP24_ERR_NULL;
+  if (M < 1 || slide_kprime(K, n) == 0 || (static_cast<int64_t>(M) * K) % 8 != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(q_lifted) || !aligned16(scale)) return SP24_ERR_ALIGN;
+  const int rc = check_workspace(workspace, ws_bytes);
+  if (rc != SP24_OK) return rc;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  return cuda_status(sp24::launch_slide_lift(X, M, K, n, static_cast<uint32_t *>(workspace), scale, q_lifted,
+                                             status, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int fp8_quantize_pertoken(const void *X, int64_t rows, int64_t cols, uint8_t *q, float *scales,
                           int32_t *status, sp24_stream_t stream) {
   if (!X || !q || !scales) return SP24_ERR_NULL;

@@ -57,6 +57,12 @@ cudaError_t launch_quantize_pertoken(const void *x, int64_t rows, int64_t cols, 
 cudaError_t launch_prune24_perchannel(const void *w, int N, int K, uint8_t *values, uint8_t *meta,
                                       float *scales, int32_t *status, cudaStream_t st);
 
+// ---- slide.cu: general (2N-2):2N (N = 3, 5); `ws` as for the streamed kernels.
+cudaError_t launch_slide_decompose(const void *w, int N, int K, int n, uint32_t *ws, float *scale,
+                                   uint8_t *values, uint8_t *meta, int32_t *status, int sms, cudaStream_t st);
+cudaError_t launch_slide_lift(const void *x, int M, int K, int n, uint32_t *ws, float *scale, uint8_t *q,
+                              int32_t *status, int sms, cudaStream_t st);
+
 // Records the CUDA error reported by sp24_last_cuda_error() (api.cu).
 void set_last_cuda_error(int e);
 

@@ -113,12 +113,25 @@ def test_validation_rejects_bad_arguments_without_a_gpu(lib):
     gs = lib.sp24_gemm_packed_scaled
     assert gs(FAKE, FAKE, 1, FAKE, FAKE, 1, FAKE, 4, 192, 128, FAKE, big, None, None) == _lib.SP24_ERR_SHAPE
     assert gs(FAKE, None, 1, FAKE, FAKE, 1, FAKE, 4, 128, 128, FAKE, big, None, None) == _lib.SP24_ERR_NULL
+    # general (2n-2):2n: 3 <= n <= 5, K % 2n == 0, K' % 16 == 0
+    sd, sl = lib.slide_decompose, lib.slide_lift
+    assert sd(FAKE, 64, 120, 6, FAKE, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert sd(FAKE, 64, 120, 2, FAKE, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert sd(FAKE, 64, 100, 3, FAKE, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert sd(FAKE, 64, 66, 3, FAKE, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE  # K-prime 88
+    assert sd(FAKE, 0, 120, 5, FAKE, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert sd(FAKE, 64, 120, 3, FAKE, None, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_NULL
+    assert sl(FAKE, 0, 120, 3, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert sl(FAKE, 4, 125, 5, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert sl(FAKE, 4, 120, 5, None, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_NULL
     # alignment
     odd = ctypes.c_void_p((1 << 20) + 8)
     assert qg(FAKE, 4, 128, 128, FAKE, None, odd, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.fp8_quantize_pertoken(FAKE, 4, 16, odd, FAKE, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.sp24_prune_compress_packed(FAKE, 128, 128, odd, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.fp8_quantize_pertensor(odd, 4, 32, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
+    assert lib.slide_decompose(FAKE, 64, 120, 3, odd, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
+    assert lib.slide_lift(odd, 4, 120, 5, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.sp24_gemm(FAKE, None, odd, FAKE, None, FAKE, 4, 128, 128, 0, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
 
 

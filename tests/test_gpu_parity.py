@@ -701,3 +701,120 @@ def _scaled_check(m, n, k, x_vec, w_vec, seed):
 @pytest.mark.parametrize("x_vec,w_vec", [(True, True), (True, False), (False, True), (False, False)])
 def test_sparse_gemm_packed_scaled(m, n, k, x_vec, w_vec):
     _scaled_check(m, n, k, x_vec, w_vec, m + n)
+
+
+# ------------------------------------------------------------ general (2N-2):2N
+
+@pytest.mark.parametrize("n", [3, 5])
+@pytest.mark.parametrize("rows,k,dist", [(40, 120, "normal"), (33, 600, "ties"), (257, 1920, "student_t3")])
+def test_slide_decompose_bit_exact(n, rows, k, dist):
+    """4:6 and 8:10 windows: values, metadata and scale byte for byte (ragged
+    row counts; the ties case exercises the lower-index tie rule)."""
+    if (k // (2 * n) * 4 * (n - 1)) % 16:
+        pytest.skip("K' not a multiple of 16")
+    w = WL.random_bits((rows, k), 3100 + n, scale=0.02, dist=dist)
+    st = new_status()
+    d = sp().slide_decompose(dev_bf16(w), n, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = O.slide_decompose(w, n)
+    assert host(d["scale"])[0] == ref["scale"]
+    assert np.array_equal(host(d["meta"]), ref["meta"])
+    assert np.array_equal(host(d["values"]), ref["values"])
+
+
+@pytest.mark.parametrize("n", [3, 5])
+@pytest.mark.parametrize("m,k", [(1, 120), (7, 600), (300, 1920)])
+def test_slide_lift_bit_exact(n, m, k):
+    x = WL.random_bits((m, k), 3200 + n)
+    q, s = sp().slide_lift(dev_bf16(x), n)
+    ref_q, ref_s = O.slide_lift(x, n)
+    assert host(s)[0] == ref_s and np.array_equal(host(q), ref_q)
+
+
+@pytest.mark.parametrize("n,rows,k", [(3, 512, 1920), (5, 1024, 1920)])
+def test_slide_decompose_table_form_bit_exact(n, rows, k):
+    """Above 2 x 148 x 512 groups the kernel encodes through its shared-memory
+    code table instead of dividing: the whole tensor byte for byte, with
+    heavy-tailed values (codes across the table's band and tiny magnitudes in
+    its signed-zero region)."""
+    w = WL.random_bits((rows, k), 3500 + n, scale=0.02, dist="student_t3")
+    st = new_status()
+    d = sp().slide_decompose(dev_bf16(w), n, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = O.slide_decompose(w, n)
+    assert host(d["scale"])[0] == ref["scale"]
+    assert np.array_equal(host(d["meta"]), ref["meta"])
+    assert np.array_equal(host(d["values"]), ref["values"])
+
+
+@pytest.mark.parametrize("n,k", [(3, 4608), (5, 3840)])
+def test_slide_lift_table_form_bit_exact(n, k):
+    x = WL.random_bits((2048, k), 3600 + n, dist="student_t3")
+    q, s = sp().slide_lift(dev_bf16(x), n)
+    ref_q, ref_s = O.slide_lift(x, n)
+    assert host(s)[0] == ref_s and np.array_equal(host(q), ref_q)
+
+
+def test_slide_general_n4_is_the_68_path():
+    w = WL.random_bits((64, 512), 3300, scale=0.02, dist="ties")
+    x = WL.random_bits((5, 512), 3301)
+    d = sp().slide_decompose(dev_bf16(w), 4)
+    d68 = sp().slide68_decompose(dev_bf16(w), "e4m3")
+    q, s = sp().slide_lift(dev_bf16(x), 4)
+    q68, s68 = sp().slide68_lift(dev_bf16(x))
+    for key in ("values", "meta", "scale"):
+        assert torch.equal(d[key], d68[key]), key
+    assert torch.equal(q, q68) and torch.equal(s, s68)
+
+
+def test_slide_workspace_reused_across_calls():
+    """The counters return to zero: a second call on a smaller tensor through
+    the same workspace gives the oracle's scale, not the first call's amax."""
+    ws = sp().Workspace(torch.device(DEV))
+    big = WL.random_bits((64, 600), 3400, scale=4.0)
+    small = WL.random_bits((64, 600), 3401, scale=0.01)
+    sp().slide_decompose(dev_bf16(big), 3, workspace=ws)
+    d = sp().slide_decompose(dev_bf16(small), 3, workspace=ws)
+    _, s = sp().slide_lift(dev_bf16(small), 5, workspace=ws)
+    torch.cuda.synchronize()
+    assert host(d["scale"])[0] == O.slide_decompose(small, 3)["scale"]
+    assert host(s)[0] == O.slide_lift(small, 5)[1]
+
+
+@pytest.mark.parametrize("n,k", [(3, 4608), (5, 3840)])
+def test_slide_workload_gemm(n, k):
+    """The 4096-row layer with K chosen so that K' = 6144 for 4:6 and 8:10:
+    decompose (sampled rows checked byte for byte), lift (every code), GEMM
+    over K' (canonical and tile-packed) within tolerance on sampled rows."""
+    w, x = WL.weight_bits(5, k=k), WL.activation_bits(5, 64, k=k)
+    st = new_status()
+    d = sp().slide_decompose(dev_bf16(w), n, status=st)
+    xl, sxl = sp().slide_lift(dev_bf16(x), n, status=st)
+    y = sp().sp24_gemm(xl, sxl, d["values"], d["meta"], d["scale"], status=st)
+    packed = sp().sp24_pack_weights(d["values"], d["meta"])
+    yp = sp().sp24_gemm_packed(xl, sxl, packed, d["scale"], w.shape[0], status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    kp = k // (2 * n) * 4 * (n - 1)
+    assert kp == 6144
+    s = O.scale_from_amax(O.amax(w))
+    assert host(d["scale"])[0] == s
+    rows = np.sort(np.random.default_rng(56).choice(w.shape[0], size=32, replace=False))
+    ref = O.slide_decompose(w[rows], n)
+    codes = O.quantize_with_scale(w[rows], s)
+    rr, cc = np.nonzero(ref["emask"])
+    want = np.zeros_like(ref["expanded"], dtype=np.uint8)
+    want[rr, cc] = codes[rr, ref["src"][rr, cc]]
+    vals, meta = O.compress24(ref["emask"], want)
+    assert np.array_equal(host(d["meta"])[rows], meta)
+    assert np.array_equal(host(d["values"])[rows], vals)
+    ref_q, ref_s = O.slide_lift(x, n)
+    assert host(sxl)[0] == ref_s and np.array_equal(host(xl), ref_q)
+    # Y[:, rows] = X' W'[rows]^T, checked on the sampled output channels
+    y_ref, b = O.gemm_ref(O.e4m3_decode(ref_q), O.e4m3_decode(want), ref_s, s)
+    for yy, what in ((y, "canonical"), (yp, "packed")):
+        yh = host(yy)[:, rows]
+        assert_gemm_close(torch.from_numpy(np.ascontiguousarray(yh).view(np.int16)).view(torch.bfloat16),
+                          y_ref, b, f"{2 * n - 2}:{2 * n} {what}")

@@ -18,6 +18,8 @@ the function's docstring.  Pages cited:
   SlideSparse summary) -- Resumen tecnico §2 Metodologia: "Descomposicion de
   Ventana Deslizante", "Levantamiento de Activacion", "Pipeline de
   Implementacion"; the lay "Analogia de la Ventana Deslizante".
+* the cookbook's Comparison Tables ("INT8 W8A8" recipe) and the SlideSparse
+  summary's §3-§4 (INT8 among its precisions) for the INT8 functions.
 * "La Densite Dynamique et les Noyaux Non Structures ..." (the roadmap) --
   §Lacunes des noyaux (compressed metadata), §Interaction avec la
   quantification (per-tensor FP8 scaling).
@@ -449,6 +451,79 @@ def gemm_ref_scaled(x_vals: np.ndarray, w_vals: np.ndarray, sx: np.ndarray, sw: 
     b = np.broadcast_to(np.asarray(sw, dtype=np.float64).reshape(-1), (w.shape[0],))
     s = a[:, None] * b[None, :]
     return s * (x @ w.T), np.abs(s) * (np.abs(x) @ np.abs(w).T)
+
+
+# ---------------------------------------------------------------------------
+# INT8 W8A8 with 2:4 weights (the cookbook, Comparison Tables: the "INT8 W8A8"
+# recipe; the SlideSparse summary, §3 Contribuciones Clave: INT8 among the
+# supported precisions, and §4: its end-to-end result measured in INT8)
+# ---------------------------------------------------------------------------
+
+INT8_MAX = 127
+
+
+def int8_scale_from_amax(a: np.float32) -> np.float32:
+    """Symmetric per-tensor INT8 scale s = amax / 127, one fp32 division; 1.0
+    when amax is 0.
+
+    Reading: the pages name the recipe but give no formula; the plainest one
+    is the E4M3 rule with the INT8 grid: a symmetric range [-127, 127] (no
+    zero point, -128 unused) and the largest magnitude mapped to 127.
+    """
+    a = np.float32(a)
+    if a == 0:
+        return np.float32(1.0)
+    return np.float32(a / np.float32(INT8_MAX))
+
+
+def int8_quantize_with_scale(bits: np.ndarray, s: np.float32) -> np.ndarray:
+    """INT8 codes q = clamp(round_half_even(RN_fp32(x / s)), -127, 127).
+
+    The quotient is one correctly rounded fp32 division, as for E4M3; it is
+    then rounded to the nearest integer, ties to even.  The clamp only
+    matters where the fp32 quotient of the largest element lands a rounding
+    error above 127.
+    """
+    x = bf16_to_f32(bits)
+    _require_finite(x, "int8 quantisation")
+    v = (x / np.float32(s)).astype(np.float32)
+    return np.clip(np.rint(v), -INT8_MAX, INT8_MAX).astype(np.int8)
+
+
+def int8_quantize_pertensor(bits: np.ndarray):
+    """Per-tensor dynamic INT8 quantisation: returns (codes int8, scale)."""
+    s = int8_scale_from_amax(amax(bits))
+    return int8_quantize_with_scale(bits, s), s
+
+
+def sp24_prune_compress_int8(w_bits: np.ndarray):
+    """The 2:4 weight path with INT8 codes: the same selection (ranking the
+    bf16 magnitudes, ties to the lower index) and layout as
+    sp24_prune_compress, each kept value stored as its INT8 code under the
+    per-tensor scale.  Returns a dict with ``values`` (int8 [N, K/2]),
+    ``meta``, ``mask``, ``scale`` and ``pruned_dense`` (int8, 0 where pruned).
+    """
+    w_bits = np.asarray(w_bits, dtype=np.uint16)
+    mask = prune24_mask(w_bits)
+    s = int8_scale_from_amax(amax(w_bits))
+    codes = int8_quantize_with_scale(w_bits, s)
+    dense = np.where(mask, codes, np.int8(0)).astype(np.int8)
+    vals, meta = compress24(mask, codes)
+    return dict(values=vals.astype(np.int8), meta=meta, mask=mask, scale=s, pruned_dense=dense)
+
+
+def gemm_ref_int8(xq: np.ndarray, wq: np.ndarray, sx=1.0, sw=1.0):
+    """INT8 GEMM: the exact integer sums acc[m, n] = sum_k xq[m, k] wq[n, k]
+    (int64; every partial sum of the shapes used fits int32), then
+    Y = sx * sw * acc in float64 and the bound B = |sx * sw| * sum_k
+    |xq wq|.  ``wq`` is the dense [N, K] code array (0 at pruned positions).
+    Returns (Y, B, acc).
+    """
+    x = np.asarray(xq, dtype=np.int64)
+    w = np.asarray(wq, dtype=np.int64)
+    acc = x @ w.T
+    s = float(np.float64(sx) * np.float64(sw))
+    return s * acc.astype(np.float64), abs(s) * (np.abs(x) @ np.abs(w).T).astype(np.float64), acc
 
 
 # ---------------------------------------------------------------------------

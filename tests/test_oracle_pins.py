@@ -417,3 +417,82 @@ def test_general_slide_reconstructs_and_gemm_is_exact(n):
     y1, _ = O.gemm_ref(O.e4m3_decode(xl), O.e4m3_decode(d["expanded"]))
     y2, _ = O.gemm_ref(O.e4m3_decode(xq), O.e4m3_decode(back))
     assert np.array_equal(y1, y2)
+
+
+# ------------------------------------------------------------ INT8 W8A8 with 2:4 weights
+
+def test_int8_golden_hand_example():
+    lines = [ln.split() for ln in open(os.path.join(GOLDEN, "int8_hand_example.txt"))
+             if ln.strip() and not ln.startswith("#")]
+    for vals, codes, scale in ((lines[0], lines[1], lines[2]), (lines[3], lines[4], lines[5])):
+        bits = WL.to_bf16_bits(np.array([float(v) for v in vals]))[None, :]
+        q, s = O.int8_quantize_pertensor(bits)
+        assert float(s) == float(scale[0])
+        assert q[0].tolist() == [int(c) for c in codes]
+
+
+def test_int8_matches_torch_quantizer_away_from_rounding_ties():
+    """torch's per-tensor qint8 quantiser (zero point 0) rounds x / s to the
+    nearest integer on its own code path; it multiplies by the reciprocal of
+    s, so the comparison leaves out quotients within 1e-5 of a half-integer."""
+    x = WL.random_bits((64, 512), 4000, dist="student_t3")
+    q, s = O.int8_quantize_pertensor(x)
+    xf = O.bf16_to_f32(x)
+    tq = torch.quantize_per_tensor(torch.from_numpy(xf), float(s), 0, torch.qint8).int_repr().numpy()
+    r = xf.astype(np.float64) / float(s)
+    far = np.abs(np.abs(r - np.floor(r)) - 0.5) > 1e-5
+    assert far.mean() > 0.99
+    assert np.array_equal(q[far], tq[far])
+
+
+def test_int8_every_bf16_value_within_half_a_step():
+    """Every finite bf16 value with |x| <= amax = 3: the code is within half a
+    step of x / s (plus the fp32 quotient's rounding), exact half-way cases go
+    to the even code, |q| <= 127 and +-amax code to +-127."""
+    s = O.int8_scale_from_amax(np.float32(3.0))
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    x = O.bf16_to_f32(bits)
+    sel = np.isfinite(x) & (np.abs(x) <= 3.0)
+    q = O.int8_quantize_with_scale(bits[sel], s).astype(np.int64)
+    r = x[sel].astype(np.float64) / np.float64(s)
+    assert (np.abs(q - r) <= 0.5 + 2.0 ** -23 * np.abs(r) + 1e-12).all()
+    half = (2 * r == np.round(2 * r)) & (r != np.round(r))
+    assert (q[half] % 2 == 0).all()
+    assert np.abs(q).max() == 127
+    ends = O.int8_quantize_with_scale(WL.to_bf16_bits(np.array([[3.0, -3.0]])), s)
+    assert ends.tolist() == [[127, -127]]
+
+
+def test_int8_zero_tensor_and_dequantisation_error():
+    q, s = O.int8_quantize_pertensor(np.zeros((4, 16), dtype=np.uint16))
+    assert s == np.float32(1.0) and not q.any()
+    x = WL.random_bits((32, 256), 4050)
+    q, s = O.int8_quantize_pertensor(x)
+    err = np.abs(q.astype(np.float64) * np.float64(s) - O.bf16_to_f32(x).astype(np.float64))
+    assert (err <= 0.5 * np.float64(s) * (1 + 1e-6)).all()
+
+
+def test_int8_prune_compress_selects_like_fp8():
+    w = WL.random_bits((64, 256), 4100, scale=0.02, dist="ties")
+    d = O.sp24_prune_compress_int8(w)
+    ref = O.sp24_prune_compress(w, "e4m3")
+    assert np.array_equal(d["mask"], ref["mask"]) and np.array_equal(d["meta"], ref["meta"])
+    assert np.array_equal(O.decompress24(d["values"], d["meta"], 256), d["pruned_dense"])
+    q, s = O.int8_quantize_pertensor(w)
+    assert s == d["scale"]
+    assert np.array_equal(np.where(d["mask"], q, 0), d["pruned_dense"])
+
+
+def test_int8_gemm_is_the_exact_integer_product():
+    """The integer sums equal a walk over the compressed operand in plain
+    loops (the pinned format), Y and B equal the pinned float64 reference on
+    the same integers, and the largest K used keeps every sum inside int32."""
+    x = WL.random_bits((3, 64), 4200)
+    w = WL.random_bits((5, 64), 4201, scale=0.02)
+    xq, sx = O.int8_quantize_pertensor(x)
+    d = O.sp24_prune_compress_int8(w)
+    y, b, acc = O.gemm_ref_int8(xq, d["pruned_dense"], sx, d["scale"])
+    assert np.array_equal(O.sparse_gemm_walk(xq, d["values"], d["meta"]), acc.astype(np.float64))
+    y2, b2 = O.gemm_ref(xq, d["pruned_dense"], sx, d["scale"])
+    assert np.array_equal(y, y2) and np.array_equal(b, b2)
+    assert 14336 // 2 * 127 * 127 < 2 ** 31

@@ -257,6 +257,28 @@ int slide68_lift_gemm_packed(const void *X, int M, int N, int K, const void *pac
                              sp24_stream_t stream);
 
 /*
+ * INT8 W8A8 with 2:4 weights (the cookbook, Comparison Tables: the "INT8
+ * W8A8" recipe; SlideSparse, §3 "Contribuciones Clave": INT8 among the
+ * supported precisions).  Symmetric per-tensor scales: s = amax / 127 (1.0
+ * for an all-zero tensor), q = clamp(round_half_even(RN_fp32(x / s)),
+ * -127, 127).
+ * int8_quantize_pertensor: X bf16 [rows, cols] (cols % 16 == 0) -> q int8
+ *   [rows, cols], *scale <- s.
+ * sp24_prune_compress_int8: W bf16 [N, K] (K % 8 == 0) -> the 2:4 selection
+ *   of sp24_prune_compress (two largest |w| per group of 4, ties to the lower
+ *   index) in the canonical layout with INT8 codes: values int8 [N, K/2],
+ *   meta [N, K/8], *w_scale <- s.
+ * Pointers are device pointers, 16-byte aligned (scale: 4-byte).  Workspace:
+ * sp24_workspace_size(SP24_OP_QUANTIZE or SP24_OP_PRUNE_COMPRESS, ...)
+ * (256 bytes of counters, zero before and after the call).  Errors as for
+ * the E4M3 calls; SP24_STATUS_NONFINITE when the input holds Inf or NaN.
+ */
+int int8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, int8_t *q, float *scale, void *workspace,
+                            size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+int sp24_prune_compress_int8(const void *W, int N, int K, int8_t *values, uint8_t *meta, float *w_scale,
+                             void *workspace, size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+
+/*
  * The general (2N-2):2N case through 2:4 windows (SlideSparse, §2
  * "Descomposicion de Ventana Deslizante": N-1 overlapping windows of 4 with
  * stride 2 per 2N-group, expansion (2N-2)/N), for n = N = 3 (4:6), 4 (6:8,

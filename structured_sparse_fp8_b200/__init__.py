@@ -10,7 +10,8 @@ Entry points (same names as the C ABI):
     slide68_lift, sp24_gemm, fp8_gemm_dense, sp24_pack_weights,
     sp24_prune_compress_packed, slide68_decompose_packed, sp24_gemm_packed,
     sp24_quantize_gemm_packed, slide68_lift_gemm_packed, fp8_quantize_pertoken,
-    sp24_prune_compress_perchannel, sp24_gemm_packed_scaled, slide_decompose, slide_lift
+    sp24_prune_compress_perchannel, sp24_gemm_packed_scaled, slide_decompose, slide_lift,
+    int8_quantize_pertensor, sp24_prune_compress_int8
 """
 from __future__ import annotations
 
@@ -24,7 +25,7 @@ __all__ = [
     "sp24_gemm", "fp8_gemm_dense", "sp24_pack_weights", "sp24_prune_compress_packed", "slide68_decompose_packed",
     "sp24_gemm_packed", "sp24_quantize_gemm_packed", "slide68_lift_gemm_packed",
     "fp8_quantize_pertoken", "sp24_prune_compress_perchannel", "sp24_gemm_packed_scaled",
-    "slide_decompose", "slide_lift",
+    "slide_decompose", "slide_lift", "int8_quantize_pertensor", "sp24_prune_compress_int8",
     "Workspace",
     "Sp24Error", "DTYPE_E4M3", "DTYPE_BF16",
 ]
@@ -137,6 +138,48 @@ def fp8_quantize_pertensor(X: torch.Tensor, status: torch.Tensor | None = None,
                                     _ptr(status), _stream(X.device))
     _lib.check(rc, "fp8_quantize_pertensor")
     return q, s
+
+
+def int8_quantize_pertensor(X: torch.Tensor, status: torch.Tensor | None = None,
+                            out: torch.Tensor | None = None, scale: torch.Tensor | None = None,
+                            workspace: Workspace | None = None):
+    """Symmetric per-tensor INT8 quantisation of X bf16 [rows, cols] -> (codes int8, scale f32[1])."""
+    lib = _lib.load()
+    _require_cuda(X, status, out, scale)
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise Sp24Error("X must be a 2-D bf16 tensor")
+    rows, cols = X.shape
+    q = out if out is not None else torch.empty((rows, cols), dtype=torch.int8, device=X.device)
+    s = scale if scale is not None else torch.empty((1,), dtype=torch.float32, device=X.device)
+    ws, wsn = _ws(X.device, _lib.OP_QUANTIZE, rows, 0, cols, DTYPE_E4M3, workspace)
+    rc = lib.int8_quantize_pertensor(_ptr(X), rows, cols, _ptr(q), _ptr(s), _ptr(ws), wsn,
+                                     _ptr(status), _stream(X.device))
+    _lib.check(rc, "int8_quantize_pertensor")
+    return q, s
+
+
+def sp24_prune_compress_int8(W: torch.Tensor, status: torch.Tensor | None = None,
+                             workspace: Workspace | None = None, out: dict | None = None):
+    """2:4 magnitude prune + symmetric per-tensor INT8 quantise + compress of
+    W bf16 [N, K]: returns dict(values int8 [N, K/2], meta u8 [N, K/8], scale);
+    ``out`` may supply any of these preallocated."""
+    lib = _lib.load()
+    out = out or {}
+    _require_cuda(W, status, *out.values())
+    if W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise Sp24Error("W must be a 2-D bf16 tensor")
+    N, K = W.shape
+    values = out.get("values")
+    values = values if values is not None else torch.empty((N, K // 2), dtype=torch.int8, device=W.device)
+    meta = out.get("meta")
+    meta = meta if meta is not None else torch.empty((N, K // 8), dtype=torch.uint8, device=W.device)
+    scale = out.get("scale")
+    scale = scale if scale is not None else torch.empty((1,), dtype=torch.float32, device=W.device)
+    ws, wsn = _ws(W.device, _lib.OP_PRUNE_COMPRESS, 0, N, K, DTYPE_E4M3, workspace)
+    rc = lib.sp24_prune_compress_int8(_ptr(W), N, K, _ptr(values), _ptr(meta), _ptr(scale), _ptr(ws), wsn,
+                                      _ptr(status), _stream(W.device))
+    _lib.check(rc, "sp24_prune_compress_int8")
+    return dict(values=values, meta=meta, scale=scale)
 
 
 def slide68_decompose(W: torch.Tensor, out_dtype="e4m3", status: torch.Tensor | None = None,

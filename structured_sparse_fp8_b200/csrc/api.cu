@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "int8_kernels.h"
 #include "kernels.h"
 #include "sp24.h"
 
@@ -175,6 +176,33 @@ int fp8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, uint8_t *q
   if (rc != SP24_OK) return rc;
   return cuda_status(sp24::launch_quantize_fused(X, nelem, static_cast<uint32_t *>(workspace), scale,
                                                  q, status, sms, st));
+}
+
+int int8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, int8_t *q, float *scale, void *workspace,
+                            size_t ws_bytes, int32_t *status, sp24_stream_t stream) {
+  if (!X || !q || !scale) return SP24_ERR_NULL;
+  if (rows < 1 || cols < 1 || cols % 16 != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(q)) return SP24_ERR_ALIGN;
+  const int rc = check_workspace(workspace, ws_bytes);
+  if (rc != SP24_OK) return rc;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  return cuda_status(sp24::launch_int8_quantize(X, rows * cols, static_cast<uint32_t *>(workspace), scale, q,
+                                                status, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sp24_prune_compress_int8(const void *W, int N, int K, int8_t *values, uint8_t *meta, float *w_scale,
+                             void *workspace, size_t ws_bytes, int32_t *status, sp24_stream_t stream) {
+  if (!W || !values || !meta || !w_scale) return SP24_ERR_NULL;
+  if (N < 1 || K < 8 || K % 8 != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(values) || !aligned16(meta)) return SP24_ERR_ALIGN;
+  const int rc = check_workspace(workspace, ws_bytes);
+  if (rc != SP24_OK) return rc;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  return cuda_status(sp24::launch_int8_prune24(W, static_cast<int64_t>(N) * K, static_cast<uint32_t *>(workspace),
+                                               w_scale, values, meta, status, sms,
+                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int slide68_decompose(const void *W, int N, int K, int out_dtype, void *values, uint8_t *meta,

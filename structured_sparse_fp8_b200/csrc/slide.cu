@@ -27,6 +27,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "amax_cta.cuh"
 #include "kernels.h"
 #include "quant_common.cuh"
 #include "sp24.h"
@@ -37,31 +38,9 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kCtasPerSm = 2;
-constexpr int kBatch = 4;          // groups (amax: 16-byte vectors) per thread per pass
+constexpr int kBatch = 4;          // groups per thread per pass (table form)
 constexpr int kTabBytes = 65536;   // one code per bf16 bit pattern
 constexpr int kBand = 24;          // binades at and below amax's that can give a nonzero code
-
-// ws[0] <- max(ws[0], amax bits of x); x has nvec 8-element vectors.
-__global__ void __launch_bounds__(kThreads) bf16_amax_kernel(const uint4 *__restrict__ x, int64_t nvec, uint32_t *ws) {
-  __shared__ uint32_t s_red[kThreads / 32];
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  uint32_t m2 = 0;
-  for (int64_t v = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; v < nvec; v += stride * kBatch) {
-    uint4 w[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u)
-      w[u] = v + stride * u < nvec ? __ldg(x + v + stride * u) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) m2 = __vmaxu2(m2, absmax8x2(w[u]));
-  }
-  const uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
-  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = mx;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    const uint32_t r = __reduce_max_sync(0xFFFFFFFFu, threadIdx.x < kThreads / 32 ? s_red[threadIdx.x] : 0u);
-    if (threadIdx.x == 0) atomicMax(&ws[0], r);
-  }
-}
 
 // The E4M3 code of a bf16 pattern h (16 bits) under the scale s: from the
 // table, or (DIRECT) by the division.
@@ -260,13 +239,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
 int64_t grid_cap(int sms) { return static_cast<int64_t>(kCtasPerSm) * sms; }
 
-unsigned amax_grid(int64_t nvec, int sms) {
-  const int64_t per = static_cast<int64_t>(kThreads) * kBatch;
-  int64_t g = (nvec + per - 1) / per;
-  if (g > grid_cap(sms)) g = grid_cap(sms);
-  return static_cast<unsigned>(g < 1 ? 1 : g);
-}
-
 // The direct form when one group per thread fits the bounded grid.
 bool direct_form(int64_t groups, int sms) { return groups <= grid_cap(sms) * kThreads; }
 
@@ -326,8 +298,8 @@ cudaError_t launch_lift_form(const uint32_t *x, int64_t groups, uint32_t *ws, fl
 cudaError_t launch_slide_decompose(const void *w, int N, int K, int n, uint32_t *ws, float *scale,
                                    uint8_t *values, uint8_t *meta, int32_t *status, int sms, cudaStream_t st) {
   if (n != 3 && n != 5) return cudaErrorInvalidValue;
-  const int64_t nvec = static_cast<int64_t>(N) * K / 8;
-  bf16_amax_kernel<<<amax_grid(nvec, sms), kThreads, 0, st>>>(static_cast<const uint4 *>(w), nvec, ws);
+  const cudaError_t e = launch_bf16_amax(w, static_cast<int64_t>(N) * K / 8, ws, grid_cap(sms), st);
+  if (e != cudaSuccess) return e;
   const int64_t groups = static_cast<int64_t>(N) * (K / (2 * n));
   const uint32_t *ww = static_cast<const uint32_t *>(w);
   return n == 3 ? launch_decompose_form<3>(ww, groups, ws, scale, values, meta, status, sms, st)
@@ -337,8 +309,8 @@ cudaError_t launch_slide_decompose(const void *w, int N, int K, int n, uint32_t 
 cudaError_t launch_slide_lift(const void *x, int M, int K, int n, uint32_t *ws, float *scale, uint8_t *q,
                               int32_t *status, int sms, cudaStream_t st) {
   if (n != 3 && n != 5) return cudaErrorInvalidValue;
-  const int64_t nvec = static_cast<int64_t>(M) * K / 8;
-  bf16_amax_kernel<<<amax_grid(nvec, sms), kThreads, 0, st>>>(static_cast<const uint4 *>(x), nvec, ws);
+  const cudaError_t e = launch_bf16_amax(x, static_cast<int64_t>(M) * K / 8, ws, grid_cap(sms), st);
+  if (e != cudaSuccess) return e;
   const int64_t groups = static_cast<int64_t>(M) * (K / (2 * n));
   const uint32_t *xx = static_cast<const uint32_t *>(x);
   return n == 3 ? launch_lift_form<3>(xx, groups, ws, scale, q, status, sms, st)

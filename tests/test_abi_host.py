@@ -124,6 +124,12 @@ def test_validation_rejects_bad_arguments_without_a_gpu(lib):
     assert sl(FAKE, 0, 120, 3, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
     assert sl(FAKE, 4, 125, 5, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
     assert sl(FAKE, 4, 120, 5, None, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_NULL
+    # INT8: cols % 16 (activations), K % 8 (weights)
+    assert lib.int8_quantize_pertensor(FAKE, 4, 24, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.int8_quantize_pertensor(FAKE, 0, 32, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.int8_quantize_pertensor(FAKE, 4, 32, FAKE, None, FAKE, ws, None, None) == _lib.SP24_ERR_NULL
+    assert lib.sp24_prune_compress_int8(FAKE, 4, 12, FAKE, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
+    assert lib.sp24_prune_compress_int8(FAKE, 4, 16, FAKE, FAKE, None, FAKE, ws, None, None) == _lib.SP24_ERR_NULL
     # alignment
     odd = ctypes.c_void_p((1 << 20) + 8)
     assert qg(FAKE, 4, 128, 128, FAKE, None, odd, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_ALIGN
@@ -132,6 +138,8 @@ def test_validation_rejects_bad_arguments_without_a_gpu(lib):
     assert lib.fp8_quantize_pertensor(odd, 4, 32, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.slide_decompose(FAKE, 64, 120, 3, odd, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.slide_lift(odd, 4, 120, 5, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
+    assert lib.int8_quantize_pertensor(FAKE, 4, 32, odd, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
+    assert lib.sp24_prune_compress_int8(FAKE, 4, 16, FAKE, odd, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.sp24_gemm(FAKE, None, odd, FAKE, None, FAKE, 4, 128, 128, 0, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
 
 

@@ -818,3 +818,33 @@ def test_slide_workload_gemm(n, k):
         yh = host(yy)[:, rows]
         assert_gemm_close(torch.from_numpy(np.ascontiguousarray(yh).view(np.int16)).view(torch.bfloat16),
                           y_ref, b, f"{2 * n - 2}:{2 * n} {what}")
+
+
+# ------------------------------------------------------------ INT8 W8A8 (2:4 weights)
+
+@pytest.mark.parametrize("rows,cols,dist", [(1, 16, "normal"), (7, 48, "ties"), (300, 1920, "student_t3"),
+                                            (2048, 4096, "student_t3")])
+def test_int8_quantize_bit_exact(rows, cols, dist):
+    """Codes and scale byte for byte: the division form for the small cases,
+    the code-table form for X[2048,4096] (above 2 x 148 x 512 vectors of 8);
+    the tie-heavy case puts fp32 quotients next to half-integers."""
+    x = WL.random_bits((rows, cols), 4300 + rows, dist=dist)
+    st = new_status()
+    q, s = sp().int8_quantize_pertensor(dev_bf16(x), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref_q, ref_s = O.int8_quantize_pertensor(x)
+    assert host(s)[0] == ref_s and np.array_equal(host(q), ref_q)
+
+
+@pytest.mark.parametrize("n,k,dist", [(40, 120, "ties"), (257, 1920, "normal"), (1024, 2048, "student_t3")])
+def test_int8_prune_compress_bit_exact(n, k, dist):
+    w = WL.random_bits((n, k), 4400 + n, scale=0.02, dist=dist)
+    st = new_status()
+    d = sp().sp24_prune_compress_int8(dev_bf16(w), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = O.sp24_prune_compress_int8(w)
+    assert host(d["scale"])[0] == ref["scale"]
+    assert np.array_equal(host(d["meta"]), ref["meta"])
+    assert np.array_equal(host(d["values"]), ref["values"])

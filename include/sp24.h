@@ -17,7 +17,10 @@
  * (2N-2):2N Structured Sparsity", Resumen tecnico §2 Metodologia): each
  * 8-group is split into three overlapping stride-2 windows that are each
  * 2:4 over a lifted K' = 1.5 K, and the activation lift is fused into the
- * FP8 quantisation pass.
+ * FP8 quantisation pass.  Beyond that path: the fused quantise + GEMM forms
+ * for decode, per-token and per-channel scales, the general (2N-2):2N
+ * decomposition for N = 3 and 5, and the INT8 W8A8 quantisers (each
+ * declared with its own citation below).
  *
  * Conventions for every entry point
  * ---------------------------------

@@ -496,3 +496,30 @@ def test_int8_gemm_is_the_exact_integer_product():
     y2, b2 = O.gemm_ref(xq, d["pruned_dense"], sx, d["scale"])
     assert np.array_equal(y, y2) and np.array_equal(b, b2)
     assert 14336 // 2 * 127 * 127 < 2 ** 31
+
+
+def _golden_cases(name):
+    cases, cur = [], None
+    for ln in open(os.path.join(GOLDEN, name)):
+        if not ln.strip() or ln.startswith("#"):
+            continue
+        key, *rest = ln.split()
+        if key == "n":
+            cur = {"n": int(rest[0])}
+            cases.append(cur)
+        else:
+            cur[key] = rest
+    return cases
+
+
+def test_general_slide_golden_hand_examples():
+    for c in _golden_cases("slide_general_hand_example.txt"):
+        n = c["n"]
+        w = WL.to_bf16_bits(np.array([[float(v) for v in c["w"]]]))
+        assert np.nonzero(O.slide_mask(w, n)[0])[0].tolist() == [int(v) for v in c["kept"]]
+        pairs = [tuple(int(p) for p in wp.split(",")) for wp in c["windows"]]
+        assert O.slide_windows(O.slide_mask(w, n)[0], n) == pairs
+        d = O.slide_decompose(w, n)
+        assert d["meta"][0].tolist() == [int(b, 16) for b in c["meta"]]
+        assert d["src"][0][d["emask"][0]].tolist() == [int(v) for v in c["src"]]
+        assert O.slide_lift_columns(2 * n, n).tolist() == [int(v) for v in c["lift"]]

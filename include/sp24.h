@@ -19,8 +19,8 @@
  * 2:4 over a lifted K' = 1.5 K, and the activation lift is fused into the
  * FP8 quantisation pass.  Beyond that path: the fused quantise + GEMM forms
  * for decode, per-token and per-channel scales, the general (2N-2):2N
- * decomposition for N = 3 and 5, and the INT8 W8A8 quantisers (each
- * declared with its own citation below).
+ * decomposition for N = 3 and 5, and INT8 W8A8 (quantisers and the sparse
+ * GEMM; each declared with its own citation below).
  *
  * Conventions for every entry point
  * ---------------------------------
@@ -280,6 +280,19 @@ int int8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, int8_t *q
                             size_t ws_bytes, int32_t *status, sp24_stream_t stream);
 int sp24_prune_compress_int8(const void *W, int N, int K, int8_t *values, uint8_t *meta, float *w_scale,
                              void *workspace, size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+/*
+ * The INT8 W8A8 sparse GEMM: Y[M, N] = x_scale * w_scale * (Xq . W^T), the
+ * integer products summed exactly in the tensor cores' s32 accumulators
+ * (kind::i8) and converted to fp32 in the epilogue, bf16 out.  Xq: int8
+ * [M, K] from int8_quantize_pertensor; packed: sp24_pack_weights applied to
+ * the values (int8, as bytes) and metadata of sp24_prune_compress_int8;
+ * scales: one device float each.  Shape rules, workspace
+ * (sp24_workspace_size(SP24_OP_GEMM_PACKED, M, N, K, 0)) and errors as for
+ * sp24_gemm_packed.
+ */
+int sp24_gemm_int8_packed(const int8_t *Xq, const float *x_scale, const void *packed, const float *w_scale,
+                          void *Y, int M, int N, int K, void *workspace, size_t ws_bytes, int32_t *status,
+                          sp24_stream_t stream);
 
 /*
  * The general (2N-2):2N case through 2:4 windows (SlideSparse, §2

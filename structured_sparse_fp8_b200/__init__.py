@@ -11,7 +11,7 @@ Entry points (same names as the C ABI):
     sp24_prune_compress_packed, slide68_decompose_packed, sp24_gemm_packed,
     sp24_quantize_gemm_packed, slide68_lift_gemm_packed, fp8_quantize_pertoken,
     sp24_prune_compress_perchannel, sp24_gemm_packed_scaled, slide_decompose, slide_lift,
-    int8_quantize_pertensor, sp24_prune_compress_int8
+    int8_quantize_pertensor, sp24_prune_compress_int8, sp24_gemm_int8_packed
 """
 from __future__ import annotations
 
@@ -26,6 +26,7 @@ __all__ = [
     "sp24_gemm_packed", "sp24_quantize_gemm_packed", "slide68_lift_gemm_packed",
     "fp8_quantize_pertoken", "sp24_prune_compress_perchannel", "sp24_gemm_packed_scaled",
     "slide_decompose", "slide_lift", "int8_quantize_pertensor", "sp24_prune_compress_int8",
+    "sp24_gemm_int8_packed",
     "Workspace",
     "Sp24Error", "DTYPE_E4M3", "DTYPE_BF16",
 ]
@@ -329,6 +330,27 @@ def sp24_gemm_packed(xq: torch.Tensor, x_scale, packed: torch.Tensor, w_scale, n
     rc = lib.sp24_gemm_packed(_ptr(xq), _ptr(x_scale), _ptr(packed), _ptr(w_scale), _ptr(y), M, n, K,
                               _ptr(ws), wsn, _ptr(status), _stream(xq.device))
     _lib.check(rc, "sp24_gemm_packed")
+    return y
+
+
+def sp24_gemm_int8_packed(xq: torch.Tensor, x_scale, packed: torch.Tensor, w_scale, n: int,
+                          out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                          workspace: Workspace | None = None):
+    """INT8 W8A8 sparse GEMM: xq int8 [M, K], tile-packed INT8 2:4 weights
+    (sp24_pack_weights of sp24_prune_compress_int8's values viewed as bytes,
+    and its metadata) -> Y bf16 [M, n]."""
+    lib = _lib.load()
+    _require_cuda(xq, x_scale, packed, w_scale, out, status)
+    if xq.dtype != torch.int8 or xq.dim() != 2:
+        raise Sp24Error("xq must be a 2-D int8 tensor")
+    M, K = xq.shape
+    if packed.numel() != n * K // 2 + n * K // 8:
+        raise Sp24Error("packed weights do not match N x K")
+    y = out if out is not None else torch.empty((M, n), dtype=torch.bfloat16, device=xq.device)
+    ws, wsn = _ws(xq.device, _lib.OP_GEMM_PACKED, M, n, K, DTYPE_E4M3, workspace)
+    rc = lib.sp24_gemm_int8_packed(_ptr(xq), _ptr(x_scale), _ptr(packed), _ptr(w_scale), _ptr(y), M, n, K,
+                                   _ptr(ws), wsn, _ptr(status), _stream(xq.device))
+    _lib.check(rc, "sp24_gemm_int8_packed")
     return y
 
 

@@ -50,6 +50,7 @@ SIGNATURES = {
     "slide_decompose": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _sz, _p, _p]),
     "int8_quantize_pertensor": (_i, [_p, _i64, _i64, _p, _p, _p, _sz, _p, _p]),
     "sp24_prune_compress_int8": (_i, [_p, _i, _i, _p, _p, _p, _p, _sz, _p, _p]),
+    "sp24_gemm_int8_packed": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _sz, _p, _p]),
     "slide_lift": (_i, [_p, _i, _i, _i, _p, _p, _p, _sz, _p, _p]),
     "sp24_prune_compress_perchannel": (_i, [_p, _i, _i, _p, _p, _p, _p, _p]),
     "sp24_gemm_packed_scaled": (_i, [_p, _p, _i, _p, _p, _i, _p, _i, _i, _i, _p, _sz, _p, _p]),

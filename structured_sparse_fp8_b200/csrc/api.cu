@@ -244,7 +244,7 @@ static int gemm_common(sp24::GemmKind kind, const void *Xq, const float *x_scale
                        const void *w_values, const uint8_t *w_meta, const float *w_scale, void *Y,
                        int M, int N, int K, void *workspace, size_t ws_bytes, int32_t *status,
                        sp24_stream_t stream) {
-  const bool sparse = kind != sp24::kDenseE4M3 && kind != sp24::kSparseE4M3Packed;
+  const bool sparse = kind != sp24::kDenseE4M3 && kind != sp24::kSparseE4M3Packed && kind != sp24::kSparseI8Packed;
   if (!Xq || !w_values || !Y || (sparse && !w_meta)) return SP24_ERR_NULL;
   const int kmod = 128;
   if (M < 1 || N < 128 || N % 128 != 0 || K < kmod || K % kmod != 0) return SP24_ERR_SHAPE;
@@ -289,6 +289,13 @@ int sp24_gemm_packed(const void *Xq, const float *x_scale, const void *packed, c
                      sp24_stream_t stream) {
   return gemm_common(sp24::kSparseE4M3Packed, Xq, x_scale, packed, nullptr, w_scale, Y, M, N, K,
                      workspace, ws_bytes, status, stream);
+}
+
+int sp24_gemm_int8_packed(const int8_t *Xq, const float *x_scale, const void *packed, const float *w_scale,
+                          void *Y, int M, int N, int K, void *workspace, size_t ws_bytes, int32_t *status,
+                          sp24_stream_t stream) {
+  return gemm_common(sp24::kSparseI8Packed, Xq, x_scale, packed, nullptr, w_scale, Y, M, N, K, workspace,
+                     ws_bytes, status, stream);
 }
 
 static int quant_gemm_common(bool lift, const void *X, int M, int N, int K, const void *packed,

@@ -54,6 +54,7 @@ struct KindTraits<kSparseE4M3> {
   static constexpr int kAStep = 32;  // A bytes per MMA along K
   static constexpr int kBStep = 64;  // B bytes per MMA along K
   static constexpr uint32_t kFmt = 0;
+  static constexpr uint32_t kDFmt = 1;       // fp32 accumulator
   static constexpr int kAElemBytes = 1;
   static constexpr int kBElemBytes = 1;
   static constexpr int kBBoxElems = 128;     // one 128-byte swizzle row of X per box
@@ -70,6 +71,15 @@ struct KindTraits<kSparseE4M3Packed> : KindTraits<kSparseE4M3> {
   static constexpr bool kPacked = true;
 };
 
+// INT8 W8A8 (kind::i8): the packed layout and the 8-bit 2:4 metadata of the
+// E4M3 kind, signed operands, an s32 accumulator converted to fp32 in the
+// epilogue.
+template <>
+struct KindTraits<kSparseI8Packed> : KindTraits<kSparseE4M3Packed> {
+  static constexpr uint32_t kFmt = 1;   // signed 8-bit
+  static constexpr uint32_t kDFmt = 2;  // s32 accumulator
+};
+
 // Dense E4M3 (comparison kernel): 128 logical K per stage, 4 MMAs of K = 32.
 template <>
 struct KindTraits<kDenseE4M3> {
@@ -84,6 +94,7 @@ struct KindTraits<kDenseE4M3> {
   static constexpr int kAStep = 32;
   static constexpr int kBStep = 32;
   static constexpr uint32_t kFmt = 0;
+  static constexpr uint32_t kDFmt = 1;
   static constexpr int kAElemBytes = 1;
   static constexpr int kBElemBytes = 1;
   static constexpr int kBBoxElems = 128;
@@ -110,6 +121,7 @@ struct KindTraits<kSparseBF16> {
   static constexpr int kAStep = 32;  // 16 compressed bf16 per MMA
   static constexpr int kBStep = 64;  // 32 bf16 per MMA
   static constexpr uint32_t kFmt = 1;
+  static constexpr uint32_t kDFmt = 1;
   static constexpr int kAElemBytes = 2;
   static constexpr int kBElemBytes = 2;
   static constexpr int kBBoxElems = 64;
@@ -277,6 +289,16 @@ struct SegIter {
 // CTA whose stream-K range holds unit u.
 __device__ __forceinline__ int cta_of_unit(int64_t u, int64_t units, int grid) {
   return static_cast<int>(((u + 1) * grid + units - 1) / units) - 1;
+}
+
+// An accumulator word as fp32: the bits themselves, or (kind::i8) the s32
+// sum converted (exact below 2^24, correctly rounded above).
+template <int KIND>
+__device__ __forceinline__ float acc_f32(uint32_t v) {
+  if constexpr (KIND == kSparseI8Packed)
+    return __int2float_rn(static_cast<int>(v));
+  else
+    return __uint_as_float(v);
 }
 
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {
@@ -563,7 +585,7 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = mma_idesc(128, BN, T::kFmt, T::kSparse);
+      constexpr uint32_t idesc = mma_idesc(128, BN, T::kFmt, T::kSparse, T::kDFmt);
       // metadata of row tile i: 4 TMEM columns after all accumulators
       const uint32_t e_tmem = tmem_base + NB * C::kAccCols;
       SegIter it;
@@ -619,6 +641,8 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
               const uint32_t d = d_tmem + rt * BN;
               if constexpr (KIND == kSparseE4M3 || KIND == kSparseE4M3Packed) {
                 mma_f8_sparse(d, ad, bd, idesc, e_tmem + 4 * rt + 2 * kk, acc);
+              } else if constexpr (KIND == kSparseI8Packed) {
+                mma_i8_sparse(d, ad, bd, idesc, e_tmem + 4 * rt + 2 * kk, acc);
               } else if constexpr (KIND == kSparseBF16) {
                 // one metadata column per MMA; columns are addressed in pairs and
                 // the instruction descriptor's selector picks the column of the pair
@@ -744,8 +768,8 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4)
               __stcg(part4(blockIdx.x, rt, c / 4 + k4),
-                     make_float4(__uint_as_float(v[4 * k4]), __uint_as_float(v[4 * k4 + 1]),
-                                 __uint_as_float(v[4 * k4 + 2]), __uint_as_float(v[4 * k4 + 3])));
+                     make_float4(acc_f32<KIND>(v[4 * k4]), acc_f32<KIND>(v[4 * k4 + 1]),
+                                 acc_f32<KIND>(v[4 * k4 + 2]), acc_f32<KIND>(v[4 * k4 + 3])));
           }
         }
         tc_fence_before();
@@ -823,7 +847,7 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
                 for (int h = 0; h < kStep / 32; ++h) {
                   if (c2 + 32 * h < mvalid)
                     store_pass(c2 + 32 * h, [&](int k) {
-                      return __uint_as_float(h < 2 ? w0[32 * h + k] : w1[32 * (h - 2) + k]);
+                      return acc_f32<KIND>(h < 2 ? w0[32 * h + k] : w1[32 * (h - 2) + k]);
                     });
                 }
               }
@@ -840,7 +864,7 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
             tmem_regs_ready(v[1]);
             float acc[32];
 #pragma unroll
-            for (int k = 0; k < kW; ++k) acc[k] = __uint_as_float(v[k >> 4][k & 15]);
+            for (int k = 0; k < kW; ++k) acc[k] = acc_f32<KIND>(v[k >> 4][k & 15]);
             if (first <= last) {
               float4 cur[8];
 #pragma unroll
@@ -972,7 +996,9 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   // two 128-row W tiles on one activation tile when N allows it.
   pl.mt = (pl.bn == 224 && kind != kSparseBF16 && N % 256 == 0) ? 2 : 1;
   // Decode-sized tiles over packed weights take two 128-K blocks per stage.
-  pl.kb = (kind == kSparseE4M3Packed && pl.bn <= 64 && pl.mt == 1 && K % 256 == 0) ? 2 : 1;
+  pl.kb = ((kind == kSparseE4M3Packed || kind == kSparseI8Packed) && pl.bn <= 64 && pl.mt == 1 && K % 256 == 0)
+              ? 2
+              : 1;
   pl.bk = 128 * pl.kb;
   pl.tiles_n = N / (128 * pl.mt);
   pl.tiles_m = (M + pl.bn - 1) / pl.bn;
@@ -1112,7 +1138,7 @@ static cudaError_t launch_kind(const GemmPlan &pl, const void *xq, const float *
                                const void *w_values, const uint8_t *w_meta, const float *w_scale,
                                void *y, int M, int N, int K, void *ws, int32_t *status,
                                cudaStream_t st) {
-  if constexpr (KIND == kSparseE4M3Packed) {
+  if constexpr (KIND == kSparseE4M3Packed || KIND == kSparseI8Packed) {
     if (pl.kb == 2) {
       switch (pl.bn) {
         case 16: return launch_typed<KIND, 16, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
@@ -1210,6 +1236,8 @@ cudaError_t launch_gemm(GemmKind kind, const GemmPlan &pl, const void *xq, const
       return launch_kind<kSparseBF16>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
     case kSparseE4M3Packed:
       return launch_kind<kSparseE4M3Packed>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
+    case kSparseI8Packed:
+      return launch_kind<kSparseI8Packed>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
     default:
       return cudaErrorInvalidValue;
   }

@@ -70,7 +70,7 @@ void set_last_cuda_error(int e);
 constexpr size_t kAmaxWorkspaceBytes = 256;
 
 // ---- gemm.cu
-enum GemmKind : int { kSparseE4M3 = 0, kDenseE4M3 = 1, kSparseBF16 = 2, kSparseE4M3Packed = 3 };
+enum GemmKind : int { kSparseE4M3 = 0, kDenseE4M3 = 1, kSparseBF16 = 2, kSparseE4M3Packed = 3, kSparseI8Packed = 4 };
 
 // How a GEMM call is cut into CTAs: tile shape, work decomposition and the
 // scratch a stream-K reduction needs.

@@ -207,11 +207,13 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
-// Instruction descriptor for tcgen05.mma kinds f16 / f8f6f4 with fp32 accumulation.
-//   fmt: kind::f8f6f4 -> 0 = E4M3; kind::f16 -> 1 = BF16.  Both operands K-major.
+// Instruction descriptor for tcgen05.mma kinds f16 / f8f6f4 / i8.
+//   fmt (A and B): kind::f8f6f4 -> 0 = E4M3; kind::f16 -> 1 = BF16;
+//   kind::i8 -> 1 = signed 8-bit.  dfmt (D): 1 = F32, 2 = S32 (kind::i8).
+//   Both operands K-major.
 __host__ __device__ constexpr uint32_t mma_idesc(uint32_t m, uint32_t n, uint32_t fmt,
-                                                 bool sparse) {
-  return (sparse ? (1u << 2) : 0u) | (1u << 4) | (fmt << 7) | (fmt << 10) | ((n >> 3) << 17) |
+                                                 bool sparse, uint32_t dfmt = 1) {
+  return (sparse ? (1u << 2) : 0u) | (dfmt << 4) | (fmt << 7) | (fmt << 10) | ((n >> 3) << 17) |
          ((m >> 4) << 24);
 }
 
@@ -235,6 +237,19 @@ __device__ __forceinline__ void mma_f8_sparse(uint32_t d_tmem, uint64_t adesc, u
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.sp.cta_group::1.kind::f8f6f4 [%0], %1, %2, [%5], %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(e_tmem)
+      : "memory");
+}
+
+// D[tmem] (+)= A_sparse[smem] * B[smem]^T, signed 8-bit integers, s32
+// accumulation, 2:4 metadata in TMEM at e_tmem (the 8-bit layout of kind::f8f6f4).
+__device__ __forceinline__ void mma_i8_sparse(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t e_tmem,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::i8 [%0], %1, %2, [%5], %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(e_tmem)
       : "memory");
 }

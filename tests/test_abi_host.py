@@ -130,6 +130,11 @@ def test_validation_rejects_bad_arguments_without_a_gpu(lib):
     assert lib.int8_quantize_pertensor(FAKE, 4, 32, FAKE, None, FAKE, ws, None, None) == _lib.SP24_ERR_NULL
     assert lib.sp24_prune_compress_int8(FAKE, 4, 12, FAKE, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_SHAPE
     assert lib.sp24_prune_compress_int8(FAKE, 4, 16, FAKE, FAKE, None, FAKE, ws, None, None) == _lib.SP24_ERR_NULL
+    gi = lib.sp24_gemm_int8_packed
+    assert gi(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 192, 128, FAKE, big, None, None) == _lib.SP24_ERR_SHAPE
+    assert gi(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 128, 192, FAKE, big, None, None) == _lib.SP24_ERR_SHAPE
+    assert gi(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 128, 128, FAKE, big, None, None) == _lib.SP24_ERR_SHAPE
+    assert gi(None, FAKE, FAKE, FAKE, FAKE, 4, 128, 128, FAKE, big, None, None) == _lib.SP24_ERR_NULL
     # alignment
     odd = ctypes.c_void_p((1 << 20) + 8)
     assert qg(FAKE, 4, 128, 128, FAKE, None, odd, FAKE, FAKE, FAKE, big, None, None) == _lib.SP24_ERR_ALIGN
@@ -140,6 +145,7 @@ def test_validation_rejects_bad_arguments_without_a_gpu(lib):
     assert lib.slide_lift(odd, 4, 120, 5, FAKE, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.int8_quantize_pertensor(FAKE, 4, 32, odd, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.sp24_prune_compress_int8(FAKE, 4, 16, FAKE, odd, FAKE, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
+    assert lib.sp24_gemm_int8_packed(odd, FAKE, FAKE, FAKE, FAKE, 4, 128, 128, FAKE, big, None, None) == _lib.SP24_ERR_ALIGN
     assert lib.sp24_gemm(FAKE, None, odd, FAKE, None, FAKE, 4, 128, 128, 0, FAKE, ws, None, None) == _lib.SP24_ERR_ALIGN
 
 

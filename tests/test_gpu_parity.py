@@ -848,3 +848,30 @@ def test_int8_prune_compress_bit_exact(n, k, dist):
     assert host(d["scale"])[0] == ref["scale"]
     assert np.array_equal(host(d["meta"]), ref["meta"])
     assert np.array_equal(host(d["values"]), ref["values"])
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 1024, 2048), (8, 1024, 2048), (64, 1024, 2048), (300, 1024, 2048),
+                                   (2048, 1024, 2048), (33, 11008, 4096)])
+def test_int8_sparse_gemm_within_tolerance(m, n, k):
+    """INT8 W8A8 end to end: quantise X, prune + quantise + compress W, pack,
+    GEMM (kind::i8, s32 accumulation); Y against the oracle's exact integer
+    GEMM scaled by sx sw.  The cases cover decode tiles with two-block
+    stages, a 128-token tile, the two-row-tile prefill path and a stream-K
+    split over W[11008,4096]."""
+    w = WL.random_bits((n, k), 5000 + n + k, scale=0.02)
+    x = WL.random_bits((m, k), 5100 + m)
+    st = new_status()
+    c = sp().sp24_prune_compress_int8(dev_bf16(w), status=st)
+    xq, sx = sp().int8_quantize_pertensor(dev_bf16(x), status=st)
+    packed = sp().sp24_pack_weights(c["values"].view(torch.uint8), c["meta"])
+    y = sp().sp24_gemm_int8_packed(xq, sx, packed, c["scale"], n, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref_w = O.sp24_prune_compress_int8(w)
+    ref_q, ref_s = O.int8_quantize_pertensor(x)
+    assert np.array_equal(host(xq), ref_q) and np.array_equal(host(c["values"]), ref_w["values"])
+    if m * n * k <= 1 << 27:
+        y_ref, b, _ = O.gemm_ref_int8(ref_q, ref_w["pruned_dense"], ref_s, ref_w["scale"])
+    else:  # the same values through float64 BLAS (exact: every sum is an integer below 2^53)
+        y_ref, b = O.gemm_ref(ref_q, ref_w["pruned_dense"], ref_s, ref_w["scale"])
+    assert_gemm_close(y, y_ref, b, f"int8 M={m} N={n} K={k}")

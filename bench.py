@@ -530,6 +530,43 @@ class GpuWorkload:
             out[f"{2 * nn - 2}:{2 * nn}"] = res
         return out
 
+    def int8_compare(self, reps=50):
+        """INT8 W8A8 on this workload's 2:4 shapes: the INT8 weight path
+        (prune + quantise + compress, canonical layout), the per-tensor INT8
+        quantiser and the INT8 sparse GEMM over tile-packed weights (rotating
+        layers, larger than L2), each a CUDA graph of back-to-back calls."""
+        if self.is68:
+            return None
+        torch, sp = self.torch, self.sp
+        n, k = self.n, self.k
+        outw = dict(values=torch.empty((n, k // 2), dtype=torch.int8, device=self.dev),
+                    meta=torch.empty((n, k // 8), dtype=torch.uint8, device=self.dev),
+                    scale=torch.empty((1,), dtype=torch.float32, device=self.dev))
+        sp.sp24_prune_compress_int8(self.w_pool[0], workspace=self.ws, out=outw)
+        packed = sp.sp24_pack_weights(outw["values"].view(torch.uint8), outw["meta"])
+        pool = [packed.clone() for _ in range(self.R_g)]
+        sw = outw["scale"].clone()
+        t = self._graph_us(lambda r: sp.sp24_prune_compress_int8(self.w_pool[r % self.R_w], workspace=self.ws,
+                                                                 out=outw), max(4, reps // 5))
+        out = {"weight_path_us": round(t, 3), "weight_path_gbs": round(bytes_prune24(n, k) / t / 1e3, 1)}
+        for m in self.ms:
+            q = torch.empty((m, k), dtype=torch.int8, device=self.dev)
+            sx = torch.empty((1,), dtype=torch.float32, device=self.dev)
+            # one eager call of each before capture (attribute set-up, warm)
+            sp.int8_quantize_pertensor(self.x_dev[m], workspace=self.ws, out=q, scale=sx)
+            sp.sp24_gemm_int8_packed(q, sx, pool[0], sw, n, out=self.y[m], workspace=self.ws)
+            tq = self._graph_us(lambda r: sp.int8_quantize_pertensor(self.x_dev[m], workspace=self.ws, out=q,
+                                                                    scale=sx), reps)
+            tg = self._graph_us(lambda r: sp.sp24_gemm_int8_packed(q, sx, pool[r % self.R_g], sw, n, out=self.y[m],
+                                                                  workspace=self.ws), reps)
+            out[str(m)] = {"quantize_us": round(tq, 3),
+                           "quantize_gbs": round(bytes_quant(m, k) / tq / 1e3, 1),
+                           "gemm_us": round(tg, 3),
+                           "gemm_gbs": round(bytes_sparse_gemm(m, n, k) / tg / 1e3, 1),
+                           "gemm_tops_dense_equiv": round(2 * m * n * k / tg / 1e6, 2)}
+        del pool
+        return out
+
     def fusion_compare(self, reps=50):
         """For every M that the step runs fused: the fused launch against the
         activation kernel + GEMM pair it replaces, each as a CUDA graph of
@@ -671,6 +708,12 @@ def run_gpu(args, wl, rank, world, local_rank):
     fusion = gw.fusion_compare() if rank == 0 and not args.no_compare else None
     finer = gw.finer_scales() if rank == 0 and not args.no_compare else None
     general = gw.general_slide() if rank == 0 and not args.no_compare else None
+    int8 = None
+    if rank == 0 and not args.no_compare:
+        try:
+            int8 = gw.int8_compare()
+        except Exception as e:  # a failure here is recorded, never fatal to the bench line
+            int8 = {"error": f"{type(e).__name__}: {e}"[:300]}
     e2e_t, h2d, d2h = gw.e2e(args.steps)
     e2e_t = max_over_ranks(e2e_t, device)
     del g_timed, g_detail, g_warm
@@ -705,6 +748,7 @@ def run_gpu(args, wl, rank, world, local_rank):
         "fused_vs_unfused": fusion,
         "finer_scales": finer,
         "general_slide": general,
+        "int8_w8a8": int8,
         "e2e": {"value": round(aggregate_gbs(step_bytes, args.steps, world, e2e_t), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": gw.step_launches() * args.steps,

@@ -156,3 +156,98 @@ def test_no_silent_fallback_without_a_sm100_device(lib):
     # valid arguments on a machine without an sm_100 device: the call must refuse
     rc = lib.fp8_quantize_pertensor(FAKE, 4, 32, FAKE, FAKE, FAKE, 256, None, None)
     assert rc == _lib.SP24_ERR_ARCH
+
+
+def _header_declarations():
+    import re
+    text = re.sub(r"/\*.*?\*/", "", open(_lib.HEADER).read(), flags=re.S)
+    decls = {}
+    for ret, name, params in re.findall(r"^\s*((?:const\s+)?[a-z_0-9]+\s*\**)\s*([a-z_0-9]+)\s*\(([^)]*)\)\s*;",
+                                        text, flags=re.M):
+        plist = [p.strip() for p in params.split(",") if p.strip() and p.strip() != "void"]
+        decls[name] = (ret.strip(), plist)
+    return decls
+
+
+def _ctype_of(param):
+    if "*" in param or "sp24_stream_t" in param:
+        return ctypes.c_void_p
+    if "int64_t" in param:
+        return ctypes.c_int64
+    if "size_t" in param:
+        return ctypes.c_size_t
+    if param.startswith("int ") or param == "int":
+        return ctypes.c_int
+    raise AssertionError(f"unclassified parameter {param!r}")
+
+
+def test_binding_signatures_match_the_header():
+    """Every ctypes signature has the header's parameter count and kinds
+    (pointer, int, int64_t, size_t) and return type: a binding that passed
+    an argument in the wrong slot or width would fail here, not on a GPU."""
+    decls = _header_declarations()
+    assert set(decls) == set(_lib.header_functions())
+    rets = {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "const char *": ctypes.c_char_p}
+    for name, (ret, params) in decls.items():
+        res, args = _lib.SIGNATURES[name]
+        assert rets[" ".join(ret.replace("*", " *").split())] is res, name
+        assert [_ctype_of(p) for p in params] == list(args), name
+
+
+def test_bindings_marshal_arguments_in_header_order(monkeypatch):
+    """The Python bindings of the sliding-window and INT8 entry points pass
+    the right tensors, sizes and stream in the header's order, and size their
+    outputs as the header states (a recording stand-in for the library, CPU
+    tensors; nothing is computed)."""
+    import torch
+
+    import structured_sparse_fp8_b200 as sp
+
+    calls = {}
+
+    class Recorder:
+        def __getattr__(self, name):
+            def f(*args):
+                calls[name] = args
+                return 512 if name == "sp24_workspace_size" else 0
+            return f
+
+    monkeypatch.setattr(sp._lib, "load", lambda: Recorder())
+    monkeypatch.setattr(sp, "_require_cuda", lambda *ts: None)
+    monkeypatch.setattr(sp, "_stream", lambda device: 777)
+    ws = sp.Workspace("cpu")
+    wsp = ws.get(512).data_ptr()
+
+    def check(name, expect):
+        got = calls[name]
+        assert len(got) == len(_lib.SIGNATURES[name][1]), name
+        assert got[:-3] + got[-2:] == expect[:-3] + expect[-2:], name   # all but the workspace size
+        assert got[-3] >= 512 or name.endswith("packed"), name
+
+    W = torch.zeros((8, 120), dtype=torch.bfloat16)
+    d = sp.slide_decompose(W, 3, workspace=ws)
+    assert d["values"].shape == (8, 80) and d["meta"].shape == (8, 20)   # K' = 120 * 4 / 3 = 160
+    check("slide_decompose", (W.data_ptr(), 8, 120, 3, d["values"].data_ptr(), d["meta"].data_ptr(),
+                              d["scale"].data_ptr(), wsp, 512, None, 777))
+    X = torch.zeros((4, 120), dtype=torch.bfloat16)
+    q, s = sp.slide_lift(X, 5, workspace=ws)
+    assert q.shape == (4, 192) and q.dtype == torch.uint8                  # K' = 120 * 8 / 5
+    check("slide_lift", (X.data_ptr(), 4, 120, 5, q.data_ptr(), s.data_ptr(), wsp, 512, None, 777))
+    X = torch.zeros((4, 32), dtype=torch.bfloat16)
+    q, s = sp.int8_quantize_pertensor(X, workspace=ws)
+    assert q.shape == (4, 32) and q.dtype == torch.int8
+    check("int8_quantize_pertensor", (X.data_ptr(), 4, 32, q.data_ptr(), s.data_ptr(), wsp, 512, None, 777))
+    W = torch.zeros((8, 64), dtype=torch.bfloat16)
+    c = sp.sp24_prune_compress_int8(W, workspace=ws)
+    assert c["values"].shape == (8, 32) and c["values"].dtype == torch.int8 and c["meta"].shape == (8, 8)
+    check("sp24_prune_compress_int8", (W.data_ptr(), 8, 64, c["values"].data_ptr(), c["meta"].data_ptr(),
+                                       c["scale"].data_ptr(), wsp, 512, None, 777))
+    xq = torch.zeros((4, 128), dtype=torch.int8)
+    packed = torch.zeros(128 * 128 // 2 + 128 * 128 // 8, dtype=torch.uint8)
+    sx, sw = torch.ones(1), torch.ones(1)
+    y = sp.sp24_gemm_int8_packed(xq, sx, packed, sw, 128, workspace=ws)
+    assert y.shape == (4, 128) and y.dtype == torch.bfloat16
+    check("sp24_gemm_int8_packed", (xq.data_ptr(), sx.data_ptr(), packed.data_ptr(), sw.data_ptr(), y.data_ptr(),
+                                    4, 128, 128, wsp, 512, None, 777))
+    with pytest.raises(sp.Sp24Error):
+        sp.sp24_gemm_int8_packed(xq.view(torch.uint8), sx, packed, sw, 128, workspace=ws)

@@ -19,7 +19,8 @@ the function's docstring.  Pages cited:
   Ventana Deslizante", "Levantamiento de Activacion", "Pipeline de
   Implementacion"; the lay "Analogia de la Ventana Deslizante".
 * the cookbook's Comparison Tables ("INT8 W8A8" recipe) and the SlideSparse
-  summary's §3-§4 (INT8 among its precisions) for the INT8 functions.
+  summary's §3-§4 (INT8 and FP4 among its precisions) for the INT8 and FP4
+  functions.
 * "La Densite Dynamique et les Noyaux Non Structures ..." (the roadmap) --
   §Lacunes des noyaux (compressed metadata), §Interaction avec la
   quantification (per-tensor FP8 scaling).
@@ -524,6 +525,84 @@ def gemm_ref_int8(xq: np.ndarray, wq: np.ndarray, sx=1.0, sw=1.0):
     acc = x @ w.T
     s = float(np.float64(sx) * np.float64(sw))
     return s * acc.astype(np.float64), abs(s) * (np.abs(x) @ np.abs(w).T).astype(np.float64), acc
+
+
+# ---------------------------------------------------------------------------
+# FP4 (E2M1) with 2:4 weights (the SlideSparse summary, §3 Contribuciones
+# Clave: FP4 among the supported precisions)
+# ---------------------------------------------------------------------------
+
+E2M1_MAX = 6.0
+# magnitude of code c (bits: sign 3, exponent 2-1, mantissa 0; bias 1;
+# exponent 0 is subnormal: 0 and 0.5)
+_E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def e2m1_decode(codes: np.ndarray) -> np.ndarray:
+    """Values (float64) of FP4 E2M1 codes 0..15 (bit 3 is the sign)."""
+    c = np.asarray(codes, dtype=np.uint8)
+    mag = _E2M1_GRID[c & 7]
+    return np.where(c & 8, -mag, mag)
+
+
+def e2m1_encode(v: np.ndarray) -> np.ndarray:
+    """FP4 E2M1 code of each fp32 value: round to the nearest grid value,
+    ties to the even code (mantissa bit 0), saturate at +-6, and keep the sign
+    of a value that rounds to zero (code 8 for negatives), as E4M3 does."""
+    v = np.asarray(v, dtype=np.float32)
+    _require_finite(v, "e2m1_encode")
+    a = np.abs(v).astype(np.float64)
+    d = np.abs(a[..., None] - _E2M1_GRID)           # distance to each magnitude
+    best = d.min(axis=-1, keepdims=True)
+    # candidates at the minimal distance: one, or two at a tie; take the even index
+    cand = d == best
+    idx = np.where(cand[..., ::2].any(axis=-1),
+                   np.argmax(cand & (np.arange(8) % 2 == 0), axis=-1),
+                   np.argmax(cand, axis=-1))
+    idx = np.where(a > E2M1_MAX, 7, idx)
+    sign = np.signbit(v)
+    return (idx + np.where(sign, 8, 0)).astype(np.uint8)
+
+
+def fp4_scale_from_amax(a: np.float32) -> np.float32:
+    """Per-tensor FP4 scale s = amax / 6 (one fp32 division); 1.0 when amax is 0.
+
+    Reading: the pages list FP4 without a format; the plainest one in keeping
+    with the per-tensor E4M3 and INT8 rules is the same rule on the E2M1 grid
+    (largest magnitude 6), with no block scales.
+    """
+    a = np.float32(a)
+    if a == 0:
+        return np.float32(1.0)
+    return np.float32(a / np.float32(E2M1_MAX))
+
+
+def fp4_quantize_with_scale(bits: np.ndarray, s: np.float32) -> np.ndarray:
+    """E2M1 codes of x / s, the quotient one correctly rounded fp32 division."""
+    x = bf16_to_f32(bits)
+    return e2m1_encode((x / np.float32(s)).astype(np.float32))
+
+
+def fp4_quantize_pertensor(bits: np.ndarray):
+    """Per-tensor dynamic FP4 quantisation: returns (codes uint8 0..15, scale)."""
+    s = fp4_scale_from_amax(amax(bits))
+    return fp4_quantize_with_scale(bits, s), s
+
+
+def sp24_prune_compress_fp4(w_bits: np.ndarray):
+    """The 2:4 weight path with FP4 codes: the selection and layout of
+    sp24_prune_compress, each kept value stored as its E2M1 code (one code per
+    entry of values [N, K/2]; how codes are packed into bytes is a storage
+    matter for the kernels) under the per-tensor FP4 scale.  Returns a dict
+    with ``values``, ``meta``, ``mask``, ``scale`` and ``pruned_dense`` (codes,
+    0 where pruned)."""
+    w_bits = np.asarray(w_bits, dtype=np.uint16)
+    mask = prune24_mask(w_bits)
+    s = fp4_scale_from_amax(amax(w_bits))
+    codes = fp4_quantize_with_scale(w_bits, s)
+    dense = np.where(mask, codes, np.uint8(0)).astype(np.uint8)
+    vals, meta = compress24(mask, codes)
+    return dict(values=vals.astype(np.uint8), meta=meta, mask=mask, scale=s, pruned_dense=dense)
 
 
 # ---------------------------------------------------------------------------

@@ -523,3 +523,66 @@ def test_general_slide_golden_hand_examples():
         assert d["meta"][0].tolist() == [int(b, 16) for b in c["meta"]]
         assert d["src"][0][d["emask"][0]].tolist() == [int(v) for v in c["src"]]
         assert O.slide_lift_columns(2 * n, n).tolist() == [int(v) for v in c["lift"]]
+
+
+# ------------------------------------------------------------ FP4 (E2M1) with 2:4 weights
+
+def test_e2m1_decode_all_codes_match_ml_dtypes():
+    codes = np.arange(16, dtype=np.uint8)
+    want = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    assert np.array_equal(O.e2m1_decode(codes), want)
+    assert np.array_equal(np.signbit(O.e2m1_decode(codes)), codes >= 8)
+
+
+def test_e2m1_encode_every_bf16_value_matches_ml_dtypes():
+    """ml_dtypes' float4_e2m1fn cast (round to nearest even, saturating, sign
+    kept on zero) over every finite bf16 value up to |x| = 16, and a strided
+    fp32 sweep through every tie."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    x = O.bf16_to_f32(bits)
+    x = x[np.isfinite(x) & (np.abs(x) <= 16)]
+    assert np.array_equal(O.e2m1_encode(x), x.astype(ml_dtypes.float4_e2m1fn).view(np.uint8))
+    sweep = np.linspace(-7, 7, 56001, dtype=np.float32)
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], dtype=np.float32)
+    sweep = np.concatenate([sweep, ties, -ties, np.nextafter(ties, 0), np.nextafter(ties, 9)])
+    assert np.array_equal(O.e2m1_encode(sweep), sweep.astype(ml_dtypes.float4_e2m1fn).view(np.uint8))
+
+
+def test_fp4_golden_hand_example():
+    lines = [ln.split() for ln in open(os.path.join(GOLDEN, "fp4_hand_example.txt"))
+             if ln.strip() and not ln.startswith("#")]
+    for vals, codes, scale in ((lines[0], lines[1], lines[2]), (lines[3], lines[4], lines[5])):
+        bits = WL.to_bf16_bits(np.array([float(v) for v in vals]))[None, :]
+        q, s = O.fp4_quantize_pertensor(bits)
+        assert float(s) == float(scale[0])
+        assert q[0].tolist() == [int(c) for c in codes]
+
+
+def test_fp4_scale_maps_amax_to_six_and_zero_tensor():
+    x = WL.random_bits((16, 128), 4500, dist="student_t3")
+    q, s = O.fp4_quantize_pertensor(x)
+    xf = O.bf16_to_f32(x)
+    top = np.abs(xf) == np.abs(xf).max()
+    assert (q[top] & 7 == 7).all()
+    dq = O.e2m1_decode(q) * np.float64(s)
+    # relative error of a normal E2M1 value is at most a quarter (half of 2^-1)
+    big = np.abs(xf) >= np.float64(s)
+    assert (np.abs(dq[big] - xf[big]) <= 0.25 * np.abs(xf[big]) + 1e-12).all()
+    q0, s0 = O.fp4_quantize_pertensor(np.zeros((2, 8), dtype=np.uint16))
+    assert s0 == np.float32(1.0) and not q0.any()
+
+
+def test_fp4_prune_compress_and_gemm_reduce_to_pinned_functions():
+    w = WL.random_bits((32, 128), 4600, scale=0.02, dist="ties")
+    d = O.sp24_prune_compress_fp4(w)
+    ref = O.sp24_prune_compress(w, "e4m3")
+    assert np.array_equal(d["mask"], ref["mask"]) and np.array_equal(d["meta"], ref["meta"])
+    assert np.array_equal(O.decompress24(d["values"], d["meta"], 128), d["pruned_dense"])
+    q, s = O.fp4_quantize_pertensor(w)
+    assert s == d["scale"] and np.array_equal(np.where(d["mask"], q, 0), d["pruned_dense"])
+    x = WL.random_bits((3, 128), 4601)
+    xq, sx = O.fp4_quantize_pertensor(x)
+    xv, wv = O.e2m1_decode(xq), O.e2m1_decode(d["pruned_dense"])
+    y, _ = O.gemm_ref(xv, wv, sx, d["scale"])
+    walk = O.sparse_gemm_walk(xv, O.e2m1_decode(d["values"]), d["meta"], sx, d["scale"])
+    assert np.allclose(walk, y, rtol=0, atol=1e-12 * np.abs(y).max())

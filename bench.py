@@ -144,6 +144,19 @@ def load_traffic():
     return out
 
 
+def runs_of_equal_names(names):
+    """[start, end) index ranges of the maximal runs of consecutive equal
+    names: the launches one event pair brackets in the per-kernel timing."""
+    runs, i = [], 0
+    while i < len(names):
+        j = i + 1
+        while j < len(names) and names[j] == names[i]:
+            j += 1
+        runs.append((i, j))
+        i = j
+    return runs
+
+
 # ---------------------------------------------------------------- ranks
 
 def max_over_ranks(seconds: float, device=None) -> float:
@@ -351,16 +364,23 @@ class GpuWorkload:
         evs = []
         with torch.cuda.graph(g):
             for s in range(first, first + steps):
-                for (name, fn, nb, fl, nl) in self.ops_of_step(s):
-                    if events:
-                        e0 = torch.cuda.Event(enable_timing=True, external=True)
-                        e1 = torch.cuda.Event(enable_timing=True, external=True)
-                        e0.record()
-                        fn()
-                        e1.record()
-                        evs.append((name, nb, fl, e0, e1))
-                    else:
-                        fn()
+                ops = list(self.ops_of_step(s))
+                if not events:
+                    for op in ops:
+                        op[1]()
+                    continue
+                # one event pair per run of consecutive launches of one kernel,
+                # so launches of the same kernel keep their programmatic
+                # launch overlap (an event between them would serialise them)
+                for i, j in runs_of_equal_names([op[0] for op in ops]):
+                    e0 = torch.cuda.Event(enable_timing=True, external=True)
+                    e1 = torch.cuda.Event(enable_timing=True, external=True)
+                    e0.record()
+                    for op in ops[i:j]:
+                        op[1]()
+                    e1.record()
+                    evs.append((ops[i][0], sum(op[2] for op in ops[i:j]), sum(op[3] for op in ops[i:j]),
+                                j - i, e0, e1))
         return g, evs
 
     # dense FP8 comparison for the GEMM shapes of this workload ------------
@@ -662,16 +682,17 @@ def run_gpu(args, wl, rank, world, local_rank):
             dist.barrier()
     elapsed = max_over_ranks(start.elapsed_time(end) / 1e3, device)
 
-    # per-call durations (second replay of the same K steps, events between calls)
+    # per-kernel durations (second replay of the same K steps, an event pair
+    # around each run of consecutive launches of one kernel)
     g_detail.replay()
     torch.cuda.synchronize()
     per = {}
-    for name, nb, fl, e0, e1 in evs:
+    for name, nb, fl, cnt, e0, e1 in evs:
         d = per.setdefault(name, dict(t=0.0, bytes=0, flops=0, n=0))
         d["t"] += e0.elapsed_time(e1) / 1e3
         d["bytes"] += nb
         d["flops"] += fl
-        d["n"] += 1
+        d["n"] += cnt
     assert int(gw.status.item()) == 0, "device status word set during the benchmark"
 
     step_bytes = gw.step_bytes()

@@ -1,0 +1,63 @@
+"""Planted mistakes in the oracle (CPU only) must fail its pins: evidence
+that the pins of the INT8, FP4 and general sliding-window functions pin them.
+Each case replaces one oracle function by a plausibly wrong version for the
+duration of the test and runs the pin that should catch it."""
+import numpy as np
+import pytest
+
+import test_oracle_pins as P
+from oracle import sp24_oracle as O
+
+
+def _fails(pin):
+    with pytest.raises(AssertionError):
+        pin()
+
+
+def test_int8_ties_away_from_zero_is_caught(monkeypatch):
+    def wrong(bits, s):
+        v = (O.bf16_to_f32(bits) / np.float32(s)).astype(np.float32)
+        q = np.sign(v) * np.floor(np.abs(v) + np.float32(0.5))
+        return np.clip(q, -127, 127).astype(np.int8)
+    monkeypatch.setattr(O, "int8_quantize_with_scale", wrong)
+    _fails(P.test_int8_golden_hand_example)   # the half-step bound alone cannot see a tie's direction
+
+
+def test_int8_scale_of_128_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "int8_scale_from_amax", lambda a: np.float32(np.float32(a) / np.float32(128)) if a else np.float32(1))
+    _fails(P.test_int8_golden_hand_example)
+
+
+def test_fp4_ties_away_from_zero_is_caught(monkeypatch):
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+    def wrong(v):
+        v = np.asarray(v, dtype=np.float32)
+        a = np.abs(v).astype(np.float64)
+        d = np.abs(a[..., None] - grid)
+        idx = 7 - np.argmin(d[..., ::-1], axis=-1)     # ties to the larger magnitude
+        idx = np.where(a > 6, 7, idx)
+        return (idx + np.where(np.signbit(v), 8, 0)).astype(np.uint8)
+    monkeypatch.setattr(O, "e2m1_encode", wrong)
+    _fails(P.test_e2m1_encode_every_bf16_value_matches_ml_dtypes)
+    _fails(P.test_fp4_golden_hand_example)
+
+
+def test_slide_windows_from_the_right_are_caught(monkeypatch):
+    def wrong(kept, n):
+        kept = [int(p) for p in np.nonzero(np.asarray(kept, dtype=bool))[0]]
+        taken, out = set(), []
+        for j in range(n - 1):
+            cand = [p for p in kept if 2 * j <= p <= 2 * j + 3 and p not in taken]
+            pick = cand[-2:] if len(cand) >= 2 else cand
+            taken.update(pick)
+            out.append(tuple(pick))
+        return out
+    monkeypatch.setattr(O, "slide_windows", wrong)
+    _fails(P.test_general_slide_golden_hand_examples)
+
+
+def test_gemm_ref_int8_dropping_a_scale_is_caught(monkeypatch):
+    real = O.gemm_ref_int8
+    monkeypatch.setattr(O, "gemm_ref_int8", lambda xq, wq, sx=1.0, sw=1.0: real(xq, wq, sx, 1.0))
+    _fails(P.test_int8_gemm_is_the_exact_integer_product)

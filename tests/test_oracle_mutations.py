@@ -61,3 +61,83 @@ def test_gemm_ref_int8_dropping_a_scale_is_caught(monkeypatch):
     real = O.gemm_ref_int8
     monkeypatch.setattr(O, "gemm_ref_int8", lambda xq, wq, sx=1.0, sw=1.0: real(xq, wq, sx, 1.0))
     _fails(P.test_int8_gemm_is_the_exact_integer_product)
+
+
+# ------------------------------------------------------------ the core path's functions
+
+def test_e4m3_decode_with_bias_8_is_caught(monkeypatch):
+    real = O.e4m3_decode
+    monkeypatch.setattr(O, "e4m3_decode", lambda codes: real(codes) / 2.0)
+    _fails(P.test_e4m3_decode_all_codes_match_ml_dtypes)
+
+
+def test_e4m3_truncation_instead_of_rounding_is_caught(monkeypatch):
+    real_enc, real_dec = O.e4m3_encode, O.e4m3_decode
+
+    def wrong(v):
+        c = real_enc(v)
+        up = np.abs(real_dec(c)) > np.abs(np.asarray(v, dtype=np.float64))
+        return np.where(up & ((c & 0x7F) > 0), c - 1, c).astype(np.uint8)
+    monkeypatch.setattr(O, "e4m3_encode", wrong)
+    _fails(P.test_e4m3_encode_every_bf16_value_in_range)
+
+
+def test_prune_ties_to_the_higher_index_are_caught(monkeypatch):
+    def wrong(bits, group, keep):
+        w = O.bf16_to_f32(bits)
+        a = np.abs(w).reshape(*w.shape[:-1], w.shape[-1] // group, group).astype(np.float64)
+        idx = np.arange(group)
+        ai, aj = a[..., :, None], a[..., None, :]
+        beats = (aj > ai) | ((aj == ai) & (idx[None, :] > idx[:, None]))
+        return (beats.sum(axis=-1) < keep).reshape(w.shape)
+    monkeypatch.setattr(O, "keep_mask", wrong)
+    _fails(P.test_prune24_exhaustive_over_tie_alphabet)
+    _fails(P.test_prune24_golden_hand_example)
+
+
+def test_swapped_metadata_nibble_order_is_caught(monkeypatch):
+    real = O.compress24
+
+    def wrong(mask, payload):
+        vals, meta = real(mask, payload)
+        return vals, ((meta & 0x0F) << 4 | (meta >> 4)).astype(np.uint8)
+    monkeypatch.setattr(O, "compress24", wrong)
+    _fails(P.test_prune24_golden_hand_example)
+
+
+def test_68_windows_from_the_right_are_caught(monkeypatch):
+    def wrong(kept):
+        kept = [int(p) for p in np.nonzero(np.asarray(kept, dtype=bool))[0]]
+        taken, out = set(), []
+        for j in range(3):
+            cand = [p for p in kept if 2 * j <= p <= 2 * j + 3 and p not in taken][-2:]
+            taken.update(cand)
+            out.append(tuple(cand))
+        return out
+    monkeypatch.setattr(O, "window_assignment", wrong)
+    _fails(P.test_slide68_golden_hand_example)
+
+
+def test_e4m3_scale_with_the_wrong_maximum_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "scale_from_amax",
+                        lambda a: np.float32(np.float32(a) / np.float32(240.0)) if a else np.float32(1.0))
+    _fails(P.test_scale_closed_form_and_zero_tensor)
+
+
+def test_pertoken_with_the_tensor_scale_is_caught(monkeypatch):
+    def wrong(bits):
+        codes, s = O.quantize_pertensor(bits)
+        return codes, np.full(bits.shape[0], s, dtype=np.float32)
+    monkeypatch.setattr(O, "quantize_pertoken", wrong)
+    _fails(P.test_pertoken_scales_follow_row_magnitude_exactly)
+
+
+def test_gemm_dropping_the_last_k_column_is_caught(monkeypatch):
+    real = O.gemm_ref
+
+    def wrong(x_vals, w_vals, sx=1.0, sw=1.0):
+        x = np.array(x_vals, dtype=np.float64)
+        x[:, -1] = 0.0
+        return real(x, w_vals, sx, sw)
+    monkeypatch.setattr(O, "gemm_ref", wrong)
+    _fails(lambda: P.test_sparse_walk_equals_dense_reference("normal"))

@@ -141,3 +141,25 @@ def test_gemm_dropping_the_last_k_column_is_caught(monkeypatch):
         return real(x, w_vals, sx, sw)
     monkeypatch.setattr(O, "gemm_ref", wrong)
     _fails(lambda: P.test_sparse_walk_equals_dense_reference("normal"))
+
+
+def test_perchannel_with_the_tensor_scale_is_caught(monkeypatch):
+    def wrong(w_bits):
+        r = O.sp24_prune_compress(w_bits, "e4m3")
+        return dict(values=r["values"], meta=r["meta"], mask=r["mask"],
+                    scales=np.full(w_bits.shape[0], r["scale"], dtype=np.float32), pruned_dense=r["pruned_dense"])
+    monkeypatch.setattr(O, "sp24_prune_compress_perchannel", wrong)
+    _fails(P.test_perchannel_prune_selects_like_per_tensor_and_scales_each_row)
+
+
+def test_general_lift_off_by_one_window_is_caught(monkeypatch):
+    def wrong(k, n):   # windows at stride 1 instead of 2
+        g2 = 2 * n
+        cols = np.empty(k // g2 * 4 * (n - 1), dtype=np.int64)
+        for g in range(k // g2):
+            for j in range(n - 1):
+                for r in range(4):
+                    cols[4 * ((n - 1) * g + j) + r] = g2 * g + j + r
+        return cols
+    monkeypatch.setattr(O, "slide_lift_columns", wrong)
+    _fails(P.test_general_slide_golden_hand_examples)

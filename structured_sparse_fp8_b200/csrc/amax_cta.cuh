@@ -1,6 +1,7 @@
-// amax_cta.cuh -- the first launch of the two-launch quantisers (slide.cu,
-// int8.cu): the bf16 amax of a tensor, reduced in each CTA and then by one
-// atomic per CTA into a workspace word that starts at zero.  Internal
+// amax_cta.cuh -- shared pieces of the two-launch quantisers (slide.cu,
+// int8.cu): the first launch, the bf16 amax of a tensor reduced in each CTA
+// and then by one atomic per CTA into a workspace word that starts at zero,
+// and the departure count that ends the second launch.  Internal
 // linkage: every source that includes it gets its own kernel.
 #pragma once
 
@@ -46,6 +47,19 @@ inline unsigned bf16_amax_grid(int64_t nvec, int64_t cap) {
   int64_t g = (nvec + per - 1) / per;
   if (g > cap) g = cap;
   return static_cast<unsigned>(g < 1 ? 1 : g);
+}
+
+// End of the second launch: the last CTA to leave returns the two workspace
+// words (ws[0] amax, ws[1] departures) to zero for the next call.
+__device__ __forceinline__ void workspace_depart(uint32_t *ws) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&ws[1], 1u) == gridDim.x - 1) {
+      ws[0] = 0u;
+      ws[1] = 0u;
+    }
+  }
 }
 
 inline cudaError_t launch_bf16_amax(const void *x, int64_t nvec, uint32_t *ws, int64_t cap, cudaStream_t st) {

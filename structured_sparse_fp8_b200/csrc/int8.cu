@@ -89,17 +89,6 @@ __device__ __forceinline__ Coder<DIRECT> make_coder(uint8_t *tab, const uint32_t
   return Coder<DIRECT>{tab, s};
 }
 
-__device__ __forceinline__ void depart(uint32_t *ws) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(&ws[1], 1u) == gridDim.x - 1) {
-      ws[0] = 0u;
-      ws[1] = 0u;
-    }
-  }
-}
-
 template <bool DIRECT>
 __host__ __device__ constexpr int batch() { return DIRECT ? 1 : kBatch; }
 
@@ -129,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       q[v + stride * u] = make_uint2(lo, hi);
     }
   }
-  depart(ws);
+  workspace_depart(ws);
 }
 
 // W bf16 as nvec 16-byte vectors (two groups of 4 each; K % 8 == 0, so a
@@ -174,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       meta[vu] = static_cast<uint8_t>(mb);
     }
   }
-  depart(ws);
+  workspace_depart(ws);
 }
 
 int64_t grid_cap(int sms) { return static_cast<int64_t>(kCtasPerSm) * sms; }

@@ -93,17 +93,6 @@ __device__ __forceinline__ Coder<DIRECT> make_coder(uint8_t *tab, const uint32_t
   return Coder<DIRECT>{tab, s};
 }
 
-__device__ __forceinline__ void depart(uint32_t *ws) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(&ws[1], 1u) == gridDim.x - 1) {
-      ws[0] = 0u;
-      ws[1] = 0u;
-    }
-  }
-}
-
 // Group g of thread (warp span t, slice u): t * 32 B + 32 u + lane.
 // Loads the NN words (2N bf16) of the thread's B groups, zeros past the end.
 template <int NN, int B>
@@ -196,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (g < groups) decompose_group<NN>(v[u], code, g, values, meta);
     }
   }
-  depart(ws);
+  workspace_depart(ws);
 }
 
 // One 2N-group of X: the 2N codes, written as the N-1 windows' 4 codes each
@@ -234,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         *reinterpret_cast<uint4 *>(q + g * 16) = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
-  depart(ws);
+  workspace_depart(ws);
 }
 
 int64_t grid_cap(int sms) { return static_cast<int64_t>(kCtasPerSm) * sms; }

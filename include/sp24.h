@@ -40,10 +40,15 @@
  *   use.  Its first 256 bytes (and, for a split-K GEMM, its tile counters)
  *   hold counters that every call returns to zero; the rest is scratch that
  *   a call rewrites before reading.  So one buffer can serve any sequence of
- *   calls, as long as calls sharing it never run concurrently.
+ *   calls, as long as calls sharing it never run concurrently.  After a call
+ *   that reported SP24_STATUS_TIMEOUT the counters may be left nonzero (a
+ *   late arrival can count into a tile its owner gave up on): zero-fill the
+ *   workspace again before its next use, or a later call may read partial
+ *   sums that are not ready.
  * - `status` (nullable) is a device int32 that kernels OR error bits into:
  *   SP24_STATUS_NONFINITE when an input holds NaN/Inf (the method is defined
- *   for finite inputs only).  Read it after synchronising the stream.
+ *   for finite inputs only; a NaN input element is encoded as 0x7F whatever
+ *   its sign).  Read it after synchronising the stream.
  * - The library is for sm_100a (B200).  On any other device the entry
  *   points return SP24_ERR_ARCH.
  *

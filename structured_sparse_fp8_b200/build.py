@@ -17,7 +17,6 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsp24.so")
 SOURCES = ["api.cu", "elementwise.cu", "gemm.cu", "int8.cu", "noalloc.cu", "rowscale.cu", "slide.cu", "stream.cu"]
-HEADERS = ["kernels.h", "sm100_ptx.cuh", "quant_common.cuh"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -33,7 +32,9 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "sp24.h")]
+    # every source and header the library is compiled from, whatever its name
+    deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh", ".h"))]
+    deps += [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 

@@ -22,11 +22,14 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t h) { return __uint_
 
 // E4M3 code of one fp32 value: round to nearest even, saturate to +-448, and
 // keep the sign of a value that rounds to zero (code 0x80 for negatives).
+// A NaN of either sign gives 0x7F: finite values saturate at magnitude code
+// 0x7E, so a magnitude code of 0x7F is the conversion's NaN, whatever sign it
+// carries, and it is returned without one.
 __device__ __forceinline__ uint32_t e4m3_code(float v) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
-  uint32_t c = r & 0xFFu;
-  return c | ((__float_as_uint(v) >> 24) & 0x80u);
+  const uint32_t c = r & 0xFFu;
+  return (c & 0x7Fu) == 0x7Fu ? 0x7Fu : c | ((__float_as_uint(v) >> 24) & 0x80u);
 }
 
 // Largest magnitude bit patterns of the 8 bf16 values of a 16-byte vector,

@@ -73,6 +73,15 @@ def test_device_e4m3_encode_matches_oracle():
     assert np.array_equal(got, want), np.argwhere(got != want)[:5]
 
 
+def test_device_e4m3_encode_nan_of_either_sign_is_0x7f():
+    # NaN inputs are outside the method's contract (they set the status bit);
+    # the device encoder still agrees with the oracle on them
+    nan_bits = np.array([0x7FC00000, 0xFFC00000, 0x7F800001, 0xFFFFFFFF], dtype=np.uint32)
+    v = nan_bits.view(np.float32)
+    got = host(sp().debug_e4m3_encode(torch.from_numpy(v.copy()).to(DEV)))
+    assert np.array_equal(got, O.e4m3_encode(v)) and (got == 0x7F).all(), got
+
+
 # ------------------------------------------------------------ quantisation
 
 @pytest.mark.parametrize("shape,seed", [((1, 16), 1), ((3, 48), 2), ((16, 256), 3),

@@ -163,3 +163,19 @@ def test_general_lift_off_by_one_window_is_caught(monkeypatch):
         return cols
     monkeypatch.setattr(O, "slide_lift_columns", wrong)
     _fails(P.test_general_slide_golden_hand_examples)
+
+
+def test_bf16_truncation_is_caught(monkeypatch):
+    def wrong(x):
+        u = np.asarray(x, dtype=np.float32).view(np.uint32)
+        return (u >> np.uint32(16)).astype(np.uint16)      # chops instead of rounding
+    monkeypatch.setattr(O, "f32_to_bf16_rne", wrong)
+    _fails(P.test_f32_to_bf16_rne_matches_library_casts)
+
+
+def test_bf16_ties_away_from_zero_is_caught(monkeypatch):
+    def wrong(x):
+        u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+        return ((u + np.uint64(0x8000)) >> np.uint64(16)).astype(np.uint16)
+    monkeypatch.setattr(O, "f32_to_bf16_rne", wrong)
+    _fails(P.test_f32_to_bf16_rne_matches_library_casts)

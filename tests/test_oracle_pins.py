@@ -69,6 +69,31 @@ def test_e4m3_saturates_above_448_and_keeps_sign_of_zero():
     assert (O.e4m3_encode(-tiny) == 0x80).all()
 
 
+def _lib_bf16(v32):
+    return np.asarray(v32, dtype=np.float32).astype(ml_dtypes.bfloat16).view(np.uint16)
+
+
+def test_f32_to_bf16_rne_matches_library_casts():
+    # every 65537th finite fp32 bit pattern of both signs (a stride that walks
+    # through every low-16-bit residue, so ties, near-ties and exact values)
+    u = np.arange(0, 0x7F800000, 65537, dtype=np.uint64).astype(np.uint32)
+    v = np.concatenate([u, u | np.uint32(0x80000000)]).view(np.float32)
+    assert (O.f32_to_bf16_rne(v) == _lib_bf16(v)).all()
+    t = torch.from_numpy(v.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert (O.f32_to_bf16_rne(v) == t).all()
+    # every midpoint between neighbouring bf16 values whose exponent field is
+    # below the top one, with one fp32 ulp either side: ties go to the even
+    # neighbour, everything else to the nearer one
+    hi = np.arange(0x0000, 0x7F7F, dtype=np.uint32)
+    mid = ((hi << np.uint32(16)) | np.uint32(0x8000)).view(np.float32)
+    probe = np.concatenate([mid, np.nextafter(mid, np.float32(0)), np.nextafter(mid, np.float32(np.inf))])
+    probe = np.concatenate([probe, -probe])
+    assert (O.f32_to_bf16_rne(probe) == _lib_bf16(probe)).all()
+    # bf16 values themselves are fixed points
+    exact = O.bf16_to_f32(np.arange(0x7F80, dtype=np.uint16))
+    assert (O.f32_to_bf16_rne(exact) == np.arange(0x7F80, dtype=np.uint16)).all()
+
+
 def test_e4m3_golden_landmarks():
     path = os.path.join(GOLDEN, "e4m3_landmarks.txt")
     rows = [ln.split("#")[0].split() for ln in open(path) if ln.strip() and not ln.startswith("#")]

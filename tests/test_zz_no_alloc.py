@@ -5,15 +5,17 @@ device allocation, or a hot loop that cannot pay for cudaMalloc's implicit
 synchronisation.  fp8_quantize_pertensor_static serves them with a static
 device array.  This test calls it through the C ABI twice in a row (the
 second call must not see the first call's leftovers) and checks that codes
-and scale equal those of fp8_quantize_pertensor, bit for bit, which is the
-tolerance the parity tests use for FP8 codes.  It is collected last so that
-a run stopping at the first failure has already run every other test, and it
-passes both alone in a fresh process and after the rest of the suite.
+and scale equal, bit for bit (the tolerance the parity tests use for FP8
+codes), both those of fp8_quantize_pertensor and those of the CPU oracle.
+It is collected last so that a run stopping at the first failure has already
+run every other test, and it passes both alone in a fresh process and after
+the rest of the suite.
 """
 import numpy as np
 import pytest
 import torch
 
+from oracle import sp24_oracle as O
 from structured_sparse_fp8_b200 import workloads as WL
 
 pytestmark = pytest.mark.gpu
@@ -32,7 +34,8 @@ def test_static_scratch_quantize_matches_workspace_quantize_twice():
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
     for call, (shape, seed, scale) in enumerate([((64, 4096), 11, 1.0), ((37, 14336), 12, 0.02)]):
-        x = _dev_bf16(WL.random_bits(shape, seed, scale=scale), dev)
+        bits = WL.random_bits(shape, seed, scale=scale)
+        x = _dev_bf16(bits, dev)
         q = torch.empty(shape, dtype=torch.uint8, device=dev)
         s = torch.empty(1, dtype=torch.float32, device=dev)
         st = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -44,3 +47,6 @@ def test_static_scratch_quantize_matches_workspace_quantize_twice():
         assert int(st.item()) == 0
         assert s.item() == ref_s.item(), f"call {call}: scale differs"
         assert torch.equal(q, ref_q), f"call {call}: codes differ"
+        oq, osx = O.quantize_pertensor(bits)
+        assert s.item() == float(osx), f"call {call}: scale differs from the oracle"
+        assert np.array_equal(q.cpu().numpy(), oq), f"call {call}: codes differ from the oracle"

@@ -735,6 +735,9 @@ def run_gpu(args, wl, rank, world, local_rank):
             int8 = gw.int8_compare()
         except Exception as e:  # a failure here is recorded, never fatal to the bench line
             int8 = {"error": f"{type(e).__name__}: {e}"[:300]}
+    prefill = None
+    if rank == 0 and args.workload == "decode" and not args.no_prefill:
+        prefill = prefill_headline(device, peaks)
     e2e_t, h2d, d2h = gw.e2e(args.steps)
     e2e_t = max_over_ranks(e2e_t, device)
     del g_timed, g_detail, g_warm
@@ -764,6 +767,7 @@ def run_gpu(args, wl, rank, world, local_rank):
                          f"{gw.R_g} compressed layers",
                    "parallelism": f"replicas x{world}"},
         "roofline": roof,
+        "prefill": prefill,
         "kernels": kernels,
         "sparse_vs_dense": compare,
         "fused_vs_unfused": fusion,
@@ -777,6 +781,72 @@ def run_gpu(args, wl, rank, world, local_rank):
         "peaks": peaks,
     }
     return line, gw
+
+
+def prefill_headline(device, peaks, reps=20):
+    """The tensor-bound target next to the decode headline: the prefill-shaped
+    fused-QKV sparse GEMM (M4096 N12288 K4096, X with its 41 outlier columns)
+    and the same-family dense FP8 GEMM on the same shapes, each timed as a
+    CUDA graph of `reps` launches over rotating weight copies (pools larger
+    than L2), CUDA events on the launching stream.  Roofline: 2 M N K
+    dense-equivalent FLOPs per call against the sparse FP8 peak, 4 x the
+    measured bf16 burst (the nominal ratios: FP8 = 2 x bf16, 2:4 = 2 x
+    dense)."""
+    import torch
+
+    import structured_sparse_fp8_b200 as sp
+    from structured_sparse_fp8_b200 import workloads as WL
+    wl = WORKLOADS["prefill"]
+    m, n, k = wl["ms"][0], wl["n"], wl["k"]
+    ws = sp.Workspace(device)
+    w = torch.from_numpy(WL.weight_bits(wl["cfg"]).view(np.int16)).view(torch.bfloat16).to(device)
+    x = torch.from_numpy(WL.activation_bits(wl["cfg"], m).view(np.int16)).view(torch.bfloat16).to(device)
+    packed, sw = sp.sp24_prune_compress_packed(w, workspace=ws)
+    wq, swd = sp.fp8_quantize_pertensor(w, workspace=ws)
+    xq, sx = sp.fp8_quantize_pertensor(x, workspace=ws)
+    del w
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=device)
+    ps = [packed] + [packed.clone() for _ in range(max(1, -(-3 * L2_BYTES // packed.numel())) - 1)]
+    pd = [wq] + [wq.clone() for _ in range(max(1, -(-3 * L2_BYTES // wq.numel())) - 1)]
+    ws.get(max(sp._lib.load().sp24_workspace_size(sp._lib.OP_GEMM_PACKED, m, n, k, 0),
+               sp._lib.load().sp24_workspace_size(sp._lib.OP_GEMM_DENSE, m, n, k, 0)) + 4096)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def time_graph(fn):
+        fn(0)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for r in range(reps):
+                fn(r)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) * 1e3 / reps
+
+    t_sp = time_graph(lambda r: sp.sp24_gemm_packed(xq, sx, ps[r % len(ps)], sw, n, out=y, status=status,
+                                                    workspace=ws))
+    t_dn = time_graph(lambda r: sp.fp8_gemm_dense(xq, sx, pd[r % len(pd)], swd, out=y, status=status,
+                                                  workspace=ws))
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "device status word set during the prefill timing"
+    flops = 2.0 * m * n * k
+    achieved = flops / t_sp / 1e6
+    peak = peaks["bf16_tflops"] * 4.0
+    return {"workload": wl["name"],
+            "sparse_us": round(t_sp, 3), "dense_fp8_us": round(t_dn, 3), "speedup_vs_dense": round(t_dn / t_sp, 3),
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
+                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "kernel": "sp24_gemm_packed",
+                         "peak_source": f"{peaks['source']} bf16 burst x4 (2:4 sparse FP8 dense-equivalent)",
+                         "traffic": None},
+            "dense_tflops": round(flops / t_dn / 1e6, 1),
+            "timing": f"CUDA graph of {reps} launches over {len(ps)} rotating packed weight copies "
+                      f"({len(pd)} dense), inputs larger than L2"}
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -877,6 +947,8 @@ def main():
     ap.add_argument("--unfused", action="store_true",
                     help="quantise activations in their own launch at every M (no fused quantise + GEMM)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the prefill-shaped (tensor-bound) GEMM timed next to the decode headline")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -240,7 +240,8 @@ int sp24_gemm_packed(const void *Xq, const float *x_scale, const void *packed,
  * compute the amax of X between them, encode it, and start their tensor-core
  * work on the codes, while the packed weights already stream in.  Workspace:
  * sp24_workspace_size(SP24_OP_QUANTIZE_GEMM_PACKED, M, N, K, 0) (its first
- * 256 bytes are counters, zero before the first use and after every call).
+ * 8 KB are counters and per-CTA flags, zero before the first use and after
+ * every call).
  * Shape rules: 1 <= M <= 256, N % 128 == 0, K % 128 == 0.  Xq and Y must not
  * alias X or each other.  SP24_STATUS_NONFINITE is set as by
  * fp8_quantize_pertensor.

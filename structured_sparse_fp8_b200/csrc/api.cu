@@ -83,7 +83,7 @@ size_t sp24_workspace_size(int op, int64_t M, int64_t N, int64_t K, int dtype) {
       if (M < 1 || N < 128 || Kg < 128 || M > INT32_MAX || N > INT32_MAX || Kg > INT32_MAX) return 0;
       int sms = device_sm_count();
       if (sms <= 0) sms = 148;
-      return sp24::kAmaxWorkspaceBytes +
+      return sp24::kFusedCounterBytes +
              sp24::plan_gemm(sp24::kSparseE4M3Packed, static_cast<int>(M), static_cast<int>(N),
                              static_cast<int>(Kg), sms)
                  .workspace_bytes();
@@ -310,7 +310,8 @@ static int quant_gemm_common(bool lift, const void *X, int M, int N, int K, cons
   if (sms < 0) return SP24_ERR_ARCH;
   const int Kg = lift ? K / 2 * 3 : K;
   const sp24::GemmPlan pl = sp24::plan_gemm(sp24::kSparseE4M3Packed, M, N, Kg, sms);
-  if (!workspace || ws_bytes < sp24::kAmaxWorkspaceBytes + pl.workspace_bytes()) return SP24_ERR_WORKSPACE;
+  if (pl.grid > sp24::kFusedMaxCtas) return SP24_ERR_SHAPE;
+  if (!workspace || ws_bytes < sp24::kFusedCounterBytes + pl.workspace_bytes()) return SP24_ERR_WORKSPACE;
   if (!aligned16(workspace)) return SP24_ERR_ALIGN;
   sp24::GemmFusedX fx;
   fx.x = X;
@@ -319,7 +320,7 @@ static int quant_gemm_common(bool lift, const void *X, int M, int N, int K, cons
   fx.x_scale = x_scale;
   fx.counters = static_cast<uint32_t *>(workspace);
   return cuda_status(sp24::launch_gemm_quant(pl, fx, packed, w_scale, Y, M, N, Kg,
-                                             static_cast<uint8_t *>(workspace) + sp24::kAmaxWorkspaceBytes,
+                                             static_cast<uint8_t *>(workspace) + sp24::kFusedCounterBytes,
                                              status, reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -142,7 +142,11 @@ struct KindTraits<kSparseBF16> {
 // two blocks per stage halve it.  Packed weights only: the stage's two
 // blocks of a row tile are adjacent in memory (one bulk copy) and their
 // metadata is one 128x256b copy.
-template <int KIND, int BN, int MT = 1, int KB = 1>
+// Staged activation codes of the fused local quantisation (BN = 16 kernels):
+// up to this many bytes of E4M3 codes kept in shared memory.
+constexpr uint32_t kXStageBytes = 8192;
+
+template <int KIND, int BN, int MT = 1, int KB = 1, int XQ = 0>
 struct Config {
   using T = KindTraits<KIND>;
   static_assert(KB == 1 || (KB == 2 && T::kPacked && MT == 1), "two-block stages are for packed, one-row-tile tiles");
@@ -152,6 +156,7 @@ struct Config {
   static constexpr uint32_t kEBytes = kRows * T::kERowBytes * KB;
   static constexpr uint32_t kTBytes = T::kMetaTransform ? 128 * 16 : 0;  // TMEM-ready metadata
   static constexpr uint32_t kTmaBytes = kABytes + kBBytes + kEBytes;
+  static constexpr uint32_t kWBytes = kABytes + kEBytes;  // the weight half of a stage
   static constexpr uint32_t kStageBytes = kTmaBytes + kTBytes;
   static constexpr int kBSub = T::kBRowBytes * KB / 128;  // 128-byte X boxes per stage
   static constexpr int kMmas = T::kMmas * KB;             // MMAs per row tile per stage
@@ -179,6 +184,10 @@ struct Config {
   static constexpr int kThreads = 64 + kEpiThreads;
   static constexpr int kRtPerWarp = MT * 4 / kEpiWarps;  // row tiles each epilogue warp drains
   static constexpr uint32_t kSmemBudget = BN <= 64 ? 108 * 1024 : (kEpiWarps == 8 ? 224 * 1024 : 214 * 1024);
+  // Decode-sized tiles: two CTAs must fit an SM (shared memory above, and
+  // registers: at most 65536 / (2 * kThreads) per thread), or the next
+  // kernel cannot start streaming its weights before this one ends.
+  static constexpr int kMinBlocks = BN <= 64 ? 2 : 1;
   // Wide token tiles write Y through shared memory: each epilogue warp
   // stages its 32 rows x 32 tokens of a pass (2 KB of bf16) in one of two
   // buffers of its own and stores them with a 2-D bulk tensor copy, so the
@@ -188,9 +197,10 @@ struct Config {
   static constexpr bool kTmaStoreY = BN >= 128;
   static constexpr uint32_t kStageY = 32 * 32 * 2;          // one warp's pass
   static constexpr uint32_t kYBytes = kTmaStoreY ? kEpiWarps * 2 * kStageY : 0;
-  static constexpr int kStagesRaw = static_cast<int>((kSmemBudget - kYBytes) / kStageBytes);
+  static constexpr uint32_t kXStage = (XQ != 0 && BN == 16) ? kXStageBytes : 0;
+  static constexpr int kStagesRaw = static_cast<int>((kSmemBudget - kYBytes - kXStage) / kStageBytes);
   static constexpr int kStages = kStagesRaw > 16 ? 16 : kStagesRaw;
-  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kYBytes + 1024 /*align*/ + 1024 /*bars*/;
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kYBytes + kXStage + 1024 /*align*/ + 1024 /*bars*/;
   // Accumulators: MT x BN columns each; two of them (the epilogue of one
   // output tile overlaps the main loop of the next) whenever they fit in the
   // 512 TMEM columns next to the 4 metadata columns per row tile.
@@ -238,13 +248,14 @@ struct GemmArgs {
   const uint8_t *packed;  // tile-packed weights (packed kind only)
   // Fused activation quantisation (XQ != 0): bf16 X of xvec 8-element
   // vectors in, its E4M3 codes (lifted for XQ = 2) out to xq, which is the
-  // B operand the kernel then loads; xbar = [amax bits, arrivals, codes
-  // written, departures], zero between calls.
+  // B operand the kernel then loads; xbar = the kFusedCounterBytes prefix
+  // (departure count and per-CTA slots, see kXSlotAmax), zero between calls.
   const uint16_t *x;
   uint8_t *xq;
   float *x_scale_out;
   uint32_t *xbar;
   int64_t xvec;
+  int xstaged;  // local form with the codes staged in shared memory (kXStage)
   // Scale vectors (VS kernels): x_scale holds M per-token scales when x_vec,
   // w_scale N per-channel scales when w_vec; otherwise one value each.
   int x_vec, w_vec;
@@ -319,6 +330,16 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
   return v;
 }
 
+__device__ __forceinline__ void st_release_gpu(uint32_t *p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Spin (bounded) until *p reaches `expect`; acquire semantics.
 __device__ __forceinline__ void wait_count_gpu(const uint32_t *p, uint32_t expect, int32_t *status) {
   const uint64_t t0 = global_timer_ns();
@@ -334,104 +355,213 @@ __device__ __forceinline__ void wait_count_gpu(const uint32_t *p, uint32_t expec
 
 // Per-tensor E4M3 quantisation of the activations fused in front of the
 // GEMM, run by the 128 epilogue threads (t = 0..127) while the producer
-// already streams weights.  Two forms:
+// already streams weights.  Each thread loads its vectors of X once (up to
+// kXReg 16-byte vectors kept in registers; more are loaded again to encode)
+// and encodes them with e4m3_code_quot, which equals the correctly rounded
+// division on every input.  Two forms:
 //  * grid-wide (the usual one): (1) amax of this CTA's slice of X (a
-//    contiguous range of 8-element vectors), (2) a grid-wide max through
-//    xbar[0] and an arrival count, (3) s = amax / 448 (1 when amax = 0) and
-//    this slice's codes E4M3(RN_fp32(x / s)) written to xq, (4) a second
-//    count, xbar[2], that every CTA's producer waits for before it loads X
-//    codes.  Every CTA is resident (at most one per SM, cooperative launch),
-//    so both counts complete; each wait is bounded anyway.
+//    contiguous range of 8-element vectors), (2) written to the CTA's amax
+//    slot; CTA 0 takes the max over every slot and publishes it (see
+//    kXCopies), (3) s = amax / 448 (1 when amax = 0) and this slice's codes
+//    E4M3(RN_fp32(x / s)) written to xq, (4) the CTA's codes slot set; CTA
+//    0's producer waits for every codes slot and publishes, and every
+//    producer waits for that before it loads X codes, then counts its CTA's
+//    departure in xbar[3].  Every CTA becomes resident (at most one per SM,
+//    and one fits), so the slots fill; each wait is bounded anyway.
 //  * local (X of at most kLocalXVec vectors): every CTA takes the amax of
-//    all of X and encodes all of it itself, so no CTA waits for another; the
-//    codes every CTA writes are identical, and each CTA's producer waits
-//    only for its own CTA (x_ready).
-//  * between the two (X of at most kLocalAmaxXVec vectors): every CTA takes
-//    the amax of all of X (no first count), then encodes its slice as in
-//    the grid-wide form.
+//    all of X and encodes all of it itself, so no CTA waits for another and
+//    the counters are not touched.  When the codes fit kXStageBytes
+//    (`xstage`, BN = 16 kernels) they go to shared memory, from where the
+//    producer copies each stage's rows into its B tile, and only CTA 0
+//    writes them to xq for the caller; otherwise every CTA writes the
+//    (identical) codes to xq and its producer TMA-loads them.  Either way
+//    the producer waits for this CTA only (x_ready).
 // XQ = 2 writes the SlideSparse lift: each 8-group g of a row becomes the 12
 // codes of windows 2j..2j+3, j = 0..2.  Returns s.
 constexpr int64_t kLocalXVec = 1024;
-constexpr int64_t kLocalAmaxXVec = 4096;
+constexpr int kXReg = 8;
+// Grid-wide form: 32-bit words of the counter prefix (kFusedCounterBytes).
+// CTA g writes its amax | 0x10000 (nonzero) to slot kXSlotAmax + g and, once
+// its codes are written, 1 to kXSlotCodes + g; each slot is written once per
+// call.  CTA 0 alone polls the slots (one warp: every CTA polling the same
+// few lines made their writes queue behind the reads for microseconds) and
+// publishes the result to kXCopies copies, one per 128-byte line, which the
+// other CTAs poll (CTA g the copy g % kXCopies).  Word 3 counts departures;
+// the last CTA to leave clears slots and copies.  GPU-scope fences are few:
+// the release before a codes slot, CTA 0's acquire-and-release before the
+// codes copies and before its departure, and each reader's acquire.
+constexpr int kXCopies = 16;
+constexpr int kXCopyAmax = 32;                      // copy f at word kXCopyAmax + 32 f
+constexpr int kXCopyCodes = 32 * (1 + kXCopies);    // copy f at word kXCopyCodes + 32 f
+constexpr int kXSlotAmax = 32 * (1 + 2 * kXCopies);  // slot g at word kXSlotAmax + g
+constexpr int kXSlotCodes = kXSlotAmax + 256;
+
+__device__ __forceinline__ void st_relaxed_gpu(uint32_t *p, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Poll (bounded; backing off from 32 to 256 ns) until *p is nonzero and
+// return it.  No fence: the caller adds one when the word releases other
+// data.
+__device__ __forceinline__ uint32_t wait_word_gpu(const uint32_t *p, int32_t *status) {
+  uint32_t v = ld_relaxed_gpu(p);
+  if (v == 0u) {
+    const uint64_t t0 = global_timer_ns();
+    uint32_t ns = 32, polls = 0;
+    while ((v = ld_relaxed_gpu(p)) == 0u) {
+      __nanosleep(ns);
+      ns = min(ns * 2u, 256u);
+      if ((++polls & 15u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+        if (status) atomicOr(status, SP24_STATUS_TIMEOUT);
+        break;
+      }
+    }
+  }
+  return v;
+}
+
+// One warp (all 32 lanes) polls slots[0 .. n), n <= 256, until every slot is
+// nonzero (bounded; the loads of a poll are all in flight at once, and the
+// polls back off from 64 to 256 ns) and returns the largest value.  No fence:
+// the caller adds one when the slots release other data.
+__device__ __forceinline__ uint32_t wait_slots_warp(const uint32_t *slots, int n, int32_t *status) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t t0 = global_timer_ns();
+  uint32_t polls = 0, ns = 64, mx = 0;
+  while (true) {
+    uint32_t v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = lane + 32 * j < n ? ld_relaxed_gpu(slots + lane + 32 * j) : 1u;
+    uint32_t mn = 0xFFFFFFFFu;
+    mx = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      mn = min(mn, v[j]);
+      mx = max(mx, v[j]);
+    }
+    if (__all_sync(0xFFFFFFFFu, mn != 0u)) break;
+    __nanosleep(ns);
+    ns = min(ns * 2u, 256u);
+    if ((++polls & 15u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+      if (lane == 0 && status) atomicOr(status, SP24_STATUS_TIMEOUT);
+      break;
+    }
+  }
+  return __reduce_max_sync(0xFFFFFFFFu, mx);
+}
 
 template <int XQ>
-__device__ __forceinline__ void encode_xvec(const GemmArgs &p, int64_t v, const uint4 w, float sx) {
-  const uint32_t h[4] = {w.x, w.y, w.z, w.w};
-  uint32_t c[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    c[2 * i] = e4m3_code(__fdiv_rn(bf16_bits_to_float(h[i] & 0xFFFFu), sx));
-    c[2 * i + 1] = e4m3_code(__fdiv_rn(bf16_bits_to_float(h[i] >> 16), sx));
-  }
+__device__ __forceinline__ void store_xvec(uint8_t *dst, int64_t v, const uint2 c) {
   if constexpr (XQ == 1) {
-    *reinterpret_cast<uint2 *>(p.xq + 8 * v) =
-        make_uint2(c[0] | c[1] << 8 | c[2] << 16 | c[3] << 24, c[4] | c[5] << 8 | c[6] << 16 | c[7] << 24);
+    *reinterpret_cast<uint2 *>(dst + 8 * v) = c;
   } else {
-    uint32_t *o = reinterpret_cast<uint32_t *>(p.xq + 12 * v);
-    o[0] = c[0] | c[1] << 8 | c[2] << 16 | c[3] << 24;
-    o[1] = c[2] | c[3] << 8 | c[4] << 16 | c[5] << 24;
-    o[2] = c[4] | c[5] << 8 | c[6] << 16 | c[7] << 24;
+    uint32_t *o = reinterpret_cast<uint32_t *>(dst + 12 * v);
+    o[0] = c.x;
+    o[1] = __byte_perm(c.x, c.y, 0x5432);  // codes 2..5
+    o[2] = c.y;
   }
 }
 
 template <int XQ>
-__device__ float fused_quantize(const GemmArgs &p, int t, uint32_t *s_red, float *s_scale, uint64_t *x_ready) {
+__device__ float fused_quantize(const GemmArgs &p, int t, uint32_t *s_red, float *s_scale, uint64_t *x_ready,
+                                uint8_t *xstage) {
   const bool local = p.xvec <= kLocalXVec;
-  const bool local_amax = p.xvec <= kLocalAmaxXVec;
   const int64_t v0 = local ? 0 : static_cast<int64_t>(blockIdx.x) * p.xvec / gridDim.x;
   const int64_t v1 = local ? p.xvec : static_cast<int64_t>(blockIdx.x + 1) * p.xvec / gridDim.x;
   const uint4 *xv = reinterpret_cast<const uint4 *>(p.x);
-  // kXBatch independent 16-byte loads per thread in flight at a time
-  constexpr int kXBatch = 8;
+  // vectors v0 + t + 128 u, u < kXReg: all loads in flight at once, kept
+  uint4 w[kXReg];
+#pragma unroll
+  for (int u = 0; u < kXReg; ++u)
+    w[u] = v0 + t + 128 * u < v1 ? __ldg(xv + v0 + t + 128 * u) : make_uint4(0u, 0u, 0u, 0u);
   uint32_t m2 = 0;
-  {
-    const int64_t a0 = local_amax ? 0 : v0, a1 = local_amax ? p.xvec : v1;
-    for (int64_t v = a0 + t; v < a1; v += 128 * kXBatch) {
-      uint4 w[kXBatch];
 #pragma unroll
-      for (int u = 0; u < kXBatch; ++u)
-        w[u] = v + 128 * u < a1 ? __ldg(xv + v + 128 * u) : make_uint4(0u, 0u, 0u, 0u);
+  for (int u = 0; u < kXReg; ++u) m2 = __vmaxu2(m2, absmax8x2(w[u]));
+  for (int64_t v = v0 + t + 128 * kXReg; v < v1; v += 128 * kXReg) {  // large X: batches of kXReg loads
+    uint4 r[kXReg];
 #pragma unroll
-      for (int u = 0; u < kXBatch; ++u) m2 = __vmaxu2(m2, absmax8x2(w[u]));
-    }
+    for (int u = 0; u < kXReg; ++u) r[u] = v + 128 * u < v1 ? __ldg(xv + v + 128 * u) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < kXReg; ++u) m2 = __vmaxu2(m2, absmax8x2(r[u]));
   }
   uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
   if ((t & 31) == 0) s_red[t >> 5] = mx;
   named_bar_sync(1, 128);
-  if (t == 0) {
+  if (t < 32) {
     mx = max(max(s_red[0], s_red[1]), max(s_red[2], s_red[3]));
     uint32_t amax = mx;
-    if (!local_amax) {
-      red_max_relaxed_gpu(&p.xbar[0], mx);
-      red_release_add_gpu(&p.xbar[1], 1u);  // orders the max before the arrival
-      wait_count_gpu(&p.xbar[1], gridDim.x, p.status);
-      amax = ld_acquire_gpu(&p.xbar[0]);
+    if (!local) {
+      if (t == 0) st_relaxed_gpu(&p.xbar[kXSlotAmax + blockIdx.x], mx | 0x10000u);
+      if (blockIdx.x == 0) {
+        amax = wait_slots_warp(&p.xbar[kXSlotAmax], gridDim.x, p.status) & 0xFFFFu;
+        if (t < kXCopies) st_relaxed_gpu(&p.xbar[kXCopyAmax + 32 * t], amax | 0x10000u);  // the data itself
+      } else if (t == 0) {
+        amax = wait_word_gpu(&p.xbar[kXCopyAmax + 32 * (blockIdx.x % kXCopies)], p.status) & 0xFFFFu;
+      }
     }
-    const float sx = amax == 0u ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax), 448.0f);
-    if (blockIdx.x == 0) {
-      if (amax >= 0x7F80u && p.status) atomicOr(p.status, SP24_STATUS_NONFINITE);
-      *p.x_scale_out = sx;
+    if (t == 0) {
+      const float sx = amax == 0u ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax), 448.0f);
+      if (blockIdx.x == 0) {
+        if (amax >= 0x7F80u && p.status) atomicOr(p.status, SP24_STATUS_NONFINITE);
+        *p.x_scale_out = sx;
+      }
+      s_scale[0] = sx;
+      s_scale[1] = __frcp_rn(sx);
     }
-    *s_scale = sx;
   }
   named_bar_sync(1, 128);
-  const float sx = *s_scale;
-  for (int64_t v = v0 + t; v < v1; v += 128 * kXBatch) {
-    uint4 w[kXBatch];
+  const float sx = s_scale[0], rx = s_scale[1];
+  uint8_t *dst = xstage ? xstage : p.xq;
+  const bool also_out = xstage && blockIdx.x == 0;  // staged codes: CTA 0 returns them
+  {
+    // this thread's vectors in registers: v0 + t + 128 u for u < nv, encoded
+    // two at a time (the pairs interleave; no work for absent vectors)
+    const int64_t mine = v1 - v0 - t;
+    const int nv = mine <= 0 ? 0 : static_cast<int>(mine >= 128 * kXReg ? kXReg : (mine + 127) / 128);
 #pragma unroll
-    for (int u = 0; u < kXBatch; ++u)
-      if (v + 128 * u < v1) w[u] = __ldg(xv + v + 128 * u);
-#pragma unroll
-    for (int u = 0; u < kXBatch; ++u)
-      if (v + 128 * u < v1) encode_xvec<XQ>(p, v + 128 * u, w[u], sx);
+    for (int u = 0; u < kXReg; u += 2) {
+      if (u < nv) {
+        bool ok0, ok1;
+        uint2 c0 = e4m3_codes8_fast(w[u], rx, ok0);
+        uint2 c1 = e4m3_codes8_fast(w[u + 1], rx, ok1);
+        if (!ok0) c0 = e4m3_codes8_div(w[u], sx);
+        if (!ok1) c1 = e4m3_codes8_div(w[u + 1], sx);
+        const int64_t v = v0 + t + 128 * u;
+        store_xvec<XQ>(dst, v, c0);
+        if (also_out) store_xvec<XQ>(p.xq, v, c0);
+        if (u + 1 < nv) {
+          store_xvec<XQ>(dst, v + 128, c1);
+          if (also_out) store_xvec<XQ>(p.xq, v + 128, c1);
+        }
+      }
+    }
   }
-  fence_proxy_async_global();  // the codes are read back by TMA loads
+  for (int64_t v = v0 + t + 128 * kXReg; v < v1; v += 128 * kXReg) {
+    uint4 r[kXReg];
+#pragma unroll
+    for (int u = 0; u < kXReg; ++u) r[u] = v + 128 * u < v1 ? __ldg(xv + v + 128 * u) : make_uint4(0u, 0u, 0u, 0u);
+    uint2 c[kXReg];
+    bool ok[kXReg];
+#pragma unroll
+    for (int u = 0; u < kXReg; ++u) c[u] = e4m3_codes8_fast(r[u], rx, ok[u]);
+#pragma unroll
+    for (int u = 0; u < kXReg; ++u)
+      if (!ok[u]) c[u] = e4m3_codes8_div(r[u], sx);
+#pragma unroll
+    for (int u = 0; u < kXReg; ++u) {
+      if (v + 128 * u < v1) {
+        store_xvec<XQ>(dst, v + 128 * u, c[u]);
+        if (also_out) store_xvec<XQ>(p.xq, v + 128 * u, c[u]);
+      }
+    }
+  }
+  if (!xstage) fence_proxy_async_global();  // the codes are read back by TMA loads
   named_bar_sync(1, 128);
   if (t == 0) {
     if (local)
       mbar_arrive(x_ready);
     else
-      red_release_add_gpu(&p.xbar[2], 1u);
+      st_release_gpu(&p.xbar[kXSlotCodes + blockIdx.x], 1u);  // releases the codes (bar.sync above)
   }
   return sx;
 }
@@ -446,12 +576,12 @@ __device__ __forceinline__ float token_scale(const GemmArgs &p, int m, float sx)
 // ------------------------------------------------------------------ kernel
 
 template <int KIND, int BN, int MT, int XQ, int KB, bool VS>
-__global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
+__global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config<KIND, BN, MT, KB, XQ>::kMinBlocks)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
                 const GemmArgs p) {
   using T = KindTraits<KIND>;
-  using C = Config<KIND, BN, MT, KB>;
+  using C = Config<KIND, BN, MT, KB, XQ>;
   constexpr int S = C::kStages;
   constexpr int NB = C::kAccBufs;
 
@@ -459,7 +589,8 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *ystage = smem + S * C::kStageBytes;  // kYBytes: two staged Y passes
-  uint64_t *full = reinterpret_cast<uint64_t *>(ystage + C::kYBytes);
+  uint8_t *xstage = ystage + C::kYBytes;         // kXStage: staged activation codes
+  uint64_t *full = reinterpret_cast<uint64_t *>(xstage + C::kXStage);
   uint64_t *empty = full + S;
   uint64_t *meta_ready = empty + S;
   uint64_t *tmem_full = meta_ready + S;
@@ -467,7 +598,7 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
   uint64_t *x_ready = tmem_empty + NB;  // fused local quantisation: codes written
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(x_ready + 1);
   [[maybe_unused]] __shared__ uint32_t s_xred[4];
-  [[maybe_unused]] __shared__ float s_xscale;
+  [[maybe_unused]] __shared__ float s_xscale[2];
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -504,12 +635,18 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
   // not release their dependents early, so the producer may stream weight
   // tiles right away; activations, scales and Y are touched only after
   // griddepcontrol.wait, i.e. after the previous kernel has completed.
-  if (threadIdx.x != 0) grid_dependency_wait();
+  if (warp != 0) grid_dependency_wait();
   grid_launch_dependents();
 
+  // The producer and MMA warps walk the schedule with all 32 lanes, combine
+  // their barrier waits by vote and issue every TMA / tcgen05 instruction
+  // from one elected lane: the loop counters, addresses and descriptors are
+  // then warp-uniform, which the issue of those instructions needs to be
+  // cheap.
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    {
+      const bool leader = elect_one();
       const uint64_t keep_x = l2_policy_evict_last();  // X tiles are re-read by many CTAs
       // Weights are read once when there is a single token tile; otherwise
       // every token tile re-reads them and they should stay in L2.
@@ -528,8 +665,26 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
           if (T::kSparse) tma_load_2d(st + C::kEOff, &tmE, bar, kb * T::kERowBytes, n0, stream_w);
         }
       };
+      // Staged activation codes (fused local quantisation): the producer
+      // copies each stage's X rows from shared memory into the stage's B tile
+      // (the 128-byte swizzle: 16-byte chunk c of row m at c ^ (m & 7)); the
+      // rows past M are left as they are, since they only feed output
+      // columns that are never stored.
+      const bool staged = C::kXStage > 0 && p.xstaged;
+      auto copy_x_rows = [&](uint8_t *st, int kb) {
+        for (int q = lane; q < p.M * KB * 8; q += 32) {
+          const int c = q & 7, u = (q >> 3) % KB, m = q / (8 * KB);
+          const uint4 v = *reinterpret_cast<const uint4 *>(xstage + static_cast<int64_t>(m) * p.K +
+                                                           (kb * KB + u) * 128 + c * 16);
+          *reinterpret_cast<uint4 *>(st + C::kBOff + u * BN * 128 + m * 128 + ((c ^ (m & 7)) * 16)) = v;
+        }
+        fence_proxy_async_smem();  // generic writes, read by the MMA (async proxy)
+        __syncwarp();
+      };
       // Pass 1 (before the grid dependency resolves): the weight half of the
-      // first S stages.  Pass 2: everything else, in the same stage order.
+      // first S stages (with staged codes the stage's arrival waits for the
+      // X copy: only the transaction bytes are announced here).  Pass 2:
+      // everything else, in the same stage order.
       SegIter it;
       it.init(p);
       Segment sg;
@@ -544,8 +699,37 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
           const int n0 = (s0.tile % p.tiles_n) * C::kRows;
           for (int kb = s0.kb0; kb < s0.kb1 && pre < S; ++kb, ++pre) {
             uint8_t *st = smem + pre * C::kStageBytes;
-            mbar_arrive_expect_tx(&full[pre], C::kTmaBytes);
-            load_weights(st, &full[pre], n0, kb);
+            if (leader) {
+              if (staged)
+                mbar_expect_tx(&full[pre], C::kWBytes);
+              else
+                mbar_arrive_expect_tx(&full[pre], C::kTmaBytes);
+              load_weights(st, &full[pre], n0, kb);
+            }
+          }
+        }
+      }
+      // The rest of this CTA's weights, when they are read once (a single
+      // token tile): one L2 prefetch per segment, also issued before the
+      // dependency resolves, so that the CTA's whole weight share streams
+      // from HBM while the previous kernel drains, and the stages after the
+      // first S refill from L2.
+      if constexpr (T::kPacked && MT == 1) {
+        if (tiles_m == 1 && leader) {
+          const uint64_t keep_w = l2_policy_evict_normal();
+          SegIter it1;
+          it1.init(p);
+          Segment s1;
+          int st_i = 0;
+          while (it1.next(p, s1)) {
+            const int nblk = s1.kb1 - s1.kb0;
+            const int skip = min(nblk, max(0, pre - st_i));  // stages already loaded into the ring
+            if (skip < nblk) {
+              const uint8_t *src = p.packed + ((static_cast<int64_t>(s1.tile % p.tiles_n) * p.num_kb + s1.kb0 + skip) * KB) *
+                                                  kPackedBlockBytes;
+              bulk_prefetch_l2(src, static_cast<uint32_t>((nblk - skip) * KB * kPackedBlockBytes), keep_w);
+            }
+            st_i += nblk;
           }
         }
       }
@@ -553,11 +737,42 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
       if constexpr (XQ != 0) {
         // the activation codes are written by the epilogue warps: of this
         // CTA (local form) or of the whole grid
-        if (p.xvec <= kLocalXVec)
-          mbar_wait(x_ready, 0u, p.status);
-        else
-          wait_count_gpu(&p.xbar[2], gridDim.x, p.status);
-        fence_proxy_async_global();
+        if (p.xvec <= kLocalXVec) {
+          mbar_wait_warp(x_ready, 0u, p.status);
+        } else {
+          if (blockIdx.x == 0) {
+            // gather every CTA's codes slot, acquire their codes and release
+            // them again through the copies
+            wait_slots_warp(&p.xbar[kXSlotCodes], gridDim.x, p.status);
+            __syncwarp();
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");
+            if (lane < kXCopies) st_relaxed_gpu(&p.xbar[kXCopyCodes + 32 * lane], 1u);
+            __syncwarp();
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");  // the copies before the departure below
+          } else {
+            if (leader) wait_word_gpu(&p.xbar[kXCopyCodes + 32 * (blockIdx.x % kXCopies)], p.status);
+            __syncwarp();
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire every CTA's codes
+          }
+          // This CTA reads the slots and copies no more (its epilogue read
+          // the amax before setting its codes slot): count its departure;
+          // the last CTA to leave clears them.
+          uint32_t last = 0;
+          if (leader) last = atomicAdd(&p.xbar[3], 1u) == gridDim.x - 1 ? 1u : 0u;
+          if (__shfl_sync(0xFFFFFFFFu, last, 0)) {  // the leader is lane 0 of the converged warp
+            for (int g = lane; g < static_cast<int>(gridDim.x); g += 32) {
+              p.xbar[kXSlotAmax + g] = 0u;
+              p.xbar[kXSlotCodes + g] = 0u;
+            }
+            if (lane < kXCopies) {
+              p.xbar[kXCopyAmax + 32 * lane] = 0u;
+              p.xbar[kXCopyCodes + 32 * lane] = 0u;
+            }
+            if (leader) p.xbar[3] = 0u;
+          }
+        }
+        __syncwarp();
+        if (!staged) fence_proxy_async_global();
       }
       while (ok && it.next(p, sg)) {
         const int n0 = (sg.tile % p.tiles_n) * C::kRows;
@@ -567,24 +782,40 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
           const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
           uint8_t *st = smem + s * C::kStageBytes;
           if (i >= pre) {
-            if (i >= S && !mbar_wait(&empty[s], ph ^ 1u, p.status)) {
+            if (i >= S && !mbar_wait_warp(&empty[s], ph ^ 1u, p.status)) {
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&full[s], C::kTmaBytes);
-            load_weights(st, &full[s], n0, kb);
+            if (leader && !staged) {
+              mbar_arrive_expect_tx(&full[s], C::kTmaBytes);
+              load_weights(st, &full[s], n0, kb);
+            }
           }
+          if (staged) {
+            copy_x_rows(st, kb);
+            if (leader) {
+              if (i >= pre) {
+                mbar_arrive_expect_tx(&full[s], C::kWBytes);
+                load_weights(st, &full[s], n0, kb);
+              } else {
+                mbar_arrive(&full[s]);
+              }
+            }
+          } else if (leader) {
 #pragma unroll
-          for (int sub = 0; sub < C::kBSub; ++sub)
-            tma_load_2d(st + C::kBOff + sub * BN * 128, &tmB, &full[s],
-                        kb * (T::kBRowBytes * KB / T::kBElemBytes) + sub * T::kBBoxElems, m0, keep_x);
+            for (int sub = 0; sub < C::kBSub; ++sub)
+              tma_load_2d(st + C::kBOff + sub * BN * 128, &tmB, &full[s],
+                          kb * (T::kBRowBytes * KB / T::kBElemBytes) + sub * T::kBBoxElems, m0, keep_x);
+          }
+          __syncwarp();
         }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {
+      const bool leader = elect_one();
       constexpr uint32_t idesc = mma_idesc(128, BN, T::kFmt, T::kSparse, T::kDFmt);
       // metadata of row tile i: 4 TMEM columns after all accumulators
       const uint32_t e_tmem = tmem_base + NB * C::kAccCols;
@@ -596,65 +827,69 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
       while (ok && it.next(p, sg)) {
         const int b = j % NB;
         const int r = j / NB;
-        if (r >= 1 && !mbar_wait(&tmem_empty[b], static_cast<uint32_t>(r - 1) & 1u, p.status)) break;
+        if (r >= 1 && !mbar_wait_warp(&tmem_empty[b], static_cast<uint32_t>(r - 1) & 1u, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * C::kAccCols;  // row tile rt at + rt * BN
         for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++i) {
           const int s = i % S;
           const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
-          if (!mbar_wait(&full[s], ph, p.status) ||
-              (T::kMetaTransform && !mbar_wait(&meta_ready[s], ph, p.status))) {
+          if (!mbar_wait_warp(&full[s], ph, p.status) ||
+              (T::kMetaTransform && !mbar_wait_warp(&meta_ready[s], ph, p.status))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t st_addr = smem_addr(smem + s * C::kStageBytes);
           const uint32_t b_addr = st_addr + C::kBOff;
-          if (T::kSparse) {
-            // 128 rows x 16 B, rows contiguous: core matrices of 8 rows are 128 B apart.
-            if constexpr (T::kPacked && MT * KB == 2) {
-              // two packed blocks' metadata in one copy (both row tiles, or
-              // both k-blocks of one row tile): the second 16-byte column is
-              // the next block's metadata, 10240 bytes on
-              tmem_copy_128x256b(e_tmem, smem_desc(st_addr + C::e_off(0), kPackedBlockBytes, 128, kSwizzleNone));
-            } else {
-#pragma unroll
-              for (int rt = 0; rt < MT; ++rt) {
-                const uint32_t e_addr = st_addr + C::e_off(rt) + (T::kMetaTransform ? C::kEBytes : 0);
-                tmem_copy_128x128b(e_tmem + 4 * rt, smem_desc(e_addr, 2048, 128, kSwizzleNone));
-              }
-            }
-          }
-#pragma unroll
-          for (int rt = 0; rt < MT; ++rt) {
-            const uint32_t a_addr = st_addr + C::a_off(rt);
-#pragma unroll
-            for (int kk = 0; kk < C::kMmas; ++kk) {
-              // MMA kk reads block kk / kMmas of the stage (packed blocks are
-              // 10240 bytes apart), step kk % kMmas within it
-              const uint32_t a_k = KB == 1 ? kk * T::kAStep
-                                           : (kk / T::kMmas) * kPackedBlockBytes + (kk % T::kMmas) * T::kAStep;
-              const uint64_t ad = smem_desc(a_addr + a_k, 16, T::kASbo, T::kASwizzle);
-              const uint32_t boff = (kk * T::kBStep / 128) * (BN * 128) + (kk * T::kBStep) % 128;
-              const uint64_t bd = smem_desc(b_addr + boff, 16, 8 * 128, kSwizzle128B);
-              const uint32_t acc = (kb > sg.kb0 || kk > 0) ? 1u : 0u;
-              const uint32_t d = d_tmem + rt * BN;
-              if constexpr (KIND == kSparseE4M3 || KIND == kSparseE4M3Packed) {
-                mma_f8_sparse(d, ad, bd, idesc, e_tmem + 4 * rt + 2 * kk, acc);
-              } else if constexpr (KIND == kSparseI8Packed) {
-                mma_i8_sparse(d, ad, bd, idesc, e_tmem + 4 * rt + 2 * kk, acc);
-              } else if constexpr (KIND == kSparseBF16) {
-                // one metadata column per MMA; columns are addressed in pairs and
-                // the instruction descriptor's selector picks the column of the pair
-                mma_bf16_sparse(d, ad, bd, idesc | static_cast<uint32_t>(kk & 1), e_tmem + (kk & ~1), acc);
+          if (leader) {
+            if (T::kSparse) {
+              // 128 rows x 16 B, rows contiguous: core matrices of 8 rows are 128 B apart.
+              if constexpr (T::kPacked && MT * KB == 2) {
+                // two packed blocks' metadata in one copy (both row tiles, or
+                // both k-blocks of one row tile): the second 16-byte column is
+                // the next block's metadata, 10240 bytes on
+                tmem_copy_128x256b(e_tmem, smem_desc(st_addr + C::e_off(0), kPackedBlockBytes, 128, kSwizzleNone));
               } else {
-                mma_f8_dense(d, ad, bd, idesc, acc);
+#pragma unroll
+                for (int rt = 0; rt < MT; ++rt) {
+                  const uint32_t e_addr = st_addr + C::e_off(rt) + (T::kMetaTransform ? C::kEBytes : 0);
+                  tmem_copy_128x128b(e_tmem + 4 * rt, smem_desc(e_addr, 2048, 128, kSwizzleNone));
+                }
               }
             }
+#pragma unroll
+            for (int rt = 0; rt < MT; ++rt) {
+              const uint32_t a_addr = st_addr + C::a_off(rt);
+#pragma unroll
+              for (int kk = 0; kk < C::kMmas; ++kk) {
+                // MMA kk reads block kk / kMmas of the stage (packed blocks are
+                // 10240 bytes apart), step kk % kMmas within it
+                const uint32_t a_k = KB == 1 ? kk * T::kAStep
+                                             : (kk / T::kMmas) * kPackedBlockBytes + (kk % T::kMmas) * T::kAStep;
+                const uint64_t ad = smem_desc(a_addr + a_k, 16, T::kASbo, T::kASwizzle);
+                const uint32_t boff = (kk * T::kBStep / 128) * (BN * 128) + (kk * T::kBStep) % 128;
+                const uint64_t bd = smem_desc(b_addr + boff, 16, 8 * 128, kSwizzle128B);
+                const uint32_t acc = (kb > sg.kb0 || kk > 0) ? 1u : 0u;
+                const uint32_t d = d_tmem + rt * BN;
+                if constexpr (KIND == kSparseE4M3 || KIND == kSparseE4M3Packed) {
+                  mma_f8_sparse(d, ad, bd, idesc, e_tmem + 4 * rt + 2 * kk, acc);
+                } else if constexpr (KIND == kSparseI8Packed) {
+                  mma_i8_sparse(d, ad, bd, idesc, e_tmem + 4 * rt + 2 * kk, acc);
+                } else if constexpr (KIND == kSparseBF16) {
+                  // one metadata column per MMA; columns are addressed in pairs and
+                  // the instruction descriptor's selector picks the column of the pair
+                  mma_bf16_sparse(d, ad, bd, idesc | static_cast<uint32_t>(kk & 1), e_tmem + (kk & ~1), acc);
+                } else {
+                  mma_f8_dense(d, ad, bd, idesc, acc);
+                }
+              }
+            }
+            mma_commit(&empty[s]);
           }
-          mma_commit(&empty[s]);
+          __syncwarp();
         }
-        mma_commit(&tmem_full[b]);
+        if (leader) mma_commit(&tmem_full[b]);
+        __syncwarp();
         ++j;
       }
     }
@@ -669,7 +904,7 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
     const int rt0 = (e >> 2) * C::kRtPerWarp;  // first row tile this warp drains
     float sx;
     if constexpr (XQ != 0)
-      sx = fused_quantize<XQ>(p, t, s_xred, &s_xscale, x_ready);
+      sx = fused_quantize<XQ>(p, t, s_xred, s_xscale, x_ready, C::kXStage > 0 && p.xstaged ? xstage : nullptr);
     else
       sx = p.x_scale ? __ldg(p.x_scale) : 1.0f;
     const float sw = p.w_scale ? __ldg(p.w_scale) : 1.0f;
@@ -926,19 +1161,6 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
-  if constexpr (XQ != 0) {
-    // Every thread of this CTA is past its waits on xbar; the last CTA to
-    // get here returns the counters to zero for the next call.
-    if (threadIdx.x == 64) {
-      __threadfence();
-      if (atomicAdd(&p.xbar[3], 1u) == gridDim.x - 1) {
-        p.xbar[0] = 0u;
-        p.xbar[1] = 0u;
-        p.xbar[2] = 0u;
-        p.xbar[3] = 0u;
-      }
-    }
-  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -1039,13 +1261,20 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
                                 cudaStream_t st, const GemmFusedX *fx = nullptr, int x_vec = 0,
                                 int w_vec = 0) {
   using T = KindTraits<KIND>;
-  using C = Config<KIND, BN, MT, KB>;
+  using C = Config<KIND, BN, MT, KB, XQ>;
   static_assert(XQ == 0 || KIND == kSparseE4M3Packed, "fused quantisation feeds the packed E4M3 GEMM");
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
     attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN, MT, XQ, KB, VS>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (attr_err == cudaSuccess && XQ != 0) {
+      // the fused quantisation's grid-wide counts rely on one CTA fitting an SM
+      int per_sm = 0;
+      attr_err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemm_kernel<KIND, BN, MT, XQ, KB, VS>,
+                                                               C::kThreads, C::kSmemBytes);
+      if (attr_err == cudaSuccess && per_sm < 1) attr_err = cudaErrorCooperativeLaunchTooLarge;
+    }
   });
   if (attr_err != cudaSuccess) return attr_err;
 
@@ -1103,6 +1332,7 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   a.x_scale_out = nullptr;
   a.xbar = nullptr;
   a.xvec = 0;
+  a.xstaged = 0;
   a.x_vec = x_vec;
   a.w_vec = w_vec;
   if constexpr (XQ != 0) {
@@ -1111,6 +1341,7 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
     a.x_scale_out = fx->x_scale;
     a.xbar = fx->counters;
     a.xvec = static_cast<int64_t>(M) * (XQ == 2 ? K / 3 * 2 : K) / 8;
+    a.xstaged = (C::kXStage > 0 && a.xvec <= kLocalXVec && static_cast<int64_t>(M) * K <= kXStageBytes) ? 1 : 0;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(pl.grid), 1, 1);
@@ -1118,18 +1349,19 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = st;
   // Programmatic dependent launch (see the kernel).  Stream-K owners wait
-  // for contributor CTAs; with at most one CTA per SM every CTA becomes
-  // resident once the SMs still held by the previous kernel drain, and each
-  // wait is bounded anyway.
-  // The fused quantisation's grid-wide counts need every CTA resident at
-  // once: a cooperative launch, which the driver refuses otherwise.
-  cudaLaunchAttribute attrs[2];
+  // for contributor CTAs, and the fused quantisation's grid-wide counts wait
+  // for every CTA.  Both only need every CTA to become resident eventually:
+  // the grid is at most one CTA per SM and one CTA fits an SM (checked once
+  // above), so every CTA is resident as soon as the kernels ahead of it
+  // drain, and each wait is bounded anyway.  The launch is not cooperative:
+  // a cooperative grid was measured to start 1-2 us later behind the
+  // previous kernel, losing the weight prefetch that programmatic launch
+  // overlaps with it.
+  cudaLaunchAttribute attrs[1];
   attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attrs[0].val.programmaticStreamSerializationAllowed = 1;
-  attrs[1].id = cudaLaunchAttributeCooperative;
-  attrs[1].val.cooperative = 1;
   cfg.attrs = attrs;
-  cfg.numAttrs = XQ != 0 ? 2 : 1;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, MT, XQ, KB, VS>, tmA, tmB, tmE, tmY, a);
 }
 

@@ -69,6 +69,13 @@ void set_last_cuda_error(int e);
 // Bytes of scratch the amax/scale reduction uses (two counters, padded).
 constexpr size_t kAmaxWorkspaceBytes = 256;
 
+// Counter prefix of the fused quantise + GEMM workspace: a line of counters,
+// 32 lines of published copies, then one 32-bit slot per CTA (at most
+// kFusedMaxCtas) for the amax and one for "codes written" (6272 bytes,
+// padded).  Zero before the first call and after every call.
+constexpr int kFusedMaxCtas = 256;
+constexpr size_t kFusedCounterBytes = 8192;
+
 // ---- gemm.cu
 enum GemmKind : int { kSparseE4M3 = 0, kDenseE4M3 = 1, kSparseBF16 = 2, kSparseE4M3Packed = 3, kSparseI8Packed = 4 };
 
@@ -119,7 +126,7 @@ struct GemmFusedX {
   int lift;            // 0: codes [M, Kx]; 1: SlideSparse lift, codes [M, 3 Kx / 2]
   uint8_t *xq;         // out: the E4M3 codes (the GEMM's B operand)
   float *x_scale;      // out: amax|X| / 448 (1 when amax = 0)
-  uint32_t *counters;  // 4 words, zero before the call and after it
+  uint32_t *counters;  // kFusedCounterBytes, zero before the call and after it
 };
 cudaError_t launch_gemm_quant(const GemmPlan &plan, const GemmFusedX &fx, const void *packed,
                               const float *w_scale, void *y, int M, int N, int K, void *workspace,

@@ -32,6 +32,67 @@ __device__ __forceinline__ uint32_t e4m3_code(float v) {
   return (c & 0x7Fu) == 0x7Fu ? 0x7Fu : c | ((__float_as_uint(v) >> 24) & 0x80u);
 }
 
+// E4M3 codes of RN_fp32(x / s) without a division on the common path.
+// r = RN(1 / s) is given.  q = RN(x * r) differs from x / s by less than
+// three units of x / s's last place (two roundings of relative size 2^-24
+// each), so at most six fp32 steps from RN(x / s) even across a binade
+// edge.  E4M3 rounding is monotone in the value, so when the fp32 values
+// eight steps either side of q have the same code, RN(x / s) has it too.
+// The check runs on four codes at once (one byte each); when it fails for
+// any of them (a rounding boundary within reach, about one value in 2^16;
+// NaN or Inf) the correctly rounded division decides all four.  The result
+// is exactly e4m3_code(__fdiv_rn(x, s)) for every x and s > 0.
+
+// The E4M3 codes of fp32 values hi and lo, in bits 8-15 and 0-7.
+__device__ __forceinline__ uint32_t e4m3_pair(float hi, float lo) {
+  uint16_t pr;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(hi), "f"(lo));
+  return pr;
+}
+
+// Codes of the four bf16 values of h0 (elements 0, 1) and h1 (2, 3), byte i
+// = element i; false when the division must decide.
+__device__ __forceinline__ bool e4m3_codes4_quot(uint32_t h0, uint32_t h1, float r, uint32_t &out) {
+  const uint32_t hh[4] = {h0 & 0xFFFFu, h0 >> 16, h1 & 0xFFFFu, h1 >> 16};
+  uint32_t p[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t u = __float_as_uint(__fmul_rn(bf16_bits_to_float(hh[i]), r));
+    const uint32_t mag = u & 0x7FFFFFFFu, sgn = u & 0x80000000u;
+    p[i] = e4m3_pair(__uint_as_float(sgn | (mag + 8u)), __uint_as_float(sgn | (mag > 8u ? mag - 8u : 0u)));
+  }
+  // bytes (low, high) of each pair: the codes 8 steps below and above q
+  const uint32_t w01 = p[0] | p[1] << 16, w23 = p[2] | p[3] << 16;
+  const uint32_t lo = __byte_perm(w01, w23, 0x6420), hi = __byte_perm(w01, w23, 0x7531);
+  // both ends equal, and no NaN code (magnitude 0x7F)
+  const uint32_t bad = (lo ^ hi) | (((lo & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u);
+  // the sign of every input (a value that rounds to zero keeps it)
+  out = lo | (__byte_perm(h0, h1, 0x7531) & 0x80808080u);
+  return bad == 0u;
+}
+
+// The exact form, out of line: rare, and kept out of the unrolled loops.
+static __device__ __noinline__ uint2 e4m3_codes8_div(const uint4 w, float s) {
+  const uint32_t h[4] = {w.x, w.y, w.z, w.w};
+  uint32_t q[2] = {0u, 0u};
+  for (int i = 0; i < 8; ++i)
+    q[i >> 2] |= e4m3_code(__fdiv_rn(bf16_bits_to_float((h[i >> 1] >> (16 * (i & 1))) & 0xFFFFu), s)) << (8 * (i & 3));
+  return make_uint2(q[0], q[1]);
+}
+
+// The codes of the 8 bf16 values of a 16-byte vector, packed little-endian
+// into two words, by the fast path; `ok` is false when e4m3_codes8_div must
+// produce them instead.  No call and no branch: a caller encoding several
+// vectors runs their fast paths interleaved and redoes the (rare) failed
+// vectors afterwards.
+__device__ __forceinline__ uint2 e4m3_codes8_fast(const uint4 w, float r, bool &ok) {
+  uint32_t a, b;
+  const bool oa = e4m3_codes4_quot(w.x, w.y, r, a);
+  const bool ob = e4m3_codes4_quot(w.z, w.w, r, b);
+  ok = oa && ob;
+  return make_uint2(a, b);
+}
+
 // Largest magnitude bit patterns of the 8 bf16 values of a 16-byte vector,
 // per 16-bit lane (the larger lane is the vector's).  For finite bf16 the
 // unsigned order of (bits & 0x7FFF) is the order of |x|; NaN/Inf patterns

@@ -41,6 +41,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                : "memory");
 }
 
+// Announce `bytes` more transaction bytes on the current phase without
+// arriving (the arrival comes later, from this or another thread).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -66,6 +72,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_
   }
   if (status) atomicOr(status, SP24_STATUS_TIMEOUT);
   return false;
+}
+
+// Warp-wide form for the single-issuer warps: every lane polls, and the
+// result is the vote of all lanes, so that the caller's control flow (and
+// every address or descriptor computed under it) stays warp-uniform.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, int32_t *status) {
+  const bool ok = mbar_wait(bar, parity, (threadIdx.x & 31) == 0 ? status : nullptr);
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// One lane of a converged warp (the same lane every time): the issuer of
+// TMA and tcgen05 instructions whose operands the whole warp computed.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
@@ -106,6 +132,14 @@ __device__ __forceinline__ void bulk_load_g2s(void *dst, const void *src, uint32
       " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
       : "memory");
+}
+
+// Prefetch `bytes` (a multiple of 16, 16-byte aligned source) from global
+// memory into L2; nothing is written to shared memory and nothing waits.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes, uint64_t policy) {
+  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(src), "r"(bytes),
+               "l"(policy)
+               : "memory");
 }
 
 // 2-D tiled bulk tensor store shared -> global (bulk-group completion).  The

@@ -56,14 +56,14 @@ def test_workspace_sizes(lib):
     # tiny: 2 tiles x 2 k-blocks -> 2 CTAs with one whole tile each
     assert lib.sp24_workspace_size(_lib.OP_GEMM, 16, 256, 256, 0) == 0
     assert lib.sp24_workspace_size(_lib.OP_GEMM, 0, 11008, 4096, 0) == 0
-    # fused quantise (or lift) + GEMM: 256 bytes of counters, then the GEMM's
-    # workspace at K (or K' = 3K/2)
+    # fused quantise (or lift) + GEMM: 8 KB of counters, published copies and
+    # per-CTA slots, then the GEMM's workspace at K (or K' = 3K/2)
     for m in (1, 8, 32, 64, 256):
         assert (lib.sp24_workspace_size(_lib.OP_QUANTIZE_GEMM_PACKED, m, 11008, 4096, 0)
-                == 256 + lib.sp24_workspace_size(_lib.OP_GEMM_PACKED, m, 11008, 4096, 0))
+                == 8192 + lib.sp24_workspace_size(_lib.OP_GEMM_PACKED, m, 11008, 4096, 0))
         assert (lib.sp24_workspace_size(_lib.OP_LIFT_GEMM_PACKED, m, 4096, 4096, 0)
-                == 256 + lib.sp24_workspace_size(_lib.OP_GEMM_PACKED, m, 4096, 6144, 0))
-    assert lib.sp24_workspace_size(_lib.OP_QUANTIZE_GEMM_PACKED, 16, 256, 256, 0) == 256
+                == 8192 + lib.sp24_workspace_size(_lib.OP_GEMM_PACKED, m, 4096, 6144, 0))
+    assert lib.sp24_workspace_size(_lib.OP_QUANTIZE_GEMM_PACKED, 16, 256, 256, 0) == 8192
 
 
 FAKE = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: calls fail validation first

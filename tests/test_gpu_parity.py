@@ -533,7 +533,7 @@ def _fused_weights(w, lift):
     return packed, sw, wv, ref_w["scale"]
 
 
-def _fused_check(x, wts, n, what, lift=False):
+def _fused_check(x, wts, n, what, lift=False, check_y=True):
     """The fused launch against the oracle: codes and scale bit-exact, Y within
     tolerance, and Y identical to the two-launch path on the same codes."""
     packed, sw, wv, ref_sw = wts
@@ -549,14 +549,16 @@ def _fused_check(x, wts, n, what, lift=False):
     assert int(st.item()) == 0, what
     assert host(sx)[0] == ref_s, what
     assert np.array_equal(host(xq), ref_q), what
-    y_ref, b = O.gemm_ref(O.e4m3_decode(ref_q), wv, ref_s, ref_sw)
-    assert_gemm_close(y, y_ref, b, what)
     assert torch.equal(y, y2), what
+    if check_y:
+        y_ref, b = O.gemm_ref(O.e4m3_decode(ref_q), wv, ref_s, ref_sw)
+        assert_gemm_close(y, y_ref, b, what)
 
 
-# M*K/8 at most 1024: every CTA quantises all of X; at most 4096: every CTA
-# takes the whole amax and encodes a slice; above: amax and codes grid-wide
-@pytest.mark.parametrize("m,n,k", [(1, 128, 128), (7, 256, 384), (16, 256, 256), (20, 256, 1024),
+# M*K/8 at most 1024: every CTA quantises all of X (codes staged in shared
+# memory when they fit 8 KB and the tile is 16 tokens); above: amax and
+# codes grid-wide
+@pytest.mark.parametrize("m,n,k", [(1, 128, 128), (2, 256, 4096), (7, 256, 384), (16, 256, 256), (20, 256, 1024),
                                    (33, 384, 1024), (64, 128, 640), (100, 256, 512), (256, 384, 1152)])
 def test_quantize_gemm_packed_small(m, n, k):
     x = WL.random_bits((m, k), 1000 + m)
@@ -586,6 +588,45 @@ def test_lift_gemm_packed_slide68_workload():
     wts = _fused_weights(WL.weight_bits(5), True)
     for m in (1, 64):
         _fused_check(WL.activation_bits(5, m), wts, 4096, f"fused 6:8 M={m}", lift=True)
+
+
+def _every_bf16_up_to(amax_bits):
+    """Every finite bf16 pattern of magnitude <= the bf16 value amax_bits
+    (both signs), amax itself first: every rounding decision of the encoder
+    at the scale amax / 448."""
+    v = O.bf16_to_f32(np.arange(65536, dtype=np.uint16))
+    amax = O.bf16_to_f32(np.array([amax_bits], dtype=np.uint16))[0]
+    ok = np.isfinite(v) & (np.abs(v) <= amax)
+    bits = np.arange(65536, dtype=np.uint16)[ok]
+    return np.concatenate([np.array([amax_bits], dtype=np.uint16), bits])
+
+
+@pytest.mark.parametrize("amax_bits", [0x43E0, 0x3FC0, 0x3D18, 0x447A, 0x2180, 0x0080])
+def test_quantize_gemm_packed_every_bf16_value(amax_bits):
+    """The fused kernel's division-free encoder, grid-wide form (every
+    eligible bf16 value, at M > 1024 / (K / 8) rows) and the local form
+    with codes staged in shared memory (M = 1, a strided subset), against the
+    oracle's correctly rounded division, bit for bit.  amax = 2^-126 makes
+    the scale an fp32 subnormal whose reciprocal overflows, so every code
+    takes the exact division; its outputs are bf16 subnormals, coarser than
+    the GEMM tolerance, so only codes, scale and the two-launch identity
+    are checked there."""
+    check_y = amax_bits != 0x0080
+    bits = _every_bf16_up_to(amax_bits)
+    k = 1024
+    m = -(-len(bits) // k)
+    x = np.zeros(m * k, dtype=np.uint16)
+    x[:len(bits)] = bits
+    wts = _fused_weights(WL.random_bits((128, k), 1700, scale=0.02), False)
+    _fused_check(x.reshape(m, k), wts, 128, f"fused every bf16 <= {amax_bits:#x}, {m} rows", check_y=check_y)
+    k1 = 4096
+    sub = bits[np.linspace(0, len(bits) - 1, k1).astype(np.int64)]
+    sub[0] = amax_bits
+    wts1 = _fused_weights(WL.random_bits((128, k1), 1701, scale=0.02), False)
+    _fused_check(sub.reshape(1, k1), wts1, 128, f"fused staged, bf16 <= {amax_bits:#x}", check_y=check_y)
+    wts2 = _fused_weights(WL.random_bits((128, k1), 1702, scale=0.02), True)
+    _fused_check(sub.reshape(1, k1), wts2, 128, f"fused staged lift, bf16 <= {amax_bits:#x}", lift=True,
+                 check_y=check_y)
 
 
 def test_quantize_gemm_packed_zero_and_nonfinite_inputs():
@@ -619,9 +660,29 @@ def test_quantize_gemm_packed_reuses_its_workspace():
             y2 = sp().sp24_gemm_packed(xq, sx, packed, sw, 384, workspace=ws)
             outs.append((host(y), host(y2)))
     torch.cuda.synchronize()
-    assert (ws.buf[:256] == 0).all()
+    assert (ws.buf[:8192] == 0).all()        # the fused counters and per-CTA slots
     for (a, b), (c, d) in zip(outs[:3], outs[3:]):
         assert np.array_equal(a, b) and np.array_equal(a, c) and np.array_equal(c, d)
+
+
+def test_quantize_gemm_packed_back_to_back_grid_calls():
+    """Grid-wide fused calls queued back to back on one workspace, each X with
+    its own scale: a counter or flag left set by one call would let the next
+    read its codes before they are written (Y would then differ from the
+    two-launch GEMM on the same codes)."""
+    ws = sp().Workspace(DEV)
+    w = WL.random_bits((384, 1024), 1800, scale=0.02)
+    packed, sw = sp().sp24_prune_compress_packed(dev_bf16(w))
+    xs = [dev_bf16(WL.random_bits((40 + 24 * (i % 2), 1024), 1900 + i, scale=0.5 + i)) for i in range(24)]
+    outs = [sp().sp24_quantize_gemm_packed(x, packed, sw, 384, workspace=ws) for x in xs]
+    refs = [sp().sp24_gemm_packed(xq, sx, packed, sw, 384, workspace=ws) for (_, xq, sx) in outs]
+    torch.cuda.synchronize()
+    assert (ws.buf[:8192] == 0).all()
+    for i, ((y, xq, sx), y2) in enumerate(zip(outs, refs)):
+        assert torch.equal(y, y2), f"call {i}"
+    for i in (0, 23):
+        ref_q, ref_s = O.quantize_pertensor(host(xs[i]))
+        assert host(outs[i][2])[0] == ref_s and np.array_equal(host(outs[i][1]), ref_q), f"call {i}"
 
 
 # ------------------------------------------------------------ per-token / per-channel scales

@@ -849,6 +849,100 @@ def prefill_headline(device, peaks, reps=20):
                       f"({len(pd)} dense), inputs larger than L2"}
 
 
+# ---------------------------------------------------------------- single-kernel cases
+# `bench.py --kernel-case NAME` runs one library call on a fixed workload
+# shape, twice as warm-up and then three times, and exits: the command the
+# per-kernel ncu summaries under profiles/ are captured from (one kernel per
+# case; inputs larger than L2 where the workload is).
+
+def kernel_case(name, device):
+    import torch
+
+    import structured_sparse_fp8_b200 as sp
+    from structured_sparse_fp8_b200 import workloads as WL
+
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+    ws = sp.Workspace(device)
+    ws.get(256 << 20)
+    w2 = None
+
+    def w_decode():
+        return bf(WL.weight_bits(2))
+
+    if name == "quantize":                       # X[4096, 4096] per-tensor E4M3
+        x = bf(WL.activation_bits(3, 4096))
+        call = lambda: sp.fp8_quantize_pertensor(x, workspace=ws)
+    elif name == "lift":                         # X[2048, 4096] 6:8 lift + quantise
+        x = bf(WL.activation_bits(5, 2048))
+        call = lambda: sp.slide68_lift(x, workspace=ws)
+    elif name == "prune_packed":                 # W[11008, 4096] 2:4 prune + compress, packed
+        w = w_decode()
+        call = lambda: sp.sp24_prune_compress_packed(w, workspace=ws)
+    elif name == "slide68_packed":               # W[4096, 4096] 6:8 decompose, packed
+        w = bf(WL.weight_bits(5))
+        call = lambda: sp.slide68_decompose_packed(w, workspace=ws)
+    elif name in ("gemm_packed_decode", "gemm_dense_decode", "gemm_int8_decode", "fused_decode"):
+        m = 64
+        w = w_decode()
+        x = bf(WL.activation_bits(2, m))
+        if name == "gemm_dense_decode":
+            wq, swd = sp.fp8_quantize_pertensor(w, workspace=ws)
+            xq, sx = sp.fp8_quantize_pertensor(x, workspace=ws)
+            call = lambda: sp.fp8_gemm_dense(xq, sx, wq, swd, workspace=ws)
+        elif name == "gemm_int8_decode":
+            c = sp.sp24_prune_compress_int8(w, workspace=ws)
+            packed = sp.sp24_pack_weights(c["values"].view(torch.uint8), c["meta"])
+            xq, sx = sp.int8_quantize_pertensor(x, workspace=ws)
+            call = lambda: sp.sp24_gemm_int8_packed(xq, sx, packed, c["scale"], w.shape[0], workspace=ws)
+        else:
+            packed, sw = sp.sp24_prune_compress_packed(w, workspace=ws)
+            xq, sx = sp.fp8_quantize_pertensor(x, workspace=ws)
+            if name == "fused_decode":
+                call = lambda: sp.sp24_quantize_gemm_packed(x, packed, sw, w.shape[0], workspace=ws)
+            else:
+                call = lambda: sp.sp24_gemm_packed(xq, sx, packed, sw, w.shape[0], workspace=ws)
+    elif name == "gemm_bf16_downproj":           # M256 N4096 K14336, bf16 operands
+        w = bf(WL.weight_bits(4))
+        x = bf(WL.activation_bits(4, 256))
+        c = sp.sp24_prune_compress(w, "bf16", workspace=ws)
+        call = lambda: sp.sp24_gemm(x, None, c["values"], c["meta"], None, dtype="bf16", workspace=ws)
+    elif name == "gemm_scaled_prefill":          # M4096 N12288 K4096, per-token x per-channel scales
+        w = bf(WL.weight_bits(3))
+        x = bf(WL.activation_bits(3, 4096))
+        c = sp.sp24_prune_compress_perchannel(w)
+        packed = sp.sp24_pack_weights(c["values"], c["meta"])
+        xq, sx = sp.fp8_quantize_pertoken(x)
+        call = lambda: sp.sp24_gemm_packed_scaled(xq, sx, packed, c["scales"], w.shape[0], workspace=ws)
+    elif name == "pertoken":                     # X[4096, 4096] per-token E4M3
+        x = bf(WL.activation_bits(3, 4096))
+        call = lambda: sp.fp8_quantize_pertoken(x)
+    elif name == "perchannel":                   # W[11008, 4096] per-channel 2:4 prune
+        w = w_decode()
+        call = lambda: sp.sp24_prune_compress_perchannel(w)
+    elif name == "int8_quantize":                # X[4096, 4096] per-tensor INT8
+        x = bf(WL.activation_bits(3, 4096))
+        call = lambda: sp.int8_quantize_pertensor(x, workspace=ws)
+    elif name == "int8_prune":                   # W[11008, 4096] INT8 2:4 weight path
+        w = w_decode()
+        call = lambda: sp.sp24_prune_compress_int8(w, workspace=ws)
+    elif name in ("slide46_decompose", "slide46_lift"):   # 4:6 at K = 4608 (K' = 6144)
+        if name == "slide46_decompose":
+            w = bf(WL.random_bits((4096, 4608), 2301, scale=0.02))
+            call = lambda: sp.slide_decompose(w, 3, workspace=ws)
+        else:
+            x = bf(WL.random_bits((2048, 4608), 2302))
+            call = lambda: sp.slide_lift(x, 3, workspace=ws)
+    else:
+        raise SystemExit(f"unknown kernel case {name}")
+    for _ in range(5):
+        call()
+    torch.cuda.synchronize()
+    del w2
+    print(json.dumps({"kernel_case": name, "ok": True}))
+
+
 # ---------------------------------------------------------------- CPU oracle
 
 def oracle_sample_step(wl, rows, rng_seed, m_cap=64):
@@ -947,12 +1041,21 @@ def main():
     ap.add_argument("--unfused", action="store_true",
                     help="quantise activations in their own launch at every M (no fused quantise + GEMM)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-case", default=None,
+                    help="run one library call on a fixed shape five times and exit (for per-kernel ncu captures)")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the prefill-shaped (tensor-bound) GEMM timed next to the decode headline")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = WORKLOADS[args.workload]
+    if args.kernel_case:
+        import torch
+
+        import __graft_entry__
+        __graft_entry__.build()
+        kernel_case(args.kernel_case, torch.device("cuda", 0))
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

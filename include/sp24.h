@@ -19,8 +19,8 @@
  * 2:4 over a lifted K' = 1.5 K, and the activation lift is fused into the
  * FP8 quantisation pass.  Beyond that path: the fused quantise + GEMM forms
  * for decode, per-token and per-channel scales, the general (2N-2):2N
- * decomposition for N = 3 and 5, and INT8 W8A8 (quantisers and the sparse
- * GEMM; each declared with its own citation below).
+ * decomposition for N = 3 and 5, INT8 W8A8 and FP4 (quantisers and the
+ * sparse GEMMs; each declared with its own citation below).
  *
  * Conventions for every entry point
  * ---------------------------------
@@ -99,6 +99,7 @@ typedef struct CUstream_st *sp24_stream_t; /* identical to cudaStream_t */
 #define SP24_OP_GEMM_PACKED 6
 #define SP24_OP_QUANTIZE_GEMM_PACKED 7 /* K = the columns of X */
 #define SP24_OP_LIFT_GEMM_PACKED 8     /* K = the columns of X (the GEMM runs over 3K/2) */
+#define SP24_OP_GEMM_FP4 9
 
 /*
  * Weight path, 2:4.  W: bf16 [N, K].  For every row and every group of 4
@@ -299,6 +300,44 @@ int sp24_prune_compress_int8(const void *W, int N, int K, int8_t *values, uint8_
 int sp24_gemm_int8_packed(const int8_t *Xq, const float *x_scale, const void *packed, const float *w_scale,
                           void *Y, int M, int N, int K, void *workspace, size_t ws_bytes, int32_t *status,
                           sp24_stream_t stream);
+
+/*
+ * FP4 (OCP E2M1) with 2:4 weights (SlideSparse, §3 "Contribuciones Clave":
+ * FP4 among the supported precisions).  The pages give no format; the rule
+ * is the per-tensor E4M3 one on the E2M1 grid (magnitudes 0, 0.5, 1, 1.5,
+ * 2, 3, 4, 6): s = amax / 6 (1.0 for an all-zero tensor), code =
+ * E2M1(RN_fp32(x / s)) to the nearest grid value, ties to the even code,
+ * saturating at 6, the sign kept on a value that rounds to zero (code 8);
+ * no block scales.  Codes are 4 bits (bit 3 the sign), packed two per byte,
+ * element 2i in the low nibble of byte i.
+ * fp4_quantize_pertensor: X bf16 [rows, cols] (cols % 32 == 0) -> q u8
+ *   [rows, cols / 2], *scale <- s.
+ * sp24_prune_compress_fp4: W bf16 [N, K] (K % 64 == 0) -> the 2:4 selection
+ *   of sp24_prune_compress in the canonical layout with FP4 codes: values
+ *   [N, K/2] codes = u8 [N, K/4], meta [N, K/8], *w_scale <- s.
+ * Pointers are device pointers, 16-byte aligned (scale: 4-byte).  Workspace:
+ * sp24_workspace_size(SP24_OP_QUANTIZE or SP24_OP_PRUNE_COMPRESS, ...)
+ * (256 bytes of counters, zero before and after the call).  Errors as for
+ * the E4M3 calls; SP24_STATUS_NONFINITE when the input holds Inf or NaN.
+ */
+int fp4_quantize_pertensor(const void *X, int64_t rows, int64_t cols, uint8_t *q, float *scale, void *workspace,
+                           size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+int sp24_prune_compress_fp4(const void *W, int N, int K, uint8_t *values, uint8_t *meta, float *w_scale,
+                            void *workspace, size_t ws_bytes, int32_t *status, sp24_stream_t stream);
+/*
+ * The FP4 sparse GEMM: Y[M, N] = x_scale * w_scale * (Xq . W^T) on the
+ * tensor cores (tcgen05.mma.sp kind::f8f6f4 with E2M1 operands, fp32
+ * accumulation), bf16 out.  Xq: u8 [M, K / 2] from fp4_quantize_pertensor;
+ * values u8 [N, K / 4] and meta [N, K / 8] from sp24_prune_compress_fp4;
+ * scales: one device float each.  Shape rules: M >= 1, N % 128 == 0,
+ * K % 256 == 0.  Xq and values must be 32-byte aligned (the 4-bit tensor
+ * maps), meta and Y 16-byte aligned.  Workspace:
+ * sp24_workspace_size(SP24_OP_GEMM_FP4, M, N, K, 0) (zero-filled before the
+ * first use, its counters zero again after every call, as for sp24_gemm).
+ */
+int sp24_gemm_fp4(const uint8_t *Xq, const float *x_scale, const uint8_t *w_values, const uint8_t *w_meta,
+                  const float *w_scale, void *Y, int M, int N, int K, void *workspace, size_t ws_bytes,
+                  int32_t *status, sp24_stream_t stream);
 
 /*
  * The general (2N-2):2N case through 2:4 windows (SlideSparse, §2

@@ -354,6 +354,70 @@ def sp24_gemm_int8_packed(xq: torch.Tensor, x_scale, packed: torch.Tensor, w_sca
     return y
 
 
+def fp4_quantize_pertensor(X: torch.Tensor, status: torch.Tensor | None = None,
+                           out: torch.Tensor | None = None, scale: torch.Tensor | None = None,
+                           workspace: Workspace | None = None):
+    """Per-tensor FP4 (E2M1) quantisation of X bf16 [rows, cols] -> (codes u8
+    [rows, cols / 2], two per byte, element 2i in the low nibble; scale f32[1])."""
+    lib = _lib.load()
+    _require_cuda(X, status, out, scale)
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise Sp24Error("X must be a 2-D bf16 tensor")
+    rows, cols = X.shape
+    q = out if out is not None else torch.empty((rows, cols // 2), dtype=torch.uint8, device=X.device)
+    s = scale if scale is not None else torch.empty((1,), dtype=torch.float32, device=X.device)
+    ws, wsn = _ws(X.device, _lib.OP_QUANTIZE, rows, 0, cols, DTYPE_E4M3, workspace)
+    rc = lib.fp4_quantize_pertensor(_ptr(X), rows, cols, _ptr(q), _ptr(s), _ptr(ws), wsn,
+                                    _ptr(status), _stream(X.device))
+    _lib.check(rc, "fp4_quantize_pertensor")
+    return q, s
+
+
+def sp24_prune_compress_fp4(W: torch.Tensor, status: torch.Tensor | None = None,
+                            workspace: Workspace | None = None, out: dict | None = None):
+    """2:4 magnitude prune + per-tensor FP4 (E2M1) quantise + compress of W bf16
+    [N, K]: returns dict(values u8 [N, K/4] (K/2 codes, two per byte), meta u8
+    [N, K/8], scale); ``out`` may supply any of these preallocated."""
+    lib = _lib.load()
+    out = out or {}
+    _require_cuda(W, status, *out.values())
+    if W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise Sp24Error("W must be a 2-D bf16 tensor")
+    N, K = W.shape
+    values = out.get("values")
+    values = values if values is not None else torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    meta = out.get("meta")
+    meta = meta if meta is not None else torch.empty((N, K // 8), dtype=torch.uint8, device=W.device)
+    scale = out.get("scale")
+    scale = scale if scale is not None else torch.empty((1,), dtype=torch.float32, device=W.device)
+    ws, wsn = _ws(W.device, _lib.OP_PRUNE_COMPRESS, 0, N, K, DTYPE_E4M3, workspace)
+    rc = lib.sp24_prune_compress_fp4(_ptr(W), N, K, _ptr(values), _ptr(meta), _ptr(scale), _ptr(ws), wsn,
+                                     _ptr(status), _stream(W.device))
+    _lib.check(rc, "sp24_prune_compress_fp4")
+    return dict(values=values, meta=meta, scale=scale)
+
+
+def sp24_gemm_fp4(xq: torch.Tensor, x_scale, values: torch.Tensor, meta: torch.Tensor, w_scale,
+                  out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                  workspace: Workspace | None = None):
+    """FP4 sparse GEMM: xq u8 [M, K/2] (fp4_quantize_pertensor), values u8 [N, K/4]
+    and meta u8 [N, K/8] (sp24_prune_compress_fp4) -> Y bf16 [M, N]."""
+    lib = _lib.load()
+    _require_cuda(xq, x_scale, values, meta, w_scale, out, status)
+    if xq.dtype != torch.uint8 or xq.dim() != 2 or values.dim() != 2:
+        raise Sp24Error("xq and values must be 2-D uint8 tensors of packed FP4 codes")
+    M, K = xq.shape[0], xq.shape[1] * 2
+    N = values.shape[0]
+    if values.shape[1] * 4 != K or meta.shape != (N, K // 8):
+        raise Sp24Error("values / meta do not match N x K")
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    ws, wsn = _ws(xq.device, _lib.OP_GEMM_FP4, M, N, K, DTYPE_E4M3, workspace)
+    rc = lib.sp24_gemm_fp4(_ptr(xq), _ptr(x_scale), _ptr(values), _ptr(meta), _ptr(w_scale), _ptr(y), M, N, K,
+                           _ptr(ws), wsn, _ptr(status), _stream(xq.device))
+    _lib.check(rc, "sp24_gemm_fp4")
+    return y
+
+
 def _quant_gemm(name, op, klift, X, packed, w_scale, n, out, xq_out, x_scale_out, status, workspace):
     lib = _lib.load()
     _require_cuda(X, packed, w_scale, out, xq_out, x_scale_out, status)

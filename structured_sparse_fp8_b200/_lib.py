@@ -25,7 +25,7 @@ SP24_STATUS_TIMEOUT = 2
 DTYPE_E4M3 = 0
 DTYPE_BF16 = 1
 (OP_QUANTIZE, OP_PRUNE_COMPRESS, OP_SLIDE68_DECOMPOSE, OP_SLIDE68_LIFT, OP_GEMM, OP_GEMM_DENSE,
- OP_GEMM_PACKED, OP_QUANTIZE_GEMM_PACKED, OP_LIFT_GEMM_PACKED) = range(9)
+ OP_GEMM_PACKED, OP_QUANTIZE_GEMM_PACKED, OP_LIFT_GEMM_PACKED, OP_GEMM_FP4) = range(10)
 
 _p = ctypes.c_void_p
 _i = ctypes.c_int
@@ -51,6 +51,9 @@ SIGNATURES = {
     "int8_quantize_pertensor": (_i, [_p, _i64, _i64, _p, _p, _p, _sz, _p, _p]),
     "sp24_prune_compress_int8": (_i, [_p, _i, _i, _p, _p, _p, _p, _sz, _p, _p]),
     "sp24_gemm_int8_packed": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _sz, _p, _p]),
+    "fp4_quantize_pertensor": (_i, [_p, _i64, _i64, _p, _p, _p, _sz, _p, _p]),
+    "sp24_prune_compress_fp4": (_i, [_p, _i, _i, _p, _p, _p, _p, _sz, _p, _p]),
+    "sp24_gemm_fp4": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _p, _sz, _p, _p]),
     "slide_lift": (_i, [_p, _i, _i, _i, _p, _p, _p, _sz, _p, _p]),
     "sp24_prune_compress_perchannel": (_i, [_p, _i, _i, _p, _p, _p, _p, _p]),
     "sp24_gemm_packed_scaled": (_i, [_p, _p, _i, _p, _p, _i, _p, _i, _i, _i, _p, _sz, _p, _p]),

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "fp4_kernels.h"
 #include "int8_kernels.h"
 #include "kernels.h"
 #include "sp24.h"
@@ -87,6 +88,13 @@ size_t sp24_workspace_size(int op, int64_t M, int64_t N, int64_t K, int dtype) {
              sp24::plan_gemm(sp24::kSparseE4M3Packed, static_cast<int>(M), static_cast<int>(N),
                              static_cast<int>(Kg), sms)
                  .workspace_bytes();
+    }
+    case SP24_OP_GEMM_FP4: {
+      if (M < 1 || N < 128 || K < 256 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return 0;
+      int sms = device_sm_count();
+      if (sms <= 0) sms = 148;
+      return sp24::plan_gemm(sp24::kSparseFP4, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sms)
+          .workspace_bytes();
     }
     case SP24_OP_GEMM:
     case SP24_OP_GEMM_PACKED:
@@ -289,6 +297,53 @@ int sp24_gemm_packed(const void *Xq, const float *x_scale, const void *packed, c
                      sp24_stream_t stream) {
   return gemm_common(sp24::kSparseE4M3Packed, Xq, x_scale, packed, nullptr, w_scale, Y, M, N, K,
                      workspace, ws_bytes, status, stream);
+}
+
+int fp4_quantize_pertensor(const void *X, int64_t rows, int64_t cols, uint8_t *q, float *scale, void *workspace,
+                           size_t ws_bytes, int32_t *status, sp24_stream_t stream) {
+  if (!X || !q || !scale) return SP24_ERR_NULL;
+  if (rows < 1 || cols < 1 || cols % 32 != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(q)) return SP24_ERR_ALIGN;
+  const int rc = check_workspace(workspace, ws_bytes);
+  if (rc != SP24_OK) return rc;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  return cuda_status(sp24::launch_fp4_quantize(X, rows * cols, static_cast<uint32_t *>(workspace), scale, q,
+                                               status, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sp24_prune_compress_fp4(const void *W, int N, int K, uint8_t *values, uint8_t *meta, float *w_scale,
+                            void *workspace, size_t ws_bytes, int32_t *status, sp24_stream_t stream) {
+  if (!W || !values || !meta || !w_scale) return SP24_ERR_NULL;
+  if (N < 1 || K < 64 || K % 64 != 0) return SP24_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(values) || !aligned16(meta)) return SP24_ERR_ALIGN;
+  const int rc = check_workspace(workspace, ws_bytes);
+  if (rc != SP24_OK) return rc;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  return cuda_status(sp24::launch_fp4_prune24(W, static_cast<int64_t>(N) * K, static_cast<uint32_t *>(workspace),
+                                              w_scale, values, meta, status, sms,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sp24_gemm_fp4(const uint8_t *Xq, const float *x_scale, const uint8_t *w_values, const uint8_t *w_meta,
+                  const float *w_scale, void *Y, int M, int N, int K, void *workspace, size_t ws_bytes,
+                  int32_t *status, sp24_stream_t stream) {
+  if (!Xq || !w_values || !w_meta || !Y) return SP24_ERR_NULL;
+  if (M < 1 || N < 128 || N % 128 != 0 || K < 256 || K % 256 != 0) return SP24_ERR_SHAPE;
+  // the 4-bit tensor maps want 32-byte aligned bases
+  if ((reinterpret_cast<uintptr_t>(Xq) & 31u) || (reinterpret_cast<uintptr_t>(w_values) & 31u) ||
+      !aligned16(w_meta) || !aligned16(Y))
+    return SP24_ERR_ALIGN;
+  const int sms = device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
+  const sp24::GemmPlan pl = sp24::plan_gemm(sp24::kSparseFP4, M, N, K, sms);
+  if (pl.workspace_bytes() > 0) {
+    if (!workspace || ws_bytes < pl.workspace_bytes()) return SP24_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SP24_ERR_ALIGN;
+  }
+  return cuda_status(sp24::launch_gemm(sp24::kSparseFP4, pl, Xq, x_scale, w_values, w_meta, w_scale, Y, M, N, K,
+                                       workspace, status, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int sp24_gemm_int8_packed(const int8_t *Xq, const float *x_scale, const void *packed, const float *w_scale,

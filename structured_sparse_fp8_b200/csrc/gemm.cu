@@ -61,6 +61,7 @@ struct KindTraits<kSparseE4M3> {
   static constexpr bool kMetaTransform = false;
   static constexpr int kMetaColsPerMma = 2;  // 64 metadata bits per row per MMA
   static constexpr bool kPacked = false;
+  static constexpr bool kFp4 = false;
 };
 
 // The same MMA with the weights in the tile-packed layout: each stage's
@@ -78,6 +79,22 @@ template <>
 struct KindTraits<kSparseI8Packed> : KindTraits<kSparseE4M3Packed> {
   static constexpr uint32_t kFmt = 1;   // signed 8-bit
   static constexpr uint32_t kDFmt = 2;  // s32 accumulator
+};
+
+// 2:4 sparse FP4 (E2M1 A and B, kind::f8f6f4): the codes are packed two per
+// byte in global memory and loaded with 4-bit tensor maps
+// (CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B), which lay every 16 codes out in 16
+// bytes of shared memory (8 bytes of codes, 8 of padding): the byte geometry
+// of the E4M3 tiles, one byte per element.  Such a box is 128 elements wide,
+// so a stage covers two 128-K blocks (KB = 2): 128 stored values = 128
+// bytes per W row (128-byte swizzle), 2 x 128 bytes per token, and the two
+// blocks' metadata (16 bytes per row each, two 2 KB boxes).
+template <>
+struct KindTraits<kSparseFP4> : KindTraits<kSparseE4M3> {
+  static constexpr uint32_t kASwizzle = kSwizzle128B;
+  static constexpr int kASbo = 8 * 128;  // 8 rows of one stage's 128 bytes
+  static constexpr uint32_t kFmt = 5;     // E2M1
+  static constexpr bool kFp4 = true;
 };
 
 // Dense E4M3 (comparison kernel): 128 logical K per stage, 4 MMAs of K = 32.
@@ -101,6 +118,7 @@ struct KindTraits<kDenseE4M3> {
   static constexpr bool kMetaTransform = false;
   static constexpr int kMetaColsPerMma = 0;
   static constexpr bool kPacked = false;
+  static constexpr bool kFp4 = false;
 };
 
 // 2:4 sparse BF16 (kind::f16): per stage 128 logical K = 64 bf16 values (128 B)
@@ -128,6 +146,7 @@ struct KindTraits<kSparseBF16> {
   static constexpr bool kMetaTransform = true;
   static constexpr int kMetaColsPerMma = 1;
   static constexpr bool kPacked = false;
+  static constexpr bool kFp4 = false;
 };
 
 // MT = 128-row W tiles per CTA tile (1 or 2).  With MT = 2 each stage
@@ -149,15 +168,21 @@ constexpr uint32_t kXStageBytes = 8192;
 template <int KIND, int BN, int MT = 1, int KB = 1, int XQ = 0>
 struct Config {
   using T = KindTraits<KIND>;
-  static_assert(KB == 1 || (KB == 2 && T::kPacked && MT == 1), "two-block stages are for packed, one-row-tile tiles");
+  static_assert(KB == 1 || (KB == 2 && (T::kPacked || T::kFp4) && MT == 1),
+                "two-block stages are for packed or FP4, one-row-tile tiles");
+  static_assert(!T::kFp4 || (KB == 2 && MT == 1), "FP4 stages are two 128-K blocks of one row tile");
   static constexpr int kRows = 128 * MT;
   static constexpr uint32_t kABytes = kRows * T::kARowBytes * KB;
   static constexpr uint32_t kBBytes = BN * T::kBRowBytes * KB;
   static constexpr uint32_t kEBytes = kRows * T::kERowBytes * KB;
   static constexpr uint32_t kTBytes = T::kMetaTransform ? 128 * 16 : 0;  // TMEM-ready metadata
-  static constexpr uint32_t kTmaBytes = kABytes + kBBytes + kEBytes;
+  // Transaction bytes of a stage's copies: a 4-bit box moves its packed
+  // bytes (half its shared-memory footprint, which pads every 8 bytes of
+  // codes to 16).
+  static constexpr uint32_t kTmaBytes = (T::kFp4 ? (kABytes + kBBytes) / 2 : kABytes + kBBytes) + kEBytes;
   static constexpr uint32_t kWBytes = kABytes + kEBytes;  // the weight half of a stage
-  static constexpr uint32_t kStageBytes = kTmaBytes + kTBytes;
+  // shared-memory footprint of a stage (the padded size for 4-bit boxes)
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes + kEBytes + kTBytes;
   static constexpr int kBSub = T::kBRowBytes * KB / 128;  // 128-byte X boxes per stage
   static constexpr int kMmas = T::kMmas * KB;             // MMAs per row tile per stage
   // Stage layout: [A][B][E][T] (tensor-mapped weights; A and E hold all kRows
@@ -660,6 +685,14 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
                                  ((static_cast<int64_t>(n0 / 128 + i) * p.num_kb + kb) * KB) * kPackedBlockBytes;
             bulk_load_g2s(st + C::a_off(i), blk, KB * kPackedBlockBytes, bar, stream_w);
           }
+        } else if constexpr (T::kFp4) {
+          // stage kb = stored codes 128 kb .. 128 kb + 127 of each row (one
+          // 4-bit box), and the metadata of 128-K blocks 2 kb, 2 kb + 1
+          tma_load_2d(st, &tmA, bar, kb * 128, n0, stream_w);
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            tma_load_2d(st + C::kEOff + j * 128 * T::kERowBytes, &tmE, bar, (2 * kb + j) * T::kERowBytes, n0,
+                        stream_w);
         } else {
           tma_load_2d(st, &tmA, bar, kb * (T::kARowBytes / T::kAElemBytes), n0, stream_w);
           if (T::kSparse) tma_load_2d(st + C::kEOff, &tmE, bar, kb * T::kERowBytes, n0, stream_w);
@@ -844,7 +877,10 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
           if (leader) {
             if (T::kSparse) {
               // 128 rows x 16 B, rows contiguous: core matrices of 8 rows are 128 B apart.
-              if constexpr (T::kPacked && MT * KB == 2) {
+              if constexpr (T::kFp4) {
+                // the two blocks' metadata boxes, 2048 bytes apart
+                tmem_copy_128x256b(e_tmem, smem_desc(st_addr + C::kEOff, 128 * T::kERowBytes, 128, kSwizzleNone));
+              } else if constexpr (T::kPacked && MT * KB == 2) {
                 // two packed blocks' metadata in one copy (both row tiles, or
                 // both k-blocks of one row tile): the second 16-byte column is
                 // the next block's metadata, 10240 bytes on
@@ -864,14 +900,14 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
               for (int kk = 0; kk < C::kMmas; ++kk) {
                 // MMA kk reads block kk / kMmas of the stage (packed blocks are
                 // 10240 bytes apart), step kk % kMmas within it
-                const uint32_t a_k = KB == 1 ? kk * T::kAStep
-                                             : (kk / T::kMmas) * kPackedBlockBytes + (kk % T::kMmas) * T::kAStep;
+                const uint32_t a_k = (KB == 1 || T::kFp4) ? kk * T::kAStep
+                                                          : (kk / T::kMmas) * kPackedBlockBytes + (kk % T::kMmas) * T::kAStep;
                 const uint64_t ad = smem_desc(a_addr + a_k, 16, T::kASbo, T::kASwizzle);
                 const uint32_t boff = (kk * T::kBStep / 128) * (BN * 128) + (kk * T::kBStep) % 128;
                 const uint64_t bd = smem_desc(b_addr + boff, 16, 8 * 128, kSwizzle128B);
                 const uint32_t acc = (kb > sg.kb0 || kk > 0) ? 1u : 0u;
                 const uint32_t d = d_tmem + rt * BN;
-                if constexpr (KIND == kSparseE4M3 || KIND == kSparseE4M3Packed) {
+                if constexpr (KIND == kSparseE4M3 || KIND == kSparseE4M3Packed || KIND == kSparseFP4) {
                   mma_f8_sparse(d, ad, bd, idesc, e_tmem + 4 * rt + 2 * kk, acc);
                 } else if constexpr (KIND == kSparseI8Packed) {
                   mma_i8_sparse(d, ad, bd, idesc, e_tmem + 4 * rt + 2 * kk, acc);
@@ -1183,14 +1219,15 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major 2-D map: `inner` elements per row (contiguous), `outer` rows.
+// Row-major 2-D map: `inner` elements per row (contiguous), `outer` rows;
+// elem_bytes = 0 marks 4-bit elements (two per byte).
 bool make_tensor_map_2d(CUtensorMap *map, const void *ptr, CUtensorMapDataType dt, int elem_bytes,
                         uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
                         CUtensorMapSwizzle sw) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elem_bytes)};
+  cuuint64_t strides[1] = {elem_bytes == 0 ? inner / 2 : inner * static_cast<uint64_t>(elem_bytes)};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
@@ -1217,8 +1254,11 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   // Large token tiles (224 tokens: many tiles, bound by operand ingest) pair
   // two 128-row W tiles on one activation tile when N allows it.
   pl.mt = (pl.bn == 224 && kind != kSparseBF16 && N % 256 == 0) ? 2 : 1;
-  // Decode-sized tiles over packed weights take two 128-K blocks per stage.
-  pl.kb = ((kind == kSparseE4M3Packed || kind == kSparseI8Packed) && pl.bn <= 64 && pl.mt == 1 && K % 256 == 0)
+  // Decode-sized tiles over packed weights take two 128-K blocks per stage;
+  // FP4 always does (one 4-bit box spans two blocks) and uses one row tile.
+  if (kind == kSparseFP4) pl.mt = 1;
+  pl.kb = (kind == kSparseFP4 ||
+           ((kind == kSparseE4M3Packed || kind == kSparseI8Packed) && pl.bn <= 64 && pl.mt == 1 && K % 256 == 0))
               ? 2
               : 1;
   pl.bk = 128 * pl.kb;
@@ -1279,20 +1319,27 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   if (attr_err != cudaSuccess) return attr_err;
 
   CUtensorMap tmA, tmB, tmE;
-  const CUtensorMapDataType dtA =
-      T::kAElemBytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  const CUtensorMapDataType dtB =
-      T::kBElemBytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const CUtensorMapDataType dtA = T::kFp4                 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B
+                                  : T::kAElemBytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16
+                                                        : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const CUtensorMapDataType dtB = T::kFp4                 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B
+                                  : T::kBElemBytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16
+                                                        : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const uint64_t a_row = T::kSparse ? static_cast<uint64_t>(K) / 2 : static_cast<uint64_t>(K);
   const CUtensorMapSwizzle a_sw =
       T::kASwizzle == kSwizzle64B ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   if (T::kPacked) {
     tmA = {};
+  } else if (T::kFp4) {
+    // the stored codes of 128 rows x 256 K: one 128-element 4-bit box
+    if (!make_tensor_map_2d(&tmA, w_values, dtA, 0, a_row, N, 128, C::kRows, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
   } else if (!make_tensor_map_2d(&tmA, w_values, dtA, T::kAElemBytes, a_row, N,
                                  T::kARowBytes / T::kAElemBytes, C::kRows, a_sw)) {
     return cudaErrorInvalidValue;
   }
-  if (!make_tensor_map_2d(&tmB, xq, dtB, T::kBElemBytes, K, M, T::kBBoxElems, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_tensor_map_2d(&tmB, xq, dtB, T::kFp4 ? 0 : T::kBElemBytes, K, M, T::kBBoxElems, BN,
+                          CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (T::kSparse && !T::kPacked) {
     if (!make_tensor_map_2d(&tmE, w_meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(K) / 8, N,
@@ -1370,29 +1417,41 @@ static cudaError_t launch_kind(const GemmPlan &pl, const void *xq, const float *
                                const void *w_values, const uint8_t *w_meta, const float *w_scale,
                                void *y, int M, int N, int K, void *ws, int32_t *status,
                                cudaStream_t st) {
-  if constexpr (KIND == kSparseE4M3Packed || KIND == kSparseI8Packed) {
-    if (pl.kb == 2) {
-      switch (pl.bn) {
-        case 16: return launch_typed<KIND, 16, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-        case 32: return launch_typed<KIND, 32, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-        case 64: return launch_typed<KIND, 64, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-        default: return cudaErrorInvalidValue;
+  if constexpr (KIND == kSparseFP4) {
+    switch (pl.bn) {
+      case 16: return launch_typed<KIND, 16, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+      case 32: return launch_typed<KIND, 32, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+      case 64: return launch_typed<KIND, 64, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+      case 128: return launch_typed<KIND, 128, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+      case 224: return launch_typed<KIND, 224, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+      case 256: return launch_typed<KIND, 256, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+      default: return cudaErrorInvalidValue;
+    }
+  } else {
+    if constexpr (KIND == kSparseE4M3Packed || KIND == kSparseI8Packed) {
+      if (pl.kb == 2) {
+        switch (pl.bn) {
+          case 16: return launch_typed<KIND, 16, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+          case 32: return launch_typed<KIND, 32, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+          case 64: return launch_typed<KIND, 64, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+          default: return cudaErrorInvalidValue;
+        }
       }
     }
-  }
-  switch (pl.bn) {
-    case 16: return launch_typed<KIND, 16, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-    case 32: return launch_typed<KIND, 32, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-    case 64: return launch_typed<KIND, 64, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-    case 128: return launch_typed<KIND, 128, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-    case 224:
-      if constexpr (KIND != kSparseBF16) {
-        if (pl.mt == 2)
-          return launch_typed<KIND, 224, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-      }
-      return launch_typed<KIND, 224, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-    case 256: return launch_typed<KIND, 256, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
-    default: return cudaErrorInvalidValue;
+    switch (pl.bn) {
+      case 16: return launch_typed<KIND, 16, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+      case 32: return launch_typed<KIND, 32, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+      case 64: return launch_typed<KIND, 64, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+      case 128: return launch_typed<KIND, 128, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+      case 224:
+        if constexpr (KIND != kSparseBF16) {
+          if (pl.mt == 2)
+            return launch_typed<KIND, 224, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+        }
+        return launch_typed<KIND, 224, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+      case 256: return launch_typed<KIND, 256, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+      default: return cudaErrorInvalidValue;
+    }
   }
 }
 
@@ -1470,6 +1529,8 @@ cudaError_t launch_gemm(GemmKind kind, const GemmPlan &pl, const void *xq, const
       return launch_kind<kSparseE4M3Packed>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
     case kSparseI8Packed:
       return launch_kind<kSparseI8Packed>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
+    case kSparseFP4:
+      return launch_kind<kSparseFP4>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
     default:
       return cudaErrorInvalidValue;
   }

@@ -77,7 +77,14 @@ constexpr int kFusedMaxCtas = 256;
 constexpr size_t kFusedCounterBytes = 8192;
 
 // ---- gemm.cu
-enum GemmKind : int { kSparseE4M3 = 0, kDenseE4M3 = 1, kSparseBF16 = 2, kSparseE4M3Packed = 3, kSparseI8Packed = 4 };
+enum GemmKind : int {
+  kSparseE4M3 = 0,
+  kDenseE4M3 = 1,
+  kSparseBF16 = 2,
+  kSparseE4M3Packed = 3,
+  kSparseI8Packed = 4,
+  kSparseFP4 = 5  // E2M1 codes, two per byte, canonical 2:4 layout; stages of 256 K
+};
 
 // How a GEMM call is cut into CTAs: tile shape, work decomposition and the
 // scratch a stream-K reduction needs.

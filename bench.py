@@ -10,9 +10,10 @@ W[11008, 4096] (bf16, N(0, 0.02)) with X[M, 4096] (N(0, 1)) for M in
     2:4 prune/quantise/compress, written in the GEMM's tile-packed layout:
     ``sp24_prune_compress_packed``), and
   * for each M: quantises X and runs the sparse GEMM against another layer's
-    compressed weights: for M <= 256 in one launch
-    (``sp24_quantize_gemm_packed``), otherwise as ``fp8_quantize_pertensor``
-    followed by ``sp24_gemm_packed``.
+    compressed weights: for M <= 64 through ``sp24_quantize_gemm_packed``
+    (one launch when M * K <= 8192, else the one-cluster quantiser and the
+    GEMM behind it), otherwise as ``fp8_quantize_pertensor`` followed by
+    ``sp24_gemm_packed``.
 The 6:8 workload decomposes into the packed layout
 (``slide68_decompose_packed``) and lifts and quantises X instead
 (``slide68_lift_gemm_packed``, or ``slide68_lift`` + ``sp24_gemm_packed``).
@@ -78,6 +79,18 @@ def bytes_bf16_sparse_gemm(m, n, k):
     return n * k + n * k // 8 + 2 * m * k + 2 * m * n
 
 
+def bytes_prune24_fp4(n, k):
+    return 2 * n * k + n * k // 4 + n * k // 8 + 4
+
+
+def bytes_quant_fp4(m, k):
+    return 2 * m * k + m * k // 2 + 4
+
+
+def bytes_sparse_gemm_fp4(m, n, k):
+    return n * k // 4 + n * k // 8 + m * k // 2 + 2 * m * n + 8
+
+
 def bytes_slide68(n, k):
     return 2 * n * k + 3 * n * k // 4 + 3 * n * k // 16 + 4
 
@@ -93,6 +106,7 @@ def bytes_fused_gemm(m, n, k, kc):
 
 
 FUSED_MAX_M = 64  # above this the full-grid quantiser launch is faster
+FUSED_ONE_LAUNCH = 8192  # X elements up to which the fused call is one launch
 
 
 WORKLOADS = {
@@ -342,8 +356,10 @@ class GpuWorkload:
         for j, m in enumerate(self.ms):
             layer = (s * len(self.ms) + j) % self.R_g
             if self.fused[m]:
+                # one launch when every CTA can quantise X itself, else the
+                # quantiser and the GEMM behind it
                 ops.append((self.fused_name(), (lambda m=m, layer=layer: self.fused_op(m, layer)),
-                            bytes_fused_gemm(m, n, k, kc), 2 * m * n * kc, 1))
+                            bytes_fused_gemm(m, n, k, kc), 2 * m * n * kc, 1 if m * k <= FUSED_ONE_LAUNCH else 2))
                 continue
             aname = "slide68_lift" if self.is68 else "fp8_quantize_pertensor"
             abytes = bytes_lift(m, k) if self.is68 else bytes_quant(m, k)
@@ -587,6 +603,42 @@ class GpuWorkload:
         del pool
         return out
 
+    def fp4_compare(self, reps=50):
+        """FP4 (E2M1) with 2:4 weights on this workload's shapes: the FP4
+        weight path (prune + quantise + compress), the per-tensor FP4
+        quantiser and the FP4 sparse GEMM (rotating layers, larger than L2),
+        each a CUDA graph of back-to-back calls."""
+        if self.is68:
+            return None
+        torch, sp = self.torch, self.sp
+        n, k = self.n, self.k
+        outw = dict(values=torch.empty((n, k // 4), dtype=torch.uint8, device=self.dev),
+                    meta=torch.empty((n, k // 8), dtype=torch.uint8, device=self.dev),
+                    scale=torch.empty((1,), dtype=torch.float32, device=self.dev))
+        sp.sp24_prune_compress_fp4(self.w_pool[0], workspace=self.ws, out=outw)
+        npool = max(2, -(-3 * L2_BYTES // (n * k // 4 + n * k // 8)))
+        pool = [(outw["values"].clone(), outw["meta"].clone()) for _ in range(npool)]
+        sw = outw["scale"].clone()
+        t = self._graph_us(lambda r: sp.sp24_prune_compress_fp4(self.w_pool[r % self.R_w], workspace=self.ws,
+                                                                out=outw), max(4, reps // 5))
+        out = {"weight_path_us": round(t, 3), "weight_path_gbs": round(bytes_prune24_fp4(n, k) / t / 1e3, 1)}
+        for m in self.ms:
+            q = torch.empty((m, k // 2), dtype=torch.uint8, device=self.dev)
+            sx = torch.empty((1,), dtype=torch.float32, device=self.dev)
+            sp.fp4_quantize_pertensor(self.x_dev[m], workspace=self.ws, out=q, scale=sx)
+            sp.sp24_gemm_fp4(q, sx, pool[0][0], pool[0][1], sw, out=self.y[m], workspace=self.ws)
+            tq = self._graph_us(lambda r: sp.fp4_quantize_pertensor(self.x_dev[m], workspace=self.ws, out=q,
+                                                                   scale=sx), reps)
+            tg = self._graph_us(lambda r: sp.sp24_gemm_fp4(q, sx, pool[r % npool][0], pool[r % npool][1], sw,
+                                                          out=self.y[m], workspace=self.ws), reps)
+            out[str(m)] = {"quantize_us": round(tq, 3),
+                           "quantize_gbs": round(bytes_quant_fp4(m, k) / tq / 1e3, 1),
+                           "gemm_us": round(tg, 3),
+                           "gemm_gbs": round(bytes_sparse_gemm_fp4(m, n, k) / tg / 1e3, 1),
+                           "gemm_tflops_dense_equiv": round(2 * m * n * k / tg / 1e6, 2)}
+        del pool
+        return out
+
     def fusion_compare(self, reps=50):
         """For every M that the step runs fused: the fused launch against the
         activation kernel + GEMM pair it replaces, each as a CUDA graph of
@@ -735,6 +787,12 @@ def run_gpu(args, wl, rank, world, local_rank):
             int8 = gw.int8_compare()
         except Exception as e:  # a failure here is recorded, never fatal to the bench line
             int8 = {"error": f"{type(e).__name__}: {e}"[:300]}
+    fp4 = None
+    if rank == 0 and not args.no_compare:
+        try:
+            fp4 = gw.fp4_compare()
+        except Exception as e:  # a failure here is recorded, never fatal to the bench line
+            fp4 = {"error": f"{type(e).__name__}: {e}"[:300]}
     prefill = None
     if rank == 0 and args.workload == "decode" and not args.no_prefill:
         prefill = prefill_headline(device, peaks)
@@ -774,6 +832,7 @@ def run_gpu(args, wl, rank, world, local_rank):
         "finer_scales": finer,
         "general_slide": general,
         "int8_w8a8": int8,
+        "fp4_e2m1": fp4,
         "e2e": {"value": round(aggregate_gbs(step_bytes, args.steps, world, e2e_t), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": gw.step_launches() * args.steps,
@@ -927,6 +986,18 @@ def kernel_case(name, device):
     elif name == "int8_prune":                   # W[11008, 4096] INT8 2:4 weight path
         w = w_decode()
         call = lambda: sp.sp24_prune_compress_int8(w, workspace=ws)
+    elif name == "fp4_quantize":                 # X[4096, 4096] per-tensor FP4 E2M1
+        x = bf(WL.activation_bits(3, 4096))
+        call = lambda: sp.fp4_quantize_pertensor(x, workspace=ws)
+    elif name == "fp4_prune":                    # W[11008, 4096] FP4 2:4 weight path
+        w = w_decode()
+        call = lambda: sp.sp24_prune_compress_fp4(w, workspace=ws)
+    elif name == "gemm_fp4_decode":              # M64 N11008 K4096, FP4 A and B
+        w = w_decode()
+        x = bf(WL.activation_bits(2, 64))
+        c = sp.sp24_prune_compress_fp4(w, workspace=ws)
+        xq, sx = sp.fp4_quantize_pertensor(x, workspace=ws)
+        call = lambda: sp.sp24_gemm_fp4(xq, sx, c["values"], c["meta"], c["scale"], workspace=ws)
     elif name in ("slide46_decompose", "slide46_lift"):   # 4:6 at K = 4608 (K' = 6144)
         if name == "slide46_decompose":
             w = bf(WL.random_bits((4096, 4608), 2301, scale=0.02))

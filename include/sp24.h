@@ -125,6 +125,10 @@ int sp24_prune_compress(const void *W, int N, int K, int out_dtype, void *values
  * X: bf16 [rows, cols] -> q: u8 [rows, cols], scale <- amax|X| / 448 (1.0 when
  * amax = 0), q = E4M3(x / scale) as above.  Also used for the weights of the
  * dense FP8 comparison GEMM.  Shape rules: rows >= 1, cols >= 1, cols % 16 == 0.
+ * A decode-sized X (rows * cols <= 262144) is done by one thread-block
+ * cluster that leaves the workspace untouched and lets the next kernel on
+ * `stream` launch at once (it must wait for this one before reading q or
+ * scale, as every kernel of this library does).
  */
 int fp8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, uint8_t *q, float *scale,
                            void *workspace, size_t ws_bytes, int32_t *status,
@@ -149,7 +153,8 @@ int slide68_decompose(const void *W, int N, int K, int out_dtype, void *values, 
  * Activation lift fused with per-tensor E4M3 quantisation (SlideSparse, §2
  * "Levantamiento de Activacion").  X: bf16 [M, K] -> q_lifted: u8 [M, 3K/2]
  * with q_lifted[m, 12g + 4j + r] = E4M3(X[m, 8g + 2j + r] / scale), scale <-
- * amax|X| / 448.  Shape rules: M >= 1, K % 16 == 0.
+ * amax|X| / 448.  Shape rules: M >= 1, K % 16 == 0.  M * K <= 262144: one
+ * thread-block cluster, as for fp8_quantize_pertensor.
  */
 int slide68_lift(const void *X, int M, int K, uint8_t *q_lifted, float *scale, void *workspace,
                  size_t ws_bytes, int32_t *status, sp24_stream_t stream);
@@ -231,17 +236,20 @@ int sp24_gemm_packed(const void *Xq, const float *x_scale, const void *packed,
                      size_t ws_bytes, int32_t *status, sp24_stream_t stream);
 
 /*
- * Per-tensor activation quantisation and the packed sparse GEMM in one
- * launch, for small token counts (decode).  Computes exactly what
+ * Per-tensor activation quantisation and the packed sparse GEMM, for small
+ * token counts (decode).  Computes exactly what
  *   fp8_quantize_pertensor(X, M, K, Xq, x_scale, ...) followed by
  *   sp24_gemm_packed(Xq, x_scale, packed, w_scale, Y, M, N, K, ...)
  * computes: Xq u8 [M, K] <- E4M3(x / x_scale), x_scale <- amax|X| / 448
  * (1.0 when amax = 0), Y bf16 [M, N]; Xq and x_scale are outputs (the codes
- * can feed further GEMMs of the same X).  X: bf16 [M, K].  The GEMM's CTAs
- * compute the amax of X between them, encode it, and start their tensor-core
- * work on the codes, while the packed weights already stream in.  Workspace:
+ * can feed further GEMMs of the same X).  X: bf16 [M, K].  When M * K <=
+ * 8192 it is ONE launch: every CTA of the GEMM quantises all of X itself and
+ * starts its tensor-core work on the codes while the packed weights already
+ * stream in.  Otherwise the quantiser runs first (one thread-block cluster up
+ * to M * K = 262144) and the GEMM, launched right behind it, streams its
+ * weights while it runs.  Workspace:
  * sp24_workspace_size(SP24_OP_QUANTIZE_GEMM_PACKED, M, N, K, 0) (its first
- * 8 KB are counters and per-CTA flags, zero before the first use and after
+ * 8 KB hold the quantiser's counters, zero before the first use and after
  * every call).
  * Shape rules: 1 <= M <= 256, N % 128 == 0, K % 128 == 0.  Xq and Y must not
  * alias X or each other.  SP24_STATUS_NONFINITE is set as by

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsp24.so")
-SOURCES = ["api.cu", "elementwise.cu", "fp4.cu", "gemm.cu", "int8.cu", "noalloc.cu", "rowscale.cu", "slide.cu",
+SOURCES = ["api.cu", "elementwise.cu", "fp4.cu", "gemm.cu", "int8.cu", "noalloc.cu", "rowscale.cu", "slide.cu", "smallx.cu",
            "stream.cu"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]

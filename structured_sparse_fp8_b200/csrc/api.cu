@@ -182,6 +182,8 @@ int fp8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, uint8_t *q
   const int64_t nelem = rows * cols;
   const int rc = check_workspace(workspace, ws_bytes);
   if (rc != SP24_OK) return rc;
+  if (sp24::small_quantize_fits(nelem))
+    return cuda_status(sp24::launch_quantize_small(X, nelem, false, scale, q, status, st));
   return cuda_status(sp24::launch_quantize_fused(X, nelem, static_cast<uint32_t *>(workspace), scale,
                                                  q, status, sms, st));
 }
@@ -244,6 +246,8 @@ int slide68_lift(const void *X, int M, int K, uint8_t *q_lifted, float *scale, v
   const int64_t nelem = static_cast<int64_t>(M) * K;
   const int rc = check_workspace(workspace, ws_bytes);
   if (rc != SP24_OK) return rc;
+  if (sp24::small_quantize_fits(nelem))
+    return cuda_status(sp24::launch_quantize_small(X, nelem, true, scale, q_lifted, status, st));
   return cuda_status(sp24::launch_lift_fused(X, nelem, static_cast<uint32_t *>(workspace), scale,
                                              q_lifted, status, sms, st));
 }
@@ -365,18 +369,33 @@ static int quant_gemm_common(bool lift, const void *X, int M, int N, int K, cons
   if (sms < 0) return SP24_ERR_ARCH;
   const int Kg = lift ? K / 2 * 3 : K;
   const sp24::GemmPlan pl = sp24::plan_gemm(sp24::kSparseE4M3Packed, M, N, Kg, sms);
-  if (pl.grid > sp24::kFusedMaxCtas) return SP24_ERR_SHAPE;
   if (!workspace || ws_bytes < sp24::kFusedCounterBytes + pl.workspace_bytes()) return SP24_ERR_WORKSPACE;
   if (!aligned16(workspace)) return SP24_ERR_ALIGN;
-  sp24::GemmFusedX fx;
-  fx.x = X;
-  fx.lift = lift ? 1 : 0;
-  fx.xq = Xq;
-  fx.x_scale = x_scale;
-  fx.counters = static_cast<uint32_t *>(workspace);
-  return cuda_status(sp24::launch_gemm_quant(pl, fx, packed, w_scale, Y, M, N, Kg,
-                                             static_cast<uint8_t *>(workspace) + sp24::kFusedCounterBytes,
-                                             status, reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void *gemm_ws = static_cast<uint8_t *>(workspace) + sp24::kFusedCounterBytes;
+  const int64_t nelem = static_cast<int64_t>(M) * K;
+  if (nelem / 8 <= sp24::kFusedXVec) {
+    // one launch: every CTA quantises all of X in front of its GEMM tiles
+    sp24::GemmFusedX fx;
+    fx.x = X;
+    fx.lift = lift ? 1 : 0;
+    fx.xq = Xq;
+    fx.x_scale = x_scale;
+    return cuda_status(sp24::launch_gemm_quant(pl, fx, packed, w_scale, Y, M, N, Kg, gemm_ws, status, st));
+  }
+  // Larger X: the quantiser (one cluster for decode-sized X, which lets the
+  // GEMM launch at once and stream its weights meanwhile; the streamed
+  // kernel beyond that), then the GEMM on its codes.
+  cudaError_t e;
+  if (sp24::small_quantize_fits(nelem))
+    e = sp24::launch_quantize_small(X, nelem, lift, x_scale, Xq, status, st);
+  else if (lift)
+    e = sp24::launch_lift_fused(X, nelem, static_cast<uint32_t *>(workspace), x_scale, Xq, status, sms, st);
+  else
+    e = sp24::launch_quantize_fused(X, nelem, static_cast<uint32_t *>(workspace), x_scale, Xq, status, sms, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  return cuda_status(sp24::launch_gemm(sp24::kSparseE4M3Packed, pl, Xq, x_scale, packed, nullptr, w_scale, Y, M,
+                                       N, Kg, gemm_ws, status, st));
 }
 
 int sp24_quantize_gemm_packed(const void *X, int M, int N, int K, const void *packed,

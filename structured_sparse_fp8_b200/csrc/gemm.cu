@@ -273,14 +273,12 @@ struct GemmArgs {
   const uint8_t *packed;  // tile-packed weights (packed kind only)
   // Fused activation quantisation (XQ != 0): bf16 X of xvec 8-element
   // vectors in, its E4M3 codes (lifted for XQ = 2) out to xq, which is the
-  // B operand the kernel then loads; xbar = the kFusedCounterBytes prefix
-  // (departure count and per-CTA slots, see kXSlotAmax), zero between calls.
+  // B operand the kernel then loads.
   const uint16_t *x;
   uint8_t *xq;
   float *x_scale_out;
-  uint32_t *xbar;
   int64_t xvec;
-  int xstaged;  // local form with the codes staged in shared memory (kXStage)
+  int xstaged;  // codes staged in shared memory (kXStage)
   // Scale vectors (VS kernels): x_scale holds M per-token scales when x_vec,
   // w_scale N per-channel scales when w_vec; otherwise one value each.
   int x_vec, w_vec;
@@ -355,16 +353,6 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
   return v;
 }
 
-__device__ __forceinline__ void st_release_gpu(uint32_t *p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t *p) {
-  uint32_t v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
 // Spin (bounded) until *p reaches `expect`; acquire semantics.
 __device__ __forceinline__ void wait_count_gpu(const uint32_t *p, uint32_t expect, int32_t *status) {
   const uint64_t t0 = global_timer_ns();
@@ -379,101 +367,22 @@ __device__ __forceinline__ void wait_count_gpu(const uint32_t *p, uint32_t expec
 }
 
 // Per-tensor E4M3 quantisation of the activations fused in front of the
-// GEMM, run by the 128 epilogue threads (t = 0..127) while the producer
-// already streams weights.  Each thread loads its vectors of X once (up to
-// kXReg 16-byte vectors kept in registers; more are loaded again to encode)
-// and encodes them with e4m3_code_quot, which equals the correctly rounded
-// division on every input.  Two forms:
-//  * grid-wide (the usual one): (1) amax of this CTA's slice of X (a
-//    contiguous range of 8-element vectors), (2) written to the CTA's amax
-//    slot; CTA 0 takes the max over every slot and publishes it (see
-//    kXCopies), (3) s = amax / 448 (1 when amax = 0) and this slice's codes
-//    E4M3(RN_fp32(x / s)) written to xq, (4) the CTA's codes slot set; CTA
-//    0's producer waits for every codes slot and publishes, and every
-//    producer waits for that before it loads X codes, then counts its CTA's
-//    departure in xbar[3].  Every CTA becomes resident (at most one per SM,
-//    and one fits), so the slots fill; each wait is bounded anyway.
-//  * local (X of at most kLocalXVec vectors): every CTA takes the amax of
-//    all of X and encodes all of it itself, so no CTA waits for another and
-//    the counters are not touched.  When the codes fit kXStageBytes
-//    (`xstage`, BN = 16 kernels) they go to shared memory, from where the
-//    producer copies each stage's rows into its B tile, and only CTA 0
-//    writes them to xq for the caller; otherwise every CTA writes the
-//    (identical) codes to xq and its producer TMA-loads them.  Either way
-//    the producer waits for this CTA only (x_ready).
+// GEMM (X of at most kFusedXVec 8-element vectors: decode batches of a few
+// tokens), run by the 128 epilogue threads (t = 0..127) while the producer
+// already streams weights.  Every CTA takes the amax of all of X and encodes
+// all of it itself (each thread holds up to kXReg 16-byte vectors in
+// registers), so no CTA waits for another: s = amax / 448 (1 when amax = 0),
+// codes E4M3(RN_fp32(x / s)) by e4m3_codes8_fast, which equals the correctly
+// rounded division on every input (e4m3_codes8_div where it cannot decide).
+// When the codes fit kXStageBytes (`xstage`, BN = 16 kernels) they go to
+// shared memory, from where the producer copies each stage's rows into its B
+// tile, and only CTA 0 writes them to xq for the caller; otherwise every CTA
+// writes the (identical) codes to xq and its producer TMA-loads them.  Either
+// way the producer waits for this CTA only (x_ready).
 // XQ = 2 writes the SlideSparse lift: each 8-group g of a row becomes the 12
 // codes of windows 2j..2j+3, j = 0..2.  Returns s.
-constexpr int64_t kLocalXVec = 1024;
 constexpr int kXReg = 8;
-// Grid-wide form: 32-bit words of the counter prefix (kFusedCounterBytes).
-// CTA g writes its amax | 0x10000 (nonzero) to slot kXSlotAmax + g and, once
-// its codes are written, 1 to kXSlotCodes + g; each slot is written once per
-// call.  CTA 0 alone polls the slots (one warp: every CTA polling the same
-// few lines made their writes queue behind the reads for microseconds) and
-// publishes the result to kXCopies copies, one per 128-byte line, which the
-// other CTAs poll (CTA g the copy g % kXCopies).  Word 3 counts departures;
-// the last CTA to leave clears slots and copies.  GPU-scope fences are few:
-// the release before a codes slot, CTA 0's acquire-and-release before the
-// codes copies and before its departure, and each reader's acquire.
-constexpr int kXCopies = 16;
-constexpr int kXCopyAmax = 32;                      // copy f at word kXCopyAmax + 32 f
-constexpr int kXCopyCodes = 32 * (1 + kXCopies);    // copy f at word kXCopyCodes + 32 f
-constexpr int kXSlotAmax = 32 * (1 + 2 * kXCopies);  // slot g at word kXSlotAmax + g
-constexpr int kXSlotCodes = kXSlotAmax + 256;
-
-__device__ __forceinline__ void st_relaxed_gpu(uint32_t *p, uint32_t v) {
-  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Poll (bounded; backing off from 32 to 256 ns) until *p is nonzero and
-// return it.  No fence: the caller adds one when the word releases other
-// data.
-__device__ __forceinline__ uint32_t wait_word_gpu(const uint32_t *p, int32_t *status) {
-  uint32_t v = ld_relaxed_gpu(p);
-  if (v == 0u) {
-    const uint64_t t0 = global_timer_ns();
-    uint32_t ns = 32, polls = 0;
-    while ((v = ld_relaxed_gpu(p)) == 0u) {
-      __nanosleep(ns);
-      ns = min(ns * 2u, 256u);
-      if ((++polls & 15u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
-        if (status) atomicOr(status, SP24_STATUS_TIMEOUT);
-        break;
-      }
-    }
-  }
-  return v;
-}
-
-// One warp (all 32 lanes) polls slots[0 .. n), n <= 256, until every slot is
-// nonzero (bounded; the loads of a poll are all in flight at once, and the
-// polls back off from 64 to 256 ns) and returns the largest value.  No fence:
-// the caller adds one when the slots release other data.
-__device__ __forceinline__ uint32_t wait_slots_warp(const uint32_t *slots, int n, int32_t *status) {
-  const int lane = threadIdx.x & 31;
-  const uint64_t t0 = global_timer_ns();
-  uint32_t polls = 0, ns = 64, mx = 0;
-  while (true) {
-    uint32_t v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = lane + 32 * j < n ? ld_relaxed_gpu(slots + lane + 32 * j) : 1u;
-    uint32_t mn = 0xFFFFFFFFu;
-    mx = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      mn = min(mn, v[j]);
-      mx = max(mx, v[j]);
-    }
-    if (__all_sync(0xFFFFFFFFu, mn != 0u)) break;
-    __nanosleep(ns);
-    ns = min(ns * 2u, 256u);
-    if ((++polls & 15u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
-      if (lane == 0 && status) atomicOr(status, SP24_STATUS_TIMEOUT);
-      break;
-    }
-  }
-  return __reduce_max_sync(0xFFFFFFFFu, mx);
-}
+static_assert(kFusedXVec <= 128 * kXReg, "every thread holds its vectors of X in registers");
 
 template <int XQ>
 __device__ __forceinline__ void store_xvec(uint8_t *dst, int64_t v, const uint2 c) {
@@ -490,104 +399,57 @@ __device__ __forceinline__ void store_xvec(uint8_t *dst, int64_t v, const uint2 
 template <int XQ>
 __device__ float fused_quantize(const GemmArgs &p, int t, uint32_t *s_red, float *s_scale, uint64_t *x_ready,
                                 uint8_t *xstage) {
-  const bool local = p.xvec <= kLocalXVec;
-  const int64_t v0 = local ? 0 : static_cast<int64_t>(blockIdx.x) * p.xvec / gridDim.x;
-  const int64_t v1 = local ? p.xvec : static_cast<int64_t>(blockIdx.x + 1) * p.xvec / gridDim.x;
+  const int64_t nvec = p.xvec;
   const uint4 *xv = reinterpret_cast<const uint4 *>(p.x);
-  // vectors v0 + t + 128 u, u < kXReg: all loads in flight at once, kept
+  // vectors t + 128 u, u < kXReg: all loads in flight at once, kept
   uint4 w[kXReg];
 #pragma unroll
   for (int u = 0; u < kXReg; ++u)
-    w[u] = v0 + t + 128 * u < v1 ? __ldg(xv + v0 + t + 128 * u) : make_uint4(0u, 0u, 0u, 0u);
+    w[u] = t + 128 * u < nvec ? __ldg(xv + t + 128 * u) : make_uint4(0u, 0u, 0u, 0u);
   uint32_t m2 = 0;
 #pragma unroll
   for (int u = 0; u < kXReg; ++u) m2 = __vmaxu2(m2, absmax8x2(w[u]));
-  for (int64_t v = v0 + t + 128 * kXReg; v < v1; v += 128 * kXReg) {  // large X: batches of kXReg loads
-    uint4 r[kXReg];
-#pragma unroll
-    for (int u = 0; u < kXReg; ++u) r[u] = v + 128 * u < v1 ? __ldg(xv + v + 128 * u) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-    for (int u = 0; u < kXReg; ++u) m2 = __vmaxu2(m2, absmax8x2(r[u]));
-  }
-  uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
-  if ((t & 31) == 0) s_red[t >> 5] = mx;
+  const uint32_t mw = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
+  if ((t & 31) == 0) s_red[t >> 5] = mw;
   named_bar_sync(1, 128);
-  if (t < 32) {
-    mx = max(max(s_red[0], s_red[1]), max(s_red[2], s_red[3]));
-    uint32_t amax = mx;
-    if (!local) {
-      if (t == 0) st_relaxed_gpu(&p.xbar[kXSlotAmax + blockIdx.x], mx | 0x10000u);
-      if (blockIdx.x == 0) {
-        amax = wait_slots_warp(&p.xbar[kXSlotAmax], gridDim.x, p.status) & 0xFFFFu;
-        if (t < kXCopies) st_relaxed_gpu(&p.xbar[kXCopyAmax + 32 * t], amax | 0x10000u);  // the data itself
-      } else if (t == 0) {
-        amax = wait_word_gpu(&p.xbar[kXCopyAmax + 32 * (blockIdx.x % kXCopies)], p.status) & 0xFFFFu;
-      }
+  if (t == 0) {
+    const uint32_t amax = max(max(s_red[0], s_red[1]), max(s_red[2], s_red[3]));
+    const float sx = amax == 0u ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax), 448.0f);
+    if (blockIdx.x == 0) {
+      if (amax >= 0x7F80u && p.status) atomicOr(p.status, SP24_STATUS_NONFINITE);
+      *p.x_scale_out = sx;
     }
-    if (t == 0) {
-      const float sx = amax == 0u ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax), 448.0f);
-      if (blockIdx.x == 0) {
-        if (amax >= 0x7F80u && p.status) atomicOr(p.status, SP24_STATUS_NONFINITE);
-        *p.x_scale_out = sx;
-      }
-      s_scale[0] = sx;
-      s_scale[1] = __frcp_rn(sx);
-    }
+    s_scale[0] = sx;
+    s_scale[1] = __frcp_rn(sx);
   }
   named_bar_sync(1, 128);
   const float sx = s_scale[0], rx = s_scale[1];
   uint8_t *dst = xstage ? xstage : p.xq;
   const bool also_out = xstage && blockIdx.x == 0;  // staged codes: CTA 0 returns them
-  {
-    // this thread's vectors in registers: v0 + t + 128 u for u < nv, encoded
-    // two at a time (the pairs interleave; no work for absent vectors)
-    const int64_t mine = v1 - v0 - t;
-    const int nv = mine <= 0 ? 0 : static_cast<int>(mine >= 128 * kXReg ? kXReg : (mine + 127) / 128);
+  // this thread's nv vectors, encoded two at a time (the pairs interleave; no
+  // work for absent vectors)
+  const int64_t mine = nvec - t;
+  const int nv = mine <= 0 ? 0 : static_cast<int>(mine >= 128 * kXReg ? kXReg : (mine + 127) / 128);
 #pragma unroll
-    for (int u = 0; u < kXReg; u += 2) {
-      if (u < nv) {
-        bool ok0, ok1;
-        uint2 c0 = e4m3_codes8_fast(w[u], rx, ok0);
-        uint2 c1 = e4m3_codes8_fast(w[u + 1], rx, ok1);
-        if (!ok0) c0 = e4m3_codes8_div(w[u], sx);
-        if (!ok1) c1 = e4m3_codes8_div(w[u + 1], sx);
-        const int64_t v = v0 + t + 128 * u;
-        store_xvec<XQ>(dst, v, c0);
-        if (also_out) store_xvec<XQ>(p.xq, v, c0);
-        if (u + 1 < nv) {
-          store_xvec<XQ>(dst, v + 128, c1);
-          if (also_out) store_xvec<XQ>(p.xq, v + 128, c1);
-        }
-      }
-    }
-  }
-  for (int64_t v = v0 + t + 128 * kXReg; v < v1; v += 128 * kXReg) {
-    uint4 r[kXReg];
-#pragma unroll
-    for (int u = 0; u < kXReg; ++u) r[u] = v + 128 * u < v1 ? __ldg(xv + v + 128 * u) : make_uint4(0u, 0u, 0u, 0u);
-    uint2 c[kXReg];
-    bool ok[kXReg];
-#pragma unroll
-    for (int u = 0; u < kXReg; ++u) c[u] = e4m3_codes8_fast(r[u], rx, ok[u]);
-#pragma unroll
-    for (int u = 0; u < kXReg; ++u)
-      if (!ok[u]) c[u] = e4m3_codes8_div(r[u], sx);
-#pragma unroll
-    for (int u = 0; u < kXReg; ++u) {
-      if (v + 128 * u < v1) {
-        store_xvec<XQ>(dst, v + 128 * u, c[u]);
-        if (also_out) store_xvec<XQ>(p.xq, v + 128 * u, c[u]);
+  for (int u = 0; u < kXReg; u += 2) {
+    if (u < nv) {
+      bool ok0, ok1;
+      uint2 c0 = e4m3_codes8_fast(w[u], rx, ok0);
+      uint2 c1 = e4m3_codes8_fast(w[u + 1], rx, ok1);
+      if (!ok0) c0 = e4m3_codes8_div(w[u], sx);
+      if (!ok1) c1 = e4m3_codes8_div(w[u + 1], sx);
+      const int64_t v = t + 128 * u;
+      store_xvec<XQ>(dst, v, c0);
+      if (also_out) store_xvec<XQ>(p.xq, v, c0);
+      if (u + 1 < nv) {
+        store_xvec<XQ>(dst, v + 128, c1);
+        if (also_out) store_xvec<XQ>(p.xq, v + 128, c1);
       }
     }
   }
   if (!xstage) fence_proxy_async_global();  // the codes are read back by TMA loads
   named_bar_sync(1, 128);
-  if (t == 0) {
-    if (local)
-      mbar_arrive(x_ready);
-    else
-      st_release_gpu(&p.xbar[kXSlotCodes + blockIdx.x], 1u);  // releases the codes (bar.sync above)
-  }
+  if (t == 0) mbar_arrive(x_ready);
   return sx;
 }
 
@@ -620,7 +482,7 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
   uint64_t *meta_ready = empty + S;
   uint64_t *tmem_full = meta_ready + S;
   uint64_t *tmem_empty = tmem_full + NB;
-  uint64_t *x_ready = tmem_empty + NB;  // fused local quantisation: codes written
+  uint64_t *x_ready = tmem_empty + NB;  // fused quantisation: codes written
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(x_ready + 1);
   [[maybe_unused]] __shared__ uint32_t s_xred[4];
   [[maybe_unused]] __shared__ float s_xscale[2];
@@ -768,42 +630,8 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
       }
       grid_dependency_wait();
       if constexpr (XQ != 0) {
-        // the activation codes are written by the epilogue warps: of this
-        // CTA (local form) or of the whole grid
-        if (p.xvec <= kLocalXVec) {
-          mbar_wait_warp(x_ready, 0u, p.status);
-        } else {
-          if (blockIdx.x == 0) {
-            // gather every CTA's codes slot, acquire their codes and release
-            // them again through the copies
-            wait_slots_warp(&p.xbar[kXSlotCodes], gridDim.x, p.status);
-            __syncwarp();
-            asm volatile("fence.acq_rel.gpu;" ::: "memory");
-            if (lane < kXCopies) st_relaxed_gpu(&p.xbar[kXCopyCodes + 32 * lane], 1u);
-            __syncwarp();
-            asm volatile("fence.acq_rel.gpu;" ::: "memory");  // the copies before the departure below
-          } else {
-            if (leader) wait_word_gpu(&p.xbar[kXCopyCodes + 32 * (blockIdx.x % kXCopies)], p.status);
-            __syncwarp();
-            asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire every CTA's codes
-          }
-          // This CTA reads the slots and copies no more (its epilogue read
-          // the amax before setting its codes slot): count its departure;
-          // the last CTA to leave clears them.
-          uint32_t last = 0;
-          if (leader) last = atomicAdd(&p.xbar[3], 1u) == gridDim.x - 1 ? 1u : 0u;
-          if (__shfl_sync(0xFFFFFFFFu, last, 0)) {  // the leader is lane 0 of the converged warp
-            for (int g = lane; g < static_cast<int>(gridDim.x); g += 32) {
-              p.xbar[kXSlotAmax + g] = 0u;
-              p.xbar[kXSlotCodes + g] = 0u;
-            }
-            if (lane < kXCopies) {
-              p.xbar[kXCopyAmax + 32 * lane] = 0u;
-              p.xbar[kXCopyCodes + 32 * lane] = 0u;
-            }
-            if (leader) p.xbar[3] = 0u;
-          }
-        }
+        // the activation codes are written by this CTA's epilogue warps
+        mbar_wait_warp(x_ready, 0u, p.status);
         __syncwarp();
         if (!staged) fence_proxy_async_global();
       }
@@ -1308,13 +1136,6 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   std::call_once(attr_once, [] {
     attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN, MT, XQ, KB, VS>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (attr_err == cudaSuccess && XQ != 0) {
-      // the fused quantisation's grid-wide counts rely on one CTA fitting an SM
-      int per_sm = 0;
-      attr_err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemm_kernel<KIND, BN, MT, XQ, KB, VS>,
-                                                               C::kThreads, C::kSmemBytes);
-      if (attr_err == cudaSuccess && per_sm < 1) attr_err = cudaErrorCooperativeLaunchTooLarge;
-    }
   });
   if (attr_err != cudaSuccess) return attr_err;
 
@@ -1377,7 +1198,6 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   a.x = nullptr;
   a.xq = nullptr;
   a.x_scale_out = nullptr;
-  a.xbar = nullptr;
   a.xvec = 0;
   a.xstaged = 0;
   a.x_vec = x_vec;
@@ -1386,9 +1206,9 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
     a.x = static_cast<const uint16_t *>(fx->x);
     a.xq = fx->xq;
     a.x_scale_out = fx->x_scale;
-    a.xbar = fx->counters;
     a.xvec = static_cast<int64_t>(M) * (XQ == 2 ? K / 3 * 2 : K) / 8;
-    a.xstaged = (C::kXStage > 0 && a.xvec <= kLocalXVec && static_cast<int64_t>(M) * K <= kXStageBytes) ? 1 : 0;
+    if (a.xvec > kFusedXVec) return cudaErrorInvalidValue;
+    a.xstaged = (C::kXStage > 0 && static_cast<int64_t>(M) * K <= kXStageBytes) ? 1 : 0;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(pl.grid), 1, 1);
@@ -1396,14 +1216,12 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = st;
   // Programmatic dependent launch (see the kernel).  Stream-K owners wait
-  // for contributor CTAs, and the fused quantisation's grid-wide counts wait
-  // for every CTA.  Both only need every CTA to become resident eventually:
-  // the grid is at most one CTA per SM and one CTA fits an SM (checked once
-  // above), so every CTA is resident as soon as the kernels ahead of it
-  // drain, and each wait is bounded anyway.  The launch is not cooperative:
-  // a cooperative grid was measured to start 1-2 us later behind the
-  // previous kernel, losing the weight prefetch that programmatic launch
-  // overlaps with it.
+  // for contributor CTAs, which only needs every CTA to become resident
+  // eventually: the grid is at most one CTA per SM, so every CTA is resident
+  // as soon as the kernels ahead of it drain, and each wait is bounded
+  // anyway.  The launch is not cooperative: a cooperative grid was measured
+  // to start 1-2 us later behind the previous kernel, losing the weight
+  // prefetch that programmatic launch overlaps with it.
   cudaLaunchAttribute attrs[1];
   attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attrs[0].val.programmaticStreamSerializationAllowed = 1;

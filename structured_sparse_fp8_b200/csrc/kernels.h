@@ -69,12 +69,19 @@ void set_last_cuda_error(int e);
 // Bytes of scratch the amax/scale reduction uses (two counters, padded).
 constexpr size_t kAmaxWorkspaceBytes = 256;
 
-// Counter prefix of the fused quantise + GEMM workspace: a line of counters,
-// 32 lines of published copies, then one 32-bit slot per CTA (at most
-// kFusedMaxCtas) for the amax and one for "codes written" (6272 bytes,
-// padded).  Zero before the first call and after every call.
-constexpr int kFusedMaxCtas = 256;
+// Prefix of the fused quantise + GEMM workspace: the counters of the
+// activation quantiser that runs in front of the GEMM when X is too large for
+// the one-launch form (kAmaxWorkspaceBytes used, the rest reserved).  Zero
+// before the first call and after every call.
 constexpr size_t kFusedCounterBytes = 8192;
+
+// ---- smallx.cu: decode-sized activations (at most kSmallXVec 8-element
+// vectors, nelem % 8 == 0) quantised, or lifted (rows of 16k elements), by
+// one thread-block cluster; no workspace.
+constexpr int64_t kSmallXVec = 32768;
+bool small_quantize_fits(int64_t nelem);
+cudaError_t launch_quantize_small(const void *x, int64_t nelem, bool lift, float *scale, uint8_t *q,
+                                  int32_t *status, cudaStream_t st);
 
 // ---- gemm.cu
 enum GemmKind : int {
@@ -126,14 +133,15 @@ cudaError_t launch_gemm_scaled(const GemmPlan &plan, const void *xq, const float
                                int K, void *workspace, int32_t *status, cudaStream_t st);
 
 // The packed E4M3 GEMM with the per-tensor quantisation of its activations
-// fused in front (plan from plan_gemm(kSparseE4M3Packed, M, N, K); bn <= 128,
-// mt == 1).  K is the GEMM's K: the columns of X, or 3/2 of them with lift.
+// fused in front, for X of at most kFusedXVec 8-element vectors (plan from
+// plan_gemm(kSparseE4M3Packed, M, N, K); bn <= 128, mt == 1).  K is the
+// GEMM's K: the columns of X, or 3/2 of them with lift.
+constexpr int64_t kFusedXVec = 1024;
 struct GemmFusedX {
   const void *x;       // bf16 [M, Kx]
   int lift;            // 0: codes [M, Kx]; 1: SlideSparse lift, codes [M, 3 Kx / 2]
   uint8_t *xq;         // out: the E4M3 codes (the GEMM's B operand)
   float *x_scale;      // out: amax|X| / 448 (1 when amax = 0)
-  uint32_t *counters;  // kFusedCounterBytes, zero before the call and after it
 };
 cudaError_t launch_gemm_quant(const GemmPlan &plan, const GemmFusedX &fx, const void *packed,
                               const float *w_scale, void *y, int M, int N, int K, void *workspace,

@@ -71,7 +71,14 @@ __device__ __forceinline__ bool e4m3_codes4_quot(uint32_t h0, uint32_t h1, float
   return bad == 0u;
 }
 
-// The exact form, out of line: rare, and kept out of the unrolled loops.
+// The exact forms, out of line: rare, and kept out of the unrolled loops.
+static __device__ __noinline__ uint32_t e4m3_codes4_div(uint32_t h0, uint32_t h1, float s) {
+  const uint32_t hh[4] = {h0 & 0xFFFFu, h0 >> 16, h1 & 0xFFFFu, h1 >> 16};
+  uint32_t q = 0u;
+  for (int i = 0; i < 4; ++i) q |= e4m3_code(__fdiv_rn(bf16_bits_to_float(hh[i]), s)) << (8 * i);
+  return q;
+}
+
 static __device__ __noinline__ uint2 e4m3_codes8_div(const uint4 w, float s) {
   const uint32_t h[4] = {w.x, w.y, w.z, w.w};
   uint32_t q[2] = {0u, 0u};

@@ -82,6 +82,69 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, i
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
+// ---------------------------------------------------------- clusters
+// This CTA's rank in its thread-block cluster.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// The shared::cluster address of the object at `p` (this CTA's shared
+// memory) in the CTA of the cluster with rank `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(const void *p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_addr(p)), "r"(rank));
+  return a;
+}
+
+__device__ __forceinline__ void st_shared_cluster(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Arrive on the mbarrier at shared::cluster address `addr` (this or another
+// CTA of the cluster), releasing this thread's earlier writes at cluster
+// scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait (bounded) for a phase of `bar` whose arrivals come from other CTAs of
+// the cluster, acquiring their writes at cluster scope.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, int32_t *status) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1; i < kWaitLimitIters; ++i) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((i & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) break;
+  }
+  if (status) atomicOr(status, SP24_STATUS_TIMEOUT);
+  return false;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t *bar, uint32_t parity, int32_t *status) {
+  const bool ok = mbar_wait_cluster(bar, parity, (threadIdx.x & 31) == 0 ? status : nullptr);
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// Every thread of every CTA of the cluster: arrive (releasing) and wait
+// (acquiring).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // One lane of a converged warp (the same lane every time): the issuer of
 // TMA and tcgen05 instructions whose operands the whole warp computed.
 __device__ __forceinline__ bool elect_one() {

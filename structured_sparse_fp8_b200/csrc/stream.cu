@@ -136,7 +136,35 @@ struct CodeTable {
     else
       return tab[h];
   }
+  // codes of the bf16 values h0 (elements 0, 1) and h1 (2, 3), byte i = element i
+  __device__ __forceinline__ uint32_t codes4(uint32_t h0, uint32_t h1) const {
+    return (*this)(h0 & 0xFFFFu) | (*this)(h0 >> 16) << 8 | (*this)(h1 & 0xFFFFu) << 16 | (*this)(h1 >> 16) << 24;
+  }
 };
+
+// The same codes without a table: q = RN(x * RN(1 / s)) and the codes 8
+// steps either side of it, four values at once (e4m3_codes4_quot); the
+// correctly rounded division where that cannot decide (about one value in
+// 2^16).  Cheaper per code than the byte lookups of the table, which conflict
+// on shared-memory banks.
+struct CodeQuot {
+  float s, r;
+  __device__ __forceinline__ uint32_t operator()(uint32_t h) const {
+    return e4m3_code(__fdiv_rn(bf16_bits_to_float(h), s));
+  }
+  __device__ __forceinline__ uint32_t codes4(uint32_t h0, uint32_t h1) const {
+    uint32_t q;
+    if (!e4m3_codes4_quot(h0, h1, r, q)) q = e4m3_codes4_div(h0, h1, s);
+    return q;
+  }
+};
+
+// Every E4M3 op encodes with CodeQuot except the unpacked 2:4 prune that also
+// writes the pruned dense copy (one code per kept element, from the table).
+template <int OP, bool DENSE>
+__host__ __device__ constexpr bool quot_encoder() {
+  return !(OP == kOpPrune24 && DENSE);
+}
 
 // The table: signed zeros everywhere (zero_table, before phase 1), then the
 // 24 binades below amax (fill_table), each entry as the definition states,
@@ -280,9 +308,7 @@ __device__ __forceinline__ uint32_t prune24_codes(const uint4 v, uint32_t mb, co
                                                   const Code &code) {
   const uint32_t p0 = __byte_perm(v.x, v.y, sel16[mb & 15u]);         // kept pair of group 0
   const uint32_t p1 = __byte_perm(v.z, v.w, sel16[(mb >> 4) & 15u]);  // and of group 1
-  const uint32_t c0 = code(p0 & 0xFFFFu), c1 = code(p0 >> 16);
-  const uint32_t c2 = code(p1 & 0xFFFFu), c3 = code(p1 >> 16);
-  return c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
+  return code.codes4(p0, p1);
 }
 
 // Byte offset, in its packed block, of the 4 value bytes of unit u (row
@@ -442,7 +468,9 @@ __device__ __forceinline__ void phase2_unit(const uint8_t *p, const Chunk &ch, u
     const uint4 v0 = reinterpret_cast<const uint4 *>(p)[0];
     const uint4 v1 = reinterpret_cast<const uint4 *>(p)[1];
     const uint32_t m3 = meta_in;
-    uint32_t c[12];
+    // wp[3 gl + j] = the two kept values of window j of 8-group gl (low half
+    // first): the unit's 12 codes in output order, encoded four at a time
+    uint32_t wp[6];
 #pragma unroll
     for (int gl = 0; gl < 2; ++gl) {
       uint32_t h[8];
@@ -457,21 +485,20 @@ __device__ __forceinline__ void phase2_unit(const uint8_t *p, const Chunk &ch, u
           if (p0 == static_cast<uint32_t>(t)) h0 = h[t];
           if (p1 == static_cast<uint32_t>(t)) h1 = h[t];
         }
-        c[6 * gl + 2 * j] = code(h0);
-        c[6 * gl + 2 * j + 1] = code(h1);
+        wp[3 * gl + j] = h0 | (h1 << 16);
       }
     }
+    uint32_t c[3];
+#pragma unroll
+    for (int o = 0; o < 3; ++o) c[o] = code.codes4(wp[2 * o], wp[2 * o + 1]);
     if constexpr (OP == kOpSlide68Packed) {
       const Slide68Place pl = slide68_place(a, ch, u);
 #pragma unroll
-      for (int o = 0; o < 3; ++o)
-        *slide68_value_at(pl, 12 * pl.j + 4 * o) =
-            c[4 * o] | (c[4 * o + 1] << 8) | (c[4 * o + 2] << 16) | (c[4 * o + 3] << 24);
+      for (int o = 0; o < 3; ++o) *slide68_value_at(pl, 12 * pl.j + 4 * o) = c[o];
     } else {
       uint32_t *d = reinterpret_cast<uint32_t *>(a.out + 12 * (ch.e >> 4) + 12 * u);
 #pragma unroll
-      for (int o = 0; o < 3; ++o)
-        d[o] = c[4 * o] | (c[4 * o + 1] << 8) | (c[4 * o + 2] << 16) | (c[4 * o + 3] << 24);
+      for (int o = 0; o < 3; ++o) d[o] = c[o];
     }
   } else {
     const uint4 v = *reinterpret_cast<const uint4 *>(p);
@@ -487,21 +514,15 @@ __device__ __forceinline__ void phase2_unit(const uint8_t *p, const Chunk &ch, u
       *reinterpret_cast<uint2 *>(a.dense + ch.e + 8 * u) = dn;
       a.meta[(ch.e >> 3) + u] = static_cast<uint8_t>(mb);
     } else {
-      uint32_t h[8];
-      halves(v, h);
+      const uint32_t c03 = code.codes4(v.x, v.y), c47 = code.codes4(v.z, v.w);
       if constexpr (OP == kOpQuantize) {
-        *reinterpret_cast<uint2 *>(a.out + ch.e + 8 * u) =
-            make_uint2(code(h[0]) | (code(h[1]) << 8) | (code(h[2]) << 16) | (code(h[3]) << 24),
-                       code(h[4]) | (code(h[5]) << 8) | (code(h[6]) << 16) | (code(h[7]) << 24));
+        *reinterpret_cast<uint2 *>(a.out + ch.e + 8 * u) = make_uint2(c03, c47);
       } else if constexpr (OP == kOpLift) {
         // lifted[12 g + 4 j + r] = code(x[8 g + 2 j + r]) for the 8-group g
-        uint32_t c[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) c[t] = code(h[t]);
         uint32_t *d = reinterpret_cast<uint32_t *>(a.out + 12 * (ch.e >> 3) + 12 * u);
-        d[0] = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-        d[1] = c[2] | (c[3] << 8) | (c[4] << 16) | (c[5] << 24);
-        d[2] = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+        d[0] = c03;
+        d[1] = __byte_perm(c03, c47, 0x5432);  // codes 2..5
+        d[2] = c47;
       }
     }
   }
@@ -607,8 +628,9 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
   };
 
   // The table costs about as much as dividing 2 chunks' elements directly.
+  constexpr bool kQuot = quot_encoder<OP, DENSE>();
   const bool direct = SMALL || n_my <= 2;
-  if constexpr (FP8 && !SMALL) {
+  if constexpr (FP8 && !SMALL && !kQuot) {
     if (!direct) zero_table(tab, tid);  // ordered before its entries by the barriers below
   }
 
@@ -665,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     named_bar_sync(1, kConsumers);
     const uint32_t amax = s_amax;
     const float s = amax == 0u ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax), 448.0f);
-    if constexpr (!SMALL) {
+    if constexpr (!SMALL && !kQuot) {
       if (!direct) fill_table(tab, amax, s, tid);
     }
     named_bar_sync(1, kConsumers);
@@ -737,7 +759,9 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
         if (!resident && (tid & 31) == 0) mbar_arrive(&empty[slot]);
       }
     };
-    if constexpr (SMALL) {
+    if constexpr (kQuot) {
+      phase2(CodeQuot{s, __frcp_rn(s)});
+    } else if constexpr (SMALL) {
       phase2(CodeTable<true>{tab, s});
     } else {
       if (direct)

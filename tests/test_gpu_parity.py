@@ -96,6 +96,22 @@ def test_quantize_bit_exact(shape, seed):
     assert int(st.item()) == 0
 
 
+@pytest.mark.parametrize("shape", [(2, 131072), (1, 262160), (1, 261968)])
+def test_quantize_size_threshold(shape):
+    """262144 values (the largest X of the one-cluster quantiser), 16 more
+    (the streamed two-phase kernel), and 32746 vectors, which the 8 CTAs
+    split unevenly."""
+    x = WL.random_bits(shape, 77 + shape[0], scale=3.0)
+    st = new_status()
+    q, s = sp().fp8_quantize_pertensor(dev_bf16(x), status=st)
+    ref_q, ref_s = O.quantize_pertensor(x)
+    assert host(s)[0] == ref_s and np.array_equal(host(q), ref_q)
+    assert int(st.item()) == 0
+    q, s = sp().slide68_lift(dev_bf16(x))
+    ref_q, ref_s = O.slide68_lift(x)
+    assert host(s)[0] == ref_s and np.array_equal(host(q), ref_q)
+
+
 @pytest.mark.parametrize("m", [1, 8, 32, 64])
 def test_quantize_decode_workload(m):
     x = WL.activation_bits(2, m)
@@ -555,9 +571,9 @@ def _fused_check(x, wts, n, what, lift=False, check_y=True):
         assert_gemm_close(y, y_ref, b, what)
 
 
-# M*K/8 at most 1024: every CTA quantises all of X (codes staged in shared
-# memory when they fit 8 KB and the tile is 16 tokens); above: amax and
-# codes grid-wide
+# M*K at most 8192: one launch, every CTA quantises all of X (codes staged
+# in shared memory when they fit 8 KB and the tile is 16 tokens); above, the
+# one-cluster quantiser (M*K <= 262144) or the streamed one, then the GEMM
 @pytest.mark.parametrize("m,n,k", [(1, 128, 128), (2, 256, 4096), (7, 256, 384), (16, 256, 256), (20, 256, 1024),
                                    (33, 384, 1024), (64, 128, 640), (100, 256, 512), (256, 384, 1152)])
 def test_quantize_gemm_packed_small(m, n, k):
@@ -666,10 +682,9 @@ def test_quantize_gemm_packed_reuses_its_workspace():
 
 
 def test_quantize_gemm_packed_back_to_back_grid_calls():
-    """Grid-wide fused calls queued back to back on one workspace, each X with
-    its own scale: a counter or flag left set by one call would let the next
-    read its codes before they are written (Y would then differ from the
-    two-launch GEMM on the same codes)."""
+    """Fused calls above the one-launch size queued back to back on one
+    workspace, each X with its own scale: a GEMM that read codes before its
+    quantiser wrote them would differ from the GEMM on the same codes."""
     ws = sp().Workspace(DEV)
     w = WL.random_bits((384, 1024), 1800, scale=0.02)
     packed, sw = sp().sp24_prune_compress_packed(dev_bf16(w))
@@ -683,6 +698,32 @@ def test_quantize_gemm_packed_back_to_back_grid_calls():
     for i in (0, 23):
         ref_q, ref_s = O.quantize_pertensor(host(xs[i]))
         assert host(outs[i][2])[0] == ref_s and np.array_equal(host(outs[i][1]), ref_q), f"call {i}"
+
+
+def test_quantize_gemm_packed_back_to_back_cluster_calls():
+    """The same through the one-cluster quantiser and a 16-CTA GEMM that
+    launches behind it (programmatic launch): each call's codes and scale
+    must equal the oracle's and Y the GEMM on them."""
+    ws = sp().Workspace(DEV)
+    w = WL.random_bits((1024, 1024), 1810, scale=0.02)
+    packed, sw = sp().sp24_prune_compress_packed(dev_bf16(w))
+    xs = [dev_bf16(WL.random_bits((40 + 24 * (i % 2), 1024), 1950 + i, scale=0.5 + i)) for i in range(16)]
+    outs = [sp().sp24_quantize_gemm_packed(x, packed, sw, 1024, workspace=ws) for x in xs]
+    refs = [sp().sp24_gemm_packed(xq, sx, packed, sw, 1024, workspace=ws) for (_, xq, sx) in outs]
+    torch.cuda.synchronize()
+    assert (ws.buf[:8192] == 0).all()
+    for i, ((y, xq, sx), y2) in enumerate(zip(outs, refs)):
+        assert torch.equal(y, y2), f"call {i}"
+        ref_q, ref_s = O.quantize_pertensor(host(xs[i]))
+        assert host(sx)[0] == ref_s and np.array_equal(host(xq), ref_q), f"call {i}"
+
+
+def test_lift_gemm_packed_cluster_form():
+    """Lift + GEMM through the one-cluster lift (M32 K1024 -> K' 1536,
+    N 512)."""
+    x = WL.random_bits((32, 1024), 1240)
+    w = WL.random_bits((512, 1024), 1340, scale=0.02)
+    _fused_check(x, _fused_weights(w, True), 512, "fused lift cluster 32x512x1024", lift=True)
 
 
 # ------------------------------------------------------------ per-token / per-channel scales

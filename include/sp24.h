@@ -125,7 +125,7 @@ int sp24_prune_compress(const void *W, int N, int K, int out_dtype, void *values
  * X: bf16 [rows, cols] -> q: u8 [rows, cols], scale <- amax|X| / 448 (1.0 when
  * amax = 0), q = E4M3(x / scale) as above.  Also used for the weights of the
  * dense FP8 comparison GEMM.  Shape rules: rows >= 1, cols >= 1, cols % 16 == 0.
- * A decode-sized X (rows * cols <= 262144) is done by one thread-block
+ * A decode-sized X (rows * cols <= 131072) is done by one thread-block
  * cluster that leaves the workspace untouched and lets the next kernel on
  * `stream` launch at once (it must wait for this one before reading q or
  * scale, as every kernel of this library does).
@@ -153,7 +153,7 @@ int slide68_decompose(const void *W, int N, int K, int out_dtype, void *values, 
  * Activation lift fused with per-tensor E4M3 quantisation (SlideSparse, §2
  * "Levantamiento de Activacion").  X: bf16 [M, K] -> q_lifted: u8 [M, 3K/2]
  * with q_lifted[m, 12g + 4j + r] = E4M3(X[m, 8g + 2j + r] / scale), scale <-
- * amax|X| / 448.  Shape rules: M >= 1, K % 16 == 0.  M * K <= 262144: one
+ * amax|X| / 448.  Shape rules: M >= 1, K % 16 == 0.  M * K <= 131072: one
  * thread-block cluster, as for fp8_quantize_pertensor.
  */
 int slide68_lift(const void *X, int M, int K, uint8_t *q_lifted, float *scale, void *workspace,
@@ -246,7 +246,7 @@ int sp24_gemm_packed(const void *Xq, const float *x_scale, const void *packed,
  * 8192 it is ONE launch: every CTA of the GEMM quantises all of X itself and
  * starts its tensor-core work on the codes while the packed weights already
  * stream in.  Otherwise the quantiser runs first (one thread-block cluster up
- * to M * K = 262144) and the GEMM, launched right behind it, streams its
+ * to M * K = 131072) and the GEMM, launched right behind it, streams its
  * weights while it runs.  Workspace:
  * sp24_workspace_size(SP24_OP_QUANTIZE_GEMM_PACKED, M, N, K, 0) (its first
  * 8 KB hold the quantiser's counters, zero before the first use and after

@@ -78,7 +78,7 @@ constexpr size_t kFusedCounterBytes = 8192;
 // ---- smallx.cu: decode-sized activations (at most kSmallXVec 8-element
 // vectors, nelem % 8 == 0) quantised, or lifted (rows of 16k elements), by
 // one thread-block cluster; no workspace.
-constexpr int64_t kSmallXVec = 32768;
+constexpr int64_t kSmallXVec = 16384;
 bool small_quantize_fits(int64_t nelem);
 cudaError_t launch_quantize_small(const void *x, int64_t nelem, bool lift, float *scale, uint8_t *q,
                                   int32_t *status, cudaStream_t st);

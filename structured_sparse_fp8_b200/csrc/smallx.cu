@@ -4,7 +4,7 @@
 // The quantiser of the cookbook's FP8 recipe ("Practical Example 2": one
 // scale amax / 448 for the whole tensor, codes E4M3(x / scale)) needs the
 // amax of all of X before the first code.  For a decode batch (X of at most
-// kSmallXVec 16-byte vectors, 512 KB of bf16) a grid-wide two-phase kernel is
+// kSmallXVec 16-byte vectors, 256 KB of bf16) a grid-wide two-phase kernel is
 // all latency: its grid barrier alone costs microseconds while HBM streams
 // the GEMM's weights.  Here a single cluster of kSmallCtas CTAs does it with
 // no global synchronisation at all:
@@ -19,9 +19,11 @@
 //  4. encodes its registers with the division-free encoder (e4m3_codes8_fast,
 //     exact; the vectors it cannot decide go through the correctly rounded
 //     division) and stores 8 codes (or the 12 lifted codes) per vector.
-// The kernel releases its dependents at entry: the GEMM that consumes the
-// codes launches at once and streams its weights while this cluster runs
-// (it waits for this grid's completion before reading codes or scale).
+// The kernel releases its dependents as soon as the previous kernel has
+// completed: the GEMM that consumes the codes then launches and streams its
+// weights while this cluster runs (it waits for this grid's completion
+// before reading codes or scale).  Released at entry instead, that GEMM
+// competed with the kernel before this one and the chain was slower.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -36,7 +38,7 @@ namespace {
 
 constexpr int kSmallCtas = 8;    // one portable-size cluster
 constexpr int kSmallThreads = 256;
-constexpr int kSmallRegs = 16;   // 16-byte X vectors per thread
+constexpr int kSmallRegs = 8;    // 16-byte X vectors per thread
 
 template <bool LIFT>
 __global__ void __launch_bounds__(kSmallThreads)
@@ -53,8 +55,8 @@ __global__ void __launch_bounds__(kSmallThreads)
     fence_mbar_init();
   }
   cluster_sync_all();  // every CTA's barrier is initialised before any remote arrive
-  grid_launch_dependents();
   grid_dependency_wait();  // X may come from the previous kernel
+  grid_launch_dependents();
 
   const int64_t v0 = static_cast<int64_t>(rank) * nvec / kSmallCtas;
   const int64_t v1 = static_cast<int64_t>(rank + 1) * nvec / kSmallCtas;

@@ -96,10 +96,10 @@ def test_quantize_bit_exact(shape, seed):
     assert int(st.item()) == 0
 
 
-@pytest.mark.parametrize("shape", [(2, 131072), (1, 262160), (1, 261968)])
+@pytest.mark.parametrize("shape", [(2, 65536), (1, 131088), (1, 130960)])
 def test_quantize_size_threshold(shape):
-    """262144 values (the largest X of the one-cluster quantiser), 16 more
-    (the streamed two-phase kernel), and 32746 vectors, which the 8 CTAs
+    """131072 values (the largest X of the one-cluster quantiser), 16 more
+    (the streamed two-phase kernel), and 16370 vectors, which the 8 CTAs
     split unevenly."""
     x = WL.random_bits(shape, 77 + shape[0], scale=3.0)
     st = new_status()
@@ -573,7 +573,7 @@ def _fused_check(x, wts, n, what, lift=False, check_y=True):
 
 # M*K at most 8192: one launch, every CTA quantises all of X (codes staged
 # in shared memory when they fit 8 KB and the tile is 16 tokens); above, the
-# one-cluster quantiser (M*K <= 262144) or the streamed one, then the GEMM
+# one-cluster quantiser (M*K <= 131072) or the streamed one, then the GEMM
 @pytest.mark.parametrize("m,n,k", [(1, 128, 128), (2, 256, 4096), (7, 256, 384), (16, 256, 256), (20, 256, 1024),
                                    (33, 384, 1024), (64, 128, 640), (100, 256, 512), (256, 384, 1152)])
 def test_quantize_gemm_packed_small(m, n, k):

@@ -902,7 +902,7 @@ def prefill_headline(device, peaks, reps=20):
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
                          "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "kernel": "sp24_gemm_packed",
                          "peak_source": f"{peaks['source']} bf16 burst x4 (2:4 sparse FP8 dense-equivalent)",
-                         "traffic": None},
+                         "traffic": load_traffic().get("prefill:sp24_gemm_packed")},
             "dense_tflops": round(flops / t_dn / 1e6, 1),
             "timing": f"CUDA graph of {reps} launches over {len(ps)} rotating packed weight copies "
                       f"({len(pd)} dense), inputs larger than L2"}
@@ -930,7 +930,10 @@ def kernel_case(name, device):
     def w_decode():
         return bf(WL.weight_bits(2))
 
-    if name == "quantize":                       # X[4096, 4096] per-tensor E4M3
+    if name == "quantize_small":                 # X[32, 4096] per-tensor E4M3, one thread-block cluster
+        x = bf(WL.activation_bits(2, 32))
+        call = lambda: sp.fp8_quantize_pertensor(x, workspace=ws)
+    elif name == "quantize":                     # X[4096, 4096] per-tensor E4M3
         x = bf(WL.activation_bits(3, 4096))
         call = lambda: sp.fp8_quantize_pertensor(x, workspace=ws)
     elif name == "lift":                         # X[2048, 4096] 6:8 lift + quantise
@@ -943,7 +946,7 @@ def kernel_case(name, device):
         w = bf(WL.weight_bits(5))
         call = lambda: sp.slide68_decompose_packed(w, workspace=ws)
     elif name in ("gemm_packed_decode", "gemm_dense_decode", "gemm_int8_decode", "fused_decode"):
-        m = 64
+        m = 1 if name == "fused_decode" else 64  # the fused call is one launch up to M*K = 8192
         w = w_decode()
         x = bf(WL.activation_bits(2, m))
         if name == "gemm_dense_decode":

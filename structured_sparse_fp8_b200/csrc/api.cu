@@ -103,9 +103,10 @@ size_t sp24_workspace_size(int op, int64_t M, int64_t N, int64_t K, int dtype) {
       int sms = device_sm_count();
       if (sms <= 0) sms = 148;
       const sp24::GemmKind kind =
-          op == SP24_OP_GEMM_DENSE    ? sp24::kDenseE4M3
-          : op == SP24_OP_GEMM_PACKED ? sp24::kSparseE4M3Packed
-                                      : (dtype == SP24_DTYPE_BF16 ? sp24::kSparseBF16 : sp24::kSparseE4M3);
+          op == SP24_OP_GEMM_DENSE ? sp24::kDenseE4M3
+          : op == SP24_OP_GEMM_PACKED
+              ? sp24::packed_kind(static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sms)
+              : (dtype == SP24_DTYPE_BF16 ? sp24::kSparseBF16 : sp24::kSparseE4M3);
       return sp24::plan_gemm(kind, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sms)
           .workspace_bytes();
     }
@@ -264,6 +265,7 @@ static int gemm_common(sp24::GemmKind kind, const void *Xq, const float *x_scale
     return SP24_ERR_ALIGN;
   const int sms = device_sm_count();
   if (sms < 0) return SP24_ERR_ARCH;
+  if (kind == sp24::kSparseE4M3Packed) kind = sp24::packed_kind(M, N, K, sms);
   const sp24::GemmPlan pl = sp24::plan_gemm(kind, M, N, K, sms);
   if (pl.workspace_bytes() > 0) {
     if (!workspace || ws_bytes < pl.workspace_bytes()) return SP24_ERR_WORKSPACE;

@@ -62,6 +62,7 @@ struct KindTraits<kSparseE4M3> {
   static constexpr int kMetaColsPerMma = 2;  // 64 metadata bits per row per MMA
   static constexpr bool kPacked = false;
   static constexpr bool kFp4 = false;
+  static constexpr bool kPair = false;
 };
 
 // The same MMA with the weights in the tile-packed layout: each stage's
@@ -79,6 +80,21 @@ template <>
 struct KindTraits<kSparseI8Packed> : KindTraits<kSparseE4M3Packed> {
   static constexpr uint32_t kFmt = 1;   // signed 8-bit
   static constexpr uint32_t kDFmt = 2;  // s32 accumulator
+};
+
+// The packed E4M3 kind on SM pairs (tensor-bound tiles): a cluster of two
+// CTAs runs one M = 256 sparse MMA per K step (cta_group::2).  Each CTA
+// loads the packed blocks of its own 128 weight rows (through a 2-D tensor
+// map over the packed buffer: a 10240-byte block is 40 rows of 256 bytes)
+// and half of the activation tile, both counted on the even CTA's barrier;
+// the even CTA issues the metadata copies, MMAs and commits for both, and
+// each CTA drains the accumulator of its own rows.  Against one CTA holding
+// two row tiles the shared-memory bytes per MMA are the same, but each
+// CTA's accumulator is BN columns, so two fit tensor memory and a tile's
+// epilogue overlaps the next tile's main loop.
+template <>
+struct KindTraits<kSparseE4M3Pair> : KindTraits<kSparseE4M3Packed> {
+  static constexpr bool kPair = true;
 };
 
 // 2:4 sparse FP4 (E2M1 A and B, kind::f8f6f4): the codes are packed two per
@@ -119,6 +135,7 @@ struct KindTraits<kDenseE4M3> {
   static constexpr int kMetaColsPerMma = 0;
   static constexpr bool kPacked = false;
   static constexpr bool kFp4 = false;
+  static constexpr bool kPair = false;
 };
 
 // 2:4 sparse BF16 (kind::f16): per stage 128 logical K = 64 bf16 values (128 B)
@@ -147,6 +164,7 @@ struct KindTraits<kSparseBF16> {
   static constexpr int kMetaColsPerMma = 1;
   static constexpr bool kPacked = false;
   static constexpr bool kFp4 = false;
+  static constexpr bool kPair = false;
 };
 
 // MT = 128-row W tiles per CTA tile (1 or 2).  With MT = 2 each stage
@@ -173,7 +191,10 @@ struct Config {
   static_assert(!T::kFp4 || (KB == 2 && MT == 1), "FP4 stages are two 128-K blocks of one row tile");
   static constexpr int kRows = 128 * MT;
   static constexpr uint32_t kABytes = kRows * T::kARowBytes * KB;
-  static constexpr uint32_t kBBytes = BN * T::kBRowBytes * KB;
+  static_assert(!T::kPair || (MT == 1 && XQ == 0 && BN >= 128 && BN % 32 == 0),
+                "SM pairs run one-row-tile stages of wide token tiles");
+  static constexpr int kBRows = T::kPair ? BN / 2 : BN;  // activation rows this CTA loads
+  static constexpr uint32_t kBBytes = kBRows * T::kBRowBytes * KB;
   static constexpr uint32_t kEBytes = kRows * T::kERowBytes * KB;
   static constexpr uint32_t kTBytes = T::kMetaTransform ? 128 * 16 : 0;  // TMEM-ready metadata
   // Transaction bytes of a stage's copies: a 4-bit box moves its packed
@@ -290,15 +311,18 @@ struct Segment {
   int tile, kb0, kb1, role;
 };
 
+// `me` / `ncta`: this CTA's index and the count of schedule units (CTAs,
+// or SM pairs for the pair kind).
 struct SegIter {
   int64_t u, u_end;
-  int tile;
-  __device__ __forceinline__ void init(const GemmArgs &p) {
-    tile = blockIdx.x;
+  int tile, step;
+  __device__ __forceinline__ void init(const GemmArgs &p, int me, int ncta) {
+    tile = me;
+    step = ncta;
     u = u_end = 0;
-    if (static_cast<int>(blockIdx.x) < p.sk_grid) {
-      u = static_cast<int64_t>(blockIdx.x) * p.sk_units / p.sk_grid;
-      u_end = static_cast<int64_t>(blockIdx.x + 1) * p.sk_units / p.sk_grid;
+    if (me < p.sk_grid) {
+      u = static_cast<int64_t>(me) * p.sk_units / p.sk_grid;
+      u_end = static_cast<int64_t>(me + 1) * p.sk_units / p.sk_grid;
     }
   }
   __device__ __forceinline__ bool next(const GemmArgs &p, Segment &s) {
@@ -307,7 +331,7 @@ struct SegIter {
       s.kb0 = 0;
       s.kb1 = p.num_kb;
       s.role = kWhole;
-      tile += gridDim.x;
+      tile += step;
       return true;
     }
     if (u >= u_end) return false;
@@ -490,9 +514,18 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int tiles_m = (p.num_tiles + p.tiles_n - 1) / p.tiles_n;
+  // SM pairs: rank in the pair (0 = the CTA that issues the MMAs) and the
+  // pair's index in the schedule
+  const uint32_t rank = T::kPair ? cluster_ctarank() & 1u : 0u;
+  const int me = T::kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int ncta = T::kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  // first weight row of a tile held by this CTA
+  auto row0 = [&](int tile) {
+    return T::kPair ? (tile % p.tiles_n) * 256 + static_cast<int>(rank) * 128 : (tile % p.tiles_n) * C::kRows;
+  };
 
   if (warp == 0 && lane == 0) {
-    if (!T::kPacked) prefetch_tensormap(&tmA);
+    if (!T::kPacked || T::kPair) prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
     if (T::kSparse && !T::kPacked) prefetch_tensormap(&tmE);
     if (C::kTmaStoreY) prefetch_tensormap(&tmY);
@@ -503,17 +536,24 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
     }
     for (int b = 0; b < NB; ++b) {
       mbar_init(&tmem_full[b], 1);
-      mbar_init(&tmem_empty[b], C::kEpiThreads);
+      mbar_init(&tmem_empty[b], T::kPair ? 2 * C::kEpiThreads : C::kEpiThreads);  // pairs: both CTAs drain
     }
     mbar_init(x_ready, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
+    if constexpr (T::kPair) {
+      tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  // pairs: both CTAs' barriers exist before the first remote arrive or load
+  if constexpr (T::kPair) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // Programmatic dependent launch.  This grid may start while the previous
@@ -540,7 +580,13 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
       const uint64_t stream_w = tiles_m == 1 ? l2_policy_evict_first() : l2_policy_evict_normal();
       // weight half of a stage: values + metadata of rows n0.., k-block kb
       auto load_weights = [&](uint8_t *st, uint64_t *bar, int n0, int kb) {
-        if constexpr (T::kPacked) {
+        if constexpr (T::kPair) {
+          // this CTA's packed block (rows n0..n0+127, k-block kb): rows of
+          // 256 bytes 40 (blk) .. 40 (blk) + 39 of the packed tensor map,
+          // counted on the even CTA's barrier
+          const int blk = ((n0 / 128) * p.num_kb + kb) * KB;
+          tma_load_2d_pair(st, &tmA, mapa_shared(bar, 0u), 0, blk * (kPackedBlockBytes / 256), stream_w);
+        } else if constexpr (T::kPacked) {
 #pragma unroll
           for (int i = 0; i < MT; ++i) {
             const uint8_t *blk = p.packed +
@@ -581,24 +627,24 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
       // X copy: only the transaction bytes are announced here).  Pass 2:
       // everything else, in the same stage order.
       SegIter it;
-      it.init(p);
+      it.init(p, me, ncta);
       Segment sg;
       int i = 0;
       bool ok = true;
       int pre = 0;  // stages whose weight tiles were issued ahead
       {
         SegIter it0;
-        it0.init(p);
+        it0.init(p, me, ncta);
         Segment s0;
         while (pre < S && it0.next(p, s0)) {
-          const int n0 = (s0.tile % p.tiles_n) * C::kRows;
+          const int n0 = row0(s0.tile);
           for (int kb = s0.kb0; kb < s0.kb1 && pre < S; ++kb, ++pre) {
             uint8_t *st = smem + pre * C::kStageBytes;
             if (leader) {
               if (staged)
                 mbar_expect_tx(&full[pre], C::kWBytes);
-              else
-                mbar_arrive_expect_tx(&full[pre], C::kTmaBytes);
+              else if (!T::kPair || rank == 0)  // pairs: the even CTA expects both CTAs' bytes
+                mbar_arrive_expect_tx(&full[pre], T::kPair ? 2 * C::kTmaBytes : C::kTmaBytes);
               load_weights(st, &full[pre], n0, kb);
             }
           }
@@ -609,11 +655,11 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
       // dependency resolves, so that the CTA's whole weight share streams
       // from HBM while the previous kernel drains, and the stages after the
       // first S refill from L2.
-      if constexpr (T::kPacked && MT == 1) {
+      if constexpr (T::kPacked && MT == 1 && !T::kPair) {
         if (tiles_m == 1 && leader) {
           const uint64_t keep_w = l2_policy_evict_normal();
           SegIter it1;
-          it1.init(p);
+          it1.init(p, me, ncta);
           Segment s1;
           int st_i = 0;
           while (it1.next(p, s1)) {
@@ -636,7 +682,7 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
         if (!staged) fence_proxy_async_global();
       }
       while (ok && it.next(p, sg)) {
-        const int n0 = (sg.tile % p.tiles_n) * C::kRows;
+        const int n0 = row0(sg.tile);
         const int m0 = (sg.tile / p.tiles_n) * BN;
         for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++i) {
           const int s = i % S;
@@ -648,7 +694,8 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
               break;
             }
             if (leader && !staged) {
-              mbar_arrive_expect_tx(&full[s], C::kTmaBytes);
+              if (!T::kPair || rank == 0)
+                mbar_arrive_expect_tx(&full[s], T::kPair ? 2 * C::kTmaBytes : C::kTmaBytes);
               load_weights(st, &full[s], n0, kb);
             }
           }
@@ -663,13 +710,28 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
               }
             }
           } else if (leader) {
+            if constexpr (T::kPair) {
+              // this CTA's half of the activation tile, 128 K per box
 #pragma unroll
-            for (int sub = 0; sub < C::kBSub; ++sub)
-              tma_load_2d(st + C::kBOff + sub * BN * 128, &tmB, &full[s],
-                          kb * (T::kBRowBytes * KB / T::kBElemBytes) + sub * T::kBBoxElems, m0, keep_x);
+              for (int sub = 0; sub < C::kBSub; ++sub)
+                tma_load_2d_pair(st + C::kBOff + sub * C::kBRows * 128, &tmB, mapa_shared(&full[s], 0u),
+                                 kb * (T::kBRowBytes * KB / T::kBElemBytes) + sub * T::kBBoxElems,
+                                 m0 + static_cast<int>(rank) * C::kBRows, keep_x);
+            } else {
+#pragma unroll
+              for (int sub = 0; sub < C::kBSub; ++sub)
+                tma_load_2d(st + C::kBOff + sub * BN * 128, &tmB, &full[s],
+                            kb * (T::kBRowBytes * KB / T::kBElemBytes) + sub * T::kBBoxElems, m0, keep_x);
+            }
           }
           __syncwarp();
         }
+      }
+      if constexpr (T::kPair) {
+        // the even CTA's commits release this CTA's slots: wait for the last
+        // ones, so that none lands after this CTA has left
+        for (int k = i > S ? i - S : 0; ok && k < i; ++k)
+          if (!mbar_wait_warp(&empty[k % S], static_cast<uint32_t>(k / S) & 1u, p.status)) break;
       }
     }
     __syncwarp();
@@ -677,14 +739,14 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
     // ------------------------------------------------------ MMA issuer
     {
       const bool leader = elect_one();
-      constexpr uint32_t idesc = mma_idesc(128, BN, T::kFmt, T::kSparse, T::kDFmt);
+      constexpr uint32_t idesc = mma_idesc(T::kPair ? 256 : 128, BN, T::kFmt, T::kSparse, T::kDFmt);
       // metadata of row tile i: 4 TMEM columns after all accumulators
       const uint32_t e_tmem = tmem_base + NB * C::kAccCols;
       SegIter it;
-      it.init(p);
+      it.init(p, me, ncta);
       Segment sg;
       int i = 0, j = 0;
-      bool ok = true;
+      bool ok = !T::kPair || rank == 0;  // pairs: the even CTA issues for both
       while (ok && it.next(p, sg)) {
         const int b = j % NB;
         const int r = j / NB;
@@ -708,6 +770,14 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
               if constexpr (T::kFp4) {
                 // the two blocks' metadata boxes, 2048 bytes apart
                 tmem_copy_128x256b(e_tmem, smem_desc(st_addr + C::kEOff, 128 * T::kERowBytes, 128, kSwizzleNone));
+              } else if constexpr (T::kPair) {
+                // each CTA's block metadata into its own tensor memory (two
+                // blocks: the second 16-byte column is the next block's, 10240
+                // bytes on)
+                if constexpr (KB == 2)
+                  tmem_copy_128x256b_pair(e_tmem, smem_desc(st_addr + C::e_off(0), kPackedBlockBytes, 128, kSwizzleNone));
+                else
+                  tmem_copy_128x128b_pair(e_tmem, smem_desc(st_addr + C::e_off(0), 2048, 128, kSwizzleNone));
               } else if constexpr (T::kPacked && MT * KB == 2) {
                 // two packed blocks' metadata in one copy (both row tiles, or
                 // both k-blocks of one row tile): the second 16-byte column is
@@ -731,11 +801,13 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
                 const uint32_t a_k = (KB == 1 || T::kFp4) ? kk * T::kAStep
                                                           : (kk / T::kMmas) * kPackedBlockBytes + (kk % T::kMmas) * T::kAStep;
                 const uint64_t ad = smem_desc(a_addr + a_k, 16, T::kASbo, T::kASwizzle);
-                const uint32_t boff = (kk * T::kBStep / 128) * (BN * 128) + (kk * T::kBStep) % 128;
+                const uint32_t boff = (kk * T::kBStep / 128) * (C::kBRows * 128) + (kk * T::kBStep) % 128;
                 const uint64_t bd = smem_desc(b_addr + boff, 16, 8 * 128, kSwizzle128B);
                 const uint32_t acc = (kb > sg.kb0 || kk > 0) ? 1u : 0u;
                 const uint32_t d = d_tmem + rt * BN;
-                if constexpr (KIND == kSparseE4M3 || KIND == kSparseE4M3Packed || KIND == kSparseFP4) {
+                if constexpr (T::kPair) {
+                  mma_f8_sparse_pair(d, ad, bd, idesc, e_tmem + 2 * kk, acc);
+                } else if constexpr (KIND == kSparseE4M3 || KIND == kSparseE4M3Packed || KIND == kSparseFP4) {
                   mma_f8_sparse(d, ad, bd, idesc, e_tmem + 4 * rt + 2 * kk, acc);
                 } else if constexpr (KIND == kSparseI8Packed) {
                   mma_i8_sparse(d, ad, bd, idesc, e_tmem + 4 * rt + 2 * kk, acc);
@@ -748,11 +820,19 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
                 }
               }
             }
-            mma_commit(&empty[s]);
+            if constexpr (T::kPair)
+              mma_commit_pair(&empty[s], 3);  // both CTAs' slot
+            else
+              mma_commit(&empty[s]);
           }
           __syncwarp();
         }
-        if (leader) mma_commit(&tmem_full[b]);
+        if (leader) {
+          if constexpr (T::kPair)
+            mma_commit_pair(&tmem_full[b], 3);
+          else
+            mma_commit(&tmem_full[b]);
+        }
         __syncwarp();
         ++j;
       }
@@ -775,8 +855,15 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
     const float sc = sx * sw;
     constexpr int kW = C::kEpiCols;
     [[maybe_unused]] uint32_t ypass = 0;  // staged Y passes issued so far
+    // accumulator b drained (pairs: the even CTA's MMA warp waits for both)
+    auto release_acc = [&](int b) {
+      if (T::kPair && rank != 0)
+        mbar_arrive_cluster(mapa_shared(&tmem_empty[b], 0u));
+      else
+        mbar_arrive(&tmem_empty[b]);
+    };
     SegIter it;
-    it.init(p);
+    it.init(p, me, ncta);
     Segment sg;
     int i = 0, j = 0;
     while (it.next(p, sg)) {
@@ -808,10 +895,15 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
       // fp32 partial tile of CTA g, row tile rt, in quads of 4 token columns
       // laid out [column quad][row][4], so that a warp's 32 rows of one quad
       // are 512 contiguous bytes: quad cq of this thread's row.
+      // (g: schedule index; pairs keep one partial per CTA, 2 g + rank)
       auto part4 = [&](int g, int rt, int cq) {
+        const int slot = T::kPair ? 2 * g + static_cast<int>(rank) : g;
         return reinterpret_cast<float4 *>(p.partials) +
-               ((static_cast<size_t>(g) * MT + rt) * (BN / 4) + cq) * 128 + row;
+               ((static_cast<size_t>(slot) * MT + rt) * (BN / 4) + cq) * 128 + row;
       };
+      // the split tile's counter (pairs: one per CTA of the pair, counting
+      // the contributors' CTAs of the same rank)
+      const int ci = (sg.tile - p.dp_tiles) * (T::kPair ? 2 : 1) + static_cast<int>(rank);
       // Owner of a split tile: its contributors (the next CTAs) compute this
       // tile's later k-blocks as the first segment of their range, so they
       // are normally done before this CTA's own k-blocks are.  Wait for them
@@ -825,20 +917,20 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
       float4 nxt[8];             // the next pass's first-contributor partial
       if (sg.role == kOwner) {
         const int64_t u_first = static_cast<int64_t>(sg.tile - p.dp_tiles) * p.num_kb;
-        first = static_cast<int>(blockIdx.x) + 1;
+        first = me + 1;
         last = cta_of_unit(u_first + p.num_kb - 1, p.sk_units, p.sk_grid);
         if (t == 0) {
           const uint32_t expect = static_cast<uint32_t>(last - first + 1);
           const uint64_t t0 = global_timer_ns();
           uint32_t polls = 0;
-          while (ld_acquire_gpu(&p.counters[sg.tile - p.dp_tiles]) < expect) {
+          while (ld_acquire_gpu(&p.counters[ci]) < expect) {
             __nanosleep(20);
             if ((++polls & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
               if (p.status) atomicOr(p.status, SP24_STATUS_TIMEOUT);
               break;
             }
           }
-          p.counters[sg.tile - p.dp_tiles] = 0u;  // leave the workspace counters at zero
+          p.counters[ci] = 0u;  // leave the workspace counters at zero
         }
         named_bar_sync(1, C::kEpiThreads);  // the acquire by thread 0 covers the whole CTA's reads
         if constexpr (!C::kTmaStoreY) {
@@ -848,7 +940,7 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
       }
       mbar_wait(&tmem_full[b], static_cast<uint32_t>(r) & 1u, p.status);
       tc_fence_after();
-      const int n0 = (sg.tile % p.tiles_n) * C::kRows;
+      const int n0 = row0(sg.tile);
       const int m0 = (sg.tile / p.tiles_n) * BN;
       const int mvalid = min(BN, p.M - m0);
       // lane quarter of this warp, accumulator b; row tile rt at + rt * BN
@@ -866,17 +958,17 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
             tmem_regs_ready(v);
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4)
-              __stcg(part4(blockIdx.x, rt, c / 4 + k4),
+              __stcg(part4(me, rt, c / 4 + k4),
                      make_float4(acc_f32<KIND>(v[4 * k4]), acc_f32<KIND>(v[4 * k4 + 1]),
                                  acc_f32<KIND>(v[4 * k4 + 2]), acc_f32<KIND>(v[4 * k4 + 3])));
           }
         }
         tc_fence_before();
-        mbar_arrive(&tmem_empty[b]);
+        release_acc(b);
         // The barrier orders every thread's partial stores before thread 0's
         // release increment (release is cumulative), which the owner acquires.
         named_bar_sync(1, C::kEpiThreads);
-        if (t == 0) red_release_add_gpu(&p.counters[sg.tile - p.dp_tiles], 1u);
+        if (t == 0) red_release_add_gpu(&p.counters[ci], 1u);
       } else {
 #pragma unroll 1
         for (int rt = rt0; rt < rt0 + C::kRtPerWarp; ++rt) {
@@ -1010,7 +1102,7 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
           }
         }
         tc_fence_before();
-        mbar_arrive(&tmem_empty[b]);
+        release_acc(b);
       }
       ++j;
     }
@@ -1021,9 +1113,15 @@ __global__ void __launch_bounds__(Config<KIND, BN, MT, KB, XQ>::kThreads, Config
 
   tc_fence_before();
   __syncthreads();
+  // pairs: no CTA frees its tensor memory or leaves while the other may still
+  // use it, arrive on its barriers or load into its shared memory
+  if constexpr (T::kPair) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    if constexpr (T::kPair)
+      tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else
+      tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
@@ -1076,21 +1174,56 @@ static int choose_bn(GemmKind kind, int M) {
   return pad224 * 10 <= static_cast<long>(M) * 11 ? 224 : 256;
 }
 
+// Clusters of two CTAs of the SM-pair GEMM that the device runs at once (0
+// when it cannot run them: no device, or no room for a pair).
+static int pair_capacity() {
+  static int cap = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    using C = Config<kSparseE4M3Pair, 224, 1, 1, 0>;
+    const auto kern = gemm_kernel<kSparseE4M3Pair, 224, 1, 0, 1, false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return;
+    }
+    cudaLaunchConfig_t qc = {};
+    qc.gridDim = dim3(2, 1, 1);
+    qc.blockDim = dim3(C::kThreads, 1, 1);
+    qc.dynamicSmemBytes = C::kSmemBytes;
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = 2;
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    qc.attrs = qa;
+    qc.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &qc) == cudaSuccess)
+      cap = n;
+    else
+      (void)cudaGetLastError();
+  });
+  return cap;
+}
+
 GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   GemmPlan pl{};
+  const bool pair = kind == kSparseE4M3Pair;
   pl.bn = choose_bn(kind, M);
   // Large token tiles (224 tokens: many tiles, bound by operand ingest) pair
   // two 128-row W tiles on one activation tile when N allows it.
   pl.mt = (pl.bn == 224 && kind != kSparseBF16 && N % 256 == 0) ? 2 : 1;
   // Decode-sized tiles over packed weights take two 128-K blocks per stage;
   // FP4 always does (one 4-bit box spans two blocks) and uses one row tile.
-  if (kind == kSparseFP4) pl.mt = 1;
-  pl.kb = (kind == kSparseFP4 ||
+  // SM pairs: each CTA one row tile of a 256-row tile, scheduled by pair.
+  if (kind == kSparseFP4 || pair) pl.mt = 1;
+  if (pair) sm_count = min(sm_count / 2, pair_capacity());
+  pl.kb = (kind == kSparseFP4 || (pair && K % 256 == 0) ||
            ((kind == kSparseE4M3Packed || kind == kSparseI8Packed) && pl.bn <= 64 && pl.mt == 1 && K % 256 == 0))
               ? 2
               : 1;
   pl.bk = 128 * pl.kb;
-  pl.tiles_n = N / (128 * pl.mt);
+  pl.tiles_n = N / (pair ? 256 : 128 * pl.mt);
   pl.tiles_m = (M + pl.bn - 1) / pl.bn;
   pl.num_kb = K / pl.bk;
   pl.num_tiles = pl.tiles_n * pl.tiles_m;
@@ -1119,7 +1252,16 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
   pl.counter_bytes = pl.stream_k ? kGemmCounterBytes : 0;
   pl.partial_bytes =
       pl.stream_k ? static_cast<size_t>(pl.sk_grid) * 128 * pl.mt * pl.bn * sizeof(float) : 0;
+  if (pair) {  // the schedule counted pairs; launch and partials count CTAs
+    pl.grid *= 2;
+    pl.partial_bytes *= 2;
+  }
   return pl;
+}
+
+GemmKind packed_kind(int M, int N, int K, int sm_count) {
+  const GemmPlan pl = plan_gemm(kSparseE4M3Packed, M, N, K, sm_count);
+  return (pl.mt == 2 && pl.bn == 224 && pair_capacity() >= 2) ? kSparseE4M3Pair : kSparseE4M3Packed;
 }
 
 template <int KIND, int BN, int MT, int XQ = 0, int KB = 1, bool VS = false>
@@ -1149,7 +1291,13 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   const uint64_t a_row = T::kSparse ? static_cast<uint64_t>(K) / 2 : static_cast<uint64_t>(K);
   const CUtensorMapSwizzle a_sw =
       T::kASwizzle == kSwizzle64B ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-  if (T::kPacked) {
+  if (T::kPair) {
+    // the packed buffer as rows of 256 bytes: a 10240-byte block is 40 rows
+    const uint64_t packed_bytes = static_cast<uint64_t>(N) * K / 2 + static_cast<uint64_t>(N) * K / 8;
+    if (!make_tensor_map_2d(&tmA, w_values, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, packed_bytes / 256, 256,
+                            KB * kPackedBlockBytes / 256, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  } else if (T::kPacked) {
     tmA = {};
   } else if (T::kFp4) {
     // the stored codes of 128 rows x 256 K: one 128-element 4-bit box
@@ -1159,7 +1307,7 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
                                  T::kARowBytes / T::kAElemBytes, C::kRows, a_sw)) {
     return cudaErrorInvalidValue;
   }
-  if (!make_tensor_map_2d(&tmB, xq, dtB, T::kFp4 ? 0 : T::kBElemBytes, K, M, T::kBBoxElems, BN,
+  if (!make_tensor_map_2d(&tmB, xq, dtB, T::kFp4 ? 0 : T::kBElemBytes, K, M, T::kBBoxElems, C::kBRows,
                           CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (T::kSparse && !T::kPacked) {
@@ -1169,7 +1317,7 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   } else {
     tmE = tmB;  // unused
   }
-  if (T::kPacked) tmA = tmB;  // unused
+  if (T::kPacked && !T::kPair) tmA = tmB;  // unused
   CUtensorMap tmY = tmB;       // unused unless Y is stored through shared memory
   if (C::kTmaStoreY &&
       !make_tensor_map_2d(&tmY, y, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, N, M, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -1222,11 +1370,16 @@ static cudaError_t launch_typed(const GemmPlan &pl, const void *xq, const float 
   // anyway.  The launch is not cooperative: a cooperative grid was measured
   // to start 1-2 us later behind the previous kernel, losing the weight
   // prefetch that programmatic launch overlaps with it.
-  cudaLaunchAttribute attrs[1];
+  cudaLaunchAttribute attrs[2];
   attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  attrs[1].id = cudaLaunchAttributeClusterDimension;  // SM pairs: clusters of two
+  attrs[1].val.clusterDim.x = 2;
+  attrs[1].val.clusterDim.y = 1;
+  attrs[1].val.clusterDim.z = 1;
   cfg.attrs = attrs;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = T::kPair ? 2 : 1;
+  if (T::kPair && pl.grid % 2 != 0) return cudaErrorInvalidValue;
   return cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, MT, XQ, KB, VS>, tmA, tmB, tmE, tmY, a);
 }
 
@@ -1235,7 +1388,13 @@ static cudaError_t launch_kind(const GemmPlan &pl, const void *xq, const float *
                                const void *w_values, const uint8_t *w_meta, const float *w_scale,
                                void *y, int M, int N, int K, void *ws, int32_t *status,
                                cudaStream_t st) {
-  if constexpr (KIND == kSparseFP4) {
+  if constexpr (KIND == kSparseE4M3Pair) {
+    if (pl.bn == 224 && pl.kb == 2)
+      return launch_typed<KIND, 224, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+    if (pl.bn == 224)
+      return launch_typed<KIND, 224, 1, 0, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+    return cudaErrorInvalidValue;
+  } else if constexpr (KIND == kSparseFP4) {
     switch (pl.bn) {
       case 16: return launch_typed<KIND, 16, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
       case 32: return launch_typed<KIND, 32, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
@@ -1349,6 +1508,8 @@ cudaError_t launch_gemm(GemmKind kind, const GemmPlan &pl, const void *xq, const
       return launch_kind<kSparseI8Packed>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
     case kSparseFP4:
       return launch_kind<kSparseFP4>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
+    case kSparseE4M3Pair:
+      return launch_kind<kSparseE4M3Pair>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, workspace, status, st);
     default:
       return cudaErrorInvalidValue;
   }

@@ -521,6 +521,25 @@ def test_packed_gemm_small(m, n, k):
     assert torch.equal(y, y2)
 
 
+# 224-token tiles over N % 256 == 0 run on SM pairs (one M = 256 MMA over
+# two CTAs): whole tiles (1024 x 256), every tile split two ways
+# (1100 x 768), tiles split unevenly (4096 x 512 x 384), and full waves of
+# pairs with leftover tiles (2048 x 4096).
+@pytest.mark.parametrize("m,n,k", [(1024, 256, 256), (1100, 768, 1024), (4096, 512, 384), (2048, 4096, 256)])
+def test_packed_gemm_sm_pairs(m, n, k):
+    x = WL.random_bits((m, k), 850 + m)
+    w = WL.random_bits((n, k), 950 + n, scale=0.02)
+    st = new_status()
+    c = sp().sp24_prune_compress(dev_bf16(w), "e4m3", status=st)
+    xq, sx = sp().fp8_quantize_pertensor(dev_bf16(x), status=st)
+    packed = sp().sp24_pack_weights(c["values"], c["meta"])
+    y = sp().sp24_gemm_packed(xq, sx, packed, c["scale"], n, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    y_ref, b = _ref(host(xq), host(sx)[0], host(c["values"]), host(c["meta"]), host(c["scale"])[0], k)
+    assert_gemm_close(y, y_ref, b, f"packed on SM pairs {m}x{n}x{k}")
+
+
 @pytest.mark.parametrize("m", [1, 8, 32, 64])
 def test_packed_gemm_decode_workload(m):
     w, x = WL.weight_bits(2), WL.activation_bits(2, m)

@@ -84,10 +84,13 @@ size_t sp24_workspace_size(int op, int64_t M, int64_t N, int64_t K, int dtype) {
       if (M < 1 || N < 128 || Kg < 128 || M > INT32_MAX || N > INT32_MAX || Kg > INT32_MAX) return 0;
       int sms = device_sm_count();
       if (sms <= 0) sms = 148;
+      // the GEMM the call runs: the packed kind for the one-launch form, else
+      // the kind sp24_gemm_packed takes for the shape
+      const sp24::GemmKind gk = M * K / 8 <= sp24::kFusedXVec
+                                    ? sp24::kSparseE4M3Packed
+                                    : sp24::packed_kind(static_cast<int>(M), static_cast<int>(N), static_cast<int>(Kg), sms);
       return sp24::kFusedCounterBytes +
-             sp24::plan_gemm(sp24::kSparseE4M3Packed, static_cast<int>(M), static_cast<int>(N),
-                             static_cast<int>(Kg), sms)
-                 .workspace_bytes();
+             sp24::plan_gemm(gk, static_cast<int>(M), static_cast<int>(N), static_cast<int>(Kg), sms).workspace_bytes();
     }
     case SP24_OP_GEMM_FP4: {
       if (M < 1 || N < 128 || K < 256 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return 0;
@@ -370,13 +373,17 @@ static int quant_gemm_common(bool lift, const void *X, int M, int N, int K, cons
   const int sms = device_sm_count();
   if (sms < 0) return SP24_ERR_ARCH;
   const int Kg = lift ? K / 2 * 3 : K;
-  const sp24::GemmPlan pl = sp24::plan_gemm(sp24::kSparseE4M3Packed, M, N, Kg, sms);
+  const int64_t nelem = static_cast<int64_t>(M) * K;
+  const bool one_launch = nelem / 8 <= sp24::kFusedXVec;
+  // above the one-launch size: the GEMM sp24_gemm_packed runs for the shape
+  // (the same kind, so the same Y bit for bit)
+  const sp24::GemmKind gk = one_launch ? sp24::kSparseE4M3Packed : sp24::packed_kind(M, N, Kg, sms);
+  const sp24::GemmPlan pl = sp24::plan_gemm(gk, M, N, Kg, sms);
   if (!workspace || ws_bytes < sp24::kFusedCounterBytes + pl.workspace_bytes()) return SP24_ERR_WORKSPACE;
   if (!aligned16(workspace)) return SP24_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   void *gemm_ws = static_cast<uint8_t *>(workspace) + sp24::kFusedCounterBytes;
-  const int64_t nelem = static_cast<int64_t>(M) * K;
-  if (nelem / 8 <= sp24::kFusedXVec) {
+  if (one_launch) {
     // one launch: every CTA quantises all of X in front of its GEMM tiles
     sp24::GemmFusedX fx;
     fx.x = X;
@@ -396,8 +403,8 @@ static int quant_gemm_common(bool lift, const void *X, int M, int N, int K, cons
   else
     e = sp24::launch_quantize_fused(X, nelem, static_cast<uint32_t *>(workspace), x_scale, Xq, status, sms, st);
   if (e != cudaSuccess) return cuda_status(e);
-  return cuda_status(sp24::launch_gemm(sp24::kSparseE4M3Packed, pl, Xq, x_scale, packed, nullptr, w_scale, Y, M,
-                                       N, Kg, gemm_ws, status, st));
+  return cuda_status(sp24::launch_gemm(gk, pl, Xq, x_scale, packed, nullptr, w_scale, Y, M, N, Kg, gemm_ws, status,
+                                       st));
 }
 
 int sp24_quantize_gemm_packed(const void *X, int M, int N, int K, const void *packed,

@@ -488,7 +488,8 @@ int sp24_gemm_packed_scaled(const void *Xq, const float *x_scales, int x_per_tok
     return SP24_ERR_ALIGN;
   const int sms = device_sm_count();
   if (sms < 0) return SP24_ERR_ARCH;
-  const sp24::GemmPlan pl = sp24::plan_gemm(sp24::kSparseE4M3Packed, M, N, K, sms);
+  // the tiles sp24_gemm_packed takes for the shape (SM pairs included)
+  const sp24::GemmPlan pl = sp24::plan_gemm(sp24::packed_kind(M, N, K, sms), M, N, K, sms);
   if (pl.workspace_bytes() > 0) {
     if (!workspace || ws_bytes < pl.workspace_bytes()) return SP24_ERR_WORKSPACE;
     if (!aligned16(workspace)) return SP24_ERR_ALIGN;

@@ -1256,6 +1256,7 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
     pl.grid *= 2;
     pl.partial_bytes *= 2;
   }
+  pl.pair = pair ? 1 : 0;
   return pl;
 }
 
@@ -1458,6 +1459,15 @@ cudaError_t launch_gemm_scaled(const GemmPlan &pl, const void *xq, const float *
                                const void *packed, const float *w_scales, int w_vec, void *y, int M, int N,
                                int K, void *ws, int32_t *status, cudaStream_t st) {
   constexpr int P = kSparseE4M3Packed;
+  if (pl.pair) {
+    if (pl.bn != 224) return cudaErrorInvalidValue;
+    return pl.kb == 2 ? launch_typed<kSparseE4M3Pair, 224, 1, 0, 2, true>(pl, xq, x_scales, packed, nullptr, w_scales,
+                                                                          y, M, N, K, ws, status, st, nullptr, x_vec,
+                                                                          w_vec)
+                      : launch_typed<kSparseE4M3Pair, 224, 1, 0, 1, true>(pl, xq, x_scales, packed, nullptr, w_scales,
+                                                                          y, M, N, K, ws, status, st, nullptr, x_vec,
+                                                                          w_vec);
+  }
 #define SP24_SCALED(BN_, MT_, KB_)                                                                        \
   return launch_typed<P, BN_, MT_, 0, KB_, true>(pl, xq, x_scales, packed, nullptr, w_scales, y, M, N, K, ws, \
                                                  status, st, nullptr, x_vec, w_vec)

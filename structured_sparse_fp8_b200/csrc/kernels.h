@@ -115,6 +115,7 @@ struct GemmPlan {
   int64_t sk_units;
   size_t partial_bytes;
   size_t counter_bytes;
+  int pair;          // planned for kSparseE4M3Pair (grid counts CTAs: two per pair)
   size_t workspace_bytes() const { return stream_k ? counter_bytes + partial_bytes : 0; }
 };
 

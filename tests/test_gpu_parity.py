@@ -827,8 +827,9 @@ def _scaled_check(m, n, k, x_vec, w_vec, seed):
 
 
 # decode tiles (256-K stages), a ragged M, stream-K splits, and 256-row tiles
+# on SM pairs (one- and two-block stages)
 @pytest.mark.parametrize("m,n,k", [(1, 256, 512), (13, 384, 1024), (64, 128, 640), (300, 256, 1152),
-                                   (1100, 9728, 640)])
+                                   (1100, 9728, 640), (1500, 512, 1024)])
 @pytest.mark.parametrize("x_vec,w_vec", [(True, True), (True, False), (False, True), (False, False)])
 def test_sparse_gemm_packed_scaled(m, n, k, x_vec, w_vec):
     _scaled_check(m, n, k, x_vec, w_vec, m + n)

@@ -187,7 +187,7 @@ int fp8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, uint8_t *q
   const int rc = check_workspace(workspace, ws_bytes);
   if (rc != SP24_OK) return rc;
   if (sp24::small_quantize_fits(nelem))
-    return cuda_status(sp24::launch_quantize_small(X, nelem, false, scale, q, status, st));
+    return cuda_status(sp24::launch_quantize_small(X, nelem, sp24::kSmallE4M3, scale, q, status, st));
   return cuda_status(sp24::launch_quantize_fused(X, nelem, static_cast<uint32_t *>(workspace), scale,
                                                  q, status, sms, st));
 }
@@ -201,6 +201,10 @@ int int8_quantize_pertensor(const void *X, int64_t rows, int64_t cols, int8_t *q
   if (rc != SP24_OK) return rc;
   const int sms = device_sm_count();
   if (sms < 0) return SP24_ERR_ARCH;
+  if (sp24::small_quantize_fits(rows * cols))
+    return cuda_status(sp24::launch_quantize_small(X, rows * cols, sp24::kSmallInt8, scale,
+                                                   reinterpret_cast<uint8_t *>(q), status,
+                                                   reinterpret_cast<cudaStream_t>(stream)));
   return cuda_status(sp24::launch_int8_quantize(X, rows * cols, static_cast<uint32_t *>(workspace), scale, q,
                                                 status, sms, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -251,7 +255,7 @@ int slide68_lift(const void *X, int M, int K, uint8_t *q_lifted, float *scale, v
   const int rc = check_workspace(workspace, ws_bytes);
   if (rc != SP24_OK) return rc;
   if (sp24::small_quantize_fits(nelem))
-    return cuda_status(sp24::launch_quantize_small(X, nelem, true, scale, q_lifted, status, st));
+    return cuda_status(sp24::launch_quantize_small(X, nelem, sp24::kSmallLift, scale, q_lifted, status, st));
   return cuda_status(sp24::launch_lift_fused(X, nelem, static_cast<uint32_t *>(workspace), scale,
                                              q_lifted, status, sms, st));
 }
@@ -317,6 +321,9 @@ int fp4_quantize_pertensor(const void *X, int64_t rows, int64_t cols, uint8_t *q
   if (rc != SP24_OK) return rc;
   const int sms = device_sm_count();
   if (sms < 0) return SP24_ERR_ARCH;
+  if (sp24::small_quantize_fits(rows * cols))
+    return cuda_status(sp24::launch_quantize_small(X, rows * cols, sp24::kSmallFp4, scale, q, status,
+                                                   reinterpret_cast<cudaStream_t>(stream)));
   return cuda_status(sp24::launch_fp4_quantize(X, rows * cols, static_cast<uint32_t *>(workspace), scale, q,
                                                status, sms, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -397,7 +404,7 @@ static int quant_gemm_common(bool lift, const void *X, int M, int N, int K, cons
   // kernel beyond that), then the GEMM on its codes.
   cudaError_t e;
   if (sp24::small_quantize_fits(nelem))
-    e = sp24::launch_quantize_small(X, nelem, lift, x_scale, Xq, status, st);
+    e = sp24::launch_quantize_small(X, nelem, lift ? sp24::kSmallLift : sp24::kSmallE4M3, x_scale, Xq, status, st);
   else if (lift)
     e = sp24::launch_lift_fused(X, nelem, static_cast<uint32_t *>(workspace), x_scale, Xq, status, sms, st);
   else

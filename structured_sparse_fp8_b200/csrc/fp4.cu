@@ -39,15 +39,6 @@ constexpr int kTabBytes = 65536;   // one code per bf16 bit pattern
 // |x| > amax / 24: within 6 binades below amax's, so 7 binades in all.
 constexpr int kBand = 7;
 
-// E2M1 code (4 bits) of one fp32 value.  Both halves of the pair convert the
-// same value, so the result does not depend on which half lands in which
-// nibble; the sign is ORed in for a value that rounds to zero.
-__device__ __forceinline__ uint32_t e2m1_code(float v) {
-  uint16_t r;
-  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %1;\n\tcvt.u16.u8 %0, t;\n\t}" : "=h"(r) : "f"(v));
-  return (r & 0x7u) | ((__float_as_uint(v) >> 28) & 0x8u);
-}
-
 __device__ __forceinline__ uint32_t fp4_code(uint32_t h, float s) {
   return e2m1_code(__fdiv_rn(bf16_bits_to_float(h), s));
 }

@@ -36,11 +36,6 @@ constexpr int kBatch = 4;          // vectors per thread per pass (table form)
 constexpr int kTabBytes = 65536;   // one code per bf16 bit pattern
 constexpr int kBand = 10;          // |x| >= amax / 254 lies within 9 binades of amax's
 
-__device__ __forceinline__ int32_t int8_code(uint32_t h, float s) {
-  const int32_t q = __float2int_rn(__fdiv_rn(bf16_bits_to_float(h), s));
-  return min(max(q, -127), 127);
-}
-
 // INT8 code (as its byte) of a bf16 pattern h (16 bits): from the table, or
 // (DIRECT) by the division.
 template <bool DIRECT>

@@ -76,11 +76,13 @@ constexpr size_t kAmaxWorkspaceBytes = 256;
 constexpr size_t kFusedCounterBytes = 8192;
 
 // ---- smallx.cu: decode-sized activations (at most kSmallXVec 8-element
-// vectors, nelem % 8 == 0) quantised, or lifted (rows of 16k elements), by
-// one thread-block cluster; no workspace.
+// vectors, nelem % 8 == 0) quantised by one thread-block cluster, no
+// workspace: E4M3 codes [nelem], their 6:8 lift (rows of 16k elements)
+// [3 nelem / 2], INT8 codes [nelem] or FP4 codes [nelem / 2] (two per byte).
 constexpr int64_t kSmallXVec = 16384;
+enum SmallEnc : int { kSmallE4M3 = 0, kSmallLift = 1, kSmallInt8 = 2, kSmallFp4 = 3 };
 bool small_quantize_fits(int64_t nelem);
-cudaError_t launch_quantize_small(const void *x, int64_t nelem, bool lift, float *scale, uint8_t *q,
+cudaError_t launch_quantize_small(const void *x, int64_t nelem, SmallEnc enc, float *scale, uint8_t *q,
                                   int32_t *status, cudaStream_t st);
 
 // ---- gemm.cu

@@ -71,6 +71,22 @@ __device__ __forceinline__ bool e4m3_codes4_quot(uint32_t h0, uint32_t h1, float
   return bad == 0u;
 }
 
+// INT8 code of the bf16 pattern h at scale s: the correctly rounded quotient
+// rounded half to even and clamped to +-127.
+__device__ __forceinline__ int32_t int8_code(uint32_t h, float s) {
+  const int32_t q = __float2int_rn(__fdiv_rn(bf16_bits_to_float(h), s));
+  return min(max(q, -127), 127);
+}
+
+// E2M1 code (4 bits) of one fp32 value.  Both halves of the pair convert the
+// same value, so the result does not depend on which half lands in which
+// nibble; the sign is ORed in for a value that rounds to zero.
+__device__ __forceinline__ uint32_t e2m1_code(float v) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %1;\n\tcvt.u16.u8 %0, t;\n\t}" : "=h"(r) : "f"(v));
+  return (r & 0x7u) | ((__float_as_uint(v) >> 28) & 0x8u);
+}
+
 // The exact forms, out of line: rare, and kept out of the unrolled loops.
 static __device__ __noinline__ uint32_t e4m3_codes4_div(uint32_t h0, uint32_t h1, float s) {
   const uint32_t hh[4] = {h0 & 0xFFFFu, h0 >> 16, h1 & 0xFFFFu, h1 >> 16};

@@ -1,5 +1,6 @@
-// smallx.cu -- per-tensor E4M3 quantisation (and the SlideSparse 6:8 lift)
-// of decode-sized activations by ONE thread-block cluster.
+// smallx.cu -- per-tensor quantisation of decode-sized activations by ONE
+// thread-block cluster: E4M3 codes, the SlideSparse 6:8 lift of them, INT8
+// codes or FP4 (E2M1) codes.
 //
 // The quantiser of the cookbook's FP8 recipe ("Practical Example 2": one
 // scale amax / 448 for the whole tensor, codes E4M3(x / scale)) needs the
@@ -16,9 +17,12 @@
 //  3. waits for its own barrier's kSmallCtas arrivals (acquire, cluster
 //     scope), takes the max of the slots and the scale s = amax / 448
 //     (1 when amax = 0);
-//  4. encodes its registers with the division-free encoder (e4m3_codes8_fast,
-//     exact; the vectors it cannot decide go through the correctly rounded
-//     division) and stores 8 codes (or the 12 lifted codes) per vector.
+//  4. encodes its registers and stores them: E4M3 with the division-free
+//     encoder (e4m3_codes8_fast, exact; the vectors it cannot decide go
+//     through the correctly rounded division), 8 codes or the 12 lifted
+//     codes per vector; INT8 (s = amax / 127) and FP4 (s = amax / 6) by the
+//     correctly rounded division, 8 bytes or 8 nibbles (element 2i in the
+//     low nibble of byte i) per vector.
 // The kernel releases its dependents as soon as the previous kernel has
 // completed: the GEMM that consumes the codes then launches and streams its
 // weights while this cluster runs (it waits for this grid's completion
@@ -40,7 +44,12 @@ constexpr int kSmallCtas = 8;    // one portable-size cluster
 constexpr int kSmallThreads = 256;
 constexpr int kSmallRegs = 8;    // 16-byte X vectors per thread
 
-template <bool LIFT>
+// amax / (the code grid's largest magnitude) is the scale
+__host__ __device__ constexpr float grid_max(int enc) {
+  return enc == kSmallInt8 ? 127.0f : enc == kSmallFp4 ? 6.0f : 448.0f;
+}
+
+template <int ENC>
 __global__ void __launch_bounds__(kSmallThreads)
     small_quantize_kernel(const uint4 *__restrict__ x, int64_t nvec, float *scale_out, uint8_t *__restrict__ q,
                           int32_t *status) {
@@ -84,7 +93,7 @@ __global__ void __launch_bounds__(kSmallThreads)
     uint32_t amax = 0;
 #pragma unroll
     for (int r = 0; r < kSmallCtas; ++r) amax = max(amax, s_part[r]);
-    const float sx = amax == 0u ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax), 448.0f);
+    const float sx = amax == 0u ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax), grid_max(ENC));
     if (rank == 0) {
       *scale_out = sx;
       if (amax >= 0x7F80u && status) atomicOr(status, SP24_STATUS_NONFINITE);
@@ -94,23 +103,48 @@ __global__ void __launch_bounds__(kSmallThreads)
   }
   __syncthreads();
   const float sx = s_scale[0], rx = s_scale[1];
-  uint2 c[kSmallRegs];
-  bool ok[kSmallRegs];
+  if constexpr (ENC == kSmallInt8 || ENC == kSmallFp4) {
 #pragma unroll
-  for (int u = 0; u < kSmallRegs; ++u) c[u] = e4m3_codes8_fast(w[u], rx, ok[u]);
+    for (int u = 0; u < kSmallRegs; ++u) {
+      const int64_t v = v0 + t + kSmallThreads * u;
+      if (v < v1) {
+        const uint32_t h[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+        uint32_t lo = 0, hi = 0;
 #pragma unroll
-  for (int u = 0; u < kSmallRegs; ++u) {
-    const int64_t v = v0 + t + kSmallThreads * u;
-    if (v < v1) {
-      if (!ok[u]) c[u] = e4m3_codes8_div(w[u], sx);
-      if constexpr (LIFT) {
-        // 8-group g -> the 12 codes of windows 2j .. 2j + 3, j = 0..2
-        uint32_t *o = reinterpret_cast<uint32_t *>(q + 12 * v);
-        o[0] = c[u].x;
-        o[1] = __byte_perm(c[u].x, c[u].y, 0x5432);
-        o[2] = c[u].y;
-      } else {
-        *reinterpret_cast<uint2 *>(q + 8 * v) = c[u];
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t e = (h[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
+          if constexpr (ENC == kSmallInt8) {
+            const uint32_t b = static_cast<uint32_t>(int8_code(e, sx)) & 0xFFu;
+            if (i < 4) lo |= b << (8 * i); else hi |= b << (8 * (i - 4));
+          } else {
+            lo |= e2m1_code(__fdiv_rn(bf16_bits_to_float(e), sx)) << (4 * i);
+          }
+        }
+        if constexpr (ENC == kSmallInt8)
+          *reinterpret_cast<uint2 *>(q + 8 * v) = make_uint2(lo, hi);
+        else
+          *reinterpret_cast<uint32_t *>(q + 4 * v) = lo;
+      }
+    }
+  } else {
+    uint2 c[kSmallRegs];
+    bool ok[kSmallRegs];
+#pragma unroll
+    for (int u = 0; u < kSmallRegs; ++u) c[u] = e4m3_codes8_fast(w[u], rx, ok[u]);
+#pragma unroll
+    for (int u = 0; u < kSmallRegs; ++u) {
+      const int64_t v = v0 + t + kSmallThreads * u;
+      if (v < v1) {
+        if (!ok[u]) c[u] = e4m3_codes8_div(w[u], sx);
+        if constexpr (ENC == kSmallLift) {
+          // 8-group g -> the 12 codes of windows 2j .. 2j + 3, j = 0..2
+          uint32_t *o = reinterpret_cast<uint32_t *>(q + 12 * v);
+          o[0] = c[u].x;
+          o[1] = __byte_perm(c[u].x, c[u].y, 0x5432);
+          o[2] = c[u].y;
+        } else {
+          *reinterpret_cast<uint2 *>(q + 8 * v) = c[u];
+        }
       }
     }
   }
@@ -123,7 +157,7 @@ __global__ void __launch_bounds__(kSmallThreads)
 
 bool small_quantize_fits(int64_t nelem) { return nelem > 0 && nelem % 8 == 0 && nelem / 8 <= kSmallXVec; }
 
-cudaError_t launch_quantize_small(const void *x, int64_t nelem, bool lift, float *scale, uint8_t *q,
+cudaError_t launch_quantize_small(const void *x, int64_t nelem, SmallEnc enc, float *scale, uint8_t *q,
                                   int32_t *status, cudaStream_t st) {
   static_assert(kSmallXVec <= static_cast<int64_t>(kSmallCtas) * kSmallThreads * kSmallRegs,
                 "every vector of a small X is held in some thread's registers");
@@ -144,8 +178,13 @@ cudaError_t launch_quantize_small(const void *x, int64_t nelem, bool lift, float
   cfg.numAttrs = 2;
   const uint4 *xv = static_cast<const uint4 *>(x);
   const int64_t nvec = nelem / 8;
-  return lift ? cudaLaunchKernelEx(&cfg, small_quantize_kernel<true>, xv, nvec, scale, q, status)
-              : cudaLaunchKernelEx(&cfg, small_quantize_kernel<false>, xv, nvec, scale, q, status);
+  switch (enc) {
+    case kSmallE4M3: return cudaLaunchKernelEx(&cfg, small_quantize_kernel<kSmallE4M3>, xv, nvec, scale, q, status);
+    case kSmallLift: return cudaLaunchKernelEx(&cfg, small_quantize_kernel<kSmallLift>, xv, nvec, scale, q, status);
+    case kSmallInt8: return cudaLaunchKernelEx(&cfg, small_quantize_kernel<kSmallInt8>, xv, nvec, scale, q, status);
+    case kSmallFp4: return cudaLaunchKernelEx(&cfg, small_quantize_kernel<kSmallFp4>, xv, nvec, scale, q, status);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace sp24

@@ -67,13 +67,15 @@ def test_fp4_quantize_bit_exact(shape, seed, scale):
 
 @pytest.mark.parametrize("amax_bits", [0x40C0, 0x3F80, 0x3D18, 0x447A])
 def test_fp4_quantize_every_bf16_value(amax_bits):
-    """Every finite bf16 value of magnitude <= amax, both forms: every rounding
-    decision of the E2M1 encoder at the scale amax / 6."""
+    """Every finite bf16 value of magnitude <= amax, in each kernel form:
+    every rounding decision of the E2M1 encoder at the scale amax / 6."""
     v = O.bf16_to_f32(np.arange(65536, dtype=np.uint16))
     amax = O.bf16_to_f32(np.array([amax_bits], dtype=np.uint16))[0]
     bits = np.arange(65536, dtype=np.uint16)[np.isfinite(v) & (np.abs(v) <= amax)]
     bits = np.concatenate([np.array([amax_bits], dtype=np.uint16), bits])
-    for reps in (1, 40):   # direct form, then a tensor large enough for the table form
+    # one thread-block cluster (<= 131072 values), the two-launch direct form,
+    # the table form
+    for reps in (1, 5, 40):
         flat = np.tile(bits, reps)
         k = 4096
         x = np.zeros(-(-len(flat) // k) * k, dtype=np.uint16)

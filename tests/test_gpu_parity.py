@@ -954,12 +954,13 @@ def test_slide_workload_gemm(n, k):
 
 # ------------------------------------------------------------ INT8 W8A8 (2:4 weights)
 
-@pytest.mark.parametrize("rows,cols,dist", [(1, 16, "normal"), (7, 48, "ties"), (300, 1920, "student_t3"),
-                                            (2048, 4096, "student_t3")])
+@pytest.mark.parametrize("rows,cols,dist", [(1, 16, "normal"), (7, 48, "ties"), (2, 65536, "ties"),
+                                            (300, 1920, "student_t3"), (2048, 4096, "student_t3")])
 def test_int8_quantize_bit_exact(rows, cols, dist):
-    """Codes and scale byte for byte: the division form for the small cases,
+    """Codes and scale byte for byte: one thread-block cluster up to 131072
+    values (the first three), the two-launch division form for X[300,1920],
     the code-table form for X[2048,4096] (above 2 x 148 x 512 vectors of 8);
-    the tie-heavy case puts fp32 quotients next to half-integers."""
+    the tie-heavy cases put fp32 quotients next to half-integers."""
     x = WL.random_bits((rows, cols), 4300 + rows, dist=dist)
     st = new_status()
     q, s = sp().int8_quantize_pertensor(dev_bf16(x), status=st)

@@ -1262,7 +1262,9 @@ GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count) {
 
 GemmKind packed_kind(int M, int N, int K, int sm_count) {
   const GemmPlan pl = plan_gemm(kSparseE4M3Packed, M, N, K, sm_count);
-  return (pl.mt == 2 && pl.bn == 224 && pair_capacity() >= 2) ? kSparseE4M3Pair : kSparseE4M3Packed;
+  const bool wide = pl.mt == 2 && pl.bn == 224;                      // prefill-sized
+  const bool mid = pl.bn == 128 && M > 128 && N % 256 == 0;          // several 128-token tiles
+  return ((wide || mid) && pair_capacity() >= 2) ? kSparseE4M3Pair : kSparseE4M3Packed;
 }
 
 template <int KIND, int BN, int MT, int XQ = 0, int KB = 1, bool VS = false>
@@ -1394,6 +1396,10 @@ static cudaError_t launch_kind(const GemmPlan &pl, const void *xq, const float *
       return launch_typed<KIND, 224, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
     if (pl.bn == 224)
       return launch_typed<KIND, 224, 1, 0, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+    if (pl.bn == 128 && pl.kb == 2)
+      return launch_typed<KIND, 128, 1, 0, 2>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
+    if (pl.bn == 128)
+      return launch_typed<KIND, 128, 1, 0, 1>(pl, xq, x_scale, w_values, w_meta, w_scale, y, M, N, K, ws, status, st);
     return cudaErrorInvalidValue;
   } else if constexpr (KIND == kSparseFP4) {
     switch (pl.bn) {
@@ -1460,13 +1466,15 @@ cudaError_t launch_gemm_scaled(const GemmPlan &pl, const void *xq, const float *
                                int K, void *ws, int32_t *status, cudaStream_t st) {
   constexpr int P = kSparseE4M3Packed;
   if (pl.pair) {
-    if (pl.bn != 224) return cudaErrorInvalidValue;
-    return pl.kb == 2 ? launch_typed<kSparseE4M3Pair, 224, 1, 0, 2, true>(pl, xq, x_scales, packed, nullptr, w_scales,
-                                                                          y, M, N, K, ws, status, st, nullptr, x_vec,
-                                                                          w_vec)
-                      : launch_typed<kSparseE4M3Pair, 224, 1, 0, 1, true>(pl, xq, x_scales, packed, nullptr, w_scales,
-                                                                          y, M, N, K, ws, status, st, nullptr, x_vec,
-                                                                          w_vec);
+#define SP24_SCALED_PAIR(BN_, KB_)                                                                            \
+  return launch_typed<kSparseE4M3Pair, BN_, 1, 0, KB_, true>(pl, xq, x_scales, packed, nullptr, w_scales, y, M, N, \
+                                                             K, ws, status, st, nullptr, x_vec, w_vec)
+    if (pl.bn == 224 && pl.kb == 2) SP24_SCALED_PAIR(224, 2);
+    if (pl.bn == 224) SP24_SCALED_PAIR(224, 1);
+    if (pl.bn == 128 && pl.kb == 2) SP24_SCALED_PAIR(128, 2);
+    if (pl.bn == 128) SP24_SCALED_PAIR(128, 1);
+#undef SP24_SCALED_PAIR
+    return cudaErrorInvalidValue;
   }
 #define SP24_SCALED(BN_, MT_, KB_)                                                                        \
   return launch_typed<P, BN_, MT_, 0, KB_, true>(pl, xq, x_scales, packed, nullptr, w_scales, y, M, N, K, ws, \

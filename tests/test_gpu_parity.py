@@ -524,9 +524,11 @@ def test_packed_gemm_small(m, n, k):
 # 224-token tiles over N % 256 == 0 run on SM pairs (one M = 256 MMA over
 # two CTAs): whole tiles (1024 x 256), every tile split two ways
 # (1100 x 768), tiles split unevenly (4096 x 512 x 384), and full waves of
-# pairs with leftover tiles (2048 x 4096), and one-block stages (K = 1152).
+# pairs with leftover tiles (2048 x 4096), and one-block stages (K = 1152);
+# 128-token tiles of 129..1023 tokens (two-way splits at 256 x 512 x 2048, a
+# ragged token tile and one-block stages at 300 x 768 x 640).
 @pytest.mark.parametrize("m,n,k", [(1024, 256, 256), (1100, 768, 1024), (4096, 512, 384), (2048, 4096, 256),
-                                   (1500, 512, 1152)])
+                                   (1500, 512, 1152), (256, 512, 2048), (300, 768, 640)])
 def test_packed_gemm_sm_pairs(m, n, k):
     x = WL.random_bits((m, k), 850 + m)
     w = WL.random_bits((n, k), 950 + n, scale=0.02)

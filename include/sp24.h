@@ -431,12 +431,16 @@ int fp8_gemm_dense(const uint8_t *Xq, const float *x_scale, const uint8_t *Wq,
  * keeps the scratch of its amax reduction in a 256-byte static device array
  * inside the library instead; every GPU that loads the library holds those
  * bytes until the process exits.  It calls no allocating routine.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
- *   - Every call clears the array's counters on `stream` before using them.
- *     All calls share the one array, so calls that overlap on the GPU (other
- *     streams, other threads) race: serialise them.
+ *   - A decode-sized X (rows * cols <= 131072) uses no scratch at all (one
+ *     thread-block cluster, as fp8_quantize_pertensor).
+ *   - A larger X looks up the array's device address (cudaGetSymbolAddress)
+ *     on every call, with that device current; make the first such call on
+ *     a device before any stream capture (it loads the module).
+ *   - Such a call clears the array's counters on `stream` before using them
+ *     (a copy between the previous kernel and the quantiser, which then
+ *     cannot start beside that kernel).  All calls share the one array, so
+ *     calls that overlap on the GPU (other streams, other threads) race:
+ *     serialise them.
  *   - The scratch needed does not grow with the tensor; a configuration whose
  *     need exceeded the array would be rejected with SP24_ERR_WORKSPACE.
  * Shape rules and errors as fp8_quantize_pertensor.

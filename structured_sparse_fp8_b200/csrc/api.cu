@@ -49,6 +49,7 @@ int check_workspace(const void *workspace, size_t ws_bytes) {
 }  // namespace
 
 void sp24::set_last_cuda_error(int e) { g_last_cuda_error = e; }
+int sp24::current_device_sm_count() { return device_sm_count(); }
 
 extern "C" {
 

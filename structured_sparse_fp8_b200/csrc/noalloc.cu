@@ -7,12 +7,11 @@
 // engine or plugin host that owns every device allocation and forbids its
 // plugins from calling cudaMalloc, or a latency-critical loop where the
 // implicit device synchronisation of cudaMalloc/cudaFree is not acceptable.
-// This file gives them fp8_quantize_pertensor_static, which keeps the scratch
-// in a file-scope __device__ array instead.
+// This file gives them fp8_quantize_pertensor_static: a decode-sized X goes
+// to the one-cluster quantiser, which needs no scratch at all; a larger X
+// keeps its scratch in a file-scope __device__ array instead.
 #include <cuda_runtime.h>
 #include <stdint.h>
-
-#include <mutex>
 
 #include "kernels.h"
 #include "sp24.h"
@@ -24,24 +23,6 @@ namespace {
 constexpr size_t kStaticScratchBytes = 256;
 static_assert(sp24::kAmaxWorkspaceBytes <= kStaticScratchBytes, "static scratch too small");
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
-
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-void *g_scratch_ptr[kMaxDevices];  // device address of g_static_scratch, per device
-
-// In host code `g_static_scratch` only names a host-side stand-in; the
-// device address must be looked up once per device with that device current.
-cudaError_t scratch_address(int dev, void **out) {
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void *p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
-  return cudaSuccess;
-}
 
 }  // namespace
 
@@ -56,26 +37,27 @@ extern "C" int fp8_quantize_pertensor_static(const void *X, int64_t rows, int64_
   // configuration whose need would exceed the static array.
   if (sp24_workspace_size(SP24_OP_QUANTIZE, rows, 0, cols, SP24_DTYPE_E4M3) > kStaticScratchBytes)
     return SP24_ERR_WORKSPACE;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SP24_ERR_ARCH;
-  int major = 0, minor = 0, sms = 0;
-  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (major != 10 || minor != 0) return SP24_ERR_ARCH;
-  void *scratch = nullptr;
-  cudaError_t e = scratch_address(dev, &scratch);
-  if (e != cudaSuccess) {
-    sp24::set_last_cuda_error(static_cast<int>(e));
-    return SP24_ERR_CUDA;
-  }
+  const int sms = sp24::current_device_sm_count();
+  if (sms < 0) return SP24_ERR_ARCH;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // The array keeps whatever the previous call left: clear the counters.
-  e = cudaMemsetAsync(scratch, 0, sp24::kAmaxWorkspaceBytes, st);
   const int64_t nelem = rows * cols;
-  if (e == cudaSuccess)
-    e = sp24::launch_quantize_fused(X, nelem, static_cast<uint32_t *>(scratch), scale, q, status,
-                                    sms, st);
+  cudaError_t e;
+  if (sp24::small_quantize_fits(nelem)) {
+    e = sp24::launch_quantize_small(X, nelem, sp24::kSmallE4M3, scale, q, status, st);
+  } else {
+    // In host code `g_static_scratch` names a host-side stand-in; the device
+    // address is looked up on every call (cheap once the module is loaded),
+    // so that a context created after a reset never gets a stale one.
+    void *scratch = nullptr;
+    e = cudaGetSymbolAddress(&scratch, g_static_scratch);
+    // The array keeps whatever the previous call left (a timed-out call's
+    // counters): clear them.  This copy sits on the stream between the
+    // previous kernel and the quantiser, which therefore cannot start early
+    // beside that kernel (programmatic launch) as it does with a workspace.
+    if (e == cudaSuccess) e = cudaMemsetAsync(scratch, 0, sp24::kAmaxWorkspaceBytes, st);
+    if (e == cudaSuccess)
+      e = sp24::launch_quantize_fused(X, nelem, static_cast<uint32_t *>(scratch), scale, q, status, sms, st);
+  }
   if (e != cudaSuccess) {
     sp24::set_last_cuda_error(static_cast<int>(e));
     return SP24_ERR_CUDA;

@@ -33,7 +33,10 @@ def test_static_scratch_quantize_matches_workspace_quantize_twice():
     dev = torch.device("cuda:0")
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
-    for call, (shape, seed, scale) in enumerate([((64, 4096), 11, 1.0), ((37, 14336), 12, 0.02)]):
+    # the streamed kernel on the static scratch (twice), then a decode-sized X
+    # (the one-cluster quantiser, no scratch)
+    for call, (shape, seed, scale) in enumerate([((64, 4096), 11, 1.0), ((37, 14336), 12, 0.02),
+                                                 ((8, 4096), 13, 1.0)]):
         bits = WL.random_bits(shape, seed, scale=scale)
         x = _dev_bf16(bits, dev)
         q = torch.empty(shape, dtype=torch.uint8, device=dev)

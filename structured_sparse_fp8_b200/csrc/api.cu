@@ -49,7 +49,10 @@ int check_workspace(const void *workspace, size_t ws_bytes) {
 }  // namespace
 
 void sp24::set_last_cuda_error(int e) { g_last_cuda_error = e; }
-int sp24::current_device_sm_count() { return device_sm_count(); }
+namespace sp24 {
+// SM count of the current device for the other translation units (noalloc.cu)
+int current_device_sm_count() { return device_sm_count(); }
+}  // namespace sp24
 
 extern "C" {
 

@@ -65,9 +65,6 @@ cudaError_t launch_slide_lift(const void *x, int M, int K, int n, uint32_t *ws, 
 
 // Records the CUDA error reported by sp24_last_cuda_error() (api.cu).
 void set_last_cuda_error(int e);
-// SM count of the current device, or -1 when it is not sm_100 (api.cu; looked
-// up once per device).
-int current_device_sm_count();
 
 // Bytes of scratch the amax/scale reduction uses (two counters, padded).
 constexpr size_t kAmaxWorkspaceBytes = 256;

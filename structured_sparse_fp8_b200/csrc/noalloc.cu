@@ -16,6 +16,12 @@
 #include "kernels.h"
 #include "sp24.h"
 
+namespace sp24 {
+// SM count of the current device, or -1 when it is not sm_100 (api.cu; looked
+// up once per device).
+int current_device_sm_count();
+}  // namespace sp24
+
 namespace {
 
 // Scratch of the static-scratch entry point.  Every GPU that loads the

@@ -641,10 +641,11 @@ def _every_bf16_up_to(amax_bits):
 
 @pytest.mark.parametrize("amax_bits", [0x43E0, 0x3FC0, 0x3D18, 0x447A, 0x2180, 0x0080])
 def test_quantize_gemm_packed_every_bf16_value(amax_bits):
-    """The fused kernel's division-free encoder, grid-wide form (every
-    eligible bf16 value, at M > 1024 / (K / 8) rows) and the local form
-    with codes staged in shared memory (M = 1, a strided subset), against the
-    oracle's correctly rounded division, bit for bit.  amax = 2^-126 makes
+    """The division-free encoder of both forms of the fused call: above the
+    one-launch size the one-cluster quantiser (every eligible bf16 value, in
+    rows of K = 1024), and the one-launch form with codes staged in shared
+    memory (M = 1, a strided subset), against the oracle's correctly rounded
+    division, bit for bit.  amax = 2^-126 makes
     the scale an fp32 subnormal whose reciprocal overflows, so every code
     takes the exact division; its outputs are bf16 subnormals, coarser than
     the GEMM tolerance, so only codes, scale and the two-launch identity

@@ -794,8 +794,13 @@ def run_gpu(args, wl, rank, world, local_rank):
         except Exception as e:  # a failure here is recorded, never fatal to the bench line
             fp4 = {"error": f"{type(e).__name__}: {e}"[:300]}
     prefill = None
+    speedups = None
     if rank == 0 and args.workload == "decode" and not args.no_prefill:
         prefill = prefill_headline(device, peaks)
+        try:
+            speedups = speedup_headlines(device, peaks)
+        except Exception as e:  # a failure here is recorded, never fatal to the bench line
+            speedups = {"error": f"{type(e).__name__}: {e}"[:300]}
     e2e_t, h2d, d2h = gw.e2e(args.steps)
     e2e_t = max_over_ranks(e2e_t, device)
     del g_timed, g_detail, g_warm
@@ -826,6 +831,7 @@ def run_gpu(args, wl, rank, world, local_rank):
                    "parallelism": f"replicas x{world}"},
         "roofline": roof,
         "prefill": prefill,
+        "speedups": speedups,
         "kernels": kernels,
         "sparse_vs_dense": compare,
         "fused_vs_unfused": fusion,
@@ -906,6 +912,95 @@ def prefill_headline(device, peaks, reps=20):
             "dense_tflops": round(flops / t_dn / 1e6, 1),
             "timing": f"CUDA graph of {reps} launches over {len(ps)} rotating packed weight copies "
                       f"({len(pd)} dense), inputs larger than L2"}
+
+
+def speedup_headlines(device, peaks, reps=20):
+    """The sparse-over-dense targets next to the decode headline: the MLP
+    down-projection (M256 N4096 K14336, HBM-bound) against the dense FP8
+    GEMM of the same family, and the 6:8 GEMM over K' = 6144 (lifted X,
+    6:8 weights in the packed layout) against the dense FP8 GEMM over
+    K = 4096 at M = 2048 (tensor-bound), each a CUDA graph of `reps`
+    launches over rotating weight copies larger than L2, CUDA events on the
+    launching stream."""
+    import torch
+
+    import structured_sparse_fp8_b200 as sp
+    from structured_sparse_fp8_b200 import workloads as WL
+    lib = sp._lib.load()
+    ws = sp.Workspace(device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+    def pool(t):
+        return [t] + [t.clone() for _ in range(max(1, -(-3 * L2_BYTES // t.numel())) - 1)]
+
+    def graph_us(fn):
+        fn(0)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for r in range(reps):
+                fn(r)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) * 1e3 / reps
+
+    out = {}
+    wl = WORKLOADS["downproj"]
+    m, n, k = wl["ms"][0], wl["n"], wl["k"]
+    w, x = bf(WL.weight_bits(wl["cfg"])), bf(WL.activation_bits(wl["cfg"], m))
+    packed, sw = sp.sp24_prune_compress_packed(w, workspace=ws)
+    wq, swd = sp.fp8_quantize_pertensor(w, workspace=ws)
+    xq, sx = sp.fp8_quantize_pertensor(x, workspace=ws)
+    del w, x
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=device)
+    ps, pd = pool(packed), pool(wq)
+    ws.get(max(lib.sp24_workspace_size(sp._lib.OP_GEMM_PACKED, m, n, k, 0),
+               lib.sp24_workspace_size(sp._lib.OP_GEMM_DENSE, m, n, k, 0)) + 4096)
+    t_sp = graph_us(lambda r: sp.sp24_gemm_packed(xq, sx, ps[r % len(ps)], sw, n, out=y, status=status,
+                                                  workspace=ws))
+    t_dn = graph_us(lambda r: sp.fp8_gemm_dense(xq, sx, pd[r % len(pd)], swd, out=y, status=status,
+                                                workspace=ws))
+    gbs = bytes_sparse_gemm(m, n, k) / t_sp / 1e3
+    out["down_proj"] = {"workload": wl["name"], "sparse_us": round(t_sp, 3), "dense_fp8_us": round(t_dn, 3),
+                        "speedup_vs_dense": round(t_dn / t_sp, 3), "sparse_gbs": round(gbs, 1),
+                        "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    del ps, pd, packed, wq, xq, y
+    wl = WORKLOADS["slide68"]
+    m, n, k = 2048, wl["n"], wl["k"]
+    kp = k // 2 * 3
+    w, x = bf(WL.weight_bits(wl["cfg"])), bf(WL.activation_bits(wl["cfg"], m))
+    packed, sw = sp.slide68_decompose_packed(w, workspace=ws)
+    xl, sxl = sp.slide68_lift(x, workspace=ws)
+    wq, swd = sp.fp8_quantize_pertensor(w, workspace=ws)
+    xq, sx = sp.fp8_quantize_pertensor(x, workspace=ws)
+    del w, x
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=device)
+    ps, pd = pool(packed), pool(wq)
+    ws.get(max(lib.sp24_workspace_size(sp._lib.OP_GEMM_PACKED, m, n, kp, 0),
+               lib.sp24_workspace_size(sp._lib.OP_GEMM_DENSE, m, n, k, 0)) + 4096)
+    t_sp = graph_us(lambda r: sp.sp24_gemm_packed(xl, sxl, ps[r % len(ps)], sw, n, out=y, status=status,
+                                                  workspace=ws))
+    t_dn = graph_us(lambda r: sp.fp8_gemm_dense(xq, sx, pd[r % len(pd)], swd, out=y, status=status,
+                                                workspace=ws))
+    tf = 2.0 * m * n * kp / t_sp / 1e6
+    out["slide68_m2048"] = {"workload": f"6:8 W[{n},{k}] over K'={kp} vs dense FP8 over K={k}, M={m}",
+                            "sparse_us": round(t_sp, 3), "dense_fp8_us": round(t_dn, 3),
+                            "speedup_vs_dense": round(t_dn / t_sp, 3),
+                            "sparse_tflops_dense_equiv": round(tf, 1),
+                            "frac_tensor": round(tf / (peaks["bf16_tflops"] * 4.0), 4)}
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "device status word set during the speed-up timing"
+    out["timing"] = f"CUDA graphs of {reps} launches over rotating weight copies, inputs larger than L2"
+    return out
 
 
 # ---------------------------------------------------------------- single-kernel cases

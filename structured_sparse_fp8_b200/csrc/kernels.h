@@ -93,7 +93,7 @@ enum GemmKind : int {
   kSparseE4M3Packed = 3,
   kSparseI8Packed = 4,
   kSparseFP4 = 5,  // E2M1 codes, two per byte, canonical 2:4 layout; stages of 256 K
-  kSparseE4M3Pair = 6  // the packed E4M3 kind on SM pairs (wide token tiles, N % 256 == 0)
+  kSparseE4M3Pair = 6  // the packed E4M3 kind on SM pairs (128- and 224-token tiles, N % 256 == 0)
 };
 
 // How a GEMM call is cut into CTAs: tile shape, work decomposition and the
@@ -123,9 +123,10 @@ struct GemmPlan {
 
 GemmPlan plan_gemm(GemmKind kind, int M, int N, int K, int sm_count);
 
-// The kind the packed E4M3 GEMM runs as: kSparseE4M3Pair where its plan
-// takes 224-token tiles of two weight row tiles and the device runs CTA
-// pairs, else kSparseE4M3Packed.
+// The kind the packed E4M3 GEMM runs as: kSparseE4M3Pair where N % 256 == 0,
+// the device runs CTA pairs and the plan takes 224-token tiles of two weight
+// row tiles (prefill) or 128-token tiles of 129..1023 tokens, else
+// kSparseE4M3Packed.
 GemmKind packed_kind(int M, int N, int K, int sm_count);
 
 // Launch the tcgen05 GEMM.  `workspace` must hold plan.workspace_bytes()

@@ -228,8 +228,12 @@ int slide68_decompose_packed(const void *W, int N, int K, void *packed, float *w
                              sp24_stream_t stream);
 
 /*
- * sp24_gemm (E4M3) with tile-packed weights (sp24_pack_weights); same result.
- * Workspace from sp24_workspace_size(SP24_OP_GEMM_PACKED, M, N, K, 0).
+ * sp24_gemm (E4M3) with tile-packed weights (sp24_pack_weights); same result
+ * within the GEMM tolerance (split tiles may sum their K ranges in another
+ * order).  Workspace from sp24_workspace_size(SP24_OP_GEMM_PACKED, M, N, K,
+ * 0).  When N % 256 == 0 and M is above 128 (prefill- and down-projection-
+ * sized calls) the kernel launches clusters of two CTAs (one 256-row MMA
+ * over two SMs); everywhere else one CTA per SM at most.
  */
 int sp24_gemm_packed(const void *Xq, const float *x_scale, const void *packed,
                      const float *w_scale, void *Y, int M, int N, int K, void *workspace,
